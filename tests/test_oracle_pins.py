@@ -1,0 +1,373 @@
+"""Pins for the fp64 oracle, against things other than the oracle itself.
+
+Each test checks the oracle against a closed form, a hand-worked case, an invariant the
+method guarantees, an independent formulation, or a library routine (torch SDPA in
+float64 on the CPU). No expected value here comes from the CUDA path.
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _rand_bf16(shape, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(shape, generator=g) * scale).to(torch.bfloat16)
+
+
+def _f64(bits):
+    return torch.from_numpy(orc.bf16_bits_to_f64(bits))
+
+
+def _sdpa_causal(q, k, v, scale):
+    """Dense causal attention in float64 via torch SDPA. q [N,hq,d], k/v [N,hkv,d] (float64)."""
+    hq, hkv = q.shape[1], k.shape[1]
+    rep = hq // hkv
+    kk = k.repeat_interleave(rep, dim=1)
+    vv = v.repeat_interleave(rep, dim=1)
+    o = torch.nn.functional.scaled_dot_product_attention(
+        q.transpose(0, 1), kk.transpose(0, 1), vv.transpose(0, 1), is_causal=True, scale=scale)
+    return o.transpose(0, 1)
+
+
+def _exact_bf16(x: Fraction) -> int:
+    """Nearest bf16 to an exact rational, ties to even, by direct search (independent of the oracle)."""
+    if x == 0:
+        return 0
+    sign = 0x8000 if x < 0 else 0
+    a = abs(x)
+    e = math.floor(math.log2(a))
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    e = max(e, -126)
+    ulp = Fraction(2) ** (e - 7)
+    lo = (a // ulp) * ulp
+    hi = lo + ulp
+    if a - lo < hi - a:
+        r = lo
+    elif a - lo > hi - a:
+        r = hi
+    else:
+        r = lo if (lo / ulp) % 2 == 0 else hi
+    f = np.array([float(r)], dtype=np.float32)
+    return sign | int(f.view(np.uint32)[0] >> 16)
+
+
+# ---------------------------------------------------------------- bf16 rounding
+
+def test_round_bf16_matches_torch_on_float32_values():
+    g = torch.Generator().manual_seed(1)
+    x = torch.randn(20000, generator=g) * torch.exp(torch.randn(20000, generator=g) * 20)
+    x = torch.cat([x, torch.tensor([0.0, -0.0, 1e-40, -3e-39, 3.0e38, 65504.0, 1.0 + 2 ** -8])])
+    ref = _bits(x.to(torch.bfloat16))
+    got = orc.round_bf16(x.double().numpy())
+    assert np.array_equal(got, ref)
+
+
+def test_round_bf16_single_rounding_step():
+    # 1 + 2^-8 + 2^-30 lies just above the midpoint of bf16 neighbours 1.0 (0x3F80) and
+    # 1 + 2^-7 (0x3F81): the correctly rounded result is 0x3F81. Rounding through fp32
+    # first would drop the 2^-30 and then tie to even (0x3F80).
+    x = 1.0 + 2.0 ** -8 + 2.0 ** -30
+    assert orc.round_bf16(np.array([x]))[0] == 0x3F81
+    assert orc.round_bf16(np.array([1.0 + 2.0 ** -8]))[0] == 0x3F80       # exact tie -> even
+    assert orc.round_bf16(np.array([1.0 + 3 * 2.0 ** -8]))[0] == 0x3F82   # exact tie -> even
+    big = (2 - 2 ** -8) * 2.0 ** 127                                       # max + half ulp -> inf
+    assert orc.round_bf16(np.array([big, -big]))[0] == 0x7F80
+    assert orc.round_bf16(np.array([big * (1 - 2 ** -20)]))[0] == 0x7F7F  # just below -> max
+
+
+def test_round_bf16_exact_rationals():
+    rng = np.random.default_rng(7)
+    xs = rng.standard_normal(400) * np.exp2(rng.integers(-140, 120, 400))
+    got = orc.round_bf16(xs)
+    for x, b in zip(xs, got):
+        assert b == _exact_bf16(Fraction(float(x))), x
+
+
+# ---------------------------------------------------------------- compression
+
+@pytest.mark.parametrize("l,s", [(32, 16), (8, 4), (6, 3), (5, 5)])
+def test_compress_is_rounded_exact_mean(l, s):
+    T, h, d = 150, 2, 8
+    k = _bits(_rand_bf16((T, h, d), seed=l * 100 + s))
+    kc = orc.compress(k, l, s)
+    nc = (T - l) // s + 1
+    assert kc.shape == (nc, h, d)
+    kf = orc.bf16_bits_to_f64(k)
+    for i in range(nc):
+        for g in range(h):
+            for c in range(0, d, 3):
+                mean = sum(Fraction(float(kf[i * s + u, g, c])) for u in range(l)) / l
+                assert kc[i, g, c] == _exact_bf16(mean)
+
+
+def test_compress_block_one_is_identity():
+    k = _bits(_rand_bf16((40, 3, 16), seed=3))
+    assert np.array_equal(orc.compress(k, 1, 1), k)
+
+
+def test_compress_short_sequence_has_no_blocks():
+    k = _bits(_rand_bf16((31, 1, 8), seed=4))
+    assert orc.compress(k, 32, 16).shape[0] == 0
+    assert orc.num_cmp(31) == 0 and orc.num_cmp(32) == 1 and orc.num_cmp(47) == 1 and orc.num_cmp(48) == 2
+
+
+def test_compress_integer_inputs_exact():
+    rng = np.random.default_rng(5)
+    ints = rng.integers(0, 8, (96, 1, 4)).astype(np.float32)
+    k = _bits(torch.from_numpy(ints).to(torch.bfloat16))
+    kc = orc.bf16_bits_to_f64(orc.compress(k, 32, 16))
+    for i in range(kc.shape[0]):
+        assert np.array_equal(kc[i], ints[i * 16:i * 16 + 32].mean(axis=0))
+
+
+# ---------------------------------------------------------------- closed forms from the pages
+
+def test_block_counts_closed_forms():
+    assert (orc.num_cmp(131072), orc.num_sel(131072)) == (8191, 2048)
+    assert (orc.num_cmp(36096), orc.num_sel(36096)) == (2255, 564)
+    assert (orc.num_cmp(2048), orc.num_sel(2048)) == (127, 32)
+
+
+def test_page_numbers_shapes_and_dense_count():
+    pages = json.load(open(os.path.join(GOLDEN, "pages_numbers.json")))
+    from sparse_attention_long_fwd_b200.inputs import TOKENS_PER_FRAME
+
+    # a 50,176-pixel frame at 28x28 pixels per merged vision token is 64 tokens
+    assert pages["max_pixels_per_frame"]["value"] // (28 * 28) == TOKENS_PER_FRAME
+    # the dense causal (query, key) pair count at 128K tokens is the ~8.2e9 the pages quote
+    n = pages["scales_to_tokens"]["value"]
+    pairs = n * (n + 1) // 2
+    assert abs(pairs - pages["dense_attention_ops_at_128k"]["value"]) / pairs < 0.01
+    # 36K context = 564 frames of 64 tokens (36,096), the hybrid workload's video prefix
+    assert 564 * TOKENS_PER_FRAME <= pages["max_training_context_tokens"]["value"] * 1.003
+
+
+# ---------------------------------------------------------------- branches vs library / invariants
+
+def _case(N, hq, hkv, d, seed, nv=None, **kw):
+    q = _rand_bf16((N, hq, d), seed)
+    k = _rand_bf16((N, hkv, d), seed + 1)
+    v = _rand_bf16((N, hkv, d), seed + 2)
+    g = torch.rand((N, hq, 3), generator=torch.Generator().manual_seed(seed + 3))
+    cfg = orc.OracleConfig(N, N if nv is None else nv, hq, hkv, d, **kw)
+    return cfg, q, k, v, g
+
+
+def test_cmp_branch_with_unit_blocks_is_dense_causal_attention():
+    cfg, q, k, v, g = _case(96, 4, 2, 16, 11, cmp_len=1, cmp_stride=1, sel_len=8, top_n=4, window=16)
+    rows = np.arange(96)
+    o = orc.prefill_rows(cfg, _bits(q), _bits(k), _bits(v), g.numpy(), rows)
+    scale = 1 / math.sqrt(16)
+    qd, kd, vd = _f64(_bits(q)), _f64(_bits(k)), _f64(_bits(v))
+    ref = _sdpa_causal(qd, kd, vd, scale)
+    assert np.allclose(o["o_cmp"], ref.numpy(), atol=1e-12, rtol=0)
+    # log-sum-exp against torch.logsumexp of the causal score rows
+    for t in (0, 5, 95):
+        for h in range(4):
+            z = (kd[: t + 1, h // 2] @ qd[t, h]) * scale
+            assert abs(o["lse"][t, h] - torch.logsumexp(z, 0).item()) < 1e-12
+
+
+def test_full_budget_selection_and_window_are_dense_attention():
+    N = 200
+    cfg, q, k, v, g = _case(N, 6, 2, 16, 21, top_n=orc.num_sel(N, 64) + 2, window=N + 5)
+    o = orc.prefill_rows(cfg, _bits(q), _bits(k), _bits(v), g.numpy(), np.arange(N))
+    ref = _sdpa_causal(_f64(_bits(q)), _f64(_bits(k)), _f64(_bits(v)), 1 / 4.0).numpy()
+    assert np.allclose(o["o_sel"], ref, atol=1e-12, rtol=0)
+    assert np.allclose(o["o_win"], ref, atol=1e-12, rtol=0)
+
+
+def test_first_token_attends_to_itself_only():
+    cfg, q, k, v, g = _case(64, 4, 1, 8, 31, top_n=4, window=16)
+    o = orc.prefill_rows(cfg, _bits(q), _bits(k), _bits(v), g.numpy(), np.array([0]))
+    v0 = orc.bf16_bits_to_f64(_bits(v))[0, 0]
+    for h in range(4):
+        assert np.allclose(o["o_sel"][0, h], v0, atol=1e-15)
+        assert np.allclose(o["o_win"][0, h], v0, atol=1e-15)
+        assert np.all(o["o_cmp"][0, h] == 0) and o["lse"][0, h] == -np.inf
+    assert list(o["sel"][0, 0]) == [0, -1, -1, -1]
+
+
+@pytest.mark.parametrize("which", [0, 1, 2])
+def test_one_hot_gates_isolate_a_branch(which):
+    cfg, q, k, v, _ = _case(300, 4, 2, 16, 41, top_n=4, window=40)
+    g = np.zeros((300, 4, 3), dtype=np.float32)
+    g[..., which] = 1.0
+    rows = np.array([0, 31, 32, 100, 200, 299])
+    o = orc.prefill_rows(cfg, _bits(q), _bits(k), _bits(v), g, rows)
+    key = ("o_cmp", "o_sel", "o_win")[which]
+    assert np.array_equal(o["out"], o[key])
+
+
+def test_text_rows_are_dense_causal_attention():
+    N, nv = 260, 192
+    cfg, q, k, v, g = _case(N, 4, 2, 16, 51, nv=nv, top_n=4, window=32)
+    rows = np.arange(nv, N)
+    o = orc.prefill_rows(cfg, _bits(q), _bits(k), _bits(v), g.numpy(), rows)
+    ref = _sdpa_causal(_f64(_bits(q)), _f64(_bits(k)), _f64(_bits(v)), 0.25).numpy()
+    assert np.allclose(o["out"], ref[nv:], atol=1e-12, rtol=0)
+
+
+def test_outputs_are_convex_combinations_of_values():
+    cfg, q, k, v, g = _case(400, 4, 2, 16, 61, top_n=5, window=50)
+    rows = np.arange(0, 400, 7)
+    o = orc.prefill_rows(cfg, _bits(q), _bits(k), _bits(v), g.numpy(), rows)
+    vd = orc.bf16_bits_to_f64(_bits(v))
+    vcd = orc.bf16_bits_to_f64(orc.compress(_bits(v)))
+    for key, src in (("o_sel", vd), ("o_win", vd)):
+        for gi in range(2):
+            lo, hi = src[:, gi].min(0), src[:, gi].max(0)
+            blk = o[key][:, gi * 2:(gi + 1) * 2]
+            assert np.all(blk >= lo - 1e-12) and np.all(blk <= hi + 1e-12)
+    for gi in range(2):
+        blk = o["o_cmp"][:, gi * 2:(gi + 1) * 2]
+        assert np.all(blk >= vcd[:, gi].min(0) - 1e-12) and np.all(blk <= vcd[:, gi].max(0) + 1e-12)
+
+
+# ---------------------------------------------------------------- block scores and selection
+
+def test_scores_equal_token_density_formulation():
+    """Independent formulation: spread each compression block's probability evenly over its
+    l tokens, then sum the token densities inside each selection block and over the group."""
+    N, hq, hkv, d = 700, 6, 2, 16
+    cfg, q, k, v, g = _case(N, hq, hkv, d, 71, top_n=6, window=64)
+    rows = np.array([31, 47, 63, 64, 130, 333, 640, 699])
+    o = orc.prefill_rows(cfg, _bits(q), _bits(k), _bits(v), g.numpy(), rows)
+    kc = _f64(orc.compress(_bits(k)))
+    qd = _f64(_bits(q))
+    G = hq // hkv
+    for r, t in enumerate(rows):
+        nc = orc.num_cmp(t + 1)
+        for gi in range(hkv):
+            dens = torch.zeros(N, dtype=torch.float64)
+            for hh in range(G):
+                h = gi * G + hh
+                p = torch.softmax((kc[:nc, gi] @ qd[t, h]) / 4.0, 0)
+                for i in range(nc):
+                    dens[16 * i:16 * i + 32] += p[i] / 32
+            jt = t // 64
+            ref = [dens[64 * j:64 * j + 64].sum().item() for j in range(jt + 1)]
+            assert np.allclose(o["scores"][r, gi, :jt + 1], ref, atol=1e-13, rtol=0)
+            assert np.all(o["scores"][r, gi, jt + 1:] == 0)
+
+
+def test_scores_conserve_mass():
+    cfg, q, k, v, g = _case(1500, 8, 2, 16, 81, top_n=6, window=64)
+    rows = np.arange(0, 1500, 13)
+    o = orc.prefill_rows(cfg, _bits(q), _bits(k), _bits(v), g.numpy(), rows)
+    for r, t in enumerate(rows):
+        tot = o["scores"][r].sum(axis=1)
+        expect = 4.0 if t >= 31 else 0.0
+        assert np.allclose(tot, expect, atol=1e-12)
+
+
+def test_selection_invariants_on_random_scores():
+    N, n = 2000, 7
+    cfg, q, k, v, g = _case(N, 4, 2, 16, 91, top_n=n, window=64)
+    rows = np.arange(0, N, 9)
+    o = orc.prefill_rows(cfg, _bits(q), _bits(k), _bits(v), g.numpy(), rows)
+    for r, t in enumerate(rows):
+        jt = t // 64
+        for gi in range(2):
+            sel = o["sel"][r, gi]
+            chosen = [int(x) for x in sel if x >= 0]
+            assert chosen == sorted(set(chosen))
+            assert len(chosen) == min(n, jt + 1)
+            assert all(x < 0 for x in sel[len(chosen):])
+            forced = {0, jt, jt - 1} & set(range(jt + 1))
+            assert forced <= set(chosen)
+            sc = o["scores"][r, gi]
+            free = [j for j in chosen if j not in forced]
+            rest = [j for j in range(jt + 1) if j not in chosen]
+            for a in free:
+                for b in rest:
+                    assert sc[a] > sc[b] or (sc[a] == sc[b] and a < b)
+
+
+def test_constant_keys_hand_worked_case():
+    case = json.load(open(os.path.join(GOLDEN, "constant_keys_case.json")))
+    c = case["config"]
+    N, hq, hkv, d = c["n_tokens"], c["hq"], c["hkv"], c["d"]
+    q = _rand_bf16((N, hq, d), 101)
+    krow = _rand_bf16((1, hkv, d), 102)
+    k = krow.expand(N, hkv, d).contiguous()
+    v = _rand_bf16((N, hkv, d), 103)
+    g = torch.rand((N, hq, 3), generator=torch.Generator().manual_seed(104))
+    cfg = orc.OracleConfig(N, c["n_video"], hq, hkv, d, c["cmp_len"], c["cmp_stride"], c["sel_len"], c["top_n"],
+                           c["window"])
+    rows = np.array([int(x) for x in case["rows"]])
+    o = orc.prefill_rows(cfg, _bits(q), _bits(k), _bits(v), g.numpy(), rows)
+    vd = orc.bf16_bits_to_f64(_bits(v))
+    vcd = orc.bf16_bits_to_f64(orc.compress(_bits(v)))
+    for r, t in enumerate(rows):
+        exp = case["rows"][str(t)]
+        assert list(o["sel"][r, 0]) == exp["sel"]
+        for key, den in (("scores_numerators_over_61", 61), ("scores_numerators_over_7", 7)):
+            if key in exp:
+                num = exp[key]
+                assert np.allclose(o["scores"][r, 0, :len(num)], np.array(num) / den, atol=1e-14)
+        # uniform scores: each branch output is the plain mean of its values
+        keys = [tau for j in exp["sel"] if j >= 0 for tau in range(64 * j, 64 * j + 64) if tau <= t]
+        win = list(range(max(0, t - c["window"] + 1), t + 1))
+        nc = orc.num_cmp(t + 1)
+        for h in range(hq):
+            assert np.allclose(o["o_sel"][r, h], vd[keys, 0].mean(0), atol=1e-14)
+            assert np.allclose(o["o_win"][r, h], vd[win, 0].mean(0), atol=1e-14)
+            ref_cmp = vcd[:nc, 0].mean(0) if nc else np.zeros(d)
+            assert np.allclose(o["o_cmp"][r, h], ref_cmp, atol=1e-14)
+
+
+def test_replay_with_own_selection_is_identity():
+    cfg, q, k, v, g = _case(900, 4, 2, 16, 111, top_n=5, window=100)
+    rows = np.array([100, 400, 899])
+    a = orc.prefill_rows(cfg, _bits(q), _bits(k), _bits(v), g.numpy(), rows)
+    b = orc.prefill_rows(cfg, _bits(q), _bits(k), _bits(v), g.numpy(), rows, sel_override=a["sel"])
+    assert np.array_equal(a["out"], b["out"])
+    # replay with a different selection changes only the selection branch
+    alt = a["sel"].copy()
+    alt[2, 0, 1] = 3 if alt[2, 0, 1] != 3 else 4
+    c = orc.prefill_rows(cfg, _bits(q), _bits(k), _bits(v), g.numpy(), rows, sel_override=alt)
+    assert np.array_equal(c["o_cmp"], a["o_cmp"]) and np.array_equal(c["o_win"], a["o_win"])
+    assert not np.allclose(c["o_sel"][2, :2], a["o_sel"][2, :2])
+
+
+# ---------------------------------------------------------------- decode
+
+def test_decode_equals_prefill_last_row():
+    B, Lmax, hq, hkv, d = 3, 400, 4, 2, 16
+    kcache = _rand_bf16((B, Lmax, hkv, d), 121)
+    vcache = _rand_bf16((B, Lmax, hkv, d), 122)
+    q = _rand_bf16((B, hq, d), 123)
+    gates = torch.rand((B, hq, 3), generator=torch.Generator().manual_seed(124))
+    seq_lens = np.array([400, 257, 31], dtype=np.int32)
+    kcmp = np.stack([orc.compress(_bits(kcache[b])) for b in range(B)])
+    vcmp = np.stack([orc.compress(_bits(vcache[b])) for b in range(B)])
+    cfg = orc.OracleConfig(Lmax, Lmax, hq, hkv, d, top_n=5, window=64)
+    dec = orc.decode(cfg, _bits(q), _bits(kcache), _bits(vcache), kcmp, vcmp, seq_lens, gates.numpy())
+    for b in range(B):
+        L = int(seq_lens[b])
+        qq = torch.zeros((L, hq, d), dtype=torch.bfloat16)
+        qq[L - 1] = q[b]
+        gg = torch.zeros((L, hq, 3))
+        gg[L - 1] = gates[b]
+        pc = orc.OracleConfig(L, L, hq, hkv, d, top_n=5, window=64)
+        pre = orc.prefill_rows(pc, _bits(qq), _bits(kcache[b, :L].contiguous()), _bits(vcache[b, :L].contiguous()),
+                               gg.numpy(), np.array([L - 1]))
+        assert np.array_equal(dec["out"][b], pre["out"][0])
+        assert np.array_equal(dec["sel"][b], pre["sel"][0])
