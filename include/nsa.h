@@ -1,0 +1,149 @@
+/*
+ * nsa.h -- C ABI of the B200 (sm_100a) Native Sparse Attention forward pass.
+ *
+ * The operation is the attention layer of VideoNSA: video tokens get Native Sparse
+ * Attention, made of three branches -- a compressed branch over block summaries, a
+ * selected branch over the most important token blocks, and a sliding-window branch --
+ * whose outputs are mixed per token and head by gates; trailing text tokens get dense
+ * causal attention. Sources: top168.com article on VideoNSA, section
+ * "一、革命性的三重注意机制" (the three branches and their gated combination);
+ * shd-paper.top page "VideoNSA: Native Sparse Attention Scales Video Understanding",
+ * abstract (dense attention for text, NSA for video; scaling to 128K tokens); CSDN blog
+ * "VideoNSA：重新定义视频理解的稀疏注意力机制", section 2.2 (CMP / SLC / SWA branches)
+ * and section 3.1 (one gate per branch and head).
+ *
+ * The pages fix no constants. This library computes, for query token t and head h of
+ * GQA group g = h / (Hq/Hkv), with scale = softmax_scale (<= 0: 1/sqrt(head_dim)):
+ *   Kc[i] = bf16_rne(mean_{u<l} K[i*s+u])                   (compression, l = cmp_block, s = cmp_stride)
+ *   o_cmp = softmax over compressed blocks i with i*s + l - 1 <= t  (0 if there are none)
+ *   score[t,g,j] = sum_{h in g} sum_i P_cmp[t,h,i] * |tokens(i) & tokens(j)| / l
+ *   selection: blocks 0, t/l' and t/l' - 1 always, then the best top_n - |forced| other
+ *              blocks j <= t/l' by (score desc, index asc)   (l' = sel_block)
+ *   o_sel = softmax over tokens tau <= t of the selected blocks
+ *   o_win = softmax over tokens max(0, t-window+1) .. t
+ *   out   = gates[t,h,0]*o_cmp + gates[t,h,1]*o_sel + gates[t,h,2]*o_win
+ *   rows t >= n_video (text): out = dense causal softmax over tokens 0..t.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers, 16-byte aligned, contiguous, token-major.
+ *     bf16 tensors are IEEE bfloat16; gates are fp32.
+ *   - The caller owns every buffer. The library allocates nothing per call; it keeps no
+ *     state besides a device error word. Scratch memory is the caller's `workspace`,
+ *     sized by nsa_workspace_size().
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream). Host-side validation errors return before anything is enqueued.
+ *   - Return value: NSA_OK (0) or one of the nsa_status codes below. No exception
+ *     crosses the ABI. Faults inside kernels surface at the caller's next sync; a kernel
+ *     whose internal wait timed out records it in the device error word
+ *     (nsa_get_device_error) and returns early instead of hanging.
+ *   - Supported on sm_100 (B200) only: head_dim in {64, 128}; Hq % Hkv == 0 with
+ *     Hq/Hkv <= 16; cmp_block = 32, cmp_stride = 16, sel_block = 64;
+ *     3 <= top_n <= 64; window >= 1.
+ */
+#ifndef NSA_H_
+#define NSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum nsa_status {
+  NSA_OK = 0,
+  NSA_ERR_INVALID_ARG = 1,         /* null pointer, bad shape, misalignment, bad constant */
+  NSA_ERR_UNSUPPORTED = 2,         /* valid but not implemented here (head_dim, block sizes, device) */
+  NSA_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes < nsa_workspace_size() */
+  NSA_ERR_CUDA = 4                 /* a CUDA runtime call or launch failed */
+};
+
+enum nsa_out_dtype { NSA_OUT_BF16 = 0, NSA_OUT_F32 = 1 };
+
+typedef struct {
+  int32_t n_tokens;      /* prefill: N tokens; decode / compress: cache capacity Lmax */
+  int32_t n_video;       /* prefill: N_v, the NSA-attended prefix (0 <= N_v <= N); rows >= N_v are text */
+  int32_t num_q_heads;   /* Hq */
+  int32_t num_kv_heads;  /* Hkv */
+  int32_t head_dim;      /* d */
+  int32_t cmp_block;     /* l  (compression block length) */
+  int32_t cmp_stride;    /* s  (compression stride) */
+  int32_t sel_block;     /* l' (selection block length) */
+  int32_t top_n;         /* n  (selected blocks per token and group, forced blocks included) */
+  int32_t window;        /* w  (sliding-window length, the query token included) */
+  float softmax_scale;   /* <= 0 selects 1/sqrt(head_dim) */
+  int32_t out_dtype;     /* enum nsa_out_dtype */
+  int32_t batch;         /* decode / compress: number of sequences B (prefill: ignored) */
+} nsa_params_t;
+
+/*
+ * Prefill: one sequence of N tokens.
+ *   q     [N][Hq][d] bf16        k, v [N][Hkv][d] bf16       gates [N][Hq][3] fp32 (cmp, sel, win)
+ *   out   [N][Hq][d] bf16 or fp32 (params->out_dtype)
+ *   out_sel_idx  NULL, or [N_v][Hkv][top_n] int32: the selected block indices of every video
+ *                row, ascending, padded with -1.
+ *   workspace    device scratch of at least nsa_workspace_size(params, 0) bytes (256-byte aligned).
+ * Rows t < N_v follow NSA; rows t >= N_v get dense causal attention (gates unused).
+ */
+int nsa_prefill(const void* q, const void* k, const void* v, const float* gates, const nsa_params_t* params,
+                void* out, int32_t* out_sel_idx, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Decode: one query token per sequence against a KV cache and its compressed cache.
+ *   q       [B][Hq][d] bf16, the query at position seq_lens[b]-1 (its own K/V are in the cache)
+ *   kcache, vcache [B][Lmax][Hkv][d] bf16 (Lmax = params->n_tokens)
+ *   kcmp, vcmp     [B][Ncmp(Lmax)][Hkv][d] bf16, Ncmp(L) = L >= l ? (L-l)/s + 1 : 0, as written by
+ *                  nsa_compress (used as given: block i of sequence b is read only if complete,
+ *                  i*s + l <= seq_lens[b])
+ *   seq_lens [B] int32, 1 <= seq_lens[b] <= Lmax       gates [B][Hq][3] fp32
+ *   out     [B][Hq][d] bf16 or fp32                    out_sel_idx NULL or [B][Hkv][top_n] int32
+ *   workspace at least nsa_workspace_size(params, 1) bytes.
+ */
+int nsa_decode(const void* q, const void* kcache, const void* vcache, const void* kcmp, const void* vcmp,
+               const int32_t* seq_lens, const float* gates, const nsa_params_t* params, void* out,
+               int32_t* out_sel_idx, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Compression only: kcmp[b][i] = bf16_rne(mean_{u<l} k[b][i*s+u]) for every complete block
+ * i < Ncmp(Lmax), same for v. k, v [B][Lmax][Hkv][d]; kcmp, vcmp [B][Ncmp(Lmax)][Hkv][d].
+ * B = params->batch (>= 1), Lmax = params->n_tokens. Builds the decode's compressed cache.
+ */
+int nsa_compress(const void* k, const void* v, const nsa_params_t* params, void* kcmp, void* vcmp, void* stream);
+
+/* Workspace bytes nsa_prefill (is_decode = 0) or nsa_decode (is_decode = 1) needs; 0 if params are invalid. */
+size_t nsa_workspace_size(const nsa_params_t* params, int is_decode);
+
+/*
+ * Where nsa_prefill keeps its intermediates inside the workspace (byte offsets), for
+ * inspection after the stream has been synchronised. Every field is an offset from the
+ * workspace base; layouts are row-major:
+ *   kc, vc   [Ncmp(N_v)][Hkv][d] bf16     o_cmp [N_v][Hq][d] fp32     lse [N_v][Hq] fp32 (natural log)
+ *   scores   [N_v][Hkv][Nsel] fp32, Nsel = ceil(N_v / l'); only entries j <= t/l' are written
+ *   sel_idx  [N_v][Hkv][top_n] int32      o_sel [N_v][Hq][d] fp32
+ * Returns NSA_OK or NSA_ERR_INVALID_ARG.
+ */
+typedef struct {
+  size_t kc, vc, o_cmp, lse, scores, sel_idx, o_sel, total;
+  int32_t n_cmp, n_sel;
+} nsa_prefill_layout_t;
+int nsa_prefill_workspace_layout(const nsa_params_t* params, nsa_prefill_layout_t* layout);
+
+/* Human-readable text of a status code (static storage). */
+const char* nsa_error_string(int status);
+
+/*
+ * Device error word: bit 0 = a kernel's bounded wait timed out (the kernel stopped
+ * early, its output is invalid); bit 1 = a kernel met an out-of-range index and skipped
+ * the access. Synchronises the current device, reads the word and, if `clear` is
+ * non-zero, resets it. Returns NSA_OK or NSA_ERR_CUDA.
+ */
+int nsa_get_device_error(uint32_t* word, int clear);
+
+/* Library version string, e.g. "nsa-b200 0.1.0 sm_100a". */
+const char* nsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NSA_H_ */

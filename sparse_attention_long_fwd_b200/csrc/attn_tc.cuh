@@ -1,0 +1,467 @@
+// attn_tc.cuh -- tcgen05 / TMEM attention tile used by three steps of the NSA forward:
+//
+//   kModeCmp   compressed branch: queries attend to the block summaries Kc/Vc that are
+//              complete at their position (block i visible to t iff i*s + l - 1 <= t).
+//              Also bins the normalised probabilities into selection-block scores,
+//              summed over the GQA group (the selection branch's importance scores;
+//              top168.com article on VideoNSA, section "一、革命性的三重注意机制").
+//   kModeWin   sliding-window branch over tokens (t - w, t], followed by the gated
+//              combine out = g_cmp*o_cmp + g_sel*o_sel + g_win*o_win.
+//   kModeDense dense causal rows for the trailing text tokens of the hybrid scheme
+//              (shd-paper.top page "VideoNSA: ...", abstract: dense attention for text).
+//
+// One CTA owns one query tile: T = floor(128 / G) consecutive tokens times the G query
+// heads of one KV group, packed as MMA rows r = token * G + head (the heads of a GQA
+// group share every key, so they share the B operand). The tile's key range is streamed
+// in 128-key tiles through a TMA ring, twice:
+//   phase 1  S = Q K^T on the tensor core (TMEM accumulator), then each row's exact
+//            log-sum-exp with an online max (no P*V, no output rescaling);
+//   phase 2  S again, P = exp2(S*scale*log2e - lse2) already normalised, written to
+//            shared memory as bf16 and accumulated O += P V in TMEM. Because P is final,
+//            the compressed mode can bin it into block scores in the same pass.
+// The pages' kernel notes (CSDN blog, section 5.1: fixed 64x64 blocks, prefetching the
+// next block while computing the current one, tiling against register pressure) are
+// met here by TMA tiles, an mbarrier ring and TMEM accumulators.
+//
+// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues the
+// MMAs (one elected lane), warps 2..5 (128 threads, one per TMEM lane / MMA row) do the
+// softmax, the score binning and the epilogue. Every wait is bounded (sm100.cuh).
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+#include "sm100.cuh"
+
+namespace nsa {
+
+enum AttnMode { kModeCmp = 0, kModeWin = 1, kModeDense = 2 };
+
+struct AttnArgs {
+  int q_begin, q_end;      // query tokens handled: [q_begin, q_end)
+  int hq, hkv, G, T;       // heads, group size, tokens per tile
+  int n_tiles;             // ceil((q_end - q_begin) / T)
+  float scale_log2;        // softmax_scale * log2(e)
+  int cmp_len, cmp_stride;  // compressed-key visibility (kModeCmp)
+  int window;              // kModeWin
+  int sel_len;             // selection block (kModeCmp scores)
+  float* o_cmp;            // kModeCmp: write [N_v][Hq][d]; kModeWin: read
+  float* lse;              // kModeCmp: write [N_v][Hq] (natural log)
+  float* scores;           // kModeCmp: write [N_v][Hkv][nsel]
+  int nsel;
+  const float* o_sel;      // kModeWin: read [N_v][Hq][d]
+  const float* gates;      // kModeWin: read [N][Hq][3]
+  void* out;               // kModeWin / kModeDense: write [N][Hq][d]
+  int out_f32;
+};
+
+constexpr int kAttnThreads = 192;
+constexpr int kBN = 128;      // keys per tile
+constexpr int kStages = 2;    // TMA ring depth (K and V tiles)
+
+template <int D>
+struct AttnSmem {
+  static constexpr int kChunks = D / 64;             // 64-element (128 B) column chunks
+  static constexpr int kTileBytes = 128 * 128;       // one chunk of a 128-row tile
+  alignas(1024) uint8_t q[kChunks][kTileBytes];
+  alignas(1024) uint8_t k[kStages][kChunks][kTileBytes];
+  alignas(1024) uint8_t v[kStages][kChunks][kTileBytes];
+  alignas(1024) uint8_t p[2][kTileBytes];            // P tile: 128 rows x 128 keys bf16
+  float bins[128][33];
+  uint64_t q_full;
+  uint64_t full[kStages], empty[kStages];
+  uint64_t s_full[2], s_free[2];
+  uint64_t p_full, p_free, o_full, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int jobs_consumed;
+};
+
+__device__ __forceinline__ int ncmp_visible(int t, int l, int s) { return (t + 1 >= l) ? (t + 1 - l) / s + 1 : 0; }
+
+template <int D, int MODE>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_tile_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+                     const __grid_constant__ CUtensorMap vmap, const AttnArgs args) {
+  using Smem = AttnSmem<D>;
+  constexpr int kChunks = Smem::kChunks;
+  constexpr uint32_t kTmemCols = 512;
+  constexpr uint32_t kColO = 256;  // S buffers at columns 0 and 128, O at 256
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int G = args.G, T = args.T;
+  const int g = blockIdx.y;
+  // heavy tiles (most keys) first for the causal modes
+  const int tile = (MODE == kModeWin) ? blockIdx.x : (args.n_tiles - 1 - blockIdx.x);
+  const int t0 = args.q_begin + tile * T;
+  const int t_last = min(t0 + T, args.q_end) - 1;
+  int kb, ke;
+  if (MODE == kModeCmp) {
+    kb = 0;
+    ke = ncmp_visible(t_last, args.cmp_len, args.cmp_stride);
+  } else if (MODE == kModeWin) {
+    kb = max(0, t0 - args.window + 1);
+    ke = t_last + 1;
+  } else {
+    kb = 0;
+    ke = t_last + 1;
+  }
+  const int nkt = (ke - kb + kBN - 1) / kBN;
+  const int njobs = 2 * nkt;
+
+  if (tid == 0) {
+    mbar_init(&sm.q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.s_full[b], 1);
+      mbar_init(&sm.s_free[b], 4);
+    }
+    mbar_init(&sm.p_full, 4);
+    mbar_init(&sm.p_free, 1);
+    mbar_init(&sm.o_full, 1);
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    sm.jobs_consumed = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp >= 2) {
+    // rows T*G .. 127 of the Q tile are never written by TMA: keep them finite (zero)
+    const int r0 = T * G;
+    for (int i = tid - 64; i < (128 - r0) * 8 * kChunks; i += 128) {
+      const int c = i / ((128 - r0) * 8);
+      const int rem = i % ((128 - r0) * 8);
+      *reinterpret_cast<uint4*>(&sm.q[c][(r0 + rem / 8) * 128 + (rem % 8) * 16]) = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort_flag = &sm.abort_flag;
+  int issued = 0;  // producer: jobs whose TMA was issued
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0 && nkt > 0) {
+      tma_prefetch_desc(&qmap);
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&vmap);
+      mbar_arrive_expect_tx(&sm.q_full, kChunks * T * G * 128);
+      for (int c = 0; c < kChunks; ++c) tma_load_3d(&qmap, &sm.q_full, sm.q[c], c * 64, g * G, t0);
+      for (int job = 0; job < njobs; ++job) {
+        const int stage = job % kStages;
+        if (job >= kStages && !mbar_wait(&sm.empty[stage], ((job / kStages) - 1) & 1, abort_flag)) break;
+        const bool p2 = job >= nkt;
+        const int kpos = kb + (p2 ? job - nkt : job) * kBN;
+        mbar_arrive_expect_tx(&sm.full[stage], (p2 ? 2 : 1) * kChunks * Smem::kTileBytes);
+        for (int c = 0; c < kChunks; ++c) tma_load_3d(&kmap, &sm.full[stage], sm.k[stage][c], c * 64, g, kpos);
+        if (p2)
+          for (int c = 0; c < kChunks; ++c) tma_load_3d(&vmap, &sm.full[stage], sm.v[stage][c], c * 64, g, kpos);
+        issued = job + 1;
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0 && nkt > 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, kBN, false, false);
+      constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);
+      bool ok = mbar_wait(&sm.q_full, 0, abort_flag);
+      auto issue_s = [&](int job) -> bool {
+        const int stage = job % kStages;
+        const int b = job & 1;
+        if (!mbar_wait(&sm.full[stage], (job / kStages) & 1, abort_flag)) return false;
+        sm.jobs_consumed = job + 1;
+        if (job >= 2 && !mbar_wait(&sm.s_free[b], ((job >> 1) - 1) & 1, abort_flag)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const int c = k >> 2, kk = k & 3;
+          const uint64_t a = sdesc_sw128(smem_u32(sm.q[c]) + kk * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(smem_u32(sm.k[stage][c]) + kk * 32, 16, 1024);
+          umma_bf16_ss(tmem + b * kBN, a, bd, idS, k > 0 ? 1u : 0u);
+        }
+        umma_commit(&sm.s_full[b]);
+        if (job < nkt) umma_commit(&sm.empty[stage]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int job = 0; ok && job < njobs; ++job) {
+        if (job + 1 < njobs && !issue_s(job + 1)) {
+          ok = false;
+          break;
+        }
+        if (job >= nkt) {
+          const int kt2 = job - nkt;
+          const int stage = job % kStages;
+          if (!mbar_wait(&sm.p_full, kt2 & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < kBN / 16; ++k) {
+            const int c = k >> 2, kk = k & 3;
+            const uint64_t a = sdesc_sw128(smem_u32(sm.p[c]) + kk * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(smem_u32(sm.v[stage][0]) + k * 2048, Smem::kTileBytes, 1024);
+            umma_bf16_ss(tmem + kColO, a, bd, idO, (kt2 > 0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(&sm.p_free);
+          umma_commit(&sm.empty[stage]);
+        }
+      }
+      if (ok) umma_commit(&sm.o_full);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ softmax / epilogue
+    const int q4 = warp & 3;                 // TMEM lane quadrant of this warp
+    const int r = q4 * 32 + lane;            // MMA row
+    const int tok = r / G, hh = r % G;
+    const int t = t0 + tok;
+    const int h = g * G + hh;
+    const bool row_valid = (r < T * G) && (t < args.q_end);
+    int rb = 0, re = 0;                      // visible key range of this row
+    if (row_valid) {
+      if (MODE == kModeCmp) {
+        re = ncmp_visible(t, args.cmp_len, args.cmp_stride);
+      } else if (MODE == kModeWin) {
+        rb = max(0, t - args.window + 1);
+        re = t + 1;
+      } else {
+        re = t + 1;
+      }
+    }
+    const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const float sl2 = args.scale_log2;
+    bool ok = true;
+    // ---- phase 1: exact log-sum-exp (base 2) of each row
+    float m = -INFINITY, lsum = 0.f;
+    for (int kt = 0; kt < nkt && ok; ++kt) {
+      const int b = kt & 1;
+      // tcgen05.ld is warp-collective: every wait result is made warp-uniform
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (kt >> 1) & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const int kbase = kb + kt * kBN;
+#pragma unroll 1
+      for (int cb = 0; cb < kBN / 32; ++cb) {
+        float s[32];
+        __syncwarp();
+        tmem_ld32(trow + b * kBN + cb * 32, s);
+        tmem_wait_ld();
+        float cmax = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int kidx = kbase + cb * 32 + i;
+          s[i] = (kidx >= rb && kidx < re) ? s[i] * sl2 : -INFINITY;
+          cmax = fmaxf(cmax, s[i]);
+        }
+        const float mnew = fmaxf(m, cmax);
+        if (mnew != -INFINITY) {
+          float acc = 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc += ex2_approx(s[i] - mnew);
+          lsum = lsum * ex2_approx(m - mnew) + acc;
+          m = mnew;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.s_free[b]);
+    }
+    const bool has_keys = lsum > 0.f;
+    const float lse2 = has_keys ? m + __log2f(lsum) : INFINITY;
+    // ---- phase 2: normalised probabilities -> P (smem, bf16) and block scores
+    float carry = 0.f;  // half of the last compressed block of the previous tile (kModeCmp)
+    // In the compressed mode the four softmax warps meet at named barriers every tile,
+    // so they must leave this loop together: each iteration ORs their failures.
+    for (int kt2 = 0; kt2 < nkt; ++kt2) {
+      const int job = nkt + kt2;
+      const int b = job & 1;
+      if (ok) ok = mbar_wait(&sm.s_full[b], (job >> 1) & 1, abort_flag);
+      if (ok && kt2 > 0) ok = mbar_wait(&sm.p_free, (kt2 - 1) & 1, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      const bool any_fail = (MODE == kModeCmp) ? named_bar_any(2, 128, !ok) : !ok;
+      if (any_fail) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int kbase = kb + kt2 * kBN;
+#pragma unroll 1
+      for (int cb = 0; cb < kBN / 32; ++cb) {
+        float s[32];
+        __syncwarp();
+        tmem_ld32(trow + b * kBN + cb * 32, s);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int kidx = kbase + cb * 32 + i;
+          s[i] = (kidx >= rb && kidx < re) ? ex2_approx(s[i] * sl2 - lse2) : 0.f;
+        }
+        if (MODE == kModeCmp) {
+          // compressed block i covers tokens [16i, 16i+32); selection block j covers
+          // [64j, 64j+64): blocks 4j..4j+2 lie inside j, blocks 4j-1 and 4j+3 half inside.
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const float half_last = 0.5f * s[4 * u + 3];
+            sm.bins[r][cb * 8 + u] = carry + s[4 * u] + s[4 * u + 1] + s[4 * u + 2] + half_last;
+            carry = half_last;
+          }
+        }
+        // P row r, keys cb*32 .. cb*32+31 -> chunk cb/2, columns (cb%2)*32 ..
+        uint8_t* pc = sm.p[cb >> 1];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          uint4 w;
+          w.x = pack_bf16x2(s[8 * u + 0], s[8 * u + 1]);
+          w.y = pack_bf16x2(s[8 * u + 2], s[8 * u + 3]);
+          w.z = pack_bf16x2(s[8 * u + 4], s[8 * u + 5]);
+          w.w = pack_bf16x2(s[8 * u + 6], s[8 * u + 7]);
+          *reinterpret_cast<uint4*>(pc + sw128_offset(r, (cb & 1) * 32 + 8 * u)) = w;
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&sm.s_free[b]);
+        mbar_arrive(&sm.p_full);
+      }
+      if (MODE == kModeCmp) {
+        named_bar_sync(1, 128);
+        const int nb = T * 32;
+        for (int i = tid - 64; i < nb; i += 128) {
+          const int tk = i >> 5, bb = i & 31;
+          const int tt = t0 + tk;
+          const int j = kt2 * 32 + bb;
+          if (tt < args.q_end && j <= tt / args.sel_len) {
+            float acc = 0.f;
+            for (int x = 0; x < G; ++x) acc += sm.bins[tk * G + x][bb];
+            args.scores[(static_cast<size_t>(tt) * args.hkv + g) * args.nsel + j] = acc;
+          }
+        }
+        named_bar_sync(1, 128);
+      }
+    }
+    if (MODE == kModeCmp && ok) {
+      // the carried half-block after the last tile lands in selection block nkt*32;
+      // when no key tile exists at all, that is block 0 with score 0.
+      sm.bins[r][0] = carry;
+      named_bar_sync(1, 128);
+      for (int tk = tid - 64; tk < T; tk += 128) {
+        const int tt = t0 + tk;
+        const int j = nkt * 32;
+        if (tt < args.q_end && j <= tt / args.sel_len) {
+          float acc = 0.f;
+          for (int x = 0; x < G; ++x) acc += sm.bins[tk * G + x][0];
+          args.scores[(static_cast<size_t>(tt) * args.hkv + g) * args.nsel + j] = acc;
+        }
+      }
+    }
+    // ---- epilogue (every lane loads its TMEM row; only valid rows are stored)
+    if (ok && nkt > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_full, 0, abort_flag));
+      tc_fence_after();
+    }
+    if (ok) {
+      const size_t orow = (static_cast<size_t>(t) * args.hq + h) * D;
+      float g0 = 0.f, g1 = 0.f, g2 = 0.f;
+      if (MODE == kModeWin && row_valid) {
+        g0 = args.gates[(static_cast<size_t>(t) * args.hq + h) * 3 + 0];
+        g1 = args.gates[(static_cast<size_t>(t) * args.hq + h) * 3 + 1];
+        g2 = args.gates[(static_cast<size_t>(t) * args.hq + h) * 3 + 2];
+      }
+#pragma unroll 1
+      for (int cb = 0; cb < D / 32; ++cb) {
+        float o[32];
+        __syncwarp();
+        if (nkt > 0) {
+          tmem_ld32(trow + kColO + cb * 32, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0.f;
+        }
+        if (!row_valid) {
+          // nothing to store for padding rows
+        } else if (MODE == kModeCmp) {
+          float4* dst = reinterpret_cast<float4*>(args.o_cmp + orow + cb * 32);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) dst[u] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+        } else {
+          if (MODE == kModeWin) {
+            const float4* oc = reinterpret_cast<const float4*>(args.o_cmp + orow + cb * 32);
+            const float4* os = reinterpret_cast<const float4*>(args.o_sel + orow + cb * 32);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const float4 a = oc[u], c = os[u];
+              o[4 * u + 0] = g0 * a.x + g1 * c.x + g2 * o[4 * u + 0];
+              o[4 * u + 1] = g0 * a.y + g1 * c.y + g2 * o[4 * u + 1];
+              o[4 * u + 2] = g0 * a.z + g1 * c.z + g2 * o[4 * u + 2];
+              o[4 * u + 3] = g0 * a.w + g1 * c.w + g2 * o[4 * u + 3];
+            }
+          }
+          if (args.out_f32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.out) + orow + cb * 32);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) dst[u] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) + orow + cb * 32);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              dst[u] = make_uint4(pack_bf16x2(o[8 * u], o[8 * u + 1]), pack_bf16x2(o[8 * u + 2], o[8 * u + 3]),
+                                  pack_bf16x2(o[8 * u + 4], o[8 * u + 5]), pack_bf16x2(o[8 * u + 6], o[8 * u + 7]));
+          }
+        }
+      }
+      if (MODE == kModeCmp && row_valid)
+        args.lse[static_cast<size_t>(t) * args.hq + h] = has_keys ? lse2 * 0.69314718055994530942f : -INFINITY;
+    }
+    tc_fence_before();
+  }
+
+  // ------------------------------------------------------------------ teardown
+  __syncthreads();
+  if (*abort_flag) {
+    // drain: wait (bounded) for TMA loads that were issued but never consumed and for
+    // MMAs still in flight, so no async write lands after the CTA exits.
+    if (warp == 0 && lane == 0) {
+      if (nkt > 0) {
+        const long long t_start = clock64();
+        while (!mbar_test(&sm.q_full, 0) && clock64() - t_start < kWaitCycles) {
+        }
+      }
+      for (int job = sm.jobs_consumed; job < issued; ++job) {
+        const long long t_start = clock64();
+        while (!mbar_test(&sm.full[job % kStages], (job / kStages) & 1) && clock64() - t_start < kWaitCycles) {
+        }
+      }
+    }
+    if (warp == 1 && lane == 0 && nkt > 0) {
+      umma_commit(&sm.drain);
+      const long long t_start = clock64();
+      while (!mbar_test(&sm.drain, 0) && clock64() - t_start < kWaitCycles) {
+      }
+    }
+    __syncwarp();
+    __syncthreads();
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace nsa

@@ -1,0 +1,455 @@
+// nsa_api.cu -- the C ABI declared in include/nsa.h: argument validation, workspace
+// layout, TMA tensor maps and kernel launches for the NSA forward pass on sm_100a.
+// The whole library is this one translation unit (the kernels are header-only).
+#include <cuda_runtime.h>
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "nsa.h"
+#include "sm100.cuh"
+#include "tma_host.h"
+#include "pool.cuh"
+#include "attn_tc.cuh"
+#include "topn.cuh"
+#include "sel.cuh"
+#include "decode.cuh"
+
+namespace {
+
+using nsa::AttnArgs;
+
+constexpr size_t kAlign = 256;
+constexpr int kMaxWindowDecode = 4096;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+int ncmp_of(int T, int l, int s) { return T >= l ? (T - l) / s + 1 : 0; }
+int nsel_of(int T, int ls) { return (T + ls - 1) / ls; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Checks shared by every entry point. Returns NSA_OK or an error code.
+int check_common(const nsa_params_t* p) {
+  if (p == nullptr) return NSA_ERR_INVALID_ARG;
+  if (p->n_tokens < 1 || p->num_q_heads < 1 || p->num_kv_heads < 1 || p->head_dim < 1) return NSA_ERR_INVALID_ARG;
+  if (p->num_q_heads % p->num_kv_heads != 0) return NSA_ERR_INVALID_ARG;
+  if (p->cmp_block < 1 || p->cmp_stride < 1 || p->sel_block < 1 || p->window < 1 || p->top_n < 1)
+    return NSA_ERR_INVALID_ARG;
+  if (p->out_dtype != NSA_OUT_BF16 && p->out_dtype != NSA_OUT_F32) return NSA_ERR_INVALID_ARG;
+  if (p->head_dim != 64 && p->head_dim != 128) return NSA_ERR_UNSUPPORTED;
+  if (p->num_q_heads / p->num_kv_heads > 16) return NSA_ERR_UNSUPPORTED;
+  if (p->cmp_block != 32 || p->cmp_stride != 16 || p->sel_block != 64) return NSA_ERR_UNSUPPORTED;
+  if (p->top_n < 3 || p->top_n > 64) return NSA_ERR_UNSUPPORTED;
+  // element counts of the largest tensors must stay within 2^31 rows for the TMA maps
+  if (static_cast<long long>(p->n_tokens) * p->num_q_heads > (1LL << 31)) return NSA_ERR_UNSUPPORTED;
+  return NSA_OK;
+}
+
+int check_device() {
+  static std::mutex mu;
+  static int cached[64];
+  static bool init = false;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!init) {
+    for (int& c : cached) c = -1;
+    init = true;
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return NSA_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return NSA_ERR_UNSUPPORTED;
+  if (cached[dev] < 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return NSA_ERR_CUDA;
+    cached[dev] = (major == 10 && minor == 0) ? 1 : 0;
+  }
+  return cached[dev] == 1 ? NSA_OK : NSA_ERR_UNSUPPORTED;
+}
+
+struct PrefillLayout {
+  size_t kc, vc, o_cmp, lse, scores, sel_idx, o_sel, total;
+  int ncmp, nsel;
+};
+
+PrefillLayout prefill_layout(const nsa_params_t* p) {
+  PrefillLayout L{};
+  const int nv = p->n_video, hq = p->num_q_heads, hkv = p->num_kv_heads, d = p->head_dim;
+  L.ncmp = ncmp_of(nv, p->cmp_block, p->cmp_stride);
+  L.nsel = nsel_of(nv, p->sel_block);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + (bytes > 0 ? bytes : 1));
+    return at;
+  };
+  const size_t cmp_rows = static_cast<size_t>(L.ncmp > 0 ? L.ncmp : 1);
+  L.kc = take(cmp_rows * hkv * d * 2);
+  L.vc = take(cmp_rows * hkv * d * 2);
+  L.o_cmp = take(static_cast<size_t>(nv) * hq * d * 4);
+  L.lse = take(static_cast<size_t>(nv) * hq * 4);
+  L.scores = take(static_cast<size_t>(nv) * hkv * (L.nsel > 0 ? L.nsel : 1) * 4);
+  L.sel_idx = take(static_cast<size_t>(nv) * hkv * p->top_n * 4);
+  L.o_sel = take(static_cast<size_t>(nv) * hq * d * 4);
+  L.total = off;
+  return L;
+}
+
+struct DecodeLayout {
+  size_t logits, part, o_cmp, lse, scores, sel_idx, o_sel, o_win, total;
+  int ncmax, nsel_max, nsplit;
+};
+
+DecodeLayout decode_layout(const nsa_params_t* p) {
+  DecodeLayout L{};
+  const int B = p->batch, hq = p->num_q_heads, hkv = p->num_kv_heads, d = p->head_dim;
+  const int G = hq / hkv;
+  L.ncmax = ncmp_of(p->n_tokens, p->cmp_block, p->cmp_stride);
+  L.nsel_max = nsel_of(p->n_tokens, p->sel_block);
+  L.nsplit = (L.ncmax + 511) / 512;
+  if (L.nsplit < 1) L.nsplit = 1;
+  if (L.nsplit > 64) L.nsplit = 64;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + (bytes > 0 ? bytes : 1));
+    return at;
+  };
+  L.logits = take(static_cast<size_t>(B) * hkv * G * (L.ncmax > 0 ? L.ncmax : 1) * 4);
+  L.part = take(static_cast<size_t>(B) * hkv * L.nsplit * G * (2 + d) * 4);
+  L.o_cmp = take(static_cast<size_t>(B) * hq * d * 4);
+  L.lse = take(static_cast<size_t>(B) * hq * 4);
+  L.scores = take(static_cast<size_t>(B) * hkv * L.nsel_max * 4);
+  L.sel_idx = take(static_cast<size_t>(B) * hkv * p->top_n * 4);
+  L.o_sel = take(static_cast<size_t>(B) * hq * d * 4);
+  L.o_win = take(static_cast<size_t>(B) * hq * d * 4);
+  L.total = off;
+  return L;
+}
+
+// NSA_DEBUG_SYNC=1 in the environment: synchronise after every launch and report each
+// kernel's completion (and any error) on stderr. Off by default; costs a sync per kernel.
+bool debug_sync() {
+  static const bool on = [] {
+    const char* e = std::getenv("NSA_DEBUG_SYNC");
+    return e != nullptr && e[0] == '1';
+  }();
+  return on;
+}
+
+int launch_status(const char* name = "kernel", cudaStream_t st = nullptr) {
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess && debug_sync()) {
+    std::fprintf(stderr, "[nsa] %s launched\n", name);
+    std::fflush(stderr);
+    e = cudaStreamSynchronize(st);
+    unsigned int word = 0;
+    cudaMemcpyFromSymbol(&word, nsa::g_device_error, sizeof(word));
+    std::fprintf(stderr, "[nsa] %s finished: %s, device error word %u\n", name, cudaGetErrorString(e), word);
+    std::fflush(stderr);
+  }
+  return e == cudaSuccess ? NSA_OK : NSA_ERR_CUDA;
+}
+
+template <typename K>
+int set_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) ==
+                 cudaSuccess
+             ? NSA_OK
+             : NSA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ launchers
+int launch_pool(const void* k, const void* v, void* kc, void* vc, int nseq, int T, int hkv, int d, int ncmp, int l,
+                int s, cudaStream_t st) {
+  if (ncmp <= 0) return NSA_OK;
+  const long long threads = static_cast<long long>(nseq) * ncmp * hkv * (d / 2);
+  const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+  nsa::pool_kernel<<<dim3(blocks, 1, 2), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(kc),
+      static_cast<__nv_bfloat16*>(vc), nseq, T, hkv, d, ncmp, l, s);
+  return launch_status("pool", st);
+}
+
+template <int D, int MODE>
+int launch_attn(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a,
+                cudaStream_t st) {
+  if (a.n_tiles <= 0) return NSA_OK;
+  const size_t smem = sizeof(nsa::AttnSmem<D>) + 1024;
+  auto kern = nsa::attn_tile_kernel<D, MODE>;
+  if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
+  kern<<<dim3(a.n_tiles, a.hkv), nsa::kAttnThreads, smem, st>>>(qm, km, vm, a);
+  return launch_status(MODE == nsa::kModeCmp ? "attn_cmp" : MODE == nsa::kModeWin ? "attn_win" : "attn_dense", st);
+}
+
+template <int D>
+int prefill_impl(const nsa_params_t* p, const void* q, const void* k, const void* v, const float* gates, void* out,
+                 int32_t* out_sel_idx, uint8_t* ws, cudaStream_t st) {
+  const PrefillLayout L = prefill_layout(p);
+  const int N = p->n_tokens, nv = p->n_video, hq = p->num_q_heads, hkv = p->num_kv_heads;
+  const int G = hq / hkv;
+  const int T = 128 / G;
+  const float scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(D));
+  const float sl2 = scale * 1.4426950408889634f;
+  int rc;
+  CUtensorMap qmap, kmap, vmap, kcmap, vcmap;
+  const uint64_t qs1 = static_cast<uint64_t>(D) * 2, qs2 = static_cast<uint64_t>(hq) * D * 2;
+  const uint64_t ks1 = static_cast<uint64_t>(D) * 2, ks2 = static_cast<uint64_t>(hkv) * D * 2;
+  if (!nsa::make_tmap_bf16_3d(&qmap, q, D, hq, N, qs1, qs2, 64, G, T) ||
+      !nsa::make_tmap_bf16_3d(&kmap, k, D, hkv, N, ks1, ks2, 64, 1, nsa::kBN) ||
+      !nsa::make_tmap_bf16_3d(&vmap, v, D, hkv, N, ks1, ks2, 64, 1, nsa::kBN))
+    return NSA_ERR_CUDA;
+  AttnArgs a{};
+  a.hq = hq;
+  a.hkv = hkv;
+  a.G = G;
+  a.T = T;
+  a.scale_log2 = sl2;
+  a.cmp_len = p->cmp_block;
+  a.cmp_stride = p->cmp_stride;
+  a.window = p->window;
+  a.sel_len = p->sel_block;
+  a.nsel = L.nsel;
+  a.out = out;
+  a.out_f32 = p->out_dtype == NSA_OUT_F32;
+  if (nv > 0) {
+    auto* kc = ws + L.kc;
+    auto* vc = ws + L.vc;
+    const int ncmp_rows = L.ncmp > 0 ? L.ncmp : 1;
+    if (!nsa::make_tmap_bf16_3d(&kcmap, kc, D, hkv, ncmp_rows, ks1, ks2, 64, 1, nsa::kBN) ||
+        !nsa::make_tmap_bf16_3d(&vcmap, vc, D, hkv, ncmp_rows, ks1, ks2, 64, 1, nsa::kBN))
+      return NSA_ERR_CUDA;
+    // 1. compression: Kc, Vc of the video prefix
+    if ((rc = launch_pool(k, v, kc, vc, 1, nv, hkv, D, L.ncmp, p->cmp_block, p->cmp_stride, st)) != NSA_OK) return rc;
+    // 2. compressed branch + block scores
+    a.q_begin = 0;
+    a.q_end = nv;
+    a.n_tiles = (nv + T - 1) / T;
+    a.o_cmp = reinterpret_cast<float*>(ws + L.o_cmp);
+    a.lse = reinterpret_cast<float*>(ws + L.lse);
+    a.scores = reinterpret_cast<float*>(ws + L.scores);
+    if ((rc = launch_attn<D, nsa::kModeCmp>(qmap, kcmap, vcmap, a, st)) != NSA_OK) return rc;
+    // 3. top-n selection
+    {
+      const int nitems = nv * hkv;
+      const int nwords = (L.nsel + 31) / 32;
+      const size_t smem = static_cast<size_t>(nsa::kTopnWarps) * (L.nsel + nwords) * 4;
+      if (set_smem(nsa::topn_kernel, smem) != NSA_OK) return NSA_ERR_CUDA;
+      int blocks = (nitems + nsa::kTopnWarps - 1) / nsa::kTopnWarps;
+      if (blocks > 148 * 32) blocks = 148 * 32;
+      nsa::topn_kernel<<<blocks, nsa::kTopnWarps * 32, smem, st>>>(
+          a.scores, nitems, hkv, L.nsel, p->sel_block, p->top_n, reinterpret_cast<int32_t*>(ws + L.sel_idx),
+          out_sel_idx);
+      if ((rc = launch_status("topn", st)) != NSA_OK) return rc;
+    }
+    // 4. selected branch
+    {
+      const size_t smem = sizeof(nsa::SelSmem<D>) + 128;
+      auto kern = nsa::sel_branch_kernel<D>;
+      if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
+      const int blocks = (nv * hkv + nsa::kSelWarps - 1) / nsa::kSelWarps;
+      kern<<<blocks, nsa::kSelWarps * 32, smem, st>>>(
+          static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+          static_cast<const __nv_bfloat16*>(v), reinterpret_cast<const int32_t*>(ws + L.sel_idx), nv, hq, hkv,
+          p->top_n, p->sel_block, sl2, reinterpret_cast<float*>(ws + L.o_sel));
+      if ((rc = launch_status("sel_branch", st)) != NSA_OK) return rc;
+    }
+    // 5. sliding window + gated combine -> out rows [0, N_v)
+    a.o_sel = reinterpret_cast<const float*>(ws + L.o_sel);
+    a.gates = gates;
+    if ((rc = launch_attn<D, nsa::kModeWin>(qmap, kmap, vmap, a, st)) != NSA_OK) return rc;
+  }
+  // 6. trailing text rows: dense causal attention -> out rows [N_v, N)
+  if (N > nv) {
+    a.q_begin = nv;
+    a.q_end = N;
+    a.n_tiles = (N - nv + T - 1) / T;
+    if ((rc = launch_attn<D, nsa::kModeDense>(qmap, kmap, vmap, a, st)) != NSA_OK) return rc;
+  }
+  return NSA_OK;
+}
+
+template <int D>
+int decode_impl(const nsa_params_t* p, const void* q, const void* kcache, const void* vcache, const void* kcmp,
+                const void* vcmp, const int32_t* seq_lens, const float* gates, void* out, int32_t* out_sel_idx,
+                uint8_t* ws, cudaStream_t st) {
+  const DecodeLayout L = decode_layout(p);
+  nsa::DecArgs a{};
+  a.batch = p->batch;
+  a.lmax = p->n_tokens;
+  a.hq = p->num_q_heads;
+  a.hkv = p->num_kv_heads;
+  a.G = a.hq / a.hkv;
+  a.d = D;
+  a.ncmax = L.ncmax;
+  a.nsplit = L.nsplit;
+  a.cmp_len = p->cmp_block;
+  a.cmp_stride = p->cmp_stride;
+  a.sel_len = p->sel_block;
+  a.top_n = p->top_n;
+  a.window = p->window;
+  a.nsel_max = L.nsel_max;
+  const float scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(D));
+  a.sl2 = scale * 1.4426950408889634f;
+  a.logits = reinterpret_cast<float*>(ws + L.logits);
+  a.part = reinterpret_cast<float*>(ws + L.part);
+  a.o_cmp = reinterpret_cast<float*>(ws + L.o_cmp);
+  a.lse = reinterpret_cast<float*>(ws + L.lse);
+  a.scores = reinterpret_cast<float*>(ws + L.scores);
+  a.sel_idx = reinterpret_cast<int32_t*>(ws + L.sel_idx);
+  a.o_sel = reinterpret_cast<float*>(ws + L.o_sel);
+  a.o_win = reinterpret_cast<float*>(ws + L.o_win);
+  const auto* qq = static_cast<const __nv_bfloat16*>(q);
+  int rc;
+  const size_t smem = sizeof(nsa::DecSmem<D>) + 128;
+  {
+    auto kern = nsa::dec_cmp_kernel<D>;
+    if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
+    kern<<<dim3(L.nsplit, a.batch * a.hkv), nsa::kDecWarps * 32, smem, st>>>(
+        qq, static_cast<const __nv_bfloat16*>(kcmp), static_cast<const __nv_bfloat16*>(vcmp), seq_lens, a);
+    if ((rc = launch_status("dec_cmp", st)) != NSA_OK) return rc;
+  }
+  {
+    const size_t ssm = (static_cast<size_t>(L.nsel_max) + L.nsel_max / 32 + 1 + 16) * 4;
+    auto kern = nsa::dec_select_kernel<D>;
+    if (set_smem(kern, ssm) != NSA_OK) return NSA_ERR_CUDA;
+    kern<<<a.batch * a.hkv, 256, ssm, st>>>(seq_lens, a, out_sel_idx);
+    if ((rc = launch_status("dec_select", st)) != NSA_OK) return rc;
+  }
+  {
+    auto kern = nsa::dec_branch_kernel<D>;
+    if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
+    kern<<<dim3(a.batch * a.hkv, 2), nsa::kDecWarps * 32, smem, st>>>(
+        qq, static_cast<const __nv_bfloat16*>(kcache), static_cast<const __nv_bfloat16*>(vcache), seq_lens, a);
+    if ((rc = launch_status("dec_branch", st)) != NSA_OK) return rc;
+  }
+  {
+    const long long n = static_cast<long long>(a.batch) * a.hq * D;
+    nsa::dec_combine_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
+        gates, a.o_cmp, a.o_sel, a.o_win, out, p->out_dtype == NSA_OUT_F32, a.batch * a.hq, D);
+    if ((rc = launch_status("dec_combine", st)) != NSA_OK) return rc;
+  }
+  return NSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* nsa_version(void) { return "nsa-b200 0.1.0 sm_100a"; }
+
+const char* nsa_error_string(int status) {
+  switch (status) {
+    case NSA_OK:
+      return "ok";
+    case NSA_ERR_INVALID_ARG:
+      return "invalid argument (null pointer, bad shape, misalignment or bad constant)";
+    case NSA_ERR_UNSUPPORTED:
+      return "unsupported configuration or device (needs sm_100, head_dim 64/128, l=32, s=16, l'=64, 3<=top_n<=64)";
+    case NSA_ERR_WORKSPACE_TOO_SMALL:
+      return "workspace smaller than nsa_workspace_size()";
+    case NSA_ERR_CUDA:
+      return "a CUDA runtime call or kernel launch failed";
+    default:
+      return "unknown status";
+  }
+}
+
+size_t nsa_workspace_size(const nsa_params_t* params, int is_decode) {
+  if (check_common(params) != NSA_OK) return 0;
+  if (is_decode) {
+    if (params->batch < 1) return 0;
+    return decode_layout(params).total;
+  }
+  if (params->n_video < 0 || params->n_video > params->n_tokens) return 0;
+  return prefill_layout(params).total;
+}
+
+int nsa_prefill_workspace_layout(const nsa_params_t* params, nsa_prefill_layout_t* layout) {
+  if (layout == nullptr || check_common(params) != NSA_OK || params->n_video < 0 ||
+      params->n_video > params->n_tokens)
+    return NSA_ERR_INVALID_ARG;
+  const PrefillLayout L = prefill_layout(params);
+  layout->kc = L.kc;
+  layout->vc = L.vc;
+  layout->o_cmp = L.o_cmp;
+  layout->lse = L.lse;
+  layout->scores = L.scores;
+  layout->sel_idx = L.sel_idx;
+  layout->o_sel = L.o_sel;
+  layout->total = L.total;
+  layout->n_cmp = L.ncmp;
+  layout->n_sel = L.nsel;
+  return NSA_OK;
+}
+
+int nsa_prefill(const void* q, const void* k, const void* v, const float* gates, const nsa_params_t* params,
+                void* out, int32_t* out_sel_idx, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_common(params);
+  if (rc != NSA_OK) return rc;
+  if (params->n_video < 0 || params->n_video > params->n_tokens) return NSA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !out || !workspace || (!gates && params->n_video > 0)) return NSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (gates && !aligned16(gates)) ||
+      (out_sel_idx && !aligned16(out_sel_idx)) || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+    return NSA_ERR_INVALID_ARG;
+  if (nsel_of(params->n_video, params->sel_block) > 8192) return NSA_ERR_UNSUPPORTED;
+  if (workspace_bytes < prefill_layout(params).total) return NSA_ERR_WORKSPACE_TOO_SMALL;
+  if ((rc = check_device()) != NSA_OK) return rc;
+  auto* ws = static_cast<uint8_t*>(workspace);
+  auto st = static_cast<cudaStream_t>(stream);
+  if (params->head_dim == 64) return prefill_impl<64>(params, q, k, v, gates, out, out_sel_idx, ws, st);
+  return prefill_impl<128>(params, q, k, v, gates, out, out_sel_idx, ws, st);
+}
+
+int nsa_decode(const void* q, const void* kcache, const void* vcache, const void* kcmp, const void* vcmp,
+               const int32_t* seq_lens, const float* gates, const nsa_params_t* params, void* out,
+               int32_t* out_sel_idx, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_common(params);
+  if (rc != NSA_OK) return rc;
+  if (params->batch < 1) return NSA_ERR_INVALID_ARG;
+  if (params->window > kMaxWindowDecode) return NSA_ERR_UNSUPPORTED;
+  if (!q || !kcache || !vcache || !kcmp || !vcmp || !seq_lens || !gates || !out || !workspace)
+    return NSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(kcmp) || !aligned16(vcmp) ||
+      !aligned16(out) || (out_sel_idx && !aligned16(out_sel_idx)) ||
+      (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+    return NSA_ERR_INVALID_ARG;
+  if (nsel_of(params->n_tokens, params->sel_block) > 8192) return NSA_ERR_UNSUPPORTED;
+  if (workspace_bytes < decode_layout(params).total) return NSA_ERR_WORKSPACE_TOO_SMALL;
+  if ((rc = check_device()) != NSA_OK) return rc;
+  auto* ws = static_cast<uint8_t*>(workspace);
+  auto st = static_cast<cudaStream_t>(stream);
+  if (params->head_dim == 64)
+    return decode_impl<64>(params, q, kcache, vcache, kcmp, vcmp, seq_lens, gates, out, out_sel_idx, ws, st);
+  return decode_impl<128>(params, q, kcache, vcache, kcmp, vcmp, seq_lens, gates, out, out_sel_idx, ws, st);
+}
+
+int nsa_compress(const void* k, const void* v, const nsa_params_t* params, void* kcmp, void* vcmp, void* stream) {
+  int rc = check_common(params);
+  if (rc != NSA_OK) return rc;
+  if (params->batch < 1 || !k || !v || !kcmp || !vcmp) return NSA_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(kcmp) || !aligned16(vcmp)) return NSA_ERR_INVALID_ARG;
+  if ((rc = check_device()) != NSA_OK) return rc;
+  const int ncmp = ncmp_of(params->n_tokens, params->cmp_block, params->cmp_stride);
+  return launch_pool(k, v, kcmp, vcmp, params->batch, params->n_tokens, params->num_kv_heads, params->head_dim, ncmp,
+                     params->cmp_block, params->cmp_stride, static_cast<cudaStream_t>(stream));
+}
+
+int nsa_get_device_error(uint32_t* word, int clear) {
+  if (word == nullptr) return NSA_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return NSA_ERR_CUDA;
+  unsigned int w = 0;
+  if (cudaMemcpyFromSymbol(&w, nsa::g_device_error, sizeof(w)) != cudaSuccess) return NSA_ERR_CUDA;
+  *word = w;
+  if (clear) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(nsa::g_device_error, &zero, sizeof(zero)) != cudaSuccess) return NSA_ERR_CUDA;
+  }
+  return NSA_OK;
+}
+
+}  // extern "C"

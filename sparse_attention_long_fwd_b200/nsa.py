@@ -1,0 +1,229 @@
+"""Python binding of the C ABI in include/nsa.h (argument marshalling only).
+
+Every function named like the C entry point takes torch tensors (or raw device
+addresses) and forwards them unchanged; all computation happens in the sm_100a kernels
+of libnsa_b200.so. There is no fallback: if the library is missing or fails to load,
+every call raises NsaLibraryError.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+NSA_OK = 0
+NSA_ERR_INVALID_ARG = 1
+NSA_ERR_UNSUPPORTED = 2
+NSA_ERR_WORKSPACE_TOO_SMALL = 3
+NSA_ERR_CUDA = 4
+
+NSA_OUT_BF16 = 0
+NSA_OUT_F32 = 1
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnsa_b200.so")
+
+EXPORTED = (
+    "nsa_prefill", "nsa_decode", "nsa_compress", "nsa_workspace_size", "nsa_prefill_workspace_layout",
+    "nsa_error_string", "nsa_get_device_error", "nsa_version",
+)
+
+
+class NsaLibraryError(RuntimeError):
+    pass
+
+
+class NsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {nsa_error_string(status)} (status {status})")
+        self.status = status
+
+
+class NsaParams(ctypes.Structure):
+    _fields_ = [
+        ("n_tokens", ctypes.c_int32), ("n_video", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
+        ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("cmp_block", ctypes.c_int32),
+        ("cmp_stride", ctypes.c_int32), ("sel_block", ctypes.c_int32), ("top_n", ctypes.c_int32),
+        ("window", ctypes.c_int32), ("softmax_scale", ctypes.c_float), ("out_dtype", ctypes.c_int32),
+        ("batch", ctypes.c_int32),
+    ]
+
+
+class NsaPrefillLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in ("kc", "vc", "o_cmp", "lse", "scores", "sel_idx", "o_sel", "total")] + [
+        ("n_cmp", ctypes.c_int32), ("n_sel", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libnsa_b200.so (built by sparse_attention_long_fwd_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise NsaLibraryError(f"{path} is missing: build it with `python -m sparse_attention_long_fwd_b200.build`")
+    try:
+        lib = ctypes.CDLL(path)
+    except OSError as e:  # pragma: no cover
+        raise NsaLibraryError(f"cannot load {path}: {e}") from e
+    P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    PP = ctypes.POINTER(NsaParams)
+    lib.nsa_prefill.argtypes = [P, P, P, P, PP, P, P, P, S, P]
+    lib.nsa_prefill.restype = I
+    lib.nsa_decode.argtypes = [P, P, P, P, P, P, P, PP, P, P, P, S, P]
+    lib.nsa_decode.restype = I
+    lib.nsa_compress.argtypes = [P, P, PP, P, P, P]
+    lib.nsa_compress.restype = I
+    lib.nsa_workspace_size.argtypes = [PP, I]
+    lib.nsa_workspace_size.restype = S
+    lib.nsa_prefill_workspace_layout.argtypes = [PP, ctypes.POINTER(NsaPrefillLayout)]
+    lib.nsa_prefill_workspace_layout.restype = I
+    lib.nsa_error_string.argtypes = [I]
+    lib.nsa_error_string.restype = ctypes.c_char_p
+    lib.nsa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), I]
+    lib.nsa_get_device_error.restype = I
+    lib.nsa_version.argtypes = []
+    lib.nsa_version.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def make_params(n_tokens: int, n_video: int | None = None, num_q_heads: int = 28, num_kv_heads: int = 4,
+                head_dim: int = 128, cmp_block: int = 32, cmp_stride: int = 16, sel_block: int = 64, top_n: int = 16,
+                window: int = 512, softmax_scale: float = 0.0, out_dtype: int = NSA_OUT_F32,
+                batch: int = 0) -> NsaParams:
+    return NsaParams(n_tokens, n_tokens if n_video is None else n_video, num_q_heads, num_kv_heads, head_dim,
+                     cmp_block, cmp_stride, sel_block, top_n, window, softmax_scale, out_dtype, batch)
+
+
+def _addr(x) -> int | None:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+# ------------------------------------------------------------------ C entry points, same names
+
+def nsa_prefill(q, k, v, gates, params: NsaParams, out, out_sel_idx, workspace, workspace_bytes: int,
+                stream=None) -> int:
+    return load_library().nsa_prefill(_addr(q), _addr(k), _addr(v), _addr(gates), ctypes.byref(params), _addr(out),
+                                      _addr(out_sel_idx), _addr(workspace), workspace_bytes, _stream(stream))
+
+
+def nsa_decode(q, kcache, vcache, kcmp, vcmp, seq_lens, gates, params: NsaParams, out, out_sel_idx, workspace,
+               workspace_bytes: int, stream=None) -> int:
+    return load_library().nsa_decode(_addr(q), _addr(kcache), _addr(vcache), _addr(kcmp), _addr(vcmp),
+                                     _addr(seq_lens), _addr(gates), ctypes.byref(params), _addr(out),
+                                     _addr(out_sel_idx), _addr(workspace), workspace_bytes, _stream(stream))
+
+
+def nsa_compress(k, v, params: NsaParams, kcmp, vcmp, stream=None) -> int:
+    return load_library().nsa_compress(_addr(k), _addr(v), ctypes.byref(params), _addr(kcmp), _addr(vcmp),
+                                       _stream(stream))
+
+
+def nsa_workspace_size(params: NsaParams, is_decode: bool) -> int:
+    return int(load_library().nsa_workspace_size(ctypes.byref(params), int(bool(is_decode))))
+
+
+def nsa_prefill_workspace_layout(params: NsaParams) -> dict:
+    lay = NsaPrefillLayout()
+    rc = load_library().nsa_prefill_workspace_layout(ctypes.byref(params), ctypes.byref(lay))
+    if rc != NSA_OK:
+        raise NsaError(rc, "nsa_prefill_workspace_layout")
+    return {n: getattr(lay, n) for n, _ in NsaPrefillLayout._fields_}
+
+
+def nsa_error_string(status: int) -> str:
+    return load_library().nsa_error_string(status).decode()
+
+
+def nsa_get_device_error(clear: bool = True) -> int:
+    w = ctypes.c_uint32(0)
+    rc = load_library().nsa_get_device_error(ctypes.byref(w), int(bool(clear)))
+    if rc != NSA_OK:
+        raise NsaError(rc, "nsa_get_device_error")
+    return int(w.value)
+
+
+def nsa_version() -> str:
+    return load_library().nsa_version().decode()
+
+
+# ------------------------------------------------------------------ torch conveniences
+
+def _check(rc: int, where: str):
+    if rc != NSA_OK:
+        raise NsaError(rc, where)
+
+
+def alloc_workspace(params: NsaParams, is_decode: bool, device) -> torch.Tensor:
+    n = nsa_workspace_size(params, is_decode)
+    if n == 0:
+        raise NsaError(NSA_ERR_INVALID_ARG, "nsa_workspace_size")
+    # torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gates: torch.Tensor, *, n_video: int | None = None,
+            top_n: int = 16, window: int = 512, softmax_scale: float = 0.0, out_dtype=torch.float32,
+            return_sel: bool = False, workspace: torch.Tensor | None = None, stream=None):
+    """NSA prefill of one sequence: q [N,Hq,d], k/v [N,Hkv,d] bf16, gates [N,Hq,3] fp32 (device tensors)."""
+    N, hq, d = q.shape
+    hkv = k.shape[1]
+    p = make_params(N, n_video, hq, hkv, d, top_n=top_n, window=window, softmax_scale=softmax_scale,
+                    out_dtype=NSA_OUT_F32 if out_dtype == torch.float32 else NSA_OUT_BF16)
+    out = torch.empty((N, hq, d), dtype=out_dtype, device=q.device)
+    sel = torch.empty((p.n_video, hkv, top_n), dtype=torch.int32, device=q.device) if return_sel else None
+    if workspace is None:
+        workspace = alloc_workspace(p, False, q.device)
+    _check(nsa_prefill(q, k, v, gates, p, out, sel, workspace, workspace.numel(), stream), "nsa_prefill")
+    return (out, sel) if return_sel else out
+
+
+def compress(k: torch.Tensor, v: torch.Tensor, stream=None):
+    """Compressed cache of a [B, L, Hkv, d] (or [L, Hkv, d]) bf16 K/V pair."""
+    squeeze = k.dim() == 3
+    if squeeze:
+        k, v = k.unsqueeze(0), v.unsqueeze(0)
+    B, L, hkv, d = k.shape
+    p = make_params(L, L, hkv, hkv, d, batch=B)
+    nc = (L - 32) // 16 + 1 if L >= 32 else 0
+    kc = torch.empty((B, nc, hkv, d), dtype=k.dtype, device=k.device)
+    vc = torch.empty_like(kc)
+    _check(nsa_compress(k, v, p, kc, vc, stream), "nsa_compress")
+    return (kc[0], vc[0]) if squeeze else (kc, vc)
+
+
+def decode(q, kcache, vcache, kcmp, vcmp, seq_lens, gates, *, top_n: int = 16, window: int = 512,
+           softmax_scale: float = 0.0, out_dtype=torch.float32, return_sel: bool = False,
+           workspace: torch.Tensor | None = None, stream=None):
+    """NSA decode: q [B,Hq,d], caches [B,Lmax,Hkv,d], compressed caches [B,Ncmp,Hkv,d], seq_lens [B] int32."""
+    B, hq, d = q.shape
+    Lmax, hkv = kcache.shape[1], kcache.shape[2]
+    p = make_params(Lmax, Lmax, hq, hkv, d, top_n=top_n, window=window, softmax_scale=softmax_scale,
+                    out_dtype=NSA_OUT_F32 if out_dtype == torch.float32 else NSA_OUT_BF16, batch=B)
+    out = torch.empty((B, hq, d), dtype=out_dtype, device=q.device)
+    sel = torch.empty((B, hkv, top_n), dtype=torch.int32, device=q.device) if return_sel else None
+    if workspace is None:
+        workspace = alloc_workspace(p, True, q.device)
+    _check(nsa_decode(q, kcache, vcache, kcmp, vcmp, seq_lens, gates, p, out, sel, workspace, workspace.numel(),
+                      stream), "nsa_decode")
+    return (out, sel) if return_sel else out
+
+
+def default_scale(d: int) -> float:
+    return 1.0 / math.sqrt(d)

@@ -1,0 +1,105 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every entry
+point declared in include/nsa.h, validates arguments and reports error codes, and
+computes consistent workspace layouts. No kernel is launched here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_attention_long_fwd_b200 import nsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "nsa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nsa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = nsa.load_library()
+    declared = _declared_functions()
+    assert "nsa_prefill" in declared and "nsa_decode" in declared and "nsa_compress" in declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(nsa.EXPORTED) <= set(declared)
+
+
+def test_version_and_error_strings():
+    assert "sm_100a" in nsa.nsa_version()
+    for s in range(5):
+        assert nsa.nsa_error_string(s)
+    assert nsa.nsa_error_string(99) == "unknown status"
+
+
+def _p(**kw):
+    base = dict(n_tokens=4096, n_video=4096, num_q_heads=28, num_kv_heads=4, head_dim=128, top_n=16, window=512)
+    base.update(kw)
+    return nsa.make_params(**base)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(head_dim=96), nsa.NSA_ERR_UNSUPPORTED),
+    (dict(num_q_heads=30), nsa.NSA_ERR_INVALID_ARG),          # Hq % Hkv != 0
+    (dict(num_q_heads=68, num_kv_heads=4), nsa.NSA_ERR_UNSUPPORTED),  # G = 17 > 16
+    (dict(top_n=0), nsa.NSA_ERR_INVALID_ARG),
+    (dict(top_n=2), nsa.NSA_ERR_UNSUPPORTED),
+    (dict(top_n=65), nsa.NSA_ERR_UNSUPPORTED),
+    (dict(cmp_block=64), nsa.NSA_ERR_UNSUPPORTED),
+    (dict(window=0), nsa.NSA_ERR_INVALID_ARG),
+    (dict(n_video=5000), nsa.NSA_ERR_INVALID_ARG),
+    (dict(n_tokens=0, n_video=0), nsa.NSA_ERR_INVALID_ARG),
+])
+def test_prefill_validation_codes(kw, code):
+    p = _p(**kw)
+    fake = 1 << 20  # never dereferenced: validation fails first
+    assert nsa.nsa_prefill(fake, fake, fake, fake, p, fake, None, fake, 1 << 40, None) == code
+
+
+def test_null_and_misaligned_pointers_rejected():
+    p = _p()
+    f = 1 << 20
+    assert nsa.nsa_prefill(None, f, f, f, p, f, None, f, 1 << 40, None) == nsa.NSA_ERR_INVALID_ARG
+    assert nsa.nsa_prefill(f + 2, f, f, f, p, f, None, f, 1 << 40, None) == nsa.NSA_ERR_INVALID_ARG
+    assert nsa.nsa_prefill(f, f, f, f, p, f, None, f + 16, 1 << 40, None) == nsa.NSA_ERR_INVALID_ARG
+    assert nsa.nsa_prefill(f, f, f, f, p, f, None, f, 1000, None) == nsa.NSA_ERR_WORKSPACE_TOO_SMALL
+    pd = nsa.make_params(1024, batch=0)
+    assert nsa.nsa_decode(f, f, f, f, f, f, f, pd, f, None, f, 1 << 40, None) == nsa.NSA_ERR_INVALID_ARG
+    pd = nsa.make_params(1024, batch=2, window=5000)
+    assert nsa.nsa_decode(f, f, f, f, f, f, f, pd, f, None, f, 1 << 40, None) == nsa.NSA_ERR_UNSUPPORTED
+    assert nsa.nsa_compress(None, f, nsa.make_params(64, batch=1), f, f, None) == nsa.NSA_ERR_INVALID_ARG
+
+
+def test_prefill_layout_is_aligned_and_disjoint():
+    for n, nv in ((131072, 131072), (36352, 36096), (2048, 2048), (300, 0), (20, 20)):
+        p = _p(n_tokens=n, n_video=nv)
+        lay = nsa.nsa_prefill_workspace_layout(p)
+        assert lay["total"] == nsa.nsa_workspace_size(p, False)
+        ncmp = (nv - 32) // 16 + 1 if nv >= 32 else 0
+        assert lay["n_cmp"] == ncmp and lay["n_sel"] == (nv + 63) // 64
+        keys = ["kc", "vc", "o_cmp", "lse", "scores", "sel_idx", "o_sel"]
+        offs = [lay[k] for k in keys] + [lay["total"]]
+        assert all(o % 256 == 0 for o in offs)
+        sizes = [max(ncmp, 1) * 4 * 128 * 2] * 2 + [nv * 28 * 128 * 4, nv * 28 * 4, nv * 4 * max(lay["n_sel"], 1) * 4,
+                                                    nv * 4 * 16 * 4, nv * 28 * 128 * 4]
+        for i, sz in enumerate(sizes):
+            assert offs[i] + sz <= offs[i + 1], keys[i]
+
+
+def test_decode_workspace_scales_with_batch():
+    a = nsa.nsa_workspace_size(nsa.make_params(131072, batch=1), True)
+    b = nsa.nsa_workspace_size(nsa.make_params(131072, batch=64), True)
+    assert 0 < a < b
+    assert nsa.nsa_workspace_size(nsa.make_params(131072, head_dim=80, batch=64), True) == 0
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(nsa.NsaLibraryError):
+        nsa._lib_saved = nsa._lib
+        try:
+            nsa._lib = None
+            nsa.load_library(str(tmp_path / "absent.so"))
+        finally:
+            nsa._lib = nsa._lib_saved

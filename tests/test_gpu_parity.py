@@ -1,0 +1,182 @@
+"""GPU parity: the CUDA path (called through the C ABI) against the fp64 oracle.
+
+Sizes the oracle finishes in seconds compare every row and every intermediate; the
+full-size workloads (36K hybrid, 128K, 64 x 128K decode) compare sampled rows, in the
+same launch configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as orc
+from sparse_attention_long_fwd_b200 import nsa
+from sparse_attention_long_fwd_b200.inputs import WORKLOADS, bf16_bits, decode_inputs, prefill_inputs, scaled
+
+from nsa_check import (MAX_ABS, MEAN_ABS, assert_close, check_selection, compare_prefill_rows, oracle_cfg,
+                       run_prefill, sample_rows)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _prefill_case(w, seed, rows=None, out_dtype=torch.float32, nthreads=0):
+    q, k, v, g = prefill_inputs(w, seed=seed, device=DEV)
+    out, sel, ws, lay = run_prefill(w, q, k, v, g, out_dtype=out_dtype)
+    if rows is None:
+        rows = np.arange(w.n_tokens)
+    return compare_prefill_rows(w, q, k, v, g, rows, out, sel, ws, lay, nthreads=nthreads)
+
+
+def test_compress_bit_exact():
+    w = scaled(WORKLOADS["v128k"], n_tokens=4099, n_video=4099)
+    q, k, v, g = prefill_inputs(w, seed=3, device=DEV)
+    kc, vc = nsa.compress(k, v)
+    torch.cuda.synchronize()
+    kb, vb = bf16_bits(k), bf16_bits(v)
+    assert np.array_equal(bf16_bits(kc), orc.compress(kb))
+    assert np.array_equal(bf16_bits(vc), orc.compress(vb))
+
+
+def test_compress_batched_bit_exact():
+    w = scaled(WORKLOADS["decode64x128k"], batch=3, n_tokens=1000)
+    q, kc, vc, g, sl = decode_inputs(w, seed=4, device=DEV)
+    kcmp, vcmp = nsa.compress(kc, vc)
+    torch.cuda.synchronize()
+    for b in range(3):
+        assert np.array_equal(bf16_bits(kcmp[b]), orc.compress(bf16_bits(kc[b])))
+        assert np.array_equal(bf16_bits(vcmp[b]), orc.compress(bf16_bits(vc[b])))
+
+
+def test_prefill_tiny_all_rows():
+    """The 2048-token, 4-head, d=64 workload: every row and every intermediate."""
+    st = _prefill_case(WORKLOADS["tiny"], seed=0)
+    print(st)
+
+
+@pytest.mark.parametrize("n,hq,hkv,d,top_n,window", [
+    (1000, 28, 4, 128, 16, 512),     # several tiles, ragged tail (1000 = 55 * 18 + 10)
+    (777, 8, 1, 64, 5, 100),         # G = 8, d = 64, tiny window
+    (1500, 16, 16, 128, 4, 300),     # G = 1 (no GQA)
+    (640, 12, 3, 128, 64, 2048),     # top_n and window cover everything: dense special case
+])
+def test_prefill_shapes_all_rows(n, hq, hkv, d, top_n, window):
+    w = scaled(WORKLOADS["v128k"], n_tokens=n, n_video=n, hq=hq, hkv=hkv, d=d, top_n=top_n, window=window)
+    st = _prefill_case(w, seed=n)
+    print(st)
+
+
+def test_prefill_hybrid_small_all_rows():
+    w = scaled(WORKLOADS["qwen36k_hybrid"], n_tokens=1300, n_video=1100)
+    st = _prefill_case(w, seed=5)
+    print(st)
+
+
+def test_prefill_edge_lengths():
+    for n in (1, 17, 31, 32, 33, 64, 65, 129):
+        w = scaled(WORKLOADS["qwen36k_hybrid"], n_tokens=n, n_video=n)
+        _prefill_case(w, seed=100 + n)
+    # all text (no video prefix): dense causal only
+    w = scaled(WORKLOADS["qwen36k_hybrid"], n_tokens=300, n_video=0)
+    _prefill_case(w, seed=7)
+
+
+def test_prefill_bf16_output():
+    w = scaled(WORKLOADS["qwen36k_hybrid"], n_tokens=900, n_video=800)
+    _prefill_case(w, seed=9, out_dtype=torch.bfloat16)
+
+
+def test_prefill_one_hot_gates_isolate_branches():
+    w = scaled(WORKLOADS["qwen36k_hybrid"], n_tokens=700, n_video=700)
+    q, k, v, g = prefill_inputs(w, seed=11, device=DEV)
+    outs = []
+    for which in range(3):
+        gg = torch.zeros_like(g)
+        gg[..., which] = 1.0
+        out, sel, ws, lay = run_prefill(w, q, k, v, gg)
+        outs.append((out.clone(), ws, lay))
+    from nsa_check import ws_view
+    ocmp = ws_view(outs[0][1], outs[0][2]["o_cmp"], (700, w.hq, w.d), torch.float32)
+    osel = ws_view(outs[1][1], outs[1][2]["o_sel"], (700, w.hq, w.d), torch.float32)
+    assert torch.equal(outs[0][0], ocmp)
+    assert torch.equal(outs[1][0], osel)
+
+
+def test_prefill_qwen36k_hybrid_sampled():
+    w = WORKLOADS["qwen36k_hybrid"]
+    q, k, v, g = prefill_inputs(w, seed=1, device=DEV)
+    out, sel, ws, lay = run_prefill(w, q, k, v, g)
+    rows = sample_rows(w.n_video, w.n_tokens, 64, seed=1)
+    st = compare_prefill_rows(w, q, k, v, g, rows, out, sel, ws, lay)
+    print(st)
+
+
+def test_prefill_v128k_sampled():
+    w = WORKLOADS["v128k"]
+    q, k, v, g = prefill_inputs(w, seed=2, device=DEV)
+    out, sel, ws, lay = run_prefill(w, q, k, v, g)
+    rows = sample_rows(w.n_video, w.n_tokens, 48, seed=2)
+    st = compare_prefill_rows(w, q, k, v, g, rows, out, sel, ws, lay)
+    print(st)
+
+
+@pytest.mark.parametrize("name", ["sweep128k_n4_w256", "sweep128k_n48_w1024"])
+def test_prefill_sweep_points_sampled(name):
+    w = WORKLOADS[name]
+    q, k, v, g = prefill_inputs(w, seed=2, device=DEV)
+    out, sel, ws, lay = run_prefill(w, q, k, v, g)
+    rows = sample_rows(w.n_video, w.n_tokens, 16, seed=3)
+    compare_prefill_rows(w, q, k, v, g, rows, out, sel, ws, lay, check_intermediates=False)
+
+
+# ---------------------------------------------------------------- decode
+
+def _decode_case(w, seed, seq_lens=None, seqs=None):
+    q, kc, vc, g, sl = decode_inputs(w, seed=seed, device=DEV, seq_lens=seq_lens)
+    kcmp, vcmp = nsa.compress(kc, vc)
+    out, sel = nsa.decode(q, kc, vc, kcmp, vcmp, sl, g, top_n=w.top_n, window=w.window, return_sel=True)
+    torch.cuda.synchronize()
+    assert nsa.nsa_get_device_error(clear=True) == 0
+    cfg = orc.OracleConfig(w.n_tokens, w.n_tokens, w.hq, w.hkv, w.d, top_n=w.top_n, window=w.window)
+    qb, kb, vb, kcb, vcb = (bf16_bits(t) for t in (q, kc, vc, kcmp, vcmp))
+    gh, slh = g.cpu().numpy(), sl.cpu().numpy()
+    if seqs is None:
+        seqs = np.arange(w.batch)
+    o = orc.decode(cfg, qb, kb, vb, kcb, vcb, slh, gh, seqs=seqs)
+    gsel = sel.cpu().numpy()[seqs]
+    replay, ties = check_selection(gsel, o["sel"], o["scores"])
+    ref = o["out"]
+    if replay:
+        o2 = orc.decode(cfg, qb, kb, vb, kcb, vcb, slh, gh, seqs=np.asarray(seqs)[replay], sel_override=gsel[replay])
+        ref[replay] = o2["out"]
+    return assert_close(out.cpu().numpy()[seqs], ref, "decode out"), ties
+
+
+def test_decode_small_varied_lengths():
+    w = scaled(WORKLOADS["decode64x128k"], batch=8, n_tokens=3000)
+    lens = [3000, 1, 31, 32, 33, 64, 1000, 2049]
+    print(_decode_case(w, seed=21, seq_lens=lens))
+
+
+def test_decode_d64_window_covers_all():
+    w = scaled(WORKLOADS["decode64x128k"], batch=4, n_tokens=700, hq=8, hkv=2, d=64, top_n=12, window=1024)
+    print(_decode_case(w, seed=22, seq_lens=[700, 350, 64, 129]))
+
+
+def test_decode_64x128k_sampled():
+    w = WORKLOADS["decode64x128k"]
+    print(_decode_case(w, seed=4, seqs=np.arange(0, 64, 4)))
+
+
+# ---------------------------------------------------------------- error paths on a device
+
+def test_device_errors_are_reported_not_raised():
+    w = scaled(WORKLOADS["tiny"], n_tokens=256, n_video=256)
+    q, k, v, g = prefill_inputs(w, seed=0, device=DEV)
+    p = nsa.make_params(256, 256, 4, 1, 64, top_n=4, window=64)
+    ws = nsa.alloc_workspace(p, False, DEV)
+    out = torch.empty((256, 4, 64), device=DEV)
+    assert nsa.nsa_prefill(q, k, v, g, p, out, None, ws, ws.numel() - 256) == nsa.NSA_ERR_WORKSPACE_TOO_SMALL
+    assert nsa.nsa_prefill(q, k, v, g, p, out, None, ws[1:], ws.numel() - 1) == nsa.NSA_ERR_INVALID_ARG
+    bad = nsa.make_params(256, 256, 4, 1, 96, top_n=4, window=64)
+    assert nsa.nsa_prefill(q, k, v, g, bad, out, None, ws, ws.numel()) == nsa.NSA_ERR_UNSUPPORTED
+    assert nsa.nsa_get_device_error(clear=True) == 0
