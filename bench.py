@@ -1,0 +1,457 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 NSA forward pass.
+
+Headline: NSA prefill of one 131,072-token video sequence (2048 frames x 64 tokens,
+Hq=28, Hkv=4, d=128, l=32, s=16, l'=64, n=16, w=512, per-frame correlated keys) in
+video tokens/s, with attended TFLOP/s against the measured bf16 peak; the 64 x 128K
+decode's HBM GB/s is reported beside it. One step = one nsa_prefill call over inputs
+already resident in HBM (every kernel of the path: pooling, compressed branch with
+block scores, top-n, selected branch, window + gated combine). L2 is flushed (a
+256 MiB write) before every timed step, outside the step's events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+
+Under torchrun each rank runs its own sequence on its own GPU (independent problems,
+no collective on the data path): value = all ranks' tokens / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_attention_long_fwd_b200 import nsa  # noqa: E402
+from sparse_attention_long_fwd_b200.inputs import WORKLOADS, decode_inputs, prefill_inputs  # noqa: E402
+
+METRIC = "NSA prefill video tokens/s at 128K & TFLOP/s vs peak; decode HBM GB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PREFILL_STAGES = ["pool", "cmp_attn_scores", "topn", "sel_branch", "win_combine", "dense_text"]
+DECODE_STAGES = ["dec_cmp", "dec_select", "dec_branches", "dec_combine"]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------- work counts
+
+def prefill_counts(w):
+    """Attended keys per head for every query row, from the definition (no GPU output)."""
+    t = np.arange(w.n_video, dtype=np.int64)
+    nc = np.where(t + 1 >= w.cmp_len, (t + 1 - w.cmp_len) // w.cmp_stride + 1, 0)
+    jt = t // w.sel_len
+    nblk = np.minimum(w.top_n, jt + 1)
+    sel = (nblk - 1) * w.sel_len + (t % w.sel_len) + 1
+    win = np.minimum(w.window, t + 1)
+    text = np.arange(w.n_video, w.n_tokens, dtype=np.int64) + 1
+    per_key = 4.0 * w.d * w.hq  # QK^T and PV multiply-adds, 2 flops each
+    return {
+        "cmp_flops": per_key * nc.sum(), "sel_flops": per_key * sel.sum(), "win_flops": per_key * win.sum(),
+        "text_flops": per_key * text.sum(),
+        "keys_per_head": {"cmp": int(nc.sum()), "sel": int(sel.sum()), "win": int(win.sum()),
+                          "text": int(text.sum())},
+        "dense_causal_pairs": int(w.n_tokens) * (int(w.n_tokens) + 1) // 2,
+    }
+
+
+def decode_bytes(w, seq_lens, sel):
+    """Algorithmic HBM bytes of one decode step: visible compressed K/V, the union of selected
+    and window tokens of every (sequence, group), q, gates and the bf16 output."""
+    row = w.d * 2
+    total = 0
+    for b in range(w.batch):
+        L = int(seq_lens[b])
+        nc = (L - w.cmp_len) // w.cmp_stride + 1 if L >= w.cmp_len else 0
+        total += nc * w.hkv * row * 2
+        for g in range(w.hkv):
+            toks = np.zeros(L, dtype=bool)
+            toks[max(0, L - w.window):] = True
+            for j in sel[b, g]:
+                if j >= 0:
+                    toks[j * w.sel_len: min(L, (j + 1) * w.sel_len)] = True
+            total += int(toks.sum()) * row * 2
+    total += w.batch * w.hq * (w.d * 2 + 3 * 4 + w.d * 2)
+    return total
+
+
+# ---------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ["pci.bus_id", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device: int):
+        self.bus = None
+        try:
+            pr = torch.cuda.get_device_properties(device)
+            self.bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+        except Exception:
+            pass
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}", "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == len(self.FIELDS):
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = self.rows
+        if self.bus is not None:
+            mine = [r for r in rows if r[0].upper().endswith(self.bus[-12:])]
+            rows = mine or rows
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------- helpers
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def timed_steps(fn, steps, warmup, flush, n_stage_events):
+    """Run warmup + timed steps; per step: flush L2 (untimed), events around fn()."""
+    for _ in range(warmup):
+        flush.zero_()
+        fn(None)
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_stage_events)] for _ in range(steps)]
+    for ev in stage_ev:  # torch creates the CUDA event on its first record: do that before handing it over
+        for e in ev:
+            e.record()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()
+        starts[i].record()
+        fn(stage_ev[i])
+        ends[i].record()
+    torch.cuda.synchronize()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    return step_ms, stage_ev
+
+
+def stage_times(stage_ev, names, nrec):
+    """Average duration of each recorded stage over the timed steps."""
+    out = {}
+    for j in range(min(nrec, len(names))):
+        ms = [ev[j].elapsed_time(ev[j + 1]) for ev in stage_ev]
+        out[names[j]] = sum(ms) / len(ms)
+    return out
+
+
+# ---------------------------------------------------------------------------- arms
+
+def run_b200(args, world, rank, local):
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peaks_src = load_peaks()
+    w = WORKLOADS[args.workload]
+    counts = prefill_counts(w)
+    q, k, v, g = prefill_inputs(w, seed=2 + rank, device=dev)
+    p = nsa.make_params(w.n_tokens, w.n_video, w.hq, w.hkv, w.d, w.cmp_len, w.cmp_stride, w.sel_len, w.top_n,
+                        w.window, out_dtype=nsa.NSA_OUT_BF16)
+    ws = nsa.alloc_workspace(p, False, dev)
+    out = torch.empty((w.n_tokens, w.hq, w.d), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    n_stages = 5 + (1 if w.n_tokens > w.n_video else 0)
+
+    def step(events):
+        nsa.nsa_profile_stages(events or [])
+        rc = nsa.nsa_prefill(q, k, v, g, p, out, None, ws, ws.numel())
+        if rc != nsa.NSA_OK:
+            raise nsa.NsaError(rc, "nsa_prefill")
+
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    step_ms, stage_ev = timed_steps(step, args.steps, args.warmup, flush, n_stages + 1)
+    clk = clocks.stop()
+    nsa.nsa_profile_stages([])
+    barrier(world)
+    assert nsa.nsa_get_device_error(clear=True) == 0, "device error word set during the benchmark"
+    total_ms = max_over_ranks(sum(step_ms), world)
+    ms_per_step = total_ms / args.steps
+    tokens = w.n_video * world
+    value = tokens / (ms_per_step / 1e3)
+    stages = stage_times(stage_ev, PREFILL_STAGES, n_stages)
+    flops = counts["cmp_flops"] + counts["sel_flops"] + counts["win_flops"] + counts["text_flops"]
+    tflops = flops / (sum(step_ms) / args.steps / 1e3) / 1e12
+
+    # dominant kernel and its roofline (live CUDA-event durations of this run)
+    dom = max(stages, key=stages.get)
+    stage_flops = {"cmp_attn_scores": counts["cmp_flops"], "sel_branch": counts["sel_flops"],
+                   "win_combine": counts["win_flops"], "dense_text": counts["text_flops"]}
+    peak_t = peaks["bf16_tflops_sustained"]
+    if dom in stage_flops:
+        ach = stage_flops[dom] / (stages[dom] / 1e3) / 1e12
+        roofline = {"kernel": dom, "bound": "tensor", "achieved": round(ach, 2), "peak": peak_t, "unit": "TFLOP/s",
+                    "frac": round(ach / peak_t, 4), "traffic": None,
+                    "peak_source": f"{peaks_src} bf16_tflops_sustained (kernel timed inside a long step loop)",
+                    "algorithmic": f"{stage_flops[dom]:.4e} FLOP per launch (attended keys only)"}
+    else:
+        roofline = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": None, "traffic": None}
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "video tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{w.name}: one {w.n_tokens}-token sequence ({w.n_tokens // 64} frames x 64 tokens), "
+                               f"Hq={w.hq}, Hkv={w.hkv}, d={w.d}, l={w.cmp_len}, s={w.cmp_stride}, l'={w.sel_len}, "
+                               f"n={w.top_n}, w={w.window}, bf16 in/out", "n_tokens": w.n_tokens,
+                   "n_video": w.n_video, "top_n": w.top_n, "window": w.window,
+                   "l2": "flushed (256 MiB write) before every timed step; inputs also exceed L2",
+                   "parallelism": f"independent sequence per rank x{world}"},
+        "attended_tflops": round(tflops, 2), "attended_frac_of_peak": round(tflops / peak_t, 4),
+        "attended_keys_per_head": counts["keys_per_head"],
+        "attended_fraction_of_dense_pairs": round(sum(counts["keys_per_head"].values()) / counts["dense_causal_pairs"], 4),
+        "stages_ms": {kk: round(vv, 4) for kk, vv in stages.items()},
+        "roofline": roofline, "clocks": clk, "gpu_launches": n_stages * args.steps,
+    }
+
+    # end to end through the public call: pinned host inputs in, bf16 output back, every step
+    qh, kh, vh, gh = (t.cpu().pin_memory() for t in (q, k, v, g))
+    outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh, gh))
+    d2h = outh.numel() * outh.element_size()
+
+    def e2e_step(events):
+        q.copy_(qh, non_blocking=True)
+        k.copy_(kh, non_blocking=True)
+        v.copy_(vh, non_blocking=True)
+        g.copy_(gh, non_blocking=True)
+        step(None)
+        outh.copy_(out, non_blocking=True)
+
+    barrier(world)
+    e2e_ms, _ = timed_steps(e2e_step, args.steps, min(args.warmup, 3), flush, 0)
+    barrier(world)
+    e2e_total = max_over_ranks(sum(e2e_ms), world)
+    result["e2e"] = {"value": round(tokens / (e2e_total / args.steps / 1e3), 1), "unit": "video tokens/s",
+                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                     "ms_per_step": round(e2e_total / args.steps, 3)}
+    del qh, kh, vh, gh, outh
+
+    if not args.no_decode:
+        result["decode"] = run_decode(args, dev, peaks, peaks_src, flush, world)
+        result["gpu_launches"] += 4 * args.steps
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, q, k, v, g, args.cpu_seconds)
+    return result
+
+
+def run_decode(args, dev, peaks, peaks_src, flush, world):
+    w = WORKLOADS["decode64x128k"]
+    q, kc, vc, g, sl = decode_inputs(w, seed=4, device=dev)
+    kcmp, vcmp = nsa.compress(kc, vc)
+    p = nsa.make_params(w.n_tokens, w.n_tokens, w.hq, w.hkv, w.d, top_n=w.top_n, window=w.window,
+                        out_dtype=nsa.NSA_OUT_BF16, batch=w.batch)
+    ws = nsa.alloc_workspace(p, True, dev)
+    out = torch.empty((w.batch, w.hq, w.d), dtype=torch.bfloat16, device=dev)
+    sel = torch.empty((w.batch, w.hkv, w.top_n), dtype=torch.int32, device=dev)
+
+    def step(events):
+        nsa.nsa_profile_stages(events or [])
+        rc = nsa.nsa_decode(q, kc, vc, kcmp, vcmp, sl, g, p, out, sel, ws, ws.numel())
+        if rc != nsa.NSA_OK:
+            raise nsa.NsaError(rc, "nsa_decode")
+
+    steps = max(args.steps, 20)
+    step_ms, stage_ev = timed_steps(step, steps, args.warmup, flush, 5)
+    nsa.nsa_profile_stages([])
+    assert nsa.nsa_get_device_error(clear=True) == 0
+    total = max_over_ranks(sum(step_ms), world)
+    ms = total / steps
+    nbytes = decode_bytes(w, sl.cpu().numpy(), sel.cpu().numpy())
+    gbs = nbytes / (ms / 1e3) / 1e9
+    stages = stage_times(stage_ev, DECODE_STAGES, 4)
+    cmp_bytes = w.batch * ((w.n_tokens - 32) // 16 + 1) * w.hkv * w.d * 2 * 2
+    cmp_gbs = cmp_bytes / (stages["dec_cmp"] / 1e3) / 1e9
+    del kc, vc
+    return {"workload": "decode64x128k: 64 sequences x 131,072-token bf16 cache, Hq=28, Hkv=4, d=128, n=16, w=512",
+            "ms_per_step": round(ms, 4), "hbm_gbs": round(gbs * world, 1), "unit": "GB/s",
+            "algorithmic_bytes_per_step": nbytes, "frac_of_peak": round(gbs / peaks["hbm_gbs"], 4),
+            "peak_gbs": peaks["hbm_gbs"], "peak_source": f"{peaks_src} hbm_gbs",
+            "steps": steps, "stages_ms": {kk: round(vv, 4) for kk, vv in stages.items()},
+            "dec_cmp_roofline": {"bound": "hbm", "achieved": round(cmp_gbs, 1), "peak": peaks["hbm_gbs"],
+                                 "unit": "GB/s", "frac": round(cmp_gbs / peaks["hbm_gbs"], 4),
+                                 "algorithmic": f"{cmp_bytes} bytes per launch (compressed K and V read once)"}}
+
+
+def cpu_baseline(w, q, k, v, g, seconds):
+    """The fp64 oracle, as it stands, on this host's cores over a stratified row sample."""
+    from oracle import oracle as orc  # test infrastructure: the CPU baseline only
+    from sparse_attention_long_fwd_b200.inputs import bf16_bits
+
+    qb, kb, vb = bf16_bits(q), bf16_bits(k), bf16_bits(v)
+    gh = g.cpu().numpy()
+    cfg = orc.OracleConfig(w.n_tokens, w.n_video, w.hq, w.hkv, w.d, w.cmp_len, w.cmp_stride, w.sel_len, w.top_n,
+                           w.window)
+    t0 = time.perf_counter()
+    kc, vc = orc.compress(kb[: w.n_video]), orc.compress(vb[: w.n_video])
+    t_cmp = time.perf_counter() - t0
+    # probe, then size the sample for roughly `seconds` of work
+    probe = np.linspace(0, w.n_video - 1, 32).astype(np.int32)
+    t0 = time.perf_counter()
+    orc.prefill_rows(cfg, qb, kb, vb, gh, probe, kc=kc, vc=vc, want=())
+    t_probe = time.perf_counter() - t0
+    nrows = int(min(w.n_video, max(64, 32 * seconds / max(t_probe, 1e-3))))
+    rows = np.linspace(0, w.n_video - 1, nrows).astype(np.int32)
+    t0 = time.perf_counter()
+    orc.prefill_rows(cfg, qb, kb, vb, gh, rows, kc=kc, vc=vc, want=())
+    t_rows = time.perf_counter() - t0
+    est = t_cmp + t_rows * w.n_video / nrows
+    return {"value": round(w.n_video / est, 2), "unit": "video tokens/s", "cores": orc.max_threads(), "kind": "oracle",
+            "sample": f"{nrows} query rows evenly spaced over the {w.n_video}-token workload (all heads, all "
+                      f"branches) plus the full compression; time extrapolated by rows",
+            "seconds_measured": round(t_cmp + t_rows, 2)}
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the fp64 oracle on the host cores, same workload and metric."""
+    if rank != 0:
+        return None
+    from oracle import oracle as orc
+    from sparse_attention_long_fwd_b200.inputs import bf16_bits
+
+    w = WORKLOADS[args.workload]
+    q, k, v, g = prefill_inputs(w, seed=2, device="cpu")
+    qb, kb, vb = bf16_bits(q), bf16_bits(k), bf16_bits(v)
+    gh = g.numpy()
+    cfg = orc.OracleConfig(w.n_tokens, w.n_video, w.hq, w.hkv, w.d, w.cmp_len, w.cmp_stride, w.sel_len, w.top_n,
+                           w.window)
+    t0 = time.perf_counter()
+    kc, vc = orc.compress(kb[: w.n_video]), orc.compress(vb[: w.n_video])
+    t_cmp = time.perf_counter() - t0
+    rows_per_step = 256
+    rng = np.random.default_rng(0)
+    times = []
+    for i in range(args.warmup + args.steps):
+        # stratified: one row from each of rows_per_step equal slices of the sequence
+        edges = np.linspace(0, w.n_video, rows_per_step + 1).astype(np.int64)
+        rows = np.array([rng.integers(a, max(a + 1, b)) for a, b in zip(edges[:-1], edges[1:])], dtype=np.int32)
+        t0 = time.perf_counter()
+        orc.prefill_rows(cfg, qb, kb, vb, gh, rows, kc=kc, vc=vc, want=())
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    per_step = statistics.mean(times) * w.n_video / rows_per_step + t_cmp
+    value = w.n_video / per_step
+    cores = orc.max_threads()
+    return {
+        "metric": METRIC, "value": round(value, 2), "unit": "video tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(per_step * 1e3, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": f"{w.name}: one {w.n_tokens}-token sequence, Hq={w.hq}, Hkv={w.hkv}, d={w.d}, "
+                               f"n={w.top_n}, w={w.window}", "n_tokens": w.n_tokens},
+        "cpu_baseline": {"value": round(value, 2), "unit": "video tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {rows_per_step} rows, one per equal slice of the sequence, "
+                                   f"extrapolated to all {w.n_video} rows, plus the full compression"},
+        "e2e": {"value": round(value, 2), "unit": "video tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    ap.add_argument("--workload", default="v128k", choices=[k for k, v in WORKLOADS.items() if not v.is_decode])
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "b200":
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, world, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    world, rank, local = dist_setup()
+    try:
+        res = run_b200(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

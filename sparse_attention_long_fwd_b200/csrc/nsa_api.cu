@@ -141,8 +141,21 @@ bool debug_sync() {
   return on;
 }
 
+// Caller-registered stage events (nsa_profile_stages); g_stage_next counts the events
+// recorded by the current call.
+void* const* g_stage_events = nullptr;
+int g_stage_count = 0;
+int g_stage_next = 0;
+
+void stage_begin(cudaStream_t st) {
+  g_stage_next = 0;
+  if (g_stage_count > 0) cudaEventRecord(static_cast<cudaEvent_t>(g_stage_events[g_stage_next++]), st);
+}
+
 int launch_status(const char* name = "kernel", cudaStream_t st = nullptr) {
   cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess && g_stage_next < g_stage_count)
+    e = cudaEventRecord(static_cast<cudaEvent_t>(g_stage_events[g_stage_next++]), st);
   if (e == cudaSuccess && debug_sync()) {
     std::fprintf(stderr, "[nsa] %s launched\n", name);
     std::fflush(stderr);
@@ -401,6 +414,7 @@ int nsa_prefill(const void* q, const void* k, const void* v, const float* gates,
   if ((rc = check_device()) != NSA_OK) return rc;
   auto* ws = static_cast<uint8_t*>(workspace);
   auto st = static_cast<cudaStream_t>(stream);
+  stage_begin(st);
   if (params->head_dim == 64) return prefill_impl<64>(params, q, k, v, gates, out, out_sel_idx, ws, st);
   return prefill_impl<128>(params, q, k, v, gates, out, out_sel_idx, ws, st);
 }
@@ -423,6 +437,7 @@ int nsa_decode(const void* q, const void* kcache, const void* vcache, const void
   if ((rc = check_device()) != NSA_OK) return rc;
   auto* ws = static_cast<uint8_t*>(workspace);
   auto st = static_cast<cudaStream_t>(stream);
+  stage_begin(st);
   if (params->head_dim == 64)
     return decode_impl<64>(params, q, kcache, vcache, kcmp, vcmp, seq_lens, gates, out, out_sel_idx, ws, st);
   return decode_impl<128>(params, q, kcache, vcache, kcmp, vcmp, seq_lens, gates, out, out_sel_idx, ws, st);
@@ -437,6 +452,14 @@ int nsa_compress(const void* k, const void* v, const nsa_params_t* params, void*
   const int ncmp = ncmp_of(params->n_tokens, params->cmp_block, params->cmp_stride);
   return launch_pool(k, v, kcmp, vcmp, params->batch, params->n_tokens, params->num_kv_heads, params->head_dim, ncmp,
                      params->cmp_block, params->cmp_stride, static_cast<cudaStream_t>(stream));
+}
+
+int nsa_profile_stages(void* const* events, int count) {
+  if (count < 0 || (count > 0 && events == nullptr)) return NSA_ERR_INVALID_ARG;
+  g_stage_events = count > 0 ? events : nullptr;
+  g_stage_count = count > 0 ? count : 0;
+  g_stage_next = 0;
+  return NSA_OK;
 }
 
 int nsa_get_device_error(uint32_t* word, int clear) {

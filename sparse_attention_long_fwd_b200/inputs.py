@@ -49,6 +49,8 @@ WORKLOADS = {
                                    frame_mean_var=0.5),
     "sweep128k_n48_w1024": Workload("sweep128k_n48_w1024", 131072, 131072, top_n=48, window=1024,
                                     frame_mean_var=0.5),
+    # a 32,768-token cut of the 128K workload (inputs still larger than L2), for kernel profiles
+    "v32k": Workload("v32k", 32768, 32768, frame_mean_var=0.5),
     # 64 sequences x 131,072-token cache, one query each
     "decode64x128k": Workload("decode64x128k", 131072, 131072, batch=64),
 }

@@ -26,7 +26,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnsa_b200
 
 EXPORTED = (
     "nsa_prefill", "nsa_decode", "nsa_compress", "nsa_workspace_size", "nsa_prefill_workspace_layout",
-    "nsa_error_string", "nsa_get_device_error", "nsa_version",
+    "nsa_error_string", "nsa_get_device_error", "nsa_version", "nsa_profile_stages",
 )
 
 
@@ -87,6 +87,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.nsa_get_device_error.restype = I
     lib.nsa_version.argtypes = []
     lib.nsa_version.restype = ctypes.c_char_p
+    lib.nsa_profile_stages.argtypes = [ctypes.POINTER(ctypes.c_void_p), I]
+    lib.nsa_profile_stages.restype = I
     _lib = lib
     return lib
 
@@ -161,6 +163,18 @@ def nsa_get_device_error(clear: bool = True) -> int:
 
 def nsa_version() -> str:
     return load_library().nsa_version().decode()
+
+
+_stage_handles = None
+
+
+def nsa_profile_stages(events) -> int:
+    """Register torch.cuda.Event objects (or raw cudaEvent_t handles) recorded at stage
+    boundaries of every following call; an empty list switches recording off."""
+    global _stage_handles
+    handles = [e.cuda_event if hasattr(e, "cuda_event") else int(e) for e in (events or [])]
+    _stage_handles = (ctypes.c_void_p * max(len(handles), 1))(*handles)
+    return load_library().nsa_profile_stages(_stage_handles if handles else None, len(handles))
 
 
 # ------------------------------------------------------------------ torch conveniences
