@@ -55,7 +55,8 @@ enum nsa_status {
   NSA_ERR_INVALID_ARG = 1,         /* null pointer, bad shape, misalignment, bad constant */
   NSA_ERR_UNSUPPORTED = 2,         /* valid but not implemented here (head_dim, block sizes, device) */
   NSA_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes < nsa_workspace_size() */
-  NSA_ERR_CUDA = 4                 /* a CUDA runtime call or launch failed */
+  NSA_ERR_CUDA = 4,                /* a CUDA runtime call or launch failed */
+  NSA_ERR_NOALLOC_TOO_LARGE = 5    /* nsa_decode_noalloc: the problem needs more than its fixed scratch */
 };
 
 enum nsa_out_dtype { NSA_OUT_BF16 = 0, NSA_OUT_F32 = 1 };
@@ -102,6 +103,31 @@ int nsa_prefill(const void* q, const void* k, const void* v, const float* gates,
 int nsa_decode(const void* q, const void* kcache, const void* vcache, const void* kcmp, const void* vcmp,
                const int32_t* seq_lens, const float* gates, const nsa_params_t* params, void* out,
                int32_t* out_sel_idx, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Decode that allocates nothing and takes no workspace. The pages describe no such
+ * variant; it exists for callers that cannot call cudaMalloc or hand over scratch memory:
+ * for example a plugin or C program whose device memory is owned and pre-partitioned by
+ * a host framework that forbids allocation on its serving path, or a caller with a device
+ * memory budget fixed at start-up. Same arguments, results and kernels as nsa_decode,
+ * except that the scratch lives in one fixed device array of NSA_NOALLOC_SCRATCH_BYTES
+ * (32 MiB) compiled into the library; every GPU that loads the library holds that array
+ * until the process exits.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call before any
+ *     stream capture on the device.
+ *   - A problem whose scratch (nsa_workspace_size(params, 1)) exceeds the array returns
+ *     NSA_ERR_NOALLOC_TOO_LARGE before anything is enqueued; use nsa_decode for it.
+ *   - All calls share the one array and it keeps the last call's contents; no kernel reads
+ *     scratch it has not written in the same call, so nothing needs clearing. Calls whose
+ *     execution overlaps on the GPU (other streams, other threads) race on the array:
+ *     serialise them.
+ * Calls no cudaMalloc, cudaFree or allocating library routine.
+ */
+#define NSA_NOALLOC_SCRATCH_BYTES (32u << 20)
+int nsa_decode_noalloc(const void* q, const void* kcache, const void* vcache, const void* kcmp, const void* vcmp,
+                       const int32_t* seq_lens, const float* gates, const nsa_params_t* params, void* out,
+                       int32_t* out_sel_idx, void* stream);
 
 /*
  * Compression only: kcmp[b][i] = bf16_rne(mean_{u<l} k[b][i*s+u]) for every complete block

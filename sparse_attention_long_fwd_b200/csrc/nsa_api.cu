@@ -367,6 +367,8 @@ const char* nsa_error_string(int status) {
       return "workspace smaller than nsa_workspace_size()";
     case NSA_ERR_CUDA:
       return "a CUDA runtime call or kernel launch failed";
+    case NSA_ERR_NOALLOC_TOO_LARGE:
+      return "the decode needs more scratch than nsa_decode_noalloc's fixed array (NSA_NOALLOC_SCRATCH_BYTES)";
     default:
       return "unknown status";
   }
@@ -436,6 +438,53 @@ int nsa_decode(const void* q, const void* kcache, const void* vcache, const void
   if (workspace_bytes < decode_layout(params).total) return NSA_ERR_WORKSPACE_TOO_SMALL;
   if ((rc = check_device()) != NSA_OK) return rc;
   auto* ws = static_cast<uint8_t*>(workspace);
+  auto st = static_cast<cudaStream_t>(stream);
+  stage_begin(st);
+  if (params->head_dim == 64)
+    return decode_impl<64>(params, q, kcache, vcache, kcmp, vcmp, seq_lens, gates, out, out_sel_idx, ws, st);
+  return decode_impl<128>(params, q, kcache, vcache, kcmp, vcmp, seq_lens, gates, out, out_sel_idx, ws, st);
+}
+
+// ------------------------------------------------------------------ decode with no caller scratch
+// nsa_decode_noalloc keeps its scratch in this fixed device array instead of a caller
+// workspace. Every GPU that loads the library holds the array until the process exits.
+// Host code must not pass the symbol itself to a kernel: on the host it is only a
+// stand-in, so the device address is looked up with cudaGetSymbolAddress, once per
+// device, with that device current.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NSA_NOALLOC_SCRATCH_BYTES];
+
+static int noalloc_scratch_address(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NSA_ERR_CUDA;
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return NSA_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return NSA_OK;
+}
+
+int nsa_decode_noalloc(const void* q, const void* kcache, const void* vcache, const void* kcmp, const void* vcmp,
+                       const int32_t* seq_lens, const float* gates, const nsa_params_t* params, void* out,
+                       int32_t* out_sel_idx, void* stream) {
+  int rc = check_common(params);
+  if (rc != NSA_OK) return rc;
+  if (params->batch < 1) return NSA_ERR_INVALID_ARG;
+  if (params->window > kMaxWindowDecode) return NSA_ERR_UNSUPPORTED;
+  if (!q || !kcache || !vcache || !kcmp || !vcmp || !seq_lens || !gates || !out) return NSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(kcmp) || !aligned16(vcmp) ||
+      !aligned16(out) || (out_sel_idx && !aligned16(out_sel_idx)))
+    return NSA_ERR_INVALID_ARG;
+  if (nsel_of(params->n_tokens, params->sel_block) > 8192) return NSA_ERR_UNSUPPORTED;
+  if (decode_layout(params).total > NSA_NOALLOC_SCRATCH_BYTES) return NSA_ERR_NOALLOC_TOO_LARGE;
+  if ((rc = check_device()) != NSA_OK) return rc;
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch_address(&scratch)) != NSA_OK) return rc;
+  auto* ws = static_cast<uint8_t*>(scratch);
   auto st = static_cast<cudaStream_t>(stream);
   stage_begin(st);
   if (params->head_dim == 64)

@@ -18,6 +18,8 @@ NSA_ERR_INVALID_ARG = 1
 NSA_ERR_UNSUPPORTED = 2
 NSA_ERR_WORKSPACE_TOO_SMALL = 3
 NSA_ERR_CUDA = 4
+NSA_ERR_NOALLOC_TOO_LARGE = 5
+NSA_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 NSA_OUT_BF16 = 0
 NSA_OUT_F32 = 1
@@ -26,7 +28,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnsa_b200
 
 EXPORTED = (
     "nsa_prefill", "nsa_decode", "nsa_compress", "nsa_workspace_size", "nsa_prefill_workspace_layout",
-    "nsa_error_string", "nsa_get_device_error", "nsa_version", "nsa_profile_stages",
+    "nsa_error_string", "nsa_get_device_error", "nsa_version", "nsa_profile_stages", "nsa_decode_noalloc",
 )
 
 
@@ -75,6 +77,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.nsa_prefill.restype = I
     lib.nsa_decode.argtypes = [P, P, P, P, P, P, P, PP, P, P, P, S, P]
     lib.nsa_decode.restype = I
+    lib.nsa_decode_noalloc.argtypes = [P, P, P, P, P, P, P, PP, P, P, P]
+    lib.nsa_decode_noalloc.restype = I
     lib.nsa_compress.argtypes = [P, P, PP, P, P, P]
     lib.nsa_compress.restype = I
     lib.nsa_workspace_size.argtypes = [PP, I]
@@ -130,6 +134,15 @@ def nsa_decode(q, kcache, vcache, kcmp, vcmp, seq_lens, gates, params: NsaParams
     return load_library().nsa_decode(_addr(q), _addr(kcache), _addr(vcache), _addr(kcmp), _addr(vcmp),
                                      _addr(seq_lens), _addr(gates), ctypes.byref(params), _addr(out),
                                      _addr(out_sel_idx), _addr(workspace), workspace_bytes, _stream(stream))
+
+
+def nsa_decode_noalloc(q, kcache, vcache, kcmp, vcmp, seq_lens, gates, params: NsaParams, out, out_sel_idx,
+                       stream=None) -> int:
+    """nsa_decode without a workspace: for callers that cannot allocate device memory
+    (scratch lives in the library's fixed NSA_NOALLOC_SCRATCH_BYTES device array)."""
+    return load_library().nsa_decode_noalloc(_addr(q), _addr(kcache), _addr(vcache), _addr(kcmp), _addr(vcmp),
+                                             _addr(seq_lens), _addr(gates), ctypes.byref(params), _addr(out),
+                                             _addr(out_sel_idx), _stream(stream))
 
 
 def nsa_compress(k, v, params: NsaParams, kcmp, vcmp, stream=None) -> int:
