@@ -23,9 +23,10 @@
 // next block while computing the current one, tiling against register pressure) are
 // met here by TMA tiles, an mbarrier ring and TMEM accumulators.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues the
-// MMAs (one elected lane), warps 2..5 (128 threads, one per TMEM lane / MMA row) do the
-// softmax, the score binning and the epilogue. Every wait is bounded (sm100.cuh).
+// Warp roles (320 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues the
+// MMAs (one elected lane), warps 2..9 (two warpgroups; each thread owns one TMEM lane /
+// MMA row and one half of the key columns) do the softmax, the score binning and the
+// epilogue. Every wait is bounded (sm100.cuh).
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -38,6 +39,7 @@ enum AttnMode { kModeCmp = 0, kModeWin = 1, kModeDense = 2 };
 struct AttnArgs {
   int q_begin, q_end;      // query tokens handled: [q_begin, q_end)
   int hq, hkv, G, T;       // heads, group size, tokens per tile
+  int Gp;                  // MMA rows per token: G, or (kModeCmp) G rounded up to a power of two
   int n_tiles;             // ceil((q_end - q_begin) / T)
   float scale_log2;        // softmax_scale * log2(e)
   int cmp_len, cmp_stride;  // compressed-key visibility (kModeCmp)
@@ -53,7 +55,7 @@ struct AttnArgs {
   int out_f32;
 };
 
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 320;  // producer, MMA, 2 x 4 softmax warps
 constexpr int kBN = 128;      // keys per tile
 constexpr int kStages = 2;    // TMA ring depth (K and V tiles)
 
@@ -65,7 +67,7 @@ struct AttnSmem {
   alignas(1024) uint8_t k[kStages][kChunks][kTileBytes];
   alignas(1024) uint8_t v[kStages][kChunks][kTileBytes];
   alignas(1024) uint8_t p[2][kTileBytes];            // P tile: 128 rows x 128 keys bf16
-  float bins[128][33];
+  float lse_x[2][128][2];     // per warpgroup: (scaled max, sum) of the row's half
   uint64_t q_full;
   uint64_t full[kStages], empty[kStages];
   uint64_t s_full[2], s_free[2];
@@ -76,6 +78,22 @@ struct AttnSmem {
 };
 
 __device__ __forceinline__ int ncmp_visible(int t, int l, int s) { return (t + 1 >= l) ? (t + 1 - l) / s + 1 : 0; }
+
+// Reduce-scatter of 16 per-lane values over groups of GP adjacent lanes: afterwards
+// bin[0 .. 16/GP) of lane l holds the group sums of entries [(l%GP)*16/GP, ...).
+template <int GP>
+__device__ __forceinline__ void group_reduce_scatter(float (&bin)[16], int lane) {
+#pragma unroll
+  for (int o = GP / 2, n = 16; o >= 1; o >>= 1, n >>= 1) {
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < n / 2; ++i) {
+      const float send = upper ? bin[i] : bin[i + n / 2];
+      const float keep = upper ? bin[i + n / 2] : bin[i];
+      bin[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+}
 
 template <int D, int MODE>
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -119,9 +137,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.s_full[b], 1);
-      mbar_init(&sm.s_free[b], 4);
+      mbar_init(&sm.s_free[b], 8);
     }
-    mbar_init(&sm.p_full, 4);
+    mbar_init(&sm.p_full, 8);
     mbar_init(&sm.p_free, 1);
     mbar_init(&sm.o_full, 1);
     mbar_init(&sm.drain, 1);
@@ -134,9 +152,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tmem_relinquish();
   }
   if (warp >= 2) {
-    // rows T*G .. 127 of the Q tile are never written by TMA: keep them finite (zero)
-    const int r0 = T * G;
-    for (int i = tid - 64; i < (128 - r0) * 8 * kChunks; i += 128) {
+    // rows T*Gp .. 127 of the Q tile are never written by TMA: keep them finite (zero)
+    const int r0 = T * args.Gp;
+    for (int i = tid - 64; i < (128 - r0) * 8 * kChunks; i += 256) {
       const int c = i / ((128 - r0) * 8);
       const int rem = i % ((128 - r0) * 8);
       *reinterpret_cast<uint4*>(&sm.q[c][(r0 + rem / 8) * 128 + (rem % 8) * 16]) = make_uint4(0, 0, 0, 0);
@@ -156,7 +174,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tma_prefetch_desc(&qmap);
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
-      mbar_arrive_expect_tx(&sm.q_full, kChunks * T * G * 128);
+      mbar_arrive_expect_tx(&sm.q_full, kChunks * T * args.Gp * 128);
       for (int c = 0; c < kChunks; ++c) tma_load_3d(&qmap, &sm.q_full, sm.q[c], c * 64, g * G, t0);
       for (int job = 0; job < njobs; ++job) {
         const int stage = job % kStages;
@@ -225,12 +243,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ softmax / epilogue
+    // Two warpgroups share every S tile: warpgroup `wg` owns keys [64*wg, 64*wg + 64) of
+    // each 128-key tile (and output columns [wg*D/2, (wg+1)*D/2) in the epilogue); the
+    // thread of TMEM lane r in each warpgroup handles MMA row r.
+    const int sw = warp - 2;                 // softmax warp 0..7
+    const int wg = sw >> 2;                  // column half
     const int q4 = warp & 3;                 // TMEM lane quadrant of this warp
     const int r = q4 * 32 + lane;            // MMA row
-    const int tok = r / G, hh = r % G;
+    const int stid = sw * 32 + lane;         // 0..255
+    const int Gp = args.Gp;
+    const int tok = r / Gp, hh = r % Gp;
     const int t = t0 + tok;
     const int h = g * G + hh;
-    const bool row_valid = (r < T * G) && (t < args.q_end);
+    const bool row_valid = (r < T * Gp) && (hh < G) && (t < args.q_end);
     int rb = 0, re = 0;                      // visible key range of this row
     if (row_valid) {
       if (MODE == kModeCmp) {
@@ -243,132 +268,180 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
     }
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const int col0 = wg * 64;
     const float sl2 = args.scale_log2;
     bool ok = true;
-    // ---- phase 1: exact log-sum-exp (base 2) of each row
-    float m = -INFINITY, lsum = 0.f;
+    // ---- phase 1: log-sum-exp (base 2) of this row's half, combined across halves below
+    float m = -INFINITY, lsum = 0.f;         // m: running max of the raw (unscaled) scores
     for (int kt = 0; kt < nkt && ok; ++kt) {
       const int b = kt & 1;
       // tcgen05.ld is warp-collective: every wait result is made warp-uniform
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (kt >> 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      const int kbase = kb + kt * kBN;
-#pragma unroll 1
-      for (int cb = 0; cb < kBN / 32; ++cb) {
-        float s[32];
-        __syncwarp();
-        tmem_ld32(trow + b * kBN + cb * 32, s);
-        tmem_wait_ld();
-        float cmax = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int kidx = kbase + cb * 32 + i;
-          s[i] = (kidx >= rb && kidx < re) ? s[i] * sl2 : -INFINITY;
-          cmax = fmaxf(cmax, s[i]);
-        }
-        const float mnew = fmaxf(m, cmax);
-        if (mnew != -INFINITY) {
-          float acc = 0.f;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) acc += ex2_approx(s[i] - mnew);
-          lsum = lsum * ex2_approx(m - mnew) + acc;
-          m = mnew;
-        }
-      }
+      const int kbase = kb + kt * kBN + col0;
+      const bool full = kbase >= rb && kbase + 64 <= re;
+      float s[64];
+      __syncwarp();
+      tmem_ld32(trow + b * kBN + col0, *reinterpret_cast<float(*)[32]>(&s[0]));
+      tmem_ld32(trow + b * kBN + col0 + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.s_free[b]);
+      if (lane == 0) mbar_arrive(&sm.s_free[b]);  // S is in registers: the buffer may be reused
+      if (!full) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const int kidx = kbase + i;
+          s[i] = (kidx >= rb && kidx < re) ? s[i] : -INFINITY;
+        }
+      }
+      float mx[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) mx[c] = s[c];
+#pragma unroll
+      for (int i = 8; i < 64; i += 8)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) mx[c] = fmaxf(mx[c], s[i + c]);
+      const float cmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      const float mnew = fmaxf(m, cmax);
+      if (mnew != -INFINITY) {
+        const float ms = mnew * sl2;
+        float acc[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[c] = ex2_approx(fmaf(s[c], sl2, -ms));
+#pragma unroll
+        for (int i = 8; i < 64; i += 8)
+#pragma unroll
+          for (int c = 0; c < 8; ++c) acc[c] += ex2_approx(fmaf(s[i + c], sl2, -ms));
+        lsum = lsum * ex2_approx((m - mnew) * sl2) +
+               (((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7])));
+        m = mnew;
+      }
     }
-    const bool has_keys = lsum > 0.f;
-    const float lse2 = has_keys ? m + __log2f(lsum) : INFINITY;
+    sm.lse_x[wg][r][0] = (m == -INFINITY) ? -INFINITY : m * sl2;
+    sm.lse_x[wg][r][1] = lsum;
+    named_bar_sync(3, 256);
+    float lse2;
+    bool has_keys;
+    {
+      const float ma = sm.lse_x[0][r][0], la = sm.lse_x[0][r][1];
+      const float mb = sm.lse_x[1][r][0], lb = sm.lse_x[1][r][1];
+      const float M = fmaxf(ma, mb);
+      float L = 0.f;
+      if (M != -INFINITY) L = la * ex2_approx(ma - M) + lb * ex2_approx(mb - M);
+      has_keys = L > 0.f;
+      lse2 = has_keys ? M + __log2f(L) : INFINITY;
+    }
     // ---- phase 2: normalised probabilities -> P (smem, bf16) and block scores
-    float carry = 0.f;  // half of the last compressed block of the previous tile (kModeCmp)
-    // In the compressed mode the four softmax warps meet at named barriers every tile,
-    // so they must leave this loop together: each iteration ORs their failures.
+    // Block scores (kModeCmp): compressed block i covers tokens [16i, 16i+32) and selection
+    // block j covers [64j, 64j+64), so block j takes all of compressed blocks 4j..4j+2 and
+    // half of 4j-1 and 4j+3. A 128-key tile holds selection blocks kt2*32 .. kt2*32+31;
+    // this warpgroup's 64 keys hold 16 of them. The one compressed block that straddles
+    // the previous 64 keys is re-read from TMEM by this thread (column 63 for warpgroup 1,
+    // the previous tile's column 127 for warpgroup 0, kept from the previous iteration),
+    // so the halves never exchange data. The G heads of a token sit in Gp adjacent lanes;
+    // a shuffle reduce-scatter sums them, leaving 16/Gp consecutive blocks per lane.
+    float carry = 0.f;  // warpgroup 0: half of the previous tile's last compressed block
+    const int bpl = 16 / Gp;  // blocks per lane after the reduce-scatter (kModeCmp)
     for (int kt2 = 0; kt2 < nkt; ++kt2) {
       const int job = nkt + kt2;
       const int b = job & 1;
       if (ok) ok = mbar_wait(&sm.s_full[b], (job >> 1) & 1, abort_flag);
       if (ok && kt2 > 0) ok = mbar_wait(&sm.p_free, (kt2 - 1) & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
-      const bool any_fail = (MODE == kModeCmp) ? named_bar_any(2, 128, !ok) : !ok;
-      if (any_fail) {
-        ok = false;
-        break;
-      }
+      if (!ok) break;
       tc_fence_after();
-      const int kbase = kb + kt2 * kBN;
-#pragma unroll 1
-      for (int cb = 0; cb < kBN / 32; ++cb) {
-        float s[32];
-        __syncwarp();
-        tmem_ld32(trow + b * kBN + cb * 32, s);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int kidx = kbase + cb * 32 + i;
-          s[i] = (kidx >= rb && kidx < re) ? ex2_approx(s[i] * sl2 - lse2) : 0.f;
-        }
-        if (MODE == kModeCmp) {
-          // compressed block i covers tokens [16i, 16i+32); selection block j covers
-          // [64j, 64j+64): blocks 4j..4j+2 lie inside j, blocks 4j-1 and 4j+3 half inside.
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const float half_last = 0.5f * s[4 * u + 3];
-            sm.bins[r][cb * 8 + u] = carry + s[4 * u] + s[4 * u + 1] + s[4 * u + 2] + half_last;
-            carry = half_last;
-          }
-        }
-        // P row r, keys cb*32 .. cb*32+31 -> chunk cb/2, columns (cb%2)*32 ..
-        uint8_t* pc = sm.p[cb >> 1];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          uint4 w;
-          w.x = pack_bf16x2(s[8 * u + 0], s[8 * u + 1]);
-          w.y = pack_bf16x2(s[8 * u + 2], s[8 * u + 3]);
-          w.z = pack_bf16x2(s[8 * u + 4], s[8 * u + 5]);
-          w.w = pack_bf16x2(s[8 * u + 6], s[8 * u + 7]);
-          *reinterpret_cast<uint4*>(pc + sw128_offset(r, (cb & 1) * 32 + 8 * u)) = w;
-        }
-      }
-      fence_proxy_async_smem();
+      const int kbase = kb + kt2 * kBN + col0;
+      const bool full = kbase >= rb && kbase + 64 <= re;
+      float bin[16];
+      float half_in = 0.f;
+      float s[64];
+      uint32_t xv = 0;
+      const int xcol = wg == 1 ? 63 : 127;  // (kModeCmp) the straddling block's column
+      __syncwarp();
+      tmem_ld32(trow + b * kBN + col0, *reinterpret_cast<float(*)[32]>(&s[0]));
+      tmem_ld32(trow + b * kBN + col0 + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
+      if (MODE == kModeCmp)
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(xv) : "r"(trow + b * kBN + xcol));
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&sm.s_free[b]);
-        mbar_arrive(&sm.p_full);
+      if (lane == 0) mbar_arrive(&sm.s_free[b]);  // S is in registers: the buffer may be reused
+      if (MODE == kModeCmp) {
+        // the straddling block's probability: column 63 (wg 1) or this tile's column 127
+        // (wg 0, carried into the next tile)
+        const int xk = kb + kt2 * kBN + xcol;
+        const float px = (xk >= rb && xk < re) ? ex2_approx(fmaf(__uint_as_float(xv), sl2, -lse2)) : 0.f;
+        if (wg == 1) {
+          half_in = 0.5f * px;
+        } else {
+          half_in = carry;
+          carry = 0.5f * px;
+        }
+      }
+      if (full) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) s[i] = ex2_approx(fmaf(s[i], sl2, -lse2));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const int kidx = kbase + i;
+          s[i] = (kidx >= rb && kidx < re) ? ex2_approx(fmaf(s[i], sl2, -lse2)) : 0.f;
+        }
       }
       if (MODE == kModeCmp) {
-        named_bar_sync(1, 128);
-        const int nb = T * 32;
-        for (int i = tid - 64; i < nb; i += 128) {
-          const int tk = i >> 5, bb = i & 31;
-          const int tt = t0 + tk;
-          const int j = kt2 * 32 + bb;
-          if (tt < args.q_end && j <= tt / args.sel_len) {
-            float acc = 0.f;
-            for (int x = 0; x < G; ++x) acc += sm.bins[tk * G + x][bb];
-            args.scores[(static_cast<size_t>(tt) * args.hkv + g) * args.nsel + j] = acc;
-          }
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const float half_last = 0.5f * s[4 * u + 3];
+          bin[u] = (u == 0 ? half_in : 0.5f * s[4 * u - 1]) + s[4 * u] + s[4 * u + 1] + s[4 * u + 2] + half_last;
         }
-        named_bar_sync(1, 128);
+      }
+      // P row r, keys col0 .. col0+63 -> chunk wg
+      uint8_t* pc = sm.p[wg];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        uint4 w;
+        w.x = pack_bf16x2(s[8 * u + 0], s[8 * u + 1]);
+        w.y = pack_bf16x2(s[8 * u + 2], s[8 * u + 3]);
+        w.z = pack_bf16x2(s[8 * u + 4], s[8 * u + 5]);
+        w.w = pack_bf16x2(s[8 * u + 6], s[8 * u + 7]);
+        *reinterpret_cast<uint4*>(pc + sw128_offset(r, 8 * u)) = w;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.p_full);
+      if (MODE == kModeCmp) {
+        // reduce-scatter over the Gp lanes of this token: afterwards lane hh holds the
+        // group sums of blocks [hh*bpl, (hh+1)*bpl) of this warpgroup's 16
+        switch (Gp) {
+          case 2: group_reduce_scatter<2>(bin, lane); break;
+          case 4: group_reduce_scatter<4>(bin, lane); break;
+          case 8: group_reduce_scatter<8>(bin, lane); break;
+          case 16: group_reduce_scatter<16>(bin, lane); break;
+          default: break;
+        }
+        if (t < args.q_end && r < T * Gp) {
+          const int jt = t / args.sel_len;
+          const int j0 = kt2 * 32 + wg * 16 + hh * bpl;
+          float* dst = args.scores + (static_cast<size_t>(t) * args.hkv + g) * args.nsel;
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (i < bpl && j0 + i <= jt) dst[j0 + i] = bin[i];
+        }
       }
     }
-    if (MODE == kModeCmp && ok) {
-      // the carried half-block after the last tile lands in selection block nkt*32;
-      // when no key tile exists at all, that is block 0 with score 0.
-      sm.bins[r][0] = carry;
-      named_bar_sync(1, 128);
-      for (int tk = tid - 64; tk < T; tk += 128) {
-        const int tt = t0 + tk;
-        const int j = nkt * 32;
-        if (tt < args.q_end && j <= tt / args.sel_len) {
-          float acc = 0.f;
-          for (int x = 0; x < G; ++x) acc += sm.bins[tk * G + x][0];
-          args.scores[(static_cast<size_t>(tt) * args.hkv + g) * args.nsel + j] = acc;
-        }
-      }
+    if (MODE == kModeCmp && ok && wg == 0) {
+      // the carried half-block after the last tile lands in selection block nkt*32; when no
+      // key tile exists at all, that is block 0 with score 0
+      float c = carry;
+#pragma unroll
+      for (int o = 1; o < 16; o <<= 1)
+        if (o < Gp) c += __shfl_xor_sync(0xffffffffu, c, o);
+      const int j = nkt * 32;
+      if (hh == 0 && t < args.q_end && r < T * Gp && j <= t / args.sel_len)
+        args.scores[(static_cast<size_t>(t) * args.hkv + g) * args.nsel + j] = c;
     }
     // ---- epilogue (every lane loads its TMEM row; only valid rows are stored)
     if (ok && nkt > 0) {
@@ -384,11 +457,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         g2 = args.gates[(static_cast<size_t>(t) * args.hq + h) * 3 + 2];
       }
 #pragma unroll 1
-      for (int cb = 0; cb < D / 32; ++cb) {
+      for (int cc = 0; cc < D / 64; ++cc) {
+        const int c0 = wg * (D / 2) + cc * 32;  // output columns c0 .. c0+31
         float o[32];
         __syncwarp();
         if (nkt > 0) {
-          tmem_ld32(trow + kColO + cb * 32, o);
+          tmem_ld32(trow + kColO + c0, o);
           tmem_wait_ld();
         } else {
 #pragma unroll
@@ -397,13 +471,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!row_valid) {
           // nothing to store for padding rows
         } else if (MODE == kModeCmp) {
-          float4* dst = reinterpret_cast<float4*>(args.o_cmp + orow + cb * 32);
+          float4* dst = reinterpret_cast<float4*>(args.o_cmp + orow + c0);
 #pragma unroll
           for (int u = 0; u < 8; ++u) dst[u] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
         } else {
           if (MODE == kModeWin) {
-            const float4* oc = reinterpret_cast<const float4*>(args.o_cmp + orow + cb * 32);
-            const float4* os = reinterpret_cast<const float4*>(args.o_sel + orow + cb * 32);
+            const float4* oc = reinterpret_cast<const float4*>(args.o_cmp + orow + c0);
+            const float4* os = reinterpret_cast<const float4*>(args.o_sel + orow + c0);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
               const float4 a = oc[u], c = os[u];
@@ -414,11 +488,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
           }
           if (args.out_f32) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.out) + orow + cb * 32);
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.out) + orow + c0);
 #pragma unroll
             for (int u = 0; u < 8; ++u) dst[u] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
           } else {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) + orow + cb * 32);
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) + orow + c0);
 #pragma unroll
             for (int u = 0; u < 4; ++u)
               dst[u] = make_uint4(pack_bf16x2(o[8 * u], o[8 * u + 1]), pack_bf16x2(o[8 * u + 2], o[8 * u + 3]),
@@ -426,7 +500,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
       }
-      if (MODE == kModeCmp && row_valid)
+      if (MODE == kModeCmp && row_valid && wg == 0)
         args.lse[static_cast<size_t>(t) * args.hq + h] = has_keys ? lse2 * 0.69314718055994530942f : -INFINITY;
     }
     tc_fence_before();

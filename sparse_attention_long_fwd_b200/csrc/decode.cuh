@@ -140,7 +140,8 @@ __global__ void __launch_bounds__(256) dec_select_kernel(const int32_t* __restri
                                                          int32_t* __restrict__ out_sel_idx) {
   extern __shared__ float ds_smem[];
   float* sc = ds_smem;                                        // [nsel_max]
-  uint32_t* bits = reinterpret_cast<uint32_t*>(sc + a.nsel_max);  // [nsel_max/32 + 1]
+  int* list = reinterpret_cast<int*>(sc + a.nsel_max);        // [nsel_max]
+  uint32_t* bits = reinterpret_cast<uint32_t*>(list + a.nsel_max);  // [nsel_max/32 + 1]
   float* lse2 = reinterpret_cast<float*>(bits + a.nsel_max / 32 + 1);  // [G]
   const int bg = blockIdx.x, b = bg / a.hkv, g = bg % a.hkv;
   const int tid = threadIdx.x;
@@ -190,7 +191,7 @@ __global__ void __launch_bounds__(256) dec_select_kernel(const int32_t* __restri
   }
   __syncthreads();
   if (tid < 32) {
-    warp_topn(sc, bits, sc, jt, a.top_n, a.sel_idx + static_cast<size_t>(bg) * a.top_n,
+    warp_topn(sc, bits, list, sc, jt, a.top_n, a.sel_idx + static_cast<size_t>(bg) * a.top_n,
               out_sel_idx ? out_sel_idx + static_cast<size_t>(bg) * a.top_n : nullptr, tid);
   }
 }

@@ -206,10 +206,13 @@ int prefill_impl(const nsa_params_t* p, const void* q, const void* k, const void
   const int N = p->n_tokens, nv = p->n_video, hq = p->num_q_heads, hkv = p->num_kv_heads;
   const int G = hq / hkv;
   const int T = 128 / G;
+  int Gc = 1;  // compressed mode: G rounded up to a power of two, so a token's heads share a warp
+  while (Gc < G) Gc <<= 1;
+  const int Tc = 128 / Gc;
   const float scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(D));
   const float sl2 = scale * 1.4426950408889634f;
   int rc;
-  CUtensorMap qmap, kmap, vmap, kcmap, vcmap;
+  CUtensorMap qmap, qcmap, kmap, vmap, kcmap, vcmap;
   const uint64_t qs1 = static_cast<uint64_t>(D) * 2, qs2 = static_cast<uint64_t>(hq) * D * 2;
   const uint64_t ks1 = static_cast<uint64_t>(D) * 2, ks2 = static_cast<uint64_t>(hkv) * D * 2;
   if (!nsa::make_tmap_bf16_3d(&qmap, q, D, hq, N, qs1, qs2, 64, G, T) ||
@@ -221,6 +224,7 @@ int prefill_impl(const nsa_params_t* p, const void* q, const void* k, const void
   a.hkv = hkv;
   a.G = G;
   a.T = T;
+  a.Gp = G;
   a.scale_log2 = sl2;
   a.cmp_len = p->cmp_block;
   a.cmp_stride = p->cmp_stride;
@@ -234,23 +238,30 @@ int prefill_impl(const nsa_params_t* p, const void* q, const void* k, const void
     auto* vc = ws + L.vc;
     const int ncmp_rows = L.ncmp > 0 ? L.ncmp : 1;
     if (!nsa::make_tmap_bf16_3d(&kcmap, kc, D, hkv, ncmp_rows, ks1, ks2, 64, 1, nsa::kBN) ||
-        !nsa::make_tmap_bf16_3d(&vcmap, vc, D, hkv, ncmp_rows, ks1, ks2, 64, 1, nsa::kBN))
+        !nsa::make_tmap_bf16_3d(&vcmap, vc, D, hkv, ncmp_rows, ks1, ks2, 64, 1, nsa::kBN) ||
+        !nsa::make_tmap_bf16_3d(&qcmap, q, D, hq, N, qs1, qs2, 64, Gc, Tc))
       return NSA_ERR_CUDA;
     // 1. compression: Kc, Vc of the video prefix
     if ((rc = launch_pool(k, v, kc, vc, 1, nv, hkv, D, L.ncmp, p->cmp_block, p->cmp_stride, st)) != NSA_OK) return rc;
     // 2. compressed branch + block scores
     a.q_begin = 0;
     a.q_end = nv;
-    a.n_tiles = (nv + T - 1) / T;
     a.o_cmp = reinterpret_cast<float*>(ws + L.o_cmp);
     a.lse = reinterpret_cast<float*>(ws + L.lse);
     a.scores = reinterpret_cast<float*>(ws + L.scores);
-    if ((rc = launch_attn<D, nsa::kModeCmp>(qmap, kcmap, vcmap, a, st)) != NSA_OK) return rc;
+    {
+      AttnArgs ac = a;
+      ac.Gp = Gc;
+      ac.T = Tc;
+      ac.n_tiles = (nv + Tc - 1) / Tc;
+      if ((rc = launch_attn<D, nsa::kModeCmp>(qcmap, kcmap, vcmap, ac, st)) != NSA_OK) return rc;
+    }
+    a.n_tiles = (nv + T - 1) / T;
     // 3. top-n selection
     {
       const int nitems = nv * hkv;
       const int nwords = (L.nsel + 31) / 32;
-      const size_t smem = static_cast<size_t>(nsa::kTopnWarps) * (L.nsel + nwords) * 4;
+      const size_t smem = static_cast<size_t>(nsa::kTopnWarps) * (2 * L.nsel + nwords) * 4;
       if (set_smem(nsa::topn_kernel, smem) != NSA_OK) return NSA_ERR_CUDA;
       int blocks = (nitems + nsa::kTopnWarps - 1) / nsa::kTopnWarps;
       if (blocks > 148 * 32) blocks = 148 * 32;
@@ -327,7 +338,7 @@ int decode_impl(const nsa_params_t* p, const void* q, const void* kcache, const 
     if ((rc = launch_status("dec_cmp", st)) != NSA_OK) return rc;
   }
   {
-    const size_t ssm = (static_cast<size_t>(L.nsel_max) + L.nsel_max / 32 + 1 + 16) * 4;
+    const size_t ssm = (2 * static_cast<size_t>(L.nsel_max) + L.nsel_max / 32 + 1 + 16) * 4;
     auto kern = nsa::dec_select_kernel<D>;
     if (set_smem(kern, ssm) != NSA_OK) return NSA_ERR_CUDA;
     kern<<<a.batch * a.hkv, 256, ssm, st>>>(seq_lens, a, out_sel_idx);

@@ -7,11 +7,7 @@
 // j <= t/l' ordered by score (descending) and block index (ascending) on ties. The
 // result is written ascending and padded with -1.
 //
-// One warp per (row, group). The row's candidate scores are staged in shared memory;
-// each lane keeps the best of its strided subset as a 64-bit key
-// (score bits << 32 | ~j): scores are >= 0, so unsigned comparison of the float bits
-// orders them, and the complemented index makes the lower block win a tie. Each round
-// takes the warp-wide maximum key, removes it, and the owning lane rescans its subset.
+// One warp per (row, group); see warp_topn for the selection itself.
 #pragma once
 #include <cstdint>
 #include "sm100.cuh"
@@ -29,47 +25,111 @@ __device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long x)
   return x;
 }
 
-// Warp-cooperative top-n of one (row, group). `sc` (shared, >= jt+1 floats) holds the
-// candidate scores of blocks 0..jt; `bits` (shared, >= jt/32+1 words) receives the
-// selection bitmap. Writes top_n entries to dst (and dst2 if non-null).
-__device__ __forceinline__ void warp_topn(float* sc, uint32_t* bits, const float* __restrict__ src, int jt,
-                                          int top_n, int32_t* __restrict__ dst, int32_t* __restrict__ dst2,
-                                          int lane) {
+// Warp-cooperative top-n of one (row, group). `sc` (shared, >= jt+1 floats) receives the
+// candidate scores of blocks 0..jt; `bits` (shared, >= jt/32+1 words) the selection
+// bitmap; `list` (shared, >= jt+1 ints) is scratch. Writes top_n entries to dst (and dst2
+// if non-null).
+//
+// Keys are (score bits << 32 | ~j), unique per block. Each lane first keeps the two
+// largest keys of its strided subset; the k-th largest of those 64 keys is a lower bound
+// on the k-th largest key overall (they are a subset of all keys), so only candidates at
+// or above it can be selected. Those survivors -- usually about k of them -- are
+// compacted and the exact top-k is taken from them by rounds of warp-wide maxima.
+__device__ __forceinline__ unsigned long long cand_key(float x, int j) {
+  return x >= 0.f ? (static_cast<unsigned long long>(__float_as_uint(x)) << 32) |
+                        (0xFFFFFFFFu - static_cast<uint32_t>(j))
+                  : 0ull;
+}
+
+__device__ __forceinline__ void warp_topn(float* sc, uint32_t* bits, int* list, const float* __restrict__ src,
+                                          int jt, int top_n, int32_t* __restrict__ dst,
+                                          int32_t* __restrict__ dst2, int lane) {
   const int nwords = jt / 32 + 1;
   for (int w = lane; w < nwords; w += 32) bits[w] = 0u;
   __syncwarp();
-  // forced blocks are marked selected and kept out of the candidate set (score -1)
-  for (int j = lane; j <= jt; j += 32) {
-    const bool forced = (j == 0) || (j == jt) || (j == jt - 1);
-    sc[j] = forced ? -1.f : src[j];
-    if (forced) atomicOr(&bits[j >> 5], 1u << (j & 31));
+  // stage the candidate scores, 8 independent loads per lane in flight; forced blocks are
+  // marked selected and kept out of the candidate set (score -1)
+  for (int base = 0; base <= jt; base += 256) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = base + u * 32 + lane;
+      v[u] = j <= jt ? src[j] : -1.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = base + u * 32 + lane;
+      if (j <= jt) sc[j] = (j == 0 || j == jt || j == jt - 1) ? -1.f : v[u];
+    }
+  }
+  if (lane == 0) {
+    bits[0] |= 1u;
+    if (jt >= 1) bits[jt >> 5] |= 1u << (jt & 31);
+    if (jt >= 2) bits[(jt - 1) >> 5] |= 1u << ((jt - 1) & 31);
   }
   __syncwarp();
   const int nf = 1 + (jt >= 1 ? 1 : 0) + (jt >= 2 ? 1 : 0);
   const int k = min(top_n - nf, jt + 1 - nf);
-  auto local_best = [&]() -> unsigned long long {
-    unsigned long long best = 0ull;
+  if (k > 0) {
+    // 1. the two largest keys of this lane's subset
+    unsigned long long k1 = 0ull, k2 = 0ull;
     for (int j = lane; j <= jt; j += 32) {
-      const float x = sc[j];
-      if (x >= 0.f) {
-        const unsigned long long key =
-            (static_cast<unsigned long long>(__float_as_uint(x)) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(j));
-        best = key > best ? key : best;
+      const unsigned long long key = cand_key(sc[j], j);
+      if (key > k1) {
+        k2 = k1;
+        k1 = key;
+      } else if (key > k2) {
+        k2 = key;
       }
     }
-    return best;
-  };
-  unsigned long long mine = local_best();
-  for (int round = 0; round < k; ++round) {
-    const unsigned long long win = warp_max_u64(mine);
-    if (win == 0ull) break;
-    const int j = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(win & 0xFFFFFFFFull));
-    if ((j & 31) == lane) {
-      sc[j] = -1.f;
-      bits[j >> 5] |= 1u << (j & 31);
-      mine = local_best();
+    // 2. threshold = k-th largest of the 64 lane-top-2 keys (0 if fewer exist)
+    unsigned long long thr = 0ull;
+    {
+      unsigned long long a = k1, b2 = k2;
+      for (int round = 0; round < k && round < 64; ++round) {
+        const unsigned long long w = warp_max_u64(a);
+        thr = w;
+        if (w == 0ull) break;
+        if (a == w) {
+          a = b2;
+          b2 = 0ull;
+        }
+      }
+      if (k > 64) thr = 0ull;
+    }
+    // 3. compact the survivors (keys >= threshold)
+    int nsurv = 0;
+    for (int base = 0; base <= jt; base += 32) {
+      const int j = base + lane;
+      const unsigned long long key = j <= jt ? cand_key(sc[j], j) : 0ull;
+      const bool keep = key != 0ull && key >= thr;
+      const uint32_t m = __ballot_sync(0xffffffffu, keep);
+      if (keep) list[nsurv + __popc(m & ((1u << lane) - 1u))] = j;
+      nsurv += __popc(m);
     }
     __syncwarp();
+    // 4. exact top-k among the survivors
+    auto local_best = [&]() -> unsigned long long {
+      unsigned long long best = 0ull;
+      for (int i = lane; i < nsurv; i += 32) {
+        const int j = list[i];
+        const unsigned long long key = cand_key(sc[j], j);
+        best = key > best ? key : best;
+      }
+      return best;
+    };
+    unsigned long long mine = local_best();
+    for (int round = 0; round < k; ++round) {
+      const unsigned long long win = warp_max_u64(mine);
+      if (win == 0ull) break;
+      const int j = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(win & 0xFFFFFFFFull));
+      if (win == mine) {
+        sc[j] = -1.f;
+        bits[j >> 5] |= 1u << (j & 31);
+        mine = local_best();
+      }
+      __syncwarp();
+    }
   }
   // emit the selected set in ascending order, then -1 padding
   int pos = 0;
@@ -99,8 +159,9 @@ __global__ void __launch_bounds__(kTopnWarps * 32) topn_kernel(const float* __re
   extern __shared__ float tsm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwords = (nsel + 31) / 32;
-  float* sc = tsm + static_cast<size_t>(warp) * (nsel + nwords);
-  uint32_t* bits = reinterpret_cast<uint32_t*>(sc + nsel);
+  float* sc = tsm + static_cast<size_t>(warp) * (2 * nsel + nwords);
+  int* list = reinterpret_cast<int*>(sc + nsel);
+  uint32_t* bits = reinterpret_cast<uint32_t*>(list + nsel);
   for (int item = blockIdx.x * kTopnWarps + warp; item < nitems; item += gridDim.x * kTopnWarps) {
     const int t = item / hkv;
     const int jt = t / sel_len;
@@ -108,7 +169,8 @@ __global__ void __launch_bounds__(kTopnWarps * 32) topn_kernel(const float* __re
       if (lane == 0) record_error(kErrBadIndex);
       continue;
     }
-    warp_topn(sc, bits, scores + static_cast<size_t>(item) * nsel, jt, top_n, idx + static_cast<size_t>(item) * top_n,
+    warp_topn(sc, bits, list, scores + static_cast<size_t>(item) * nsel, jt, top_n,
+              idx + static_cast<size_t>(item) * top_n,
               idx_copy ? idx_copy + static_cast<size_t>(item) * top_n : nullptr, lane);
   }
 }
