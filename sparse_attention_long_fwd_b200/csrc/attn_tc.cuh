@@ -23,9 +23,9 @@
 // next block while computing the current one, tiling against register pressure) are
 // met here by TMA tiles, an mbarrier ring and TMEM accumulators.
 //
-// Warp roles (320 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues the
-// MMAs (one elected lane), warps 2..9 (two warpgroups; each thread owns one TMEM lane /
-// MMA row and one half of the key columns) do the softmax, the score binning and the
+// Warp roles (576 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues the
+// MMAs (one elected lane), warps 2..17 (four warpgroups; each thread owns one TMEM lane /
+// MMA row and a quarter of the key columns) do the softmax, the score binning and the
 // epilogue. Every wait is bounded (sm100.cuh).
 #pragma once
 #include <cuda_bf16.h>
@@ -55,7 +55,11 @@ struct AttnArgs {
   int out_f32;
 };
 
-constexpr int kAttnThreads = 320;  // producer, MMA, 2 x 4 softmax warps
+constexpr int kSoftmaxWG = 4;                        // softmax warpgroups sharing each S tile
+constexpr int kSoftmaxThreads = 128 * kSoftmaxWG;
+constexpr int kAttnThreads = 64 + kSoftmaxThreads;    // producer warp, MMA warp, softmax warps
+constexpr int kColsPerWG = 128 / kSoftmaxWG;          // key columns (and output columns / D*128) per warpgroup
+constexpr int kBinsPerWG = kColsPerWG / 4;            // selection blocks per warpgroup per tile
 constexpr int kBN = 128;      // keys per tile
 constexpr int kStages = 2;    // TMA ring depth (K and V tiles)
 
@@ -67,7 +71,7 @@ struct AttnSmem {
   alignas(1024) uint8_t k[kStages][kChunks][kTileBytes];
   alignas(1024) uint8_t v[kStages][kChunks][kTileBytes];
   alignas(1024) uint8_t p[2][kTileBytes];            // P tile: 128 rows x 128 keys bf16
-  float lse_x[2][128][2];     // per warpgroup: (scaled max, sum) of the row's half
+  float lse_x[kSoftmaxWG][128][2];  // per warpgroup: (scaled max, sum) of the row's columns
   uint64_t q_full;
   uint64_t full[kStages], empty[kStages];
   uint64_t s_full[2], s_free[2];
@@ -79,18 +83,25 @@ struct AttnSmem {
 
 __device__ __forceinline__ int ncmp_visible(int t, int l, int s) { return (t + 1 >= l) ? (t + 1 - l) / s + 1 : 0; }
 
-// Reduce-scatter of 16 per-lane values over groups of GP adjacent lanes: afterwards
-// bin[0 .. 16/GP) of lane l holds the group sums of entries [(l%GP)*16/GP, ...).
-template <int GP>
-__device__ __forceinline__ void group_reduce_scatter(float (&bin)[16], int lane) {
+// Reduce over groups of GP adjacent lanes of NB per-lane values. With GP <= NB each lane
+// ends with NB/GP group sums, bin[0 .. NB/GP) = entries [(l%GP)*NB/GP, ...). With GP > NB
+// the halving stops at one entry and the remaining stages add; lane l then holds entry
+// (l%GP) / (GP/NB), shared with the GP/NB - 1 lanes next to it.
+template <int GP, int NB>
+__device__ __forceinline__ void group_reduce_scatter(float (&bin)[NB], int lane) {
 #pragma unroll
-  for (int o = GP / 2, n = 16; o >= 1; o >>= 1, n >>= 1) {
-    const bool upper = (lane & o) != 0;
+  for (int o = GP / 2, n = NB; o >= 1; o >>= 1) {
+    if (n > 1) {
+      const bool upper = (lane & o) != 0;
 #pragma unroll
-    for (int i = 0; i < n / 2; ++i) {
-      const float send = upper ? bin[i] : bin[i + n / 2];
-      const float keep = upper ? bin[i + n / 2] : bin[i];
-      bin[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      for (int i = 0; i < n / 2; ++i) {
+        const float send = upper ? bin[i] : bin[i + n / 2];
+        const float keep = upper ? bin[i + n / 2] : bin[i];
+        bin[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+      n >>= 1;
+    } else {
+      bin[0] += __shfl_xor_sync(0xffffffffu, bin[0], o);
     }
   }
 }
@@ -137,9 +148,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.s_full[b], 1);
-      mbar_init(&sm.s_free[b], 8);
+      mbar_init(&sm.s_free[b], 4 * kSoftmaxWG);
     }
-    mbar_init(&sm.p_full, 8);
+    mbar_init(&sm.p_full, 4 * kSoftmaxWG);
     mbar_init(&sm.p_free, 1);
     mbar_init(&sm.o_full, 1);
     mbar_init(&sm.drain, 1);
@@ -154,7 +165,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (warp >= 2) {
     // rows T*Gp .. 127 of the Q tile are never written by TMA: keep them finite (zero)
     const int r0 = T * args.Gp;
-    for (int i = tid - 64; i < (128 - r0) * 8 * kChunks; i += 256) {
+    for (int i = tid - 64; i < (128 - r0) * 8 * kChunks; i += kSoftmaxThreads) {
       const int c = i / ((128 - r0) * 8);
       const int rem = i % ((128 - r0) * 8);
       *reinterpret_cast<uint4*>(&sm.q[c][(r0 + rem / 8) * 128 + (rem % 8) * 16]) = make_uint4(0, 0, 0, 0);
@@ -243,14 +254,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ softmax / epilogue
-    // Two warpgroups share every S tile: warpgroup `wg` owns keys [64*wg, 64*wg + 64) of
-    // each 128-key tile (and output columns [wg*D/2, (wg+1)*D/2) in the epilogue); the
-    // thread of TMEM lane r in each warpgroup handles MMA row r.
-    const int sw = warp - 2;                 // softmax warp 0..7
-    const int wg = sw >> 2;                  // column half
+    // kSoftmaxWG warpgroups share every S tile: warpgroup `wg` owns key columns
+    // [wg*kColsPerWG, (wg+1)*kColsPerWG) of each 128-key tile (and the same slice of the D
+    // output columns in the epilogue); its thread of TMEM lane r handles MMA row r.
+    const int sw = warp - 2;                 // softmax warp
+    const int wg = sw >> 2;                  // column slice
     const int q4 = warp & 3;                 // TMEM lane quadrant of this warp
     const int r = q4 * 32 + lane;            // MMA row
-    const int stid = sw * 32 + lane;         // 0..255
     const int Gp = args.Gp;
     const int tok = r / Gp, hh = r % Gp;
     const int t = t0 + tok;
@@ -268,10 +278,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
     }
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-    const int col0 = wg * 64;
+    const int col0 = wg * kColsPerWG;
     const float sl2 = args.scale_log2;
     bool ok = true;
-    // ---- phase 1: log-sum-exp (base 2) of this row's half, combined across halves below
+    // ---- phase 1: log-sum-exp (base 2) of this row's column slice, combined below
     float m = -INFINITY, lsum = 0.f;         // m: running max of the raw (unscaled) scores
     for (int kt = 0; kt < nkt && ok; ++kt) {
       const int b = kt & 1;
@@ -280,18 +290,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const int kbase = kb + kt * kBN + col0;
-      const bool full = kbase >= rb && kbase + 64 <= re;
-      float s[64];
+      const bool full = kbase >= rb && kbase + kColsPerWG <= re;
+      float s[kColsPerWG];
       __syncwarp();
-      tmem_ld32(trow + b * kBN + col0, *reinterpret_cast<float(*)[32]>(&s[0]));
-      tmem_ld32(trow + b * kBN + col0 + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
+#pragma unroll
+      for (int c = 0; c < kColsPerWG / 32; ++c)
+        tmem_ld32(trow + b * kBN + col0 + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.s_free[b]);  // S is in registers: the buffer may be reused
       if (!full) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
+        for (int i = 0; i < kColsPerWG; ++i) {
           const int kidx = kbase + i;
           s[i] = (kidx >= rb && kidx < re) ? s[i] : -INFINITY;
         }
@@ -300,7 +311,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
       for (int c = 0; c < 8; ++c) mx[c] = s[c];
 #pragma unroll
-      for (int i = 8; i < 64; i += 8)
+      for (int i = 8; i < kColsPerWG; i += 8)
 #pragma unroll
         for (int c = 0; c < 8; ++c) mx[c] = fmaxf(mx[c], s[i + c]);
       const float cmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
@@ -312,7 +323,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int c = 0; c < 8; ++c) acc[c] = ex2_approx(fmaf(s[c], sl2, -ms));
 #pragma unroll
-        for (int i = 8; i < 64; i += 8)
+        for (int i = 8; i < kColsPerWG; i += 8)
 #pragma unroll
           for (int c = 0; c < 8; ++c) acc[c] += ex2_approx(fmaf(s[i + c], sl2, -ms));
         lsum = lsum * ex2_approx((m - mnew) * sl2) +
@@ -322,15 +333,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     sm.lse_x[wg][r][0] = (m == -INFINITY) ? -INFINITY : m * sl2;
     sm.lse_x[wg][r][1] = lsum;
-    named_bar_sync(3, 256);
+    named_bar_sync(3, kSoftmaxThreads);
     float lse2;
     bool has_keys;
     {
-      const float ma = sm.lse_x[0][r][0], la = sm.lse_x[0][r][1];
-      const float mb = sm.lse_x[1][r][0], lb = sm.lse_x[1][r][1];
-      const float M = fmaxf(ma, mb);
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kSoftmaxWG; ++w) M = fmaxf(M, sm.lse_x[w][r][0]);
       float L = 0.f;
-      if (M != -INFINITY) L = la * ex2_approx(ma - M) + lb * ex2_approx(mb - M);
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < kSoftmaxWG; ++w) L += sm.lse_x[w][r][1] * ex2_approx(sm.lse_x[w][r][0] - M);
+      }
       has_keys = L > 0.f;
       lse2 = has_keys ? M + __log2f(L) : INFINITY;
     }
@@ -338,13 +352,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // Block scores (kModeCmp): compressed block i covers tokens [16i, 16i+32) and selection
     // block j covers [64j, 64j+64), so block j takes all of compressed blocks 4j..4j+2 and
     // half of 4j-1 and 4j+3. A 128-key tile holds selection blocks kt2*32 .. kt2*32+31;
-    // this warpgroup's 64 keys hold 16 of them. The one compressed block that straddles
-    // the previous 64 keys is re-read from TMEM by this thread (column 63 for warpgroup 1,
-    // the previous tile's column 127 for warpgroup 0, kept from the previous iteration),
-    // so the halves never exchange data. The G heads of a token sit in Gp adjacent lanes;
-    // a shuffle reduce-scatter sums them, leaving 16/Gp consecutive blocks per lane.
+    // this warpgroup's columns hold kBinsPerWG of them. The one compressed block that
+    // straddles the previous column slice is re-read from TMEM by this thread (column
+    // col0-1, or for warpgroup 0 the previous tile's column 127, kept from the previous
+    // iteration), so the slices never exchange data. The G heads of a token sit in Gp
+    // adjacent lanes; a shuffle reduce-scatter sums them.
     float carry = 0.f;  // warpgroup 0: half of the previous tile's last compressed block
-    const int bpl = 16 / Gp;  // blocks per lane after the reduce-scatter (kModeCmp)
     for (int kt2 = 0; kt2 < nkt; ++kt2) {
       const int job = nkt + kt2;
       const int b = job & 1;
@@ -354,15 +367,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const int kbase = kb + kt2 * kBN + col0;
-      const bool full = kbase >= rb && kbase + 64 <= re;
-      float bin[16];
+      const bool full = kbase >= rb && kbase + kColsPerWG <= re;
+      float bin[kBinsPerWG];
       float half_in = 0.f;
-      float s[64];
+      float s[kColsPerWG];
       uint32_t xv = 0;
-      const int xcol = wg == 1 ? 63 : 127;  // (kModeCmp) the straddling block's column
+      const int xcol = wg > 0 ? col0 - 1 : 127;  // (kModeCmp) the straddling block's column
       __syncwarp();
-      tmem_ld32(trow + b * kBN + col0, *reinterpret_cast<float(*)[32]>(&s[0]));
-      tmem_ld32(trow + b * kBN + col0 + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
+#pragma unroll
+      for (int c = 0; c < kColsPerWG / 32; ++c)
+        tmem_ld32(trow + b * kBN + col0 + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
       if (MODE == kModeCmp)
         asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(xv) : "r"(trow + b * kBN + xcol));
       tmem_wait_ld();
@@ -370,11 +384,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.s_free[b]);  // S is in registers: the buffer may be reused
       if (MODE == kModeCmp) {
-        // the straddling block's probability: column 63 (wg 1) or this tile's column 127
-        // (wg 0, carried into the next tile)
         const int xk = kb + kt2 * kBN + xcol;
         const float px = (xk >= rb && xk < re) ? ex2_approx(fmaf(__uint_as_float(xv), sl2, -lse2)) : 0.f;
-        if (wg == 1) {
+        if (wg > 0) {
           half_in = 0.5f * px;
         } else {
           half_in = carry;
@@ -383,51 +395,53 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       if (full) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) s[i] = ex2_approx(fmaf(s[i], sl2, -lse2));
+        for (int i = 0; i < kColsPerWG; ++i) s[i] = ex2_approx(fmaf(s[i], sl2, -lse2));
       } else {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
+        for (int i = 0; i < kColsPerWG; ++i) {
           const int kidx = kbase + i;
           s[i] = (kidx >= rb && kidx < re) ? ex2_approx(fmaf(s[i], sl2, -lse2)) : 0.f;
         }
       }
       if (MODE == kModeCmp) {
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
+        for (int u = 0; u < kBinsPerWG; ++u) {
           const float half_last = 0.5f * s[4 * u + 3];
           bin[u] = (u == 0 ? half_in : 0.5f * s[4 * u - 1]) + s[4 * u] + s[4 * u + 1] + s[4 * u + 2] + half_last;
         }
       }
-      // P row r, keys col0 .. col0+63 -> chunk wg
-      uint8_t* pc = sm.p[wg];
+      // P row r, keys col0 .. col0+kColsPerWG-1 -> chunk col0/64, columns col0%64 ..
+      uint8_t* pc = sm.p[col0 >> 6];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < kColsPerWG / 8; ++u) {
         uint4 w;
         w.x = pack_bf16x2(s[8 * u + 0], s[8 * u + 1]);
         w.y = pack_bf16x2(s[8 * u + 2], s[8 * u + 3]);
         w.z = pack_bf16x2(s[8 * u + 4], s[8 * u + 5]);
         w.w = pack_bf16x2(s[8 * u + 6], s[8 * u + 7]);
-        *reinterpret_cast<uint4*>(pc + sw128_offset(r, 8 * u)) = w;
+        *reinterpret_cast<uint4*>(pc + sw128_offset(r, (col0 & 63) + 8 * u)) = w;
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full);
       if (MODE == kModeCmp) {
-        // reduce-scatter over the Gp lanes of this token: afterwards lane hh holds the
-        // group sums of blocks [hh*bpl, (hh+1)*bpl) of this warpgroup's 16
         switch (Gp) {
-          case 2: group_reduce_scatter<2>(bin, lane); break;
-          case 4: group_reduce_scatter<4>(bin, lane); break;
-          case 8: group_reduce_scatter<8>(bin, lane); break;
-          case 16: group_reduce_scatter<16>(bin, lane); break;
+          case 2: group_reduce_scatter<2, kBinsPerWG>(bin, lane); break;
+          case 4: group_reduce_scatter<4, kBinsPerWG>(bin, lane); break;
+          case 8: group_reduce_scatter<8, kBinsPerWG>(bin, lane); break;
+          case 16: group_reduce_scatter<16, kBinsPerWG>(bin, lane); break;
           default: break;
         }
-        if (t < args.q_end && r < T * Gp) {
+        // lane hh now holds blocks [hh*bpl, (hh+1)*bpl) of this slice (Gp <= kBinsPerWG),
+        // or block hh/(Gp/kBinsPerWG) shared with its neighbours (Gp > kBinsPerWG)
+        const int bpl = Gp <= kBinsPerWG ? kBinsPerWG / Gp : 1;
+        const int share = Gp <= kBinsPerWG ? 1 : Gp / kBinsPerWG;
+        if (t < args.q_end && (hh % share) == 0) {
           const int jt = t / args.sel_len;
-          const int j0 = kt2 * 32 + wg * 16 + hh * bpl;
+          const int j0 = kt2 * 32 + wg * kBinsPerWG + (hh / share) * bpl;
           float* dst = args.scores + (static_cast<size_t>(t) * args.hkv + g) * args.nsel;
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
+          for (int i = 0; i < kBinsPerWG; ++i)
             if (i < bpl && j0 + i <= jt) dst[j0 + i] = bin[i];
         }
       }
@@ -440,7 +454,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int o = 1; o < 16; o <<= 1)
         if (o < Gp) c += __shfl_xor_sync(0xffffffffu, c, o);
       const int j = nkt * 32;
-      if (hh == 0 && t < args.q_end && r < T * Gp && j <= t / args.sel_len)
+      if (hh == 0 && t < args.q_end && j <= t / args.sel_len)
         args.scores[(static_cast<size_t>(t) * args.hkv + g) * args.nsel + j] = c;
     }
     // ---- epilogue (every lane loads its TMEM row; only valid rows are stored)
@@ -457,12 +471,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         g2 = args.gates[(static_cast<size_t>(t) * args.hq + h) * 3 + 2];
       }
 #pragma unroll 1
-      for (int cc = 0; cc < D / 64; ++cc) {
-        const int c0 = wg * (D / 2) + cc * 32;  // output columns c0 .. c0+31
+      for (int cc = 0; cc < (D / kSoftmaxWG + 31) / 32; ++cc) {
+        constexpr int kOC = D / kSoftmaxWG < 32 ? D / kSoftmaxWG : 32;  // output columns per load
+        const int c0 = wg * (D / kSoftmaxWG) + cc * 32;                 // output columns c0 .. c0+kOC-1
         float o[32];
         __syncwarp();
         if (nkt > 0) {
-          tmem_ld32(trow + kColO + c0, o);
+          if (kOC == 32) {
+            tmem_ld32(trow + kColO + c0, o);
+          } else {
+            tmem_ld16(trow + kColO + c0, *reinterpret_cast<float(*)[16]>(&o[0]));
+          }
           tmem_wait_ld();
         } else {
 #pragma unroll
@@ -473,13 +492,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         } else if (MODE == kModeCmp) {
           float4* dst = reinterpret_cast<float4*>(args.o_cmp + orow + c0);
 #pragma unroll
-          for (int u = 0; u < 8; ++u) dst[u] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+          for (int u = 0; u < kOC / 4; ++u) dst[u] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
         } else {
           if (MODE == kModeWin) {
             const float4* oc = reinterpret_cast<const float4*>(args.o_cmp + orow + c0);
             const float4* os = reinterpret_cast<const float4*>(args.o_sel + orow + c0);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
+            for (int u = 0; u < kOC / 4; ++u) {
               const float4 a = oc[u], c = os[u];
               o[4 * u + 0] = g0 * a.x + g1 * c.x + g2 * o[4 * u + 0];
               o[4 * u + 1] = g0 * a.y + g1 * c.y + g2 * o[4 * u + 1];
@@ -490,11 +509,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (args.out_f32) {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.out) + orow + c0);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) dst[u] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+            for (int u = 0; u < kOC / 4; ++u) dst[u] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
           } else {
             uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) + orow + c0);
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
+            for (int u = 0; u < kOC / 8; ++u)
               dst[u] = make_uint4(pack_bf16x2(o[8 * u], o[8 * u + 1]), pack_bf16x2(o[8 * u + 2], o[8 * u + 3]),
                                   pack_bf16x2(o[8 * u + 4], o[8 * u + 5]), pack_bf16x2(o[8 * u + 6], o[8 * u + 7]));
           }

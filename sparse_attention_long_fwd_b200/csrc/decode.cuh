@@ -50,7 +50,7 @@ struct DecArgs {
 
 template <int D>
 struct DecSmem {
-  WarpChunkBuf<D> buf[kDecWarps];
+  WarpChunkBuf<D, kChunkKeys, 2> buf[kDecWarps];
   WarpPartial<D> part[kDecWarps];
   int chunk_start[kDecWarps][128];
 };
@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) dec_cmp_kernel(const __nv_bflo
   const __nv_bfloat16* kb = kcmp + static_cast<size_t>(b) * a.ncmax * rs + static_cast<size_t>(g) * D;
   const __nv_bfloat16* vb = vcmp + static_cast<size_t>(b) * a.ncmax * rs + static_cast<size_t>(g) * D;
   float* lg = a.logits + static_cast<size_t>(bg) * a.G * a.ncmax;
-  WarpChunkBuf<D>& buf = sm.buf[warp];
+  auto& buf = sm.buf[warp];
   WarpAttnState<D> st;
   state_init(st);
   const int nch = w1 > w0 ? (w1 - w0 + kChunkKeys - 1) / kChunkKeys : 0;
@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) dec_branch_kernel(const __nv_b
   const size_t rs = static_cast<size_t>(a.hkv) * D;
   const __nv_bfloat16* kb = kcache + static_cast<size_t>(b) * a.lmax * rs + static_cast<size_t>(g) * D;
   const __nv_bfloat16* vb = vcache + static_cast<size_t>(b) * a.lmax * rs + static_cast<size_t>(g) * D;
-  WarpChunkBuf<D>& buf = sm.buf[warp];
+  auto& buf = sm.buf[warp];
   WarpAttnState<D> st;
   state_init(st);
   const int my = nch > warp ? (nch - warp + kDecWarps - 1) / kDecWarps : 0;

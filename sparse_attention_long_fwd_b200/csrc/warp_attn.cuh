@@ -18,10 +18,11 @@ namespace nsa {
 
 constexpr int kChunkKeys = 32;
 
-template <int D>
+// Per-warp ring of NST stages, each CK key rows and CK value rows of D bf16; 16-byte
+// units are XOR-swizzled by (key & 7) so ldmatrix reads are conflict-free.
+template <int D, int CK = kChunkKeys, int NST = 2>
 struct WarpChunkBuf {
-  // [2 stages][K/V][32 keys][D] bf16, 16-byte units XOR-swizzled by (key & 7)
-  alignas(128) __nv_bfloat16 kv[2][2][kChunkKeys * D];
+  alignas(128) __nv_bfloat16 kv[NST][2][CK * D];
 };
 
 template <int D>
@@ -75,16 +76,16 @@ __device__ __forceinline__ void load_q_frags(uint32_t (&a)[D / 16][4], const __n
   }
 }
 
-// Copy 32 key rows (and value rows) starting at token `start` into ring stage `st`.
+// Copy CK key rows (and value rows) starting at token `start` into ring stage `st`.
 // Rows at or beyond `row_end` are zero-filled and never read from global memory.
 // K/V row `tok` of the head lives at base + tok * row_stride.
-template <int D>
-__device__ __forceinline__ void load_chunk(WarpChunkBuf<D>& buf, int st, const __nv_bfloat16* kbase,
+template <int D, int CK, int NST>
+__device__ __forceinline__ void load_chunk(WarpChunkBuf<D, CK, NST>& buf, int st, const __nv_bfloat16* kbase,
                                            const __nv_bfloat16* vbase, size_t row_stride, int start, int row_end,
                                            int lane) {
   constexpr int kUnits = D / 8;  // 16-byte units per row
 #pragma unroll
-  for (int i = lane; i < kChunkKeys * kUnits; i += 32) {
+  for (int i = lane; i < CK * kUnits; i += 32) {
     const int row = i / kUnits, unit = i % kUnits;
     const int tok = start + row;
     const bool valid = tok < row_end;
@@ -103,23 +104,25 @@ __device__ __forceinline__ void state_init(WarpAttnState<D>& s) {
   for (int n = 0; n < D / 8; ++n) s.o[n][0] = s.o[n][1] = s.o[n][2] = s.o[n][3] = 0.f;
 }
 
-// One 32-key chunk from ring stage `st`: keys start .. start+31; key `start + c` is
+// One CK-key chunk from ring stage `st`: keys start .. start+CK-1; key `start + c` is
 // used iff key_lo <= start + c < key_hi. `sl2` = softmax scale * log2(e).
 // If `logits` is non-null, the scaled base-2 logits of rows < G are stored there:
 // logits[row * logit_stride + (start + c - logit_base)] for valid keys.
-template <int D>
+template <int D, int CK, int NST>
 __device__ __forceinline__ void attend_chunk(WarpAttnState<D>& s, const uint32_t (&qa)[D / 16][4],
-                                             const WarpChunkBuf<D>& buf, int st, int start, int key_lo,
+                                             const WarpChunkBuf<D, CK, NST>& buf, int st, int start, int key_lo,
                                              int key_hi, float sl2, int lane, float* logits = nullptr,
                                              int logit_stride = 0, int logit_base = 0, int G = 0) {
+  constexpr int NT = CK / 8;   // n-tiles of 8 keys
+  constexpr int KS = CK / 16;  // 16-key k-steps of P V
   const uint32_t kaddr = smem_u32(&buf.kv[st][0][0]);
   const uint32_t vaddr = smem_u32(&buf.kv[st][1][0]);
-  // ---- S = Q K^T : 16 rows x 32 keys (4 n-tiles of 8 keys)
-  float sc[4][4];
+  // ---- S = Q K^T : 16 rows x CK keys (NT n-tiles of 8 keys)
+  float sc[NT][4];
 #pragma unroll
-  for (int nt = 0; nt < 4; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+  for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
 #pragma unroll
-  for (int nt = 0; nt < 4; ++nt) {
+  for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
     for (int ks = 0; ks < D / 16; ks += 2) {
       const int row = nt * 8 + (lane & 7);
@@ -133,7 +136,7 @@ __device__ __forceinline__ void attend_chunk(WarpAttnState<D>& s, const uint32_t
   // ---- online softmax (rows r0 = lane/4 -> elements 0,1; r1 = r0+8 -> elements 2,3)
   float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-  for (int nt = 0; nt < 4; ++nt) {
+  for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int key = start + nt * 8 + 2 * (lane & 3) + (e & 1);
@@ -145,7 +148,7 @@ __device__ __forceinline__ void attend_chunk(WarpAttnState<D>& s, const uint32_t
   if (logits != nullptr) {
     const int r0 = lane >> 2;
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
+    for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int row = r0 + (e >> 1) * 8;
@@ -169,9 +172,9 @@ __device__ __forceinline__ void attend_chunk(WarpAttnState<D>& s, const uint32_t
   }
   s.l[0] *= alpha[0];
   s.l[1] *= alpha[1];
-  uint32_t pa[2][4];  // P as A fragments for the two 16-key k-steps
+  uint32_t pa[KS][4];  // P as A fragments for the 16-key k-steps
 #pragma unroll
-  for (int nt = 0; nt < 4; ++nt) {
+  for (int nt = 0; nt < NT; ++nt) {
     float p[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -193,7 +196,7 @@ __device__ __forceinline__ void attend_chunk(WarpAttnState<D>& s, const uint32_t
   }
   // ---- O += P V : V chunk rows are keys (k), columns are output dims (n)
 #pragma unroll
-  for (int kk = 0; kk < 2; ++kk) {
+  for (int kk = 0; kk < KS; ++kk) {
 #pragma unroll
     for (int n = 0; n < D / 8; n += 2) {
       const int row = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
