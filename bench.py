@@ -32,6 +32,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from sparse_attention_long_fwd_b200 import dist as dist_helpers  # noqa: E402
 from sparse_attention_long_fwd_b200 import nsa  # noqa: E402
 from sparse_attention_long_fwd_b200.inputs import WORKLOADS, decode_inputs, prefill_inputs  # noqa: E402
 
@@ -152,29 +153,19 @@ class ClockSampler:
 # ---------------------------------------------------------------------------- helpers
 
 def dist_setup():
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = dist_helpers.rank_env()
     if world > 1:
-        import datetime
-
         torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
+    dist_helpers.init("nccl", 120, torch.device("cuda", local) if world > 1 else None)
     return world, rank, local
 
 
 def barrier(world):
-    if world > 1:
-        torch.distributed.barrier()
+    dist_helpers.barrier(world)
 
 
 def max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    return float(t.item())
+    return dist_helpers.max_over_ranks(x, world, device="cuda")
 
 
 def timed_steps(fn, steps, warmup, flush, n_stage_events):
@@ -243,7 +234,7 @@ def run_b200(args, world, rank, local):
     total_ms = max_over_ranks(sum(step_ms), world)
     ms_per_step = total_ms / args.steps
     tokens = w.n_video * world
-    value = tokens / (ms_per_step / 1e3)
+    value = dist_helpers.aggregate_rate(w.n_video, world, ms_per_step / 1e3)
     stages = stage_times(stage_ev, PREFILL_STAGES, n_stages)
     flops = counts["cmp_flops"] + counts["sel_flops"] + counts["win_flops"] + counts["text_flops"]
     tflops = flops / (sum(step_ms) / args.steps / 1e3) / 1e12
