@@ -16,9 +16,12 @@
 // in 128-key tiles through a TMA ring, twice:
 //   phase 1  S = Q K^T on the tensor core (TMEM accumulator), then each row's exact
 //            log-sum-exp with an online max (no P*V, no output rescaling);
-//   phase 2  S again, P = exp2(S*scale*log2e - lse2) already normalised, written to
-//            shared memory as bf16 and accumulated O += P V in TMEM. Because P is final,
-//            the compressed mode can bin it into block scores in the same pass.
+//   phase 2  S again, P = exp2(S*scale*log2e - lse2) already normalised, written to TMEM
+//            as bf16 and accumulated O += P V in TMEM by a tcgen05 MMA that reads P
+//            from TMEM. Because P is final, the compressed mode
+//            can bin it into block scores in the same pass.
+// K and V tiles stream through a ring of shared-memory slots (one tile each); the MMA
+// releases a slot as soon as the MMA that read it is done.
 // The pages' kernel notes (CSDN blog, section 5.1: fixed 64x64 blocks, prefetching the
 // next block while computing the current one, tiling against register pressure) are
 // met here by TMA tiles, an mbarrier ring and TMEM accumulators.
@@ -61,25 +64,45 @@ constexpr int kAttnThreads = 64 + kSoftmaxThreads;    // producer warp, MMA warp
 constexpr int kColsPerWG = 128 / kSoftmaxWG;          // key columns (and output columns / D*128) per warpgroup
 constexpr int kBinsPerWG = kColsPerWG / 4;            // selection blocks per warpgroup per tile
 constexpr int kBN = 128;      // keys per tile
-constexpr int kStages = 2;    // TMA ring depth (K and V tiles)
 
 template <int D>
 struct AttnSmem {
   static constexpr int kChunks = D / 64;             // 64-element (128 B) column chunks
   static constexpr int kTileBytes = 128 * 128;       // one chunk of a 128-row tile
+  static constexpr int kSlotBytes = kChunks * kTileBytes;
+  // ring of K/V tile slots: as many as fit beside the Q tile in 227 KB
+  static constexpr int kSlots = D == 128 ? 5 : 8;
   alignas(1024) uint8_t q[kChunks][kTileBytes];
-  alignas(1024) uint8_t k[kStages][kChunks][kTileBytes];
-  alignas(1024) uint8_t v[kStages][kChunks][kTileBytes];
-  alignas(1024) uint8_t p[2][kTileBytes];            // P tile: 128 rows x 128 keys bf16
+  alignas(1024) uint8_t slot[kSlots][kChunks][kTileBytes];
   float lse_x[kSoftmaxWG][128][2];  // per warpgroup: (scaled max, sum) of the row's columns
   uint64_t q_full;
-  uint64_t full[kStages], empty[kStages];
+  uint64_t full[kSlots], empty[kSlots];
   uint64_t s_full[2], s_free[2];
   uint64_t p_full, p_free, o_full, drain;
   uint32_t tmem_base;
   int abort_flag;
-  int jobs_consumed;
 };
+
+// P (bf16, packed in pairs) goes to its own double-buffered TMEM columns and is read back
+// by the tensor core as the A operand of the P.V MMA ("TS" form: A from TMEM; a column
+// holds two consecutive keys, the lower key in the low half).
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
 
 __device__ __forceinline__ int ncmp_visible(int t, int l, int s) { return (t + 1 >= l) ? (t + 1 - l) / s + 1 : 0; }
 
@@ -114,6 +137,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   constexpr int kChunks = Smem::kChunks;
   constexpr uint32_t kTmemCols = 512;
   constexpr uint32_t kColO = 256;  // S buffers at columns 0 and 128, O at 256
+  constexpr uint32_t kColP = 384;  // P buffers (bf16 pairs, 64 columns each) at 384 and 448
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -138,13 +162,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     ke = t_last + 1;
   }
   const int nkt = (ke - kb + kBN - 1) / kBN;
-  const int njobs = 2 * nkt;
+  const int njobs = 2 * nkt;   // MMA jobs: nkt score tiles (phase 1), then nkt score + P.V tiles
+  const int nloads = 3 * nkt;  // TMA loads: K tiles (phase 1), then K and V per tile (phase 2)
+  constexpr int kSlots = Smem::kSlots;
 
   if (tid == 0) {
     mbar_init(&sm.q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], 1);
+    for (int x = 0; x < Smem::kSlots; ++x) {
+      mbar_init(&sm.full[x], 1);
+      mbar_init(&sm.empty[x], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.s_full[b], 1);
@@ -155,7 +181,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(&sm.o_full, 1);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
-    sm.jobs_consumed = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -177,26 +202,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort_flag = &sm.abort_flag;
-  int issued = 0;  // producer: jobs whose TMA was issued
+  int issued = 0;  // producer: loads whose TMA was issued
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
+    // load L: L < nkt -> K tile L (phase 1); else x = L - nkt -> K (x even) or V (x odd) of
+    // tile x/2 (phase 2). Load L goes to slot L % kSlots once the MMA has released the
+    // load kSlots before it.
     if (lane == 0 && nkt > 0) {
       tma_prefetch_desc(&qmap);
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
       mbar_arrive_expect_tx(&sm.q_full, kChunks * T * args.Gp * 128);
       for (int c = 0; c < kChunks; ++c) tma_load_3d(&qmap, &sm.q_full, sm.q[c], c * 64, g * G, t0);
-      for (int job = 0; job < njobs; ++job) {
-        const int stage = job % kStages;
-        if (job >= kStages && !mbar_wait(&sm.empty[stage], ((job / kStages) - 1) & 1, abort_flag)) break;
-        const bool p2 = job >= nkt;
-        const int kpos = kb + (p2 ? job - nkt : job) * kBN;
-        mbar_arrive_expect_tx(&sm.full[stage], (p2 ? 2 : 1) * kChunks * Smem::kTileBytes);
-        for (int c = 0; c < kChunks; ++c) tma_load_3d(&kmap, &sm.full[stage], sm.k[stage][c], c * 64, g, kpos);
-        if (p2)
-          for (int c = 0; c < kChunks; ++c) tma_load_3d(&vmap, &sm.full[stage], sm.v[stage][c], c * 64, g, kpos);
-        issued = job + 1;
+      for (int L = 0; L < nloads; ++L) {
+        const int x = L % kSlots;
+        if (L >= kSlots && !mbar_wait(&sm.empty[x], ((L / kSlots) - 1) & 1, abort_flag)) break;
+        const bool is_v = L >= nkt && ((L - nkt) & 1);
+        const int kt = L < nkt ? L : (L - nkt) >> 1;
+        const int kpos = kb + kt * kBN;
+        mbar_arrive_expect_tx(&sm.full[x], Smem::kSlotBytes);
+        for (int c = 0; c < kChunks; ++c)
+          tma_load_3d(is_v ? &vmap : &kmap, &sm.full[x], sm.slot[x][c], c * 64, g, kpos);
+        issued = L + 1;
       }
     }
     __syncwarp();
@@ -206,47 +234,51 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       constexpr uint32_t idS = idesc_bf16_f32(128, kBN, false, false);
       constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);
       bool ok = mbar_wait(&sm.q_full, 0, abort_flag);
+      auto wait_load = [&](int L) -> bool { return mbar_wait(&sm.full[L % kSlots], (L / kSlots) & 1, abort_flag); };
       auto issue_s = [&](int job) -> bool {
-        const int stage = job % kStages;
+        const int L = job < nkt ? job : nkt + 2 * (job - nkt);
+        const int x = L % kSlots;
         const int b = job & 1;
-        if (!mbar_wait(&sm.full[stage], (job / kStages) & 1, abort_flag)) return false;
-        sm.jobs_consumed = job + 1;
+        if (!wait_load(L)) return false;
         if (job >= 2 && !mbar_wait(&sm.s_free[b], ((job >> 1) - 1) & 1, abort_flag)) return false;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const int c = k >> 2, kk = k & 3;
           const uint64_t a = sdesc_sw128(smem_u32(sm.q[c]) + kk * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(smem_u32(sm.k[stage][c]) + kk * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(smem_u32(sm.slot[x][c]) + kk * 32, 16, 1024);
           umma_bf16_ss(tmem + b * kBN, a, bd, idS, k > 0 ? 1u : 0u);
         }
         umma_commit(&sm.s_full[b]);
-        if (job < nkt) umma_commit(&sm.empty[stage]);
+        umma_commit(&sm.empty[x]);  // the K tile is no longer needed
         return true;
       };
       if (ok) ok = issue_s(0);
       for (int job = 0; ok && job < njobs; ++job) {
+        // the next score tile goes to the tensor core before this tile's P.V, so it
+        // computes while the softmax warps turn this tile's scores into P
         if (job + 1 < njobs && !issue_s(job + 1)) {
           ok = false;
           break;
         }
         if (job >= nkt) {
           const int kt2 = job - nkt;
-          const int stage = job % kStages;
-          if (!mbar_wait(&sm.p_full, kt2 & 1, abort_flag)) {
+          const int L = nkt + 2 * kt2 + 1;  // V tile
+          const int x = L % kSlots;
+          const int b = job & 1;
+          if (!wait_load(L) || !mbar_wait(&sm.p_full, kt2 & 1, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < kBN / 16; ++k) {
-            const int c = k >> 2, kk = k & 3;
-            const uint64_t a = sdesc_sw128(smem_u32(sm.p[c]) + kk * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(smem_u32(sm.v[stage][0]) + k * 2048, Smem::kTileBytes, 1024);
-            umma_bf16_ss(tmem + kColO, a, bd, idO, (kt2 > 0 || k > 0) ? 1u : 0u);
+            const uint32_t a_tmem = tmem + kColP + b * 64 + k * 8;  // keys 16k .. 16k+15
+            const uint64_t bd = sdesc_sw128(smem_u32(sm.slot[x][0]) + k * 2048, Smem::kTileBytes, 1024);
+            umma_bf16_ts(tmem + kColO, a_tmem, bd, idO, (kt2 > 0 || k > 0) ? 1u : 0u);
           }
-          umma_commit(&sm.p_free);
-          umma_commit(&sm.empty[stage]);
+          umma_commit(&sm.p_free);   // this P.V (and its reads of P from TMEM) is done
+          umma_commit(&sm.empty[x]);  // the V tile is no longer needed
         }
       }
       if (ok) umma_commit(&sm.o_full);
@@ -362,6 +394,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int job = nkt + kt2;
       const int b = job & 1;
       if (ok) ok = mbar_wait(&sm.s_full[b], (job >> 1) & 1, abort_flag);
+      // P(kt2) is stored to TMEM only once the P.V MMA of the previous tile has finished:
+      // tcgen05.st into TMEM while a P.V that reads its A operand from TMEM was still running
+      // corrupted rows 0-31 of the output on B200, although the two P buffers are disjoint.
       if (ok && kt2 > 0) ok = mbar_wait(&sm.p_free, (kt2 - 1) & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
@@ -410,18 +445,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           bin[u] = (u == 0 ? half_in : 0.5f * s[4 * u - 1]) + s[4 * u] + s[4 * u + 1] + s[4 * u + 2] + half_last;
         }
       }
-      // P row r, keys col0 .. col0+kColsPerWG-1 -> chunk col0/64, columns col0%64 ..
-      uint8_t* pc = sm.p[col0 >> 6];
+      // P row r, keys col0 .. col0+31 -> 16 packed bf16 pairs in P buffer b (TMEM columns
+      // kColP + 64b + col0/2 ..).
+      static_assert(kColsPerWG == 32, "P placement assumes 32 key columns per warpgroup");
+      {
+        uint32_t pk[16];
 #pragma unroll
-      for (int u = 0; u < kColsPerWG / 8; ++u) {
-        uint4 w;
-        w.x = pack_bf16x2(s[8 * u + 0], s[8 * u + 1]);
-        w.y = pack_bf16x2(s[8 * u + 2], s[8 * u + 3]);
-        w.z = pack_bf16x2(s[8 * u + 4], s[8 * u + 5]);
-        w.w = pack_bf16x2(s[8 * u + 6], s[8 * u + 7]);
-        *reinterpret_cast<uint4*>(pc + sw128_offset(r, (col0 & 63) + 8 * u)) = w;
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(s[2 * i], s[2 * i + 1]);
+        tmem_st16(trow + kColP + b * 64 + col0 / 2, pk);
       }
-      fence_proxy_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full);
       if (MODE == kModeCmp) {
@@ -536,9 +570,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         while (!mbar_test(&sm.q_full, 0) && clock64() - t_start < kWaitCycles) {
         }
       }
-      for (int job = sm.jobs_consumed; job < issued; ++job) {
+      // the last load issued into each slot (earlier ones completed before it was issued)
+      for (int L = issued - kSlots > 0 ? issued - kSlots : 0; L < issued; ++L) {
         const long long t_start = clock64();
-        while (!mbar_test(&sm.full[job % kStages], (job / kStages) & 1) && clock64() - t_start < kWaitCycles) {
+        while (!mbar_test(&sm.full[L % kSlots], (L / kSlots) & 1) && clock64() - t_start < kWaitCycles) {
         }
       }
     }
