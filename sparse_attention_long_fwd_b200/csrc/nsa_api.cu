@@ -16,6 +16,7 @@
 #include "attn_tc.cuh"
 #include "topn.cuh"
 #include "sel.cuh"
+#include "sel_inv.cuh"
 #include "decode.cuh"
 
 namespace {
@@ -73,6 +74,8 @@ int check_device() {
 
 struct PrefillLayout {
   size_t kc, vc, o_cmp, lse, scores, sel_idx, o_sel, total;
+  // block-major selected branch: bucket counters, offsets, bucketed entries, partials
+  size_t sel_cnt, sel_eoff, sel_toff, sel_list, part_o, part_ml;
   int ncmp, nsel;
 };
 
@@ -95,6 +98,14 @@ PrefillLayout prefill_layout(const nsa_params_t* p) {
   L.scores = take(static_cast<size_t>(nv) * hkv * (L.nsel > 0 ? L.nsel : 1) * 4);
   L.sel_idx = take(static_cast<size_t>(nv) * hkv * p->top_n * 4);
   L.o_sel = take(static_cast<size_t>(nv) * hq * d * 4);
+  const size_t buckets = static_cast<size_t>(hkv) * (L.nsel > 0 ? L.nsel : 1);
+  const size_t entries = static_cast<size_t>(nv) * hkv * p->top_n;
+  L.sel_cnt = take(2 * buckets * 4);
+  L.sel_eoff = take((buckets + 1) * 4);
+  L.sel_toff = take((buckets + 1) * 4);
+  L.sel_list = take(entries * 4);
+  L.part_o = take(static_cast<size_t>(nv) * hq * p->top_n * d * 2);
+  L.part_ml = take(static_cast<size_t>(nv) * hq * p->top_n * 16);
   L.total = off;
   return L;
 }
@@ -152,9 +163,9 @@ void stage_begin(cudaStream_t st) {
   if (g_stage_count > 0) cudaEventRecord(static_cast<cudaEvent_t>(g_stage_events[g_stage_next++]), st);
 }
 
-int launch_status(const char* name = "kernel", cudaStream_t st = nullptr) {
+int launch_status(const char* name = "kernel", cudaStream_t st = nullptr, bool stage_end = true) {
   cudaError_t e = cudaGetLastError();
-  if (e == cudaSuccess && g_stage_next < g_stage_count)
+  if (e == cudaSuccess && stage_end && g_stage_next < g_stage_count)
     e = cudaEventRecord(static_cast<cudaEvent_t>(g_stage_events[g_stage_next++]), st);
   if (e == cudaSuccess && debug_sync()) {
     std::fprintf(stderr, "[nsa] %s launched\n", name);
@@ -270,17 +281,58 @@ int prefill_impl(const nsa_params_t* p, const void* q, const void* k, const void
           out_sel_idx);
       if ((rc = launch_status("topn", st)) != NSA_OK) return rc;
     }
-    // 4. selected branch
+    // 4. selected branch, block-major: bucket (token, slot) pairs by (group, block),
+    //    one tensor-core tile per bucket tile, then merge each row's partials
     {
-      const size_t smem = sizeof(nsa::SelSmem<D>) + 128;
-      auto kern = nsa::sel_branch_kernel<D>;
+      const int m = hkv * L.nsel;
+      const int Gp = Gc;
+      const int TT = 128 / Gp;
+      const long long entries = static_cast<long long>(nv) * hkv * p->top_n;
+      nsa::SelInvArgs sa{};
+      sa.nv = nv;
+      sa.hq = hq;
+      sa.hkv = hkv;
+      sa.G = G;
+      sa.Gp = Gp;
+      sa.TT = TT;
+      sa.nsel = L.nsel;
+      sa.top_n = p->top_n;
+      sa.sel_len = p->sel_block;
+      sa.sl2 = sl2;
+      sa.sel_idx = reinterpret_cast<const int32_t*>(ws + L.sel_idx);
+      sa.cnt = reinterpret_cast<int*>(ws + L.sel_cnt);
+      sa.cursor = sa.cnt + m;
+      sa.ent_off = reinterpret_cast<int*>(ws + L.sel_eoff);
+      sa.tile_off = reinterpret_cast<int*>(ws + L.sel_toff);
+      sa.list = reinterpret_cast<int*>(ws + L.sel_list);
+      sa.part_o = reinterpret_cast<__half*>(ws + L.part_o);
+      sa.part_ml = reinterpret_cast<float4*>(ws + L.part_ml);
+      sa.o_sel = reinterpret_cast<float*>(ws + L.o_sel);
+      CUtensorMap qsmap, k64map, v64map;
+      if (!nsa::make_tmap_bf16_3d(&qsmap, q, D, hq, N, qs1, qs2, 64, Gp, 1) ||
+          !nsa::make_tmap_bf16_3d(&k64map, k, D, hkv, N, ks1, ks2, 64, 1, 64) ||
+          !nsa::make_tmap_bf16_3d(&v64map, v, D, hkv, N, ks1, ks2, 64, 1, 64))
+        return NSA_ERR_CUDA;
+      if (cudaMemsetAsync(sa.cnt, 0, 2 * static_cast<size_t>(m) * 4, st) != cudaSuccess) return NSA_ERR_CUDA;
+      long long eb = (entries + 255) / 256;
+      const unsigned ebl = static_cast<unsigned>(eb < 148 * 16 ? (eb > 0 ? eb : 1) : 148 * 16);
+      nsa::sel_count_kernel<<<ebl, 256, 0, st>>>(sa);
+      if ((rc = launch_status("sel_count", st, false)) != NSA_OK) return rc;
+      nsa::sel_scan_kernel<<<1, 1024, 0, st>>>(sa);
+      if ((rc = launch_status("sel_scan", st, false)) != NSA_OK) return rc;
+      nsa::sel_scatter_kernel<<<ebl, 256, 0, st>>>(sa);
+      if ((rc = launch_status("sel_scatter", st)) != NSA_OK) return rc;
+      // at most 2 CTAs per SM (256 TMEM columns each): request more than a third of the SM's shared memory
+      size_t smem = sizeof(nsa::SelInvSmem<D>) + 1024;
+      if (smem < 80 * 1024) smem = 80 * 1024;
+      auto kern = nsa::sel_partial_kernel<D>;
       if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
-      const int blocks = (nv * hkv + nsa::kSelWarps - 1) / nsa::kSelWarps;
-      kern<<<blocks, nsa::kSelWarps * 32, smem, st>>>(
-          static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-          static_cast<const __nv_bfloat16*>(v), reinterpret_cast<const int32_t*>(ws + L.sel_idx), nv, hq, hkv,
-          p->top_n, p->sel_block, sl2, reinterpret_cast<float*>(ws + L.o_sel));
-      if ((rc = launch_status("sel_branch", st)) != NSA_OK) return rc;
+      const long long max_tiles = (entries + TT - 1) / TT + m;
+      kern<<<static_cast<unsigned>(max_tiles), nsa::kSelInvThreads, smem, st>>>(qsmap, k64map, v64map, sa);
+      if ((rc = launch_status("sel_partial", st)) != NSA_OK) return rc;
+      const long long rows = static_cast<long long>(nv) * hq;
+      nsa::sel_merge_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(sa);
+      if ((rc = launch_status("sel_merge", st)) != NSA_OK) return rc;
     }
     // 5. sliding window + gated combine -> out rows [0, N_v)
     a.o_sel = reinterpret_cast<const float*>(ws + L.o_sel);
