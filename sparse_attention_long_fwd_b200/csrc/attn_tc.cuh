@@ -20,6 +20,9 @@
 //            as bf16 and accumulated O += P V in TMEM by a tcgen05 MMA that reads P
 //            from TMEM. Because P is final, the compressed mode
 //            can bin it into block scores in the same pass.
+// The window and dense modes need no block scores: their phase 1 finds only the row max,
+// phase 2 leaves P = exp2(S*scale*log2e - max) unnormalised, and the epilogue divides O
+// by the row sum of P (half the exponentials of the two exact passes).
 // K and V tiles stream through a ring of shared-memory slots (one tile each); the MMA
 // releases a slot as soon as the MMA that read it is done.
 // The pages' kernel notes (CSDN blog, section 5.1: fixed 64x64 blocks, prefetching the
@@ -349,7 +352,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float cmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       const float mnew = fmaxf(m, cmax);
-      if (mnew != -INFINITY) {
+      if (MODE != kModeCmp) {
+        m = mnew;  // the window and dense branches need only the row max here
+      } else if (mnew != -INFINITY) {
         const float ms = mnew * sl2;
         float acc[8];
 #pragma unroll
@@ -377,9 +382,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int w = 0; w < kSoftmaxWG; ++w) L += sm.lse_x[w][r][1] * ex2_approx(sm.lse_x[w][r][0] - M);
       }
-      has_keys = L > 0.f;
-      lse2 = has_keys ? M + __log2f(L) : INFINITY;
+      if (MODE == kModeCmp) {
+        has_keys = L > 0.f;
+        lse2 = has_keys ? M + __log2f(L) : INFINITY;
+      } else {
+        // P = exp2(S*scale*log2e - max) unnormalised; the row sum divides O at the end
+        has_keys = M != -INFINITY;
+        lse2 = has_keys ? M : INFINITY;
+      }
     }
+    float psum = 0.f;  // (window, dense) this thread's part of the row sum of P
     // ---- phase 2: normalised probabilities -> P (smem, bf16) and block scores
     // Block scores (kModeCmp): compressed block i covers tokens [16i, 16i+32) and selection
     // block j covers [64j, 64j+64), so block j takes all of compressed blocks 4j..4j+2 and
@@ -438,6 +450,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           s[i] = (kidx >= rb && kidx < re) ? ex2_approx(fmaf(s[i], sl2, -lse2)) : 0.f;
         }
       }
+      if (MODE != kModeCmp) {
+        float ps[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int i = 0; i < kColsPerWG; ++i) ps[i & 3] += s[i];
+        psum += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+      }
       if (MODE == kModeCmp) {
 #pragma unroll
         for (int u = 0; u < kBinsPerWG; ++u) {
@@ -491,6 +509,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (hh == 0 && t < args.q_end && j <= t / args.sel_len)
         args.scores[(static_cast<size_t>(t) * args.hkv + g) * args.nsel + j] = c;
     }
+    float inv_l = 1.f;  // (window, dense) 1 / row sum of P over all column slices
+    if (MODE != kModeCmp) {
+      sm.lse_x[wg][r][1] = psum;
+      named_bar_sync(3, kSoftmaxThreads);
+      float L = 0.f;
+#pragma unroll
+      for (int w = 0; w < kSoftmaxWG; ++w) L += sm.lse_x[w][r][1];
+      inv_l = L > 0.f ? 1.f / L : 0.f;
+    }
     // ---- epilogue (every lane loads its TMEM row; only valid rows are stored)
     if (ok && nkt > 0) {
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_full, 0, abort_flag));
@@ -534,11 +561,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
             for (int u = 0; u < kOC / 4; ++u) {
               const float4 a = oc[u], c = os[u];
-              o[4 * u + 0] = g0 * a.x + g1 * c.x + g2 * o[4 * u + 0];
-              o[4 * u + 1] = g0 * a.y + g1 * c.y + g2 * o[4 * u + 1];
-              o[4 * u + 2] = g0 * a.z + g1 * c.z + g2 * o[4 * u + 2];
-              o[4 * u + 3] = g0 * a.w + g1 * c.w + g2 * o[4 * u + 3];
+              o[4 * u + 0] = g0 * a.x + g1 * c.x + g2 * (o[4 * u + 0] * inv_l);
+              o[4 * u + 1] = g0 * a.y + g1 * c.y + g2 * (o[4 * u + 1] * inv_l);
+              o[4 * u + 2] = g0 * a.z + g1 * c.z + g2 * (o[4 * u + 2] * inv_l);
+              o[4 * u + 3] = g0 * a.w + g1 * c.w + g2 * (o[4 * u + 3] * inv_l);
             }
+          } else {
+#pragma unroll
+            for (int u = 0; u < kOC; ++u) o[u] *= inv_l;
           }
           if (args.out_f32) {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.out) + orow + c0);

@@ -75,7 +75,8 @@ int check_device() {
 struct PrefillLayout {
   size_t kc, vc, o_cmp, lse, scores, sel_idx, o_sel, total;
   // block-major selected branch: bucket counters, offsets, bucketed entries, partials
-  size_t sel_cnt, sel_eoff, sel_toff, sel_list, part_o, part_ml;
+  size_t sel_cnt, sel_eoff, sel_toff, sel_list, sel_row, part_o, part_ml;
+  long long part_rows;  // 128 x the bound on selected-branch tiles
   int ncmp, nsel;
 };
 
@@ -104,8 +105,15 @@ PrefillLayout prefill_layout(const nsa_params_t* p) {
   L.sel_eoff = take((buckets + 1) * 4);
   L.sel_toff = take((buckets + 1) * 4);
   L.sel_list = take(entries * 4);
-  L.part_o = take(static_cast<size_t>(nv) * hq * p->top_n * d * 2);
-  L.part_ml = take(static_cast<size_t>(nv) * hq * p->top_n * 16);
+  L.sel_row = take(entries * 4);
+  {
+    int gc = 1;  // heads per token in a tile row block: G rounded up to a power of two
+    while (gc < hq / (hkv > 0 ? hkv : 1)) gc <<= 1;
+    const size_t tiles = (entries + (128 / gc) - 1) / (128 / gc) + buckets;
+    L.part_rows = static_cast<long long>(tiles) * 128;
+  }
+  L.part_o = take(static_cast<size_t>(L.part_rows) * d * 2);
+  L.part_ml = take(static_cast<size_t>(L.part_rows) * 16);
   L.total = off;
   return L;
 }
@@ -177,6 +185,19 @@ int launch_status(const char* name = "kernel", cudaStream_t st = nullptr, bool s
     std::fflush(stderr);
   }
   return e == cudaSuccess ? NSA_OK : NSA_ERR_CUDA;
+}
+
+// Streaming multiprocessors of the current device (cached per device); 0 on error.
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cached[dev] = n;
+  }
+  return cached[dev];
 }
 
 template <typename K>
@@ -305,11 +326,15 @@ int prefill_impl(const nsa_params_t* p, const void* q, const void* k, const void
       sa.ent_off = reinterpret_cast<int*>(ws + L.sel_eoff);
       sa.tile_off = reinterpret_cast<int*>(ws + L.sel_toff);
       sa.list = reinterpret_cast<int*>(ws + L.sel_list);
-      sa.part_o = reinterpret_cast<__half*>(ws + L.part_o);
+      sa.row_of = reinterpret_cast<int*>(ws + L.sel_row);
+      sa.part_rows = L.part_rows;
+      sa.part_o = reinterpret_cast<const __half*>(ws + L.part_o);
       sa.part_ml = reinterpret_cast<float4*>(ws + L.part_ml);
       sa.o_sel = reinterpret_cast<float*>(ws + L.o_sel);
-      CUtensorMap qsmap, k64map, v64map;
-      if (!nsa::make_tmap_bf16_3d(&qsmap, q, D, hq, N, qs1, qs2, 64, Gp, 1) ||
+      sa.q = static_cast<const __nv_bfloat16*>(q);
+      CUtensorMap k64map, v64map, omap;
+      if (!nsa::make_tmap_f16_3d(&omap, ws + L.part_o, 64, static_cast<uint64_t>(L.part_rows), D / 64, 128,
+                                 static_cast<uint64_t>(L.part_rows) * 128, 64, 32, 1) ||
           !nsa::make_tmap_bf16_3d(&k64map, k, D, hkv, N, ks1, ks2, 64, 1, 64) ||
           !nsa::make_tmap_bf16_3d(&v64map, v, D, hkv, N, ks1, ks2, 64, 1, 64))
         return NSA_ERR_CUDA;
@@ -322,14 +347,18 @@ int prefill_impl(const nsa_params_t* p, const void* q, const void* k, const void
       if ((rc = launch_status("sel_scan", st, false)) != NSA_OK) return rc;
       nsa::sel_scatter_kernel<<<ebl, 256, 0, st>>>(sa);
       if ((rc = launch_status("sel_scatter", st)) != NSA_OK) return rc;
-      // at most 2 CTAs per SM (256 TMEM columns each): request more than a third of the SM's shared memory
-      size_t smem = sizeof(nsa::SelInvSmem<D>) + 1024;
-      if (smem < 80 * 1024) smem = 80 * 1024;
-      auto kern = nsa::sel_partial_kernel<D>;
+      // persistent: one CTA per SM (512 TMEM columns each; the shared-memory request keeps
+      // a second CTA off the SM)
+      size_t smem = sizeof(nsa::SelTileSmem<D>) + 1024;
+      if (smem < 116 * 1024) smem = 116 * 1024;
+      auto kern = nsa::sel_tile_kernel<D>;
       if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
-      const long long max_tiles = (entries + TT - 1) / TT + m;
-      kern<<<static_cast<unsigned>(max_tiles), nsa::kSelInvThreads, smem, st>>>(qsmap, k64map, v64map, sa);
-      if ((rc = launch_status("sel_partial", st)) != NSA_OK) return rc;
+      const long long max_tiles = L.part_rows / 128;
+      const int nsm = sm_count();
+      if (nsm <= 0) return NSA_ERR_CUDA;
+      const unsigned grid = static_cast<unsigned>(max_tiles < nsm ? max_tiles : nsm);
+      kern<<<grid, nsa::kSelTileThreads, smem, st>>>(k64map, v64map, omap, sa);
+      if ((rc = launch_status("sel_tile", st)) != NSA_OK) return rc;
       const long long rows = static_cast<long long>(nv) * hq;
       nsa::sel_merge_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(sa);
       if ((rc = launch_status("sel_merge", st)) != NSA_OK) return rc;

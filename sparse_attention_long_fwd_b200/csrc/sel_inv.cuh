@@ -9,14 +9,17 @@
 // padded to Gp, a power of two). Each row's softmax over that block gives a partial
 // (max, sum, output / sum); sel_merge_kernel combines a row's partials as an online softmax
 // would. The sum is taken over the bf16-rounded P that the tensor core multiplies, so each
-// partial is an exact convex combination of values. The partial output is stored in fp16
-// (2^-12 relative rounding); a row whose largest magnitude would overflow fp16 is stored
-// divided by a power of two c, kept with the row's (max, sum).
+// partial is an exact convex combination of values. Partials live in tile order: tile k
+// owns rows 128k .. 128k+127 (MMA row r = token slot r / Gp, head slot r % Gp), so a warp
+// writes its 32 rows with one TMA store per 64 output columns; sel_scatter_kernel records
+// where each (token, group, slot) landed. The partial output is stored in fp16 (2^-12
+// relative rounding); a 64-column half whose largest magnitude would overflow fp16 is
+// stored divided by a power of two c, kept with the row's (max, sum).
 //
 //   sel_count_kernel    entries per (group, block)
 //   sel_scan_kernel     exclusive scans of entries and of tiles per (group, block)
 //   sel_scatter_kernel  bucket (token, slot) pairs
-//   sel_partial_kernel  one 128-row tcgen05 tile per CTA: S = Q K^T, softmax, O = P V
+//   sel_tile_kernel     persistent 128-row tcgen05 tiles: S = Q K^T, softmax, O = P V
 //   sel_merge_kernel    o_sel[t][h] from the row's partials
 #pragma once
 #include <cuda_fp16.h>
@@ -34,8 +37,11 @@ struct SelInvArgs {
   int* ent_off;                 // [hkv*nsel + 1] exclusive scan of cnt
   int* tile_off;                // [hkv*nsel + 1] exclusive scan of ceil(cnt/TT)
   int* list;                    // [nv*hkv*top_n] bucketed entries: t * 64 + slot
-  __half* part_o;               // [nv][hq][top_n][D] output / (sum * c) of each partial
-  float4* part_ml;              // [nv][hq][top_n] (max in log2 units, sum, c, 0)
+  int* row_of;                  // [nv][hkv][top_n] first partial row of each (token, group, slot)
+  const __nv_bfloat16* q;       // [nv][hq][D]
+  long long part_rows;          // rows per 64-column half of part_o (128 x the tile bound)
+  const __half* part_o;         // [D/64][part_rows][64] output / (sum * c_half) of each partial
+  float4* part_ml;              // [part_rows] (max in log2 units, sum, c of half 0, c of half 1)
   float* o_sel;                 // [nv][hq][D]
 };
 
@@ -124,148 +130,344 @@ __global__ void __launch_bounds__(256) sel_scatter_kernel(const SelInvArgs a) {
     const int g = static_cast<int>(tg % a.hkv);
     const int t = static_cast<int>(tg / a.hkv);
     const int key = g * a.nsel + j;
-    const int pos = a.ent_off[key] + atomicAdd(&a.cursor[key], 1);
-    a.list[pos] = t * 64 + slot;
+    const int local = atomicAdd(&a.cursor[key], 1);
+    a.list[a.ent_off[key] + local] = t * 64 + slot;
+    a.row_of[e] = (a.tile_off[key] + local / a.TT) * 128 + (local % a.TT) * a.Gp;
   }
 }
 
-// 32 fp32 values times `scale` to fp16 (round to nearest even), 64 contiguous bytes
-__device__ __forceinline__ void store_half32(__half* dst, const float (&o)[32], float scale) {
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    uint32_t w[4];
-#pragma unroll
-    for (int x = 0; x < 4; ++x) {
-      __half2 h = __floats2half2_rn(o[8 * u + 2 * x] * scale, o[8 * u + 2 * x + 1] * scale);
-      w[x] = *reinterpret_cast<uint32_t*>(&h);
-    }
-    d4[u] = make_uint4(w[0], w[1], w[2], w[3]);
-  }
-}
+// ---------------------------------------------------------------- partial attention tiles
+// Persistent: one CTA per SM takes a contiguous range of bucket tiles, so consecutive
+// tiles of the same (group, block) reuse the K and V already in shared memory.
+//   warps 0..2   producers: warp 0 writes the tile records (list entries prefetched two
+//                tiles ahead) and loads K and V by TMA once per bucket; all three gather
+//                the tile's Q rows (32-row blocks) with 16-byte cp.async straight into the
+//                128-byte-swizzled layout (one small TMA box per token was issue-bound)
+//   warp 3       MMA issuer: S = Q K^T into the TMEM of the tile's warpgroup, then O = P V,
+//                issuing whichever of the next S or the next P.V has its inputs ready
+//   warps 4..15  three softmax / epilogue warpgroups taking tiles in turn; thread = MMA row
+// A warpgroup's 128 TMEM columns hold S (64 columns) and, once S has been read, O over it.
+// P goes from registers to shared memory (128-byte swizzled, K-major) and the P.V product
+// reads it there, so no thread writes TMEM while an MMA runs.
+constexpr int kSelWG = 3;
+constexpr int kSelProducers = 3;
+constexpr int kSelMmaWarp = kSelProducers;
+constexpr int kSelFirstSmxWarp = kSelProducers + 1;
+constexpr int kSelTileThreads = 32 * kSelFirstSmxWarp + kSelWG * 128;  // 16 warps: 128 registers each
+constexpr int kSelQStages = 3;
+constexpr int kSelKVStages = 2;
+constexpr int kSelInfo = 8;
 
-constexpr int kSelInvThreads = 192;  // TMA warp, MMA warp, 4 softmax / epilogue warps
-
-template <int D>
-struct SelInvSmem {
-  static constexpr int kChunks = D / 64;
-  alignas(1024) uint8_t q[kChunks][128 * 128];  // 128 rows x 128 B per chunk
-  alignas(1024) uint8_t k[kChunks][64 * 128];   // the block's 64 keys
-  alignas(1024) uint8_t v[kChunks][64 * 128];   // and values
-  uint64_t full, s_full, p_full, o_full, drain;
-  uint32_t tmem_base;
-  int abort_flag;
-  int g, j, e0, cnt;
-  int ent[128];  // t * 64 + slot of this tile's tokens
+struct SelTileInfo {
+  int key, cnt, kvs, flags;  // flags: 1 = first tile of its K/V stage, 2 = last
+  int ent[128];
 };
 
-// grid: an upper bound on the tile count; CTAs past tile_off[hkv*nsel] return at once.
 template <int D>
-__global__ void __launch_bounds__(kSelInvThreads, 1)
-    sel_partial_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
-                       const __grid_constant__ CUtensorMap vmap, const SelInvArgs a) {
-  using Smem = SelInvSmem<D>;
+struct SelTileSmem {
+  static constexpr int kChunks = D / 64;
+  alignas(1024) uint8_t q[kSelQStages][kChunks][128 * 128];
+  alignas(1024) uint8_t k[kSelKVStages][kChunks][64 * 128];
+  alignas(1024) uint8_t v[kSelKVStages][kChunks][64 * 128];
+  alignas(1024) uint8_t p[kSelWG][128 * 128];  // 128 rows x 64 keys bf16
+  SelTileInfo info[kSelInfo];
+  uint64_t q_full[kSelQStages], q_empty[kSelQStages];
+  uint64_t kv_full[kSelKVStages], kv_empty[kSelKVStages];
+  uint64_t info_full[kSelInfo], info_empty[kSelInfo];
+  uint64_t s_full[kSelWG], p_full[kSelWG], o_full[kSelWG], o_free[kSelWG];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// Bounded wait by every lane of a warp, with a warp-uniform result.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+}
+
+__device__ __forceinline__ void cp_async16_cg(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+// The barrier receives one arrival once all of this thread's earlier cp.async copies land.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Tile record of the producer: bucket, first list entry, entry count, last-of-bucket, and
+// (prefetched) list entries x = lane + 32k.
+struct SelTileMeta {
+  int key, e0, cnt, last;
+  int e[4];
+};
+
+template <int D>
+__global__ void __launch_bounds__(kSelTileThreads, 1)
+    sel_tile_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                    const __grid_constant__ CUtensorMap omap, const SelInvArgs a) {
+  using Smem = SelTileSmem<D>;
   constexpr int kChunks = Smem::kChunks;
-  constexpr uint32_t kTmemCols = 256;  // S at 0 (64), O at 64 (D <= 128), P at 192 (32)
-  constexpr uint32_t kColO = 64, kColP = 192;
+  constexpr int kCpr = D / 8;          // 16-byte pieces per Q row
+  constexpr uint32_t kTmemCols = 512;  // warpgroup w: columns 128w .. 128w+127 (S, then O)
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int m = a.hkv * a.nsel;
-  const int tile = blockIdx.x;
-  if (tile >= a.tile_off[m]) return;  // uniform across the CTA
+  const long long total = a.tile_off[m];
+  const int tile_begin = static_cast<int>(total * blockIdx.x / gridDim.x);
+  const int tile_end = static_cast<int>(total * (blockIdx.x + 1) / gridDim.x);
+  const int n = tile_end - tile_begin;
+  if (n <= 0) return;  // uniform across the CTA
   if (tid == 0) {
-    // (group, block) of this tile: last key with tile_off[key] <= tile
-    int lo = 0, hi = m - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (a.tile_off[mid] <= tile) lo = mid; else hi = mid - 1;
+    for (int s = 0; s < kSelQStages; ++s) {
+      mbar_init(&sm.q_full[s], kSelProducers * 32);  // one cp.async arrival per producer lane
+      mbar_init(&sm.q_empty[s], 1);
     }
-    const int first = a.ent_off[lo] + (tile - a.tile_off[lo]) * a.TT;
-    sm.g = lo / a.nsel;
-    sm.j = lo % a.nsel;
-    sm.e0 = first;
-    sm.cnt = min(a.TT, a.ent_off[lo + 1] - first);
-    mbar_init(&sm.full, 1);
-    mbar_init(&sm.s_full, 1);
-    mbar_init(&sm.p_full, 4);
-    mbar_init(&sm.o_full, 1);
+    for (int s = 0; s < kSelKVStages; ++s) {
+      mbar_init(&sm.kv_full[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
+    }
+    for (int s = 0; s < kSelInfo; ++s) {
+      mbar_init(&sm.info_full[s], 1);
+      mbar_init(&sm.info_empty[s], 4);
+    }
+    for (int w = 0; w < kSelWG; ++w) {
+      mbar_init(&sm.s_full[w], 1);
+      mbar_init(&sm.p_full[w], 4);
+      mbar_init(&sm.o_full[w], 1);
+      mbar_init(&sm.o_free[w], 4);
+    }
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == kSelMmaWarp) {
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  __syncthreads();
-  const int g = sm.g, j = sm.j, cnt = sm.cnt;
-  for (int i = tid; i < cnt; i += kSelInvThreads) sm.ent[i] = a.list[sm.e0 + i];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort_flag = &sm.abort_flag;
   const int Gp = a.Gp, G = a.G;
+  const int lg_gp = __ffs(Gp) - 1;  // Gp is a power of two
+  int kv_issued = 0;  // warp 0: K-V loads issued
 
-  if (warp == 0) {
-    if (lane == 0) {
-      mbar_arrive_expect_tx(&sm.full, kChunks * (cnt * Gp * 128 + 2 * 64 * 128));
-      for (int c = 0; c < kChunks; ++c) {
-        for (int i = 0; i < cnt; ++i)
-          tma_load_3d(&qmap, &sm.full, &sm.q[c][i * Gp * 128], c * 64, g * G, sm.ent[i] >> 6);
-        tma_load_3d(&kmap, &sm.full, sm.k[c], c * 64, g, j * a.sel_len);
-        tma_load_3d(&vmap, &sm.full, sm.v[c], c * 64, g, j * a.sel_len);
+  if (warp < kSelProducers) {
+    // ------------------------------------------------------------------ producers
+    int key = 0, t_base = 0, t_next = 0, e_base = 0, e_next = 0;
+    SelTileMeta m0{}, m1{}, m2{};
+    auto fetch = [&](int tile) {
+      SelTileMeta r;
+      while (t_next <= tile) {  // next bucket with tiles
+        ++key;
+        t_base = t_next;
+        e_base = e_next;
+        t_next = a.tile_off[key + 1];
+        e_next = a.ent_off[key + 1];
       }
+      r.key = key;
+      r.e0 = e_base + (tile - t_base) * a.TT;
+      r.cnt = min(a.TT, e_next - r.e0);
+      r.last = (tile == tile_end - 1) || (t_next == tile + 1);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) r.e[k] = (lane + 32 * k < r.cnt) ? a.list[r.e0 + lane + 32 * k] : 0;
+      return r;
+    };
+    if (warp == 0) {
+      if (lane == 0) {
+        tma_prefetch_desc(&kmap);
+        tma_prefetch_desc(&vmap);
+        int lo = 0, hi = m - 1;  // bucket of the first tile: the last key with tile_off[key] <= tile_begin
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (a.tile_off[mid] <= tile_begin) lo = mid; else hi = mid - 1;
+        }
+        key = lo;
+      }
+      key = __shfl_sync(0xffffffffu, key, 0);
+      t_base = a.tile_off[key];
+      t_next = a.tile_off[key + 1];
+      e_base = a.ent_off[key];
+      e_next = a.ent_off[key + 1];
+      m0 = fetch(tile_begin);
+      if (n > 1) m1 = fetch(tile_begin + 1);
+      if (n > 2) m2 = fetch(tile_begin + 2);
     }
-    __syncwarp();
-  } else if (warp == 1) {
+    int kv_key = -1;
+    // one tile; `cur` is warp 0's record of tile i, refilled with tile i + 3 at the end (in
+    // place: moving records whose list loads are in flight would wait for those loads)
+    auto tile_step = [&](int i, SelTileMeta& cur) -> bool {
+      const int si = i % kSelInfo, sq = i % kSelQStages;
+      SelTileInfo& inf = sm.info[si];
+      if (warp == 0) {
+        if (i >= kSelInfo && !warp_wait(&sm.info_empty[si], ((i / kSelInfo) - 1) & 1, abort_flag)) return false;
+        const bool first = cur.key != kv_key;
+        const int kvs = first ? kv_issued % kSelKVStages : (kv_issued - 1) % kSelKVStages;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (lane + 32 * k < cur.cnt) inf.ent[lane + 32 * k] = cur.e[k];
+        if (lane == 0) {
+          inf.key = cur.key;
+          inf.cnt = cur.cnt;
+          inf.kvs = kvs;
+          inf.flags = (first ? 1 : 0) | (cur.last ? 2 : 0);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.info_full[si]);
+      } else if (!warp_wait(&sm.info_full[si], (i / kSelInfo) & 1, abort_flag)) {
+        return false;
+      }
+      // Q rows of this tile: row R = token slot R / Gp, head slot R % Gp; this warp takes the
+      // 32-row blocks b with b % kSelProducers == (warp + 1) % kSelProducers (warp 0, which
+      // also writes the records, takes the fewest)
+      if (i >= kSelQStages && !warp_wait(&sm.q_empty[sq], ((i / kSelQStages) - 1) & 1, abort_flag)) return false;
+      {
+        const int cnt = inf.cnt;
+        const int g = inf.key / a.nsel;
+        for (int b = (warp + 1) % kSelProducers; b < 4; b += kSelProducers) {
+          const int rbase = b * 32;
+          // lane L finds the source row of tile row rbase + L (-1: not loaded); the copy loop
+          // then takes row it * kRpi + lane / kCpr in iteration it, piece lane % kCpr of it
+          int my_row = -1;
+          {
+            const int R = rbase + lane;
+            const int hh = R & (Gp - 1), tok = R >> lg_gp;
+            if (tok < cnt && hh < G && g * G + hh < a.hq) my_row = (inf.ent[tok] >> 6) * a.hq + g * G + hh;
+          }
+          constexpr int kRpi = 32 / kCpr;  // rows per iteration
+          const int sub = lane / kCpr, c16 = lane % kCpr;
+          const char* src_lane = reinterpret_cast<const char*>(a.q) + c16 * 16;
+          // 128-byte swizzle: piece (c16 & 7) of row R sits at unit (c16 & 7) ^ (R & 7); R & 7 =
+          // ((it * kRpi) & 7) ^ sub because rbase is a multiple of 32 and sub < kRpi
+          const uint32_t dst_lane = smem_u32(sm.q[sq][0]) + (c16 >> 3) * (128 * 128) + (rbase + sub) * 128;
+          const uint32_t x_lane = (c16 & 7) ^ sub;
+#pragma unroll
+          for (int it = 0; it < kCpr; ++it) {
+            const int row = __shfl_sync(0xffffffffu, my_row, it * kRpi + sub);
+            const uint32_t dst = dst_lane + it * kRpi * 128 + ((x_lane ^ ((it * kRpi) & 7)) << 4);
+            if (row >= 0) cp_async16_cg(dst, src_lane + static_cast<size_t>(row) * (D * 2));
+          }
+        }
+        cp_async_arrive_noinc(&sm.q_full[sq]);
+      }
+      if (warp == 0) {
+        if (cur.key != kv_key) {
+          const int u = kv_issued;  // K-V load number
+          const int kvs = u % kSelKVStages;
+          if (u >= kSelKVStages && !warp_wait(&sm.kv_empty[kvs], ((u / kSelKVStages) - 1) & 1, abort_flag)) return false;
+          if (lane == 0) {
+            const int g = cur.key / a.nsel, j = cur.key % a.nsel;
+            mbar_arrive_expect_tx(&sm.kv_full[kvs], kChunks * 2 * 64 * 128);
+            for (int c = 0; c < kChunks; ++c) {
+              tma_load_3d(&kmap, &sm.kv_full[kvs], sm.k[kvs][c], c * 64, g, j * a.sel_len);
+              tma_load_3d(&vmap, &sm.kv_full[kvs], sm.v[kvs][c], c * 64, g, j * a.sel_len);
+            }
+          }
+          __syncwarp();
+          kv_issued = u + 1;
+          kv_key = cur.key;
+        }
+        if (i + 3 < n) cur = fetch(tile_begin + i + 3);
+      }
+      return true;
+    };
+    for (int i = 0; i < n; i += 3) {
+      if (!tile_step(i, m0)) break;
+      if (i + 1 < n && !tile_step(i + 1, m1)) break;
+      if (i + 2 < n && !tile_step(i + 2, m2)) break;
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  } else if (warp == kSelMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 64, false, false);
       constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);
-      bool ok = mbar_wait(&sm.full, 0, abort_flag);
-      if (ok) {
-        tc_fence_after();
+      int ns = 0, np = 0, kv_seen = 0;  // next S tile, next P.V tile, K-V loads consumed
+      long long last = clock64();
+      while (np < n) {
+        if (*abort_flag) break;
+        bool did = false;
+        if (np < ns && mbar_ready(&sm.p_full[np % kSelWG], (np / kSelWG) & 1)) {
+          // O = P V over the warpgroup's columns (S there has been read)
+          const int w = np % kSelWG;
+          const SelTileInfo& inf = sm.info[np % kSelInfo];
+          const int kvs = inf.kvs, flags = inf.flags;
+          tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const int c = k >> 2, kk = k & 3;
-          umma_bf16_ss(tmem, sdesc_sw128(smem_u32(sm.q[c]) + kk * 32, 16, 1024),
-                       sdesc_sw128(smem_u32(sm.k[c]) + kk * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
+          for (int k = 0; k < 4; ++k)  // 64 keys, 16 per MMA
+            umma_bf16_ss(tmem + w * 128, sdesc_sw128(smem_u32(sm.p[w]) + k * 32, 16, 1024),
+                         sdesc_sw128(smem_u32(sm.v[kvs][0]) + k * 2048, 64 * 128, 1024), idO, k > 0 ? 1u : 0u);
+          umma_commit(&sm.o_full[w]);
+          if (flags & 2) umma_commit(&sm.kv_empty[kvs]);
+          ++np;
+          did = true;
+        } else if (ns < n) {
+          const int w = ns % kSelWG, jj = ns / kSelWG;
+          const int si = ns % kSelInfo, sq = ns % kSelQStages;
+          bool ready = mbar_ready(&sm.info_full[si], (ns / kSelInfo) & 1);
+          int kvs = 0, flags = 0;
+          if (ready) {
+            kvs = sm.info[si].kvs;
+            flags = sm.info[si].flags;
+            if (flags & 1) ready = mbar_ready(&sm.kv_full[kvs], (kv_seen / kSelKVStages) & 1);
+          }
+          if (ready) ready = mbar_ready(&sm.q_full[sq], (ns / kSelQStages) & 1);
+          if (ready && jj >= 1) ready = mbar_ready(&sm.o_free[w], (jj - 1) & 1);  // O of the last tile read
+          if (ready) {
+            if (flags & 1) ++kv_seen;
+            fence_proxy_async_smem();  // Q was written by cp.async (generic proxy); the MMA reads it
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+              const int c = k >> 2, kk = k & 3;
+              umma_bf16_ss(tmem + w * 128, sdesc_sw128(smem_u32(sm.q[sq][c]) + kk * 32, 16, 1024),
+                           sdesc_sw128(smem_u32(sm.k[kvs][c]) + kk * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
+            }
+            umma_commit(&sm.s_full[w]);
+            umma_commit(&sm.q_empty[sq]);
+            ++ns;
+            did = true;
+          }
         }
-        umma_commit(&sm.s_full);
-        ok = mbar_wait(&sm.p_full, 0, abort_flag);
-      }
-      if (ok) {
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < 4; ++k)  // 64 keys, 16 per MMA
-          umma_bf16_ts(tmem + kColO, tmem + kColP + k * 8,
-                       sdesc_sw128(smem_u32(sm.v[0]) + k * 2048, 64 * 128, 1024), idO, k > 0 ? 1u : 0u);
-        umma_commit(&sm.o_full);
+        if (did) {
+          last = clock64();
+        } else if (clock64() - last > kWaitCycles) {
+          *abort_flag = 1;
+          record_error(kErrWaitTimeout);
+          break;
+        }
       }
     }
     __syncwarp();
-  } else {
-    // one thread per MMA row: token slot i = r / Gp, head slot hh = r % Gp
-    const int q4 = warp & 3;
-    const int r = q4 * 32 + lane;
-    const int i = r / Gp, hh = r % Gp;
-    const bool valid = i < cnt && hh < G;
-    const int ent = i < cnt ? sm.ent[i] : 0;
-    const int t = ent >> 6, slot = ent & 63;
-    const int key_hi = valid ? min(64, t + 1 - j * a.sel_len) : 0;  // keys j*64 + c, c < key_hi
-    const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-    bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full, 0, abort_flag));
-    float mrow = -INFINITY, lrow = 0.f;
-    if (ok) {
+  } else if (warp >= kSelFirstSmxWarp) {
+    // ------------------------------------------------------------------ softmax / epilogue
+    const int w = (warp - kSelFirstSmxWarp) >> 2;  // warpgroup
+    const int q4 = warp & 3;         // TMEM lane quadrant
+    const int r = q4 * 32 + lane;    // MMA row: token slot r / Gp, head slot r % Gp
+    const int hh = r % Gp;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16) + w * 128;
+    uint8_t* prow_smem = sm.p[w] + r * 128;
+    for (int i = w; i < n; i += kSelWG) {
+      const int jj = i / kSelWG;
+      const int si = i % kSelInfo;
+      if (!warp_wait(&sm.info_full[si], (i / kSelInfo) & 1, abort_flag)) break;
+      const SelTileInfo& inf = sm.info[si];
+      const int cnt = inf.cnt, key = inf.key;
+      const int j = key % a.nsel;
+      const int tok = r / Gp;
+      const bool valid = tok < cnt && hh < G;
+      const int ent = tok < cnt ? inf.ent[tok] : 0;
+      const int t = ent >> 6;
+      const int key_hi = valid ? min(64, t + 1 - j * a.sel_len) : 0;  // keys j*64 + c, c < key_hi
+      if (!warp_wait(&sm.s_full[w], jj & 1, abort_flag)) break;
       tc_fence_after();
       float s[64];
-      __syncwarp();
       tmem_ld32(trow, *reinterpret_cast<float(*)[32]>(&s[0]));
       tmem_ld32(trow + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
       tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 64; ++c) s[c] = c < key_hi ? s[c] * a.sl2 : -INFINITY;
+      for (int c = 0; c < 64; ++c) s[c] = c < key_hi ? s[c] : -INFINITY;
       float mx[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) mx[c] = s[c];
@@ -273,68 +475,116 @@ __global__ void __launch_bounds__(kSelInvThreads, 1)
       for (int c = 8; c < 64; c += 8)
 #pragma unroll
         for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], s[c + u]);
-      mrow = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      const float mraw =
+          fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      const float mrow = mraw * a.sl2;  // row max in log2 units (the scale is positive)
+      const float bias = mraw == -INFINITY ? 0.f : -mrow;
+      // this warp's rows of P were the staging buffer of its previous tile's partial store
+      if (lane == 0) bulk_wait_read_all();
+      __syncwarp();
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        const float p0 = mrow == -INFINITY ? 0.f : ex2_approx(s[c] - mrow);
-        const float p1 = mrow == -INFINITY ? 0.f : ex2_approx(s[c + 1] - mrow);
-        const uint32_t w = pack_bf16x2(p0, p1);
-        pk[c >> 1] = w;
-        acc[(c >> 1) & 7] += __uint_as_float(w << 16) + __uint_as_float(w & 0xffff0000u);
+      for (int ch = 0; ch < 8; ++ch) {  // 8 keys = one 16-byte chunk of the swizzled P row
+        uint32_t wv[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const int c = ch * 8 + 2 * x;
+          const uint32_t pw =
+              pack_bf16x2(ex2_approx(fmaf(s[c], a.sl2, bias)), ex2_approx(fmaf(s[c + 1], a.sl2, bias)));
+          wv[x] = pw;
+          acc[x + (ch & 1) * 4] += __uint_as_float(pw << 16) + __uint_as_float(pw & 0xffff0000u);
+        }
+        const uint32_t dst = smem_u32(prow_smem + ((ch ^ (r & 7)) << 4));
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(wv[0]), "r"(wv[1]), "r"(wv[2]),
+                     "r"(wv[3])
+                     : "memory");
       }
-      lrow = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-      tmem_st16(trow + kColP, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
-      tmem_st16(trow + kColP + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
-      tmem_wait_st();
+      const float lrow = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+      fence_proxy_async_smem();  // P is read by the tensor core (async proxy)
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.p_full);
-      ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_full, 0, abort_flag));
-    }
-    if (ok) {
+      if (lane == 0) mbar_arrive(&sm.p_full[w]);
+      if (!warp_wait(&sm.o_full[w], jj & 1, abort_flag)) break;
       tc_fence_after();
       const float inv = lrow > 0.f ? 1.f / lrow : 0.f;
-      const size_t prow = (static_cast<size_t>(t) * a.hq + g * G + hh) * a.top_n + slot;
-      // fp16 stores; 65504 is the largest finite fp16 value
-      float amax = 0.f;
+      // partial rows: fp16, staged in this warp's 32 rows of P (the P.V product is done with
+      // them) in the 128-byte-swizzled layout, then one TMA store per 64-column half
+      const int prow = (tile_begin + i) * 128 + r;
+      uint8_t* stg = sm.p[w] + q4 * 32 * 128;
+      float c_lo = 1.f, c_hi = 1.f;
 #pragma unroll 1
-      for (int cb = 0; cb < D / 32; ++cb) {
-        float o[32];
-        __syncwarp();
-        tmem_ld32(trow + kColO + cb * 32, o);
+      for (int h = 0; h < kChunks; ++h) {
+        float o[64];
+        tmem_ld32(trow + h * 64, *reinterpret_cast<float(*)[32]>(&o[0]));
+        tmem_ld32(trow + h * 64 + 32, *reinterpret_cast<float(*)[32]>(&o[32]));
         tmem_wait_ld();
+        float am[8];
 #pragma unroll
-        for (int u = 0; u < 32; ++u) amax = fmaxf(amax, fabsf(o[u] * inv));
-        if (valid) store_half32(a.part_o + prow * D + cb * 32, o, inv);
-      }
-      float c = 1.f;
-      if (__any_sync(0xffffffffu, valid && !(amax < 65504.f))) {
-        // rare: rescale the row by a power of two (exact) and store it again
-        if (amax > 65504.f && amax <= 3.0e38f) c = exp2f(ceilf(log2f(amax / 32768.f)));
-        const float inv_c = inv / c;
-#pragma unroll 1
-        for (int cb = 0; cb < D / 32; ++cb) {
-          float o[32];
+        for (int u = 0; u < 8; ++u) am[u] = fabsf(o[u]);
+#pragma unroll
+        for (int u = 8; u < 64; u += 8)
+#pragma unroll
+          for (int x = 0; x < 8; ++x) am[x] = fmaxf(am[x], fabsf(o[u + x]));
+        const float amax =
+            fmaxf(fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3])), fmaxf(fmaxf(am[4], am[5]), fmaxf(am[6], am[7]))) *
+            inv;
+        // 65504 is the largest finite fp16 value; rare rows are scaled down by a power of two
+        float c = 1.f, sc = inv;
+        if (amax > 65504.f) {
+          if (amax <= 3.0e38f) c = exp2f(ceilf(log2f(amax / 32768.f)));
+          sc = inv / c;
+        }
+        if (h == 0) c_lo = c; else c_hi = c;
+        if (h > 0) {
+          if (lane == 0) bulk_wait_read_all();
           __syncwarp();
-          tmem_ld32(trow + kColO + cb * 32, o);
-          tmem_wait_ld();
-          if (valid) store_half32(a.part_o + prow * D + cb * 32, o, inv_c);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          uint32_t wv[4];
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            __half2 hv = __floats2half2_rn(o[8 * u + 2 * x] * sc, o[8 * u + 2 * x + 1] * sc);
+            wv[x] = *reinterpret_cast<uint32_t*>(&hv);
+          }
+          const uint32_t dst = smem_u32(stg + lane * 128 + ((u ^ (lane & 7)) << 4));
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(wv[0]), "r"(wv[1]), "r"(wv[2]),
+                       "r"(wv[3])
+                       : "memory");
+        }
+        fence_proxy_async_smem();  // the TMA store reads the staged rows (async proxy)
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&omap, stg, 0, (tile_begin + i) * 128 + q4 * 32, h);
+          bulk_commit_group();
         }
       }
-      if (valid) a.part_ml[prow] = make_float4(mrow, lrow, c, 0.f);
-    }
-    tc_fence_before();
-  }
-  __syncthreads();
-  if (*abort_flag) {
-    if (warp == 0 && lane == 0) {
-      const long long t_start = clock64();
-      while (!mbar_test(&sm.full, 0) && clock64() - t_start < kWaitCycles) {
+      if (valid) a.part_ml[prow] = make_float4(mrow, lrow, c_lo, c_hi);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&sm.o_free[w]);
+        mbar_arrive(&sm.info_empty[si]);
       }
     }
-    if (warp == 1 && lane == 0) {
+    if (lane == 0) bulk_wait_all();  // partial rows written before the CTA exits
+    __syncwarp();
+  }
+
+  // ------------------------------------------------------------------ teardown
+  __syncthreads();
+  if (*abort_flag) {
+    // drain: wait (bounded) for the last TMA load issued into each stage and for MMAs in
+    // flight, so no async write lands after the CTA exits
+    if (warp == 0 && lane == 0) {
+      for (int u = kv_issued - kSelKVStages > 0 ? kv_issued - kSelKVStages : 0; u < kv_issued; ++u) {
+        const long long t_start = clock64();
+        while (!mbar_test(&sm.kv_full[u % kSelKVStages], (u / kSelKVStages) & 1) &&
+               clock64() - t_start < kWaitCycles) {
+        }
+      }
+    }
+    if (warp == kSelMmaWarp && lane == 0) {
       umma_commit(&sm.drain);
       const long long t_start = clock64();
       while (!mbar_test(&sm.drain, 0) && clock64() - t_start < kWaitCycles) {
@@ -343,7 +593,7 @@ __global__ void __launch_bounds__(kSelInvThreads, 1)
     __syncwarp();
     __syncthreads();
   }
-  if (warp == 1) {
+  if (warp == kSelMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -356,7 +606,8 @@ __device__ __forceinline__ float warp_sum(float x) {
 }
 
 // One warp per (token, head): merges the row's partials (the slots holding a block index).
-// Lane l owns output elements [l * D/32, (l+1) * D/32).
+// Lane l owns output elements [l * D/32, (l+1) * D/32), all in 64-column half
+// (l * D/32) / 64 of the partial rows.
 template <int D>
 __global__ void __launch_bounds__(256) sel_merge_kernel(const SelInvArgs a) {
   constexpr int kPer = D / 32;
@@ -364,18 +615,24 @@ __global__ void __launch_bounds__(256) sel_merge_kernel(const SelInvArgs a) {
   const int lane = threadIdx.x & 31;
   if (row >= static_cast<long long>(a.nv) * a.hq) return;
   const int t = static_cast<int>(row / a.hq), h = static_cast<int>(row % a.hq);
-  const int g = h / a.G;
-  const int32_t* sel = a.sel_idx + (static_cast<size_t>(t) * a.hkv + g) * a.top_n;
-  const float4* ml = a.part_ml + static_cast<size_t>(row) * a.top_n;
-  // lane s holds slot s's (max, sum, c); top_n <= 64
-  float4 x0 = make_float4(-INFINITY, 0.f, 1.f, 0.f), x1 = x0;
+  const int g = h / a.G, hh = h - g * a.G;
+  const size_t base = (static_cast<size_t>(t) * a.hkv + g) * a.top_n;
+  // lane s holds slot s's (max, sum, c0, c1) and partial row; top_n <= 64
+  float4 x0 = make_float4(-INFINITY, 0.f, 1.f, 1.f), x1 = x0;
+  int r0 = 0, r1 = 0;
   if (lane < a.top_n) {
-    const int j = sel[lane];
-    if (j >= 0 && j < a.nsel) x0 = ml[lane];
+    const int j = a.sel_idx[base + lane];
+    if (j >= 0 && j < a.nsel) {
+      r0 = a.row_of[base + lane] + hh;
+      x0 = a.part_ml[r0];
+    }
   }
   if (lane + 32 < a.top_n) {
-    const int j = sel[lane + 32];
-    if (j >= 0 && j < a.nsel) x1 = ml[lane + 32];
+    const int j = a.sel_idx[base + lane + 32];
+    if (j >= 0 && j < a.nsel) {
+      r1 = a.row_of[base + lane + 32] + hh;
+      x1 = a.part_ml[r1];
+    }
   }
   float M = fmaxf(x0.y > 0.f ? x0.x : -INFINITY, x1.y > 0.f ? x1.x : -INFINITY);
 #pragma unroll
@@ -383,29 +640,47 @@ __global__ void __launch_bounds__(256) sel_merge_kernel(const SelInvArgs a) {
   const float w0 = (x0.y > 0.f) ? x0.y * ex2_approx(x0.x - M) : 0.f;
   const float w1 = (x1.y > 0.f) ? x1.y * ex2_approx(x1.x - M) : 0.f;
   const float L = warp_sum(w0 + w1);
-  const float wc0 = w0 * x0.z, wc1 = w1 * x1.z;
+  const int half = (lane * kPer) >> 6;
+  const int col = (lane * kPer) & 63;
+  const __half* po = a.part_o + static_cast<size_t>(half) * a.part_rows * 64 + col;
   float acc[kPer];
 #pragma unroll
   for (int u = 0; u < kPer; ++u) acc[u] = 0.f;
-  const __half* po = a.part_o + static_cast<size_t>(row) * a.top_n * D + lane * kPer;
-  for (int s = 0; s < a.top_n; ++s) {
-    const float w = __shfl_sync(0xffffffffu, s < 32 ? wc0 : wc1, s & 31);
-    if (w == 0.f) continue;  // uniform across the warp
-    const __half* src = po + static_cast<size_t>(s) * D;
-    if constexpr (kPer == 4) {
-      const uint2 raw = *reinterpret_cast<const uint2*>(src);
-      const float2 y0 = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-      const float2 y1 = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-      acc[0] += w * y0.x;
-      acc[1] += w * y0.y;
-      acc[2] += w * y1.x;
-      acc[3] += w * y1.y;
-    } else {
-      const uint32_t raw = *reinterpret_cast<const uint32_t*>(src);
-      const float2 y0 = __half22float2(*reinterpret_cast<const __half2*>(&raw));
-      acc[0] += w * y0.x;
-      acc[1] += w * y0.y;
+  // 16 slots per round: all loads issue before the first use
+  for (int s0 = 0; s0 < a.top_n; s0 += 16) {
+    const bool lo = s0 < 32;
+    float wc[16];
+    uint32_t raw[16][kPer / 2];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int src = (s0 + k) & 31;
+      const float w = __shfl_sync(0xffffffffu, lo ? w0 : w1, src);
+      const float c0 = __shfl_sync(0xffffffffu, lo ? x0.z : x1.z, src);
+      const float c1 = __shfl_sync(0xffffffffu, lo ? x0.w : x1.w, src);
+      const int prow = __shfl_sync(0xffffffffu, lo ? r0 : r1, src);
+      wc[k] = (s0 + k < a.top_n) ? w * (half == 0 ? c0 : c1) : 0.f;
+      const __half* p = po + static_cast<size_t>(prow) * 64;
+      if (wc[k] != 0.f) {
+        if constexpr (kPer == 4) {
+          const uint2 v = *reinterpret_cast<const uint2*>(p);
+          raw[k][0] = v.x;
+          raw[k][1] = v.y;
+        } else {
+          raw[k][0] = *reinterpret_cast<const uint32_t*>(p);
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < kPer / 2; ++u) raw[k][u] = 0u;
+      }
     }
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+#pragma unroll
+      for (int u = 0; u < kPer / 2; ++u) {
+        const float2 y = __half22float2(*reinterpret_cast<const __half2*>(&raw[k][u]));
+        acc[2 * u] += wc[k] * y.x;
+        acc[2 * u + 1] += wc[k] * y.y;
+      }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   float* dst = a.o_sel + static_cast<size_t>(row) * D + lane * kPer;
