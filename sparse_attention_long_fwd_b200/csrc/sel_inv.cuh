@@ -607,9 +607,10 @@ __device__ __forceinline__ float warp_sum(float x) {
 
 // One warp per (token, head): merges the row's partials (the slots holding a block index).
 // Lane l owns output elements [l * D/32, (l+1) * D/32), all in 64-column half
-// (l * D/32) / 64 of the partial rows.
+// (l * D/32) / 64 of the partial rows. The partial rows are loaded as soon as their row
+// numbers are known, alongside the (max, sum) records that weight them.
 template <int D>
-__global__ void __launch_bounds__(256) sel_merge_kernel(const SelInvArgs a) {
+__global__ void __launch_bounds__(256, 3) sel_merge_kernel(const SelInvArgs a) {
   constexpr int kPer = D / 32;
   const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -617,50 +618,38 @@ __global__ void __launch_bounds__(256) sel_merge_kernel(const SelInvArgs a) {
   const int t = static_cast<int>(row / a.hq), h = static_cast<int>(row % a.hq);
   const int g = h / a.G, hh = h - g * a.G;
   const size_t base = (static_cast<size_t>(t) * a.hkv + g) * a.top_n;
-  // lane s holds slot s's (max, sum, c0, c1) and partial row; top_n <= 64
-  float4 x0 = make_float4(-INFINITY, 0.f, 1.f, 1.f), x1 = x0;
-  int r0 = 0, r1 = 0;
+  // lane s holds slot s (and s + 32): its partial row, or -1; top_n <= 64
+  int r0 = -1, r1 = -1;
   if (lane < a.top_n) {
     const int j = a.sel_idx[base + lane];
-    if (j >= 0 && j < a.nsel) {
-      r0 = a.row_of[base + lane] + hh;
-      x0 = a.part_ml[r0];
-    }
+    const int rb = a.row_of[base + lane];
+    if (j >= 0 && j < a.nsel) r0 = rb + hh;
   }
   if (lane + 32 < a.top_n) {
     const int j = a.sel_idx[base + lane + 32];
-    if (j >= 0 && j < a.nsel) {
-      r1 = a.row_of[base + lane + 32] + hh;
-      x1 = a.part_ml[r1];
-    }
+    const int rb = a.row_of[base + lane + 32];
+    if (j >= 0 && j < a.nsel) r1 = rb + hh;
   }
-  float M = fmaxf(x0.y > 0.f ? x0.x : -INFINITY, x1.y > 0.f ? x1.x : -INFINITY);
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  const float w0 = (x0.y > 0.f) ? x0.y * ex2_approx(x0.x - M) : 0.f;
-  const float w1 = (x1.y > 0.f) ? x1.y * ex2_approx(x1.x - M) : 0.f;
-  const float L = warp_sum(w0 + w1);
+  const float4 none = make_float4(-INFINITY, 0.f, 1.f, 1.f);
+  const float4 x0 = r0 >= 0 ? a.part_ml[r0] : none;
+  const float4 x1 = r1 >= 0 ? a.part_ml[r1] : none;
   const int half = (lane * kPer) >> 6;
   const int col = (lane * kPer) & 63;
   const __half* po = a.part_o + static_cast<size_t>(half) * a.part_rows * 64 + col;
   float acc[kPer];
 #pragma unroll
   for (int u = 0; u < kPer; ++u) acc[u] = 0.f;
-  // 16 slots per round: all loads issue before the first use
+  float M = -INFINITY, w0 = 0.f, w1 = 0.f, L = 0.f;
   for (int s0 = 0; s0 < a.top_n; s0 += 16) {
     const bool lo = s0 < 32;
-    float wc[16];
     uint32_t raw[16][kPer / 2];
+    int prow[16];
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
-      const int src = (s0 + k) & 31;
-      const float w = __shfl_sync(0xffffffffu, lo ? w0 : w1, src);
-      const float c0 = __shfl_sync(0xffffffffu, lo ? x0.z : x1.z, src);
-      const float c1 = __shfl_sync(0xffffffffu, lo ? x0.w : x1.w, src);
-      const int prow = __shfl_sync(0xffffffffu, lo ? r0 : r1, src);
-      wc[k] = (s0 + k < a.top_n) ? w * (half == 0 ? c0 : c1) : 0.f;
-      const __half* p = po + static_cast<size_t>(prow) * 64;
-      if (wc[k] != 0.f) {
+      prow[k] = __shfl_sync(0xffffffffu, lo ? r0 : r1, (s0 + k) & 31);
+      if (s0 + k >= a.top_n) prow[k] = -1;
+      const __half* p = po + static_cast<size_t>(prow[k] < 0 ? 0 : prow[k]) * 64;
+      if (prow[k] >= 0) {
         if constexpr (kPer == 4) {
           const uint2 v = *reinterpret_cast<const uint2*>(p);
           raw[k][0] = v.x;
@@ -673,14 +662,27 @@ __global__ void __launch_bounds__(256) sel_merge_kernel(const SelInvArgs a) {
         for (int u = 0; u < kPer / 2; ++u) raw[k][u] = 0u;
       }
     }
+    if (s0 == 0) {  // weights: exp2(max - M) * sum over the slots with keys
+      M = fmaxf(x0.y > 0.f ? x0.x : -INFINITY, x1.y > 0.f ? x1.x : -INFINITY);
 #pragma unroll
-    for (int k = 0; k < 16; ++k)
+      for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      w0 = (x0.y > 0.f) ? x0.y * ex2_approx(x0.x - M) : 0.f;
+      w1 = (x1.y > 0.f) ? x1.y * ex2_approx(x1.x - M) : 0.f;
+      L = warp_sum(w0 + w1);
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int src = (s0 + k) & 31;
+      const float w = __shfl_sync(0xffffffffu, lo ? w0 : w1, src);
+      const float c = __shfl_sync(0xffffffffu, lo ? (half == 0 ? x0.z : x0.w) : (half == 0 ? x1.z : x1.w), src);
+      const float wc = prow[k] >= 0 ? w * c : 0.f;
 #pragma unroll
       for (int u = 0; u < kPer / 2; ++u) {
         const float2 y = __half22float2(*reinterpret_cast<const __half2*>(&raw[k][u]));
-        acc[2 * u] += wc[k] * y.x;
-        acc[2 * u + 1] += wc[k] * y.y;
+        acc[2 * u] += wc * y.x;
+        acc[2 * u + 1] += wc * y.y;
       }
+    }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   float* dst = a.o_sel + static_cast<size_t>(row) * D + lane * kPer;
