@@ -150,6 +150,136 @@ __device__ __forceinline__ void warp_topn(float* sc, uint32_t* bits, int* list, 
   __syncwarp();
 }
 
+// Register-resident variant for rows with at most 32 * PL candidate blocks (jt < 32 * PL):
+// lane l holds blocks l, l + 32, ... as 32-bit keys (score bits + 1 for a candidate, so a
+// zero score stays selectable; 0 for none); key order is score order because scores are
+// non-negative. Warp-wide maxima are single __reduce_max_sync instructions.
+//   1. each lane's two half-slice maxima: the k-th largest of those 64 keys is a lower
+//      bound on the k-th largest key overall (they are distinct blocks of the row);
+//   2. candidates at or above that bound are compacted to `list` (as block indices);
+//   3. k rounds take the largest key among them, the smallest block index on ties.
+template <int PL>
+__device__ __forceinline__ void warp_topn_regs(uint32_t* bits, int* list, const float* __restrict__ src, int jt,
+                                               int top_n, int32_t* __restrict__ dst, int32_t* __restrict__ dst2,
+                                               int lane) {
+  const int nwords = jt / 32 + 1;
+  for (int w = lane; w < nwords; w += 32) bits[w] = 0u;
+  float v[PL];
+#pragma unroll
+  for (int u = 0; u < PL; ++u) {
+    const int j = lane + 32 * u;
+    v[u] = j <= jt ? src[j] : -1.f;
+  }
+  uint32_t key[PL];
+#pragma unroll
+  for (int u = 0; u < PL; ++u) {
+    const int j = lane + 32 * u;
+    const bool forced = j == 0 || j == jt || j == jt - 1;
+    key[u] = (j <= jt && !forced && v[u] >= 0.f) ? __float_as_uint(v[u]) + 1u : 0u;
+  }
+  __syncwarp();
+  if (lane == 0) {
+    bits[0] |= 1u;
+    if (jt >= 1) bits[jt >> 5] |= 1u << (jt & 31);
+    if (jt >= 2) bits[(jt - 1) >> 5] |= 1u << ((jt - 1) & 31);
+  }
+  const int nf = 1 + (jt >= 1 ? 1 : 0) + (jt >= 2 ? 1 : 0);
+  const int k = min(top_n - nf, jt + 1 - nf);
+  if (k > 0) {
+    // 1. lower bound: k-th largest of the 64 half-slice maxima (0 when fewer exist)
+    uint32_t a = 0u, b = 0u;
+#pragma unroll
+    for (int u = 0; u < PL; ++u) {
+      if (u < PL / 2 || PL == 1) a = max(a, key[u]);
+      else b = max(b, key[u]);
+    }
+    uint32_t thr = 0u;
+    if (k <= 64) {
+      for (int round = 0; round < k; ++round) {
+        const uint32_t w = __reduce_max_sync(0xffffffffu, max(a, b));
+        thr = w;
+        if (w == 0u) break;
+        // remove one instance of w: the lowest lane holding it, its first slot
+        const uint32_t holders = __ballot_sync(0xffffffffu, a == w || b == w);
+        if (lane == __ffs(holders) - 1) {
+          if (a == w) a = 0u; else b = 0u;
+        }
+      }
+    }
+    // 2. compact the candidates with key >= thr (block indices, in lane-slot order)
+    int cnt = 0;
+#pragma unroll
+    for (int u = 0; u < PL; ++u) cnt += (key[u] != 0u && key[u] >= thr) ? 1 : 0;
+    int off = cnt;  // inclusive scan over lanes
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, off, o);
+      if (lane >= o) off += y;
+    }
+    const int nsurv = __shfl_sync(0xffffffffu, off, 31);
+    off -= cnt;
+#pragma unroll
+    for (int u = 0; u < PL; ++u)
+      if (key[u] != 0u && key[u] >= thr) list[off++] = lane + 32 * u;
+    __syncwarp();
+    // 3. exact top-k among them: largest key, smallest block index on ties
+    if (nsurv <= 64) {
+      const int j0 = lane < nsurv ? list[lane] : -1, j1 = lane + 32 < nsurv ? list[lane + 32] : -1;
+      // the keys again from the (cached) scores of the compacted blocks
+      uint32_t q0 = j0 >= 0 ? __float_as_uint(src[j0]) + 1u : 0u;
+      uint32_t q1 = j1 >= 0 ? __float_as_uint(src[j1]) + 1u : 0u;
+      for (int round = 0; round < k; ++round) {
+        const uint32_t w = __reduce_max_sync(0xffffffffu, max(q0, q1));
+        if (w == 0u) break;
+        const uint32_t c0 = q0 == w ? static_cast<uint32_t>(j0) : 0xFFFFFFFFu;
+        const uint32_t c1 = q1 == w ? static_cast<uint32_t>(j1) : 0xFFFFFFFFu;
+        const uint32_t jw = __reduce_min_sync(0xffffffffu, min(c0, c1));
+        if (static_cast<uint32_t>(j0) == jw) q0 = 0u;
+        if (static_cast<uint32_t>(j1) == jw) q1 = 0u;
+        if (lane == 0) bits[jw >> 5] |= 1u << (jw & 31);
+      }
+    } else {
+      // many ties at the bound: rounds over the compacted list (keys reloaded by block)
+      for (int round = 0; round < k; ++round) {
+        uint32_t best = 0u, bj = 0xFFFFFFFFu;
+        for (int i = lane; i < nsurv; i += 32) {
+          const int j = list[i];
+          const uint32_t x = (j >= 0 && src[j] >= 0.f) ? __float_as_uint(src[j]) + 1u : 0u;
+          if (x > best || (x == best && x != 0u && static_cast<uint32_t>(j) < bj)) {
+            best = x;
+            bj = static_cast<uint32_t>(j);
+          }
+        }
+        const uint32_t w = __reduce_max_sync(0xffffffffu, best);
+        if (w == 0u) break;
+        const uint32_t jw = __reduce_min_sync(0xffffffffu, best == w ? bj : 0xFFFFFFFFu);
+        for (int i = lane; i < nsurv; i += 32)
+          if (list[i] == static_cast<int>(jw)) list[i] = -1;
+        if (lane == 0) bits[jw >> 5] |= 1u << (jw & 31);
+        __syncwarp();
+      }
+    }
+  }
+  __syncwarp();
+  // emit the selected set in ascending order, then -1 padding
+  int pos = 0;
+  for (int w = 0; w < nwords; ++w) {
+    const uint32_t word = bits[w];
+    const bool set = (word >> lane) & 1u;
+    const int p = pos + __popc(word & ((1u << lane) - 1u));
+    if (set && p < top_n) {
+      dst[p] = w * 32 + lane;
+      if (dst2) dst2[p] = w * 32 + lane;
+    }
+    pos += __popc(word);
+  }
+  for (int p = pos + lane; p < top_n; p += 32) {
+    dst[p] = -1;
+    if (dst2) dst2[p] = -1;
+  }
+  __syncwarp();
+}
+
 // scores: [nitems][nsel] fp32 (item = row * hkv + g); idx / idx_copy: [nitems][top_n].
 // Row position t = row (prefill rows are token positions).
 __global__ void __launch_bounds__(kTopnWarps * 32) topn_kernel(const float* __restrict__ scores, int nitems, int hkv,
@@ -169,9 +299,14 @@ __global__ void __launch_bounds__(kTopnWarps * 32) topn_kernel(const float* __re
       if (lane == 0) record_error(kErrBadIndex);
       continue;
     }
-    warp_topn(sc, bits, list, scores + static_cast<size_t>(item) * nsel, jt, top_n,
-              idx + static_cast<size_t>(item) * top_n,
-              idx_copy ? idx_copy + static_cast<size_t>(item) * top_n : nullptr, lane);
+    const float* src = scores + static_cast<size_t>(item) * nsel;
+    int32_t* d = idx + static_cast<size_t>(item) * top_n;
+    int32_t* d2 = idx_copy ? idx_copy + static_cast<size_t>(item) * top_n : nullptr;
+    if (jt < 32 * 4) warp_topn_regs<4>(bits, list, src, jt, top_n, d, d2, lane);
+    else if (jt < 32 * 16) warp_topn_regs<16>(bits, list, src, jt, top_n, d, d2, lane);
+    else if (jt < 32 * 32) warp_topn_regs<32>(bits, list, src, jt, top_n, d, d2, lane);
+    else if (jt < 32 * 64) warp_topn_regs<64>(bits, list, src, jt, top_n, d, d2, lane);
+    else warp_topn(sc, bits, list, src, jt, top_n, d, d2, lane);
   }
 }
 

@@ -51,6 +51,8 @@ WORKLOADS = {
                                     frame_mean_var=0.5),
     # a 32,768-token cut of the 128K workload (inputs still larger than L2), for kernel profiles
     "v32k": Workload("v32k", 32768, 32768, frame_mean_var=0.5),
+    # a 16,384-token cut (about 3 GB on the device), for multi-pass kernel profiles
+    "v16k": Workload("v16k", 16384, 16384, frame_mean_var=0.5),
     # 64 sequences x 131,072-token cache, one query each
     "decode64x128k": Workload("decode64x128k", 131072, 131072, batch=64),
 }
