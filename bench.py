@@ -43,6 +43,10 @@ PREFILL_STAGES = ["pool", "cmp_attn_scores", "topn", "sel_bucket", "sel_tile", "
 # kernels of ours launched per prefill step: pool, compressed tile, top-n, bucket count / scan / scatter,
 # selected partial, merge, window tile (+ the dense text tile)
 PREFILL_KERNELS = 9
+# DRAM bytes per launch of a stage's kernel on the 128K workload, from one ncu capture of the
+# current kernel version (profiles/dram_traffic_v128k.md); an entry is removed when its kernel
+# changes, and the roofline then reports traffic null.
+STAGE_TRAFFIC_V128K = {"cmp_attn_scores": 1109649920 + 4012024576}
 DECODE_STAGES = ["dec_cmp", "dec_select", "dec_branches", "dec_combine"]
 
 
@@ -251,8 +255,11 @@ def run_b200(args, world, rank, local):
     peak_t = peaks["bf16_tflops_sustained"]
     if dom in stage_flops:
         ach = stage_flops[dom] / (stages[dom] / 1e3) / 1e12
+        traffic = STAGE_TRAFFIC_V128K.get(dom) if w.name == "v128k" else None
         roofline = {"kernel": dom, "bound": "tensor", "achieved": round(ach, 2), "peak": peak_t, "unit": "TFLOP/s",
-                    "frac": round(ach / peak_t, 4), "traffic": None,
+                    "frac": round(ach / peak_t, 4), "traffic": traffic,
+                    "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one full-size launch"
+                    if traffic else None,
                     "peak_source": f"{peaks_src} bf16_tflops_sustained (kernel timed inside a long step loop)",
                     "algorithmic": f"{stage_flops[dom]:.4e} FLOP per launch (attended keys only)"}
     else:
