@@ -107,9 +107,8 @@ PrefillLayout prefill_layout(const nsa_params_t* p) {
   L.sel_list = take(entries * 4);
   L.sel_row = take(entries * 4);
   {
-    int gc = 1;  // heads per token in a tile row block: G rounded up to a power of two
-    while (gc < hq / (hkv > 0 ? hkv : 1)) gc <<= 1;
-    const size_t tiles = (entries + (128 / gc) - 1) / (128 / gc) + buckets;
+    const int G = hq / (hkv > 0 ? hkv : 1);  // a token's heads take G consecutive tile rows
+    const size_t tiles = (entries + (128 / G) - 1) / (128 / G) + buckets;
     L.part_rows = static_cast<long long>(tiles) * 128;
   }
   L.part_o = take(static_cast<size_t>(L.part_rows) * d * 2);
@@ -306,7 +305,7 @@ int prefill_impl(const nsa_params_t* p, const void* q, const void* k, const void
     //    one tensor-core tile per bucket tile, then merge each row's partials
     {
       const int m = hkv * L.nsel;
-      const int Gp = Gc;
+      const int Gp = G;  // tile rows token * G + head: no padding heads
       const int TT = 128 / Gp;
       const long long entries = static_cast<long long>(nv) * hkv * p->top_n;
       nsa::SelInvArgs sa{};

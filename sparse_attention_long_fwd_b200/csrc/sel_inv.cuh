@@ -11,7 +11,8 @@
 // would. The sum is taken over the bf16-rounded P that the tensor core multiplies, so each
 // partial is an exact convex combination of values. Partials live in tile order: tile k
 // owns rows 128k .. 128k+127 (MMA row r = token slot r / Gp, head slot r % Gp), so a warp
-// writes its 32 rows with one TMA store per 64 output columns; sel_scatter_kernel records
+// writes its 32 rows with one TMA store per 64 output columns (Gp = G: 7 heads pack 18 tokens
+// into 126 rows; the last two rows are unused); sel_scatter_kernel records
 // where each (token, group, slot) landed. The partial output is stored in fp16 (2^-12
 // relative rounding); a 64-column half whose largest magnitude would overflow fp16 is
 // stored divided by a power of two c, kept with the row's (max, sum).
@@ -250,7 +251,6 @@ __global__ void __launch_bounds__(kSelTileThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort_flag = &sm.abort_flag;
   const int Gp = a.Gp, G = a.G;
-  const int lg_gp = __ffs(Gp) - 1;  // Gp is a power of two
   int kv_issued = 0;  // warp 0: K-V loads issued
 
   if (warp < kSelProducers) {
@@ -332,7 +332,7 @@ __global__ void __launch_bounds__(kSelTileThreads, 1)
           int my_row = -1;
           {
             const int R = rbase + lane;
-            const int hh = R & (Gp - 1), tok = R >> lg_gp;
+            const int tok = R / Gp, hh = R - tok * Gp;
             if (tok < cnt && hh < G && g * G + hh < a.hq) my_row = (inf.ent[tok] >> 6) * a.hq + g * G + hh;
           }
           constexpr int kRpi = 32 / kCpr;  // rows per iteration
