@@ -402,6 +402,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // iteration), so the slices never exchange data. The G heads of a token sit in Gp
     // adjacent lanes; a shuffle reduce-scatter sums them.
     float carry = 0.f;  // warpgroup 0: half of the previous tile's last compressed block
+    // (kModeCmp) after the head reduce-scatter, lane hh holds blocks [hh*bpl, (hh+1)*bpl) of
+    // its warpgroup's slice (Gp <= kBinsPerWG), or block hh/share shared with its neighbours
+    // (Gp > kBinsPerWG); these store invariants do not change from tile to tile
+    const int sc_bpl = Gp <= kBinsPerWG ? kBinsPerWG / Gp : 1;
+    const int sc_share = Gp <= kBinsPerWG ? 1 : Gp / kBinsPerWG;
+    const bool sc_store = MODE == kModeCmp && t < args.q_end && (hh % sc_share) == 0;
+    const int sc_jt = t / args.sel_len;
+    const int sc_j0 = wg * kBinsPerWG + (hh / sc_share) * sc_bpl;
+    float* const sc_dst = args.scores + (static_cast<size_t>(t) * args.hkv + g) * args.nsel;
     for (int kt2 = 0; kt2 < nkt; ++kt2) {
       const int job = nkt + kt2;
       const int b = job & 1;
@@ -484,17 +493,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           case 16: group_reduce_scatter<16, kBinsPerWG>(bin, lane); break;
           default: break;
         }
-        // lane hh now holds blocks [hh*bpl, (hh+1)*bpl) of this slice (Gp <= kBinsPerWG),
-        // or block hh/(Gp/kBinsPerWG) shared with its neighbours (Gp > kBinsPerWG)
-        const int bpl = Gp <= kBinsPerWG ? kBinsPerWG / Gp : 1;
-        const int share = Gp <= kBinsPerWG ? 1 : Gp / kBinsPerWG;
-        if (t < args.q_end && (hh % share) == 0) {
-          const int jt = t / args.sel_len;
-          const int j0 = kt2 * 32 + wg * kBinsPerWG + (hh / share) * bpl;
-          float* dst = args.scores + (static_cast<size_t>(t) * args.hkv + g) * args.nsel;
+        if (sc_store) {
+          const int j0 = kt2 * 32 + sc_j0;
+          if (sc_bpl == 1) {
+            if (j0 <= sc_jt) sc_dst[j0] = bin[0];
+          } else {
 #pragma unroll
-          for (int i = 0; i < kBinsPerWG; ++i)
-            if (i < bpl && j0 + i <= jt) dst[j0 + i] = bin[i];
+            for (int i = 0; i < kBinsPerWG; ++i)
+              if (i < sc_bpl && j0 + i <= sc_jt) sc_dst[j0 + i] = bin[i];
+          }
         }
       }
     }
