@@ -342,15 +342,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           s[i] = (kidx >= rb && kidx < re) ? s[i] : -INFINITY;
         }
       }
+      static_assert(kColsPerWG == 32, "the max tree below covers 32 columns");
       float mx[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) mx[c] = s[c];
-#pragma unroll
-      for (int i = 8; i < kColsPerWG; i += 8)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) mx[c] = fmaxf(mx[c], s[i + c]);
-      const float cmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      for (int c = 0; c < 8; ++c) mx[c] = fmaxf(fmax3f(s[c], s[c + 8], s[c + 16]), s[c + 24]);
+      const float cmax = fmax3f(fmax3f(mx[0], mx[1], mx[2]), fmax3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
       const float mnew = fmaxf(m, cmax);
       if (MODE != kModeCmp) {
         m = mnew;  // the window and dense branches need only the row max here

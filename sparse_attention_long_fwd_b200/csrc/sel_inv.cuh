@@ -470,13 +470,12 @@ __global__ void __launch_bounds__(kSelTileThreads, 1)
       for (int c = 0; c < 64; ++c) s[c] = c < key_hi ? s[c] : -INFINITY;
       float mx[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) mx[c] = s[c];
+      for (int c = 0; c < 8; ++c) mx[c] = fmax3f(s[c], s[c + 8], s[c + 16]);
 #pragma unroll
-      for (int c = 8; c < 64; c += 8)
+      for (int c = 24; c < 64; c += 16)
 #pragma unroll
-        for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], s[c + u]);
-      const float mraw =
-          fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        for (int u = 0; u < 8; ++u) mx[u] = fmax3f(mx[u], s[c + u], s[c + 8 + u]);
+      const float mraw = fmax3f(fmax3f(mx[0], mx[1], mx[2]), fmax3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
       const float mrow = mraw * a.sl2;  // row max in log2 units (the scale is positive)
       const float bias = mraw == -INFINITY ? 0.f : -mrow;
       // this warp's rows of P were the staging buffer of its previous tile's partial store
@@ -520,14 +519,12 @@ __global__ void __launch_bounds__(kSelTileThreads, 1)
         tmem_wait_ld();
         float am[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) am[u] = fabsf(o[u]);
+        for (int x = 0; x < 8; ++x) am[x] = fmax3f(fabsf(o[x]), fabsf(o[x + 8]), fabsf(o[x + 16]));
 #pragma unroll
-        for (int u = 8; u < 64; u += 8)
+        for (int u = 24; u < 64; u += 16)
 #pragma unroll
-          for (int x = 0; x < 8; ++x) am[x] = fmaxf(am[x], fabsf(o[u + x]));
-        const float amax =
-            fmaxf(fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3])), fmaxf(fmaxf(am[4], am[5]), fmaxf(am[6], am[7]))) *
-            inv;
+          for (int x = 0; x < 8; ++x) am[x] = fmax3f(am[x], fabsf(o[u + x]), fabsf(o[u + 8 + x]));
+        const float amax = fmax3f(fmax3f(am[0], am[1], am[2]), fmax3f(am[3], am[4], am[5]), fmaxf(am[6], am[7])) * inv;
         // 65504 is the largest finite fp16 value; rare rows are scaled down by a power of two
         float c = 1.f, sc = inv;
         if (amax > 65504.f) {
