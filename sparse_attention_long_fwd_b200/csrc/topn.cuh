@@ -150,7 +150,8 @@ __device__ __forceinline__ void warp_topn(float* sc, uint32_t* bits, int* list, 
   __syncwarp();
 }
 
-// Register-resident variant for rows with at most 32 * PL candidate blocks (jt < 32 * PL):
+// Register-resident variant for rows with at most 32 * PL candidate blocks (jt < 32 * PL)
+// and top_n <= 32 (the selected set is held one block per lane, then sorted):
 // lane l holds blocks l, l + 32, ... as 32-bit keys (score bits + 1 for a candidate, so a
 // zero score stays selectable; 0 for none); key order is score order because scores are
 // non-negative. Warp-wide maxima are single __reduce_max_sync instructions.
@@ -159,11 +160,8 @@ __device__ __forceinline__ void warp_topn(float* sc, uint32_t* bits, int* list, 
 //   2. candidates at or above that bound are compacted to `list` (as block indices);
 //   3. k rounds take the largest key among them, the smallest block index on ties.
 template <int PL>
-__device__ __forceinline__ void warp_topn_regs(uint32_t* bits, int* list, const float* __restrict__ src, int jt,
-                                               int top_n, int32_t* __restrict__ dst, int32_t* __restrict__ dst2,
-                                               int lane) {
-  const int nwords = jt / 32 + 1;
-  for (int w = lane; w < nwords; w += 32) bits[w] = 0u;
+__device__ __forceinline__ void warp_topn_regs(int* list, const float* __restrict__ src, int jt, int top_n,
+                                               int32_t* __restrict__ dst, int32_t* __restrict__ dst2, int lane) {
   float v[PL];
 #pragma unroll
   for (int u = 0; u < PL; ++u) {
@@ -177,20 +175,16 @@ __device__ __forceinline__ void warp_topn_regs(uint32_t* bits, int* list, const 
     const bool forced = j == 0 || j == jt || j == jt - 1;
     key[u] = (j <= jt && !forced && v[u] >= 0.f) ? __float_as_uint(v[u]) + 1u : 0u;
   }
-  __syncwarp();
-  if (lane == 0) {
-    bits[0] |= 1u;
-    if (jt >= 1) bits[jt >> 5] |= 1u << (jt & 31);
-    if (jt >= 2) bits[(jt - 1) >> 5] |= 1u << ((jt - 1) & 31);
-  }
+  // the selected blocks, one per lane (INT_MAX: none): forced blocks in lanes 0..nf-1
   const int nf = 1 + (jt >= 1 ? 1 : 0) + (jt >= 2 ? 1 : 0);
+  int mine = lane == 0 ? 0 : (lane == 1 && jt >= 1) ? jt : (lane == 2 && jt >= 2) ? jt - 1 : 0x7fffffff;
   const int k = min(top_n - nf, jt + 1 - nf);
   if (k > 0) {
     // 1. lower bound: k-th largest of the 64 half-slice maxima (0 when fewer exist)
     uint32_t a = 0u, b = 0u;
 #pragma unroll
     for (int u = 0; u < PL; ++u) {
-      if (u < PL / 2 || PL == 1) a = max(a, key[u]);
+      if (u < PL / 2) a = max(a, key[u]);
       else b = max(b, key[u]);
     }
     uint32_t thr = 0u;
@@ -222,7 +216,8 @@ __device__ __forceinline__ void warp_topn_regs(uint32_t* bits, int* list, const 
     for (int u = 0; u < PL; ++u)
       if (key[u] != 0u && key[u] >= thr) list[off++] = lane + 32 * u;
     __syncwarp();
-    // 3. exact top-k among them: largest key, smallest block index on ties
+    // 3. exact top-k among them: largest key, smallest block index on ties; the winner of
+    //    round r goes to lane nf + r
     if (nsurv <= 64) {
       const int j0 = lane < nsurv ? list[lane] : -1, j1 = lane + 32 < nsurv ? list[lane + 32] : -1;
       // the keys again from the (cached) scores of the compacted blocks
@@ -236,7 +231,7 @@ __device__ __forceinline__ void warp_topn_regs(uint32_t* bits, int* list, const 
         const uint32_t jw = __reduce_min_sync(0xffffffffu, min(c0, c1));
         if (static_cast<uint32_t>(j0) == jw) q0 = 0u;
         if (static_cast<uint32_t>(j1) == jw) q1 = 0u;
-        if (lane == 0) bits[jw >> 5] |= 1u << (jw & 31);
+        if (lane == nf + round) mine = static_cast<int>(jw);
       }
     } else {
       // many ties at the bound: rounds over the compacted list (keys reloaded by block)
@@ -255,27 +250,26 @@ __device__ __forceinline__ void warp_topn_regs(uint32_t* bits, int* list, const 
         const uint32_t jw = __reduce_min_sync(0xffffffffu, best == w ? bj : 0xFFFFFFFFu);
         for (int i = lane; i < nsurv; i += 32)
           if (list[i] == static_cast<int>(jw)) list[i] = -1;
-        if (lane == 0) bits[jw >> 5] |= 1u << (jw & 31);
+        if (lane == nf + round) mine = static_cast<int>(jw);
         __syncwarp();
       }
     }
   }
-  __syncwarp();
-  // emit the selected set in ascending order, then -1 padding
-  int pos = 0;
-  for (int w = 0; w < nwords; ++w) {
-    const uint32_t word = bits[w];
-    const bool set = (word >> lane) & 1u;
-    const int p = pos + __popc(word & ((1u << lane) - 1u));
-    if (set && p < top_n) {
-      dst[p] = w * 32 + lane;
-      if (dst2) dst2[p] = w * 32 + lane;
+  // ascending order: bitonic sort of the 32 lanes' values (empty lanes sort last)
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const int other = __shfl_xor_sync(0xffffffffu, mine, stride);
+      const bool up = (lane & size) == 0;           // this block sorts ascending
+      const bool low = (lane & stride) == 0;        // this lane keeps the smaller value
+      mine = (low == up) ? min(mine, other) : max(mine, other);
     }
-    pos += __popc(word);
   }
-  for (int p = pos + lane; p < top_n; p += 32) {
-    dst[p] = -1;
-    if (dst2) dst2[p] = -1;
+  if (lane < top_n) {
+    const int out = mine == 0x7fffffff ? -1 : mine;
+    dst[lane] = out;
+    if (dst2) dst2[lane] = out;
   }
   __syncwarp();
 }
@@ -302,11 +296,11 @@ __global__ void __launch_bounds__(kTopnWarps * 32) topn_kernel(const float* __re
     const float* src = scores + static_cast<size_t>(item) * nsel;
     int32_t* d = idx + static_cast<size_t>(item) * top_n;
     int32_t* d2 = idx_copy ? idx_copy + static_cast<size_t>(item) * top_n : nullptr;
-    if (jt < 32 * 4) warp_topn_regs<4>(bits, list, src, jt, top_n, d, d2, lane);
-    else if (jt < 32 * 16) warp_topn_regs<16>(bits, list, src, jt, top_n, d, d2, lane);
-    else if (jt < 32 * 32) warp_topn_regs<32>(bits, list, src, jt, top_n, d, d2, lane);
-    else if (jt < 32 * 64) warp_topn_regs<64>(bits, list, src, jt, top_n, d, d2, lane);
-    else warp_topn(sc, bits, list, src, jt, top_n, d, d2, lane);
+    if (top_n > 32 || jt >= 32 * 64) warp_topn(sc, bits, list, src, jt, top_n, d, d2, lane);
+    else if (jt < 32 * 4) warp_topn_regs<4>(list, src, jt, top_n, d, d2, lane);
+    else if (jt < 32 * 16) warp_topn_regs<16>(list, src, jt, top_n, d, d2, lane);
+    else if (jt < 32 * 32) warp_topn_regs<32>(list, src, jt, top_n, d, d2, lane);
+    else warp_topn_regs<64>(list, src, jt, top_n, d, d2, lane);
   }
 }
 
