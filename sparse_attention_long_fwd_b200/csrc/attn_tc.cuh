@@ -314,6 +314,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int col0 = wg * kColsPerWG;
+    if (MODE == kModeWin && row_valid) {
+      // the epilogue reads this row's o_cmp, o_sel and gates: start bringing them into L2
+      const size_t orow = (static_cast<size_t>(t) * args.hq + h) * D + wg * (D / kSoftmaxWG);
+#pragma unroll
+      for (int c = 0; c < D / kSoftmaxWG; c += 32) {
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(args.o_cmp + orow + c));
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(args.o_sel + orow + c));
+      }
+      if (wg == 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(args.gates + (static_cast<size_t>(t) * args.hq + h) * 3));
+    }
     const float sl2 = args.scale_log2;
     bool ok = true;
     // ---- phase 1: log-sum-exp (base 2) of this row's column slice, combined below
