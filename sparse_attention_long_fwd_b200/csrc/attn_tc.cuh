@@ -78,7 +78,7 @@ struct AttnSmem {
   alignas(1024) uint8_t q[kChunks][kTileBytes];
   alignas(1024) uint8_t slot[kSlots][kChunks][kTileBytes];
   float lse_x[kSoftmaxWG][128][2];  // per warpgroup: (scaled max, sum) of the row's columns
-  uint64_t q_full;
+  uint64_t q_full, q_tmem;
   uint64_t full[kSlots], empty[kSlots];
   uint64_t s_full[2], s_free[2];
   uint64_t p_full, p_free, o_full, drain;
@@ -97,6 +97,11 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, u
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
 }
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
@@ -140,7 +145,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   constexpr int kChunks = Smem::kChunks;
   constexpr uint32_t kTmemCols = 512;
   constexpr uint32_t kColO = 256;  // S buffers at columns 0 and 128, O at 256
-  constexpr uint32_t kColP = 384;  // P buffers (bf16 pairs, 64 columns each) at 384 and 448
+  constexpr uint32_t kColP = 384;  // P (bf16 pairs, 64 columns)
+  constexpr uint32_t kColQ = 448;  // Q (bf16 pairs, D/2 columns): the A operand of every S MMA
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -171,6 +177,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (tid == 0) {
     mbar_init(&sm.q_full, 1);
+    mbar_init(&sm.q_tmem, 4 * kSoftmaxWG);
     for (int x = 0; x < Smem::kSlots; ++x) {
       mbar_init(&sm.full[x], 1);
       mbar_init(&sm.empty[x], 1);
@@ -236,7 +243,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (lane == 0 && nkt > 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, kBN, false, false);
       constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);
-      bool ok = mbar_wait(&sm.q_full, 0, abort_flag);
+      bool ok = mbar_wait(&sm.q_tmem, 0, abort_flag);  // Q staged in TMEM by the softmax warps
       auto wait_load = [&](int L) -> bool { return mbar_wait(&sm.full[L % kSlots], (L / kSlots) & 1, abort_flag); };
       auto issue_s = [&](int job) -> bool {
         const int L = job < nkt ? job : nkt + 2 * (job - nkt);
@@ -245,12 +252,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!wait_load(L)) return false;
         if (job >= 2 && !mbar_wait(&sm.s_free[b], ((job >> 1) - 1) & 1, abort_flag)) return false;
         tc_fence_after();
+        // A = Q from TMEM (dims 16k .. 16k+15 in columns kColQ + 8k ..), B = K from smem:
+        // the operand read from shared memory per MMA halves
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const int c = k >> 2, kk = k & 3;
-          const uint64_t a = sdesc_sw128(smem_u32(sm.q[c]) + kk * 32, 16, 1024);
           const uint64_t bd = sdesc_sw128(smem_u32(sm.slot[x][c]) + kk * 32, 16, 1024);
-          umma_bf16_ss(tmem + b * kBN, a, bd, idS, k > 0 ? 1u : 0u);
+          umma_bf16_ts(tmem + b * kBN, tmem + kColQ + k * 8, bd, idS, k > 0 ? 1u : 0u);
         }
         umma_commit(&sm.s_full[b]);
         umma_commit(&sm.empty[x]);  // the K tile is no longer needed
@@ -268,7 +276,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const int kt2 = job - nkt;
           const int L = nkt + 2 * kt2 + 1;  // V tile
           const int x = L % kSlots;
-          const int b = job & 1;
           if (!wait_load(L) || !mbar_wait(&sm.p_full, kt2 & 1, abort_flag)) {
             ok = false;
             break;
@@ -276,7 +283,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < kBN / 16; ++k) {
-            const uint32_t a_tmem = tmem + kColP + b * 64 + k * 8;  // keys 16k .. 16k+15
+            const uint32_t a_tmem = tmem + kColP + k * 8;  // keys 16k .. 16k+15
             const uint64_t bd = sdesc_sw128(smem_u32(sm.slot[x][0]) + k * 2048, Smem::kTileBytes, 1024);
             umma_bf16_ts(tmem + kColO, a_tmem, bd, idO, (kt2 > 0 || k > 0) ? 1u : 0u);
           }
@@ -326,6 +333,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     const float sl2 = args.scale_log2;
     bool ok = true;
+    // ---- Q row r into TMEM, packed in bf16 pairs like P: this warpgroup copies dims
+    // [wg*D/4, (wg+1)*D/4) from the 128-byte-swizzled smem image (16-byte unit u of a row
+    // sits at unit u ^ (row & 7)); rows past the tile are the zeros written at the start.
+    // A tile without keys loads no Q and runs no MMA.
+    if (nkt > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_full, 0, abort_flag));
+      if (ok) {
+        constexpr int kDimsPerWG = D / kSoftmaxWG;  // 32 (D=128) or 16 (D=64)
+        uint32_t qv[kDimsPerWG / 2];
+#pragma unroll
+        for (int i = 0; i < kDimsPerWG / 8; ++i) {
+          const int dim0 = wg * kDimsPerWG + 8 * i;
+          const int c = dim0 / 64, u = (dim0 % 64) / 8;
+          const uint4 w4 = *reinterpret_cast<const uint4*>(&sm.q[c][r * 128 + ((u ^ (r & 7)) << 4)]);
+          qv[4 * i] = w4.x;
+          qv[4 * i + 1] = w4.y;
+          qv[4 * i + 2] = w4.z;
+          qv[4 * i + 3] = w4.w;
+        }
+        __syncwarp();
+        if constexpr (kDimsPerWG / 2 == 16) {
+          tmem_st16(trow + kColQ + wg * 16, qv);
+        } else {
+          tmem_st8(trow + kColQ + wg * 8, qv);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.q_tmem);
+      }
+    }
     // ---- phase 1: log-sum-exp (base 2) of this row's column slice, combined below
     float m = -INFINITY, lsum = 0.f;         // m: running max of the raw (unscaled) scores
     for (int kt = 0; kt < nkt && ok; ++kt) {
@@ -423,7 +461,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (ok) ok = mbar_wait(&sm.s_full[b], (job >> 1) & 1, abort_flag);
       // P(kt2) is stored to TMEM only once the P.V MMA of the previous tile has finished:
       // tcgen05.st into TMEM while a P.V that reads its A operand from TMEM was still running
-      // corrupted rows 0-31 of the output on B200, although the two P buffers are disjoint.
+      // corrupted rows 0-31 of the output on B200 even while P was double-buffered in disjoint
+      // columns; with that wait in place one P buffer suffices.
       if (ok && kt2 > 0) ok = mbar_wait(&sm.p_free, (kt2 - 1) & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
@@ -478,14 +517,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           bin[u] = (u == 0 ? half_in : 0.5f * s[4 * u - 1]) + s[4 * u] + s[4 * u + 1] + s[4 * u + 2] + half_last;
         }
       }
-      // P row r, keys col0 .. col0+31 -> 16 packed bf16 pairs in P buffer b (TMEM columns
-      // kColP + 64b + col0/2 ..).
+      // P row r, keys col0 .. col0+31 -> 16 packed bf16 pairs in TMEM columns kColP + col0/2 ..
+      // (one P buffer: P(k) is stored only after the P.V of tile k-1 has finished).
       static_assert(kColsPerWG == 32, "P placement assumes 32 key columns per warpgroup");
       {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(s[2 * i], s[2 * i + 1]);
-        tmem_st16(trow + kColP + b * 64 + col0 / 2, pk);
+        tmem_st16(trow + kColP + col0 / 2, pk);
       }
       tmem_wait_st();
       tc_fence_before();
