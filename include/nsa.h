@@ -90,6 +90,33 @@ int nsa_prefill(const void* q, const void* k, const void* v, const float* gates,
                 void* out, int32_t* out_sel_idx, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Varlen prefill: B independent sequences packed back to back, the batch form a server
+ * uses. Sequence lengths vary from clip to clip (CSDN blog on VideoNSA, vcloud.csdn.net,
+ * section 5.2, item 3), and a hybrid sequence carries text rows after its video tokens
+ * (shd-paper.top page "VideoNSA: Native Sparse Attention Scales Video Understanding",
+ * abstract).
+ *   cu_seqlens  HOST array [B+1]: sequence b owns packed tokens [cu_seqlens[b], cu_seqlens[b+1]);
+ *               cu_seqlens[0] = 0, non-decreasing, cu_seqlens[B] = params->n_tokens.
+ *   n_video     HOST array [B]: sequence b's NSA-attended prefix, 0 <= n_video[b] <= its
+ *               length (params->n_video is ignored).
+ *   q, k, v, gates, out: as nsa_prefill, over the params->n_tokens packed tokens.
+ *   out_sel_idx NULL, or [sum of n_video][Hkv][top_n] int32: the video rows of every sequence,
+ *               sequence after sequence.
+ *   workspace   at least nsa_prefill_varlen_workspace_size(params, cu_seqlens, n_video, B) bytes.
+ * Each sequence gets exactly what nsa_prefill computes for it alone; positions restart at 0
+ * in every sequence. The sequences run one after another on `stream` and share the workspace,
+ * so the caller must not run two calls on one workspace concurrently. Errors as nsa_prefill,
+ * plus NSA_ERR_INVALID_ARG for malformed cu_seqlens / n_video; nothing is enqueued then.
+ */
+int nsa_prefill_varlen(const void* q, const void* k, const void* v, const float* gates, const int32_t* cu_seqlens,
+                       const int32_t* n_video, int batch, const nsa_params_t* params, void* out,
+                       int32_t* out_sel_idx, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes nsa_prefill_varlen needs (the largest single sequence's); 0 if the arguments are invalid. */
+size_t nsa_prefill_varlen_workspace_size(const nsa_params_t* params, const int32_t* cu_seqlens,
+                                         const int32_t* n_video, int batch);
+
+/*
  * Decode: one query token per sequence against a KV cache and its compressed cache.
  *   q       [B][Hq][d] bf16, the query at position seq_lens[b]-1 (its own K/V are in the cache)
  *   kcache, vcache [B][Lmax][Hkv][d] bf16 (Lmax = params->n_tokens)

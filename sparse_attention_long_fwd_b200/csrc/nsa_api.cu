@@ -440,6 +440,26 @@ int decode_impl(const nsa_params_t* p, const void* q, const void* kcache, const 
   return NSA_OK;
 }
 
+// Host-side checks of a packed batch; on success the per-sequence parameter sets are valid.
+int check_varlen(const nsa_params_t* params, const int32_t* cu, const int32_t* nv, int batch) {
+  int rc = check_common(params);
+  if (rc != NSA_OK) return rc;
+  if (!cu || !nv || batch < 1 || cu[0] != 0 || cu[batch] != params->n_tokens) return NSA_ERR_INVALID_ARG;
+  for (int b = 0; b < batch; ++b) {
+    const int len = cu[b + 1] - cu[b];
+    if (len < 0 || nv[b] < 0 || nv[b] > len) return NSA_ERR_INVALID_ARG;
+    if (nsel_of(nv[b], params->sel_block) > 8192) return NSA_ERR_UNSUPPORTED;
+  }
+  return NSA_OK;
+}
+
+nsa_params_t varlen_sequence(const nsa_params_t* params, const int32_t* cu, const int32_t* nv, int b) {
+  nsa_params_t pb = *params;
+  pb.n_tokens = cu[b + 1] - cu[b];
+  pb.n_video = nv[b];
+  return pb;
+}
+
 }  // namespace
 
 extern "C" {
@@ -510,6 +530,56 @@ int nsa_prefill(const void* q, const void* k, const void* v, const float* gates,
   stage_begin(st);
   if (params->head_dim == 64) return prefill_impl<64>(params, q, k, v, gates, out, out_sel_idx, ws, st);
   return prefill_impl<128>(params, q, k, v, gates, out, out_sel_idx, ws, st);
+}
+
+size_t nsa_prefill_varlen_workspace_size(const nsa_params_t* params, const int32_t* cu_seqlens,
+                                         const int32_t* n_video, int batch) {
+  if (check_varlen(params, cu_seqlens, n_video, batch) != NSA_OK) return 0;
+  size_t most = 0;
+  for (int b = 0; b < batch; ++b) {
+    const nsa_params_t pb = varlen_sequence(params, cu_seqlens, n_video, b);
+    const size_t need = prefill_layout(&pb).total;
+    if (need > most) most = need;
+  }
+  return most;
+}
+
+int nsa_prefill_varlen(const void* q, const void* k, const void* v, const float* gates, const int32_t* cu_seqlens,
+                       const int32_t* n_video, int batch, const nsa_params_t* params, void* out,
+                       int32_t* out_sel_idx, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_varlen(params, cu_seqlens, n_video, batch);
+  if (rc != NSA_OK) return rc;
+  long long video_rows = 0;
+  for (int b = 0; b < batch; ++b) video_rows += n_video[b];
+  if (!q || !k || !v || !out || !workspace || (!gates && video_rows > 0)) return NSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (gates && !aligned16(gates)) ||
+      (out_sel_idx && !aligned16(out_sel_idx)) || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+    return NSA_ERR_INVALID_ARG;
+  if (workspace_bytes < nsa_prefill_varlen_workspace_size(params, cu_seqlens, n_video, batch))
+    return NSA_ERR_WORKSPACE_TOO_SMALL;
+  if ((rc = check_device()) != NSA_OK) return rc;
+  auto* ws = static_cast<uint8_t*>(workspace);
+  auto st = static_cast<cudaStream_t>(stream);
+  const size_t hq = params->num_q_heads, hkv = params->num_kv_heads, d = params->head_dim;
+  const size_t out_elem = params->out_dtype == NSA_OUT_F32 ? 4 : 2;
+  stage_begin(st);
+  long long sel_row = 0;  // video rows of the earlier sequences
+  for (int b = 0; b < batch; ++b) {
+    const nsa_params_t pb = varlen_sequence(params, cu_seqlens, n_video, b);
+    if (pb.n_tokens == 0) continue;
+    const size_t t0 = static_cast<size_t>(cu_seqlens[b]);
+    const auto* qb = static_cast<const uint8_t*>(q) + t0 * hq * d * 2;
+    const auto* kb = static_cast<const uint8_t*>(k) + t0 * hkv * d * 2;
+    const auto* vb = static_cast<const uint8_t*>(v) + t0 * hkv * d * 2;
+    const float* gb = gates ? gates + t0 * hq * 3 : nullptr;
+    auto* ob = static_cast<uint8_t*>(out) + t0 * hq * d * out_elem;
+    int32_t* sb = out_sel_idx ? out_sel_idx + static_cast<size_t>(sel_row) * hkv * params->top_n : nullptr;
+    rc = params->head_dim == 64 ? prefill_impl<64>(&pb, qb, kb, vb, gb, ob, sb, ws, st)
+                                : prefill_impl<128>(&pb, qb, kb, vb, gb, ob, sb, ws, st);
+    if (rc != NSA_OK) return rc;
+    sel_row += pb.n_video;
+  }
+  return NSA_OK;
 }
 
 int nsa_decode(const void* q, const void* kcache, const void* vcache, const void* kcmp, const void* vcmp,

@@ -29,6 +29,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnsa_b200
 EXPORTED = (
     "nsa_prefill", "nsa_decode", "nsa_compress", "nsa_workspace_size", "nsa_prefill_workspace_layout",
     "nsa_error_string", "nsa_get_device_error", "nsa_version", "nsa_profile_stages", "nsa_decode_noalloc",
+    "nsa_prefill_varlen", "nsa_prefill_varlen_workspace_size",
 )
 
 
@@ -75,6 +76,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     PP = ctypes.POINTER(NsaParams)
     lib.nsa_prefill.argtypes = [P, P, P, P, PP, P, P, P, S, P]
     lib.nsa_prefill.restype = I
+    I32P = ctypes.POINTER(ctypes.c_int32)
+    lib.nsa_prefill_varlen.argtypes = [P, P, P, P, I32P, I32P, I, PP, P, P, P, S, P]
+    lib.nsa_prefill_varlen.restype = I
+    lib.nsa_prefill_varlen_workspace_size.argtypes = [PP, I32P, I32P, I]
+    lib.nsa_prefill_varlen_workspace_size.restype = S
     lib.nsa_decode.argtypes = [P, P, P, P, P, P, P, PP, P, P, P, S, P]
     lib.nsa_decode.restype = I
     lib.nsa_decode_noalloc.argtypes = [P, P, P, P, P, P, P, PP, P, P, P]
@@ -127,6 +133,26 @@ def nsa_prefill(q, k, v, gates, params: NsaParams, out, out_sel_idx, workspace, 
                 stream=None) -> int:
     return load_library().nsa_prefill(_addr(q), _addr(k), _addr(v), _addr(gates), ctypes.byref(params), _addr(out),
                                       _addr(out_sel_idx), _addr(workspace), workspace_bytes, _stream(stream))
+
+
+def _host_i32(values):
+    """A host int32 array (ctypes) from a sequence of ints."""
+    vals = [int(x) for x in values]
+    return (ctypes.c_int32 * len(vals))(*vals)
+
+
+def nsa_prefill_varlen(q, k, v, gates, cu_seqlens, n_video, params: NsaParams, out, out_sel_idx, workspace,
+                       workspace_bytes: int, stream=None) -> int:
+    """Packed batch prefill; cu_seqlens ([B+1]) and n_video ([B]) are host integer sequences."""
+    cu, nv = _host_i32(cu_seqlens), _host_i32(n_video)
+    return load_library().nsa_prefill_varlen(_addr(q), _addr(k), _addr(v), _addr(gates), cu, nv, len(nv),
+                                             ctypes.byref(params), _addr(out), _addr(out_sel_idx),
+                                             _addr(workspace), workspace_bytes, _stream(stream))
+
+
+def nsa_prefill_varlen_workspace_size(params: NsaParams, cu_seqlens, n_video) -> int:
+    cu, nv = _host_i32(cu_seqlens), _host_i32(n_video)
+    return load_library().nsa_prefill_varlen_workspace_size(ctypes.byref(params), cu, nv, len(nv))
 
 
 def nsa_decode(q, kcache, vcache, kcmp, vcmp, seq_lens, gates, params: NsaParams, out, out_sel_idx, workspace,

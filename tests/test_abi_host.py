@@ -103,3 +103,34 @@ def test_missing_library_fails_loudly(tmp_path):
             nsa.load_library(str(tmp_path / "absent.so"))
         finally:
             nsa._lib = nsa._lib_saved
+
+
+@pytest.mark.parametrize("cu,nv,code", [
+    ([0, 100, 4096], [100, 3000], nsa.NSA_OK),              # well formed (stops at the device check)
+    ([1, 100, 4096], [99, 100], nsa.NSA_ERR_INVALID_ARG),   # does not start at 0
+    ([0, 200, 100, 4096], [10, 0, 10], nsa.NSA_ERR_INVALID_ARG),  # decreasing
+    ([0, 100, 4000], [100, 100], nsa.NSA_ERR_INVALID_ARG),  # does not end at n_tokens
+    ([0, 100, 4096], [101, 100], nsa.NSA_ERR_INVALID_ARG),  # video prefix longer than its sequence
+    ([0, 100, 4096], [-1, 100], nsa.NSA_ERR_INVALID_ARG),
+])
+def test_prefill_varlen_validation(cu, nv, code):
+    p = _p()
+    f = 1 << 20
+    rc = nsa.nsa_prefill_varlen(f, f, f, f, cu, nv, p, f, None, f, 1 << 40, None)
+    if code == nsa.NSA_OK:
+        assert rc not in (nsa.NSA_ERR_INVALID_ARG, nsa.NSA_ERR_WORKSPACE_TOO_SMALL)  # only the device check fails here
+        assert nsa.nsa_prefill_varlen_workspace_size(p, cu, nv) > 0
+    else:
+        assert rc == code
+        assert nsa.nsa_prefill_varlen_workspace_size(p, cu, nv) == 0
+
+
+def test_prefill_varlen_workspace_is_the_largest_sequence():
+    p = _p(n_tokens=5000)
+    cu, nv = [0, 700, 700, 2200, 5000], [600, 0, 1500, 2800]
+    need = nsa.nsa_prefill_varlen_workspace_size(p, cu, nv)
+    single = max(nsa.nsa_workspace_size(_p(n_tokens=cu[b + 1] - cu[b], n_video=nv[b]), 0)
+                 for b in range(4) if cu[b + 1] > cu[b])
+    assert need == single
+    f = 1 << 20
+    assert nsa.nsa_prefill_varlen(f, f, f, f, cu, nv, p, f, None, f, need - 1, None) == nsa.NSA_ERR_WORKSPACE_TOO_SMALL

@@ -180,3 +180,40 @@ def test_device_errors_are_reported_not_raised():
     bad = nsa.make_params(256, 256, 4, 1, 96, top_n=4, window=64)
     assert nsa.nsa_prefill(q, k, v, g, bad, out, None, ws, ws.numel()) == nsa.NSA_ERR_UNSUPPORTED
     assert nsa.nsa_get_device_error(clear=True) == 0
+
+
+def test_prefill_varlen_packed_batch():
+    """A packed batch (hybrid, empty, all-video, shorter-than-a-block and ragged sequences)
+    equals nsa_prefill on each sequence alone, bit for bit; the single-sequence results are
+    in turn checked against the oracle on every row."""
+    base = scaled(WORKLOADS["qwen36k_hybrid"], n_tokens=700, n_video=600)
+    lens, nvs = [700, 0, 1500, 33, 257], [600, 0, 1500, 33, 200]
+    parts = []
+    for b, (n, nv) in enumerate(zip(lens, nvs)):
+        w = scaled(base, n_tokens=max(n, 1), n_video=min(nv, max(n, 1)))
+        parts.append(prefill_inputs(w, seed=20 + b, device=DEV) if n > 0 else None)
+    cat = lambda i: torch.cat([pp[i] for pp in parts if pp is not None], dim=0)
+    q, k, v, g = cat(0), cat(1), cat(2), cat(3)
+    cu = np.concatenate([[0], np.cumsum(lens)]).tolist()
+    p = nsa.make_params(cu[-1], 0, base.hq, base.hkv, base.d, base.cmp_len, base.cmp_stride, base.sel_len,
+                        base.top_n, base.window, out_dtype=nsa.NSA_OUT_F32)
+    need = nsa.nsa_prefill_varlen_workspace_size(p, cu, nvs)
+    ws = torch.empty(need, dtype=torch.uint8, device=DEV)
+    out = torch.empty((cu[-1], base.hq, base.d), dtype=torch.float32, device=DEV)
+    sel = torch.full((sum(nvs), base.hkv, base.top_n), -7, dtype=torch.int32, device=DEV)
+    rc = nsa.nsa_prefill_varlen(q, k, v, g, cu, nvs, p, out, sel, ws, need)
+    assert rc == nsa.NSA_OK, nsa.nsa_error_string(rc)
+    torch.cuda.synchronize()
+    assert nsa.nsa_get_device_error(clear=True) == 0
+    srow = 0
+    for b, (n, nv) in enumerate(zip(lens, nvs)):
+        if n == 0:
+            continue
+        w = scaled(base, n_tokens=n, n_video=nv)
+        qb, kb, vb, gb = (t[cu[b]: cu[b + 1]].contiguous() for t in (q, k, v, g))
+        o1, s1, ws1, lay1 = run_prefill(w, qb, kb, vb, gb)
+        assert torch.equal(out[cu[b]: cu[b + 1]], o1), f"sequence {b}: out differs from the single call"
+        assert torch.equal(sel[srow: srow + nv], s1), f"sequence {b}: selection differs from the single call"
+        if b in (0, 3, 4):
+            compare_prefill_rows(w, qb, kb, vb, gb, np.arange(n), o1, s1, ws1, lay1)
+        srow += nv
