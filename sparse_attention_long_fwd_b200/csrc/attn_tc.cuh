@@ -61,11 +61,17 @@ struct AttnArgs {
   int out_f32;
 };
 
-constexpr int kSoftmaxWG = 4;                        // softmax warpgroups sharing each S tile
-constexpr int kSoftmaxThreads = 128 * kSoftmaxWG;
-constexpr int kAttnThreads = 64 + kSoftmaxThreads;    // producer warp, MMA warp, softmax warps
-constexpr int kColsPerWG = 128 / kSoftmaxWG;          // key columns (and output columns / D*128) per warpgroup
-constexpr int kBinsPerWG = kColsPerWG / 4;            // selection blocks per warpgroup per tile
+// Softmax warpgroups sharing each S tile, by mode: the compressed mode (two exponentials and
+// the block scores per element) keeps four for latency hiding; the window and dense modes
+// run two, each with twice the columns, so per-tile fixed costs weigh half as much.
+template <int MODE>
+struct AttnCfg {
+  static constexpr int kWG = MODE == 0 ? 4 : 2;
+  static constexpr int kThreads = 64 + 128 * kWG;  // producer warp, MMA warp, softmax warps
+  static constexpr int kCols = 128 / kWG;           // key columns per warpgroup per tile
+  static constexpr int kBins = kCols / 4;           // selection blocks per warpgroup per tile
+};
+constexpr int kMaxSoftmaxWG = 4;
 constexpr int kBN = 128;      // keys per tile
 
 template <int D>
@@ -77,7 +83,7 @@ struct AttnSmem {
   static constexpr int kSlots = D == 128 ? 5 : 8;
   alignas(1024) uint8_t q[kChunks][kTileBytes];
   alignas(1024) uint8_t slot[kSlots][kChunks][kTileBytes];
-  float lse_x[kSoftmaxWG][128][2];  // per warpgroup: (scaled max, sum) of the row's columns
+  float lse_x[kMaxSoftmaxWG][128][2];  // per warpgroup: (scaled max, sum) of the row's columns
   uint64_t q_full, q_tmem;
   uint64_t full[kSlots], empty[kSlots];
   uint64_t s_full[2], s_free[2];
@@ -138,11 +144,15 @@ __device__ __forceinline__ void group_reduce_scatter(float (&bin)[NB], int lane)
 }
 
 template <int D, int MODE>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
     attn_tile_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap vmap, const AttnArgs args) {
   using Smem = AttnSmem<D>;
   constexpr int kChunks = Smem::kChunks;
+  constexpr int kSoftmaxWG = AttnCfg<MODE>::kWG;
+  constexpr int kSoftmaxThreads = 128 * kSoftmaxWG;
+  constexpr int kColsPerWG = AttnCfg<MODE>::kCols;
+  constexpr int kBinsPerWG = AttnCfg<MODE>::kBins;
   constexpr uint32_t kTmemCols = 512;
   constexpr uint32_t kColO = 256;  // S buffers at columns 0 and 128, O at 256
   constexpr uint32_t kColP = 384;  // P (bf16 pairs, 64 columns)
@@ -254,11 +264,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_fence_after();
         // A = Q from TMEM (dims 16k .. 16k+15 in columns kColQ + 8k ..), B = K from smem:
         // the operand read from shared memory per MMA halves
+        // descriptors advance by constant offsets (start address field in 16-byte units):
+        // the issuing thread shares its scheduler with four softmax warps, so every
+        // instruction it saves shortens the MMA issue
+        const uint64_t kdesc = sdesc_sw128(smem_u32(sm.slot[x][0]), 16, 1024);
+        const uint32_t sbuf = tmem + b * kBN, qcol = tmem + kColQ;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const int c = k >> 2, kk = k & 3;
-          const uint64_t bd = sdesc_sw128(smem_u32(sm.slot[x][c]) + kk * 32, 16, 1024);
-          umma_bf16_ts(tmem + b * kBN, tmem + kColQ + k * 8, bd, idS, k > 0 ? 1u : 0u);
+          const uint64_t bd = kdesc + static_cast<uint64_t>((c * Smem::kTileBytes + kk * 32) >> 4);
+          umma_bf16_ts(sbuf, qcol + k * 8, bd, idS, k > 0 ? 1u : 0u);
         }
         umma_commit(&sm.s_full[b]);
         umma_commit(&sm.empty[x]);  // the K tile is no longer needed
@@ -281,12 +296,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             break;
           }
           tc_fence_after();
+          const uint64_t vdesc = sdesc_sw128(smem_u32(sm.slot[x][0]), Smem::kTileBytes, 1024);
+          const uint32_t ocol = tmem + kColO, pcol = tmem + kColP;
 #pragma unroll
-          for (int k = 0; k < kBN / 16; ++k) {
-            const uint32_t a_tmem = tmem + kColP + k * 8;  // keys 16k .. 16k+15
-            const uint64_t bd = sdesc_sw128(smem_u32(sm.slot[x][0]) + k * 2048, Smem::kTileBytes, 1024);
-            umma_bf16_ts(tmem + kColO, a_tmem, bd, idO, (kt2 > 0 || k > 0) ? 1u : 0u);
-          }
+          for (int k = 0; k < kBN / 16; ++k)  // keys 16k .. 16k+15 (P columns kColP + 8k ..)
+            umma_bf16_ts(ocol, pcol + k * 8, vdesc + static_cast<uint64_t>(k * (2048 >> 4)), idO,
+                         (kt2 > 0 || k > 0) ? 1u : 0u);
           umma_commit(&sm.p_free);   // this P.V (and its reads of P from TMEM) is done
           umma_commit(&sm.empty[x]);  // the V tile is no longer needed
         }
@@ -340,7 +355,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (nkt > 0) {
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_full, 0, abort_flag));
       if (ok) {
-        constexpr int kDimsPerWG = D / kSoftmaxWG;  // 32 (D=128) or 16 (D=64)
+        constexpr int kDimsPerWG = D / kSoftmaxWG;  // 64 (D=128) or 32 (D=64)
         uint32_t qv[kDimsPerWG / 2];
 #pragma unroll
         for (int i = 0; i < kDimsPerWG / 8; ++i) {
@@ -353,10 +368,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           qv[4 * i + 3] = w4.w;
         }
         __syncwarp();
-        if constexpr (kDimsPerWG / 2 == 16) {
-          tmem_st16(trow + kColQ + wg * 16, qv);
+        if constexpr (kDimsPerWG / 2 >= 16) {
+#pragma unroll
+          for (int h = 0; h < kDimsPerWG / 32; ++h)
+            tmem_st16(trow + kColQ + wg * (kDimsPerWG / 2) + 16 * h, *reinterpret_cast<const uint32_t(*)[16]>(&qv[16 * h]));
         } else {
-          tmem_st8(trow + kColQ + wg * 8, qv);
+          tmem_st8(trow + kColQ + wg * 8, *reinterpret_cast<const uint32_t(*)[8]>(&qv[0]));
         }
         tmem_wait_st();
         tc_fence_before();
@@ -390,10 +407,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           s[i] = (kidx >= rb && kidx < re) ? s[i] : -INFINITY;
         }
       }
-      static_assert(kColsPerWG == 32, "the max tree below covers 32 columns");
+      static_assert(kColsPerWG % 16 == 0 && kColsPerWG >= 32, "max tree: 8 chains over 16-column steps");
       float mx[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) mx[c] = fmaxf(fmax3f(s[c], s[c + 8], s[c + 16]), s[c + 24]);
+      for (int c = 0; c < 8; ++c) mx[c] = fmaxf(s[c], s[c + 8]);
+#pragma unroll
+      for (int i = 16; i < kColsPerWG; i += 16)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) mx[c] = fmax3f(mx[c], s[i + c], s[i + 8 + c]);
       const float cmax = fmax3f(fmax3f(mx[0], mx[1], mx[2]), fmax3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
       const float mnew = fmaxf(m, cmax);
       if (MODE != kModeCmp) {
@@ -517,14 +538,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           bin[u] = (u == 0 ? half_in : 0.5f * s[4 * u - 1]) + s[4 * u] + s[4 * u + 1] + s[4 * u + 2] + half_last;
         }
       }
-      // P row r, keys col0 .. col0+31 -> 16 packed bf16 pairs in TMEM columns kColP + col0/2 ..
-      // (one P buffer: P(k) is stored only after the P.V of tile k-1 has finished).
-      static_assert(kColsPerWG == 32, "P placement assumes 32 key columns per warpgroup");
-      {
+      // P row r, keys col0 .. col0+kColsPerWG-1 -> packed bf16 pairs in TMEM columns
+      // kColP + col0/2 .. (one P buffer: P(k) is stored only after the P.V of tile k-1 has
+      // finished).
+      static_assert(kColsPerWG % 32 == 0, "P is stored 16 columns (32 keys) at a time");
+#pragma unroll
+      for (int h = 0; h < kColsPerWG / 32; ++h) {
         uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(s[2 * i], s[2 * i + 1]);
-        tmem_st16(trow + kColP + col0 / 2, pk);
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(s[32 * h + 2 * i], s[32 * h + 2 * i + 1]);
+        tmem_st16(trow + kColP + col0 / 2 + 16 * h, pk);
       }
       tmem_wait_st();
       tc_fence_before();

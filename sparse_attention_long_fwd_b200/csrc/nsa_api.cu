@@ -226,7 +226,7 @@ int launch_attn(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap&
   const size_t smem = sizeof(nsa::AttnSmem<D>) + 1024;
   auto kern = nsa::attn_tile_kernel<D, MODE>;
   if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
-  kern<<<dim3(a.n_tiles, a.hkv), nsa::kAttnThreads, smem, st>>>(qm, km, vm, a);
+  kern<<<dim3(a.n_tiles, a.hkv), nsa::AttnCfg<MODE>::kThreads, smem, st>>>(qm, km, vm, a);
   return launch_status(MODE == nsa::kModeCmp ? "attn_cmp" : MODE == nsa::kModeWin ? "attn_win" : "attn_dense", st);
 }
 
