@@ -124,21 +124,22 @@ __device__ __forceinline__ int ncmp_visible(int t, int l, int s) { return (t + 1
 // ends with NB/GP group sums, bin[0 .. NB/GP) = entries [(l%GP)*NB/GP, ...). With GP > NB
 // the halving stops at one entry and the remaining stages add; lane l then holds entry
 // (l%GP) / (GP/NB), shared with the GP/NB - 1 lanes next to it.
-template <int GP, int NB>
+template <int GP, int NB, int O = GP / 2, int N = NB>
 __device__ __forceinline__ void group_reduce_scatter(float (&bin)[NB], int lane) {
+  // one halving stage per lane bit O (compile-time recursion: every bin index is static)
+  if constexpr (O >= 1) {
+    if constexpr (N > 1) {
+      const bool upper = (lane & O) != 0;
 #pragma unroll
-  for (int o = GP / 2, n = NB; o >= 1; o >>= 1) {
-    if (n > 1) {
-      const bool upper = (lane & o) != 0;
-#pragma unroll
-      for (int i = 0; i < n / 2; ++i) {
-        const float send = upper ? bin[i] : bin[i + n / 2];
-        const float keep = upper ? bin[i + n / 2] : bin[i];
-        bin[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      for (int i = 0; i < N / 2; ++i) {
+        const float send = upper ? bin[i] : bin[i + N / 2];
+        const float keep = upper ? bin[i + N / 2] : bin[i];
+        bin[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
       }
-      n >>= 1;
+      group_reduce_scatter<GP, NB, O / 2, N / 2>(bin, lane);
     } else {
-      bin[0] += __shfl_xor_sync(0xffffffffu, bin[0], o);
+      bin[0] += __shfl_xor_sync(0xffffffffu, bin[0], O);
+      group_reduce_scatter<GP, NB, O / 2, N>(bin, lane);
     }
   }
 }
