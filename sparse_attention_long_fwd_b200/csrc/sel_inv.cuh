@@ -46,14 +46,24 @@ struct SelInvArgs {
   float* o_sel;                 // [nv][hq][D]
 };
 
+// Block 0 is kept by every token, so its buckets take one entry per token of their group:
+// those entries are counted (and, in the scatter, placed) per CTA in shared memory and
+// added to the global counters once per CTA, instead of by one global atomic each.
 __global__ void __launch_bounds__(256) sel_count_kernel(const SelInvArgs a) {
+  __shared__ int zero_cnt[16];
+  if (threadIdx.x < 16) zero_cnt[threadIdx.x] = 0;
+  __syncthreads();
   const long long n = static_cast<long long>(a.nv) * a.hkv * a.top_n;
   for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
        e += static_cast<long long>(gridDim.x) * blockDim.x) {
     const int j = a.sel_idx[e];
     const int g = static_cast<int>((e / a.top_n) % a.hkv);
-    if (j >= 0 && j < a.nsel) atomicAdd(&a.cnt[g * a.nsel + j], 1);
+    if (j == 0 && g < 16) atomicAdd(&zero_cnt[g], 1);
+    else if (j >= 0 && j < a.nsel) atomicAdd(&a.cnt[g * a.nsel + j], 1);
   }
+  __syncthreads();
+  if (threadIdx.x < min(a.hkv, 16) && zero_cnt[threadIdx.x] > 0)
+    atomicAdd(&a.cnt[threadIdx.x * a.nsel], zero_cnt[threadIdx.x]);
 }
 
 // One CTA of 1024 threads scans hkv*nsel counters (<= 16 * 8192).
@@ -121,19 +131,35 @@ __global__ void __launch_bounds__(1024) sel_scan_kernel(const SelInvArgs a) {
 }
 
 __global__ void __launch_bounds__(256) sel_scatter_kernel(const SelInvArgs a) {
+  __shared__ int zero_cnt[16], zero_base[16];
   const long long n = static_cast<long long>(a.nv) * a.hkv * a.top_n;
-  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
-       e += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int j = a.sel_idx[e];
-    if (j < 0 || j >= a.nsel) continue;
+  // rounds of blockDim.x consecutive entries; every thread takes part in every round
+  for (long long base = static_cast<long long>(blockIdx.x) * blockDim.x; base < n;
+       base += static_cast<long long>(gridDim.x) * blockDim.x) {
+    if (threadIdx.x < 16) zero_cnt[threadIdx.x] = 0;
+    __syncthreads();
+    const long long e = base + threadIdx.x;
+    const int j = e < n ? a.sel_idx[e] : -1;
+    const bool valid = j >= 0 && j < a.nsel;
     const int slot = static_cast<int>(e % a.top_n);
     const long long tg = e / a.top_n;
     const int g = static_cast<int>(tg % a.hkv);
     const int t = static_cast<int>(tg / a.hkv);
-    const int key = g * a.nsel + j;
-    const int local = atomicAdd(&a.cursor[key], 1);
-    a.list[a.ent_off[key] + local] = t * 64 + slot;
-    a.row_of[e] = (a.tile_off[key] + local / a.TT) * 128 + (local % a.TT) * a.Gp;
+    const int key = g * a.nsel + (valid ? j : 0);
+    const bool agg = valid && j == 0 && g < 16;  // groups past 16 use the global counter directly
+    int local = 0;
+    if (agg) local = atomicAdd(&zero_cnt[g], 1);
+    else if (valid) local = atomicAdd(&a.cursor[key], 1);
+    __syncthreads();
+    if (threadIdx.x < min(a.hkv, 16) && zero_cnt[threadIdx.x] > 0)
+      zero_base[threadIdx.x] = atomicAdd(&a.cursor[threadIdx.x * a.nsel], zero_cnt[threadIdx.x]);
+    __syncthreads();
+    if (valid) {
+      if (agg) local += zero_base[g];
+      a.list[a.ent_off[key] + local] = t * 64 + slot;
+      a.row_of[e] = (a.tile_off[key] + local / a.TT) * 128 + (local % a.TT) * a.Gp;
+    }
+    __syncthreads();
   }
 }
 
