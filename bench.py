@@ -46,7 +46,7 @@ PREFILL_KERNELS = 9
 # DRAM bytes per launch of a stage's kernel on the 128K workload, from one ncu capture of the
 # current kernel version (profiles/dram_traffic_v128k.md); an entry is removed when its kernel
 # changes, and the roofline then reports traffic null.
-STAGE_TRAFFIC_V128K = {"cmp_attn_scores": 1109649920 + 4012024576}
+STAGE_TRAFFIC_V128K = {"cmp_attn_scores": 1118705408 + 4013818880}
 DECODE_STAGES = ["dec_cmp", "dec_select", "dec_branches", "dec_combine"]
 
 
