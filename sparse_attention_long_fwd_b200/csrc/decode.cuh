@@ -191,8 +191,13 @@ __global__ void __launch_bounds__(256) dec_select_kernel(const int32_t* __restri
   }
   __syncthreads();
   if (tid < 32) {
-    warp_topn(sc, bits, list, sc, jt, a.top_n, a.sel_idx + static_cast<size_t>(bg) * a.top_n,
-              out_sel_idx ? out_sel_idx + static_cast<size_t>(bg) * a.top_n : nullptr, tid);
+    int32_t* d = a.sel_idx + static_cast<size_t>(bg) * a.top_n;
+    int32_t* d2 = out_sel_idx ? out_sel_idx + static_cast<size_t>(bg) * a.top_n : nullptr;
+    if (a.top_n > 32 || jt >= 32 * 64) warp_topn(sc, bits, list, sc, jt, a.top_n, d, d2, tid);
+    else if (jt < 32 * 4) warp_topn_regs<4>(list, sc, jt, a.top_n, d, d2, tid);
+    else if (jt < 32 * 16) warp_topn_regs<16>(list, sc, jt, a.top_n, d, d2, tid);
+    else if (jt < 32 * 32) warp_topn_regs<32>(list, sc, jt, a.top_n, d, d2, tid);
+    else warp_topn_regs<64>(list, sc, jt, a.top_n, d, d2, tid);
   }
 }
 
