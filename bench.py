@@ -356,6 +356,10 @@ def run_b200(args, world, rank, local):
     result["gpu_launches_e2e"] = n_kernels * args.steps
     del qh, kh, vh, gh, outh, bufs
 
+    if not args.no_sweep and w.name == "v128k":
+        result["sweep"] = run_sweep(args, dev, q, k, v, g, flush, peak_t, world)
+        result["gpu_launches"] += PREFILL_KERNELS * args.steps * len(result["sweep"]["points"])
+
     if not args.no_decode:
         result["decode"] = run_decode(args, dev, peaks, peaks_src, flush, world)
         result["gpu_launches"] += 4 * args.steps
@@ -363,6 +367,45 @@ def run_b200(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, q, k, v, g, args.cpu_seconds)
     return result
+
+
+SWEEP_POINTS = ("sweep128k_n4_w256", "sweep128k_n16_w512", "sweep128k_n48_w1024")
+
+
+def run_sweep(args, dev, q, k, v, g, flush, peak_t, world):
+    """Attended-key budget sweep at 128K: the same inputs, each (n, w) point timed like the headline."""
+    ws = None
+    points = []
+    for name in SWEEP_POINTS:
+        w = WORKLOADS[name]
+        p = nsa.make_params(w.n_tokens, w.n_video, w.hq, w.hkv, w.d, w.cmp_len, w.cmp_stride, w.sel_len, w.top_n,
+                            w.window, out_dtype=nsa.NSA_OUT_BF16)
+        need = nsa.nsa_workspace_size(p, False)
+        if ws is None or ws.numel() < need:
+            ws = None
+            ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        out = torch.empty((w.n_tokens, w.hq, w.d), dtype=torch.bfloat16, device=dev)
+
+        def step(events, p=p, out=out):
+            rc = nsa.nsa_prefill(q, k, v, g, p, out, None, ws, ws.numel())
+            if rc != nsa.NSA_OK:
+                raise nsa.NsaError(rc, "nsa_prefill")
+
+        barrier(world)
+        step_ms, _ = timed_steps(step, args.steps, args.warmup, flush, 0)
+        assert nsa.nsa_get_device_error(clear=True) == 0, "device error word set during the sweep"
+        ms = max_over_ranks(sum(step_ms), world) / args.steps
+        c = prefill_counts(w)
+        flops = c["cmp_flops"] + c["sel_flops"] + c["win_flops"] + c["text_flops"]
+        tf = flops / (ms / 1e3) / 1e12
+        budget = sum(c["keys_per_head"].values()) / c["dense_causal_pairs"]
+        points.append({"workload": name, "top_n": w.top_n, "window": w.window, "ms_per_step": round(ms, 4),
+                       "value": round(w.n_video * world / (ms / 1e3), 1), "unit": "video tokens/s",
+                       "attended_tflops": round(tf, 2), "attended_frac_of_peak": round(tf / peak_t, 4),
+                       "attended_fraction_of_dense_pairs": round(budget, 4)})
+        del out
+    return {"points": points, "inputs": "the headline 128K tensors (same seed); only n and w change",
+            "l2": "flushed before every timed step", "steps": args.steps, "warmup": args.warmup}
 
 
 def run_decode(args, dev, peaks, peaks_src, flush, world):
@@ -484,6 +527,7 @@ def main():
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--workload", default="v128k", choices=[k for k, v in WORKLOADS.items() if not v.is_decode])
     ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the 128K (n, w) budget sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     args = ap.parse_args()

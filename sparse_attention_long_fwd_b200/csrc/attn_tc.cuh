@@ -29,10 +29,10 @@
 // next block while computing the current one, tiling against register pressure) are
 // met here by TMA tiles, an mbarrier ring and TMEM accumulators.
 //
-// Warp roles (576 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues the
-// MMAs (one elected lane), warps 2..17 (four warpgroups; each thread owns one TMEM lane /
-// MMA row and a quarter of the key columns) do the softmax, the score binning and the
-// epilogue. Every wait is bounded (sm100.cuh).
+// Warp roles: warp 0 issues TMA loads, warp 1 owns TMEM and issues the MMAs (one elected
+// lane), the softmax warpgroups (four in the compressed mode, two pairs taking turns on the
+// key tiles; two otherwise; each thread owns one TMEM lane / MMA row and 64 key columns of a
+// tile) do the softmax, the score binning and the epilogue. Every wait is bounded (sm100.cuh).
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -61,14 +61,18 @@ struct AttnArgs {
   int out_f32;
 };
 
-// Softmax warpgroups sharing each S tile, by mode: the compressed mode (two exponentials and
-// the block scores per element) keeps four for latency hiding; the window and dense modes
-// run two, each with twice the columns, so per-tile fixed costs weigh half as much.
+// Softmax warpgroups, by mode. Two warpgroups share each S tile, one per 64-column half.
+// The compressed mode (two exponentials and the block scores per element) runs two such
+// pairs that take turns on the key tiles (pair p owns S buffer p): while one pair is in its
+// exponentials the other loads, reduces and stores, so the exponential unit and the issue
+// slots are not left idle by warps that all reach the same step at once. The window and
+// dense modes run one pair.
 template <int MODE>
 struct AttnCfg {
-  static constexpr int kWG = MODE == 0 ? 4 : 2;
+  static constexpr int kPairs = MODE == 0 ? 2 : 1;  // warpgroup pairs taking turns on key tiles
+  static constexpr int kWG = 2 * kPairs;
   static constexpr int kThreads = 64 + 128 * kWG;  // producer warp, MMA warp, softmax warps
-  static constexpr int kCols = 128 / kWG;           // key columns per warpgroup per tile
+  static constexpr int kCols = 64;                  // key columns per warpgroup per tile
   static constexpr int kBins = kCols / 4;           // selection blocks per warpgroup per tile
 };
 constexpr int kMaxSoftmaxWG = 4;
@@ -84,6 +88,8 @@ struct AttnSmem {
   alignas(1024) uint8_t q[kChunks][kTileBytes];
   alignas(1024) uint8_t slot[kSlots][kChunks][kTileBytes];
   float lse_x[kMaxSoftmaxWG][128][2];  // per warpgroup: (scaled max, sum) of the row's columns
+  float carry[2][128];                 // (compressed, two pairs) half of a tile's last block, per row
+  uint64_t carry_full[2], carry_free[2];
   uint64_t q_full, q_tmem;
   uint64_t full[kSlots], empty[kSlots];
   uint64_t s_full[2], s_free[2];
@@ -116,6 +122,53 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
+}
+
+// Sum over 32 columns of 2^(s*sl2 - ms), in 8 independent chains.
+__device__ __forceinline__ float chunk_sum_ex2(const float (&s)[32], float sl2, float ms) {
+  float acc[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) acc[c] = ex2_approx(fmaf(s[c], sl2, -ms));
+#pragma unroll
+  for (int i = 8; i < 32; i += 8)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[c] += ex2_approx(fmaf(s[i + c], sl2, -ms));
+  return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+}
+
+// s[i] = 2^(s[i]*sl2 - off) for the columns kbase+i in [rb, re), 0 elsewhere.
+__device__ __forceinline__ void chunk_ex2(float (&s)[32], float sl2, float off, bool full, int kbase, int rb, int re) {
+  if (full) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) s[i] = ex2_approx(fmaf(s[i], sl2, -off));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int kidx = kbase + i;
+      s[i] = (kidx >= rb && kidx < re) ? ex2_approx(fmaf(s[i], sl2, -off)) : 0.f;
+    }
+  }
+}
+
+// TMA load sequence of a tile: phase 1 reads K(0 .. nkt-1); phase 2 reads K(0), K(1), V(0),
+// K(2), V(1), ..., K(nkt-1), V(nkt-2), V(nkt-1): each K tile comes one step ahead of the V
+// tile issued beside it, because the score MMA runs two jobs ahead of the P.V MMA.
+__device__ __forceinline__ int p2_k_pos(int x) { return x == 0 ? 0 : 2 * x - 1; }
+__device__ __forceinline__ int p2_v_pos(int x, int nkt) { return min(2 * x + 2, 2 * nkt - 1); }
+__device__ __forceinline__ void p2_item(int p, int nkt, bool& is_v, int& x) {
+  if (p == 0) {
+    is_v = false;
+    x = 0;
+  } else if (p == 2 * nkt - 1) {
+    is_v = true;
+    x = nkt - 1;
+  } else if (p & 1) {
+    is_v = false;
+    x = (p + 1) >> 1;
+  } else {
+    is_v = true;
+    x = (p >> 1) - 1;
+  }
 }
 
 __device__ __forceinline__ int ncmp_visible(int t, int l, int s) { return (t + 1 >= l) ? (t + 1 - l) / s + 1 : 0; }
@@ -151,6 +204,8 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
   using Smem = AttnSmem<D>;
   constexpr int kChunks = Smem::kChunks;
   constexpr int kSoftmaxWG = AttnCfg<MODE>::kWG;
+  constexpr int kPairs = AttnCfg<MODE>::kPairs;
+  constexpr int kTileWG = kSoftmaxWG / kPairs;  // warpgroups that share one S tile
   constexpr int kSoftmaxThreads = 128 * kSoftmaxWG;
   constexpr int kColsPerWG = AttnCfg<MODE>::kCols;
   constexpr int kBinsPerWG = AttnCfg<MODE>::kBins;
@@ -195,9 +250,11 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.s_full[b], 1);
-      mbar_init(&sm.s_free[b], 4 * kSoftmaxWG);
+      mbar_init(&sm.s_free[b], 4 * kTileWG);
+      mbar_init(&sm.carry_full[b], 4);
+      mbar_init(&sm.carry_free[b], 4);
     }
-    mbar_init(&sm.p_full, 4 * kSoftmaxWG);
+    mbar_init(&sm.p_full, 4 * kTileWG);
     mbar_init(&sm.p_free, 1);
     mbar_init(&sm.o_full, 1);
     mbar_init(&sm.drain, 1);
@@ -227,9 +284,9 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
-    // load L: L < nkt -> K tile L (phase 1); else x = L - nkt -> K (x even) or V (x odd) of
-    // tile x/2 (phase 2). Load L goes to slot L % kSlots once the MMA has released the
-    // load kSlots before it.
+    // load L: L < nkt -> K tile L (phase 1); else position L - nkt of the phase-2 sequence
+    // (p2_item). Load L goes to slot L % kSlots once the MMA has released the load kSlots
+    // before it.
     if (lane == 0 && nkt > 0) {
       tma_prefetch_desc(&qmap);
       tma_prefetch_desc(&kmap);
@@ -239,8 +296,9 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
       for (int L = 0; L < nloads; ++L) {
         const int x = L % kSlots;
         if (L >= kSlots && !mbar_wait(&sm.empty[x], ((L / kSlots) - 1) & 1, abort_flag)) break;
-        const bool is_v = L >= nkt && ((L - nkt) & 1);
-        const int kt = L < nkt ? L : (L - nkt) >> 1;
+        bool is_v = false;
+        int kt = L;
+        if (L >= nkt) p2_item(L - nkt, nkt, is_v, kt);
         const int kpos = kb + kt * kBN;
         mbar_arrive_expect_tx(&sm.full[x], Smem::kSlotBytes);
         for (int c = 0; c < kChunks; ++c)
@@ -251,72 +309,87 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0 && nkt > 0) {
+    // The whole warp runs the issue loop (waits, descriptor arithmetic) in lockstep and one
+    // elected lane issues each tcgen05 instruction: the operands stay warp-uniform, so the
+    // issuing warp needs few of the scheduler's slots, which it shares with four softmax warps.
+    if (nkt > 0) {
+      const bool leader = elect_one_sync();
       constexpr uint32_t idS = idesc_bf16_f32(128, kBN, false, false);
       constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);
-      bool ok = mbar_wait(&sm.q_tmem, 0, abort_flag);  // Q staged in TMEM by the softmax warps
-      auto wait_load = [&](int L) -> bool { return mbar_wait(&sm.full[L % kSlots], (L / kSlots) & 1, abort_flag); };
+      auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+      };
+      bool ok = wait_all(&sm.q_tmem, 0);  // Q staged in TMEM by the softmax warps
+      auto wait_load = [&](int L) -> bool { return wait_all(&sm.full[L % kSlots], (L / kSlots) & 1); };
       auto issue_s = [&](int job) -> bool {
-        const int L = job < nkt ? job : nkt + 2 * (job - nkt);
+        const int L = job < nkt ? job : nkt + p2_k_pos(job - nkt);
         const int x = L % kSlots;
         const int b = job & 1;
         if (!wait_load(L)) return false;
-        if (job >= 2 && !mbar_wait(&sm.s_free[b], ((job >> 1) - 1) & 1, abort_flag)) return false;
+        if (job >= 2 && !wait_all(&sm.s_free[b], ((job >> 1) - 1) & 1)) return false;
         tc_fence_after();
-        // A = Q from TMEM (dims 16k .. 16k+15 in columns kColQ + 8k ..), B = K from smem:
-        // the operand read from shared memory per MMA halves
-        // descriptors advance by constant offsets (start address field in 16-byte units):
-        // the issuing thread shares its scheduler with four softmax warps, so every
-        // instruction it saves shortens the MMA issue
+        // A = Q from TMEM (dims 16k .. 16k+15 in columns kColQ + 8k ..), B = K from smem;
+        // the B descriptor advances by constant offsets (start address field in 16-byte units)
         const uint64_t kdesc = sdesc_sw128(smem_u32(sm.slot[x][0]), 16, 1024);
         const uint32_t sbuf = tmem + b * kBN, qcol = tmem + kColQ;
+        if (leader) {
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const int c = k >> 2, kk = k & 3;
-          const uint64_t bd = kdesc + static_cast<uint64_t>((c * Smem::kTileBytes + kk * 32) >> 4);
-          umma_bf16_ts(sbuf, qcol + k * 8, bd, idS, k > 0 ? 1u : 0u);
+          for (int k = 0; k < D / 16; ++k) {
+            const int c = k >> 2, kk = k & 3;
+            const uint64_t bd = kdesc + static_cast<uint64_t>((c * Smem::kTileBytes + kk * 32) >> 4);
+            umma_bf16_ts(sbuf, qcol + k * 8, bd, idS, k > 0 ? 1u : 0u);
+          }
+          umma_commit(&sm.s_full[b]);
+          umma_commit(&sm.empty[x]);  // the K tile is no longer needed
         }
-        umma_commit(&sm.s_full[b]);
-        umma_commit(&sm.empty[x]);  // the K tile is no longer needed
+        __syncwarp();
         return true;
       };
+      // Score tiles run two jobs ahead: S(job + 2) waits only for its buffer, which the pair
+      // that read S(job) frees as soon as the scores are in registers, so it computes while
+      // that pair is still in its softmax; P.V(job) follows once P(job) is in TMEM.
       if (ok) ok = issue_s(0);
+      if (ok && njobs > 1) ok = issue_s(1);
       for (int job = 0; ok && job < njobs; ++job) {
-        // the next score tile goes to the tensor core before this tile's P.V, so it
-        // computes while the softmax warps turn this tile's scores into P
-        if (job + 1 < njobs && !issue_s(job + 1)) {
+        if (job + 2 < njobs && !issue_s(job + 2)) {
           ok = false;
           break;
         }
         if (job >= nkt) {
           const int kt2 = job - nkt;
-          const int L = nkt + 2 * kt2 + 1;  // V tile
+          const int L = nkt + p2_v_pos(kt2, nkt);  // V tile
           const int x = L % kSlots;
-          if (!wait_load(L) || !mbar_wait(&sm.p_full, kt2 & 1, abort_flag)) {
+          if (!wait_load(L) || !wait_all(&sm.p_full, kt2 & 1)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint64_t vdesc = sdesc_sw128(smem_u32(sm.slot[x][0]), Smem::kTileBytes, 1024);
           const uint32_t ocol = tmem + kColO, pcol = tmem + kColP;
+          if (leader) {
 #pragma unroll
-          for (int k = 0; k < kBN / 16; ++k)  // keys 16k .. 16k+15 (P columns kColP + 8k ..)
-            umma_bf16_ts(ocol, pcol + k * 8, vdesc + static_cast<uint64_t>(k * (2048 >> 4)), idO,
-                         (kt2 > 0 || k > 0) ? 1u : 0u);
-          umma_commit(&sm.p_free);   // this P.V (and its reads of P from TMEM) is done
-          umma_commit(&sm.empty[x]);  // the V tile is no longer needed
+            for (int k = 0; k < kBN / 16; ++k)  // keys 16k .. 16k+15 (P columns kColP + 8k ..)
+              umma_bf16_ts(ocol, pcol + k * 8, vdesc + static_cast<uint64_t>(k * (2048 >> 4)), idO,
+                           (kt2 > 0 || k > 0) ? 1u : 0u);
+            umma_commit(&sm.p_free);    // this P.V (and its reads of P from TMEM) is done
+            umma_commit(&sm.empty[x]);  // the V tile is no longer needed
+          }
+          __syncwarp();
         }
       }
-      if (ok) umma_commit(&sm.o_full);
+      if (ok && leader) umma_commit(&sm.o_full);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ softmax / epilogue
-    // kSoftmaxWG warpgroups share every S tile: warpgroup `wg` owns key columns
-    // [wg*kColsPerWG, (wg+1)*kColsPerWG) of each 128-key tile (and the same slice of the D
-    // output columns in the epilogue); its thread of TMEM lane r handles MMA row r.
+    // Warpgroup `wg` belongs to pair wg / kTileWG, which handles the MMA jobs (S tiles) of
+    // parity `pair` (S buffer `pair`); within the pair it owns key columns
+    // [half*64, half*64+64) of each 128-key tile. In the epilogue it owns D/kSoftmaxWG output
+    // columns. Its thread of TMEM lane r handles MMA row r.
     const int sw = warp - 2;                 // softmax warp
-    const int wg = sw >> 2;                  // column slice
+    const int wg = sw >> 2;                  // warpgroup
+    const int pair = wg / kTileWG;
+    const int half = wg % kTileWG;           // column slice within a tile
     const int q4 = warp & 3;                 // TMEM lane quadrant of this warp
     const int r = q4 * 32 + lane;            // MMA row
     const int Gp = args.Gp;
@@ -336,7 +409,7 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
       }
     }
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-    const int col0 = wg * kColsPerWG;
+    const int col0 = half * kColsPerWG;
     if (MODE == kModeWin && row_valid) {
       // the epilogue reads this row's o_cmp, o_sel and gates: start bringing them into L2
       const size_t orow = (static_cast<size_t>(t) * args.hq + h) * D + wg * (D / kSoftmaxWG);
@@ -384,54 +457,49 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
     }
     // ---- phase 1: log-sum-exp (base 2) of this row's column slice, combined below
     float m = -INFINITY, lsum = 0.f;         // m: running max of the raw (unscaled) scores
-    for (int kt = 0; kt < nkt && ok; ++kt) {
+    for (int kt = kPairs == 1 ? 0 : pair; kt < nkt && ok; kt += kPairs) {
       const int b = kt & 1;
       // tcgen05.ld is warp-collective: every wait result is made warp-uniform
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (kt >> 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       const int kbase = kb + kt * kBN + col0;
-      const bool full = kbase >= rb && kbase + kColsPerWG <= re;
-      float s[kColsPerWG];
-      __syncwarp();
+      // warp-uniform: the unmasked path only when every row of the warp sees the whole
+      // slice; rows without keys (head padding, past the end) follow the others, their
+      // probabilities being forced to 0 through lse2 = +inf
+      const bool full = __all_sync(0xffffffffu, !row_valid || (kbase >= rb && kbase + kColsPerWG <= re));
+      // 32 columns at a time (an online max across the chunks keeps one chunk in registers)
+      static_assert(kColsPerWG % 32 == 0, "phase 1 reads 32-column chunks");
 #pragma unroll
-      for (int c = 0; c < kColsPerWG / 32; ++c)
-        tmem_ld32(trow + b * kBN + col0 + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.s_free[b]);  // S is in registers: the buffer may be reused
-      if (!full) {
-#pragma unroll
-        for (int i = 0; i < kColsPerWG; ++i) {
-          const int kidx = kbase + i;
-          s[i] = (kidx >= rb && kidx < re) ? s[i] : -INFINITY;
+      for (int h = 0; h < kColsPerWG / 32; ++h) {
+        float s[32];
+        __syncwarp();
+        tmem_ld32(trow + b * kBN + col0 + 32 * h, s);
+        tmem_wait_ld();
+        if (h == kColsPerWG / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.s_free[b]);  // S is in registers: the buffer may be reused
         }
-      }
-      static_assert(kColsPerWG % 16 == 0 && kColsPerWG >= 32, "max tree: 8 chains over 16-column steps");
-      float mx[8];
+        if (!full) {
 #pragma unroll
-      for (int c = 0; c < 8; ++c) mx[c] = fmaxf(s[c], s[c + 8]);
+          for (int i = 0; i < 32; ++i) {
+            const int kidx = kbase + 32 * h + i;
+            s[i] = (kidx >= rb && kidx < re) ? s[i] : -INFINITY;
+          }
+        }
+        float mx[8];
 #pragma unroll
-      for (int i = 16; i < kColsPerWG; i += 16)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) mx[c] = fmax3f(mx[c], s[i + c], s[i + 8 + c]);
-      const float cmax = fmax3f(fmax3f(mx[0], mx[1], mx[2]), fmax3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-      const float mnew = fmaxf(m, cmax);
-      if (MODE != kModeCmp) {
-        m = mnew;  // the window and dense branches need only the row max here
-      } else if (mnew != -INFINITY) {
-        const float ms = mnew * sl2;
-        float acc[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[c] = ex2_approx(fmaf(s[c], sl2, -ms));
-#pragma unroll
-        for (int i = 8; i < kColsPerWG; i += 8)
-#pragma unroll
-          for (int c = 0; c < 8; ++c) acc[c] += ex2_approx(fmaf(s[i + c], sl2, -ms));
-        lsum = lsum * ex2_approx((m - mnew) * sl2) +
-               (((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7])));
-        m = mnew;
+        for (int c = 0; c < 8; ++c) mx[c] = fmax3f(fmaxf(s[c], s[c + 8]), s[c + 16], s[c + 24]);
+        const float cmax = fmax3f(fmax3f(mx[0], mx[1], mx[2]), fmax3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+        const float mnew = fmaxf(m, cmax);
+        if (MODE != kModeCmp) {
+          m = mnew;  // the window and dense branches need only the row max here
+        } else if (mnew != -INFINITY) {
+          const float ms = mnew * sl2;
+          lsum = lsum * ex2_approx((m - mnew) * sl2) + chunk_sum_ex2(s, sl2, ms);
+          m = mnew;
+        }
       }
     }
     sm.lse_x[wg][r][0] = (m == -INFINITY) ? -INFINITY : m * sl2;
@@ -449,11 +517,11 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
         for (int w = 0; w < kSoftmaxWG; ++w) L += sm.lse_x[w][r][1] * ex2_approx(sm.lse_x[w][r][0] - M);
       }
       if (MODE == kModeCmp) {
-        has_keys = L > 0.f;
+        has_keys = row_valid && L > 0.f;
         lse2 = has_keys ? M + __log2f(L) : INFINITY;
       } else {
         // P = exp2(S*scale*log2e - max) unnormalised; the row sum divides O at the end
-        has_keys = M != -INFINITY;
+        has_keys = row_valid && M != -INFINITY;
         lse2 = has_keys ? M : INFINITY;
       }
     }
@@ -462,122 +530,142 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
     // Block scores (kModeCmp): compressed block i covers tokens [16i, 16i+32) and selection
     // block j covers [64j, 64j+64), so block j takes all of compressed blocks 4j..4j+2 and
     // half of 4j-1 and 4j+3. A 128-key tile holds selection blocks kt2*32 .. kt2*32+31;
-    // this warpgroup's columns hold kBinsPerWG of them. The one compressed block that
-    // straddles the previous column slice is re-read from TMEM by this thread (column
-    // col0-1, or for warpgroup 0 the previous tile's column 127, kept from the previous
-    // iteration), so the slices never exchange data. The G heads of a token sit in Gp
-    // adjacent lanes; a shuffle reduce-scatter sums them.
-    float carry = 0.f;  // warpgroup 0: half of the previous tile's last compressed block
-    // (kModeCmp) after the head reduce-scatter, lane hh holds blocks [hh*bpl, (hh+1)*bpl) of
-    // its warpgroup's slice (Gp <= kBinsPerWG), or block hh/share shared with its neighbours
-    // (Gp > kBinsPerWG); these store invariants do not change from tile to tile
-    const int sc_bpl = Gp <= kBinsPerWG ? kBinsPerWG / Gp : 1;
-    const int sc_share = Gp <= kBinsPerWG ? 1 : Gp / kBinsPerWG;
+    // this warpgroup's columns hold kBinsPerWG of them. The compressed block that straddles
+    // the two column halves (column 63) is re-read from TMEM by the upper half. The one that
+    // straddles two tiles (column 127 of the previous tile, which the other pair handled)
+    // arrives through a shared-memory slot: the upper half of each tile leaves half of its
+    // column-127 probability there and the lower half of the next tile picks it up (slot
+    // kt2 & 1, guarded by carry_full / carry_free). The G heads of a token sit in Gp adjacent
+    // lanes; a shuffle reduce-scatter sums them.
+    float carry_last = 0.f;  // upper half, last tile: half of its last compressed block
+    // (kModeCmp) the scores are reduced over the heads per 32-column chunk (8 selection
+    // blocks): lane hh then holds blocks [hh*bpl, (hh+1)*bpl) of the chunk (Gp <= 8), or block
+    // hh/share shared with its neighbours (Gp > 8); these store invariants do not change from
+    // tile to tile
+    constexpr int kChunkBins = 8;  // selection blocks per 32-column chunk
+    const int sc_bpl = Gp <= kChunkBins ? kChunkBins / Gp : 1;
+    const int sc_share = Gp <= kChunkBins ? 1 : Gp / kChunkBins;
     const bool sc_store = MODE == kModeCmp && t < args.q_end && (hh % sc_share) == 0;
     const int sc_jt = t / args.sel_len;
-    const int sc_j0 = wg * kBinsPerWG + (hh / sc_share) * sc_bpl;
+    const int sc_j0 = half * kBinsPerWG + (hh / sc_share) * sc_bpl;
     float* const sc_dst = args.scores + (static_cast<size_t>(t) * args.hkv + g) * args.nsel;
-    for (int kt2 = 0; kt2 < nkt; ++kt2) {
+    // this pair's phase-2 jobs are those of parity `pair`: job nkt + kt2
+    for (int kt2 = kPairs == 1 ? 0 : ((pair + nkt) & 1); kt2 < nkt; kt2 += kPairs) {
       const int job = nkt + kt2;
       const int b = job & 1;
       if (ok) ok = mbar_wait(&sm.s_full[b], (job >> 1) & 1, abort_flag);
-      // P(kt2) is stored to TMEM only once the P.V MMA of the previous tile has finished:
-      // tcgen05.st into TMEM while a P.V that reads its A operand from TMEM was still running
-      // corrupted rows 0-31 of the output on B200 even while P was double-buffered in disjoint
-      // columns; with that wait in place one P buffer suffices.
-      if (ok && kt2 > 0) ok = mbar_wait(&sm.p_free, (kt2 - 1) & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
       const int kbase = kb + kt2 * kBN + col0;
-      const bool full = kbase >= rb && kbase + kColsPerWG <= re;
-      float bin[kBinsPerWG];
+      // warp-uniform: the unmasked path only when every row of the warp sees the whole
+      // slice; rows without keys (head padding, past the end) follow the others, their
+      // probabilities being forced to 0 through lse2 = +inf
+      const bool full = __all_sync(0xffffffffu, !row_valid || (kbase >= rb && kbase + kColsPerWG <= re));
       float half_in = 0.f;
-      float s[kColsPerWG];
-      uint32_t xv = 0;
-      const int xcol = wg > 0 ? col0 - 1 : 127;  // (kModeCmp) the straddling block's column
-      __syncwarp();
-#pragma unroll
-      for (int c = 0; c < kColsPerWG / 32; ++c)
-        tmem_ld32(trow + b * kBN + col0 + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
-      if (MODE == kModeCmp)
-        asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(xv) : "r"(trow + b * kBN + xcol));
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.s_free[b]);  // S is in registers: the buffer may be reused
-      if (MODE == kModeCmp) {
-        const int xk = kb + kt2 * kBN + xcol;
-        const float px = (xk >= rb && xk < re) ? ex2_approx(fmaf(__uint_as_float(xv), sl2, -lse2)) : 0.f;
-        if (wg > 0) {
-          half_in = 0.5f * px;
-        } else {
-          half_in = carry;
-          carry = 0.5f * px;
-        }
-      }
-      if (full) {
-#pragma unroll
-        for (int i = 0; i < kColsPerWG; ++i) s[i] = ex2_approx(fmaf(s[i], sl2, -lse2));
-      } else {
-#pragma unroll
-        for (int i = 0; i < kColsPerWG; ++i) {
-          const int kidx = kbase + i;
-          s[i] = (kidx >= rb && kidx < re) ? ex2_approx(fmaf(s[i], sl2, -lse2)) : 0.f;
-        }
-      }
-      if (MODE != kModeCmp) {
-        float ps[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int i = 0; i < kColsPerWG; ++i) ps[i & 3] += s[i];
-        psum += (ps[0] + ps[1]) + (ps[2] + ps[3]);
-      }
-      if (MODE == kModeCmp) {
-#pragma unroll
-        for (int u = 0; u < kBinsPerWG; ++u) {
-          const float half_last = 0.5f * s[4 * u + 3];
-          bin[u] = (u == 0 ? half_in : 0.5f * s[4 * u - 1]) + s[4 * u] + s[4 * u + 1] + s[4 * u + 2] + half_last;
-        }
-      }
-      // P row r, keys col0 .. col0+kColsPerWG-1 -> packed bf16 pairs in TMEM columns
-      // kColP + col0/2 .. (one P buffer: P(k) is stored only after the P.V of tile k-1 has
-      // finished).
+      // 32 columns at a time: read from TMEM, exponentials, then (kModeCmp) the chunk's 8
+      // block scores, then the chunk's P packed to bf16 pairs, so only one chunk is ever held
+      // in fp32
       static_assert(kColsPerWG % 32 == 0, "P is stored 16 columns (32 keys) at a time");
+      uint32_t pk[kColsPerWG / 2];
+      float prev_last = 0.f;  // (kModeCmp) p of the previous chunk's last column
 #pragma unroll
       for (int h = 0; h < kColsPerWG / 32; ++h) {
-        uint32_t pk[16];
+        float sc[32];
+        uint32_t xv = 0;
+        __syncwarp();
+        tmem_ld32(trow + b * kBN + col0 + 32 * h, sc);
+        if (MODE == kModeCmp && h == 0 && half > 0)
+          asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(xv) : "r"(trow + b * kBN + col0 - 1));
+        tmem_wait_ld();
+        if (h == kColsPerWG / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.s_free[b]);  // S is in registers: the buffer may be reused
+        }
+        if (MODE == kModeCmp && h == 0 && half > 0) {
+          const int xk = kb + kt2 * kBN + col0 - 1;
+          half_in = (xk >= rb && xk < re) ? 0.5f * ex2_approx(fmaf(__uint_as_float(xv), sl2, -lse2)) : 0.f;
+        }
+        chunk_ex2(sc, sl2, lse2, full, kbase + 32 * h, rb, re);
+        if (MODE != kModeCmp) {
+          float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(s[32 * h + 2 * i], s[32 * h + 2 * i + 1]);
-        tmem_st16(trow + kColP + col0 / 2 + 16 * h, pk);
+          for (int i = 0; i < 32; ++i) ps[i & 3] += sc[i];
+          psum += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+        }
+        if (MODE == kModeCmp) {
+          if (h == 0 && half == 0 && kt2 > 0) {
+            // half of the previous tile's column 127, left by the other pair
+            const int slot = (kt2 - 1) & 1;
+            if (ok) ok = mbar_wait(&sm.carry_full[slot], ((kt2 - 1) >> 1) & 1, abort_flag);
+            half_in = sm.carry[slot][r];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.carry_free[slot]);
+          }
+          if (h == kColsPerWG / 32 - 1 && half == kTileWG - 1) {
+            // hand half of column 127 to the next tile's lower half (the other pair)
+            const float c127 = 0.5f * sc[31];
+            if (kt2 + 1 < nkt) {
+              const int slot = kt2 & 1;
+              if (kt2 >= 2 && ok) ok = mbar_wait(&sm.carry_free[slot], ((kt2 >> 1) - 1) & 1, abort_flag);
+              sm.carry[slot][r] = c127;
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&sm.carry_full[slot]);
+            } else {
+              carry_last = c127;
+            }
+          }
+          float bin[kChunkBins];
+#pragma unroll
+          for (int u = 0; u < kChunkBins; ++u) {
+            const float left = u > 0 ? 0.5f * sc[4 * u - 1] : (h == 0 ? half_in : 0.5f * prev_last);
+            bin[u] = left + sc[4 * u] + sc[4 * u + 1] + sc[4 * u + 2] + 0.5f * sc[4 * u + 3];
+          }
+          prev_last = sc[31];
+          switch (Gp) {
+            case 2: group_reduce_scatter<2, kChunkBins>(bin, lane); break;
+            case 4: group_reduce_scatter<4, kChunkBins>(bin, lane); break;
+            case 8: group_reduce_scatter<8, kChunkBins>(bin, lane); break;
+            case 16: group_reduce_scatter<16, kChunkBins>(bin, lane); break;
+            default: break;
+          }
+          if (sc_store) {
+            const int j0 = kt2 * 32 + h * kChunkBins + sc_j0;
+            if (sc_bpl == 1) {
+              if (j0 <= sc_jt) sc_dst[j0] = bin[0];
+            } else {
+#pragma unroll
+              for (int i = 0; i < kChunkBins; ++i)
+                if (i < sc_bpl && j0 + i <= sc_jt) sc_dst[j0 + i] = bin[i];
+            }
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[16 * h + i] = pack_bf16x2(sc[2 * i], sc[2 * i + 1]);
       }
+      // P row r, keys col0 .. col0+kColsPerWG-1 -> packed bf16 pairs in TMEM columns
+      // kColP + col0/2 .. . P(kt2) is stored only once the P.V MMA of the previous tile has
+      // finished: tcgen05.st into TMEM while a P.V that reads its A operand from TMEM was
+      // still running corrupted rows 0-31 of the output on B200 even while P was
+      // double-buffered in disjoint columns; with that wait in place one P buffer suffices.
+      // The wait comes after the exponentials, which overlap the previous P.V.
+      if (ok && kt2 > 0) ok = mbar_wait(&sm.p_free, (kt2 - 1) & 1, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+#pragma unroll
+      for (int h = 0; h < kColsPerWG / 32; ++h)
+        tmem_st16(trow + kColP + col0 / 2 + 16 * h, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * h]));
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full);
-      if (MODE == kModeCmp) {
-        switch (Gp) {
-          case 2: group_reduce_scatter<2, kBinsPerWG>(bin, lane); break;
-          case 4: group_reduce_scatter<4, kBinsPerWG>(bin, lane); break;
-          case 8: group_reduce_scatter<8, kBinsPerWG>(bin, lane); break;
-          case 16: group_reduce_scatter<16, kBinsPerWG>(bin, lane); break;
-          default: break;
-        }
-        if (sc_store) {
-          const int j0 = kt2 * 32 + sc_j0;
-          if (sc_bpl == 1) {
-            if (j0 <= sc_jt) sc_dst[j0] = bin[0];
-          } else {
-#pragma unroll
-            for (int i = 0; i < kBinsPerWG; ++i)
-              if (i < sc_bpl && j0 + i <= sc_jt) sc_dst[j0 + i] = bin[i];
-          }
-        }
-      }
     }
-    if (MODE == kModeCmp && ok && wg == 0) {
-      // the carried half-block after the last tile lands in selection block nkt*32; when no
-      // key tile exists at all, that is block 0 with score 0
-      float c = carry;
+    if (MODE == kModeCmp && ok && wg == kSoftmaxWG - 1) {
+      // the half-block after the last tile lands in selection block nkt*32; the last
+      // phase-2 job (2*nkt - 1) is odd, so this warpgroup (upper half of pair 1) holds it.
+      // When no key tile exists at all, that is block 0 with score 0.
+      float c = carry_last;
 #pragma unroll
       for (int o = 1; o < 16; o <<= 1)
         if (o < Gp) c += __shfl_xor_sync(0xffffffffu, c, o);
@@ -683,10 +771,13 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
         }
       }
     }
-    if (warp == 1 && lane == 0 && nkt > 0) {
-      umma_commit(&sm.drain);
-      const long long t_start = clock64();
-      while (!mbar_test(&sm.drain, 0) && clock64() - t_start < kWaitCycles) {
+    if (warp == 1 && nkt > 0) {
+      // the commit tracks the MMAs of the lane that issued them: the same elected lane
+      if (elect_one_sync()) {
+        umma_commit(&sm.drain);
+        const long long t_start = clock64();
+        while (!mbar_test(&sm.drain, 0) && clock64() - t_start < kWaitCycles) {
+        }
       }
     }
     __syncwarp();
