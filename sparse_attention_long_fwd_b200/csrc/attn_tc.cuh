@@ -66,7 +66,8 @@ struct AttnArgs {
 // pairs that take turns on the key tiles (pair p owns S buffer p): while one pair is in its
 // exponentials the other loads, reduces and stores, so the exponential unit and the issue
 // slots are not left idle by warps that all reach the same step at once. The window and
-// dense modes run one pair.
+// dense modes (one exponential per element, a few tiles per item) run one pair, which
+// measured faster for them than two.
 template <int MODE>
 struct AttnCfg {
   static constexpr int kPairs = MODE == 0 ? 2 : 1;  // warpgroup pairs taking turns on key tiles
@@ -74,6 +75,7 @@ struct AttnCfg {
   static constexpr int kThreads = 64 + 128 * kWG;  // producer warp, MMA warp, softmax warps
   static constexpr int kCols = 64;                  // key columns per warpgroup per tile
   static constexpr int kBins = kCols / 4;           // selection blocks per warpgroup per tile
+  static constexpr bool kPersistent = MODE != 0;    // one CTA per SM looping over the items
 };
 constexpr int kMaxSoftmaxWG = 4;
 constexpr int kBN = 128;      // keys per tile
@@ -90,10 +92,10 @@ struct AttnSmem {
   float lse_x[kMaxSoftmaxWG][128][2];  // per warpgroup: (scaled max, sum) of the row's columns
   float carry[2][128];                 // (compressed, two pairs) half of a tile's last block, per row
   uint64_t carry_full[2], carry_free[2];
-  uint64_t q_full, q_tmem;
+  uint64_t q_full, q_tmem, q_empty, qcols_free;
   uint64_t full[kSlots], empty[kSlots];
   uint64_t s_full[2], s_free[2];
-  uint64_t p_full, p_free, o_full, drain;
+  uint64_t p_full, p_free[2], o_full, o_free, drain;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -213,6 +215,7 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
   constexpr uint32_t kColO = 256;  // S buffers at columns 0 and 128, O at 256
   constexpr uint32_t kColP = 384;  // P (bf16 pairs, 64 columns)
   constexpr uint32_t kColQ = 448;  // Q (bf16 pairs, D/2 columns): the A operand of every S MMA
+  constexpr int kSlots = Smem::kSlots;
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -220,30 +223,38 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int G = args.G, T = args.T;
-  const int g = blockIdx.y;
-  // heavy tiles (most keys) first for the causal modes
-  const int tile = (MODE == kModeWin) ? blockIdx.x : (args.n_tiles - 1 - blockIdx.x);
-  const int t0 = args.q_begin + tile * T;
-  const int t_last = min(t0 + T, args.q_end) - 1;
-  int kb, ke;
-  if (MODE == kModeCmp) {
-    kb = 0;
-    ke = ncmp_visible(t_last, args.cmp_len, args.cmp_stride);
-  } else if (MODE == kModeWin) {
-    kb = max(0, t0 - args.window + 1);
-    ke = t_last + 1;
-  } else {
-    kb = 0;
-    ke = t_last + 1;
-  }
-  const int nkt = (ke - kb + kBN - 1) / kBN;
-  const int njobs = 2 * nkt;   // MMA jobs: nkt score tiles (phase 1), then nkt score + P.V tiles
-  const int nloads = 3 * nkt;  // TMA loads: K tiles (phase 1), then K and V per tile (phase 2)
-  constexpr int kSlots = Smem::kSlots;
+  // Work items (query tile, KV group), heavy tiles (most keys) first for the causal modes.
+  // Window and dense: one CTA per SM, persistent, CTA c taking items c, c + gridDim.x, ...,
+  // so each item's start overlaps the previous item's epilogue (these items are short).
+  // Compressed: one item per CTA (its items are long, and the hardware's launch order then
+  // balances them); the loops below run once and compile as such.
+  constexpr bool kPersist = AttnCfg<MODE>::kPersistent;
+  const int n_items = args.n_tiles * args.hkv;
+  auto item_geo = [&](int item, int& g, int& t0, int& kb, int& nkt) {
+    const int rank = item / args.hkv;
+    g = item % args.hkv;
+    const int tile = (MODE == kModeWin) ? rank : (args.n_tiles - 1 - rank);
+    t0 = args.q_begin + tile * T;
+    const int t_last = min(t0 + T, args.q_end) - 1;
+    int ke;
+    if (MODE == kModeCmp) {
+      kb = 0;
+      ke = ncmp_visible(t_last, args.cmp_len, args.cmp_stride);
+    } else if (MODE == kModeWin) {
+      kb = max(0, t0 - args.window + 1);
+      ke = t_last + 1;
+    } else {
+      kb = 0;
+      ke = t_last + 1;
+    }
+    nkt = (ke - kb + kBN - 1) / kBN;
+  };
 
   if (tid == 0) {
     mbar_init(&sm.q_full, 1);
     mbar_init(&sm.q_tmem, 4 * kSoftmaxWG);
+    mbar_init(&sm.q_empty, 4 * kSoftmaxWG);
+    mbar_init(&sm.qcols_free, 1);
     for (int x = 0; x < Smem::kSlots; ++x) {
       mbar_init(&sm.full[x], 1);
       mbar_init(&sm.empty[x], 1);
@@ -255,8 +266,10 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
       mbar_init(&sm.carry_free[b], 4);
     }
     mbar_init(&sm.p_full, 4 * kTileWG);
-    mbar_init(&sm.p_free, 1);
+    mbar_init(&sm.p_free[0], 1);
+    mbar_init(&sm.p_free[1], 1);
     mbar_init(&sm.o_full, 1);
+    mbar_init(&sm.o_free, 4 * kSoftmaxWG);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
@@ -280,30 +293,61 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort_flag = &sm.abort_flag;
-  int issued = 0;  // producer: loads whose TMA was issued
+  int issued = 0;    // producer: K/V loads whose TMA was issued
+  int q_issued = 0;  // producer: Q tiles whose TMA was issued
+  bool leader = false;  // MMA warp: the lane that issues every tcgen05 op
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
-    // load L: L < nkt -> K tile L (phase 1); else position L - nkt of the phase-2 sequence
-    // (p2_item). Load L goes to slot L % kSlots once the MMA has released the load kSlots
-    // before it.
-    if (lane == 0 && nkt > 0) {
+    // Per item: its Q tile (into the single Q buffer, once the softmax warps have moved the
+    // previous one into TMEM), then its K/V loads. Load l of an item: l < nkt -> K tile l
+    // (phase 1); else position l - nkt of the phase-2 sequence (p2_item). The CTA-wide load
+    // counter L picks slot L % kSlots, which is reused once the MMA has released load
+    // L - kSlots. The next item's Q is issued as soon as the buffer frees up.
+    if (lane == 0 && blockIdx.x < n_items) {
       tma_prefetch_desc(&qmap);
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
-      mbar_arrive_expect_tx(&sm.q_full, kChunks * T * args.Gp * 128);
-      for (int c = 0; c < kChunks; ++c) tma_load_3d(&qmap, &sm.q_full, sm.q[c], c * 64, g * G, t0);
-      for (int L = 0; L < nloads; ++L) {
-        const int x = L % kSlots;
-        if (L >= kSlots && !mbar_wait(&sm.empty[x], ((L / kSlots) - 1) & 1, abort_flag)) break;
-        bool is_v = false;
-        int kt = L;
-        if (L >= nkt) p2_item(L - nkt, nkt, is_v, kt);
-        const int kpos = kb + kt * kBN;
-        mbar_arrive_expect_tx(&sm.full[x], Smem::kSlotBytes);
-        for (int c = 0; c < kChunks; ++c)
-          tma_load_3d(is_v ? &vmap : &kmap, &sm.full[x], sm.slot[x][c], c * 64, g, kpos);
-        issued = L + 1;
+      auto load_q = [&](int item) {
+        int g, t0, kb, nkt;
+        item_geo(item, g, t0, kb, nkt);
+        mbar_arrive_expect_tx(&sm.q_full, kChunks * T * args.Gp * 128);
+        for (int c = 0; c < kChunks; ++c) tma_load_3d(&qmap, &sm.q_full, sm.q[c], c * 64, g * G, t0);
+        ++q_issued;
+      };
+      load_q(blockIdx.x);
+      bool ok = true;
+      int L = 0;
+      for (int it = 0; ok && (kPersist || it == 0); ++it) {
+        const int item = blockIdx.x + it * gridDim.x;
+        if (item >= n_items) break;
+        int g, t0, kb, nkt;
+        item_geo(item, g, t0, kb, nkt);
+        const bool has_next = kPersist && item + static_cast<int>(gridDim.x) < n_items;
+        bool next_q = !has_next;
+        for (int l = 0; l < 3 * nkt; ++l, ++L) {
+          if (!next_q && mbar_ready(&sm.q_empty, it & 1)) {
+            load_q(item + gridDim.x);
+            next_q = true;
+          }
+          const int x = L % kSlots;
+          if (L >= kSlots && !mbar_wait(&sm.empty[x], ((L / kSlots) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          bool is_v = false;
+          int kt = l;
+          if (l >= nkt) p2_item(l - nkt, nkt, is_v, kt);
+          const int kpos = kb + kt * kBN;
+          mbar_arrive_expect_tx(&sm.full[x], Smem::kSlotBytes);
+          for (int c = 0; c < kChunks; ++c)
+            tma_load_3d(is_v ? &vmap : &kmap, &sm.full[x], sm.slot[x][c], c * 64, g, kpos);
+          issued = L + 1;
+        }
+        if (ok && !next_q) {
+          if (!mbar_wait(&sm.q_empty, it & 1, abort_flag)) break;
+          load_q(item + gridDim.x);
+        }
       }
     }
     __syncwarp();
@@ -312,21 +356,35 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
     // The whole warp runs the issue loop (waits, descriptor arithmetic) in lockstep and one
     // elected lane issues each tcgen05 instruction: the operands stay warp-uniform, so the
     // issuing warp needs few of the scheduler's slots, which it shares with four softmax warps.
-    if (nkt > 0) {
-      const bool leader = elect_one_sync();
-      constexpr uint32_t idS = idesc_bf16_f32(128, kBN, false, false);
-      constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);
-      auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
-        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+    // Barrier phases run on across items: an item has 2*nkt MMA jobs (nkt per S buffer),
+    // nkt P.V products and 3*nkt loads, so `base` (the CTA's tiles so far) fixes every parity.
+    leader = elect_one_sync();
+    constexpr uint32_t idS = idesc_bf16_f32(128, kBN, false, false);
+    constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+    };
+    bool ok = true;
+    int base = 0;
+    for (int it = 0; ok && (kPersist || it == 0); ++it) {
+      const int item = blockIdx.x + it * gridDim.x;
+      if (item >= n_items) break;
+      int g, t0, kb, nkt;
+      item_geo(item, g, t0, kb, nkt);
+      const int njobs = 2 * nkt;
+      ok = wait_all(&sm.q_tmem, it & 1);  // Q staged in TMEM by the softmax warps
+      auto wait_load = [&](int l) -> bool {
+        const int L = 3 * base + l;
+        return wait_all(&sm.full[L % kSlots], (L / kSlots) & 1);
       };
-      bool ok = wait_all(&sm.q_tmem, 0);  // Q staged in TMEM by the softmax warps
-      auto wait_load = [&](int L) -> bool { return wait_all(&sm.full[L % kSlots], (L / kSlots) & 1); };
       auto issue_s = [&](int job) -> bool {
-        const int L = job < nkt ? job : nkt + p2_k_pos(job - nkt);
-        const int x = L % kSlots;
+        const int l = job < nkt ? job : nkt + p2_k_pos(job - nkt);
+        const int x = (3 * base + l) % kSlots;
         const int b = job & 1;
-        if (!wait_load(L)) return false;
-        if (job >= 2 && !wait_all(&sm.s_free[b], ((job >> 1) - 1) & 1)) return false;
+        if (!wait_load(l)) return false;
+        // S(job) reuses the buffer of the job two before it (possibly of the previous item)
+        const int use = base + (job >> 1);
+        if (use >= 1 && !wait_all(&sm.s_free[b], (use - 1) & 1)) return false;
         tc_fence_after();
         // A = Q from TMEM (dims 16k .. 16k+15 in columns kColQ + 8k ..), B = K from smem;
         // the B descriptor advances by constant offsets (start address field in 16-byte units)
@@ -341,6 +399,8 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
           }
           umma_commit(&sm.s_full[b]);
           umma_commit(&sm.empty[x]);  // the K tile is no longer needed
+          // after the item's last score tile, Q's TMEM columns may take the next item's Q
+          if (job == njobs - 1) umma_commit(&sm.qcols_free);
         }
         __syncwarp();
         return true;
@@ -348,7 +408,7 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
       // Score tiles run two jobs ahead: S(job + 2) waits only for its buffer, which the pair
       // that read S(job) frees as soon as the scores are in registers, so it computes while
       // that pair is still in its softmax; P.V(job) follows once P(job) is in TMEM.
-      if (ok) ok = issue_s(0);
+      if (ok && njobs > 0) ok = issue_s(0);
       if (ok && njobs > 1) ok = issue_s(1);
       for (int job = 0; ok && job < njobs; ++job) {
         if (job + 2 < njobs && !issue_s(job + 2)) {
@@ -357,9 +417,14 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
         }
         if (job >= nkt) {
           const int kt2 = job - nkt;
-          const int L = nkt + p2_v_pos(kt2, nkt);  // V tile
-          const int x = L % kSlots;
-          if (!wait_load(L) || !wait_all(&sm.p_full, kt2 & 1)) {
+          const int l = nkt + p2_v_pos(kt2, nkt);  // V tile
+          const int x = (3 * base + l) % kSlots;
+          if (!wait_load(l) || !wait_all(&sm.p_full, (base + kt2) & 1)) {
+            ok = false;
+            break;
+          }
+          // the first P.V of an item overwrites O: the previous item's epilogue has read it
+          if (kt2 == 0 && it > 0 && !wait_all(&sm.o_free, (it - 1) & 1)) {
             ok = false;
             break;
           }
@@ -371,13 +436,23 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
             for (int k = 0; k < kBN / 16; ++k)  // keys 16k .. 16k+15 (P columns kColP + 8k ..)
               umma_bf16_ts(ocol, pcol + k * 8, vdesc + static_cast<uint64_t>(k * (2048 >> 4)), idO,
                            (kt2 > 0 || k > 0) ? 1u : 0u);
-            umma_commit(&sm.p_free);    // this P.V (and its reads of P from TMEM) is done
+            // this P.V (and its reads of P from TMEM) is done; counted per pair of the tile
+            umma_commit(&sm.p_free[kPairs == 1 ? 0 : (job & 1)]);
             umma_commit(&sm.empty[x]);  // the V tile is no longer needed
           }
           __syncwarp();
         }
       }
-      if (ok && leader) umma_commit(&sm.o_full);
+      // An item without keys commits at once; it still waits for the previous item's epilogue,
+      // so o_full never completes twice before the softmax warps have waited for the first
+      // of the two (the waits tell phases apart by parity only).
+      if (ok && njobs == 0 && it > 0) ok = wait_all(&sm.o_free, (it - 1) & 1);
+      if (ok && leader) {
+        if (njobs == 0) umma_commit(&sm.qcols_free);  // (no MMA of this item: arrives at once)
+        umma_commit(&sm.o_full);
+      }
+      __syncwarp();
+      base += nkt;
     }
     __syncwarp();
   } else {
@@ -394,300 +469,342 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
     const int r = q4 * 32 + lane;            // MMA row
     const int Gp = args.Gp;
     const int tok = r / Gp, hh = r % Gp;
-    const int t = t0 + tok;
-    const int h = g * G + hh;
-    const bool row_valid = (r < T * Gp) && (hh < G) && (t < args.q_end);
-    int rb = 0, re = 0;                      // visible key range of this row
-    if (row_valid) {
-      if (MODE == kModeCmp) {
-        re = ncmp_visible(t, args.cmp_len, args.cmp_stride);
-      } else if (MODE == kModeWin) {
-        rb = max(0, t - args.window + 1);
-        re = t + 1;
-      } else {
-        re = t + 1;
-      }
-    }
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int col0 = half * kColsPerWG;
-    if (MODE == kModeWin && row_valid) {
-      // the epilogue reads this row's o_cmp, o_sel and gates: start bringing them into L2
-      const size_t orow = (static_cast<size_t>(t) * args.hq + h) * D + wg * (D / kSoftmaxWG);
-#pragma unroll
-      for (int c = 0; c < D / kSoftmaxWG; c += 32) {
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(args.o_cmp + orow + c));
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(args.o_sel + orow + c));
-      }
-      if (wg == 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(args.gates + (static_cast<size_t>(t) * args.hq + h) * 3));
-    }
     const float sl2 = args.scale_log2;
-    bool ok = true;
-    // ---- Q row r into TMEM, packed in bf16 pairs like P: this warpgroup copies dims
-    // [wg*D/4, (wg+1)*D/4) from the 128-byte-swizzled smem image (16-byte unit u of a row
-    // sits at unit u ^ (row & 7)); rows past the tile are the zeros written at the start.
-    // A tile without keys loads no Q and runs no MMA.
-    if (nkt > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_full, 0, abort_flag));
-      if (ok) {
-        constexpr int kDimsPerWG = D / kSoftmaxWG;  // 64 (D=128) or 32 (D=64)
-        uint32_t qv[kDimsPerWG / 2];
-#pragma unroll
-        for (int i = 0; i < kDimsPerWG / 8; ++i) {
-          const int dim0 = wg * kDimsPerWG + 8 * i;
-          const int c = dim0 / 64, u = (dim0 % 64) / 8;
-          const uint4 w4 = *reinterpret_cast<const uint4*>(&sm.q[c][r * 128 + ((u ^ (r & 7)) << 4)]);
-          qv[4 * i] = w4.x;
-          qv[4 * i + 1] = w4.y;
-          qv[4 * i + 2] = w4.z;
-          qv[4 * i + 3] = w4.w;
-        }
-        __syncwarp();
-        if constexpr (kDimsPerWG / 2 >= 16) {
-#pragma unroll
-          for (int h = 0; h < kDimsPerWG / 32; ++h)
-            tmem_st16(trow + kColQ + wg * (kDimsPerWG / 2) + 16 * h, *reinterpret_cast<const uint32_t(*)[16]>(&qv[16 * h]));
-        } else {
-          tmem_st8(trow + kColQ + wg * 8, *reinterpret_cast<const uint32_t(*)[8]>(&qv[0]));
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.q_tmem);
-      }
-    }
-    // ---- phase 1: log-sum-exp (base 2) of this row's column slice, combined below
-    float m = -INFINITY, lsum = 0.f;         // m: running max of the raw (unscaled) scores
-    for (int kt = kPairs == 1 ? 0 : pair; kt < nkt && ok; kt += kPairs) {
-      const int b = kt & 1;
-      // tcgen05.ld is warp-collective: every wait result is made warp-uniform
-      ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (kt >> 1) & 1, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      const int kbase = kb + kt * kBN + col0;
-      // warp-uniform: the unmasked path only when every row of the warp sees the whole
-      // slice; rows without keys (head padding, past the end) follow the others, their
-      // probabilities being forced to 0 through lse2 = +inf
-      const bool full = __all_sync(0xffffffffu, !row_valid || (kbase >= rb && kbase + kColsPerWG <= re));
-      // 32 columns at a time (an online max across the chunks keeps one chunk in registers)
-      static_assert(kColsPerWG % 32 == 0, "phase 1 reads 32-column chunks");
-#pragma unroll
-      for (int h = 0; h < kColsPerWG / 32; ++h) {
-        float s[32];
-        __syncwarp();
-        tmem_ld32(trow + b * kBN + col0 + 32 * h, s);
-        tmem_wait_ld();
-        if (h == kColsPerWG / 32 - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.s_free[b]);  // S is in registers: the buffer may be reused
-        }
-        if (!full) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int kidx = kbase + 32 * h + i;
-            s[i] = (kidx >= rb && kidx < re) ? s[i] : -INFINITY;
-          }
-        }
-        float mx[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) mx[c] = fmax3f(fmaxf(s[c], s[c + 8]), s[c + 16], s[c + 24]);
-        const float cmax = fmax3f(fmax3f(mx[0], mx[1], mx[2]), fmax3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-        const float mnew = fmaxf(m, cmax);
-        if (MODE != kModeCmp) {
-          m = mnew;  // the window and dense branches need only the row max here
-        } else if (mnew != -INFINITY) {
-          const float ms = mnew * sl2;
-          lsum = lsum * ex2_approx((m - mnew) * sl2) + chunk_sum_ex2(s, sl2, ms);
-          m = mnew;
-        }
-      }
-    }
-    sm.lse_x[wg][r][0] = (m == -INFINITY) ? -INFINITY : m * sl2;
-    sm.lse_x[wg][r][1] = lsum;
-    named_bar_sync(3, kSoftmaxThreads);
-    float lse2;
-    bool has_keys;
-    {
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kSoftmaxWG; ++w) M = fmaxf(M, sm.lse_x[w][r][0]);
-      float L = 0.f;
-      if (M != -INFINITY) {
-#pragma unroll
-        for (int w = 0; w < kSoftmaxWG; ++w) L += sm.lse_x[w][r][1] * ex2_approx(sm.lse_x[w][r][0] - M);
-      }
-      if (MODE == kModeCmp) {
-        has_keys = row_valid && L > 0.f;
-        lse2 = has_keys ? M + __log2f(L) : INFINITY;
-      } else {
-        // P = exp2(S*scale*log2e - max) unnormalised; the row sum divides O at the end
-        has_keys = row_valid && M != -INFINITY;
-        lse2 = has_keys ? M : INFINITY;
-      }
-    }
-    float psum = 0.f;  // (window, dense) this thread's part of the row sum of P
-    // ---- phase 2: normalised probabilities -> P (smem, bf16) and block scores
-    // Block scores (kModeCmp): compressed block i covers tokens [16i, 16i+32) and selection
-    // block j covers [64j, 64j+64), so block j takes all of compressed blocks 4j..4j+2 and
-    // half of 4j-1 and 4j+3. A 128-key tile holds selection blocks kt2*32 .. kt2*32+31;
-    // this warpgroup's columns hold kBinsPerWG of them. The compressed block that straddles
-    // the two column halves (column 63) is re-read from TMEM by the upper half. The one that
-    // straddles two tiles (column 127 of the previous tile, which the other pair handled)
-    // arrives through a shared-memory slot: the upper half of each tile leaves half of its
-    // column-127 probability there and the lower half of the next tile picks it up (slot
-    // kt2 & 1, guarded by carry_full / carry_free). The G heads of a token sit in Gp adjacent
-    // lanes; a shuffle reduce-scatter sums them.
-    float carry_last = 0.f;  // upper half, last tile: half of its last compressed block
     // (kModeCmp) the scores are reduced over the heads per 32-column chunk (8 selection
     // blocks): lane hh then holds blocks [hh*bpl, (hh+1)*bpl) of the chunk (Gp <= 8), or block
-    // hh/share shared with its neighbours (Gp > 8); these store invariants do not change from
-    // tile to tile
+    // hh/share shared with its neighbours (Gp > 8)
     constexpr int kChunkBins = 8;  // selection blocks per 32-column chunk
     const int sc_bpl = Gp <= kChunkBins ? kChunkBins / Gp : 1;
     const int sc_share = Gp <= kChunkBins ? 1 : Gp / kChunkBins;
-    const bool sc_store = MODE == kModeCmp && t < args.q_end && (hh % sc_share) == 0;
-    const int sc_jt = t / args.sel_len;
     const int sc_j0 = half * kBinsPerWG + (hh / sc_share) * sc_bpl;
-    float* const sc_dst = args.scores + (static_cast<size_t>(t) * args.hkv + g) * args.nsel;
-    // this pair's phase-2 jobs are those of parity `pair`: job nkt + kt2
-    for (int kt2 = kPairs == 1 ? 0 : ((pair + nkt) & 1); kt2 < nkt; kt2 += kPairs) {
-      const int job = nkt + kt2;
-      const int b = job & 1;
-      if (ok) ok = mbar_wait(&sm.s_full[b], (job >> 1) & 1, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
+    // (kModeCmp) carry slot `p` takes half of column 127 of the tiles of pair p (written by
+    // its upper half, read by the lower half of the other pair); uses counted across items
+    int carry_writes = 0, carry_reads = 0;
+    int other_pv = 0;  // (two pairs) P.V products of the other pair's tiles in earlier items
+    bool ok = true;
+
+    // ---- Q rows into TMEM, packed in bf16 pairs like P: this warpgroup copies dims
+    // [wg*D/kSoftmaxWG, ...) of row r from the 128-byte-swizzled smem image (16-byte unit u
+    // of a row sits at unit u ^ (row & 7)); rows past the tile are the zeros written at the
+    // start. Q of item `it` waits for its TMA and, after the first item, for the last score
+    // MMA of the previous item (which read the same TMEM columns).
+    auto stage_q = [&](int it) -> bool {
+      bool w = mbar_wait(&sm.q_full, it & 1, abort_flag);
+      if (w && it > 0) w = mbar_wait(&sm.qcols_free, (it - 1) & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, w)) return false;
       tc_fence_after();
-      const int kbase = kb + kt2 * kBN + col0;
-      // warp-uniform: the unmasked path only when every row of the warp sees the whole
-      // slice; rows without keys (head padding, past the end) follow the others, their
-      // probabilities being forced to 0 through lse2 = +inf
-      const bool full = __all_sync(0xffffffffu, !row_valid || (kbase >= rb && kbase + kColsPerWG <= re));
-      float half_in = 0.f;
-      // 32 columns at a time: read from TMEM, exponentials, then (kModeCmp) the chunk's 8
-      // block scores, then the chunk's P packed to bf16 pairs, so only one chunk is ever held
-      // in fp32
-      static_assert(kColsPerWG % 32 == 0, "P is stored 16 columns (32 keys) at a time");
-      uint32_t pk[kColsPerWG / 2];
-      float prev_last = 0.f;  // (kModeCmp) p of the previous chunk's last column
+      constexpr int kDimsPerWG = D / kSoftmaxWG;  // 32 or 64 (D=128), 16 or 32 (D=64)
+      uint32_t qv[kDimsPerWG / 2];
 #pragma unroll
-      for (int h = 0; h < kColsPerWG / 32; ++h) {
-        float sc[32];
-        uint32_t xv = 0;
-        __syncwarp();
-        tmem_ld32(trow + b * kBN + col0 + 32 * h, sc);
-        if (MODE == kModeCmp && h == 0 && half > 0)
-          asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(xv) : "r"(trow + b * kBN + col0 - 1));
-        tmem_wait_ld();
-        if (h == kColsPerWG / 32 - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.s_free[b]);  // S is in registers: the buffer may be reused
-        }
-        if (MODE == kModeCmp && h == 0 && half > 0) {
-          const int xk = kb + kt2 * kBN + col0 - 1;
-          half_in = (xk >= rb && xk < re) ? 0.5f * ex2_approx(fmaf(__uint_as_float(xv), sl2, -lse2)) : 0.f;
-        }
-        chunk_ex2(sc, sl2, lse2, full, kbase + 32 * h, rb, re);
-        if (MODE != kModeCmp) {
-          float ps[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ps[i & 3] += sc[i];
-          psum += (ps[0] + ps[1]) + (ps[2] + ps[3]);
-        }
-        if (MODE == kModeCmp) {
-          if (h == 0 && half == 0 && kt2 > 0) {
-            // half of the previous tile's column 127, left by the other pair
-            const int slot = (kt2 - 1) & 1;
-            if (ok) ok = mbar_wait(&sm.carry_full[slot], ((kt2 - 1) >> 1) & 1, abort_flag);
-            half_in = sm.carry[slot][r];
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.carry_free[slot]);
-          }
-          if (h == kColsPerWG / 32 - 1 && half == kTileWG - 1) {
-            // hand half of column 127 to the next tile's lower half (the other pair)
-            const float c127 = 0.5f * sc[31];
-            if (kt2 + 1 < nkt) {
-              const int slot = kt2 & 1;
-              if (kt2 >= 2 && ok) ok = mbar_wait(&sm.carry_free[slot], ((kt2 >> 1) - 1) & 1, abort_flag);
-              sm.carry[slot][r] = c127;
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&sm.carry_full[slot]);
-            } else {
-              carry_last = c127;
-            }
-          }
-          float bin[kChunkBins];
-#pragma unroll
-          for (int u = 0; u < kChunkBins; ++u) {
-            const float left = u > 0 ? 0.5f * sc[4 * u - 1] : (h == 0 ? half_in : 0.5f * prev_last);
-            bin[u] = left + sc[4 * u] + sc[4 * u + 1] + sc[4 * u + 2] + 0.5f * sc[4 * u + 3];
-          }
-          prev_last = sc[31];
-          switch (Gp) {
-            case 2: group_reduce_scatter<2, kChunkBins>(bin, lane); break;
-            case 4: group_reduce_scatter<4, kChunkBins>(bin, lane); break;
-            case 8: group_reduce_scatter<8, kChunkBins>(bin, lane); break;
-            case 16: group_reduce_scatter<16, kChunkBins>(bin, lane); break;
-            default: break;
-          }
-          if (sc_store) {
-            const int j0 = kt2 * 32 + h * kChunkBins + sc_j0;
-            if (sc_bpl == 1) {
-              if (j0 <= sc_jt) sc_dst[j0] = bin[0];
-            } else {
-#pragma unroll
-              for (int i = 0; i < kChunkBins; ++i)
-                if (i < sc_bpl && j0 + i <= sc_jt) sc_dst[j0 + i] = bin[i];
-            }
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) pk[16 * h + i] = pack_bf16x2(sc[2 * i], sc[2 * i + 1]);
+      for (int i = 0; i < kDimsPerWG / 8; ++i) {
+        const int dim0 = wg * kDimsPerWG + 8 * i;
+        const int c = dim0 / 64, u = (dim0 % 64) / 8;
+        const uint4 w4 = *reinterpret_cast<const uint4*>(&sm.q[c][r * 128 + ((u ^ (r & 7)) << 4)]);
+        qv[4 * i] = w4.x;
+        qv[4 * i + 1] = w4.y;
+        qv[4 * i + 2] = w4.z;
+        qv[4 * i + 3] = w4.w;
       }
-      // P row r, keys col0 .. col0+kColsPerWG-1 -> packed bf16 pairs in TMEM columns
-      // kColP + col0/2 .. . P(kt2) is stored only once the P.V MMA of the previous tile has
-      // finished: tcgen05.st into TMEM while a P.V that reads its A operand from TMEM was
-      // still running corrupted rows 0-31 of the output on B200 even while P was
-      // double-buffered in disjoint columns; with that wait in place one P buffer suffices.
-      // The wait comes after the exponentials, which overlap the previous P.V.
-      if (ok && kt2 > 0) ok = mbar_wait(&sm.p_free, (kt2 - 1) & 1, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
+      __syncwarp();
+      if constexpr (kDimsPerWG / 2 >= 16) {
 #pragma unroll
-      for (int h = 0; h < kColsPerWG / 32; ++h)
-        tmem_st16(trow + kColP + col0 / 2 + 16 * h, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * h]));
+        for (int hx = 0; hx < kDimsPerWG / 32; ++hx)
+          tmem_st16(trow + kColQ + wg * (kDimsPerWG / 2) + 16 * hx,
+                    *reinterpret_cast<const uint32_t(*)[16]>(&qv[16 * hx]));
+      } else {
+        tmem_st8(trow + kColQ + wg * 8, *reinterpret_cast<const uint32_t(*)[8]>(&qv[0]));
+      }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.p_full);
-    }
-    if (MODE == kModeCmp && ok && wg == kSoftmaxWG - 1) {
-      // the half-block after the last tile lands in selection block nkt*32; the last
-      // phase-2 job (2*nkt - 1) is odd, so this warpgroup (upper half of pair 1) holds it.
-      // When no key tile exists at all, that is block 0 with score 0.
-      float c = carry_last;
+      if (lane == 0) {
+        mbar_arrive(&sm.q_tmem);
+        mbar_arrive(&sm.q_empty);  // the smem Q buffer may take the next item's tile
+      }
+      return true;
+    };
+    if (blockIdx.x < n_items) ok = stage_q(0);
+
+    // Every softmax thread runs every item, also after a failed wait (its waits are then
+    // skipped): the named barriers below are passed the same number of times by all of them.
+    int base = 0;
+    for (int it = 0; kPersist || it == 0; ++it) {
+      const int item = blockIdx.x + it * gridDim.x;
+      if (item >= n_items) break;
+      int g, t0, kb, nkt;
+      item_geo(item, g, t0, kb, nkt);
+      const int t = t0 + tok;
+      const int h = g * G + hh;
+      const bool row_valid = (r < T * Gp) && (hh < G) && (t < args.q_end);
+      int rb = 0, re = 0;  // visible key range of this row
+      if (row_valid) {
+        if (MODE == kModeCmp) {
+          re = ncmp_visible(t, args.cmp_len, args.cmp_stride);
+        } else if (MODE == kModeWin) {
+          rb = max(0, t - args.window + 1);
+          re = t + 1;
+        } else {
+          re = t + 1;
+        }
+      }
+      if (MODE == kModeWin && row_valid) {
+        // the epilogue reads this row's o_cmp, o_sel and gates: start bringing them into L2
+        const size_t orow = (static_cast<size_t>(t) * args.hq + h) * D + wg * (D / kSoftmaxWG);
 #pragma unroll
-      for (int o = 1; o < 16; o <<= 1)
-        if (o < Gp) c += __shfl_xor_sync(0xffffffffu, c, o);
-      const int j = nkt * 32;
-      if (hh == 0 && t < args.q_end && j <= t / args.sel_len)
-        args.scores[(static_cast<size_t>(t) * args.hkv + g) * args.nsel + j] = c;
-    }
-    float inv_l = 1.f;  // (window, dense) 1 / row sum of P over all column slices
-    if (MODE != kModeCmp) {
-      sm.lse_x[wg][r][1] = psum;
+        for (int c = 0; c < D / kSoftmaxWG; c += 32) {
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(args.o_cmp + orow + c));
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(args.o_sel + orow + c));
+        }
+        if (wg == 0)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(args.gates + (static_cast<size_t>(t) * args.hq + h) * 3));
+      }
+
+      // ---- phase 1: log-sum-exp (base 2) of this row's column slice, combined below
+      float m = -INFINITY, lsum = 0.f;  // m: running max of the raw (unscaled) scores
+      for (int kt = kPairs == 1 ? 0 : pair; kt < nkt && ok; kt += kPairs) {
+        const int b = kt & 1;
+        // tcgen05.ld is warp-collective: every wait result is made warp-uniform
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (base + (kt >> 1)) & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        const int kbase = kb + kt * kBN + col0;
+        // warp-uniform: the unmasked path only when every row of the warp sees the whole
+        // slice; rows without keys (head padding, past the end) follow the others, their
+        // probabilities being forced to 0 through lse2 = +inf
+        const bool full = __all_sync(0xffffffffu, !row_valid || (kbase >= rb && kbase + kColsPerWG <= re));
+        // 32 columns at a time (an online max across the chunks keeps one chunk in registers)
+        static_assert(kColsPerWG % 32 == 0, "phase 1 reads 32-column chunks");
+#pragma unroll
+        for (int hc = 0; hc < kColsPerWG / 32; ++hc) {
+          float s[32];
+          __syncwarp();
+          tmem_ld32(trow + b * kBN + col0 + 32 * hc, s);
+          tmem_wait_ld();
+          if (hc == kColsPerWG / 32 - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.s_free[b]);  // S is in registers: the buffer may be reused
+          }
+          if (!full) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int kidx = kbase + 32 * hc + i;
+              s[i] = (kidx >= rb && kidx < re) ? s[i] : -INFINITY;
+            }
+          }
+          float mx[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) mx[c] = fmax3f(fmaxf(s[c], s[c + 8]), s[c + 16], s[c + 24]);
+          const float cmax = fmax3f(fmax3f(mx[0], mx[1], mx[2]), fmax3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+          const float mnew = fmaxf(m, cmax);
+          if (MODE != kModeCmp) {
+            m = mnew;  // the window and dense branches need only the row max here
+          } else if (mnew != -INFINITY) {
+            const float ms = mnew * sl2;
+            lsum = lsum * ex2_approx((m - mnew) * sl2) + chunk_sum_ex2(s, sl2, ms);
+            m = mnew;
+          }
+        }
+      }
+      sm.lse_x[wg][r][0] = (m == -INFINITY) ? -INFINITY : m * sl2;
+      sm.lse_x[wg][r][1] = lsum;
       named_bar_sync(3, kSoftmaxThreads);
-      float L = 0.f;
+      float lse2;
+      bool has_keys;
+      {
+        float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < kSoftmaxWG; ++w) L += sm.lse_x[w][r][1];
-      inv_l = L > 0.f ? 1.f / L : 0.f;
-    }
-    // ---- epilogue (every lane loads its TMEM row; only valid rows are stored)
-    if (ok && nkt > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_full, 0, abort_flag));
-      tc_fence_after();
-    }
-    if (ok) {
+        for (int w = 0; w < kSoftmaxWG; ++w) M = fmaxf(M, sm.lse_x[w][r][0]);
+        float Lsum = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+          for (int w = 0; w < kSoftmaxWG; ++w) Lsum += sm.lse_x[w][r][1] * ex2_approx(sm.lse_x[w][r][0] - M);
+        }
+        if (MODE == kModeCmp) {
+          has_keys = row_valid && Lsum > 0.f;
+          lse2 = has_keys ? M + __log2f(Lsum) : INFINITY;
+        } else {
+          // P = exp2(S*scale*log2e - max) unnormalised; the row sum divides O at the end
+          has_keys = row_valid && M != -INFINITY;
+          lse2 = has_keys ? M : INFINITY;
+        }
+      }
+      float psum = 0.f;  // (window, dense) this thread's part of the row sum of P
+      // ---- phase 2: normalised probabilities -> P (TMEM, bf16) and block scores
+      // Block scores (kModeCmp): compressed block i covers tokens [16i, 16i+32) and selection
+      // block j covers [64j, 64j+64), so block j takes all of compressed blocks 4j..4j+2 and
+      // half of 4j-1 and 4j+3. A 128-key tile holds selection blocks kt2*32 .. kt2*32+31;
+      // this warpgroup's columns hold kBinsPerWG of them. The compressed block that straddles
+      // the two column halves (column 63) is re-read from TMEM by the upper half. The one that
+      // straddles two tiles (column 127 of the previous tile, which the other pair handled)
+      // arrives through a shared-memory slot: the upper half of each tile leaves half of its
+      // column-127 probability there and the lower half of the next tile picks it up (guarded
+      // by carry_full / carry_free). The G heads of a token sit in Gp adjacent lanes; a shuffle
+      // reduce-scatter sums them.
+      float carry_last = 0.f;  // upper half, last tile: half of its last compressed block
+      const bool sc_store = MODE == kModeCmp && t < args.q_end && (hh % sc_share) == 0;
+      const int sc_jt = t / args.sel_len;
+      float* const sc_dst = args.scores + (static_cast<size_t>(t) * args.hkv + g) * args.nsel;
+      // this pair's phase-2 jobs are those of parity `pair`: job nkt + kt2
+      for (int kt2 = kPairs == 1 ? 0 : ((pair + nkt) & 1); ok && kt2 < nkt; kt2 += kPairs) {
+        const int job = nkt + kt2;
+        const int b = job & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (base + (job >> 1)) & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        const int kbase = kb + kt2 * kBN + col0;
+        const bool full = __all_sync(0xffffffffu, !row_valid || (kbase >= rb && kbase + kColsPerWG <= re));
+        float half_in = 0.f;
+        // 32 columns at a time: read from TMEM, exponentials, then (kModeCmp) the chunk's 8
+        // block scores, then the chunk's P packed to bf16 pairs, so only one chunk is ever held
+        // in fp32
+        static_assert(kColsPerWG % 32 == 0, "P is stored 16 columns (32 keys) at a time");
+        uint32_t pk[kColsPerWG / 2];
+        float prev_last = 0.f;  // (kModeCmp) p of the previous chunk's last column
+#pragma unroll
+        for (int hc = 0; hc < kColsPerWG / 32; ++hc) {
+          float sc[32];
+          uint32_t xv = 0;
+          __syncwarp();
+          tmem_ld32(trow + b * kBN + col0 + 32 * hc, sc);
+          if (MODE == kModeCmp && hc == 0 && half > 0)
+            asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(xv) : "r"(trow + b * kBN + col0 - 1));
+          tmem_wait_ld();
+          if (hc == kColsPerWG / 32 - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.s_free[b]);  // S is in registers: the buffer may be reused
+          }
+          if (MODE == kModeCmp && hc == 0 && half > 0) {
+            const int xk = kb + kt2 * kBN + col0 - 1;
+            half_in = (xk >= rb && xk < re) ? 0.5f * ex2_approx(fmaf(__uint_as_float(xv), sl2, -lse2)) : 0.f;
+          }
+          chunk_ex2(sc, sl2, lse2, full, kbase + 32 * hc, rb, re);
+          if (MODE != kModeCmp) {
+            float ps[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ps[i & 3] += sc[i];
+            psum += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+          }
+          if (MODE == kModeCmp) {
+            if (hc == 0 && half == 0 && kt2 > 0) {
+              // half of the previous tile's column 127, left by the other pair in its slot
+              const int slot = pair ^ 1;
+              if (ok) ok = mbar_wait(&sm.carry_full[slot], carry_reads & 1, abort_flag);
+              half_in = sm.carry[slot][r];
+              ++carry_reads;
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&sm.carry_free[slot]);
+            }
+            if (hc == kColsPerWG / 32 - 1 && half == kTileWG - 1) {
+              // hand half of column 127 to the next tile's lower half (the other pair)
+              const float c127 = 0.5f * sc[31];
+              if (kt2 + 1 < nkt) {
+                const int slot = pair;
+                if (carry_writes > 0 && ok)
+                  ok = mbar_wait(&sm.carry_free[slot], (carry_writes - 1) & 1, abort_flag);
+                sm.carry[slot][r] = c127;
+                ++carry_writes;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.carry_full[slot]);
+              } else {
+                carry_last = c127;
+              }
+            }
+            float bin[kChunkBins];
+#pragma unroll
+            for (int u = 0; u < kChunkBins; ++u) {
+              const float left = u > 0 ? 0.5f * sc[4 * u - 1] : (hc == 0 ? half_in : 0.5f * prev_last);
+              bin[u] = left + sc[4 * u] + sc[4 * u + 1] + sc[4 * u + 2] + 0.5f * sc[4 * u + 3];
+            }
+            prev_last = sc[31];
+            switch (Gp) {
+              case 2: group_reduce_scatter<2, kChunkBins>(bin, lane); break;
+              case 4: group_reduce_scatter<4, kChunkBins>(bin, lane); break;
+              case 8: group_reduce_scatter<8, kChunkBins>(bin, lane); break;
+              case 16: group_reduce_scatter<16, kChunkBins>(bin, lane); break;
+              default: break;
+            }
+            if (sc_store) {
+              const int j0 = kt2 * 32 + hc * kChunkBins + sc_j0;
+              if (sc_bpl == 1) {
+                if (j0 <= sc_jt) sc_dst[j0] = bin[0];
+              } else {
+#pragma unroll
+                for (int i = 0; i < kChunkBins; ++i)
+                  if (i < sc_bpl && j0 + i <= sc_jt) sc_dst[j0 + i] = bin[i];
+              }
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[16 * hc + i] = pack_bf16x2(sc[2 * i], sc[2 * i + 1]);
+        }
+        // P row r, keys col0 .. col0+kColsPerWG-1 -> packed bf16 pairs in TMEM columns
+        // kColP + col0/2 .. . P(kt2) is stored only once the P.V MMA of the previous tile has
+        // finished: tcgen05.st into TMEM while a P.V that reads its A operand from TMEM was
+        // still running corrupted rows 0-31 of the output on B200 even while P was
+        // double-buffered in disjoint columns; with that wait in place one P buffer suffices.
+        // The wait comes after the exponentials, which overlap the previous P.V. The P.V of
+        // tile kt2 - 1 is the last one before it: its completion (counted on the barrier of the
+        // pair that owned that tile) means every earlier P.V has finished too. For the first
+        // tile of an item the previous item's epilogue already saw all of its P.V products
+        // finish.
+        if (ok && kt2 > 0) {
+          if (kPairs == 1) {
+            ok = mbar_wait(&sm.p_free[0], (base + kt2 - 1) & 1, abort_flag);
+          } else {
+            // P.V products of the other pair up to tile kt2 - 1 (its tiles are those whose job
+            // nkt + k has its parity): the last of them is the one to wait for
+            const int other = pair ^ 1;
+            const int n = other_pv + ((kt2 + (other == (nkt & 1) ? 1 : 0)) >> 1) - 1;
+            ok = mbar_wait(&sm.p_free[other], n & 1, abort_flag);
+          }
+        }
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+#pragma unroll
+        for (int hc = 0; hc < kColsPerWG / 32; ++hc)
+          tmem_st16(trow + kColP + col0 / 2 + 16 * hc, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * hc]));
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.p_full);
+      }
+      if (MODE == kModeCmp && ok && wg == kSoftmaxWG - 1) {
+        // the half-block after the last tile lands in selection block nkt*32; the last
+        // phase-2 job (2*nkt - 1) is odd, so this warpgroup (upper half of pair 1) holds it.
+        // When no key tile exists at all, that is block 0 with score 0.
+        float c = carry_last;
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1)
+          if (o < Gp) c += __shfl_xor_sync(0xffffffffu, c, o);
+        const int j = nkt * 32;
+        if (hh == 0 && t < args.q_end && j <= t / args.sel_len)
+          args.scores[(static_cast<size_t>(t) * args.hkv + g) * args.nsel + j] = c;
+      }
+      float inv_l = 1.f;  // (window, dense) 1 / row sum of P over all column slices
+      if (MODE != kModeCmp) {
+        sm.lse_x[wg][r][1] = psum;
+        named_bar_sync(3, kSoftmaxThreads);
+        float Lsum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kSoftmaxWG; ++w) Lsum += sm.lse_x[w][r][1];
+        inv_l = Lsum > 0.f ? 1.f / Lsum : 0.f;
+      }
+      // the next item's Q goes into TMEM now, so its score MMAs overlap this epilogue
+      if (kPersist && ok && item + static_cast<int>(gridDim.x) < n_items) ok = stage_q(it + 1);
+      // ---- epilogue (every lane loads its TMEM row; only valid rows are stored)
+      if (ok) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_full, it & 1, abort_flag));
+        tc_fence_after();
+      }
+      if (!ok) {
+        base += nkt;
+        other_pv += (nkt + ((pair ^ 1) == (nkt & 1) ? 1 : 0)) >> 1;
+        continue;
+      }
       const size_t orow = (static_cast<size_t>(t) * args.hq + h) * D;
       float g0 = 0.f, g1 = 0.f, g2 = 0.f;
       if (MODE == kModeWin && row_valid) {
@@ -695,60 +812,75 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
         g1 = args.gates[(static_cast<size_t>(t) * args.hq + h) * 3 + 1];
         g2 = args.gates[(static_cast<size_t>(t) * args.hq + h) * 3 + 2];
       }
-#pragma unroll 1
-      for (int cc = 0; cc < (D / kSoftmaxWG + 31) / 32; ++cc) {
-        constexpr int kOC = D / kSoftmaxWG < 32 ? D / kSoftmaxWG : 32;  // output columns per load
-        const int c0 = wg * (D / kSoftmaxWG) + cc * 32;                 // output columns c0 .. c0+kOC-1
-        float o[32];
-        __syncwarp();
-        if (nkt > 0) {
-          if (kOC == 32) {
-            tmem_ld32(trow + kColO + c0, o);
-          } else {
-            tmem_ld16(trow + kColO + c0, *reinterpret_cast<float(*)[16]>(&o[0]));
-          }
-          tmem_wait_ld();
-        } else {
+      constexpr int kOC = D / kSoftmaxWG < 32 ? D / kSoftmaxWG : 32;  // output columns per load
+      constexpr int kOLoads = (D / kSoftmaxWG + 31) / 32;
+      float o[kOLoads][32];
+      // O row r, this warpgroup's columns: into registers, then O's TMEM may take the next
+      // item's P.V while the stores run
+      __syncwarp();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0.f;
+      for (int cc = 0; cc < kOLoads; ++cc) {
+        const int c0 = wg * (D / kSoftmaxWG) + cc * 32;
+        if (kOC == 32) {
+          tmem_ld32(trow + kColO + c0, o[cc]);
+        } else {
+          tmem_ld16(trow + kColO + c0, *reinterpret_cast<float(*)[16]>(&o[cc][0]));
         }
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.o_free);
+      if (nkt == 0) {
+#pragma unroll
+        for (int cc = 0; cc < kOLoads; ++cc)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[cc][i] = 0.f;
+      }
+#pragma unroll
+      for (int cc = 0; cc < kOLoads; ++cc) {
+        const int c0 = wg * (D / kSoftmaxWG) + cc * 32;  // output columns c0 .. c0+kOC-1
+        float* oc_ = o[cc];
         if (!row_valid) {
           // nothing to store for padding rows
         } else if (MODE == kModeCmp) {
           float4* dst = reinterpret_cast<float4*>(args.o_cmp + orow + c0);
 #pragma unroll
-          for (int u = 0; u < kOC / 4; ++u) dst[u] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+          for (int u = 0; u < kOC / 4; ++u) dst[u] = make_float4(oc_[4 * u], oc_[4 * u + 1], oc_[4 * u + 2], oc_[4 * u + 3]);
         } else {
           if (MODE == kModeWin) {
-            const float4* oc = reinterpret_cast<const float4*>(args.o_cmp + orow + c0);
-            const float4* os = reinterpret_cast<const float4*>(args.o_sel + orow + c0);
+            const float4* ocp = reinterpret_cast<const float4*>(args.o_cmp + orow + c0);
+            const float4* osp = reinterpret_cast<const float4*>(args.o_sel + orow + c0);
 #pragma unroll
             for (int u = 0; u < kOC / 4; ++u) {
-              const float4 a = oc[u], c = os[u];
-              o[4 * u + 0] = g0 * a.x + g1 * c.x + g2 * (o[4 * u + 0] * inv_l);
-              o[4 * u + 1] = g0 * a.y + g1 * c.y + g2 * (o[4 * u + 1] * inv_l);
-              o[4 * u + 2] = g0 * a.z + g1 * c.z + g2 * (o[4 * u + 2] * inv_l);
-              o[4 * u + 3] = g0 * a.w + g1 * c.w + g2 * (o[4 * u + 3] * inv_l);
+              const float4 a4 = ocp[u], c4 = osp[u];
+              oc_[4 * u + 0] = g0 * a4.x + g1 * c4.x + g2 * (oc_[4 * u + 0] * inv_l);
+              oc_[4 * u + 1] = g0 * a4.y + g1 * c4.y + g2 * (oc_[4 * u + 1] * inv_l);
+              oc_[4 * u + 2] = g0 * a4.z + g1 * c4.z + g2 * (oc_[4 * u + 2] * inv_l);
+              oc_[4 * u + 3] = g0 * a4.w + g1 * c4.w + g2 * (oc_[4 * u + 3] * inv_l);
             }
           } else {
 #pragma unroll
-            for (int u = 0; u < kOC; ++u) o[u] *= inv_l;
+            for (int u = 0; u < kOC; ++u) oc_[u] *= inv_l;
           }
           if (args.out_f32) {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.out) + orow + c0);
 #pragma unroll
-            for (int u = 0; u < kOC / 4; ++u) dst[u] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+            for (int u = 0; u < kOC / 4; ++u)
+              dst[u] = make_float4(oc_[4 * u], oc_[4 * u + 1], oc_[4 * u + 2], oc_[4 * u + 3]);
           } else {
             uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) + orow + c0);
 #pragma unroll
             for (int u = 0; u < kOC / 8; ++u)
-              dst[u] = make_uint4(pack_bf16x2(o[8 * u], o[8 * u + 1]), pack_bf16x2(o[8 * u + 2], o[8 * u + 3]),
-                                  pack_bf16x2(o[8 * u + 4], o[8 * u + 5]), pack_bf16x2(o[8 * u + 6], o[8 * u + 7]));
+              dst[u] = make_uint4(pack_bf16x2(oc_[8 * u], oc_[8 * u + 1]), pack_bf16x2(oc_[8 * u + 2], oc_[8 * u + 3]),
+                                  pack_bf16x2(oc_[8 * u + 4], oc_[8 * u + 5]), pack_bf16x2(oc_[8 * u + 6], oc_[8 * u + 7]));
           }
         }
       }
       if (MODE == kModeCmp && row_valid && wg == 0)
         args.lse[static_cast<size_t>(t) * args.hq + h] = has_keys ? lse2 * 0.69314718055994530942f : -INFINITY;
+      base += nkt;
+      other_pv += (nkt + ((pair ^ 1) == (nkt & 1) ? 1 : 0)) >> 1;
     }
     tc_fence_before();
   }
@@ -759,9 +891,9 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
     // drain: wait (bounded) for TMA loads that were issued but never consumed and for
     // MMAs still in flight, so no async write lands after the CTA exits.
     if (warp == 0 && lane == 0) {
-      if (nkt > 0) {
+      if (q_issued > 0) {
         const long long t_start = clock64();
-        while (!mbar_test(&sm.q_full, 0) && clock64() - t_start < kWaitCycles) {
+        while (!mbar_test(&sm.q_full, (q_issued - 1) & 1) && clock64() - t_start < kWaitCycles) {
         }
       }
       // the last load issued into each slot (earlier ones completed before it was issued)
@@ -771,9 +903,9 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
         }
       }
     }
-    if (warp == 1 && nkt > 0) {
-      // the commit tracks the MMAs of the lane that issued them: the same elected lane
-      if (elect_one_sync()) {
+    if (warp == 1) {
+      // the commit tracks the MMAs of the lane that issued them
+      if (leader) {
         umma_commit(&sm.drain);
         const long long t_start = clock64();
         while (!mbar_test(&sm.drain, 0) && clock64() - t_start < kWaitCycles) {

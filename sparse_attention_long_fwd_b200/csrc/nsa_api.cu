@@ -226,7 +226,13 @@ int launch_attn(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap&
   const size_t smem = sizeof(nsa::AttnSmem<D>) + 1024;
   auto kern = nsa::attn_tile_kernel<D, MODE>;
   if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
-  kern<<<dim3(a.n_tiles, a.hkv), nsa::AttnCfg<MODE>::kThreads, smem, st>>>(qm, km, vm, a);
+  // persistent modes: one CTA per SM walks the (tile, group) items; otherwise one CTA per item
+  const long long items = static_cast<long long>(a.n_tiles) * a.hkv;
+  const int sms = sm_count();
+  if (sms <= 0) return NSA_ERR_CUDA;
+  const unsigned grid =
+      static_cast<unsigned>(nsa::AttnCfg<MODE>::kPersistent && items > sms ? sms : items);
+  kern<<<grid, nsa::AttnCfg<MODE>::kThreads, smem, st>>>(qm, km, vm, a);
   return launch_status(MODE == nsa::kModeCmp ? "attn_cmp" : MODE == nsa::kModeWin ? "attn_win" : "attn_dense", st);
 }
 
