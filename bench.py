@@ -38,10 +38,10 @@ from sparse_attention_long_fwd_b200.inputs import WORKLOADS, decode_inputs, pref
 
 METRIC = "NSA prefill video tokens/s at 128K & TFLOP/s vs peak; decode HBM GB/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-PREFILL_STAGES = ["pool", "cmp_attn_scores", "topn", "sel_bucket", "sel_tile", "sel_merge", "win_combine",
+PREFILL_STAGES = ["pool", "cmp_attn_scores", "topn", "sel_bucket", "sel_tile", "win", "sel_merge_combine",
                   "dense_text"]
 # kernels of ours launched per prefill step: pool, compressed tile, top-n, bucket count / scan / scatter,
-# selected partial, merge, window tile (+ the dense text tile)
+# selected tiles, window tile, merge + gated combine (+ the dense text tile)
 PREFILL_KERNELS = 9
 # DRAM bytes per launch of a stage's kernel on the 128K workload, from one ncu capture of the
 # current kernel version (profiles/dram_traffic_v128k.md); an entry is removed when its kernel
@@ -251,7 +251,7 @@ def run_b200(args, world, rank, local):
     # dominant kernel and its roofline (live CUDA-event durations of this run)
     dom = max(stages, key=stages.get)
     stage_flops = {"cmp_attn_scores": counts["cmp_flops"], "sel_tile": counts["sel_flops"],
-                   "win_combine": counts["win_flops"], "dense_text": counts["text_flops"]}
+                   "win": counts["win_flops"], "dense_text": counts["text_flops"]}
     peak_t = peaks["bf16_tflops_sustained"]
     if dom in stage_flops:
         ach = stage_flops[dom] / (stages[dom] / 1e3) / 1e12

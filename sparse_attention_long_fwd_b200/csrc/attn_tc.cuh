@@ -5,8 +5,8 @@
 //              Also bins the normalised probabilities into selection-block scores,
 //              summed over the GQA group (the selection branch's importance scores;
 //              top168.com article on VideoNSA, section "一、革命性的三重注意机制").
-//   kModeWin   sliding-window branch over tokens (t - w, t], followed by the gated
-//              combine out = g_cmp*o_cmp + g_sel*o_sel + g_win*o_win.
+//   kModeWin   sliding-window branch over tokens (t - w, t]: o_win (fp16), which the
+//              selected branch's merge then folds into the gated combine.
 //   kModeDense dense causal rows for the trailing text tokens of the hybrid scheme
 //              (shd-paper.top page "VideoNSA: ...", abstract: dense attention for text).
 //
@@ -35,6 +35,7 @@
 // tile) do the softmax, the score binning and the epilogue. Every wait is bounded (sm100.cuh).
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cstdint>
 #include "sm100.cuh"
 
@@ -51,13 +52,12 @@ struct AttnArgs {
   int cmp_len, cmp_stride;  // compressed-key visibility (kModeCmp)
   int window;              // kModeWin
   int sel_len;             // selection block (kModeCmp scores)
-  float* o_cmp;            // kModeCmp: write [N_v][Hq][d]; kModeWin: read
+  float* o_cmp;            // kModeCmp: write [N_v][Hq][d]
   float* lse;              // kModeCmp: write [N_v][Hq] (natural log)
   float* scores;           // kModeCmp: write [N_v][Hkv][nsel]
   int nsel;
-  const float* o_sel;      // kModeWin: read [N_v][Hq][d]
-  const float* gates;      // kModeWin: read [N][Hq][3]
-  void* out;               // kModeWin / kModeDense: write [N][Hq][d]
+  __half* o_win;           // kModeWin: write [N_v][Hq][d]
+  void* out;               // kModeDense: write [N][Hq][d]
   int out_f32;
 };
 
@@ -80,7 +80,7 @@ struct AttnCfg {
 constexpr int kMaxSoftmaxWG = 4;
 constexpr int kBN = 128;      // keys per tile
 
-template <int D>
+template <int D, int MODE>
 struct AttnSmem {
   static constexpr int kChunks = D / 64;             // 64-element (128 B) column chunks
   static constexpr int kTileBytes = 128 * 128;       // one chunk of a 128-row tile
@@ -203,7 +203,7 @@ template <int D, int MODE>
 __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
     attn_tile_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap vmap, const AttnArgs args) {
-  using Smem = AttnSmem<D>;
+  using Smem = AttnSmem<D, MODE>;
   constexpr int kChunks = Smem::kChunks;
   constexpr int kSoftmaxWG = AttnCfg<MODE>::kWG;
   constexpr int kPairs = AttnCfg<MODE>::kPairs;
@@ -549,18 +549,6 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
           re = t + 1;
         }
       }
-      if (MODE == kModeWin && row_valid) {
-        // the epilogue reads this row's o_cmp, o_sel and gates: start bringing them into L2
-        const size_t orow = (static_cast<size_t>(t) * args.hq + h) * D + wg * (D / kSoftmaxWG);
-#pragma unroll
-        for (int c = 0; c < D / kSoftmaxWG; c += 32) {
-          asm volatile("prefetch.global.L2 [%0];" ::"l"(args.o_cmp + orow + c));
-          asm volatile("prefetch.global.L2 [%0];" ::"l"(args.o_sel + orow + c));
-        }
-        if (wg == 0)
-          asm volatile("prefetch.global.L2 [%0];" ::"l"(args.gates + (static_cast<size_t>(t) * args.hq + h) * 3));
-      }
-
       // ---- phase 1: log-sum-exp (base 2) of this row's column slice, combined below
       float m = -INFINITY, lsum = 0.f;  // m: running max of the raw (unscaled) scores
       for (int kt = kPairs == 1 ? 0 : pair; kt < nkt && ok; kt += kPairs) {
@@ -800,84 +788,88 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_full, it & 1, abort_flag));
         tc_fence_after();
       }
-      if (!ok) {
-        base += nkt;
-        other_pv += (nkt + ((pair ^ 1) == (nkt & 1) ? 1 : 0)) >> 1;
-        continue;
-      }
+      // (after a failed wait the work below is skipped, but the named barrier is still passed)
       const size_t orow = (static_cast<size_t>(t) * args.hq + h) * D;
-      float g0 = 0.f, g1 = 0.f, g2 = 0.f;
-      if (MODE == kModeWin && row_valid) {
-        g0 = args.gates[(static_cast<size_t>(t) * args.hq + h) * 3 + 0];
-        g1 = args.gates[(static_cast<size_t>(t) * args.hq + h) * 3 + 1];
-        g2 = args.gates[(static_cast<size_t>(t) * args.hq + h) * 3 + 2];
-      }
       constexpr int kOC = D / kSoftmaxWG < 32 ? D / kSoftmaxWG : 32;  // output columns per load
       constexpr int kOLoads = (D / kSoftmaxWG + 31) / 32;
       float o[kOLoads][32];
       // O row r, this warpgroup's columns: into registers, then O's TMEM may take the next
       // item's P.V while the stores run
       __syncwarp();
+      if (ok) {
 #pragma unroll
-      for (int cc = 0; cc < kOLoads; ++cc) {
-        const int c0 = wg * (D / kSoftmaxWG) + cc * 32;
-        if (kOC == 32) {
-          tmem_ld32(trow + kColO + c0, o[cc]);
-        } else {
-          tmem_ld16(trow + kColO + c0, *reinterpret_cast<float(*)[16]>(&o[cc][0]));
+        for (int cc = 0; cc < kOLoads; ++cc) {
+          const int c0 = wg * (D / kSoftmaxWG) + cc * 32;
+          if (kOC == 32) {
+            tmem_ld32(trow + kColO + c0, o[cc]);
+          } else {
+            tmem_ld16(trow + kColO + c0, *reinterpret_cast<float(*)[16]>(&o[cc][0]));
+          }
         }
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.o_free);
       }
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.o_free);
-      if (nkt == 0) {
+      if (!ok || nkt == 0) {
 #pragma unroll
         for (int cc = 0; cc < kOLoads; ++cc)
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[cc][i] = 0.f;
       }
+      if constexpr (MODE == kModeWin) {
+        // o_win = O / row sum in fp16, this warpgroup's columns of row r (the gated combine
+        // reads it in the selected branch's merge, whole rows per warp)
+        static_assert(kOC % 8 == 0, "o_win is written in 8-column units");
+        if (ok && row_valid) {
 #pragma unroll
-      for (int cc = 0; cc < kOLoads; ++cc) {
-        const int c0 = wg * (D / kSoftmaxWG) + cc * 32;  // output columns c0 .. c0+kOC-1
-        float* oc_ = o[cc];
-        if (!row_valid) {
-          // nothing to store for padding rows
-        } else if (MODE == kModeCmp) {
-          float4* dst = reinterpret_cast<float4*>(args.o_cmp + orow + c0);
+          for (int cc = 0; cc < kOLoads; ++cc) {
+            const int c0 = wg * (D / kSoftmaxWG) + cc * 32;
+            uint4* dst = reinterpret_cast<uint4*>(args.o_win + orow + c0);
 #pragma unroll
-          for (int u = 0; u < kOC / 4; ++u) dst[u] = make_float4(oc_[4 * u], oc_[4 * u + 1], oc_[4 * u + 2], oc_[4 * u + 3]);
-        } else {
-          if (MODE == kModeWin) {
-            const float4* ocp = reinterpret_cast<const float4*>(args.o_cmp + orow + c0);
-            const float4* osp = reinterpret_cast<const float4*>(args.o_sel + orow + c0);
+            for (int u8 = 0; u8 < kOC / 8; ++u8) {
+              uint4 w4;
+              uint32_t* wp = reinterpret_cast<uint32_t*>(&w4);
 #pragma unroll
-            for (int u = 0; u < kOC / 4; ++u) {
-              const float4 a4 = ocp[u], c4 = osp[u];
-              oc_[4 * u + 0] = g0 * a4.x + g1 * c4.x + g2 * (oc_[4 * u + 0] * inv_l);
-              oc_[4 * u + 1] = g0 * a4.y + g1 * c4.y + g2 * (oc_[4 * u + 1] * inv_l);
-              oc_[4 * u + 2] = g0 * a4.z + g1 * c4.z + g2 * (oc_[4 * u + 2] * inv_l);
-              oc_[4 * u + 3] = g0 * a4.w + g1 * c4.w + g2 * (oc_[4 * u + 3] * inv_l);
+              for (int i = 0; i < 4; ++i) {
+                const __half2 hv =
+                    __floats2half2_rn(o[cc][u8 * 8 + 2 * i] * inv_l, o[cc][u8 * 8 + 2 * i + 1] * inv_l);
+                wp[i] = *reinterpret_cast<const uint32_t*>(&hv);
+              }
+              dst[u8] = w4;
             }
+          }
+        }
+      } else {
+#pragma unroll
+        for (int cc = 0; cc < kOLoads; ++cc) {
+          const int c0 = wg * (D / kSoftmaxWG) + cc * 32;  // output columns c0 .. c0+kOC-1
+          float* oc_ = o[cc];
+          if (!row_valid || !ok) {
+            // nothing to store for padding rows
+          } else if (MODE == kModeCmp) {
+            float4* dst = reinterpret_cast<float4*>(args.o_cmp + orow + c0);
+#pragma unroll
+            for (int u = 0; u < kOC / 4; ++u) dst[u] = make_float4(oc_[4 * u], oc_[4 * u + 1], oc_[4 * u + 2], oc_[4 * u + 3]);
           } else {
 #pragma unroll
             for (int u = 0; u < kOC; ++u) oc_[u] *= inv_l;
-          }
-          if (args.out_f32) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.out) + orow + c0);
+            if (args.out_f32) {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.out) + orow + c0);
 #pragma unroll
-            for (int u = 0; u < kOC / 4; ++u)
-              dst[u] = make_float4(oc_[4 * u], oc_[4 * u + 1], oc_[4 * u + 2], oc_[4 * u + 3]);
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) + orow + c0);
+              for (int u = 0; u < kOC / 4; ++u)
+                dst[u] = make_float4(oc_[4 * u], oc_[4 * u + 1], oc_[4 * u + 2], oc_[4 * u + 3]);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) + orow + c0);
 #pragma unroll
-            for (int u = 0; u < kOC / 8; ++u)
-              dst[u] = make_uint4(pack_bf16x2(oc_[8 * u], oc_[8 * u + 1]), pack_bf16x2(oc_[8 * u + 2], oc_[8 * u + 3]),
-                                  pack_bf16x2(oc_[8 * u + 4], oc_[8 * u + 5]), pack_bf16x2(oc_[8 * u + 6], oc_[8 * u + 7]));
+              for (int u = 0; u < kOC / 8; ++u)
+                dst[u] = make_uint4(pack_bf16x2(oc_[8 * u], oc_[8 * u + 1]), pack_bf16x2(oc_[8 * u + 2], oc_[8 * u + 3]),
+                                    pack_bf16x2(oc_[8 * u + 4], oc_[8 * u + 5]), pack_bf16x2(oc_[8 * u + 6], oc_[8 * u + 7]));
+            }
           }
         }
       }
-      if (MODE == kModeCmp && row_valid && wg == 0)
+      if (MODE == kModeCmp && ok && row_valid && wg == 0)
         args.lse[static_cast<size_t>(t) * args.hq + h] = has_keys ? lse2 * 0.69314718055994530942f : -INFINITY;
       base += nkt;
       other_pv += (nkt + ((pair ^ 1) == (nkt & 1) ? 1 : 0)) >> 1;

@@ -73,7 +73,7 @@ int check_device() {
 }
 
 struct PrefillLayout {
-  size_t kc, vc, o_cmp, lse, scores, sel_idx, o_sel, total;
+  size_t kc, vc, o_cmp, lse, scores, sel_idx, o_win, total;
   // block-major selected branch: bucket counters, offsets, bucketed entries, partials
   size_t sel_cnt, sel_eoff, sel_toff, sel_list, sel_row, part_o, part_ml;
   long long part_rows;  // 128 x the bound on selected-branch tiles
@@ -98,7 +98,7 @@ PrefillLayout prefill_layout(const nsa_params_t* p) {
   L.lse = take(static_cast<size_t>(nv) * hq * 4);
   L.scores = take(static_cast<size_t>(nv) * hkv * (L.nsel > 0 ? L.nsel : 1) * 4);
   L.sel_idx = take(static_cast<size_t>(nv) * hkv * p->top_n * 4);
-  L.o_sel = take(static_cast<size_t>(nv) * hq * d * 4);
+  L.o_win = take(static_cast<size_t>(nv) * hq * d * 2);
   const size_t buckets = static_cast<size_t>(hkv) * (L.nsel > 0 ? L.nsel : 1);
   const size_t entries = static_cast<size_t>(nv) * hkv * p->top_n;
   L.sel_cnt = take(2 * buckets * 4);
@@ -223,7 +223,7 @@ template <int D, int MODE>
 int launch_attn(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a,
                 cudaStream_t st) {
   if (a.n_tiles <= 0) return NSA_OK;
-  const size_t smem = sizeof(nsa::AttnSmem<D>) + 1024;
+  const size_t smem = sizeof(nsa::AttnSmem<D, MODE>) + 1024;
   auto kern = nsa::attn_tile_kernel<D, MODE>;
   if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
   // persistent modes: one CTA per SM walks the (tile, group) items; otherwise one CTA per item
@@ -335,7 +335,11 @@ int prefill_impl(const nsa_params_t* p, const void* q, const void* k, const void
       sa.part_rows = L.part_rows;
       sa.part_o = reinterpret_cast<const __half*>(ws + L.part_o);
       sa.part_ml = reinterpret_cast<float4*>(ws + L.part_ml);
-      sa.o_sel = reinterpret_cast<float*>(ws + L.o_sel);
+      sa.o_cmp = reinterpret_cast<const float*>(ws + L.o_cmp);
+      sa.o_win = reinterpret_cast<const __half*>(ws + L.o_win);
+      sa.gates = gates;
+      sa.out = out;
+      sa.out_f32 = p->out_dtype == NSA_OUT_F32;
       sa.q = static_cast<const __nv_bfloat16*>(q);
       CUtensorMap k64map, v64map, omap;
       if (!nsa::make_tmap_f16_3d(&omap, ws + L.part_o, 64, static_cast<uint64_t>(L.part_rows), D / 64, 128,
@@ -364,16 +368,16 @@ int prefill_impl(const nsa_params_t* p, const void* q, const void* k, const void
       const unsigned grid = static_cast<unsigned>(max_tiles < nsm ? max_tiles : nsm);
       kern<<<grid, nsa::kSelTileThreads, smem, st>>>(k64map, v64map, omap, sa);
       if ((rc = launch_status("sel_tile", st)) != NSA_OK) return rc;
+      // 5. sliding window -> o_win
+      a.o_win = reinterpret_cast<__half*>(ws + L.o_win);
+      if ((rc = launch_attn<D, nsa::kModeWin>(qmap, kmap, vmap, a, st)) != NSA_OK) return rc;
+      // 6. merge of the selected partials + gated combine -> out rows [0, N_v)
       const long long rows = static_cast<long long>(nv) * hq;
       nsa::sel_merge_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(sa);
       if ((rc = launch_status("sel_merge", st)) != NSA_OK) return rc;
     }
-    // 5. sliding window + gated combine -> out rows [0, N_v)
-    a.o_sel = reinterpret_cast<const float*>(ws + L.o_sel);
-    a.gates = gates;
-    if ((rc = launch_attn<D, nsa::kModeWin>(qmap, kmap, vmap, a, st)) != NSA_OK) return rc;
   }
-  // 6. trailing text rows: dense causal attention -> out rows [N_v, N)
+  // 7. trailing text rows: dense causal attention -> out rows [N_v, N)
   if (N > nv) {
     a.q_begin = nv;
     a.q_end = N;
@@ -512,7 +516,7 @@ int nsa_prefill_workspace_layout(const nsa_params_t* params, nsa_prefill_layout_
   layout->lse = L.lse;
   layout->scores = L.scores;
   layout->sel_idx = L.sel_idx;
-  layout->o_sel = L.o_sel;
+  layout->o_win = L.o_win;
   layout->total = L.total;
   layout->n_cmp = L.ncmp;
   layout->n_sel = L.nsel;

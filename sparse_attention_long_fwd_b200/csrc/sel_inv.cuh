@@ -21,7 +21,8 @@
 //   sel_scan_kernel     exclusive scans of entries and of tiles per (group, block)
 //   sel_scatter_kernel  bucket (token, slot) pairs
 //   sel_tile_kernel     persistent 128-row tcgen05 tiles: S = Q K^T, softmax, O = P V
-//   sel_merge_kernel    o_sel[t][h] from the row's partials
+//   sel_merge_kernel    o_sel[t][h] from the row's partials, then the gated combine
+//                       out = g_cmp*o_cmp + g_sel*o_sel + g_win*o_win (o_sel is not stored)
 #pragma once
 #include <cuda_fp16.h>
 #include "attn_tc.cuh"
@@ -43,7 +44,11 @@ struct SelInvArgs {
   long long part_rows;          // rows per 64-column half of part_o (128 x the tile bound)
   const __half* part_o;         // [D/64][part_rows][64] output / (sum * c_half) of each partial
   float4* part_ml;              // [part_rows] (max in log2 units, sum, c of half 0, c of half 1)
-  float* o_sel;                 // [nv][hq][D]
+  const float* o_cmp;           // [nv][hq][D] compressed branch
+  const __half* o_win;          // [nv][hq][D] sliding-window branch
+  const float* gates;           // [N][hq][3] (g_cmp, g_sel, g_win)
+  void* out;                    // [N][hq][D] rows < nv: the gated combine, bf16 or fp32
+  int out_f32;
 };
 
 // Block 0 is kept by every token, so its buckets take one entry per token of their group:
@@ -641,6 +646,26 @@ __global__ void __launch_bounds__(256, 3) sel_merge_kernel(const SelInvArgs a) {
   const int t = static_cast<int>(row / a.hq), h = static_cast<int>(row % a.hq);
   const int g = h / a.G, hh = h - g * a.G;
   const size_t base = (static_cast<size_t>(t) * a.hkv + g) * a.top_n;
+  // the combine's other inputs go out first: their latency overlaps the partials' loads
+  const size_t orow = static_cast<size_t>(row) * D + lane * kPer;
+  const float gc = __ldg(a.gates + static_cast<size_t>(row) * 3 + 0);
+  const float gs = __ldg(a.gates + static_cast<size_t>(row) * 3 + 1);
+  const float gw = __ldg(a.gates + static_cast<size_t>(row) * 3 + 2);
+  float oc[kPer], ow[kPer];
+  if constexpr (kPer == 4) {
+    const float4 c4 = __ldg(reinterpret_cast<const float4*>(a.o_cmp + orow));
+    const uint2 w2 = __ldg(reinterpret_cast<const uint2*>(a.o_win + orow));
+    oc[0] = c4.x; oc[1] = c4.y; oc[2] = c4.z; oc[3] = c4.w;
+    const float2 wa = __half22float2(*reinterpret_cast<const __half2*>(&w2.x));
+    const float2 wb = __half22float2(*reinterpret_cast<const __half2*>(&w2.y));
+    ow[0] = wa.x; ow[1] = wa.y; ow[2] = wb.x; ow[3] = wb.y;
+  } else {
+    const float2 c2 = __ldg(reinterpret_cast<const float2*>(a.o_cmp + orow));
+    const uint32_t w1 = __ldg(reinterpret_cast<const unsigned int*>(a.o_win + orow));
+    oc[0] = c2.x; oc[1] = c2.y;
+    const float2 wa = __half22float2(*reinterpret_cast<const __half2*>(&w1));
+    ow[0] = wa.x; ow[1] = wa.y;
+  }
   // lane s holds slot s (and s + 32): its partial row, or -1; top_n <= 64
   int r0 = -1, r1 = -1;
   if (lane < a.top_n) {
@@ -708,11 +733,22 @@ __global__ void __launch_bounds__(256, 3) sel_merge_kernel(const SelInvArgs a) {
     }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
-  float* dst = a.o_sel + static_cast<size_t>(row) * D + lane * kPer;
-  if constexpr (kPer == 4)
-    *reinterpret_cast<float4*>(dst) = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-  else
-    *reinterpret_cast<float2*>(dst) = make_float2(acc[0] * inv, acc[1] * inv);
+  float res[kPer];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) res[u] = gc * oc[u] + gs * (acc[u] * inv) + gw * ow[u];
+  if (a.out_f32) {
+    float* dst = static_cast<float*>(a.out) + orow;
+    if constexpr (kPer == 4)
+      *reinterpret_cast<float4*>(dst) = make_float4(res[0], res[1], res[2], res[3]);
+    else
+      *reinterpret_cast<float2*>(dst) = make_float2(res[0], res[1]);
+  } else {
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + orow;
+    if constexpr (kPer == 4)
+      *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(res[0], res[1]), pack_bf16x2(res[2], res[3]));
+    else
+      *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(res[0], res[1]);
+  }
 }
 
 }  // namespace nsa

@@ -100,6 +100,8 @@ def compare_prefill_rows(w: Workload, q, k, v, gates, rows, out, sel, ws, layout
         if len(vrows):
             ocmp = ws_view(ws, layout["o_cmp"], (w.n_video, w.hq, w.d), torch.float32)[vrows].cpu().numpy()
             stats["o_cmp"] = assert_close(ocmp, o["o_cmp"][vid], "o_cmp")
+            owin = ws_view(ws, layout["o_win"], (w.n_video, w.hq, w.d), torch.float16)[vrows].float().cpu().numpy()
+            stats["o_win"] = assert_close(owin, o["o_win"][vid], "o_win")
             lse = ws_view(ws, layout["lse"], (w.n_video, w.hq), torch.float32)[vrows].cpu().numpy()
             fin = np.isfinite(o["lse"][vid])
             assert np.array_equal(np.isfinite(lse), fin)
@@ -123,10 +125,6 @@ def compare_prefill_rows(w: Workload, q, k, v, gates, rows, out, sel, ws, layout
             o2 = orc.prefill_rows(cfg, qb, kb, vb, g, rr, kc=kc_o, vc=vc_o, sel_override=gsel[replay],
                                   want=("o_sel",), nthreads=nthreads)
             ref[vidx[replay]] = o2["out"]
-            o["o_sel"][vidx[replay]] = o2["o_sel"]
-        if check_intermediates:
-            osel = ws_view(ws, layout["o_sel"], (w.n_video, w.hq, w.d), torch.float32)[vrows].cpu().numpy()
-            stats["o_sel"] = assert_close(osel, o["o_sel"][vid], "o_sel")
     if out.dtype == torch.float32:
         stats["out"] = assert_close(out_h, ref, "out")
     else:

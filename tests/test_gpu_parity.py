@@ -93,12 +93,21 @@ def test_prefill_one_hot_gates_isolate_branches():
         gg = torch.zeros_like(g)
         gg[..., which] = 1.0
         out, sel, ws, lay = run_prefill(w, q, k, v, gg)
-        outs.append((out.clone(), ws, lay))
-    from nsa_check import ws_view
+        outs.append((out.clone(), ws, lay, sel.clone()))
+    from nsa_check import ws_view, host_bits
     ocmp = ws_view(outs[0][1], outs[0][2]["o_cmp"], (700, w.hq, w.d), torch.float32)
-    osel = ws_view(outs[1][1], outs[1][2]["o_sel"], (700, w.hq, w.d), torch.float32)
+    owin = ws_view(outs[2][1], outs[2][2]["o_win"], (700, w.hq, w.d), torch.float16)
     assert torch.equal(outs[0][0], ocmp)
-    assert torch.equal(outs[1][0], osel)
+    assert torch.equal(outs[2][0], owin.float())
+    # the selected branch is never stored on its own: with g_sel = 1 the output is o_sel,
+    # checked against the oracle on the blocks this run selected (near-ties may differ)
+    qb, kb, vb = host_bits(q, k, v)
+    rows = np.arange(0, 700, 7, dtype=np.int32)
+    gg = torch.zeros_like(g)
+    gg[..., 1] = 1.0
+    o = orc.prefill_rows(oracle_cfg(w), qb, kb, vb, gg.cpu().numpy(), rows,
+                         sel_override=outs[1][3][rows].cpu().numpy(), want=("o_sel",))
+    assert_close(outs[1][0][rows].cpu().numpy(), o["o_sel"], "o_sel through g_sel = 1")
 
 
 def test_prefill_qwen36k_hybrid_sampled():
