@@ -46,7 +46,7 @@ PREFILL_KERNELS = 9
 # DRAM bytes per launch of a stage's kernel on the 128K workload, from one ncu capture of the
 # current kernel version (profiles/dram_traffic_v128k.md); an entry is removed when its kernel
 # changes, and the roofline then reports traffic null.
-STAGE_TRAFFIC_V128K = {"cmp_attn_scores": 1118705408 + 4013818880}
+STAGE_TRAFFIC_V128K = {"cmp_attn_scores": 4989331456}
 DECODE_STAGES = ["dec_cmp", "dec_select", "dec_branches", "dec_combine"]
 
 
@@ -362,7 +362,7 @@ def run_b200(args, world, rank, local):
 
     if not args.no_decode:
         result["decode"] = run_decode(args, dev, peaks, peaks_src, flush, world)
-        result["gpu_launches"] += 4 * args.steps
+        result["gpu_launches"] += 4 * result["decode"]["steps"]
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, q, k, v, g, args.cpu_seconds)
