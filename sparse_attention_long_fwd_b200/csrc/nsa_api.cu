@@ -298,13 +298,17 @@ int prefill_impl(const nsa_params_t* p, const void* q, const void* k, const void
     {
       const int nitems = nv * hkv;
       const int nwords = (L.nsel + 31) / 32;
-      const size_t smem = static_cast<size_t>(nsa::kTopnWarps) * (2 * L.nsel + nwords) * 4;
-      if (set_smem(nsa::topn_kernel, smem) != NSA_OK) return NSA_ERR_CUDA;
+      // every row on the register path (fewer than 2,048 blocks, top_n <= 32): 64 list
+      // entries per warp, so shared memory does not limit the warps per SM
+      const bool regs_only = L.nsel <= 32 * 64 && p->top_n <= 32;
+      const size_t smem =
+          static_cast<size_t>(nsa::kTopnWarps) * (regs_only ? 64 : 2 * L.nsel + nwords) * 4;
+      auto kern = regs_only ? nsa::topn_kernel<true> : nsa::topn_kernel<false>;
+      if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
       int blocks = (nitems + nsa::kTopnWarps - 1) / nsa::kTopnWarps;
       if (blocks > 148 * 32) blocks = 148 * 32;
-      nsa::topn_kernel<<<blocks, nsa::kTopnWarps * 32, smem, st>>>(
-          a.scores, nitems, hkv, L.nsel, p->sel_block, p->top_n, reinterpret_cast<int32_t*>(ws + L.sel_idx),
-          out_sel_idx);
+      kern<<<blocks, nsa::kTopnWarps * 32, smem, st>>>(a.scores, nitems, hkv, L.nsel, p->sel_block, p->top_n,
+                                                        reinterpret_cast<int32_t*>(ws + L.sel_idx), out_sel_idx);
       if ((rc = launch_status("topn", st)) != NSA_OK) return rc;
     }
     // 4. selected branch, block-major: bucket (token, slot) pairs by (group, block),

@@ -157,8 +157,10 @@ __device__ __forceinline__ void warp_topn(float* sc, uint32_t* bits, int* list, 
 // non-negative. Warp-wide maxima are single __reduce_max_sync instructions.
 //   1. each lane's two half-slice maxima: the k-th largest of those 64 keys is a lower
 //      bound on the k-th largest key overall (they are distinct blocks of the row);
-//   2. candidates at or above that bound are compacted to `list` (as block indices);
-//   3. k rounds take the largest key among them, the smallest block index on ties.
+//   2. candidates at or above that bound are compacted to `list` (block indices; the first
+//      64 are kept, `list` holds 64 ints);
+//   3. k rounds take the largest key among them, the smallest block index on ties (from the
+//      list when at most 64 survived, else by scanning the candidates again).
 template <int PL>
 __device__ __forceinline__ void warp_topn_regs(int* list, const float* __restrict__ src, int jt, int top_n,
                                                int32_t* __restrict__ dst, int32_t* __restrict__ dst2, int lane) {
@@ -201,9 +203,16 @@ __device__ __forceinline__ void warp_topn_regs(int* list, const float* __restric
       }
     }
     // 2. compact the candidates with key >= thr (block indices, in lane-slot order)
-    int cnt = 0;
+    static_assert(PL <= 64, "candidate bits");
+    uint32_t cand = 0u, cand_hi = 0u;  // bit u (u - 32): block lane + 32u is a candidate
 #pragma unroll
-    for (int u = 0; u < PL; ++u) cnt += (key[u] != 0u && key[u] >= thr) ? 1 : 0;
+    for (int u = 0; u < PL; ++u) {
+      if (key[u] != 0u && key[u] >= thr) {
+        if (u < 32) cand |= 1u << (u & 31);
+        else cand_hi |= 1u << (u & 31);
+      }
+    }
+    const int cnt = __popc(cand) + __popc(cand_hi);
     int off = cnt;  // inclusive scan over lanes
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -213,8 +222,13 @@ __device__ __forceinline__ void warp_topn_regs(int* list, const float* __restric
     const int nsurv = __shfl_sync(0xffffffffu, off, 31);
     off -= cnt;
 #pragma unroll
-    for (int u = 0; u < PL; ++u)
-      if (key[u] != 0u && key[u] >= thr) list[off++] = lane + 32 * u;
+    for (int u = 0; u < PL; ++u) {
+      const bool c = u < 32 ? ((cand >> (u & 31)) & 1u) : ((cand_hi >> (u & 31)) & 1u);
+      if (c) {
+        if (off < 64) list[off] = lane + 32 * u;  // the exact pass below needs only 64
+        ++off;
+      }
+    }
     __syncwarp();
     // 3. exact top-k among them: largest key, smallest block index on ties; the winner of
     //    round r goes to lane nf + r
@@ -234,24 +248,30 @@ __device__ __forceinline__ void warp_topn_regs(int* list, const float* __restric
         if (lane == nf + round) mine = static_cast<int>(jw);
       }
     } else {
-      // many ties at the bound: rounds over the compacted list (keys reloaded by block)
+      // many ties at the bound (rare): rounds over the candidate bits, the keys read again
+      // from the row (the list holds only the first 64 candidates)
       for (int round = 0; round < k; ++round) {
         uint32_t best = 0u, bj = 0xFFFFFFFFu;
-        for (int i = lane; i < nsurv; i += 32) {
-          const int j = list[i];
-          const uint32_t x = (j >= 0 && src[j] >= 0.f) ? __float_as_uint(src[j]) + 1u : 0u;
-          if (x > best || (x == best && x != 0u && static_cast<uint32_t>(j) < bj)) {
-            best = x;
-            bj = static_cast<uint32_t>(j);
+        for (int u = 0; u < PL; ++u) {  // slots in block order: the first maximum has the lowest index
+          const bool c = u < 32 ? ((cand >> (u & 31)) & 1u) : ((cand_hi >> (u & 31)) & 1u);
+          if (c) {
+            const float x = src[lane + 32 * u];
+            const uint32_t kx = __float_as_uint(x) + 1u;
+            if (kx > best) {
+              best = kx;
+              bj = static_cast<uint32_t>(lane + 32 * u);
+            }
           }
         }
         const uint32_t w = __reduce_max_sync(0xffffffffu, best);
         if (w == 0u) break;
         const uint32_t jw = __reduce_min_sync(0xffffffffu, best == w ? bj : 0xFFFFFFFFu);
-        for (int i = lane; i < nsurv; i += 32)
-          if (list[i] == static_cast<int>(jw)) list[i] = -1;
+        if (static_cast<int>(jw & 31u) == lane) {  // taken: clear its candidate bit
+          const int u = static_cast<int>(jw >> 5);
+          if (u < 32) cand &= ~(1u << u);
+          else cand_hi &= ~(1u << (u - 32));
+        }
         if (lane == nf + round) mine = static_cast<int>(jw);
-        __syncwarp();
       }
     }
   }
@@ -276,6 +296,11 @@ __device__ __forceinline__ void warp_topn_regs(int* list, const float* __restric
 
 // scores: [nitems][nsel] fp32 (item = row * hkv + g); idx / idx_copy: [nitems][top_n].
 // Row position t = row (prefill rows are token positions).
+// One warp per (row, group). kRegsOnly: every row has fewer than 2,048 candidate blocks and
+// top_n <= 32 (checked by the host), so only the register path runs and each warp needs just
+// the 64-entry candidate list in shared memory; otherwise each warp also has the score row,
+// the list and the bitmap of the shared-memory path.
+template <bool kRegsOnly>
 __global__ void __launch_bounds__(kTopnWarps * 32) topn_kernel(const float* __restrict__ scores, int nitems, int hkv,
                                                                 int nsel, int sel_len, int top_n,
                                                                 int32_t* __restrict__ idx,
@@ -283,20 +308,21 @@ __global__ void __launch_bounds__(kTopnWarps * 32) topn_kernel(const float* __re
   extern __shared__ float tsm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwords = (nsel + 31) / 32;
-  float* sc = tsm + static_cast<size_t>(warp) * (2 * nsel + nwords);
-  int* list = reinterpret_cast<int*>(sc + nsel);
+  float* sc = tsm + static_cast<size_t>(warp) * (kRegsOnly ? 64 : 2 * nsel + nwords);
+  int* list = kRegsOnly ? reinterpret_cast<int*>(sc) : reinterpret_cast<int*>(sc + nsel);
   uint32_t* bits = reinterpret_cast<uint32_t*>(list + nsel);
   for (int item = blockIdx.x * kTopnWarps + warp; item < nitems; item += gridDim.x * kTopnWarps) {
     const int t = item / hkv;
     const int jt = t / sel_len;
-    if (jt >= nsel) {  // cannot happen for valid arguments; never index past the row
+    if (jt >= nsel || (kRegsOnly && (top_n > 32 || jt >= 32 * 64))) {
+      // cannot happen for valid arguments; never index past the row
       if (lane == 0) record_error(kErrBadIndex);
       continue;
     }
     const float* src = scores + static_cast<size_t>(item) * nsel;
     int32_t* d = idx + static_cast<size_t>(item) * top_n;
     int32_t* d2 = idx_copy ? idx_copy + static_cast<size_t>(item) * top_n : nullptr;
-    if (top_n > 32 || jt >= 32 * 64) warp_topn(sc, bits, list, src, jt, top_n, d, d2, lane);
+    if (!kRegsOnly && (top_n > 32 || jt >= 32 * 64)) warp_topn(sc, bits, list, src, jt, top_n, d, d2, lane);
     else if (jt < 32 * 4) warp_topn_regs<4>(list, src, jt, top_n, d, d2, lane);
     else if (jt < 32 * 16) warp_topn_regs<16>(list, src, jt, top_n, d, d2, lane);
     else if (jt < 32 * 32) warp_topn_regs<32>(list, src, jt, top_n, d, d2, lane);

@@ -110,6 +110,20 @@ def test_prefill_one_hot_gates_isolate_branches():
     assert_close(outs[1][0][rows].cpu().numpy(), o["o_sel"], "o_sel through g_sel = 1")
 
 
+@pytest.mark.parametrize("n", [9000, 40000])
+def test_prefill_constant_keys_exact_ties(n):
+    """Every key equal: the compressed probabilities are uniform, so all interior selection
+    blocks tie exactly (in fp32 here and in fp64 in the oracle) and thousands of candidates
+    sit at the top-n bound; the lower block index must win every tie."""
+    w = scaled(WORKLOADS["v128k"], n_tokens=n, n_video=n)
+    q, k, v, g = prefill_inputs(w, seed=13, device=DEV)
+    k = k[:1].expand_as(k).contiguous()
+    out, sel, ws, lay = run_prefill(w, q, k, v, g)
+    rows = np.unique(np.concatenate([np.arange(0, n, 97), np.arange(n - 64, n)])).astype(np.int32)
+    st = compare_prefill_rows(w, q, k, v, g, rows, out, sel, ws, lay)
+    assert st["ties"] == 0, st  # exact ties resolve the same way on both sides
+
+
 def test_prefill_qwen36k_hybrid_sampled():
     w = WORKLOADS["qwen36k_hybrid"]
     q, k, v, g = prefill_inputs(w, seed=1, device=DEV)
