@@ -170,7 +170,7 @@ size_t nsa_workspace_size(const nsa_params_t* params, int is_decode);
  * Where nsa_prefill keeps its intermediates inside the workspace (byte offsets), for
  * inspection after the stream has been synchronised. Every field is an offset from the
  * workspace base; layouts are row-major:
- *   kc, vc   [Ncmp(N_v)][Hkv][d] bf16     o_cmp [N_v][Hq][d] fp32     lse [N_v][Hq] fp32 (natural log)
+ *   kc, vc   [Ncmp(N_v)][Hkv][d] bf16     o_cmp [N_v][Hq][d] fp16     lse [N_v][Hq] fp32 (natural log)
  *   scores   [N_v][Hkv][Nsel] fp32, Nsel = ceil(N_v / l'); only entries j <= t/l' are written
  *   sel_idx  [N_v][Hkv][top_n] int32      o_win [N_v][Hq][d] fp16 (window branch)
  * The selected branch's output goes straight into the gated combine and is not kept.

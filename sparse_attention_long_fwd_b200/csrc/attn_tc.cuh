@@ -52,7 +52,7 @@ struct AttnArgs {
   int cmp_len, cmp_stride;  // compressed-key visibility (kModeCmp)
   int window;              // kModeWin
   int sel_len;             // selection block (kModeCmp scores)
-  float* o_cmp;            // kModeCmp: write [N_v][Hq][d]
+  __half* o_cmp;           // kModeCmp: write [N_v][Hq][d]
   float* lse;              // kModeCmp: write [N_v][Hq] (natural log)
   float* scores;           // kModeCmp: write [N_v][Hkv][nsel]
   int nsel;
@@ -848,9 +848,18 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
           if (!row_valid || !ok) {
             // nothing to store for padding rows
           } else if (MODE == kModeCmp) {
-            float4* dst = reinterpret_cast<float4*>(args.o_cmp + orow + c0);
+            uint4* dst = reinterpret_cast<uint4*>(args.o_cmp + orow + c0);
 #pragma unroll
-            for (int u = 0; u < kOC / 4; ++u) dst[u] = make_float4(oc_[4 * u], oc_[4 * u + 1], oc_[4 * u + 2], oc_[4 * u + 3]);
+            for (int u = 0; u < kOC / 8; ++u) {
+              uint4 w4;
+              uint32_t* wp = reinterpret_cast<uint32_t*>(&w4);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const __half2 hv = __floats2half2_rn(oc_[8 * u + 2 * i], oc_[8 * u + 2 * i + 1]);
+                wp[i] = *reinterpret_cast<const uint32_t*>(&hv);
+              }
+              dst[u] = w4;
+            }
           } else {
 #pragma unroll
             for (int u = 0; u < kOC; ++u) oc_[u] *= inv_l;

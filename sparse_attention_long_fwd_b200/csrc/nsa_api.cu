@@ -94,7 +94,7 @@ PrefillLayout prefill_layout(const nsa_params_t* p) {
   const size_t cmp_rows = static_cast<size_t>(L.ncmp > 0 ? L.ncmp : 1);
   L.kc = take(cmp_rows * hkv * d * 2);
   L.vc = take(cmp_rows * hkv * d * 2);
-  L.o_cmp = take(static_cast<size_t>(nv) * hq * d * 4);
+  L.o_cmp = take(static_cast<size_t>(nv) * hq * d * 2);
   L.lse = take(static_cast<size_t>(nv) * hq * 4);
   L.scores = take(static_cast<size_t>(nv) * hkv * (L.nsel > 0 ? L.nsel : 1) * 4);
   L.sel_idx = take(static_cast<size_t>(nv) * hkv * p->top_n * 4);
@@ -283,7 +283,7 @@ int prefill_impl(const nsa_params_t* p, const void* q, const void* k, const void
     // 2. compressed branch + block scores
     a.q_begin = 0;
     a.q_end = nv;
-    a.o_cmp = reinterpret_cast<float*>(ws + L.o_cmp);
+    a.o_cmp = reinterpret_cast<__half*>(ws + L.o_cmp);
     a.lse = reinterpret_cast<float*>(ws + L.lse);
     a.scores = reinterpret_cast<float*>(ws + L.scores);
     {
@@ -339,7 +339,7 @@ int prefill_impl(const nsa_params_t* p, const void* q, const void* k, const void
       sa.part_rows = L.part_rows;
       sa.part_o = reinterpret_cast<const __half*>(ws + L.part_o);
       sa.part_ml = reinterpret_cast<float4*>(ws + L.part_ml);
-      sa.o_cmp = reinterpret_cast<const float*>(ws + L.o_cmp);
+      sa.o_cmp = reinterpret_cast<const __half*>(ws + L.o_cmp);
       sa.o_win = reinterpret_cast<const __half*>(ws + L.o_win);
       sa.gates = gates;
       sa.out = out;

@@ -44,7 +44,7 @@ struct SelInvArgs {
   long long part_rows;          // rows per 64-column half of part_o (128 x the tile bound)
   const __half* part_o;         // [D/64][part_rows][64] output / (sum * c_half) of each partial
   float4* part_ml;              // [part_rows] (max in log2 units, sum, c of half 0, c of half 1)
-  const float* o_cmp;           // [nv][hq][D] compressed branch
+  const __half* o_cmp;          // [nv][hq][D] compressed branch
   const __half* o_win;          // [nv][hq][D] sliding-window branch
   const float* gates;           // [N][hq][3] (g_cmp, g_sel, g_win)
   void* out;                    // [N][hq][D] rows < nv: the gated combine, bf16 or fp32
@@ -653,16 +653,19 @@ __global__ void __launch_bounds__(256, 3) sel_merge_kernel(const SelInvArgs a) {
   const float gw = __ldg(a.gates + static_cast<size_t>(row) * 3 + 2);
   float oc[kPer], ow[kPer];
   if constexpr (kPer == 4) {
-    const float4 c4 = __ldg(reinterpret_cast<const float4*>(a.o_cmp + orow));
+    const uint2 c2 = __ldg(reinterpret_cast<const uint2*>(a.o_cmp + orow));
     const uint2 w2 = __ldg(reinterpret_cast<const uint2*>(a.o_win + orow));
-    oc[0] = c4.x; oc[1] = c4.y; oc[2] = c4.z; oc[3] = c4.w;
+    const float2 ca = __half22float2(*reinterpret_cast<const __half2*>(&c2.x));
+    const float2 cb = __half22float2(*reinterpret_cast<const __half2*>(&c2.y));
+    oc[0] = ca.x; oc[1] = ca.y; oc[2] = cb.x; oc[3] = cb.y;
     const float2 wa = __half22float2(*reinterpret_cast<const __half2*>(&w2.x));
     const float2 wb = __half22float2(*reinterpret_cast<const __half2*>(&w2.y));
     ow[0] = wa.x; ow[1] = wa.y; ow[2] = wb.x; ow[3] = wb.y;
   } else {
-    const float2 c2 = __ldg(reinterpret_cast<const float2*>(a.o_cmp + orow));
+    const uint32_t c1 = __ldg(reinterpret_cast<const unsigned int*>(a.o_cmp + orow));
     const uint32_t w1 = __ldg(reinterpret_cast<const unsigned int*>(a.o_win + orow));
-    oc[0] = c2.x; oc[1] = c2.y;
+    const float2 ca = __half22float2(*reinterpret_cast<const __half2*>(&c1));
+    oc[0] = ca.x; oc[1] = ca.y;
     const float2 wa = __half22float2(*reinterpret_cast<const __half2*>(&w1));
     ow[0] = wa.x; ow[1] = wa.y;
   }

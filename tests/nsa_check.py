@@ -98,7 +98,7 @@ def compare_prefill_rows(w: Workload, q, k, v, gates, rows, out, sel, ws, layout
             vc_g = bf16_bits(ws_view(ws, layout["vc"], (nc, w.hkv, w.d), torch.bfloat16))
             assert np.array_equal(kc_g, kc_o) and np.array_equal(vc_g, vc_o), "compressed K/V not bit-exact"
         if len(vrows):
-            ocmp = ws_view(ws, layout["o_cmp"], (w.n_video, w.hq, w.d), torch.float32)[vrows].cpu().numpy()
+            ocmp = ws_view(ws, layout["o_cmp"], (w.n_video, w.hq, w.d), torch.float16)[vrows].float().cpu().numpy()
             stats["o_cmp"] = assert_close(ocmp, o["o_cmp"][vid], "o_cmp")
             owin = ws_view(ws, layout["o_win"], (w.n_video, w.hq, w.d), torch.float16)[vrows].float().cpu().numpy()
             stats["o_win"] = assert_close(owin, o["o_win"][vid], "o_win")

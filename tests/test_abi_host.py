@@ -82,7 +82,7 @@ def test_prefill_layout_is_aligned_and_disjoint():
         keys = ["kc", "vc", "o_cmp", "lse", "scores", "sel_idx", "o_win"]
         offs = [lay[k] for k in keys] + [lay["total"]]
         assert all(o % 256 == 0 for o in offs)
-        sizes = [max(ncmp, 1) * 4 * 128 * 2] * 2 + [nv * 28 * 128 * 4, nv * 28 * 4, nv * 4 * max(lay["n_sel"], 1) * 4,
+        sizes = [max(ncmp, 1) * 4 * 128 * 2] * 2 + [nv * 28 * 128 * 2, nv * 28 * 4, nv * 4 * max(lay["n_sel"], 1) * 4,
                                                     nv * 4 * 16 * 4, nv * 28 * 128 * 2]
         for i, sz in enumerate(sizes):
             assert offs[i] + sz <= offs[i + 1], keys[i]
