@@ -638,7 +638,7 @@ __device__ __forceinline__ float warp_sum(float x) {
 // (l * D/32) / 64 of the partial rows. The partial rows are loaded as soon as their row
 // numbers are known, alongside the (max, sum) records that weight them.
 template <int D>
-__global__ void __launch_bounds__(256, 3) sel_merge_kernel(const SelInvArgs a) {
+__global__ void __launch_bounds__(256, 4) sel_merge_kernel(const SelInvArgs a) {
   constexpr int kPer = D / 32;
   const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -691,12 +691,14 @@ __global__ void __launch_bounds__(256, 3) sel_merge_kernel(const SelInvArgs a) {
 #pragma unroll
   for (int u = 0; u < kPer; ++u) acc[u] = 0.f;
   float M = -INFINITY, w0 = 0.f, w1 = 0.f, L = 0.f;
-  for (int s0 = 0; s0 < a.top_n; s0 += 16) {
+  // partial rows in batches of kMB slots: their loads go out together
+  constexpr int kMB = 8;
+  for (int s0 = 0; s0 < a.top_n; s0 += kMB) {
     const bool lo = s0 < 32;
-    uint32_t raw[16][kPer / 2];
-    int prow[16];
+    uint32_t raw[kMB][kPer / 2];
+    int prow[kMB];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
+    for (int k = 0; k < kMB; ++k) {
       prow[k] = __shfl_sync(0xffffffffu, lo ? r0 : r1, (s0 + k) & 31);
       if (s0 + k >= a.top_n) prow[k] = -1;
       const __half* p = po + static_cast<size_t>(prow[k] < 0 ? 0 : prow[k]) * 64;
@@ -722,7 +724,7 @@ __global__ void __launch_bounds__(256, 3) sel_merge_kernel(const SelInvArgs a) {
       L = warp_sum(w0 + w1);
     }
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
+    for (int k = 0; k < kMB; ++k) {
       const int src = (s0 + k) & 31;
       const float w = __shfl_sync(0xffffffffu, lo ? w0 : w1, src);
       const float c = __shfl_sync(0xffffffffu, lo ? (half == 0 ? x0.z : x0.w) : (half == 0 ? x1.z : x1.w), src);
