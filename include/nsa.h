@@ -198,9 +198,10 @@ int nsa_get_device_error(uint32_t* word, int clear);
  * every nsa_prefill / nsa_decode call records events[i] (cudaEvent_t handles owned by
  * the caller) on its stream at its stage boundaries: events[0] before the first kernel,
  * then one event after each kernel, in launch order (prefill: pool, compressed attention,
- * top-n, selected branch, window + combine, dense text rows; decode: compressed split,
- * select, branches, combine). Stages that do not run record nothing; events beyond
- * `count` are not recorded. count = 0 (or events = NULL) switches recording off. The
+ * top-n, selected buckets, selected tiles, window, merge + gated combine, dense text rows;
+ * decode: compressed split, select, branches + gated combine). Stages that do not run
+ * record nothing; events beyond `count` are not recorded. count = 0 (or events = NULL)
+ * switches recording off. The
  * registration is process-wide and not thread-safe. Returns NSA_OK or NSA_ERR_INVALID_ARG.
  */
 int nsa_profile_stages(void* const* events, int count);

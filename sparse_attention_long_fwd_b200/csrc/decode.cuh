@@ -6,13 +6,15 @@
 // is HBM-bound and split four ways:
 //   dec_cmp_kernel      split-K over the compressed cache: each CTA attends to a slice of
 //                       the visible blocks, keeps its base-2 logits for the scoring step
-//                       and writes a partial (max, sum, unnormalised output) per head;
+//                       and writes a partial (max, sum, unnormalised output) per head; one
+//                       more CTA per (sequence, group) runs the sliding-window branch, which
+//                       needs no selection, beside the compressed stream;
 //   dec_select_kernel   merges the partials into o_cmp and the row log-sum-exp, turns
 //                       the stored logits into selection-block scores summed over the
 //                       group, and picks the top-n blocks (topn.cuh);
-//   dec_branch_kernel   the selected-block and the sliding-window branches, one CTA per
-//                       (sequence, group, branch), four warps splitting the key chunks;
-//   dec_combine_kernel  out = g_cmp*o_cmp + g_sel*o_sel + g_win*o_win.
+//   dec_branch_kernel   the selected-block branch, one CTA per (sequence, group), four
+//                       warps splitting the key chunks, then the gated combine
+//                       out = g_cmp*o_cmp + g_sel*o_sel + g_win*o_win of the group's heads.
 #pragma once
 #include "sel.cuh"
 #include "topn.cuh"
@@ -20,6 +22,10 @@
 namespace nsa {
 
 constexpr int kDecWarps = 4;
+// Cache keys per chunk and chunks in flight per warp: 16-key chunks in a 3-stage ring keep
+// two chunks loading while one is used, in 24 KB per warp (d = 128), so two CTAs fit an SM.
+constexpr int kDecChunk = 16;
+constexpr int kDecStages = 3;
 
 // Sequence length of b, clamped to [1, lmax]; an out-of-range value is recorded in the
 // device error word instead of being used to index the caches.
@@ -44,16 +50,42 @@ struct DecArgs {
   float* lse;           // [B][hq] natural log
   float* scores;        // [B][hkv][nsel_max]
   int32_t* sel_idx;     // [B][hkv][top_n]
-  float* o_sel;         // [B][hq][D]
   float* o_win;         // [B][hq][D]
+  const float* gates;   // [B][hq][3]
+  void* out;            // [B][hq][D]
+  int out_f32;
 };
 
 template <int D>
 struct DecSmem {
-  WarpChunkBuf<D, kChunkKeys, 2> buf[kDecWarps];
-  WarpPartial<D> part[kDecWarps];
-  int chunk_start[kDecWarps][128];
+  union {
+    WarpChunkBuf<D, kDecChunk, kDecStages> buf[kDecWarps];
+    WarpPartial<D> part[kDecWarps];  // after the last chunk: the warps' partial states
+  };
+  int chunk_start[512];  // chunk list of the branch kernel (flat)
 };
+static_assert(sizeof(WarpPartial<128>) * kDecWarps <= sizeof(WarpChunkBuf<128, kDecChunk, kDecStages>) * kDecWarps,
+              "partials alias the chunk ring");
+
+// Stream `nch` chunks through the warp's ring (kDecStages - 1 in flight), calling
+// use(stage, ci) on each in order; load(stage, ci) issues chunk ci's cp.async copies.
+template <typename Load, typename Use>
+__device__ __forceinline__ void dec_stream(int nch, Load&& load, Use&& use) {
+#pragma unroll
+  for (int c = 0; c < kDecStages - 1; ++c) {
+    if (c < nch) load(c, c);
+    cp_async_commit();
+  }
+  for (int ci = 0; ci < nch; ++ci) {
+    const int cn = ci + kDecStages - 1;
+    if (cn < nch) load(cn % kDecStages, cn);
+    cp_async_commit();  // (possibly empty: keeps the group count uniform)
+    asm volatile("cp.async.wait_group %0;" ::"n"(kDecStages - 1) : "memory");
+    __syncwarp();
+    use(ci % kDecStages, ci);
+    __syncwarp();
+  }
+}
 
 // Merge the four warps' partial states of rows < G; returns through the callback
 // f(row, m, l, o_ptr_scaled...) -- written inline at the two call sites below.
@@ -69,17 +101,95 @@ __device__ __forceinline__ void merge_rows(const WarpPartial<D>* parts, int npar
   }
 }
 
+// Programmatic dependent launch: a kernel lets the next one in the stream be launched
+// while it runs (its CTAs then wait, resident, in grid_dependency_wait until this grid has
+// finished and its writes are visible), so the launch gap between the decode's kernels is
+// hidden.
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// One (sequence, group)'s selected-block (is_win false) or sliding-window (is_win true)
+// branch: the four warps split the key chunks, then merge; each normalised output value
+// goes to f(row, c, value) for the lane's columns c.
+template <int D, typename F>
+__device__ __forceinline__ void dec_branch_body(DecSmem<D>& sm, const __nv_bfloat16* __restrict__ q,
+                                                const __nv_bfloat16* __restrict__ kcache,
+                                                const __nv_bfloat16* __restrict__ vcache, const DecArgs& a, int b,
+                                                int g, int L, bool is_win, F&& f) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bg = b * a.hkv + g;
+  const int t = L - 1;
+  // chunk list (shared by the four warps; warp w takes chunks w, w+4, ...); its last entry
+  // holds the count
+  int* list = sm.chunk_start;
+  int nch;
+  if (warp == 0) {
+    if (is_win) {
+      const int w0 = max(0, t - a.window + 1);
+      nch = (t + 1 - w0 + kDecChunk - 1) / kDecChunk;
+      if (nch > 511) nch = 511;  // window <= 4096 is validated on the host
+      for (int ci = lane; ci < nch; ci += 32) list[ci] = w0 + ci * kDecChunk;
+      __syncwarp();
+    } else {
+      // (top_n * sel_len / kDecChunk <= 511 entries for the validated sizes)
+      nch = build_chunk_list(a.sel_idx + static_cast<size_t>(bg) * a.top_n, a.top_n, a.sel_len, t, list, lane,
+                             kDecChunk);
+    }
+    if (lane == 0) sm.chunk_start[511] = nch;
+  }
+  __syncthreads();
+  nch = sm.chunk_start[511];
+  const int key_lo = is_win ? max(0, t - a.window + 1) : 0;
+  uint32_t qa[D / 16][4];
+  load_q_frags<D>(qa, q + (static_cast<size_t>(b) * a.hq + g * a.G) * D, a.G, lane);
+  const size_t rs = static_cast<size_t>(a.hkv) * D;
+  const __nv_bfloat16* kb = kcache + static_cast<size_t>(b) * a.lmax * rs + static_cast<size_t>(g) * D;
+  const __nv_bfloat16* vb = vcache + static_cast<size_t>(b) * a.lmax * rs + static_cast<size_t>(g) * D;
+  auto& buf = sm.buf[warp];
+  WarpAttnState<D> st;
+  state_init(st);
+  const int my = nch > warp ? (nch - warp + kDecWarps - 1) / kDecWarps : 0;
+  dec_stream(
+      my,
+      [&](int stg, int x) { load_chunk<D>(buf, stg, kb, vb, rs, list[warp + x * kDecWarps], t + 1, lane); },
+      [&](int stg, int x) { attend_chunk<D>(st, qa, buf, stg, list[warp + x * kDecWarps], key_lo, t + 1, a.sl2, lane); });
+  state_reduce_l(st);
+  cp_async_wait_0();
+  __syncthreads();  // every warp is done with the ring: the partials take its place
+  state_store(st, sm.part[warp], lane);
+  __syncthreads();
+  for (int row = warp; row < a.G; row += kDecWarps) {
+    float M, Lsum, wts[kDecWarps];
+    merge_rows<D>(sm.part, kDecWarps, a.G, row, M, Lsum, wts);
+    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+    for (int c = lane; c < D; c += 32) {
+      float acc = 0.f;
+      for (int w = 0; w < kDecWarps; ++w) acc += sm.part[w].o[row][c] * wts[w];
+      f(row, c, acc * inv);
+    }
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kDecWarps * 32) dec_cmp_kernel(const __nv_bfloat16* __restrict__ q,
                                                                  const __nv_bfloat16* __restrict__ kcmp,
                                                                  const __nv_bfloat16* __restrict__ vcmp,
+                                                                 const __nv_bfloat16* __restrict__ kcache,
+                                                                 const __nv_bfloat16* __restrict__ vcache,
                                                                  const int32_t* __restrict__ seq_lens,
                                                                  const DecArgs a) {
   extern __shared__ uint8_t dec_smem_raw[];
   DecSmem<D>& sm = *reinterpret_cast<DecSmem<D>*>((reinterpret_cast<uintptr_t>(dec_smem_raw) + 127) & ~uintptr_t(127));
+  grid_launch_dependents();  // dec_select_kernel may take free slots and wait there
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bg = blockIdx.y, b = bg / a.hkv, g = bg % a.hkv, split = blockIdx.x;
   const int L = seq_len_checked(seq_lens, b, a.lmax);
+  if (split == a.nsplit) {  // the window branch of (sequence, group)
+    float* dst = a.o_win + (static_cast<size_t>(b) * a.hq + g * a.G) * D;
+    dec_branch_body<D>(sm, q, kcache, vcache, a, b, g, L, true,
+                       [&](int row, int c, float v) { dst[static_cast<size_t>(row) * D + c] = v; });
+    return;
+  }
   const int nc = (L >= a.cmp_len) ? (L - a.cmp_len) / a.cmp_stride + 1 : 0;
   const int per = ((a.ncmax + a.nsplit - 1) / a.nsplit + kDecWarps * kChunkKeys - 1) / (kDecWarps * kChunkKeys) *
                   (kDecWarps * kChunkKeys);
@@ -97,24 +207,15 @@ __global__ void __launch_bounds__(kDecWarps * 32) dec_cmp_kernel(const __nv_bflo
   auto& buf = sm.buf[warp];
   WarpAttnState<D> st;
   state_init(st);
-  const int nch = w1 > w0 ? (w1 - w0 + kChunkKeys - 1) / kChunkKeys : 0;
-  if (nch > 0) {
-    load_chunk<D>(buf, 0, kb, vb, rs, w0, w1, lane);
-    cp_async_commit();
-  }
-  for (int ci = 0; ci < nch; ++ci) {
-    if (ci + 1 < nch) {
-      load_chunk<D>(buf, (ci + 1) & 1, kb, vb, rs, w0 + (ci + 1) * kChunkKeys, w1, lane);
-      cp_async_commit();
-      cp_async_wait_1();
-    } else {
-      cp_async_wait_0();
-    }
-    __syncwarp();
-    attend_chunk<D>(st, qa, buf, ci & 1, w0 + ci * kChunkKeys, w0, w1, a.sl2, lane, lg, a.ncmax, 0, a.G);
-    __syncwarp();
-  }
+  const int nch = w1 > w0 ? (w1 - w0 + kDecChunk - 1) / kDecChunk : 0;
+  dec_stream(
+      nch, [&](int stg, int ci) { load_chunk<D>(buf, stg, kb, vb, rs, w0 + ci * kDecChunk, w1, lane); },
+      [&](int stg, int ci) {
+        attend_chunk<D>(st, qa, buf, stg, w0 + ci * kDecChunk, w0, w1, a.sl2, lane, lg, a.ncmax, 0, a.G);
+      });
   state_reduce_l(st);
+  cp_async_wait_0();
+  __syncthreads();  // every warp is done with the ring: the partials take its place
   state_store(st, sm.part[warp], lane);
   __syncthreads();
   float* dst = a.part + (static_cast<size_t>(bg) * a.nsplit + split) * a.G * (2 + D);
@@ -138,6 +239,8 @@ __global__ void __launch_bounds__(kDecWarps * 32) dec_cmp_kernel(const __nv_bflo
 template <int D>
 __global__ void __launch_bounds__(256) dec_select_kernel(const int32_t* __restrict__ seq_lens, const DecArgs a,
                                                          int32_t* __restrict__ out_sel_idx) {
+  grid_dependency_wait();  // dec_cmp_kernel's partials and logits
+  grid_launch_dependents();
   extern __shared__ float ds_smem[];
   float* sc = ds_smem;                                        // [nsel_max]
   int* list = reinterpret_cast<int*>(sc + a.nsel_max);        // [nsel_max]
@@ -150,26 +253,39 @@ __global__ void __launch_bounds__(256) dec_select_kernel(const int32_t* __restri
   const int nc = (L >= a.cmp_len) ? (L - a.cmp_len) / a.cmp_stride + 1 : 0;
   const int jt = t / a.sel_len;
   const float* part = a.part + static_cast<size_t>(bg) * a.nsplit * a.G * (2 + D);
-  // ---- merge split partials: o_cmp and the base-2 log-sum-exp per head
+  // ---- merge split partials: o_cmp and the base-2 log-sum-exp per head. A warp per head
+  // row: lane s holds split s (and s + 32), so the (max, sum) loads go out together, and the
+  // output columns' loads are unrolled over the splits.
+  const int lane = tid & 31;
   for (int row = tid / 32; row < a.G; row += 8) {
-    float M = -INFINITY;
-    for (int s = 0; s < a.nsplit; ++s) M = fmaxf(M, part[(static_cast<size_t>(s) * a.G + row) * (2 + D)]);
-    float Lsum = 0.f;
-    for (int s = 0; s < a.nsplit; ++s) {
-      const float* pr = part + (static_cast<size_t>(s) * a.G + row) * (2 + D);
-      if (M != -INFINITY) Lsum += pr[1] * ex2_approx(pr[0] - M);
-    }
+    auto ml = [&](int s, int k) -> float {
+      return s < a.nsplit ? part[(static_cast<size_t>(s) * a.G + row) * (2 + D) + k] : (k == 0 ? -INFINITY : 0.f);
+    };
+    const float m0 = ml(lane, 0), l0 = ml(lane, 1), m1 = ml(lane + 32, 0), l1 = ml(lane + 32, 1);
+    float M = fmaxf(m0, m1);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float w0 = (M == -INFINITY || m0 == -INFINITY) ? 0.f : ex2_approx(m0 - M);
+    const float w1 = (M == -INFINITY || m1 == -INFINITY) ? 0.f : ex2_approx(m1 - M);
+    float Lsum = l0 * w0 + l1 * w1;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
     const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
     const int h = g * a.G + row;
-    for (int c = tid % 32; c < D; c += 32) {
-      float acc = 0.f;
-      for (int s = 0; s < a.nsplit; ++s) {
-        const float* pr = part + (static_cast<size_t>(s) * a.G + row) * (2 + D);
-        if (M != -INFINITY) acc += pr[2 + c] * ex2_approx(pr[0] - M);
-      }
-      a.o_cmp[(static_cast<size_t>(b) * a.hq + h) * D + c] = acc * inv;
+    constexpr int kPer = D / 32;
+    float acc[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
+#pragma unroll 4
+    for (int s = 0; s < a.nsplit; ++s) {
+      const float w = __shfl_sync(0xffffffffu, s < 32 ? w0 : w1, s & 31);
+      const float* pr = part + (static_cast<size_t>(s) * a.G + row) * (2 + D) + 2;
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) acc[k] += w * pr[lane + 32 * k];
     }
-    if (tid % 32 == 0) {
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) a.o_cmp[(static_cast<size_t>(b) * a.hq + h) * D + lane + 32 * k] = acc[k] * inv;
+    if (lane == 0) {
       lse2[row] = Lsum > 0.f ? M + __log2f(Lsum) : INFINITY;
       a.lse[static_cast<size_t>(b) * a.hq + h] = Lsum > 0.f ? (M + __log2f(Lsum)) * 0.69314718055994530942f : -INFINITY;
     }
@@ -201,7 +317,8 @@ __global__ void __launch_bounds__(256) dec_select_kernel(const int32_t* __restri
   }
 }
 
-// grid (B*hkv, 2): blockIdx.y = 0 -> selected blocks, 1 -> sliding window.
+// One CTA per (sequence, group): the selected-block branch, then the gated combine of the
+// group's heads (o_cmp from dec_select_kernel, o_win from dec_cmp_kernel's window CTAs).
 template <int D>
 __global__ void __launch_bounds__(kDecWarps * 32) dec_branch_kernel(const __nv_bfloat16* __restrict__ q,
                                                                     const __nv_bfloat16* __restrict__ kcache,
@@ -210,83 +327,19 @@ __global__ void __launch_bounds__(kDecWarps * 32) dec_branch_kernel(const __nv_b
                                                                     const DecArgs a) {
   extern __shared__ uint8_t dec_smem_raw[];
   DecSmem<D>& sm = *reinterpret_cast<DecSmem<D>*>((reinterpret_cast<uintptr_t>(dec_smem_raw) + 127) & ~uintptr_t(127));
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bg = blockIdx.x, b = bg / a.hkv, g = bg % a.hkv;
-  const bool is_win = blockIdx.y == 1;
+  grid_dependency_wait();  // dec_select_kernel's selection and o_cmp (and, before it, o_win)
   const int L = seq_len_checked(seq_lens, b, a.lmax);
-  const int t = L - 1;
-  // chunk list (shared by the four warps; warp w takes chunks w, w+4, ...)
-  int* list = sm.chunk_start[0];
-  int nch;
-  if (warp == 0) {
-    if (is_win) {
-      const int w0 = max(0, t - a.window + 1);
-      nch = (t + 1 - w0 + kChunkKeys - 1) / kChunkKeys;
-      if (nch > 128) nch = 128;  // window <= 4096 is validated on the host
-      for (int ci = lane; ci < nch; ci += 32) list[ci] = w0 + ci * kChunkKeys;
-      __syncwarp();
-    } else {
-      nch = build_chunk_list(a.sel_idx + static_cast<size_t>(bg) * a.top_n, a.top_n, a.sel_len, t, list, lane);
-    }
-    if (lane == 0) sm.chunk_start[1][0] = nch;
-  }
-  __syncthreads();
-  nch = sm.chunk_start[1][0];
-  const int key_lo = is_win ? max(0, t - a.window + 1) : 0;
-  uint32_t qa[D / 16][4];
-  load_q_frags<D>(qa, q + (static_cast<size_t>(b) * a.hq + g * a.G) * D, a.G, lane);
-  const size_t rs = static_cast<size_t>(a.hkv) * D;
-  const __nv_bfloat16* kb = kcache + static_cast<size_t>(b) * a.lmax * rs + static_cast<size_t>(g) * D;
-  const __nv_bfloat16* vb = vcache + static_cast<size_t>(b) * a.lmax * rs + static_cast<size_t>(g) * D;
-  auto& buf = sm.buf[warp];
-  WarpAttnState<D> st;
-  state_init(st);
-  const int my = nch > warp ? (nch - warp + kDecWarps - 1) / kDecWarps : 0;
-  if (my > 0) {
-    load_chunk<D>(buf, 0, kb, vb, rs, list[warp], t + 1, lane);
-    cp_async_commit();
-  }
-  for (int x = 0; x < my; ++x) {
-    const int ci = warp + x * kDecWarps;
-    if (x + 1 < my) {
-      load_chunk<D>(buf, (x + 1) & 1, kb, vb, rs, list[ci + kDecWarps], t + 1, lane);
-      cp_async_commit();
-      cp_async_wait_1();
-    } else {
-      cp_async_wait_0();
-    }
-    __syncwarp();
-    attend_chunk<D>(st, qa, buf, x & 1, list[ci], key_lo, t + 1, a.sl2, lane);
-    __syncwarp();
-  }
-  state_reduce_l(st);
-  state_store(st, sm.part[warp], lane);
-  __syncthreads();
-  float* dst = (is_win ? a.o_win : a.o_sel) + (static_cast<size_t>(b) * a.hq + g * a.G) * D;
-  for (int row = warp; row < a.G; row += kDecWarps) {
-    float M, Lsum, wts[kDecWarps];
-    merge_rows<D>(sm.part, kDecWarps, a.G, row, M, Lsum, wts);
-    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-    for (int c = lane; c < D; c += 32) {
-      float acc = 0.f;
-      for (int w = 0; w < kDecWarps; ++w) acc += sm.part[w].o[row][c] * wts[w];
-      dst[static_cast<size_t>(row) * D + c] = acc * inv;
-    }
-  }
-}
-
-__global__ void __launch_bounds__(256) dec_combine_kernel(const float* __restrict__ gates, const float* __restrict__ o_cmp,
-                                                          const float* __restrict__ o_sel,
-                                                          const float* __restrict__ o_win, void* __restrict__ out,
-                                                          int out_f32, int rows, int d) {
-  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= static_cast<long long>(rows) * d) return;
-  const long long row = i / d;
-  const float v = gates[row * 3 + 0] * o_cmp[i] + gates[row * 3 + 1] * o_sel[i] + gates[row * 3 + 2] * o_win[i];
-  if (out_f32)
-    static_cast<float*>(out)[i] = v;
-  else
-    static_cast<__nv_bfloat16*>(out)[i] = __float2bfloat16_rn(v);
+  const size_t row0 = static_cast<size_t>(b) * a.hq + g * a.G;
+  dec_branch_body<D>(sm, q, kcache, vcache, a, b, g, L, false, [&](int row, int c, float v) {
+    const size_t r = row0 + row;
+    const size_t e = r * D + c;
+    const float o = a.gates[r * 3 + 0] * a.o_cmp[e] + a.gates[r * 3 + 1] * v + a.gates[r * 3 + 2] * a.o_win[e];
+    if (a.out_f32)
+      static_cast<float*>(a.out)[e] = o;
+    else
+      static_cast<__nv_bfloat16*>(a.out)[e] = __float2bfloat16_rn(o);
+  });
 }
 
 }  // namespace nsa

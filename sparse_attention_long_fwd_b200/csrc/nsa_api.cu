@@ -118,7 +118,7 @@ PrefillLayout prefill_layout(const nsa_params_t* p) {
 }
 
 struct DecodeLayout {
-  size_t logits, part, o_cmp, lse, scores, sel_idx, o_sel, o_win, total;
+  size_t logits, part, o_cmp, lse, scores, sel_idx, o_win, total;
   int ncmax, nsel_max, nsplit;
 };
 
@@ -143,7 +143,6 @@ DecodeLayout decode_layout(const nsa_params_t* p) {
   L.lse = take(static_cast<size_t>(B) * hq * 4);
   L.scores = take(static_cast<size_t>(B) * hkv * L.nsel_max * 4);
   L.sel_idx = take(static_cast<size_t>(B) * hkv * p->top_n * 4);
-  L.o_sel = take(static_cast<size_t>(B) * hq * d * 4);
   L.o_win = take(static_cast<size_t>(B) * hq * d * 4);
   L.total = off;
   return L;
@@ -391,6 +390,25 @@ int prefill_impl(const nsa_params_t* p, const void* q, const void* k, const void
   return NSA_OK;
 }
 
+// Launch with programmatic stream serialisation: the kernel may start while the previous
+// one in the stream finishes, and waits for it (griddepcontrol.wait) before reading its
+// results.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 template <int D>
 int decode_impl(const nsa_params_t* p, const void* q, const void* kcache, const void* vcache, const void* kcmp,
                 const void* vcmp, const int32_t* seq_lens, const float* gates, void* out, int32_t* out_sel_idx,
@@ -419,37 +437,42 @@ int decode_impl(const nsa_params_t* p, const void* q, const void* kcache, const 
   a.lse = reinterpret_cast<float*>(ws + L.lse);
   a.scores = reinterpret_cast<float*>(ws + L.scores);
   a.sel_idx = reinterpret_cast<int32_t*>(ws + L.sel_idx);
-  a.o_sel = reinterpret_cast<float*>(ws + L.o_sel);
   a.o_win = reinterpret_cast<float*>(ws + L.o_win);
+  a.gates = gates;
+  a.out = out;
+  a.out_f32 = p->out_dtype == NSA_OUT_F32;
   const auto* qq = static_cast<const __nv_bfloat16*>(q);
   int rc;
   const size_t smem = sizeof(nsa::DecSmem<D>) + 128;
   {
     auto kern = nsa::dec_cmp_kernel<D>;
     if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
-    kern<<<dim3(L.nsplit, a.batch * a.hkv), nsa::kDecWarps * 32, smem, st>>>(
-        qq, static_cast<const __nv_bfloat16*>(kcmp), static_cast<const __nv_bfloat16*>(vcmp), seq_lens, a);
+    // x < nsplit: slices of the compressed cache; x = nsplit: the window branch
+    kern<<<dim3(L.nsplit + 1, a.batch * a.hkv), nsa::kDecWarps * 32, smem, st>>>(
+        qq, static_cast<const __nv_bfloat16*>(kcmp), static_cast<const __nv_bfloat16*>(vcmp),
+        static_cast<const __nv_bfloat16*>(kcache), static_cast<const __nv_bfloat16*>(vcache), seq_lens, a);
     if ((rc = launch_status("dec_cmp", st)) != NSA_OK) return rc;
   }
   {
     const size_t ssm = (2 * static_cast<size_t>(L.nsel_max) + L.nsel_max / 32 + 1 + 16) * 4;
     auto kern = nsa::dec_select_kernel<D>;
     if (set_smem(kern, ssm) != NSA_OK) return NSA_ERR_CUDA;
-    kern<<<a.batch * a.hkv, 256, ssm, st>>>(seq_lens, a, out_sel_idx);
+    if (launch_dependent(kern, dim3(a.batch * a.hkv), dim3(256), ssm, st, seq_lens, a, out_sel_idx) != cudaSuccess) {
+      cudaGetLastError();  // (clear it: the status is returned here)
+      return NSA_ERR_CUDA;
+    }
     if ((rc = launch_status("dec_select", st)) != NSA_OK) return rc;
   }
   {
     auto kern = nsa::dec_branch_kernel<D>;
     if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
-    kern<<<dim3(a.batch * a.hkv, 2), nsa::kDecWarps * 32, smem, st>>>(
-        qq, static_cast<const __nv_bfloat16*>(kcache), static_cast<const __nv_bfloat16*>(vcache), seq_lens, a);
+    if (launch_dependent(kern, dim3(a.batch * a.hkv), dim3(nsa::kDecWarps * 32), smem, st, qq,
+                         static_cast<const __nv_bfloat16*>(kcache), static_cast<const __nv_bfloat16*>(vcache), seq_lens,
+                         a) != cudaSuccess) {
+      cudaGetLastError();  // (clear it: the status is returned here)
+      return NSA_ERR_CUDA;
+    }
     if ((rc = launch_status("dec_branch", st)) != NSA_OK) return rc;
-  }
-  {
-    const long long n = static_cast<long long>(a.batch) * a.hq * D;
-    nsa::dec_combine_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
-        gates, a.o_cmp, a.o_sel, a.o_win, out, p->out_dtype == NSA_OUT_F32, a.batch * a.hq, D);
-    if ((rc = launch_status("dec_combine", st)) != NSA_OK) return rc;
   }
   return NSA_OK;
 }
