@@ -17,7 +17,8 @@
  *     ones (top168.com article, section 一, the selection-branch paragraph).
  * The pages fix none of the constants or formulas below; where they are silent the
  * plainest reading is taken (each one is named at the function that uses it):
- *   compression   Kc[i] = bf16_rne(mean_{u<l} K[i*s+u]), complete blocks only;
+ *   compression   Kc[i] = bf16_rne(mean_{u<l} K[i*s+u]), complete blocks only; the
+ *                 learnable form weights the l positions per head instead of averaging;
  *   cmp branch    block i visible to t iff i*s + l - 1 <= t; softmax over visible blocks;
  *   block scores  score[j] = sum_{h in group} sum_i P_h[i] * |tokens(i) & tokens(j)| / l;
  *   selection     blocks 0, j_t and j_t-1 always kept (j_t = t / l'); the remaining
@@ -107,6 +108,26 @@ void oracle_compress(const uint16_t* k, int T, int h, int d, int l, int s, uint1
         double sum = 0.0;
         for (int u = 0; u < l; ++u) sum += oracle_bf16_to_double(k[((size_t)(i * s + u) * h + g) * d + c]);
         kc[((size_t)i * h + g) * d + c] = oracle_double_to_bf16(sum / (double)l);
+      }
+}
+
+/* Learnable compression: the sparse pattern is steered by learned parameters
+ * (shd-paper.top page "VideoNSA: Native Sparse Attention Scales Video Understanding",
+ * section "方法详解", key design (1)). The page gives no form for them; the reading here
+ * is the plainest learnable version of the mean above: a per-head linear map over the l
+ * positions of a block, Kc[i][g] = bf16_rne(sum_u w[g][u] * K[i*s+u][g]), with w = 1/l
+ * giving the mean. Each product of an fp32 weight and a bf16 key is exact in fp64 and the
+ * sum runs in token order, rounded once.
+ * k: [T][h][d] bf16 bits; w: [h][l] fp32; kc: [Ncmp(T)][h][d] bf16 bits. */
+void oracle_compress_weighted(const uint16_t* k, const float* w, int T, int h, int d, int l, int s, uint16_t* kc) {
+  const int nc = oracle_num_cmp(T, l, s);
+  for (int i = 0; i < nc; ++i)
+    for (int g = 0; g < h; ++g)
+      for (int c = 0; c < d; ++c) {
+        double sum = 0.0;
+        for (int u = 0; u < l; ++u)
+          sum += (double)w[(size_t)g * l + u] * oracle_bf16_to_double(k[((size_t)(i * s + u) * h + g) * d + c]);
+        kc[((size_t)i * h + g) * d + c] = oracle_double_to_bf16(sum);
       }
 }
 

@@ -52,6 +52,8 @@ def _load():
         lib.oracle_num_cmp.argtypes = [ctypes.c_int] * 3
         lib.oracle_num_sel.argtypes = [ctypes.c_int] * 2
         lib.oracle_compress.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
+        lib.oracle_compress_weighted.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                 ctypes.c_int, P]
         lib.oracle_prefill_rows.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, P, P, ctypes.c_int, P, P, P, P, P,
                                             ctypes.c_int, P, P, P, P, P, ctypes.c_int]
         lib.oracle_decode.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, P, P, P, ctypes.c_int, P, P, P, P, P,
@@ -124,6 +126,20 @@ def compress(k_bits: np.ndarray, l: int = 32, s: int = 16) -> np.ndarray:
     nc = num_cmp(T, l, s)
     out = np.zeros((max(nc, 0), h, d), dtype=np.uint16)
     _load().oracle_compress(_ptr(k_bits), T, h, d, l, s, _ptr(out))
+    return out
+
+
+def compress_weighted(k_bits: np.ndarray, w: np.ndarray, l: int = 32, s: int = 16) -> np.ndarray:
+    """Learnable compression of [T, h, d] bf16 keys (values): every complete block is the
+    w-weighted sum of its l tokens, w [h, l] float32 per head, rounded once to bf16."""
+    k_bits = _u16(k_bits)
+    T, h, d = k_bits.shape
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    if w.shape != (h, l):
+        raise ValueError(f"weights must be [{h}, {l}], got {w.shape}")
+    nc = num_cmp(T, l, s)
+    out = np.zeros((max(nc, 0), h, d), dtype=np.uint16)
+    _load().oracle_compress_weighted(_ptr(k_bits), _ptr(w), T, h, d, l, s, _ptr(out))
     return out
 
 

@@ -371,3 +371,142 @@ def test_decode_equals_prefill_last_row():
                                gg.numpy(), np.array([L - 1]))
         assert np.array_equal(dec["out"][b], pre["out"][0])
         assert np.array_equal(dec["sel"][b], pre["sel"][0])
+
+
+# ---------------------------------------------------------------- learnable compression
+
+def _rand_weights(shape, seed):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.rand(shape, generator=g) * 0.1 - 0.02).numpy().astype(np.float32)
+
+
+def test_weighted_compress_is_rounded_exact_weighted_sum():
+    # the definition evaluated in exact rationals, rounded by direct search
+    T, h, d, l, s = 40, 2, 4, 8, 4
+    k = _bits(_rand_bf16((T, h, d), 31))
+    w = _rand_weights((h, l), 32)
+    got = orc.compress_weighted(k, w, l, s)
+    kf = orc.bf16_bits_to_f64(k)
+    nc = (T - l) // s + 1
+    assert got.shape == (nc, h, d)
+    for i in range(nc):
+        for g in range(h):
+            for c in range(d):
+                exact = sum(Fraction(float(w[g, u])) * Fraction(float(kf[i * s + u, g, c])) for u in range(l))
+                assert int(got[i, g, c]) == _exact_bf16(exact), (i, g, c)
+
+
+def test_weighted_compress_uniform_weights_equal_mean():
+    k = _bits(_rand_bf16((300, 3, 16), 33))
+    w = np.full((3, 32), 1.0 / 32, dtype=np.float32)  # 1/32 is exact, so the sums agree bit for bit
+    assert np.array_equal(orc.compress_weighted(k, w, 32, 16), orc.compress(k, 32, 16))
+
+
+def test_weighted_compress_one_hot_copies_a_token_per_head():
+    T, h, d, l, s = 200, 3, 8, 32, 16
+    k = _bits(_rand_bf16((T, h, d), 34))
+    w = np.zeros((h, l), dtype=np.float32)
+    pos = [0, 17, 31]
+    for g in range(h):
+        w[g, pos[g]] = 1.0
+    got = orc.compress_weighted(k, w, l, s)
+    for g in range(h):
+        want = k[pos[g]::s, g][: got.shape[0]]
+        assert np.array_equal(got[:, g], want), g
+
+
+# ---------------------------------------------------------------- gate network
+
+from oracle import gate as gate_orc  # noqa: E402
+
+# standard normal CDF at 1, -1 and 2 (textbook values)
+_PHI_1 = 0.8413447460685429
+_PHI_M1 = 0.15865525393145707
+_PHI_2 = 0.9772498680518208
+
+
+def test_gelu_textbook_values():
+    got = gate_orc.gelu(np.array([0.0, 1.0, -1.0, 2.0]))
+    assert got[0] == 0.0
+    assert got[1] == pytest.approx(_PHI_1, abs=1e-15)
+    assert got[2] == pytest.approx(-_PHI_M1, abs=1e-15)
+    assert got[3] == pytest.approx(2 * _PHI_2, abs=1e-15)
+    # x*Phi(x) - (-x)*Phi(-x) = x, for any x
+    xs = np.linspace(-6, 6, 101)
+    assert np.allclose(gate_orc.gelu(xs) - gate_orc.gelu(-xs), xs, atol=1e-14)
+
+
+def test_gates_zero_weights_are_softmax_of_bias():
+    dim = 8
+    x = _bits(_rand_bf16((5, dim), 40))
+    w1 = np.zeros((dim // 2, dim), dtype=np.uint16)
+    got = gate_orc.gate_mlp(x, w1, np.zeros(dim // 2), np.zeros((3, dim // 2)),
+                            np.array([0.0, math.log(2), math.log(3)], dtype=np.float32))
+    b2 = np.array([0.0, math.log(2), math.log(3)], dtype=np.float32).astype(np.float64)
+    want = np.exp(b2) / np.exp(b2).sum()  # (1, 2, 3)/6 up to the fp32 rounding of the logs
+    assert np.allclose(got, want[None, :], atol=1e-15)
+    assert np.allclose(want, [1 / 6, 2 / 6, 3 / 6], atol=1e-7)
+
+
+def test_gates_hand_worked_case_pins_layouts_and_gelu():
+    # hidden unit j reads input j with sign (+, -, +); gate c reads hidden unit (c + 2) % 3
+    dim, hid = 6, 3
+    x = _bits(torch.tensor([[1.0, 1.0, 2.0, 0.0, 0.0, 0.0]], dtype=torch.bfloat16))
+    w1 = torch.zeros(hid, dim)
+    w1[0, 0], w1[1, 1], w1[2, 2] = 1.0, -1.0, 1.0
+    w2 = np.zeros((3, hid), dtype=np.float32)
+    w2[0, 2], w2[1, 0], w2[2, 1] = 1.0, 1.0, 1.0
+    got = gate_orc.gate_mlp(x, _bits(w1.to(torch.bfloat16)), np.zeros(hid), w2, np.zeros(3))
+    logits = [2 * _PHI_2, _PHI_1, -_PHI_M1]
+    z = sum(math.exp(v) for v in logits)
+    assert np.allclose(got[0], [math.exp(v) / z for v in logits], atol=1e-14)
+
+
+def _torch_gate_module(dim, w1_bits, b1, w2, b2):
+    """The blog's two-layer gate module built from torch.nn layers in float64."""
+    m = torch.nn.Sequential(torch.nn.Linear(dim, dim // 2), torch.nn.GELU(), torch.nn.Linear(dim // 2, 3)).double()
+    with torch.no_grad():
+        m[0].weight.copy_(_f64(w1_bits))
+        m[0].bias.copy_(torch.from_numpy(np.asarray(b1, np.float32).astype(np.float64)))
+        m[2].weight.copy_(torch.from_numpy(np.asarray(w2, np.float32).astype(np.float64)))
+        m[2].bias.copy_(torch.from_numpy(np.asarray(b2, np.float32).astype(np.float64)))
+    return m
+
+
+def _rand_gate_weights(dim, seed):
+    g = torch.Generator().manual_seed(seed)
+    w1 = _bits((torch.randn(dim // 2, dim, generator=g) / math.sqrt(dim)).to(torch.bfloat16))
+    b1 = (torch.randn(dim // 2, generator=g) * 0.1).numpy().astype(np.float32)
+    w2 = (torch.randn(3, dim // 2, generator=g) / math.sqrt(dim // 2)).numpy().astype(np.float32)
+    b2 = (torch.randn(3, generator=g) * 0.1).numpy().astype(np.float32)
+    return w1, b1, w2, b2
+
+
+@pytest.mark.parametrize("dim", [64, 128])
+def test_gates_match_torch_module(dim):
+    w1, b1, w2, b2 = _rand_gate_weights(dim, 41)
+    x = _bits(_rand_bf16((7, 4, dim), 42))
+    got = gate_orc.gate_mlp(x, w1, b1, w2, b2)
+    m = _torch_gate_module(dim, w1, b1, w2, b2)
+    want = torch.softmax(m(_f64(x)), dim=-1).detach().numpy()
+    assert np.allclose(got, want, atol=1e-13)
+    assert np.allclose(got.sum(-1), 1.0, atol=1e-14) and (got > 0).all()
+    # adding a constant to every logit leaves the gates unchanged
+    shifted = gate_orc.gate_mlp(x, w1, b1, w2, b2 + np.float32(3.0))
+    assert np.allclose(shifted, got, atol=1e-13)
+
+
+def test_pooled_gates_match_blog_module_per_head():
+    B, T, H, dim = 2, 9, 3, 64
+    w1, b1, w2, b2 = _rand_gate_weights(dim, 43)
+    x = _bits(_rand_bf16((B, T, H, dim), 44))
+    got = gate_orc.gate_mlp_pooled(x, w1, b1, w2, b2)
+    m = _torch_gate_module(dim, w1, b1, w2, b2)
+    xf = _f64(x)
+    for h in range(H):
+        want = torch.softmax(m(xf[:, :, h, :].mean(dim=1)), dim=-1).detach().numpy()  # the blog's forward, one head
+        assert np.allclose(got[:, h], want, atol=1e-13), h
+    # tokens that are all equal pool to the per-token gate
+    same = np.repeat(x[:, :1], T, axis=1)
+    assert np.allclose(gate_orc.gate_mlp_pooled(same, w1, b1, w2, b2),
+                       gate_orc.gate_mlp(same[:, 0], w1, b1, w2, b2), atol=1e-14)
