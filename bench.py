@@ -34,7 +34,8 @@ sys.path.insert(0, ROOT)
 
 from sparse_attention_long_fwd_b200 import dist as dist_helpers  # noqa: E402
 from sparse_attention_long_fwd_b200 import nsa  # noqa: E402
-from sparse_attention_long_fwd_b200.inputs import WORKLOADS, decode_inputs, prefill_inputs  # noqa: E402
+from sparse_attention_long_fwd_b200.inputs import (WORKLOADS, decode_inputs, gate_weights, phi_weights,  # noqa: E402
+                                                   prefill_inputs)
 
 METRIC = "NSA prefill video tokens/s at 128K & TFLOP/s vs peak; decode HBM GB/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -364,6 +365,10 @@ def run_b200(args, world, rank, local):
         result["decode"] = run_decode(args, dev, peaks, peaks_src, flush, world)
         result["gpu_launches"] += len(DECODE_STAGES) * result["decode"]["steps"]
 
+    if not args.no_gates and w.name == "v128k":
+        result["gates_and_phi"] = run_gates(args, dev, q, k, v, g, peaks, peaks_src, flush, world)
+        result["gpu_launches"] += result["gates_and_phi"]["launches"]
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, q, k, v, g, args.cpu_seconds)
     return result
@@ -406,6 +411,75 @@ def run_sweep(args, dev, q, k, v, g, flush, peak_t, world):
         del out
     return {"points": points, "inputs": "the headline 128K tensors (same seed); only n and w change",
             "l2": "flushed before every timed step", "steps": args.steps, "warmup": args.warmup}
+
+
+def run_gates(args, dev, q, k, v, g, peaks, peaks_src, flush, world):
+    """The gate network over the 128K queries (one row per token and head) and the prefill
+    with the learnable compression, on the headline tensors."""
+    w = WORKLOADS["v128k"]
+    rows, dim = w.n_tokens * w.hq, w.d
+    w1, b1, w2, b2 = gate_weights(dim, seed=21, device=dev)
+    gates = torch.empty((rows, 3), dtype=torch.float32, device=dev)
+
+    def gate_step(events):
+        rc = nsa.nsa_gate_mlp(q, w1, b1, w2, b2, rows, dim, gates)
+        if rc != nsa.NSA_OK:
+            raise nsa.NsaError(rc, "nsa_gate_mlp")
+
+    barrier(world)
+    gms, _ = timed_steps(gate_step, args.steps, args.warmup, flush, 0)
+    gate_ms = max_over_ranks(sum(gms), world) / args.steps
+    gate_bytes = rows * dim * 2 + rows * 3 * 4 + w1.numel() * 2 + (b1.numel() + w2.numel() + b2.numel()) * 4
+    gate_gbs = gate_bytes / (gate_ms / 1e3) / 1e9
+
+    B, T, H = 1, w.n_tokens, w.hq
+    pooled = torch.empty((B, 1, H, 3), dtype=torch.float32, device=dev)
+    pws_n = nsa.nsa_gate_mlp_pooled_workspace_size(B, T, H, dim)
+    pws = torch.empty(pws_n, dtype=torch.uint8, device=dev)
+
+    def pooled_step(events):
+        rc = nsa.nsa_gate_mlp_pooled(q, w1, b1, w2, b2, B, T, H, dim, 1, pooled, pws, pws_n)
+        if rc != nsa.NSA_OK:
+            raise nsa.NsaError(rc, "nsa_gate_mlp_pooled")
+
+    barrier(world)
+    pms, _ = timed_steps(pooled_step, args.steps, args.warmup, flush, 0)
+    pooled_ms = max_over_ranks(sum(pms), world) / args.steps
+    pooled_gbs = rows * dim * 2 / (pooled_ms / 1e3) / 1e9
+
+    phi = phi_weights(w.hkv, w.cmp_len, seed=22, device=dev)
+    p = nsa.make_params(w.n_tokens, w.n_video, w.hq, w.hkv, w.d, w.cmp_len, w.cmp_stride, w.sel_len, w.top_n,
+                        w.window, out_dtype=nsa.NSA_OUT_BF16)
+    ws = nsa.alloc_workspace(p, False, dev)
+    out = torch.empty((w.n_tokens, w.hq, w.d), dtype=torch.bfloat16, device=dev)
+
+    def phi_step(events):
+        rc = nsa.nsa_prefill_phi(q, k, v, g, phi[0], phi[1], p, out, None, ws, ws.numel())
+        if rc != nsa.NSA_OK:
+            raise nsa.NsaError(rc, "nsa_prefill_phi")
+
+    barrier(world)
+    fms, _ = timed_steps(phi_step, args.steps, args.warmup, flush, 0)
+    assert nsa.nsa_get_device_error(clear=True) == 0, "device error word set during the gate / phi runs"
+    phi_ms = max_over_ranks(sum(fms), world) / args.steps
+    hbm = peaks["hbm_gbs"]
+    del ws, out, gates
+    return {
+        "gate_mlp": {"workload": f"{rows} rows (131,072 tokens x 28 heads) of d={dim}: W1 {dim // 2}x{dim} on the "
+                                 "tensor cores, GELU, W2 3x{0}, softmax".format(dim // 2),
+                     "ms": round(gate_ms, 4),
+                     "roofline": {"bound": "hbm", "achieved": round(gate_gbs, 1), "peak": hbm, "unit": "GB/s",
+                                  "frac": round(gate_gbs / hbm, 4), "peak_source": f"{peaks_src} hbm_gbs",
+                                  "algorithmic": f"{gate_bytes} bytes per launch (x read once, gates written)"}},
+        "gate_mlp_pooled": {"workload": "mean over 131,072 tokens per head (28 heads), then the MLP in fp64",
+                            "ms": round(pooled_ms, 4), "hbm_gbs": round(pooled_gbs, 1),
+                            "frac": round(pooled_gbs / hbm, 4)},
+        "prefill_phi": {"workload": "the headline 128K prefill with the learnable compression",
+                        "ms_per_step": round(phi_ms, 4),
+                        "value": round(w.n_video * world / (phi_ms / 1e3), 1), "unit": "video tokens/s"},
+        "steps": args.steps, "warmup": args.warmup, "l2": "flushed before every timed step",
+        "launches": args.steps * (1 + 2 + PREFILL_KERNELS),
+    }
 
 
 def run_decode(args, dev, peaks, peaks_src, flush, world):
@@ -534,6 +608,7 @@ def main():
     ap.add_argument("--workload", default="v128k", choices=[k for k, v in WORKLOADS.items() if not v.is_decode])
     ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
     ap.add_argument("--no-sweep", action="store_true", help="skip the 128K (n, w) budget sweep")
+    ap.add_argument("--no-gates", action="store_true", help="skip the gate-network and learnable-compression lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     args = ap.parse_args()

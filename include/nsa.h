@@ -163,6 +163,62 @@ int nsa_decode_noalloc(const void* q, const void* kcache, const void* vcache, co
  */
 int nsa_compress(const void* k, const void* v, const nsa_params_t* params, void* kcmp, void* vcmp, void* stream);
 
+/*
+ * Learnable compression. The pages steer the sparse pattern with learned parameters
+ * (shd-paper.top page "VideoNSA: Native Sparse Attention Scales Video Understanding",
+ * section "方法详解", key design (1)) without giving their form; this library's form is a
+ * per-head weighting of the l positions of a block in place of the mean:
+ *   kcmp[b][i][g] = bf16_rne( sum_{u<l} phi_k[g][u] * k[b][i*s+u][g] ), same for v with phi_v.
+ * phi_k, phi_v: device [Hkv][l] fp32, 4-byte aligned; everything else as nsa_compress.
+ * The fp64 sum of exact products is rounded once; phi = 1/l (l a power of two) gives
+ * exactly nsa_compress's mean.
+ */
+int nsa_compress_weighted(const void* k, const void* v, const float* phi_k, const float* phi_v,
+                          const nsa_params_t* params, void* kcmp, void* vcmp, void* stream);
+
+/*
+ * nsa_prefill with the learnable compression above building the compressed keys and
+ * values of the video prefix (phi_k, phi_v: device [Hkv][l] fp32, both required). Same
+ * arguments, workspace, results and errors as nsa_prefill otherwise.
+ */
+int nsa_prefill_phi(const void* q, const void* k, const void* v, const float* gates, const float* phi_k,
+                    const float* phi_v, const nsa_params_t* params, void* out, int32_t* out_sel_idx, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/*
+ * Gate network: three softmax-normalised gates per head from a two-layer MLP, dim -> dim/2
+ * with an exact (erf) GELU, then dim/2 -> 3 (CSDN blog "VideoNSA：重新定义视频理解的稀疏注意力
+ * 机制", vcloud.csdn.net, section 3.1 "动态门控机制详解"). Per row r:
+ *   gates[r] = softmax( W2 . GELU(W1 . x[r] + b1) + b2 )
+ *   x      [rows][dim] bf16, 16-byte aligned; e.g. a prefill's q [N][Hq][d] seen as N*Hq rows
+ *          of dim = d, which yields the [N][Hq][3] gates nsa_prefill takes.
+ *   w1     [dim/2][dim] bf16 (linear-layer layout [out][in]), 16-byte aligned
+ *   b1     [dim/2] fp32     w2 [3][dim/2] fp32     b2 [3] fp32      gates [rows][3] fp32
+ * dim must be 64 or 128 (else NSA_ERR_UNSUPPORTED). The first layer runs on the tensor
+ * cores in fp32 accumulation; rows = 0 enqueues nothing. All pointers are device memory
+ * owned by the caller; errors (NSA_ERR_INVALID_ARG for null or misaligned pointers, rows
+ * < 0) are returned before anything is enqueued.
+ */
+int nsa_gate_mlp(const void* x, const void* w1, const float* b1, const float* w2, const float* b2, int64_t rows,
+                 int dim, float* gates, void* stream);
+
+/*
+ * The blog's averaged gate: the MLP above applied, per sequence and head, to the mean of
+ * x over the sequence's tokens, all in fp64.
+ *   x       [batch][seq_len][heads][dim] bf16, 16-byte aligned
+ *   gates   [batch][repeat][heads][3] fp32: the triple of (b, h) written to every r < repeat
+ *           (repeat = 1 gives nsa_decode's [B][Hq][3]; repeat = seq_len gives per-token gates
+ *           for nsa_prefill)
+ *   workspace  device scratch of nsa_gate_mlp_pooled_workspace_size(...) bytes, 256-byte aligned
+ * Weights, dim and errors as nsa_gate_mlp, plus NSA_ERR_WORKSPACE_TOO_SMALL.
+ */
+int nsa_gate_mlp_pooled(const void* x, const void* w1, const float* b1, const float* w2, const float* b2, int batch,
+                        int seq_len, int heads, int dim, int repeat, float* gates, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/* Workspace bytes nsa_gate_mlp_pooled needs; 0 if the arguments are invalid. */
+size_t nsa_gate_mlp_pooled_workspace_size(int batch, int seq_len, int heads, int dim);
+
 /* Workspace bytes nsa_prefill (is_decode = 0) or nsa_decode (is_decode = 1) needs; 0 if params are invalid. */
 size_t nsa_workspace_size(const nsa_params_t* params, int is_decode);
 

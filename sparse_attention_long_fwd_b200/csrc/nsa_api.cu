@@ -18,6 +18,7 @@
 #include "sel.cuh"
 #include "sel_inv.cuh"
 #include "decode.cuh"
+#include "gate.cuh"
 
 namespace {
 
@@ -32,6 +33,7 @@ int ncmp_of(int T, int l, int s) { return T >= l ? (T - l) / s + 1 : 0; }
 int nsel_of(int T, int ls) { return (T + ls - 1) / ls; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 // Checks shared by every entry point. Returns NSA_OK or an error code.
 int check_common(const nsa_params_t* p) {
@@ -207,14 +209,15 @@ int set_smem(K kernel, size_t bytes) {
 }
 
 // ------------------------------------------------------------------ launchers
+// wk, wv: per-head block weights [hkv][l] of the learnable compression, or null for the mean
 int launch_pool(const void* k, const void* v, void* kc, void* vc, int nseq, int T, int hkv, int d, int ncmp, int l,
-                int s, cudaStream_t st) {
+                int s, cudaStream_t st, const float* wk = nullptr, const float* wv = nullptr) {
   if (ncmp <= 0) return NSA_OK;
   const long long threads = static_cast<long long>(nseq) * ncmp * hkv * (d / 2);
   const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
   nsa::pool_kernel<<<dim3(blocks, 1, 2), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(kc),
-      static_cast<__nv_bfloat16*>(vc), nseq, T, hkv, d, ncmp, l, s);
+      static_cast<__nv_bfloat16*>(vc), wk, wv, nseq, T, hkv, d, ncmp, l, s);
   return launch_status("pool", st);
 }
 
@@ -237,7 +240,8 @@ int launch_attn(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap&
 
 template <int D>
 int prefill_impl(const nsa_params_t* p, const void* q, const void* k, const void* v, const float* gates, void* out,
-                 int32_t* out_sel_idx, uint8_t* ws, cudaStream_t st) {
+                 int32_t* out_sel_idx, uint8_t* ws, cudaStream_t st, const float* phi_k = nullptr,
+                 const float* phi_v = nullptr) {
   const PrefillLayout L = prefill_layout(p);
   const int N = p->n_tokens, nv = p->n_video, hq = p->num_q_heads, hkv = p->num_kv_heads;
   const int G = hq / hkv;
@@ -278,7 +282,9 @@ int prefill_impl(const nsa_params_t* p, const void* q, const void* k, const void
         !nsa::make_tmap_bf16_3d(&qcmap, q, D, hq, N, qs1, qs2, 64, Gc, Tc))
       return NSA_ERR_CUDA;
     // 1. compression: Kc, Vc of the video prefix
-    if ((rc = launch_pool(k, v, kc, vc, 1, nv, hkv, D, L.ncmp, p->cmp_block, p->cmp_stride, st)) != NSA_OK) return rc;
+    if ((rc = launch_pool(k, v, kc, vc, 1, nv, hkv, D, L.ncmp, p->cmp_block, p->cmp_stride, st, phi_k, phi_v)) !=
+        NSA_OK)
+      return rc;
     // 2. compressed branch + block scores
     a.q_begin = 0;
     a.q_end = nv;
@@ -550,8 +556,12 @@ int nsa_prefill_workspace_layout(const nsa_params_t* params, nsa_prefill_layout_
   return NSA_OK;
 }
 
-int nsa_prefill(const void* q, const void* k, const void* v, const float* gates, const nsa_params_t* params,
-                void* out, int32_t* out_sel_idx, void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+int prefill_entry(const void* q, const void* k, const void* v, const float* gates, const float* phi_k,
+                  const float* phi_v, const nsa_params_t* params, void* out, int32_t* out_sel_idx, void* workspace,
+                  size_t workspace_bytes, void* stream) {
   int rc = check_common(params);
   if (rc != NSA_OK) return rc;
   if (params->n_video < 0 || params->n_video > params->n_tokens) return NSA_ERR_INVALID_ARG;
@@ -565,8 +575,24 @@ int nsa_prefill(const void* q, const void* k, const void* v, const float* gates,
   auto* ws = static_cast<uint8_t*>(workspace);
   auto st = static_cast<cudaStream_t>(stream);
   stage_begin(st);
-  if (params->head_dim == 64) return prefill_impl<64>(params, q, k, v, gates, out, out_sel_idx, ws, st);
-  return prefill_impl<128>(params, q, k, v, gates, out, out_sel_idx, ws, st);
+  if (params->head_dim == 64) return prefill_impl<64>(params, q, k, v, gates, out, out_sel_idx, ws, st, phi_k, phi_v);
+  return prefill_impl<128>(params, q, k, v, gates, out, out_sel_idx, ws, st, phi_k, phi_v);
+}
+}  // namespace
+
+extern "C" {
+
+int nsa_prefill(const void* q, const void* k, const void* v, const float* gates, const nsa_params_t* params,
+                void* out, int32_t* out_sel_idx, void* workspace, size_t workspace_bytes, void* stream) {
+  return prefill_entry(q, k, v, gates, nullptr, nullptr, params, out, out_sel_idx, workspace, workspace_bytes,
+                       stream);
+}
+
+int nsa_prefill_phi(const void* q, const void* k, const void* v, const float* gates, const float* phi_k,
+                    const float* phi_v, const nsa_params_t* params, void* out, int32_t* out_sel_idx, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  if (!phi_k || !phi_v || !aligned4(phi_k) || !aligned4(phi_v)) return NSA_ERR_INVALID_ARG;
+  return prefill_entry(q, k, v, gates, phi_k, phi_v, params, out, out_sel_idx, workspace, workspace_bytes, stream);
 }
 
 size_t nsa_prefill_varlen_workspace_size(const nsa_params_t* params, const int32_t* cu_seqlens,
@@ -699,6 +725,114 @@ int nsa_compress(const void* k, const void* v, const nsa_params_t* params, void*
   const int ncmp = ncmp_of(params->n_tokens, params->cmp_block, params->cmp_stride);
   return launch_pool(k, v, kcmp, vcmp, params->batch, params->n_tokens, params->num_kv_heads, params->head_dim, ncmp,
                      params->cmp_block, params->cmp_stride, static_cast<cudaStream_t>(stream));
+}
+
+int nsa_compress_weighted(const void* k, const void* v, const float* phi_k, const float* phi_v,
+                          const nsa_params_t* params, void* kcmp, void* vcmp, void* stream) {
+  int rc = check_common(params);
+  if (rc != NSA_OK) return rc;
+  if (params->batch < 1 || !k || !v || !kcmp || !vcmp || !phi_k || !phi_v) return NSA_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(kcmp) || !aligned16(vcmp) || !aligned4(phi_k) ||
+      !aligned4(phi_v))
+    return NSA_ERR_INVALID_ARG;
+  if ((rc = check_device()) != NSA_OK) return rc;
+  const int ncmp = ncmp_of(params->n_tokens, params->cmp_block, params->cmp_stride);
+  return launch_pool(k, v, kcmp, vcmp, params->batch, params->n_tokens, params->num_kv_heads, params->head_dim, ncmp,
+                     params->cmp_block, params->cmp_stride, static_cast<cudaStream_t>(stream), phi_k, phi_v);
+}
+
+// ------------------------------------------------------------------ gate network
+}  // extern "C"
+
+namespace {
+
+bool gate_weights_ok(const void* w1, const float* b1, const float* w2, const float* b2) {
+  return w1 && b1 && w2 && b2 && aligned16(w1) && aligned4(b1) && aligned4(w2) && aligned4(b2);
+}
+
+template <int DIM>
+int launch_gate_mlp(const void* x, const void* w1, const float* b1, const float* w2, const float* b2, int64_t rows,
+                    float* gates, cudaStream_t st) {
+  CUtensorMap xmap, wmap;
+  const uint64_t pitch = static_cast<uint64_t>(DIM) * 2;
+  if (!nsa::make_tmap_bf16_3d(&xmap, x, DIM, static_cast<uint64_t>(rows), 1, pitch, pitch * rows, 64, 128, 1) ||
+      !nsa::make_tmap_bf16_3d(&wmap, w1, DIM, DIM / 2, 1, pitch, pitch * (DIM / 2), 64, DIM / 2, 1))
+    return NSA_ERR_CUDA;
+  const size_t smem = sizeof(nsa::GateSmem<DIM>) + 1024;
+  auto kern = nsa::gate_mlp_kernel<DIM>;
+  if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>((rows + 127) / 128);
+  kern<<<grid, 128, smem, st>>>(xmap, wmap, b1, w2, b2, gates, static_cast<long long>(rows));
+  return launch_status("gate_mlp", st, false);
+}
+
+// Token chunk of the averaged gate's first pass: about 1,184 CTAs (8 per SM of a 148-SM
+// part) over the whole batch, at least 64 tokens each. Fixed by the shapes alone, so the
+// workspace size does not depend on the device.
+int gate_chunk(int batch, int seq_len) {
+  const int per_seq = batch >= 1184 ? 1 : 1184 / batch;
+  const int c = (seq_len + per_seq - 1) / per_seq;
+  return c < 64 ? 64 : c;
+}
+
+bool pooled_args_ok(int batch, int seq_len, int heads, int dim, int repeat) {
+  return batch >= 1 && seq_len >= 1 && heads >= 1 && repeat >= 1 && (dim == 64 || dim == 128) &&
+         static_cast<long long>(heads) * dim <= (1LL << 20);
+}
+
+}  // namespace
+
+extern "C" {
+
+int nsa_gate_mlp(const void* x, const void* w1, const float* b1, const float* w2, const float* b2, int64_t rows,
+                 int dim, float* gates, void* stream) {
+  if (!x || !gates || rows < 0 || !gate_weights_ok(w1, b1, w2, b2)) return NSA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned4(gates)) return NSA_ERR_INVALID_ARG;
+  if (dim != 64 && dim != 128) return NSA_ERR_UNSUPPORTED;
+  if (rows > (1LL << 31) - 128) return NSA_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
+  if (rows == 0) return NSA_OK;
+  int rc = check_device();
+  if (rc != NSA_OK) return rc;
+  auto st = static_cast<cudaStream_t>(stream);
+  return dim == 64 ? launch_gate_mlp<64>(x, w1, b1, w2, b2, rows, gates, st)
+                   : launch_gate_mlp<128>(x, w1, b1, w2, b2, rows, gates, st);
+}
+
+size_t nsa_gate_mlp_pooled_workspace_size(int batch, int seq_len, int heads, int dim) {
+  if (!pooled_args_ok(batch, seq_len, heads, dim, 1)) return 0;
+  const int chunk = gate_chunk(batch, seq_len);
+  const size_t nchunk = static_cast<size_t>((seq_len + chunk - 1) / chunk);
+  return align_up(nchunk * batch * heads * dim * sizeof(double));
+}
+
+int nsa_gate_mlp_pooled(const void* x, const void* w1, const float* b1, const float* w2, const float* b2, int batch,
+                        int seq_len, int heads, int dim, int repeat, float* gates, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  if (!x || !gates || !workspace || !gate_weights_ok(w1, b1, w2, b2)) return NSA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned4(gates) || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+    return NSA_ERR_INVALID_ARG;
+  if (!pooled_args_ok(batch, seq_len, heads, dim, repeat)) return dim == 64 || dim == 128 ? NSA_ERR_INVALID_ARG
+                                                                                           : NSA_ERR_UNSUPPORTED;
+  if (workspace_bytes < nsa_gate_mlp_pooled_workspace_size(batch, seq_len, heads, dim))
+    return NSA_ERR_WORKSPACE_TOO_SMALL;
+  int rc = check_device();
+  if (rc != NSA_OK) return rc;
+  auto st = static_cast<cudaStream_t>(stream);
+  const int chunk = gate_chunk(batch, seq_len);
+  const int nchunk = (seq_len + chunk - 1) / chunk;
+  auto* part = static_cast<double*>(workspace);
+  nsa::gate_mean_partial_kernel<<<dim3(nchunk, batch), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), part,
+                                                                      batch, seq_len, heads * dim, chunk);
+  if ((rc = launch_status("gate_mean_partial", st, false)) != NSA_OK) return rc;
+  const unsigned grid = static_cast<unsigned>(batch) * heads;
+  const auto* w1b = static_cast<const __nv_bfloat16*>(w1);
+  if (dim == 64)
+    nsa::gate_pooled_kernel<64><<<grid, 64, 0, st>>>(part, w1b, b1, w2, b2, gates, batch, seq_len, heads, nchunk,
+                                                      repeat);
+  else
+    nsa::gate_pooled_kernel<128><<<grid, 128, 0, st>>>(part, w1b, b1, w2, b2, gates, batch, seq_len, heads, nchunk,
+                                                        repeat);
+  return launch_status("gate_pooled", st, false);
 }
 
 int nsa_profile_stages(void* const* events, int count) {

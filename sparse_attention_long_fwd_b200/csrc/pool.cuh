@@ -11,6 +11,14 @@
 // odd at a precision with >= 2 extra bits makes the second rounding correct, Boldo &
 // Melquiond, "When double rounding is odd", 2005).
 //
+// Learnable form: the pages steer the sparse pattern with learned parameters
+// (shd-paper.top page "VideoNSA: Native Sparse Attention Scales Video Understanding",
+// section "方法详解", key design (1)) without giving their form. Given per-head weights
+// w [hkv][l] (fp32), a summary is the weighted sum instead of the mean:
+//   Kc[i][g] = bf16_rne( sum_{u<l} w[g][u] * K[i*s + u][g] ).
+// An fp32 weight times a bf16 key is exact in fp64, so this sum is rounded exactly like
+// the mean's; w = 1/l with l a power of two reproduces the mean bit for bit.
+//
 // HBM-bound: each token row is read by l/s = 2 overlapping blocks (the second read hits
 // L2); one thread owns two adjacent dims (a bf16x2 word) of one (sequence, block, head).
 #pragma once
@@ -26,13 +34,16 @@ __device__ __forceinline__ __nv_bfloat16 f64_to_bf16_rne(double x) {
 }
 
 // src: [nseq][T][hkv][d] bf16; dst: [nseq][ncmp][hkv][d] bf16. blockIdx.z: 0 -> K, 1 -> V.
+// wk, wv: [hkv][l] fp32 weights of the learnable form, or both null for the mean.
 // Each thread handles one bf16x2 column pair of one (seq, block i, head g).
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ k,
                                                    const __nv_bfloat16* __restrict__ v,
                                                    __nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict__ vc,
+                                                   const float* __restrict__ wk, const float* __restrict__ wv,
                                                    int nseq, int T, int hkv, int d, int ncmp, int l, int s) {
   const __nv_bfloat16* src = blockIdx.z == 0 ? k : v;
   __nv_bfloat16* dst = blockIdx.z == 0 ? kc : vc;
+  const float* w = blockIdx.z == 0 ? wk : wv;
   const int pairs = d / 2;
   const long long total = static_cast<long long>(nseq) * ncmp * hkv * pairs;
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -47,15 +58,27 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   const __nv_bfloat162* in = reinterpret_cast<const __nv_bfloat162*>(
       src + (static_cast<size_t>(b) * T + static_cast<size_t>(i) * s) * row_elems + static_cast<size_t>(g) * d) + p;
   double a0 = 0.0, a1 = 0.0;
-  for (int u = 0; u < l; ++u) {
-    const float2 x = __bfloat1622float2(in[static_cast<size_t>(u) * (row_elems / 2)]);
-    a0 += static_cast<double>(x.x);
-    a1 += static_cast<double>(x.y);
-  }
-  const double dl = static_cast<double>(l);
   __nv_bfloat162 o;
-  o.x = f64_to_bf16_rne(a0 / dl);
-  o.y = f64_to_bf16_rne(a1 / dl);
+  if (w == nullptr) {
+    for (int u = 0; u < l; ++u) {
+      const float2 x = __bfloat1622float2(in[static_cast<size_t>(u) * (row_elems / 2)]);
+      a0 += static_cast<double>(x.x);
+      a1 += static_cast<double>(x.y);
+    }
+    const double dl = static_cast<double>(l);
+    o.x = f64_to_bf16_rne(a0 / dl);
+    o.y = f64_to_bf16_rne(a1 / dl);
+  } else {
+    const float* wg = w + static_cast<size_t>(g) * l;
+    for (int u = 0; u < l; ++u) {
+      const float2 x = __bfloat1622float2(in[static_cast<size_t>(u) * (row_elems / 2)]);
+      const double wu = static_cast<double>(__ldg(wg + u));
+      a0 += wu * static_cast<double>(x.x);  // exact product: fusing it into an fma changes nothing
+      a1 += wu * static_cast<double>(x.y);
+    }
+    o.x = f64_to_bf16_rne(a0);
+    o.y = f64_to_bf16_rne(a1);
+  }
   reinterpret_cast<__nv_bfloat162*>(dst + ((static_cast<size_t>(b) * ncmp + i) * hkv + g) * d)[p] = o;
 }
 

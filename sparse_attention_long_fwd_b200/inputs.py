@@ -106,6 +106,27 @@ def decode_inputs(w: Workload, seed: int = 0, device="cpu", seq_lens=None):
     return q, kc, vc, gates, seq_lens
 
 
+def phi_weights(hkv: int, l: int = 32, seed: int = 0, device="cpu"):
+    """Weights of the learnable compression, phi_k and phi_v [hkv, l] fp32: (1 + N(0, 0.25)) / l,
+    a perturbed mean."""
+    g = _gen(seed, device)
+    wk = (1.0 + 0.5 * torch.randn((hkv, l), generator=g, device=device)) / l
+    wv = (1.0 + 0.5 * torch.randn((hkv, l), generator=g, device=device)) / l
+    return wk.contiguous(), wv.contiguous()
+
+
+def gate_weights(dim: int, seed: int = 0, device="cpu"):
+    """Gate-network weights: W1 [dim/2, dim] bf16 ~ N(0, 1/dim); b1 [dim/2] ~ N(0, 0.01);
+    W2 [3, dim/2] ~ N(0, 2/dim); b2 [3] ~ N(0, 0.01) (fp32)."""
+    g = _gen(seed, device)
+    hid = dim // 2
+    w1 = (torch.randn((hid, dim), generator=g, device=device) / dim ** 0.5).to(torch.bfloat16)
+    b1 = torch.randn((hid,), generator=g, device=device) * 0.1
+    w2 = torch.randn((3, hid), generator=g, device=device) / hid ** 0.5
+    b2 = torch.randn((3,), generator=g, device=device) * 0.1
+    return w1, b1, w2, b2
+
+
 def bf16_bits(t: torch.Tensor):
     """Raw 16-bit patterns of a bf16 tensor as a numpy uint16 array (host copy)."""
     import numpy as np

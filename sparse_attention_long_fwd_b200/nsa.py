@@ -29,7 +29,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnsa_b200
 EXPORTED = (
     "nsa_prefill", "nsa_decode", "nsa_compress", "nsa_workspace_size", "nsa_prefill_workspace_layout",
     "nsa_error_string", "nsa_get_device_error", "nsa_version", "nsa_profile_stages", "nsa_decode_noalloc",
-    "nsa_prefill_varlen", "nsa_prefill_varlen_workspace_size",
+    "nsa_prefill_varlen", "nsa_prefill_varlen_workspace_size", "nsa_compress_weighted", "nsa_prefill_phi",
+    "nsa_gate_mlp", "nsa_gate_mlp_pooled", "nsa_gate_mlp_pooled_workspace_size",
 )
 
 
@@ -87,6 +88,16 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.nsa_decode_noalloc.restype = I
     lib.nsa_compress.argtypes = [P, P, PP, P, P, P]
     lib.nsa_compress.restype = I
+    lib.nsa_compress_weighted.argtypes = [P, P, P, P, PP, P, P, P]
+    lib.nsa_compress_weighted.restype = I
+    lib.nsa_prefill_phi.argtypes = [P, P, P, P, P, P, PP, P, P, P, S, P]
+    lib.nsa_prefill_phi.restype = I
+    lib.nsa_gate_mlp.argtypes = [P, P, P, P, P, ctypes.c_int64, I, P, P]
+    lib.nsa_gate_mlp.restype = I
+    lib.nsa_gate_mlp_pooled.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P, S, P]
+    lib.nsa_gate_mlp_pooled.restype = I
+    lib.nsa_gate_mlp_pooled_workspace_size.argtypes = [I, I, I, I]
+    lib.nsa_gate_mlp_pooled_workspace_size.restype = S
     lib.nsa_workspace_size.argtypes = [PP, I]
     lib.nsa_workspace_size.restype = S
     lib.nsa_prefill_workspace_layout.argtypes = [PP, ctypes.POINTER(NsaPrefillLayout)]
@@ -176,6 +187,34 @@ def nsa_compress(k, v, params: NsaParams, kcmp, vcmp, stream=None) -> int:
                                        _stream(stream))
 
 
+def nsa_compress_weighted(k, v, phi_k, phi_v, params: NsaParams, kcmp, vcmp, stream=None) -> int:
+    return load_library().nsa_compress_weighted(_addr(k), _addr(v), _addr(phi_k), _addr(phi_v), ctypes.byref(params),
+                                                _addr(kcmp), _addr(vcmp), _stream(stream))
+
+
+def nsa_prefill_phi(q, k, v, gates, phi_k, phi_v, params: NsaParams, out, out_sel_idx, workspace,
+                    workspace_bytes: int, stream=None) -> int:
+    return load_library().nsa_prefill_phi(_addr(q), _addr(k), _addr(v), _addr(gates), _addr(phi_k), _addr(phi_v),
+                                          ctypes.byref(params), _addr(out), _addr(out_sel_idx), _addr(workspace),
+                                          workspace_bytes, _stream(stream))
+
+
+def nsa_gate_mlp(x, w1, b1, w2, b2, rows: int, dim: int, gates, stream=None) -> int:
+    return load_library().nsa_gate_mlp(_addr(x), _addr(w1), _addr(b1), _addr(w2), _addr(b2), rows, dim,
+                                       _addr(gates), _stream(stream))
+
+
+def nsa_gate_mlp_pooled(x, w1, b1, w2, b2, batch: int, seq_len: int, heads: int, dim: int, repeat: int, gates,
+                        workspace, workspace_bytes: int, stream=None) -> int:
+    return load_library().nsa_gate_mlp_pooled(_addr(x), _addr(w1), _addr(b1), _addr(w2), _addr(b2), batch, seq_len,
+                                              heads, dim, repeat, _addr(gates), _addr(workspace), workspace_bytes,
+                                              _stream(stream))
+
+
+def nsa_gate_mlp_pooled_workspace_size(batch: int, seq_len: int, heads: int, dim: int) -> int:
+    return int(load_library().nsa_gate_mlp_pooled_workspace_size(batch, seq_len, heads, dim))
+
+
 def nsa_workspace_size(params: NsaParams, is_decode: bool) -> int:
     return int(load_library().nsa_workspace_size(ctypes.byref(params), int(bool(is_decode))))
 
@@ -233,8 +272,9 @@ def alloc_workspace(params: NsaParams, is_decode: bool, device) -> torch.Tensor:
 
 def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gates: torch.Tensor, *, n_video: int | None = None,
             top_n: int = 16, window: int = 512, softmax_scale: float = 0.0, out_dtype=torch.float32,
-            return_sel: bool = False, workspace: torch.Tensor | None = None, stream=None):
-    """NSA prefill of one sequence: q [N,Hq,d], k/v [N,Hkv,d] bf16, gates [N,Hq,3] fp32 (device tensors)."""
+            return_sel: bool = False, workspace: torch.Tensor | None = None, phi=None, stream=None):
+    """NSA prefill of one sequence: q [N,Hq,d], k/v [N,Hkv,d] bf16, gates [N,Hq,3] fp32 (device tensors).
+    phi = (phi_k, phi_v), each [Hkv, 32] fp32, selects the learnable compression."""
     N, hq, d = q.shape
     hkv = k.shape[1]
     p = make_params(N, n_video, hq, hkv, d, top_n=top_n, window=window, softmax_scale=softmax_scale,
@@ -243,12 +283,17 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gates: torch.Tens
     sel = torch.empty((p.n_video, hkv, top_n), dtype=torch.int32, device=q.device) if return_sel else None
     if workspace is None:
         workspace = alloc_workspace(p, False, q.device)
-    _check(nsa_prefill(q, k, v, gates, p, out, sel, workspace, workspace.numel(), stream), "nsa_prefill")
+    if phi is None:
+        _check(nsa_prefill(q, k, v, gates, p, out, sel, workspace, workspace.numel(), stream), "nsa_prefill")
+    else:
+        _check(nsa_prefill_phi(q, k, v, gates, phi[0], phi[1], p, out, sel, workspace, workspace.numel(), stream),
+               "nsa_prefill_phi")
     return (out, sel) if return_sel else out
 
 
-def compress(k: torch.Tensor, v: torch.Tensor, stream=None):
-    """Compressed cache of a [B, L, Hkv, d] (or [L, Hkv, d]) bf16 K/V pair."""
+def compress(k: torch.Tensor, v: torch.Tensor, phi=None, stream=None):
+    """Compressed cache of a [B, L, Hkv, d] (or [L, Hkv, d]) bf16 K/V pair; phi = (phi_k, phi_v),
+    each [Hkv, 32] fp32, selects the learnable compression."""
     squeeze = k.dim() == 3
     if squeeze:
         k, v = k.unsqueeze(0), v.unsqueeze(0)
@@ -257,7 +302,10 @@ def compress(k: torch.Tensor, v: torch.Tensor, stream=None):
     nc = (L - 32) // 16 + 1 if L >= 32 else 0
     kc = torch.empty((B, nc, hkv, d), dtype=k.dtype, device=k.device)
     vc = torch.empty_like(kc)
-    _check(nsa_compress(k, v, p, kc, vc, stream), "nsa_compress")
+    if phi is None:
+        _check(nsa_compress(k, v, p, kc, vc, stream), "nsa_compress")
+    else:
+        _check(nsa_compress_weighted(k, v, phi[0], phi[1], p, kc, vc, stream), "nsa_compress_weighted")
     return (kc[0], vc[0]) if squeeze else (kc, vc)
 
 
@@ -276,6 +324,24 @@ def decode(q, kcache, vcache, kcmp, vcmp, seq_lens, gates, *, top_n: int = 16, w
     _check(nsa_decode(q, kcache, vcache, kcmp, vcmp, seq_lens, gates, p, out, sel, workspace, workspace.numel(),
                       stream), "nsa_decode")
     return (out, sel) if return_sel else out
+
+
+def gate_mlp(x: torch.Tensor, w1: torch.Tensor, b1: torch.Tensor, w2: torch.Tensor, b2: torch.Tensor, stream=None):
+    """Per-row gates: x [..., dim] bf16 -> [..., 3] fp32 (w1 [dim/2, dim] bf16; b1, w2, b2 fp32)."""
+    dim = x.shape[-1]
+    gates = torch.empty((*x.shape[:-1], 3), dtype=torch.float32, device=x.device)
+    _check(nsa_gate_mlp(x, w1, b1, w2, b2, x.numel() // dim, dim, gates, stream), "nsa_gate_mlp")
+    return gates
+
+
+def gate_mlp_pooled(x: torch.Tensor, w1, b1, w2, b2, repeat: int = 1, stream=None):
+    """Averaged gates: x [B, T, H, dim] bf16 -> [B, repeat, H, 3] fp32 (the (b, h) triple repeated)."""
+    B, T, H, dim = x.shape
+    gates = torch.empty((B, repeat, H, 3), dtype=torch.float32, device=x.device)
+    ws = torch.empty(max(nsa_gate_mlp_pooled_workspace_size(B, T, H, dim), 1), dtype=torch.uint8, device=x.device)
+    _check(nsa_gate_mlp_pooled(x, w1, b1, w2, b2, B, T, H, dim, repeat, gates, ws, ws.numel(), stream),
+           "nsa_gate_mlp_pooled")
+    return gates
 
 
 def default_scale(d: int) -> float:

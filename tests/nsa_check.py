@@ -22,14 +22,19 @@ def oracle_cfg(w: Workload) -> orc.OracleConfig:
                             w.window)
 
 
-def run_prefill(w: Workload, q, k, v, gates, out_dtype=torch.float32):
-    """Call nsa_prefill through the C ABI; returns (out, sel, workspace, layout)."""
+def run_prefill(w: Workload, q, k, v, gates, out_dtype=torch.float32, phi=None):
+    """Call nsa_prefill (nsa_prefill_phi when phi = (phi_k, phi_v) is given) through the C ABI;
+    returns (out, sel, workspace, layout)."""
     p = nsa.make_params(w.n_tokens, w.n_video, w.hq, w.hkv, w.d, w.cmp_len, w.cmp_stride, w.sel_len, w.top_n,
                         w.window, out_dtype=nsa.NSA_OUT_F32 if out_dtype == torch.float32 else nsa.NSA_OUT_BF16)
     ws = nsa.alloc_workspace(p, False, q.device)
     out = torch.empty((w.n_tokens, w.hq, w.d), dtype=out_dtype, device=q.device)
     sel = torch.full((max(w.n_video, 1), w.hkv, w.top_n), -7, dtype=torch.int32, device=q.device)
-    rc = nsa.nsa_prefill(q, k, v, gates, p, out, sel if w.n_video > 0 else None, ws, ws.numel())
+    sel_arg = sel if w.n_video > 0 else None
+    if phi is None:
+        rc = nsa.nsa_prefill(q, k, v, gates, p, out, sel_arg, ws, ws.numel())
+    else:
+        rc = nsa.nsa_prefill_phi(q, k, v, gates, phi[0], phi[1], p, out, sel_arg, ws, ws.numel())
     assert rc == nsa.NSA_OK, nsa.nsa_error_string(rc)
     torch.cuda.synchronize()
     assert nsa.nsa_get_device_error(clear=True) == 0
@@ -79,14 +84,19 @@ def assert_close(got: np.ndarray, ref: np.ndarray, what: str, max_abs=MAX_ABS, m
 
 
 def compare_prefill_rows(w: Workload, q, k, v, gates, rows, out, sel, ws, layout, check_intermediates=True,
-                         nthreads=0):
-    """Element-wise comparison of the listed rows against the oracle (plus replay on near-ties)."""
+                         nthreads=0, phi=None):
+    """Element-wise comparison of the listed rows against the oracle (plus replay on near-ties).
+    phi = (phi_k, phi_v) selects the oracle's learnable compression."""
     qb, kb, vb = host_bits(q, k, v)
     g = gates.detach().cpu().numpy()
     rows = np.asarray(rows, dtype=np.int32)
     cfg = oracle_cfg(w)
-    kc_o = orc.compress(kb[: w.n_video])
-    vc_o = orc.compress(vb[: w.n_video])
+    if phi is None:
+        kc_o = orc.compress(kb[: w.n_video])
+        vc_o = orc.compress(vb[: w.n_video])
+    else:
+        kc_o = orc.compress_weighted(kb[: w.n_video], phi[0].cpu().numpy())
+        vc_o = orc.compress_weighted(vb[: w.n_video], phi[1].cpu().numpy())
     o = orc.prefill_rows(cfg, qb, kb, vb, g, rows, kc=kc_o, vc=vc_o, nthreads=nthreads)
     vid = rows < w.n_video
     vrows = rows[vid]

@@ -134,3 +134,29 @@ def test_prefill_varlen_workspace_is_the_largest_sequence():
     assert need == single
     f = 1 << 20
     assert nsa.nsa_prefill_varlen(f, f, f, f, cu, nv, p, f, None, f, need - 1, None) == nsa.NSA_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_learnable_compression_and_gate_validation():
+    f = 1 << 20
+    p = _p()
+    pc = nsa.make_params(64, batch=1)
+    # learnable compression: both weight arrays are required and 4-byte aligned
+    assert nsa.nsa_compress_weighted(f, f, None, f, pc, f, f, None) == nsa.NSA_ERR_INVALID_ARG
+    assert nsa.nsa_compress_weighted(f, f, f, f + 2, pc, f, f, None) == nsa.NSA_ERR_INVALID_ARG
+    assert nsa.nsa_prefill_phi(f, f, f, f, None, f, p, f, None, f, 1 << 40, None) == nsa.NSA_ERR_INVALID_ARG
+    assert nsa.nsa_prefill_phi(f, f, f, f, f, f, p, f, None, f, 1000, None) == nsa.NSA_ERR_WORKSPACE_TOO_SMALL
+    # gate MLP
+    assert nsa.nsa_gate_mlp(f, f, f, f, f, 100, 128, None, None) == nsa.NSA_ERR_INVALID_ARG
+    assert nsa.nsa_gate_mlp(f + 8, f, f, f, f, 100, 128, f, None) == nsa.NSA_ERR_INVALID_ARG
+    assert nsa.nsa_gate_mlp(f, f, f, f, f, -1, 128, f, None) == nsa.NSA_ERR_INVALID_ARG
+    assert nsa.nsa_gate_mlp(f, f, f, f, f, 100, 96, f, None) == nsa.NSA_ERR_UNSUPPORTED
+    assert nsa.nsa_gate_mlp(f, f, f, f, f, 0, 128, f, None) == nsa.NSA_OK  # nothing to do, nothing enqueued
+    # averaged gate: workspace sizing and checks
+    need = nsa.nsa_gate_mlp_pooled_workspace_size(2, 131072, 28, 128)
+    assert need > 0 and need % 256 == 0 and need <= 8 * 1184 * 28 * 128 + 256
+    assert nsa.nsa_gate_mlp_pooled_workspace_size(0, 10, 28, 128) == 0
+    assert nsa.nsa_gate_mlp_pooled_workspace_size(1, 10, 28, 96) == 0
+    assert nsa.nsa_gate_mlp_pooled(f, f, f, f, f, 2, 131072, 28, 128, 1, f, f, need - 1, None) == \
+        nsa.NSA_ERR_WORKSPACE_TOO_SMALL
+    assert nsa.nsa_gate_mlp_pooled(f, f, f, f, f, 2, 131072, 28, 128, 0, f, f, need, None) == nsa.NSA_ERR_INVALID_ARG
+    assert nsa.nsa_gate_mlp_pooled(f, f, f, f, f, 1, 100, 28, 96, 1, f, f, 1 << 30, None) == nsa.NSA_ERR_UNSUPPORTED
