@@ -47,7 +47,7 @@ PREFILL_KERNELS = 9
 # DRAM bytes per launch of a stage's kernel on the 128K workload, from one ncu capture of the
 # current kernel version (profiles/dram_traffic_v128k.md); an entry is removed when its kernel
 # changes, and the roofline then reports traffic null.
-STAGE_TRAFFIC_V128K = {"cmp_attn_scores": 4989331456}
+STAGE_TRAFFIC_V128K = {"cmp_attn_scores": 4043696128}
 DECODE_STAGES = ["dec_cmp_and_window", "dec_select", "dec_selected_and_combine"]
 
 
