@@ -510,3 +510,122 @@ def test_pooled_gates_match_blog_module_per_head():
     same = np.repeat(x[:, :1], T, axis=1)
     assert np.allclose(gate_orc.gate_mlp_pooled(same, w1, b1, w2, b2),
                        gate_orc.gate_mlp(same[:, 0], w1, b1, w2, b2), atol=1e-14)
+
+
+# ---------------------------------------------------------------- backward
+
+from oracle import backward as bwd_orc  # noqa: E402
+
+
+def _bwd_case(N, nv, hq, hkv, d, seed, top_n=4, window=40):
+    cfg = orc.OracleConfig(N, nv, hq, hkv, d, top_n=top_n, window=window)
+    q = _bits(_rand_bf16((N, hq, d), seed))
+    k = _bits(_rand_bf16((N, hkv, d), seed + 1))
+    v = _bits(_rand_bf16((N, hkv, d), seed + 2))
+    g = torch.rand((N, hq, 3), generator=torch.Generator().manual_seed(seed + 3)).numpy().astype(np.float32)
+    dout = _bits(_rand_bf16((N, hq, d), seed + 4))
+    o = orc.prefill_rows(cfg, q, k, v, g, np.arange(N, dtype=np.int32), want=("sel",))
+    return cfg, q, k, v, g, dout, o
+
+
+def test_backward_forward_equals_the_forward_oracle():
+    # the backward's own forward (key sets, compression, combine, text rows) against the C oracle
+    cfg, q, k, v, g, dout, o = _bwd_case(300, 260, 4, 2, 16, 50)
+    r = bwd_orc.prefill_backward(cfg, q, k, v, g, dout, o["sel"][: cfg.n_video])
+    assert np.abs(r["out"] - o["out"]).max() < 1e-12
+
+
+def _loss_and_grads(cfg, q, k, v, g, dout, sel, phi=None):
+    kc = bwd_orc.compressed_f64(k[: cfg.n_video], cfg, phi, rounded=False)
+    vc = bwd_orc.compressed_f64(v[: cfg.n_video], cfg, phi, rounded=False)
+    r = bwd_orc.forward_backward(cfg, q, k, v, g, dout, sel, kc, vc, phi)
+    return float((r["out"] * dout).sum()), r
+
+
+@pytest.mark.parametrize("use_phi", [False, True])
+def test_backward_finite_differences(use_phi):
+    # central differences of L = <dO, out> along random directions, on the smooth forward
+    # (exact fp64 summaries): agreement to ~1e-8 relative pins every gradient term
+    cfg, qb, kb, vb, g, doutb, o = _bwd_case(150, 130, 4, 2, 8, 60, top_n=3, window=24)
+    f = orc.bf16_bits_to_f64
+    q, k, v, dout = f(qb), f(kb), f(vb), f(doutb)
+    g = g.astype(np.float64)
+    sel = o["sel"][: cfg.n_video]
+    phi = (1.0 + 0.5 * np.random.default_rng(61).standard_normal((2, 32))) / 32 if use_phi else None
+    _, r = _loss_and_grads(cfg, q, k, v, g, dout, sel, phi)
+    rng = np.random.default_rng(62)
+    eps = 1e-5
+    for name, x, grad in (("q", q, r["dq"]), ("k", k, r["dk"]), ("v", v, r["dv"]), ("gates", g, r["dgates"])):
+        delta = rng.standard_normal(x.shape)
+        if name == "gates":
+            delta[cfg.n_video:] = 0.0  # text rows ignore their gates
+        args = {"q": q, "k": k, "v": v, "gates": g}
+        hi = dict(args, **{name: x + eps * delta})
+        lo = dict(args, **{name: x - eps * delta})
+        lp, _ = _loss_and_grads(cfg, hi["q"], hi["k"], hi["v"], hi["gates"], dout, sel, phi)
+        lm, _ = _loss_and_grads(cfg, lo["q"], lo["k"], lo["v"], lo["gates"], dout, sel, phi)
+        fd = (lp - lm) / (2 * eps)
+        an = float((grad * delta).sum())
+        assert abs(fd - an) <= 1e-7 * max(1.0, abs(an)), (name, fd, an)
+
+
+def test_backward_matches_torch_autograd_dense_masks():
+    # an independent formulation: each branch as a dense masked softmax over all keys,
+    # differentiated by torch autograd in float64
+    cfg, qb, kb, vb, gb, doutb, o = _bwd_case(200, 170, 6, 2, 16, 70, top_n=3, window=30)
+    f = orc.bf16_bits_to_f64
+    q, k, v, dout = (torch.from_numpy(f(a)).requires_grad_(True) for a in (qb, kb, vb, doutb))
+    gates = torch.from_numpy(gb.astype(np.float64)).requires_grad_(True)
+    N, nv, hq, hkv, d = cfg.n_tokens, cfg.n_video, cfg.hq, cfg.hkv, cfg.d
+    G, l, s, ls = hq // hkv, cfg.cmp_len, cfg.cmp_stride, cfg.sel_len
+    sel = o["sel"][:nv]
+    scale = 1.0 / math.sqrt(d)
+    nc = (nv - l) // s + 1
+    kc = torch.stack([k[i * s: i * s + l].mean(0) for i in range(nc)])
+    vc = torch.stack([v[i * s: i * s + l].mean(0) for i in range(nc)])
+    t_idx = torch.arange(N)[:, None]
+    tok = torch.arange(N)[None, :]
+    m_cmp = ((torch.arange(nc)[None, :] * s + l - 1) <= t_idx) & (t_idx < nv)
+    m_win = (tok <= t_idx) & (tok > t_idx - cfg.window) & (t_idx < nv)
+    m_txt = (tok <= t_idx) & (t_idx >= nv)
+    m_sel = torch.zeros((hkv, N, N), dtype=torch.bool)
+    for t in range(nv):
+        for g in range(hkv):
+            for j in sel[t, g]:
+                if j >= 0:
+                    m_sel[g, t, j * ls: min((j + 1) * ls, t + 1)] = True
+
+    def attend(K, V, mask):  # mask [hkv or 1, N, n]
+        S = torch.einsum("thd,nhd->htn", q, K.repeat_interleave(G, dim=1)) * scale
+        M = mask.repeat_interleave(G, dim=0) if mask.shape[0] == hkv else mask.expand(hq, -1, -1)
+        P = torch.softmax(S.masked_fill(~M, float("-inf")), dim=-1)
+        P = torch.where(M.any(-1, keepdim=True), P, torch.zeros_like(P))
+        return torch.einsum("htn,nhd->thd", P, V.repeat_interleave(G, dim=1))
+
+    out = (gates[..., 0:1] * attend(kc, vc, m_cmp[None]) + gates[..., 1:2] * attend(k, v, m_sel)
+           + gates[..., 2:3] * attend(k, v, m_win[None]) + attend(k, v, m_txt[None]))
+    (out * dout).sum().backward()
+    _, r = _loss_and_grads(cfg, f(qb), f(kb), f(vb), gb.astype(np.float64), f(doutb), sel)
+    assert np.abs(out.detach().numpy() - r["out"]).max() < 1e-12
+    for name, tg in (("dq", q.grad), ("dk", k.grad), ("dv", v.grad)):
+        assert np.abs(tg.numpy() - r[name]).max() < 1e-11, name
+    gg = gates.grad.numpy().copy()
+    gg[nv:] = 0.0
+    assert np.abs(gg - r["dgates"]).max() < 1e-11
+
+
+def test_backward_value_gradient_sums_to_gated_output_gradient():
+    # sum over tokens of dV equals, per group, the sum of dO weighted by the gates of the
+    # non-empty branches (probabilities sum to one; the compression's weights sum to one)
+    cfg, q, k, v, g, dout, o = _bwd_case(260, 220, 4, 2, 16, 80)
+    r = bwd_orc.prefill_backward(cfg, q, k, v, g, dout, o["sel"][: cfg.n_video])
+    do = orc.bf16_bits_to_f64(dout)
+    G = cfg.hq // cfg.hkv
+    w = np.ones((cfg.n_tokens, cfg.hq))
+    rows = np.arange(cfg.n_video)
+    has_cmp = rows >= cfg.cmp_len - 1
+    w[: cfg.n_video] = g[: cfg.n_video, :, 0] * has_cmp[:, None] + g[: cfg.n_video, :, 1] + g[: cfg.n_video, :, 2]
+    for grp in range(cfg.hkv):
+        hs = slice(grp * G, (grp + 1) * G)
+        want = (w[:, hs, None] * do[:, hs]).sum(axis=(0, 1))
+        assert np.allclose(r["dv"][:, grp].sum(0), want, atol=1e-10)
