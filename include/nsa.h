@@ -219,6 +219,31 @@ int nsa_gate_mlp_pooled(const void* x, const void* w1, const float* b1, const fl
 /* Workspace bytes nsa_gate_mlp_pooled needs; 0 if the arguments are invalid. */
 size_t nsa_gate_mlp_pooled_workspace_size(int batch, int seq_len, int heads, int dim);
 
+/*
+ * Backward of nsa_prefill: the gradients of a loss L given dL/dout. The pages train the
+ * model end to end (shd-paper.top page "VideoNSA: Native Sparse Attention Scales Video
+ * Understanding", abstract); the selection is held constant (block indices carry no
+ * gradient), and the compressed keys' gradient returns to their tokens with the
+ * compression's weights (the bf16 rounding of the summaries passes gradients unchanged).
+ *   q, k, v, gates, params: as given to nsa_prefill (or nsa_prefill_phi)
+ *   d_out    [N][Hq][d] bf16, dL/dout
+ *   sel_idx  [N_v][Hkv][top_n] int32: the forward's selection (nsa_prefill's out_sel_idx)
+ *   phi_k, phi_v  both NULL (mean compression) or both the learnable weights [Hkv][l] fp32
+ *   dq       [N][Hq][d] fp32     dk, dv [N][Hkv][d] fp32    (written, not accumulated)
+ *   dgates   [N][Hq][3] fp32: <dL/dout, o_b> per branch; 0 for text rows
+ *   workspace    at least nsa_backward_workspace_size(params) bytes, 256-byte aligned
+ * All device pointers; q, k, v, d_out, dq, dk, dv 16-byte aligned. Errors as nsa_prefill,
+ * returned before anything is enqueued. dk and dv are sums of fp32 atomic adds, so their
+ * last bits vary from run to run.
+ */
+int nsa_backward(const void* q, const void* k, const void* v, const float* gates, const void* d_out,
+                 const int32_t* sel_idx, const float* phi_k, const float* phi_v, const nsa_params_t* params,
+                 float* dq, float* dk, float* dv, float* dgates, void* workspace, size_t workspace_bytes,
+                 void* stream);
+
+/* Workspace bytes nsa_backward needs; 0 if params are invalid. */
+size_t nsa_backward_workspace_size(const nsa_params_t* params);
+
 /* Workspace bytes nsa_prefill (is_decode = 0) or nsa_decode (is_decode = 1) needs; 0 if params are invalid. */
 size_t nsa_workspace_size(const nsa_params_t* params, int is_decode);
 

@@ -86,14 +86,14 @@ def compressed_f64(k: np.ndarray, cfg: orc.OracleConfig, phi=None, rounded: bool
     return out
 
 
-def forward_backward(cfg: orc.OracleConfig, q, k, v, gates, d_out, sel, kc=None, vc=None, phi=None):
+def forward_backward(cfg: orc.OracleConfig, q, k, v, gates, d_out, sel, kc=None, vc=None, phi_k=None, phi_v=None):
     """Forward outputs and gradients of one prefill.
 
     q [N, hq, d], k, v [N, hkv, d], d_out [N, hq, d]: fp64 arrays (widen bf16 inputs with
     orc.bf16_bits_to_f64); gates [N, hq, 3]; sel [n_video, hkv, top_n] block indices (-1
-    padded). kc, vc: the compressed keys and values (fp64) the forward attended; phi: the
-    learnable compression's weights [hkv, l] (None for the mean), used for the gradient's
-    way back to the tokens.
+    padded). kc, vc: the compressed keys and values (fp64) the forward attended; phi_k, phi_v:
+    the learnable compression's weights [hkv, l] for keys and values (None for the mean), used
+    for the gradient's way back to the tokens.
     Returns dict(out, dq, dk, dv, dgates); dgates of text rows are 0."""
     q, k, v, d_out = (np.asarray(a, dtype=np.float64) for a in (q, k, v, d_out))
     gates = np.asarray(gates, dtype=np.float64)
@@ -135,21 +135,24 @@ def forward_backward(cfg: orc.OracleConfig, q, k, v, gates, d_out, sel, kc=None,
                     np.add.at(dvs, (idx, g), dVb)
                 dgates[t, hs, b] = dg
     # the compressed keys' gradient flows back to their tokens with the compression's weights
-    w = np.full((hkv, cfg.cmp_len), 1.0 / cfg.cmp_len) if phi is None else np.asarray(phi, np.float64)
+    mean = np.full((hkv, cfg.cmp_len), 1.0 / cfg.cmp_len)
+    wk = mean if phi_k is None else np.asarray(phi_k, np.float64)
+    wv = mean if phi_v is None else np.asarray(phi_v, np.float64)
     for i in range(ncmp):
         for u in range(cfg.cmp_len):
             tau = i * cfg.cmp_stride + u
-            dk[tau] += w[:, u, None] * dkc[i]
-            dv[tau] += w[:, u, None] * dvc[i]
+            dk[tau] += wk[:, u, None] * dkc[i]
+            dv[tau] += wv[:, u, None] * dvc[i]
     return {"out": out, "dq": dq, "dk": dk, "dv": dv, "dgates": dgates}
 
 
-def prefill_backward(cfg: orc.OracleConfig, q_bits, k_bits, v_bits, gates, d_out_bits, sel, phi=None) -> dict:
+def prefill_backward(cfg: orc.OracleConfig, q_bits, k_bits, v_bits, gates, d_out_bits, sel, phi_k=None,
+                     phi_v=None) -> dict:
     """Gradients of the prefill the forward oracle computes, on the exact bf16 inputs it
     consumed (uint16 bit patterns) and its bf16 compressed keys and values."""
     kb = np.ascontiguousarray(k_bits)[: cfg.n_video]
     vb = np.ascontiguousarray(v_bits)[: cfg.n_video]
-    kc = compressed_f64(kb, cfg, phi)
-    vc = compressed_f64(vb, cfg, phi)
+    kc = compressed_f64(kb, cfg, phi_k)
+    vc = compressed_f64(vb, cfg, phi_v)
     f = orc.bf16_bits_to_f64
-    return forward_backward(cfg, f(q_bits), f(k_bits), f(v_bits), gates, f(d_out_bits), sel, kc, vc, phi)
+    return forward_backward(cfg, f(q_bits), f(k_bits), f(v_bits), gates, f(d_out_bits), sel, kc, vc, phi_k, phi_v)

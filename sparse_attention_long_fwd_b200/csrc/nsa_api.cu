@@ -19,6 +19,7 @@
 #include "sel_inv.cuh"
 #include "decode.cuh"
 #include "gate.cuh"
+#include "backward.cuh"
 
 namespace {
 
@@ -833,6 +834,219 @@ int nsa_gate_mlp_pooled(const void* x, const void* w1, const float* b1, const fl
     nsa::gate_pooled_kernel<128><<<grid, 128, 0, st>>>(part, w1b, b1, w2, b2, gates, batch, seq_len, heads, nchunk,
                                                         repeat);
   return launch_status("gate_pooled", st, false);
+}
+
+// ------------------------------------------------------------------ backward
+}  // extern "C"
+
+namespace {
+
+struct BwdLayout {
+  size_t kc, vc, dkc, dvc, stats, cnt, ent_off, seg_off, list, row_of, total;
+  int ncmp, nsel;
+};
+
+BwdLayout bwd_layout(const nsa_params_t* p) {
+  BwdLayout L{};
+  const size_t N = p->n_tokens, nv = p->n_video, hq = p->num_q_heads, hkv = p->num_kv_heads, d = p->head_dim;
+  L.ncmp = ncmp_of(p->n_video, p->cmp_block, p->cmp_stride);
+  L.nsel = nsel_of(p->n_video, p->sel_block);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + (bytes > 0 ? bytes : 1));
+    return at;
+  };
+  const size_t nc = L.ncmp > 0 ? L.ncmp : 1;
+  const size_t buckets = hkv * (L.nsel > 0 ? L.nsel : 1);
+  const size_t entries = nv * hkv * p->top_n;
+  L.kc = take(nc * hkv * d * 2);
+  L.vc = take(nc * hkv * d * 2);
+  L.dkc = take(nc * hkv * d * 4);
+  L.dvc = take(nc * hkv * d * 4);
+  L.stats = take(N * hq * 3 * 8);
+  L.cnt = take(2 * buckets * 4);  // counters and scatter cursors, zeroed together
+  L.ent_off = take((buckets + 1) * 4);
+  L.seg_off = take((buckets + 1) * 4);
+  L.list = take(entries * 4);
+  L.row_of = take(entries * 4);
+  L.total = off;
+  return L;
+}
+
+template <int D, int BR>
+int launch_bwd_key(const nsa::BwdArgs& a, long long n_items, cudaStream_t st) {
+  if (n_items <= 0) return NSA_OK;
+  const size_t smem = nsa::kBwdWarps * sizeof(nsa::BwdKeySmem<D>);
+  auto kern = nsa::bwd_key_kernel<D, BR>;
+  if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
+  const long long grid = (n_items + nsa::kBwdWarps - 1) / nsa::kBwdWarps;
+  if (grid > 0x7fffffffLL) return NSA_ERR_UNSUPPORTED;
+  kern<<<static_cast<unsigned>(grid), 32 * nsa::kBwdWarps, smem, st>>>(a, n_items);
+  return launch_status(BR == nsa::kBwdCmp ? "bwd_key_cmp" : BR == nsa::kBwdSel ? "bwd_key_sel"
+                                                          : BR == nsa::kBwdWin ? "bwd_key_win" : "bwd_key_dense",
+                       st);
+}
+
+template <int D>
+int backward_impl(const nsa_params_t* p, const void* q, const void* k, const void* v, const float* gates,
+                  const void* d_out, const int32_t* sel_idx, const float* phi_k, const float* phi_v, float* dq,
+                  float* dk, float* dv, float* dgates, uint8_t* ws, cudaStream_t st) {
+  const BwdLayout L = bwd_layout(p);
+  const int N = p->n_tokens, nv = p->n_video, hq = p->num_q_heads, hkv = p->num_kv_heads;
+  const int G = hq / hkv;
+  const float scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(D));
+  int rc;
+  nsa::BwdArgs a{};
+  a.N = N;
+  a.nv = nv;
+  a.hq = hq;
+  a.hkv = hkv;
+  a.G = G;
+  a.ncmp = L.ncmp;
+  a.nsel = L.nsel;
+  a.top_n = p->top_n;
+  a.cmp_len = p->cmp_block;
+  a.cmp_stride = p->cmp_stride;
+  a.sel_len = p->sel_block;
+  a.window = p->window;
+  a.scale = scale;
+  a.sl2 = scale * 1.4426950408889634f;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.kc = reinterpret_cast<const __nv_bfloat16*>(ws + L.kc);
+  a.vc = reinterpret_cast<const __nv_bfloat16*>(ws + L.vc);
+  a.dout = static_cast<const __nv_bfloat16*>(d_out);
+  a.gates = gates;
+  a.sel_idx = sel_idx;
+  a.stats = reinterpret_cast<float2*>(ws + L.stats);
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.dkc = reinterpret_cast<float*>(ws + L.dkc);
+  a.dvc = reinterpret_cast<float*>(ws + L.dvc);
+  a.dgates = dgates;
+  a.ent_off = reinterpret_cast<const int*>(ws + L.ent_off);
+  a.seg_off = reinterpret_cast<const int*>(ws + L.seg_off);
+  a.list = reinterpret_cast<const int*>(ws + L.list);
+  const size_t kv_bytes = static_cast<size_t>(N) * hkv * D * 4;
+  if (cudaMemsetAsync(dk, 0, kv_bytes, st) != cudaSuccess || cudaMemsetAsync(dv, 0, kv_bytes, st) != cudaSuccess)
+    return NSA_ERR_CUDA;
+  if (L.ncmp > 0) {
+    const size_t cb = static_cast<size_t>(L.ncmp) * hkv * D * 4;
+    if (cudaMemsetAsync(ws + L.dkc, 0, cb, st) != cudaSuccess || cudaMemsetAsync(ws + L.dvc, 0, cb, st) != cudaSuccess)
+      return NSA_ERR_CUDA;
+    // the compressed keys and values the forward attended
+    if ((rc = launch_pool(k, v, ws + L.kc, ws + L.vc, 1, nv, hkv, D, L.ncmp, p->cmp_block, p->cmp_stride, st, phi_k,
+                          phi_v)) != NSA_OK)
+      return rc;
+  }
+  // row pass: dq, the gates' gradient and the per-branch statistics
+  {
+    const size_t smem = nsa::kBwdWarps * sizeof(nsa::WarpChunkBuf<D, nsa::kBwdChunk, 2>);
+    auto kern = nsa::bwd_row_kernel<D>;
+    if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
+    const long long items = static_cast<long long>(N) * hkv;
+    kern<<<static_cast<unsigned>((items + nsa::kBwdWarps - 1) / nsa::kBwdWarps), 32 * nsa::kBwdWarps, smem, st>>>(a);
+    if ((rc = launch_status("bwd_row", st)) != NSA_OK) return rc;
+  }
+  if (nv > 0) {
+    // buckets of the selected branch: which tokens chose each (group, block)
+    const int m = hkv * L.nsel;
+    nsa::SelInvArgs sa{};
+    sa.nv = nv;
+    sa.hq = hq;
+    sa.hkv = hkv;
+    sa.G = G;
+    sa.Gp = G;
+    sa.TT = nsa::kBwdSegSel;
+    sa.nsel = L.nsel;
+    sa.top_n = p->top_n;
+    sa.sel_len = p->sel_block;
+    sa.sel_idx = sel_idx;
+    sa.cnt = reinterpret_cast<int*>(ws + L.cnt);
+    sa.cursor = sa.cnt + m;
+    sa.ent_off = reinterpret_cast<int*>(ws + L.ent_off);
+    sa.tile_off = reinterpret_cast<int*>(ws + L.seg_off);
+    sa.list = reinterpret_cast<int*>(ws + L.list);
+    sa.row_of = reinterpret_cast<int*>(ws + L.row_of);
+    if (cudaMemsetAsync(sa.cnt, 0, 2 * static_cast<size_t>(m) * 4, st) != cudaSuccess) return NSA_ERR_CUDA;
+    const long long entries = static_cast<long long>(nv) * hkv * p->top_n;
+    const long long eb = (entries + 255) / 256;
+    const unsigned ebl = static_cast<unsigned>(eb < 148 * 16 ? (eb > 0 ? eb : 1) : 148 * 16);
+    nsa::sel_count_kernel<<<ebl, 256, 0, st>>>(sa);
+    if ((rc = launch_status("bwd_sel_count", st, false)) != NSA_OK) return rc;
+    nsa::sel_scan_kernel<<<1, 1024, 0, st>>>(sa);
+    if ((rc = launch_status("bwd_sel_scan", st, false)) != NSA_OK) return rc;
+    nsa::sel_scatter_kernel<<<ebl, 256, 0, st>>>(sa);
+    if ((rc = launch_status("bwd_sel_scatter", st)) != NSA_OK) return rc;
+    // key pass, one launch per branch
+    if (L.ncmp > 0) {
+      const long long items = static_cast<long long>((L.ncmp + nsa::kBwdChunk - 1) / nsa::kBwdChunk) * hkv *
+                              ((nv + nsa::kBwdSegCmp - 1) / nsa::kBwdSegCmp);
+      if ((rc = launch_bwd_key<D, nsa::kBwdCmp>(a, items, st)) != NSA_OK) return rc;
+    }
+    {
+      const long long segs = entries / nsa::kBwdSegSel + m + 1;  // >= sum over buckets of ceil(count / segment)
+      if ((rc = launch_bwd_key<D, nsa::kBwdSel>(a, segs * (p->sel_block / nsa::kBwdChunk), st)) != NSA_OK) return rc;
+    }
+    {
+      const long long items = static_cast<long long>((nv + nsa::kBwdChunk - 1) / nsa::kBwdChunk) * hkv;
+      if ((rc = launch_bwd_key<D, nsa::kBwdWin>(a, items, st)) != NSA_OK) return rc;
+    }
+  }
+  if (N > nv) {
+    const long long items = static_cast<long long>((N + nsa::kBwdChunk - 1) / nsa::kBwdChunk) * hkv *
+                            ((N - nv + nsa::kBwdSegDense - 1) / nsa::kBwdSegDense);
+    if ((rc = launch_bwd_key<D, nsa::kBwdDense>(a, items, st)) != NSA_OK) return rc;
+  }
+  if (L.ncmp > 0) {
+    const long long total = static_cast<long long>(nv) * hkv * D;
+    nsa::pool_bwd_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(
+        a.dkc, a.dvc, phi_k, phi_v, dk, dv, nv, hkv, D, L.ncmp, p->cmp_block, p->cmp_stride);
+    if ((rc = launch_status("pool_bwd", st)) != NSA_OK) return rc;
+  }
+  return NSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t nsa_backward_workspace_size(const nsa_params_t* params) {
+  if (check_common(params) != NSA_OK || params->n_video < 0 || params->n_video > params->n_tokens) return 0;
+  return bwd_layout(params).total;
+}
+
+int nsa_backward(const void* q, const void* k, const void* v, const float* gates, const void* d_out,
+                 const int32_t* sel_idx, const float* phi_k, const float* phi_v, const nsa_params_t* params,
+                 float* dq, float* dk, float* dv, float* dgates, void* workspace, size_t workspace_bytes,
+                 void* stream) {
+  int rc = check_common(params);
+  if (rc != NSA_OK) return rc;
+  if (params->n_video < 0 || params->n_video > params->n_tokens) return NSA_ERR_INVALID_ARG;
+  const bool video = params->n_video > 0;
+  if (!q || !k || !v || !d_out || !dq || !dk || !dv || !dgates || !workspace || (video && (!gates || !sel_idx)))
+    return NSA_ERR_INVALID_ARG;
+  if ((phi_k == nullptr) != (phi_v == nullptr)) return NSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(d_out) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv) || !aligned4(dgates) || (gates && !aligned4(gates)) || (sel_idx && !aligned4(sel_idx)) ||
+      (phi_k && (!aligned4(phi_k) || !aligned4(phi_v))) || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+    return NSA_ERR_INVALID_ARG;
+  if (nsel_of(params->n_video, params->sel_block) > 8192) return NSA_ERR_UNSUPPORTED;
+  if (workspace_bytes < bwd_layout(params).total) return NSA_ERR_WORKSPACE_TOO_SMALL;
+  if ((rc = check_device()) != NSA_OK) return rc;
+  auto* ws = static_cast<uint8_t*>(workspace);
+  auto st = static_cast<cudaStream_t>(stream);
+  // stage events registered by nsa_profile_stages belong to the forward calls
+  const int saved_count = g_stage_count;
+  g_stage_count = 0;
+  rc = params->head_dim == 64
+           ? backward_impl<64>(params, q, k, v, gates, d_out, sel_idx, phi_k, phi_v, dq, dk, dv, dgates, ws, st)
+           : backward_impl<128>(params, q, k, v, gates, d_out, sel_idx, phi_k, phi_v, dq, dk, dv, dgates, ws, st);
+  g_stage_count = saved_count;
+  return rc;
 }
 
 int nsa_profile_stages(void* const* events, int count) {

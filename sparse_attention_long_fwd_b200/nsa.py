@@ -30,7 +30,8 @@ EXPORTED = (
     "nsa_prefill", "nsa_decode", "nsa_compress", "nsa_workspace_size", "nsa_prefill_workspace_layout",
     "nsa_error_string", "nsa_get_device_error", "nsa_version", "nsa_profile_stages", "nsa_decode_noalloc",
     "nsa_prefill_varlen", "nsa_prefill_varlen_workspace_size", "nsa_compress_weighted", "nsa_prefill_phi",
-    "nsa_gate_mlp", "nsa_gate_mlp_pooled", "nsa_gate_mlp_pooled_workspace_size",
+    "nsa_gate_mlp", "nsa_gate_mlp_pooled", "nsa_gate_mlp_pooled_workspace_size", "nsa_backward",
+    "nsa_backward_workspace_size",
 )
 
 
@@ -98,6 +99,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.nsa_gate_mlp_pooled.restype = I
     lib.nsa_gate_mlp_pooled_workspace_size.argtypes = [I, I, I, I]
     lib.nsa_gate_mlp_pooled_workspace_size.restype = S
+    lib.nsa_backward.argtypes = [P, P, P, P, P, P, P, P, PP, P, P, P, P, P, S, P]
+    lib.nsa_backward.restype = I
+    lib.nsa_backward_workspace_size.argtypes = [PP]
+    lib.nsa_backward_workspace_size.restype = S
     lib.nsa_workspace_size.argtypes = [PP, I]
     lib.nsa_workspace_size.restype = S
     lib.nsa_prefill_workspace_layout.argtypes = [PP, ctypes.POINTER(NsaPrefillLayout)]
@@ -215,6 +220,17 @@ def nsa_gate_mlp_pooled_workspace_size(batch: int, seq_len: int, heads: int, dim
     return int(load_library().nsa_gate_mlp_pooled_workspace_size(batch, seq_len, heads, dim))
 
 
+def nsa_backward(q, k, v, gates, d_out, sel_idx, phi_k, phi_v, params: NsaParams, dq, dk, dv, dgates, workspace,
+                 workspace_bytes: int, stream=None) -> int:
+    return load_library().nsa_backward(_addr(q), _addr(k), _addr(v), _addr(gates), _addr(d_out), _addr(sel_idx),
+                                       _addr(phi_k), _addr(phi_v), ctypes.byref(params), _addr(dq), _addr(dk),
+                                       _addr(dv), _addr(dgates), _addr(workspace), workspace_bytes, _stream(stream))
+
+
+def nsa_backward_workspace_size(params: NsaParams) -> int:
+    return int(load_library().nsa_backward_workspace_size(ctypes.byref(params)))
+
+
 def nsa_workspace_size(params: NsaParams, is_decode: bool) -> int:
     return int(load_library().nsa_workspace_size(ctypes.byref(params), int(bool(is_decode))))
 
@@ -324,6 +340,28 @@ def decode(q, kcache, vcache, kcmp, vcmp, seq_lens, gates, *, top_n: int = 16, w
     _check(nsa_decode(q, kcache, vcache, kcmp, vcmp, seq_lens, gates, p, out, sel, workspace, workspace.numel(),
                       stream), "nsa_decode")
     return (out, sel) if return_sel else out
+
+
+def backward(q, k, v, gates, d_out, sel_idx, *, n_video: int | None = None, top_n: int = 16, window: int = 512,
+             softmax_scale: float = 0.0, phi=None, workspace: torch.Tensor | None = None, stream=None):
+    """Gradients of the prefill: returns dq [N,Hq,d], dk, dv [N,Hkv,d] and dgates [N,Hq,3] (fp32),
+    given dL/dout (bf16) and the forward's selection sel_idx [N_v,Hkv,top_n]."""
+    N, hq, d = q.shape
+    hkv = k.shape[1]
+    p = make_params(N, n_video, hq, hkv, d, top_n=top_n, window=window, softmax_scale=softmax_scale)
+    dq = torch.empty((N, hq, d), dtype=torch.float32, device=q.device)
+    dk = torch.empty((N, hkv, d), dtype=torch.float32, device=q.device)
+    dv = torch.empty_like(dk)
+    dgates = torch.empty((N, hq, 3), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        n = nsa_backward_workspace_size(p)
+        if n == 0:
+            raise NsaError(NSA_ERR_INVALID_ARG, "nsa_backward_workspace_size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+    pk, pv = (None, None) if phi is None else phi
+    _check(nsa_backward(q, k, v, gates, d_out, sel_idx, pk, pv, p, dq, dk, dv, dgates, workspace, workspace.numel(),
+                        stream), "nsa_backward")
+    return dq, dk, dv, dgates
 
 
 def gate_mlp(x: torch.Tensor, w1: torch.Tensor, b1: torch.Tensor, w2: torch.Tensor, b2: torch.Tensor, stream=None):

@@ -160,3 +160,22 @@ def test_learnable_compression_and_gate_validation():
         nsa.NSA_ERR_WORKSPACE_TOO_SMALL
     assert nsa.nsa_gate_mlp_pooled(f, f, f, f, f, 2, 131072, 28, 128, 0, f, f, need, None) == nsa.NSA_ERR_INVALID_ARG
     assert nsa.nsa_gate_mlp_pooled(f, f, f, f, f, 1, 100, 28, 96, 1, f, f, 1 << 30, None) == nsa.NSA_ERR_UNSUPPORTED
+
+
+def test_backward_validation():
+    f = 1 << 20
+    p = _p()
+    need = nsa.nsa_backward_workspace_size(p)
+    assert need > 0 and need % 256 == 0
+    ok_args = [f] * 6 + [None, None, p] + [f] * 5
+    assert nsa.nsa_backward(*ok_args, need - 1, None) == nsa.NSA_ERR_WORKSPACE_TOO_SMALL
+    bad = list(ok_args)
+    bad[5] = None  # the forward's selection is required when there are video rows
+    assert nsa.nsa_backward(*bad, need, None) == nsa.NSA_ERR_INVALID_ARG
+    bad = list(ok_args)
+    bad[6] = f  # phi_k without phi_v
+    assert nsa.nsa_backward(*bad, need, None) == nsa.NSA_ERR_INVALID_ARG
+    bad = list(ok_args)
+    bad[9] = f + 4  # dq misaligned
+    assert nsa.nsa_backward(*bad, need, None) == nsa.NSA_ERR_INVALID_ARG
+    assert nsa.nsa_backward_workspace_size(_p(head_dim=96)) == 0

@@ -536,9 +536,10 @@ def test_backward_forward_equals_the_forward_oracle():
 
 
 def _loss_and_grads(cfg, q, k, v, g, dout, sel, phi=None):
-    kc = bwd_orc.compressed_f64(k[: cfg.n_video], cfg, phi, rounded=False)
-    vc = bwd_orc.compressed_f64(v[: cfg.n_video], cfg, phi, rounded=False)
-    r = bwd_orc.forward_backward(cfg, q, k, v, g, dout, sel, kc, vc, phi)
+    pk, pv = (None, None) if phi is None else phi
+    kc = bwd_orc.compressed_f64(k[: cfg.n_video], cfg, pk, rounded=False)
+    vc = bwd_orc.compressed_f64(v[: cfg.n_video], cfg, pv, rounded=False)
+    r = bwd_orc.forward_backward(cfg, q, k, v, g, dout, sel, kc, vc, pk, pv)
     return float((r["out"] * dout).sum()), r
 
 
@@ -551,7 +552,8 @@ def test_backward_finite_differences(use_phi):
     q, k, v, dout = f(qb), f(kb), f(vb), f(doutb)
     g = g.astype(np.float64)
     sel = o["sel"][: cfg.n_video]
-    phi = (1.0 + 0.5 * np.random.default_rng(61).standard_normal((2, 32))) / 32 if use_phi else None
+    prng = np.random.default_rng(61)
+    phi = tuple((1.0 + 0.5 * prng.standard_normal((2, 32))) / 32 for _ in range(2)) if use_phi else None
     _, r = _loss_and_grads(cfg, q, k, v, g, dout, sel, phi)
     rng = np.random.default_rng(62)
     eps = 1e-5
