@@ -369,6 +369,10 @@ def run_b200(args, world, rank, local):
         result["gates_and_phi"] = run_gates(args, dev, q, k, v, g, peaks, peaks_src, flush, world)
         result["gpu_launches"] += result["gates_and_phi"]["launches"]
 
+    if not args.no_backward and w.name == "v128k":
+        result["backward"] = run_backward(args, dev, q, k, v, g, peaks, flush, world)
+        result["gpu_launches"] += result["backward"]["launches"]
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, q, k, v, g, args.cpu_seconds)
     return result
@@ -480,6 +484,55 @@ def run_gates(args, dev, q, k, v, g, peaks, peaks_src, flush, world):
         "steps": args.steps, "warmup": args.warmup, "l2": "flushed before every timed step",
         "launches": args.steps * (1 + 2 + PREFILL_KERNELS),
     }
+
+
+BACKWARD_KERNELS = 9  # 128K, no text rows: pool, row pass, 3 bucket kernels, 3 key passes, pool backward
+
+
+def run_backward(args, dev, q, k, v, g, peaks, flush, world):
+    """nsa_backward on the headline 128K tensors, with the selection of one forward call and
+    a N(0,1) dL/dout."""
+    w = WORKLOADS["v128k"]
+    p = nsa.make_params(w.n_tokens, w.n_video, w.hq, w.hkv, w.d, w.cmp_len, w.cmp_stride, w.sel_len, w.top_n,
+                        w.window, out_dtype=nsa.NSA_OUT_BF16)
+    ws = nsa.alloc_workspace(p, False, dev)
+    out = torch.empty((w.n_tokens, w.hq, w.d), dtype=torch.bfloat16, device=dev)
+    sel = torch.empty((w.n_video, w.hkv, w.top_n), dtype=torch.int32, device=dev)
+    rc = nsa.nsa_prefill(q, k, v, g, p, out, sel, ws, ws.numel())
+    if rc != nsa.NSA_OK:
+        raise nsa.NsaError(rc, "nsa_prefill")
+    del ws, out
+    gen = torch.Generator(device=dev).manual_seed(31)
+    d_out = torch.randn((w.n_tokens, w.hq, w.d), generator=gen, device=dev).to(torch.bfloat16)
+    dq = torch.empty((w.n_tokens, w.hq, w.d), dtype=torch.float32, device=dev)
+    dk = torch.empty((w.n_tokens, w.hkv, w.d), dtype=torch.float32, device=dev)
+    dv = torch.empty_like(dk)
+    dgates = torch.empty((w.n_tokens, w.hq, 3), dtype=torch.float32, device=dev)
+    bws = torch.empty(nsa.nsa_backward_workspace_size(p), dtype=torch.uint8, device=dev)
+
+    def step(events):
+        rc = nsa.nsa_backward(q, k, v, g, d_out, sel, None, None, p, dq, dk, dv, dgates, bws, bws.numel())
+        if rc != nsa.NSA_OK:
+            raise nsa.NsaError(rc, "nsa_backward")
+
+    barrier(world)
+    step_ms, _ = timed_steps(step, args.steps, args.warmup, flush, 0)
+    assert nsa.nsa_get_device_error(clear=True) == 0, "device error word set during the backward"
+    ms = max_over_ranks(sum(step_ms), world) / args.steps
+    c = prefill_counts(w)
+    # QK^T, dO V^T, P^T dO, dS K and dS^T Q against the forward's QK^T and PV: 2.5x its FLOPs
+    flops = 2.5 * (c["cmp_flops"] + c["sel_flops"] + c["win_flops"] + c["text_flops"])
+    tf = flops / (ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    del bws, dq, dk, dv, dgates, d_out
+    return {"workload": "v128k backward: dq, dk, dv and the gates' gradient of the headline prefill "
+                        "(selection of its forward held constant)",
+            "ms_per_step": round(ms, 3), "value": round(w.n_video * world / (ms / 1e3), 1),
+            "unit": "video tokens/s", "steps": args.steps, "warmup": args.warmup,
+            "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(tf / peak, 4),
+                         "algorithmic": f"{flops:.4e} FLOP per step (2.5x the forward's attended FLOPs)"},
+            "launches": BACKWARD_KERNELS * args.steps}
 
 
 def run_decode(args, dev, peaks, peaks_src, flush, world):
@@ -609,6 +662,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
     ap.add_argument("--no-sweep", action="store_true", help="skip the 128K (n, w) budget sweep")
     ap.add_argument("--no-gates", action="store_true", help="skip the gate-network and learnable-compression lines")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     args = ap.parse_args()
