@@ -11,11 +11,12 @@
 // Text rows (t >= n_video) are one dense branch with gate 1.
 //
 // Three passes, all on warp-level mma.sync tiles (m16n8k16, bf16 in, fp32 accumulate):
-//   bwd_row_kernel   one warp per (token, group), the group's heads as rows of a 16-row
-//                    tile. Per branch: pass A streams the keys once for the row's
-//                    log-sum-exp and o_b, giving <dO, o_b> (the gate gradient); pass B
-//                    streams them again for dS and dq += dS K. Writes dq, the gate
-//                    gradient and (lse, <dO, o_b>) per (row, branch) for the next pass.
+//   bwd_row_kernel   one warp per (two adjacent tokens, group) when a group has at most
+//                    8 heads (else one token): the heads are the rows of a 16-row tile.
+//                    Per branch: pass A streams the keys once for each row's log-sum-exp
+//                    and o_b, giving <dO, o_b> (the gate gradient); pass B streams them
+//                    again for dS and dq += dS K. Writes dq, the gate gradient and
+//                    (lse, <dO, o_b>) per (row, branch) for the next pass.
 //   bwd_key_kernel   one warp per (branch, 16-key tile, group, segment of the rows that
 //                    attend those keys): S^T = K Q^T and dP^T = V dO^T for 16 rows at a
 //                    time, then dv += P^T dO and dk += dS^T Q in registers; the sums are
@@ -62,27 +63,32 @@ struct BwdArgs {
 };
 
 // ---------------------------------------------------------------- row pass
+// A warp's 16 MMA rows: thread rows lane/4 (half 0) and lane/4 + 8 (half 1). With G <= 8 a
+// warp takes two adjacent tokens of the same kind (half 0: token A's heads, half 1: token
+// B's), so 2G of the 16 rows do work; with G > 8 it takes one token (half 1: heads 8..G-1).
+// Keys are masked per half: adjacent tokens differ in their last compressed block, their
+// window and their selection, and attend the union with their own ranges.
 
 struct ChunkDesc {
-  const __nv_bfloat16* kb;
-  const __nv_bfloat16* vb;
-  int start, row_end, lo, hi;
+  int start, row_end;  // keys start .. start+15 are loaded where < row_end
+  int lo[2], hi[2];    // key range of each half
 };
 
-// Streams `nch` chunks through the warp's two-stage ring; use(stage, desc) runs on each.
+// Streams `nch` chunks of keys from (kb, vb) through the warp's two-stage ring.
 template <int D, class Desc, class Use>
-__device__ __forceinline__ void bwd_stream(WarpChunkBuf<D, kBwdChunk, 2>& buf, size_t stride, int nch, Desc desc,
-                                           Use use, int lane) {
+__device__ __forceinline__ void bwd_stream(WarpChunkBuf<D, kBwdChunk, 2>& buf, const __nv_bfloat16* kb,
+                                           const __nv_bfloat16* vb, size_t stride, int nch, Desc desc, Use use,
+                                           int lane) {
   if (nch <= 0) return;
   {
     const ChunkDesc d0 = desc(0);
-    load_chunk<D, kBwdChunk, 2>(buf, 0, d0.kb, d0.vb, stride, d0.start, d0.row_end, lane);
+    load_chunk<D, kBwdChunk, 2>(buf, 0, kb, vb, stride, d0.start, d0.row_end, lane);
   }
   cp_async_commit();
   for (int c = 0; c < nch; ++c) {
     if (c + 1 < nch) {
       const ChunkDesc dn = desc(c + 1);
-      load_chunk<D, kBwdChunk, 2>(buf, (c + 1) & 1, dn.kb, dn.vb, stride, dn.start, dn.row_end, lane);
+      load_chunk<D, kBwdChunk, 2>(buf, (c + 1) & 1, kb, vb, stride, dn.start, dn.row_end, lane);
     }
     cp_async_commit();
     cp_async_wait_1();
@@ -91,6 +97,102 @@ __device__ __forceinline__ void bwd_stream(WarpChunkBuf<D, kBwdChunk, 2>& buf, s
     __syncwarp();  // every lane is done with this stage before it is refilled
   }
   cp_async_wait_0();
+}
+
+// A fragments of the 16 rows: half 0 from row pointer p0, half 1 from p1 (null: zero).
+template <int D>
+__device__ __forceinline__ void bwd_load_frags(uint32_t (&a)[D / 16][4], const __nv_bfloat16* p0,
+                                               const __nv_bfloat16* p1, int lane) {
+  const int c = 2 * (lane & 3);
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks) {
+    const int col = ks * 16 + c;
+    a[ks][0] = p0 ? *reinterpret_cast<const uint32_t*>(p0 + col) : 0u;
+    a[ks][1] = p1 ? *reinterpret_cast<const uint32_t*>(p1 + col) : 0u;
+    a[ks][2] = p0 ? *reinterpret_cast<const uint32_t*>(p0 + col + 8) : 0u;
+    a[ks][3] = p1 ? *reinterpret_cast<const uint32_t*>(p1 + col + 8) : 0u;
+  }
+}
+
+// Pass A on one chunk: online softmax over the chunk's keys (per-half ranges), O += P V.
+template <int D>
+__device__ __forceinline__ void bwd_attend_chunk(WarpAttnState<D>& s, const uint32_t (&qa)[D / 16][4],
+                                                 const WarpChunkBuf<D, kBwdChunk, 2>& buf, int st,
+                                                 const ChunkDesc& cd, float sl2, int lane) {
+  constexpr int NT = kBwdChunk / 8;
+  const uint32_t kaddr = smem_u32(&buf.kv[st][0][0]);
+  const uint32_t vaddr = smem_u32(&buf.kv[st][1][0]);
+  float sc[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ks += 2) {
+      const int row = nt * 8 + (lane & 7);
+      const int unit = ks * 2 + (lane >> 3);
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(kaddr + (row * D + swz_unit(row, unit) * 8) * 2, b0, b1, b2, b3);
+      mma_bf16_16816(sc[nt], qa[ks], b0, b1);
+      mma_bf16_16816(sc[nt], qa[ks + 1], b2, b3);
+    }
+  }
+  float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int r = e >> 1;
+      const int key = cd.start + nt * 8 + 2 * (lane & 3) + (e & 1);
+      const float z = (key >= cd.lo[r] && key < cd.hi[r]) ? sc[nt][e] * sl2 : -INFINITY;
+      sc[nt][e] = z;
+      mx[r] = fmaxf(mx[r], z);
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+    mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+  }
+  float alpha[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const float mnew = fmaxf(s.m[r], mx[r]);
+    alpha[r] = (mnew == -INFINITY) ? 1.f : ex2_approx(s.m[r] - mnew);
+    s.m[r] = mnew;
+  }
+  s.l[0] *= alpha[0];
+  s.l[1] *= alpha[1];
+  uint32_t pa[4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    float p[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float mr = s.m[e >> 1];
+      p[e] = (mr == -INFINITY) ? 0.f : ex2_approx(sc[nt][e] - mr);
+    }
+    s.l[0] += p[0] + p[1];
+    s.l[1] += p[2] + p[3];
+    pa[nt * 2 + 0] = pack_bf16x2(p[0], p[1]);
+    pa[nt * 2 + 1] = pack_bf16x2(p[2], p[3]);
+  }
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) {
+    s.o[n][0] *= alpha[0];
+    s.o[n][1] *= alpha[0];
+    s.o[n][2] *= alpha[1];
+    s.o[n][3] *= alpha[1];
+  }
+#pragma unroll
+  for (int n = 0; n < D / 8; n += 2) {
+    const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
+    const int unit = n + (lane >> 4);
+    uint32_t b0, b1, b2, b3;
+    ldsm_x4_t(vaddr + (row * D + swz_unit(row, unit) * 8) * 2, b0, b1, b2, b3);
+    mma_bf16_16816(s.o[n], pa, b0, b1);
+    mma_bf16_16816(s.o[n + 1], pa, b2, b3);
+  }
 }
 
 // Pass B on one chunk: S = Q K^T, dP = dO V^T, dS = gs * P * (dP - dg), dq += dS K.
@@ -132,7 +234,7 @@ __device__ __forceinline__ void bwd_dq_chunk(float (&dq)[D / 8][4], const uint32
     for (int e = 0; e < 4; ++e) {
       const int r = e >> 1;
       const int key = cd.start + nt * 8 + 2 * (lane & 3) + (e & 1);
-      const bool ok = key >= cd.lo && key < cd.hi && lse2[r] != -INFINITY;
+      const bool ok = key >= cd.lo[r] && key < cd.hi[r] && lse2[r] != -INFINITY;
       const float p = ok ? ex2_approx(sc[nt][e] * sl2 - lse2[r]) : 0.f;
       ds[e] = gs[r] * p * (dp[nt][e] - dg[r]);
     }
@@ -150,21 +252,20 @@ __device__ __forceinline__ void bwd_dq_chunk(float (&dq)[D / 8][4], const uint32
   }
 }
 
-// <dO, o / l> for the two rows this thread holds, reduced over the quad.
+// <dO, o / l> of the two rows this thread holds (half r from dO row pointer p[r]), reduced
+// over the quad.
 template <int D>
-__device__ __forceinline__ void bwd_row_dot(const WarpAttnState<D>& s, const __nv_bfloat16* dorow, int G,
+__device__ __forceinline__ void bwd_row_dot(const WarpAttnState<D>& s, const __nv_bfloat16* const (&p)[2],
                                             int lane, float (&dg)[2]) {
-  const int r0 = lane >> 2, c = 2 * (lane & 3);
+  const int c = 2 * (lane & 3);
   float part[2] = {0.f, 0.f};
 #pragma unroll
-  for (int n = 0; n < D / 8; ++n) {
+  for (int r = 0; r < 2; ++r) {
+    if (p[r] == nullptr) continue;
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int row = r0 + 8 * r;
-      if (row < G) {
-        const float2 d = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dorow + row * D + n * 8 + c));
-        part[r] += s.o[n][2 * r] * d.x + s.o[n][2 * r + 1] * d.y;
-      }
+    for (int n = 0; n < D / 8; ++n) {
+      const float2 d = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p[r] + n * 8 + c));
+      part[r] += s.o[n][2 * r] * d.x + s.o[n][2 * r + 1] * d.y;
     }
   }
 #pragma unroll
@@ -176,105 +277,163 @@ __device__ __forceinline__ void bwd_row_dot(const WarpAttnState<D>& s, const __n
 }
 
 template <int D>
+struct BwdRowSmem {
+  WarpChunkBuf<D, kBwdChunk, 2> buf;
+  int2 blocks[128];  // the union of the tokens' selected blocks: (block, mask of the halves)
+};
+
+template <int D>
 __global__ void __launch_bounds__(32 * kBwdWarps) bwd_row_kernel(const BwdArgs a) {
   extern __shared__ __align__(128) uint8_t bwd_row_smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  auto& buf = reinterpret_cast<WarpChunkBuf<D, kBwdChunk, 2>*>(bwd_row_smem)[warp];
+  auto& sm = reinterpret_cast<BwdRowSmem<D>*>(bwd_row_smem)[warp];
+  const int G = a.G;
+  const int tpw = G <= 8 ? 2 : 1;  // tokens per warp
+  const int nv_items = (a.nv + tpw - 1) / tpw;
+  const int nt_items = (a.N - a.nv + tpw - 1) / tpw;
   const long long item = static_cast<long long>(blockIdx.x) * kBwdWarps + warp;
-  if (item >= static_cast<long long>(a.N) * a.hkv) return;  // warp-uniform; no CTA-wide barrier follows
-  const int t = static_cast<int>(item / a.hkv), g = static_cast<int>(item % a.hkv);
-  const int G = a.G, h0 = g * G;
+  if (item >= static_cast<long long>(nv_items + nt_items) * a.hkv) return;  // warp-uniform, no CTA barrier follows
+  const int g = static_cast<int>(item % a.hkv);
+  const int pi = static_cast<int>(item / a.hkv);
+  const bool video = pi < nv_items;
+  const int t_end = video ? a.nv : a.N;
+  const int tA = video ? pi * tpw : a.nv + (pi - nv_items) * tpw;
+  const int h0 = g * G;
   const int r0 = lane >> 2;
-  const __nv_bfloat16* qrow = a.q + (static_cast<size_t>(t) * a.hq + h0) * D;
-  const __nv_bfloat16* dorow = a.dout + (static_cast<size_t>(t) * a.hq + h0) * D;
+  // the two halves: token, head and validity
+  int tok[2], head[2];
+  bool ok[2];
+  if (tpw == 2) {
+    tok[0] = tA;
+    tok[1] = tA + 1;
+    head[0] = head[1] = r0;
+    ok[0] = r0 < G;
+    ok[1] = r0 < G && tA + 1 < t_end;
+  } else {
+    tok[0] = tok[1] = tA;
+    head[0] = r0;
+    head[1] = r0 + 8;
+    ok[0] = r0 < G;
+    ok[1] = r0 + 8 < G;
+  }
+  const bool has_b = tpw == 2 ? (tA + 1 < t_end) : true;  // warp-uniform: half 1 exists at all
+  const int tB = tpw == 2 ? (has_b ? tA + 1 : tA) : tA;   // the later token of the warp
+  const __nv_bfloat16* qp[2];
+  const __nv_bfloat16* dp[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const size_t row = (static_cast<size_t>(tok[r]) * a.hq + h0 + head[r]) * D;
+    qp[r] = ok[r] ? a.q + row : nullptr;
+    dp[r] = ok[r] ? a.dout + row : nullptr;
+  }
   const size_t kv_stride = static_cast<size_t>(a.hkv) * D;
   uint32_t qa[D / 16][4];
-  load_q_frags<D>(qa, qrow, G, lane);
+  bwd_load_frags<D>(qa, qp[0], qp[1], lane);
   float dq[D / 8][4];
 #pragma unroll
   for (int n = 0; n < D / 8; ++n) dq[n][0] = dq[n][1] = dq[n][2] = dq[n][3] = 0.f;
-  const bool video = t < a.nv;
   const int nb = video ? 3 : 1;
-  const int32_t* sel = video ? a.sel_idx + (static_cast<size_t>(t) * a.hkv + g) * a.top_n : nullptr;
-  for (int b = 0; b < nb; ++b) {
-    const int br = video ? b : static_cast<int>(kBwdDense);
-    // the branch's keys as chunks of 16
-    int nch = 0, lo = 0, hi = 0, nvalid = 0, tail = 0;
-    const __nv_bfloat16* kb = (br == kBwdCmp) ? a.kc + g * D : a.k + g * D;
-    const __nv_bfloat16* vb = (br == kBwdCmp) ? a.vc + g * D : a.v + g * D;
-    if (br == kBwdCmp) {
-      const int nc = t >= a.cmp_len - 1 ? min((t - a.cmp_len + 1) / a.cmp_stride + 1, a.ncmp) : 0;
-      lo = 0;
-      hi = nc;
-      nch = (nc + kBwdChunk - 1) / kBwdChunk;
-    } else if (br == kBwdWin) {
-      lo = max(0, t - a.window + 1);
-      hi = t + 1;
-      nch = (hi - lo + kBwdChunk - 1) / kBwdChunk;
-    } else if (br == kBwdDense) {
-      lo = 0;
-      hi = t + 1;
-      nch = (hi + kBwdChunk - 1) / kBwdChunk;
-    } else {
-      while (nvalid < a.top_n && sel[nvalid] >= 0) ++nvalid;
-      if (nvalid > 0) {
-        const int last = sel[nvalid - 1];
-        const int span = min(a.sel_len, t + 1 - last * a.sel_len);
-        tail = span > 0 ? (span + kBwdChunk - 1) / kBwdChunk : 0;
-        nch = (nvalid - 1) * (a.sel_len / kBwdChunk) + tail;
+  // token of each half for the key ranges (a missing token B takes A's ranges, masked off by gs = 0)
+  const int tk[2] = {tok[0], tpw == 2 ? tB : tok[1]};
+  int nblk = 0;
+  if (video) {
+    // the union of the tokens' selected blocks, ascending, with the halves that chose each
+    if (lane == 0) {
+      const int32_t* sa_ = a.sel_idx + (static_cast<size_t>(tk[0]) * a.hkv + g) * a.top_n;
+      const int32_t* sb_ = a.sel_idx + (static_cast<size_t>(tk[1]) * a.hkv + g) * a.top_n;
+      int ia = 0, ib = 0;
+      while (true) {
+        const int ja = ia < a.top_n ? sa_[ia] : -1;
+        const int jb = ib < a.top_n ? sb_[ib] : -1;
+        if (ja < 0 && jb < 0) break;
+        int j, mask;
+        if (jb < 0 || (ja >= 0 && ja < jb)) {
+          j = ja;
+          mask = 1;
+          ++ia;
+        } else if (ja < 0 || jb < ja) {
+          j = jb;
+          mask = 2;
+          ++ib;
+        } else {
+          j = ja;
+          mask = 3;
+          ++ia;
+          ++ib;
+        }
+        sm.blocks[nblk++] = make_int2(j, mask);
       }
     }
-    const int per_block = a.sel_len / kBwdChunk;
+    nblk = __shfl_sync(0xffffffffu, nblk, 0);
+    __syncwarp();
+  }
+  const int per_block = a.sel_len / kBwdChunk;
+  for (int b = 0; b < nb; ++b) {
+    const int br = video ? b : static_cast<int>(kBwdDense);
+    const __nv_bfloat16* kb = (br == kBwdCmp) ? a.kc + g * D : a.k + g * D;
+    const __nv_bfloat16* vb = (br == kBwdCmp) ? a.vc + g * D : a.v + g * D;
+    int lo[2], hi[2], nch = 0;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int t = tk[r];
+      if (br == kBwdCmp) {
+        lo[r] = 0;
+        hi[r] = t >= a.cmp_len - 1 ? min((t - a.cmp_len + 1) / a.cmp_stride + 1, a.ncmp) : 0;
+      } else if (br == kBwdWin) {
+        lo[r] = max(0, t - a.window + 1);
+        hi[r] = t + 1;
+      } else {
+        lo[r] = 0;
+        hi[r] = t + 1;
+      }
+    }
+    const int range_lo = min(lo[0], lo[1]), range_hi = max(hi[0], hi[1]);
+    if (br == kBwdSel) nch = nblk * per_block;
+    else nch = range_hi > range_lo ? (range_hi - range_lo + kBwdChunk - 1) / kBwdChunk : 0;
     auto desc = [&](int c) -> ChunkDesc {
       ChunkDesc d;
-      d.kb = kb;
-      d.vb = vb;
       if (br == kBwdSel) {
-        const int slot = min(c / per_block, nvalid - 1);
-        const int sub = c - slot * per_block;
-        const int j = sel[slot];
-        d.start = j * a.sel_len + sub * kBwdChunk;
-        d.row_end = min(j * a.sel_len + a.sel_len, t + 1);
-        d.lo = d.start;
-        d.hi = d.row_end;
+        const int2 e = sm.blocks[c / per_block];
+        d.start = e.x * a.sel_len + (c % per_block) * kBwdChunk;
+        d.row_end = d.start;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int end = min(e.x * a.sel_len + a.sel_len, tk[r] + 1);
+          const bool mine = (e.y >> r) & 1;
+          d.lo[r] = d.start;
+          d.hi[r] = mine ? end : d.start;
+          d.row_end = max(d.row_end, d.hi[r]);
+        }
       } else {
-        d.start = lo + c * kBwdChunk;
-        d.row_end = hi;
-        d.lo = lo;
-        d.hi = hi;
+        d.start = range_lo + c * kBwdChunk;
+        d.row_end = range_hi;
+        d.lo[0] = lo[0];
+        d.lo[1] = lo[1];
+        d.hi[0] = hi[0];
+        d.hi[1] = hi[1];
       }
       return d;
     };
     // pass A: log-sum-exp and o_b
     WarpAttnState<D> st;
     state_init<D>(st);
-    bwd_stream<D>(buf, kv_stride, nch, desc,
-                  [&](int stg, const ChunkDesc& cd) {
-                    attend_chunk<D, kBwdChunk, 2>(st, qa, buf, stg, cd.start, cd.lo, cd.hi, a.sl2, lane);
-                  },
+    bwd_stream<D>(sm.buf, kb, vb, kv_stride, nch, desc,
+                  [&](int stg, const ChunkDesc& cd) { bwd_attend_chunk<D>(st, qa, sm.buf, stg, cd, a.sl2, lane); },
                   lane);
     state_reduce_l<D>(st);
     float lse2[2], dg[2], gs[2];
 #pragma unroll
     for (int r = 0; r < 2; ++r) lse2[r] = st.l[r] > 0.f ? st.m[r] + __log2f(st.l[r]) : -INFINITY;
-    bwd_row_dot<D>(st, dorow, G, lane, dg);
+    bwd_row_dot<D>(st, dp, lane, dg);
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      const int row = r0 + 8 * r;
-      const float gate = row < G ? (video ? a.gates[(static_cast<size_t>(t) * a.hq + h0 + row) * 3 + b] : 1.f) : 0.f;
+      const size_t o = (static_cast<size_t>(tok[r]) * a.hq + h0 + head[r]) * 3;
+      const float gate = ok[r] ? (video ? a.gates[o + b] : 1.f) : 0.f;
       gs[r] = gate * a.scale;
-      if ((lane & 3) == 0 && row < G) {
-        const size_t o = (static_cast<size_t>(t) * a.hq + h0 + row) * 3 + b;
-        a.stats[o] = make_float2(lse2[r], dg[r]);
-        a.dgates[o] = video ? dg[r] : 0.f;
-      }
-    }
-    if (!video && (lane & 3) == 0) {
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int row = r0 + 8 * r;
-        if (row < G) {
-          const size_t o = (static_cast<size_t>(t) * a.hq + h0 + row) * 3;
+      if ((lane & 3) == 0 && ok[r]) {
+        a.stats[o + b] = make_float2(lse2[r], dg[r]);
+        a.dgates[o + b] = video ? dg[r] : 0.f;
+        if (!video) {
           a.dgates[o + 1] = 0.f;
           a.dgates[o + 2] = 0.f;
         }
@@ -282,24 +441,21 @@ __global__ void __launch_bounds__(32 * kBwdWarps) bwd_row_kernel(const BwdArgs a
     }
     // pass B: dS and dq
     uint32_t da[D / 16][4];
-    load_q_frags<D>(da, dorow, G, lane);
-    bwd_stream<D>(buf, kv_stride, nch, desc,
+    bwd_load_frags<D>(da, dp[0], dp[1], lane);
+    bwd_stream<D>(sm.buf, kb, vb, kv_stride, nch, desc,
                   [&](int stg, const ChunkDesc& cd) {
-                    bwd_dq_chunk<D>(dq, qa, da, buf, stg, cd, a.sl2, lse2, dg, gs, lane);
+                    bwd_dq_chunk<D>(dq, qa, da, sm.buf, stg, cd, a.sl2, lse2, dg, gs, lane);
                   },
                   lane);
   }
   const int c = 2 * (lane & 3);
 #pragma unroll
-  for (int n = 0; n < D / 8; ++n) {
+  for (int r = 0; r < 2; ++r) {
+    if (!ok[r]) continue;
+    float* dst = a.dq + (static_cast<size_t>(tok[r]) * a.hq + h0 + head[r]) * D + c;
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int row = r0 + 8 * r;
-      if (row < G) {
-        float* dst = a.dq + (static_cast<size_t>(t) * a.hq + h0 + row) * D + n * 8 + c;
-        *reinterpret_cast<float2*>(dst) = make_float2(dq[n][2 * r], dq[n][2 * r + 1]);
-      }
-    }
+    for (int n = 0; n < D / 8; ++n)
+      *reinterpret_cast<float2*>(dst + n * 8) = make_float2(dq[n][2 * r], dq[n][2 * r + 1]);
   }
 }
 

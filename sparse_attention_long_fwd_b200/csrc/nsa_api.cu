@@ -944,10 +944,11 @@ int backward_impl(const nsa_params_t* p, const void* q, const void* k, const voi
   }
   // row pass: dq, the gates' gradient and the per-branch statistics
   {
-    const size_t smem = nsa::kBwdWarps * sizeof(nsa::WarpChunkBuf<D, nsa::kBwdChunk, 2>);
+    const size_t smem = nsa::kBwdWarps * sizeof(nsa::BwdRowSmem<D>);
     auto kern = nsa::bwd_row_kernel<D>;
     if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
-    const long long items = static_cast<long long>(N) * hkv;
+    const int tpw = G <= 8 ? 2 : 1;  // tokens per warp, as the kernel pairs them
+    const long long items = static_cast<long long>((nv + tpw - 1) / tpw + (N - nv + tpw - 1) / tpw) * hkv;
     kern<<<static_cast<unsigned>((items + nsa::kBwdWarps - 1) / nsa::kBwdWarps), 32 * nsa::kBwdWarps, smem, st>>>(a);
     if ((rc = launch_status("bwd_row", st)) != NSA_OK) return rc;
   }
