@@ -501,7 +501,7 @@ def run_backward(args, dev, q, k, v, g, peaks, flush, world):
     rc = nsa.nsa_prefill(q, k, v, g, p, out, sel, ws, ws.numel())
     if rc != nsa.NSA_OK:
         raise nsa.NsaError(rc, "nsa_prefill")
-    del ws, out
+    del out  # ws keeps the forward's saved statistics
     gen = torch.Generator(device=dev).manual_seed(31)
     d_out = torch.randn((w.n_tokens, w.hq, w.d), generator=gen, device=dev).to(torch.bfloat16)
     dq = torch.empty((w.n_tokens, w.hq, w.d), dtype=torch.float32, device=dev)
@@ -511,7 +511,7 @@ def run_backward(args, dev, q, k, v, g, peaks, flush, world):
     bws = torch.empty(nsa.nsa_backward_workspace_size(p), dtype=torch.uint8, device=dev)
 
     def step(events):
-        rc = nsa.nsa_backward(q, k, v, g, d_out, sel, None, None, p, dq, dk, dv, dgates, bws, bws.numel())
+        rc = nsa.nsa_backward(q, k, v, g, d_out, sel, ws, None, None, p, dq, dk, dv, dgates, bws, bws.numel())
         if rc != nsa.NSA_OK:
             raise nsa.NsaError(rc, "nsa_backward")
 
@@ -524,9 +524,9 @@ def run_backward(args, dev, q, k, v, g, peaks, flush, world):
     flops = 2.5 * (c["cmp_flops"] + c["sel_flops"] + c["win_flops"] + c["text_flops"])
     tf = flops / (ms / 1e3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
-    del bws, dq, dk, dv, dgates, d_out
+    del bws, dq, dk, dv, dgates, d_out, ws
     return {"workload": "v128k backward: dq, dk, dv and the gates' gradient of the headline prefill "
-                        "(selection of its forward held constant)",
+                        "(its forward's selection held constant; its saved compressed-branch statistics reused)",
             "ms_per_step": round(ms, 3), "value": round(w.n_video * world / (ms / 1e3), 1),
             "unit": "video tokens/s", "steps": args.steps, "warmup": args.warmup,
             "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peak, "unit": "TFLOP/s",

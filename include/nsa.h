@@ -228,6 +228,9 @@ size_t nsa_gate_mlp_pooled_workspace_size(int batch, int seq_len, int heads, int
  *   q, k, v, gates, params: as given to nsa_prefill (or nsa_prefill_phi)
  *   d_out    [N][Hq][d] bf16, dL/dout
  *   sel_idx  [N_v][Hkv][top_n] int32: the forward's selection (nsa_prefill's out_sel_idx)
+ *   fwd_workspace  NULL, or the workspace of the nsa_prefill / nsa_prefill_phi call being
+ *            differentiated, unchanged since: its compressed-branch log-sum-exp and output
+ *            (nsa_prefill_workspace_layout: lse, o_cmp) then replace a recomputation
  *   phi_k, phi_v  both NULL (mean compression) or both the learnable weights [Hkv][l] fp32
  *   dq       [N][Hq][d] fp32     dk, dv [N][Hkv][d] fp32    (written, not accumulated)
  *   dgates   [N][Hq][3] fp32: <dL/dout, o_b> per branch; 0 for text rows
@@ -237,9 +240,9 @@ size_t nsa_gate_mlp_pooled_workspace_size(int batch, int seq_len, int heads, int
  * last bits vary from run to run.
  */
 int nsa_backward(const void* q, const void* k, const void* v, const float* gates, const void* d_out,
-                 const int32_t* sel_idx, const float* phi_k, const float* phi_v, const nsa_params_t* params,
-                 float* dq, float* dk, float* dv, float* dgates, void* workspace, size_t workspace_bytes,
-                 void* stream);
+                 const int32_t* sel_idx, const void* fwd_workspace, const float* phi_k, const float* phi_v,
+                 const nsa_params_t* params, float* dq, float* dk, float* dv, float* dgates, void* workspace,
+                 size_t workspace_bytes, void* stream);
 
 /* Workspace bytes nsa_backward needs; 0 if params are invalid. */
 size_t nsa_backward_workspace_size(const nsa_params_t* params);

@@ -16,7 +16,9 @@
 //                    Per branch: pass A streams the keys once for each row's log-sum-exp
 //                    and o_b, giving <dO, o_b> (the gate gradient); pass B streams them
 //                    again for dS and dq += dS K. Writes dq, the gate gradient and
-//                    (lse, <dO, o_b>) per (row, branch) for the next pass.
+//                    (lse, <dO, o_b>) per (row, branch) for the next pass. Given the
+//                    forward's saved log-sum-exp and output of the compressed branch,
+//                    that branch skips pass A.
 //   bwd_key_kernel   one warp per (branch, 16-key tile, group, segment of the rows that
 //                    attend those keys): S^T = K Q^T and dP^T = V dO^T for 16 rows at a
 //                    time, then dv += P^T dO and dk += dS^T Q in registers; the sums are
@@ -25,6 +27,7 @@
 //   pool_bwd_kernel  the compressed keys' gradient back to the tokens of each block.
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cstdint>
 
 #include "warp_attn.cuh"
@@ -60,6 +63,8 @@ struct BwdArgs {
   const int* ent_off;         // selected-branch buckets: [hkv*nsel + 1] entry offsets
   const int* seg_off;         // [hkv*nsel + 1] segment offsets (ceil(count / kBwdSegSel))
   const int* list;            // bucketed entries t * 64 + slot
+  const float* fwd_lse;       // [nv][hq] the forward's compressed-branch log-sum-exp (natural log),
+  const __half* fwd_ocmp;     // [nv][hq][D] and its output, or both null: pass A recomputes them
 };
 
 // ---------------------------------------------------------------- row pass
@@ -414,17 +419,43 @@ __global__ void __launch_bounds__(32 * kBwdWarps) bwd_row_kernel(const BwdArgs a
       }
       return d;
     };
-    // pass A: log-sum-exp and o_b
-    WarpAttnState<D> st;
-    state_init<D>(st);
-    bwd_stream<D>(sm.buf, kb, vb, kv_stride, nch, desc,
-                  [&](int stg, const ChunkDesc& cd) { bwd_attend_chunk<D>(st, qa, sm.buf, stg, cd, a.sl2, lane); },
-                  lane);
-    state_reduce_l<D>(st);
     float lse2[2], dg[2], gs[2];
+    if (br == kBwdCmp && a.fwd_lse != nullptr) {
+      // the forward's statistics: lse2 = lse / ln 2, <dO, o_cmp> from its fp16 output
+      const int c = 2 * (lane & 3);
+      float part[2] = {0.f, 0.f};
 #pragma unroll
-    for (int r = 0; r < 2; ++r) lse2[r] = st.l[r] > 0.f ? st.m[r] + __log2f(st.l[r]) : -INFINITY;
-    bwd_row_dot<D>(st, dp, lane, dg);
+      for (int r = 0; r < 2; ++r) {
+        lse2[r] = -INFINITY;
+        if (!ok[r]) continue;
+        const size_t row = static_cast<size_t>(tok[r]) * a.hq + h0 + head[r];
+        lse2[r] = a.fwd_lse[row] * 1.4426950408889634f;
+        const __half* o = a.fwd_ocmp + row * D + c;
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n) {
+          const float2 ov = __half22float2(*reinterpret_cast<const __half2*>(o + n * 8));
+          const float2 dv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dp[r] + n * 8 + c));
+          part[r] += ov.x * dv.x + ov.y * dv.y;
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        part[r] += __shfl_xor_sync(0xffffffffu, part[r], 1);
+        part[r] += __shfl_xor_sync(0xffffffffu, part[r], 2);
+        dg[r] = part[r];
+      }
+    } else {
+      // pass A: log-sum-exp and o_b
+      WarpAttnState<D> st;
+      state_init<D>(st);
+      bwd_stream<D>(sm.buf, kb, vb, kv_stride, nch, desc,
+                    [&](int stg, const ChunkDesc& cd) { bwd_attend_chunk<D>(st, qa, sm.buf, stg, cd, a.sl2, lane); },
+                    lane);
+      state_reduce_l<D>(st);
+#pragma unroll
+      for (int r = 0; r < 2; ++r) lse2[r] = st.l[r] > 0.f ? st.m[r] + __log2f(st.l[r]) : -INFINITY;
+      bwd_row_dot<D>(st, dp, lane, dg);
+    }
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
       const size_t o = (static_cast<size_t>(tok[r]) * a.hq + h0 + head[r]) * 3;

@@ -890,8 +890,8 @@ int launch_bwd_key(const nsa::BwdArgs& a, long long n_items, cudaStream_t st) {
 
 template <int D>
 int backward_impl(const nsa_params_t* p, const void* q, const void* k, const void* v, const float* gates,
-                  const void* d_out, const int32_t* sel_idx, const float* phi_k, const float* phi_v, float* dq,
-                  float* dk, float* dv, float* dgates, uint8_t* ws, cudaStream_t st) {
+                  const void* d_out, const int32_t* sel_idx, const uint8_t* fwd_ws, const float* phi_k,
+                  const float* phi_v, float* dq, float* dk, float* dv, float* dgates, uint8_t* ws, cudaStream_t st) {
   const BwdLayout L = bwd_layout(p);
   const int N = p->n_tokens, nv = p->n_video, hq = p->num_q_heads, hkv = p->num_kv_heads;
   const int G = hq / hkv;
@@ -930,6 +930,11 @@ int backward_impl(const nsa_params_t* p, const void* q, const void* k, const voi
   a.ent_off = reinterpret_cast<const int*>(ws + L.ent_off);
   a.seg_off = reinterpret_cast<const int*>(ws + L.seg_off);
   a.list = reinterpret_cast<const int*>(ws + L.list);
+  if (fwd_ws != nullptr && nv > 0) {
+    const PrefillLayout F = prefill_layout(p);
+    a.fwd_lse = reinterpret_cast<const float*>(fwd_ws + F.lse);
+    a.fwd_ocmp = reinterpret_cast<const __half*>(fwd_ws + F.o_cmp);
+  }
   const size_t kv_bytes = static_cast<size_t>(N) * hkv * D * 4;
   if (cudaMemsetAsync(dk, 0, kv_bytes, st) != cudaSuccess || cudaMemsetAsync(dv, 0, kv_bytes, st) != cudaSuccess)
     return NSA_ERR_CUDA;
@@ -1021,9 +1026,9 @@ size_t nsa_backward_workspace_size(const nsa_params_t* params) {
 }
 
 int nsa_backward(const void* q, const void* k, const void* v, const float* gates, const void* d_out,
-                 const int32_t* sel_idx, const float* phi_k, const float* phi_v, const nsa_params_t* params,
-                 float* dq, float* dk, float* dv, float* dgates, void* workspace, size_t workspace_bytes,
-                 void* stream) {
+                 const int32_t* sel_idx, const void* fwd_workspace, const float* phi_k, const float* phi_v,
+                 const nsa_params_t* params, float* dq, float* dk, float* dv, float* dgates, void* workspace,
+                 size_t workspace_bytes, void* stream) {
   int rc = check_common(params);
   if (rc != NSA_OK) return rc;
   if (params->n_video < 0 || params->n_video > params->n_tokens) return NSA_ERR_INVALID_ARG;
@@ -1033,7 +1038,8 @@ int nsa_backward(const void* q, const void* k, const void* v, const float* gates
   if ((phi_k == nullptr) != (phi_v == nullptr)) return NSA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(d_out) || !aligned16(dq) || !aligned16(dk) ||
       !aligned16(dv) || !aligned4(dgates) || (gates && !aligned4(gates)) || (sel_idx && !aligned4(sel_idx)) ||
-      (phi_k && (!aligned4(phi_k) || !aligned4(phi_v))) || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+      (phi_k && (!aligned4(phi_k) || !aligned4(phi_v))) || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 ||
+      (reinterpret_cast<uintptr_t>(fwd_workspace) % kAlign) != 0)
     return NSA_ERR_INVALID_ARG;
   if (nsel_of(params->n_video, params->sel_block) > 8192) return NSA_ERR_UNSUPPORTED;
   if (workspace_bytes < bwd_layout(params).total) return NSA_ERR_WORKSPACE_TOO_SMALL;
@@ -1044,8 +1050,10 @@ int nsa_backward(const void* q, const void* k, const void* v, const float* gates
   const int saved_count = g_stage_count;
   g_stage_count = 0;
   rc = params->head_dim == 64
-           ? backward_impl<64>(params, q, k, v, gates, d_out, sel_idx, phi_k, phi_v, dq, dk, dv, dgates, ws, st)
-           : backward_impl<128>(params, q, k, v, gates, d_out, sel_idx, phi_k, phi_v, dq, dk, dv, dgates, ws, st);
+           ? backward_impl<64>(params, q, k, v, gates, d_out, sel_idx, static_cast<const uint8_t*>(fwd_workspace),
+                               phi_k, phi_v, dq, dk, dv, dgates, ws, st)
+           : backward_impl<128>(params, q, k, v, gates, d_out, sel_idx, static_cast<const uint8_t*>(fwd_workspace),
+                                phi_k, phi_v, dq, dk, dv, dgates, ws, st);
   g_stage_count = saved_count;
   return rc;
 }

@@ -99,7 +99,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.nsa_gate_mlp_pooled.restype = I
     lib.nsa_gate_mlp_pooled_workspace_size.argtypes = [I, I, I, I]
     lib.nsa_gate_mlp_pooled_workspace_size.restype = S
-    lib.nsa_backward.argtypes = [P, P, P, P, P, P, P, P, PP, P, P, P, P, P, S, P]
+    lib.nsa_backward.argtypes = [P, P, P, P, P, P, P, P, P, PP, P, P, P, P, P, S, P]
     lib.nsa_backward.restype = I
     lib.nsa_backward_workspace_size.argtypes = [PP]
     lib.nsa_backward_workspace_size.restype = S
@@ -220,11 +220,12 @@ def nsa_gate_mlp_pooled_workspace_size(batch: int, seq_len: int, heads: int, dim
     return int(load_library().nsa_gate_mlp_pooled_workspace_size(batch, seq_len, heads, dim))
 
 
-def nsa_backward(q, k, v, gates, d_out, sel_idx, phi_k, phi_v, params: NsaParams, dq, dk, dv, dgates, workspace,
-                 workspace_bytes: int, stream=None) -> int:
+def nsa_backward(q, k, v, gates, d_out, sel_idx, fwd_workspace, phi_k, phi_v, params: NsaParams, dq, dk, dv, dgates,
+                 workspace, workspace_bytes: int, stream=None) -> int:
     return load_library().nsa_backward(_addr(q), _addr(k), _addr(v), _addr(gates), _addr(d_out), _addr(sel_idx),
-                                       _addr(phi_k), _addr(phi_v), ctypes.byref(params), _addr(dq), _addr(dk),
-                                       _addr(dv), _addr(dgates), _addr(workspace), workspace_bytes, _stream(stream))
+                                       _addr(fwd_workspace), _addr(phi_k), _addr(phi_v), ctypes.byref(params),
+                                       _addr(dq), _addr(dk), _addr(dv), _addr(dgates), _addr(workspace),
+                                       workspace_bytes, _stream(stream))
 
 
 def nsa_backward_workspace_size(params: NsaParams) -> int:
@@ -343,9 +344,11 @@ def decode(q, kcache, vcache, kcmp, vcmp, seq_lens, gates, *, top_n: int = 16, w
 
 
 def backward(q, k, v, gates, d_out, sel_idx, *, n_video: int | None = None, top_n: int = 16, window: int = 512,
-             softmax_scale: float = 0.0, phi=None, workspace: torch.Tensor | None = None, stream=None):
+             softmax_scale: float = 0.0, phi=None, fwd_workspace: torch.Tensor | None = None,
+             workspace: torch.Tensor | None = None, stream=None):
     """Gradients of the prefill: returns dq [N,Hq,d], dk, dv [N,Hkv,d] and dgates [N,Hq,3] (fp32),
-    given dL/dout (bf16) and the forward's selection sel_idx [N_v,Hkv,top_n]."""
+    given dL/dout (bf16) and the forward's selection sel_idx [N_v,Hkv,top_n]; fwd_workspace, the
+    forward call's workspace, lets the compressed branch reuse its saved statistics."""
     N, hq, d = q.shape
     hkv = k.shape[1]
     p = make_params(N, n_video, hq, hkv, d, top_n=top_n, window=window, softmax_scale=softmax_scale)
@@ -359,8 +362,8 @@ def backward(q, k, v, gates, d_out, sel_idx, *, n_video: int | None = None, top_
             raise NsaError(NSA_ERR_INVALID_ARG, "nsa_backward_workspace_size")
         workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
     pk, pv = (None, None) if phi is None else phi
-    _check(nsa_backward(q, k, v, gates, d_out, sel_idx, pk, pv, p, dq, dk, dv, dgates, workspace, workspace.numel(),
-                        stream), "nsa_backward")
+    _check(nsa_backward(q, k, v, gates, d_out, sel_idx, fwd_workspace, pk, pv, p, dq, dk, dv, dgates, workspace,
+                        workspace.numel(), stream), "nsa_backward")
     return dq, dk, dv, dgates
 
 

@@ -167,15 +167,18 @@ def test_backward_validation():
     p = _p()
     need = nsa.nsa_backward_workspace_size(p)
     assert need > 0 and need % 256 == 0
-    ok_args = [f] * 6 + [None, None, p] + [f] * 5
+    ok_args = [f] * 6 + [None, None, None, p] + [f] * 5
     assert nsa.nsa_backward(*ok_args, need - 1, None) == nsa.NSA_ERR_WORKSPACE_TOO_SMALL
     bad = list(ok_args)
     bad[5] = None  # the forward's selection is required when there are video rows
     assert nsa.nsa_backward(*bad, need, None) == nsa.NSA_ERR_INVALID_ARG
     bad = list(ok_args)
-    bad[6] = f  # phi_k without phi_v
+    bad[7] = f  # phi_k without phi_v
     assert nsa.nsa_backward(*bad, need, None) == nsa.NSA_ERR_INVALID_ARG
     bad = list(ok_args)
-    bad[9] = f + 4  # dq misaligned
+    bad[10] = f + 4  # dq misaligned
+    assert nsa.nsa_backward(*bad, need, None) == nsa.NSA_ERR_INVALID_ARG
+    bad = list(ok_args)
+    bad[6] = f + 128  # the forward's workspace must be 256-byte aligned
     assert nsa.nsa_backward(*bad, need, None) == nsa.NSA_ERR_INVALID_ARG
     assert nsa.nsa_backward_workspace_size(_p(head_dim=96)) == 0

@@ -34,14 +34,14 @@ def _grad_close(got, ref, what):
     return round(mx, 6), round(mn, 7)
 
 
-def _run(w, seed, phi=None):
+def _run(w, seed, phi=None, saved=False):
     q, k, v, g = prefill_inputs(w, seed=seed, device=DEV)
     out, sel, ws, lay = run_prefill(w, q, k, v, g, phi=phi)
     gen = torch.Generator(device=DEV).manual_seed(seed + 100)
     d_out = torch.randn((w.n_tokens, w.hq, w.d), generator=gen, device=DEV).to(torch.bfloat16)
     sel_arg = sel if w.n_video > 0 else torch.zeros(1, dtype=torch.int32, device=DEV)
     dq, dk, dv, dgates = nsa.backward(q, k, v, g, d_out, sel_arg, n_video=w.n_video, top_n=w.top_n,
-                                      window=w.window, phi=phi)
+                                      window=w.window, phi=phi, fwd_workspace=ws if saved else None)
     torch.cuda.synchronize()
     assert nsa.nsa_get_device_error(clear=True) == 0
     return q, k, v, g, d_out, sel, (dq, dk, dv, dgates)
@@ -67,10 +67,12 @@ def _compare(w, q, k, v, g, d_out, sel, grads, phi=None):
     ("v128k", 300, 0, 4, 2, 64, 4, 64),               # all text
     ("v128k", 40, 40, 4, 2, 128, 3, 16),              # shorter than two compression blocks
 ])
-def test_backward_every_element(name, n, nv, hq, hkv, d, top_n, window):
+@pytest.mark.parametrize("saved", [False, True])
+def test_backward_every_element(name, n, nv, hq, hkv, d, top_n, window, saved):
+    """saved: the compressed branch takes the forward's saved log-sum-exp and output."""
     w = WORKLOADS[name] if n is None else scaled(WORKLOADS[name], n_tokens=n, n_video=nv, hq=hq, hkv=hkv, d=d,
                                                     top_n=top_n, window=window)
-    q, k, v, g, d_out, sel, grads = _run(w, seed=21)
+    q, k, v, g, d_out, sel, grads = _run(w, seed=21, saved=saved)
     sel = sel if w.n_video > 0 else torch.zeros((0, w.hkv, w.top_n), dtype=torch.int32)
     print(_compare(w, q, k, v, g, d_out, sel, grads))
 
@@ -78,7 +80,7 @@ def test_backward_every_element(name, n, nv, hq, hkv, d, top_n, window):
 def test_backward_learnable_compression():
     w = scaled(WORKLOADS["v128k"], n_tokens=900, n_video=900)
     phi = phi_weights(w.hkv, 32, seed=22, device=DEV)
-    q, k, v, g, d_out, sel, grads = _run(w, seed=23, phi=phi)
+    q, k, v, g, d_out, sel, grads = _run(w, seed=23, phi=phi, saved=True)
     print(_compare(w, q, k, v, g, d_out, sel, grads, phi=phi))
 
 
@@ -87,7 +89,7 @@ def test_backward_sum_identities_at_16k():
     zero and the mean's weights sum to one), and the value gradients sum to the dO of each
     row weighted by the gates of its non-empty branches."""
     w = WORKLOADS["v16k"]
-    q, k, v, g, d_out, sel, (dq, dk, dv, dgates) = _run(w, seed=24)
+    q, k, v, g, d_out, sel, (dq, dk, dv, dgates) = _run(w, seed=24, saved=True)
     G = w.hq // w.hkv
     do = d_out.double()
     rows = torch.arange(w.n_tokens, device=DEV)
