@@ -7,8 +7,9 @@
 // file has both forms:
 //   gate_mlp_kernel     per row (one token of one head): the first layer is a dense
 //                       [128 rows x dim] x [dim x dim/2] contraction on the tensor cores
-//                       (tcgen05, bf16 in, fp32 accumulator in TMEM); GELU, the second
-//                       layer and the softmax run on the CUDA cores, one thread per row.
+//                       (tcgen05, bf16 in, fp32 accumulator in TMEM); GELU (erf to 1.5e-7,
+//                       Abramowitz & Stegun 7.1.26), the second layer and the softmax run
+//                       on the CUDA cores, one thread per row.
 //   gate_mean_partial_kernel + gate_pooled_kernel
 //                       the averaged form: fp64 column sums over token chunks, then one
 //                       CTA per (sequence, head) finishes the mean and evaluates the MLP in
@@ -24,6 +25,21 @@
 
 namespace nsa {
 
+// erf(x) by Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26:
+// erf(x) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-x^2), t = 1 / (1 + p x), x >= 0,
+// with |error| <= 1.5e-7; odd in x. One reciprocal, one exp2 and a degree-5 polynomial.
+__device__ __forceinline__ float erf_as7126(float x) {
+  const float ax = fabsf(x);
+  const float t = __fdividef(1.0f, fmaf(0.3275911f, ax, 1.0f));
+  float poly = fmaf(1.061405429f, t, -1.453152027f);
+  poly = fmaf(poly, t, 1.421413741f);
+  poly = fmaf(poly, t, -0.284496736f);
+  poly = fmaf(poly, t, 0.254829592f);
+  poly *= t;
+  const float e = ex2_approx(-ax * ax * 1.4426950408889634f);  // exp(-x^2)
+  return copysignf(fmaf(-poly, e, 1.0f), x);
+}
+
 template <int DIM>
 struct GateSmem {
   static constexpr int kHid = DIM / 2;
@@ -32,8 +48,7 @@ struct GateSmem {
   static constexpr uint32_t kTxBytes = static_cast<uint32_t>(kChunks) * (128 + kHid) * 128;
   alignas(1024) uint8_t x[kChunks][128 * 128];   // 128 rows x 128 B per chunk, 128B-swizzled
   alignas(1024) uint8_t w1[kChunks][kHid * 128];  // kHid rows x 128 B per chunk
-  float b1[kHid];
-  float w2[3][kHid];
+  float4 wb[kHid];  // per hidden unit j: (b1[j], W2[0][j], W2[1][j], W2[2][j])
   float b2[4];
   uint64_t full;
   uint64_t mma_done;
@@ -71,8 +86,7 @@ __global__ void __launch_bounds__(128) gate_mlp_kernel(const __grid_constant__ C
     tmem_alloc(&sm.tmem_base, S::kTmemCols);
     tmem_relinquish();
   }
-  for (int i = tid; i < kHid; i += 128) sm.b1[i] = b1[i];
-  for (int i = tid; i < 3 * kHid; i += 128) (&sm.w2[0][0])[i] = w2[i];
+  for (int j = tid; j < kHid; j += 128) sm.wb[j] = make_float4(b1[j], w2[j], w2[kHid + j], w2[2 * kHid + j]);
   if (tid < 3) sm.b2[tid] = b2[tid];
   tc_fence_before();
   __syncthreads();
@@ -123,11 +137,12 @@ __global__ void __launch_bounds__(128) gate_mlp_kernel(const __grid_constant__ C
     float l0 = sm.b2[0], l1 = sm.b2[1], l2 = sm.b2[2];
 #pragma unroll
     for (int j = 0; j < kHid; ++j) {
-      const float h = acc[j] + sm.b1[j];
-      const float g = 0.5f * h * (1.0f + erff(h * 0.70710678118654752f));
-      l0 = fmaf(sm.w2[0][j], g, l0);
-      l1 = fmaf(sm.w2[1][j], g, l1);
-      l2 = fmaf(sm.w2[2][j], g, l2);
+      const float4 w = sm.wb[j];
+      const float h = acc[j] + w.x;
+      const float g = 0.5f * h * (1.0f + erf_as7126(h * 0.70710678118654752f));
+      l0 = fmaf(w.y, g, l0);
+      l1 = fmaf(w.z, g, l1);
+      l2 = fmaf(w.w, g, l2);
     }
     const float m = fmaxf(l0, fmaxf(l1, l2));
     const float e0 = expf(l0 - m), e1 = expf(l1 - m), e2 = expf(l2 - m);
