@@ -170,7 +170,10 @@ __global__ void __launch_bounds__(128) gate_mlp_kernel(const __grid_constant__ C
 
 // Averaged form, step 1: fp64 column sums of x [B][T][cols] bf16 (cols = H*DIM) over the
 // token chunk [c*chunk, min(T, (c+1)*chunk)) of sequence b = blockIdx.y, c = blockIdx.x;
-// partial [nchunk][B][cols] fp64. One thread per bf16x2 column pair, 256 threads.
+// partial [nchunk][B][cols] fp64. A thread owns up to kGatePairs bf16x2 column pairs,
+// blockDim.x apart, and walks the chunk's tokens once, so its loads for one token are
+// independent of one another.
+constexpr int kGatePairs = 8;
 __global__ void __launch_bounds__(256) gate_mean_partial_kernel(const __nv_bfloat16* __restrict__ x,
                                                                 double* __restrict__ partial, int B, int T,
                                                                 int cols, int chunk) {
@@ -179,58 +182,75 @@ __global__ void __launch_bounds__(256) gate_mean_partial_kernel(const __nv_bfloa
   const int pairs = cols / 2;
   const __nv_bfloat162* base = reinterpret_cast<const __nv_bfloat162*>(x + static_cast<size_t>(b) * T * cols);
   double* out = partial + (static_cast<size_t>(c) * B + b) * cols;
-  for (int p = threadIdx.x; p < pairs; p += blockDim.x) {
-    double s0 = 0.0, s1 = 0.0;
-    int t = t0;
-    for (; t + 4 <= t1; t += 4) {
-      float2 v[4];
+  for (int p0 = threadIdx.x; p0 < pairs; p0 += blockDim.x * kGatePairs) {
+    double s0[kGatePairs], s1[kGatePairs];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = __bfloat1622float2(base[static_cast<size_t>(t + u) * pairs + p]);
+    for (int u = 0; u < kGatePairs; ++u) s0[u] = s1[u] = 0.0;
+    for (int t = t0; t < t1; ++t) {
+      const __nv_bfloat162* row = base + static_cast<size_t>(t) * pairs;
+      float2 v[kGatePairs];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        s0 += static_cast<double>(v[u].x);
-        s1 += static_cast<double>(v[u].y);
+      for (int u = 0; u < kGatePairs; ++u) {
+        const int p = p0 + u * blockDim.x;
+        v[u] = p < pairs ? __bfloat1622float2(row[p]) : make_float2(0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kGatePairs; ++u) {
+        s0[u] += static_cast<double>(v[u].x);
+        s1[u] += static_cast<double>(v[u].y);
       }
     }
-    for (; t < t1; ++t) {
-      const float2 v = __bfloat1622float2(base[static_cast<size_t>(t) * pairs + p]);
-      s0 += static_cast<double>(v.x);
-      s1 += static_cast<double>(v.y);
+#pragma unroll
+    for (int u = 0; u < kGatePairs; ++u) {
+      const int p = p0 + u * blockDim.x;
+      if (p < pairs) {
+        out[2 * p] = s0[u];
+        out[2 * p + 1] = s1[u];
+      }
     }
-    out[2 * p] = s0;
-    out[2 * p + 1] = s1;
   }
 }
 
 // Averaged form, step 2: CTA (b, h) = (blockIdx.x / H, blockIdx.x % H) adds the nchunk
-// partials in chunk order, divides by T and evaluates the MLP and softmax in fp64, then
-// writes the triple to gates[b][r][h][0..2] for every r < repeat. DIM threads (>= 64).
+// partials (kPooledSplit interleaved runs per column, then the runs in order), divides by
+// T and evaluates the MLP and softmax in fp64, then writes the triple to
+// gates[b][r][h][0..2] for every r < repeat. kPooledSplit * DIM threads.
+constexpr int kPooledSplit = 4;
 template <int DIM>
-__global__ void __launch_bounds__(DIM) gate_pooled_kernel(const double* __restrict__ partial,
+__global__ void __launch_bounds__(kPooledSplit * DIM) gate_pooled_kernel(const double* __restrict__ partial,
                                                           const __nv_bfloat16* __restrict__ w1,
                                                           const float* __restrict__ b1,
                                                           const float* __restrict__ w2,
                                                           const float* __restrict__ b2, float* __restrict__ gates,
                                                           int B, int T, int H, int nchunk, int repeat) {
   constexpr int kHid = DIM / 2;
+  __shared__ double run[kPooledSplit][DIM];
   __shared__ double mean[DIM];
   __shared__ double hid[kHid];
   __shared__ float res[3];
   const int b = blockIdx.x / H, h = blockIdx.x % H;
-  const int j = threadIdx.x;
+  const int j = threadIdx.x % DIM, part = threadIdx.x / DIM;
   const size_t cols = static_cast<size_t>(H) * DIM;
   double s = 0.0;
-  for (int c = 0; c < nchunk; ++c) s += partial[(static_cast<size_t>(c) * B + b) * cols + static_cast<size_t>(h) * DIM + j];
-  mean[j] = s / static_cast<double>(T);
+  for (int c = part; c < nchunk; c += kPooledSplit)
+    s += partial[(static_cast<size_t>(c) * B + b) * cols + static_cast<size_t>(h) * DIM + j];
+  run[part][j] = s;
   __syncthreads();
-  if (j < kHid) {
+  if (threadIdx.x < DIM) {
+    double m = 0.0;
+#pragma unroll
+    for (int q = 0; q < kPooledSplit; ++q) m += run[q][j];
+    mean[j] = m / static_cast<double>(T);
+  }
+  __syncthreads();
+  if (threadIdx.x < kHid) {
     double a = static_cast<double>(b1[j]);
     for (int i = 0; i < DIM; ++i)
       a += static_cast<double>(__bfloat162float(w1[static_cast<size_t>(j) * DIM + i])) * mean[i];
     hid[j] = 0.5 * a * (1.0 + erf(a * 0.70710678118654752440));
   }
   __syncthreads();
-  if (j == 0) {
+  if (threadIdx.x == 0) {
     double lg[3];
     for (int c = 0; c < 3; ++c) {
       double a = static_cast<double>(b2[c]);
@@ -245,7 +265,7 @@ __global__ void __launch_bounds__(DIM) gate_pooled_kernel(const double* __restri
     res[2] = static_cast<float>(e2 / z);
   }
   __syncthreads();
-  for (int r = j; r < repeat; r += DIM) {
+  for (int r = threadIdx.x; r < repeat; r += blockDim.x) {
     float* g = gates + ((static_cast<size_t>(b) * repeat + r) * H + h) * 3;
     g[0] = res[0];
     g[1] = res[1];

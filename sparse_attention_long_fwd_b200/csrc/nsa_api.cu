@@ -828,11 +828,11 @@ int nsa_gate_mlp_pooled(const void* x, const void* w1, const float* b1, const fl
   const unsigned grid = static_cast<unsigned>(batch) * heads;
   const auto* w1b = static_cast<const __nv_bfloat16*>(w1);
   if (dim == 64)
-    nsa::gate_pooled_kernel<64><<<grid, 64, 0, st>>>(part, w1b, b1, w2, b2, gates, batch, seq_len, heads, nchunk,
-                                                      repeat);
+    nsa::gate_pooled_kernel<64><<<grid, nsa::kPooledSplit * 64, 0, st>>>(part, w1b, b1, w2, b2, gates, batch,
+                                                                          seq_len, heads, nchunk, repeat);
   else
-    nsa::gate_pooled_kernel<128><<<grid, 128, 0, st>>>(part, w1b, b1, w2, b2, gates, batch, seq_len, heads, nchunk,
-                                                        repeat);
+    nsa::gate_pooled_kernel<128><<<grid, nsa::kPooledSplit * 128, 0, st>>>(part, w1b, b1, w2, b2, gates, batch,
+                                                                            seq_len, heads, nchunk, repeat);
   return launch_status("gate_pooled", st, false);
 }
 
