@@ -463,14 +463,14 @@ def test_gates_hand_worked_case_pins_layouts_and_gelu():
 
 
 def _torch_gate_module(dim, w1_bits, b1, w2, b2):
-    """The blog's two-layer gate module built from torch.nn layers in float64."""
-    m = torch.nn.Sequential(torch.nn.Linear(dim, dim // 2), torch.nn.GELU(), torch.nn.Linear(dim // 2, 3)).double()
-    with torch.no_grad():
-        m[0].weight.copy_(_f64(w1_bits))
-        m[0].bias.copy_(torch.from_numpy(np.asarray(b1, np.float32).astype(np.float64)))
-        m[2].weight.copy_(torch.from_numpy(np.asarray(w2, np.float32).astype(np.float64)))
-        m[2].bias.copy_(torch.from_numpy(np.asarray(b2, np.float32).astype(np.float64)))
-    return m
+    """The two-layer gate network evaluated with torch.nn.functional in float64."""
+    W1 = _f64(w1_bits)
+    B1, W2, B2 = (torch.from_numpy(np.asarray(a, np.float32).astype(np.float64)) for a in (b1, w2, b2))
+
+    def mlp(x):
+        return torch.nn.functional.linear(torch.nn.functional.gelu(torch.nn.functional.linear(x, W1, B1)), W2, B2)
+
+    return mlp
 
 
 def _rand_gate_weights(dim, seed):
@@ -488,7 +488,7 @@ def test_gates_match_torch_module(dim):
     x = _bits(_rand_bf16((7, 4, dim), 42))
     got = gate_orc.gate_mlp(x, w1, b1, w2, b2)
     m = _torch_gate_module(dim, w1, b1, w2, b2)
-    want = torch.softmax(m(_f64(x)), dim=-1).detach().numpy()
+    want = torch.softmax(m(_f64(x)), dim=-1).numpy()
     assert np.allclose(got, want, atol=1e-13)
     assert np.allclose(got.sum(-1), 1.0, atol=1e-14) and (got > 0).all()
     # adding a constant to every logit leaves the gates unchanged
@@ -496,7 +496,7 @@ def test_gates_match_torch_module(dim):
     assert np.allclose(shifted, got, atol=1e-13)
 
 
-def test_pooled_gates_match_blog_module_per_head():
+def test_pooled_gates_match_torch_per_head():
     B, T, H, dim = 2, 9, 3, 64
     w1, b1, w2, b2 = _rand_gate_weights(dim, 43)
     x = _bits(_rand_bf16((B, T, H, dim), 44))
@@ -504,7 +504,7 @@ def test_pooled_gates_match_blog_module_per_head():
     m = _torch_gate_module(dim, w1, b1, w2, b2)
     xf = _f64(x)
     for h in range(H):
-        want = torch.softmax(m(xf[:, :, h, :].mean(dim=1)), dim=-1).detach().numpy()  # the blog's forward, one head
+        want = torch.softmax(m(xf[:, :, h, :].mean(dim=1)), dim=-1).numpy()  # averaged over tokens, one head
         assert np.allclose(got[:, h], want, atol=1e-13), h
     # tokens that are all equal pool to the per-token gate
     same = np.repeat(x[:, :1], T, axis=1)
