@@ -182,3 +182,25 @@ def test_backward_validation():
     bad[6] = f + 128  # the forward's workspace must be 256-byte aligned
     assert nsa.nsa_backward(*bad, need, None) == nsa.NSA_ERR_INVALID_ARG
     assert nsa.nsa_backward_workspace_size(_p(head_dim=96)) == 0
+
+
+def test_gate_kernel_erf_constants_meet_their_published_bound():
+    """The gate kernel's erf follows Abramowitz & Stegun 7.1.26, |error| <= 1.5e-7. Read the
+    constants from the kernel source and evaluate the formula in float64 against math.erf,
+    so a mistyped digit fails here even where the gate tolerance would hide it."""
+    import math
+
+    src = open(os.path.join(ROOT, "sparse_attention_long_fwd_b200", "csrc", "gate.cuh")).read()
+    body = src[src.index("float erf_as7126(float x)"):]
+    body = body[: body.index("\n}\n")]
+    consts = [float(c) for c in re.findall(r"(-?\d+\.\d+)f", body) if float(c) != 1.0]
+    # in source order (the 1.0 literals aside): p, then the Horner coefficients a5 .. a1, then log2(e)
+    p, a5, a4, a3, a2, a1, log2e = consts
+    assert abs(log2e - 1 / math.log(2)) < 1e-12
+    worst = 0.0
+    for i in range(6001):
+        x = i * 1e-3
+        t = 1.0 / (1.0 + p * x)
+        poly = ((((a5 * t + a4) * t + a3) * t + a2) * t + a1) * t
+        worst = max(worst, abs(1.0 - poly * math.exp(-x * x) - math.erf(x)))
+    assert worst <= 1.5e-7, worst
