@@ -11,8 +11,10 @@ block scores, top-n, selected branch, window + gated combine). L2 is flushed (a
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
 
-Under torchrun each rank runs its own sequence on its own GPU (independent problems,
-no collective on the data path): value = all ranks' tokens / max-over-ranks time.
+With --gpus N > 1 and no launcher environment, the script starts N ranks itself
+(torch.distributed.run on 127.0.0.1); under torchrun WORLD_SIZE must equal N. Each rank
+runs its own sequence on its own GPU (independent problems, no collective on the data
+path): value = all ranks' tokens / max-over-ranks time.
 """
 from __future__ import annotations
 
@@ -39,14 +41,17 @@ from sparse_attention_long_fwd_b200.inputs import (WORKLOADS, decode_inputs, gat
 
 METRIC = "NSA prefill video tokens/s at 128K & TFLOP/s vs peak; decode HBM GB/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# B200 datasheet figures, reported beside the measured-peak fractions: dense bf16 tensor
+# throughput (the 2:4-sparse figure halved) and HBM3e bandwidth
+DATASHEET = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0}
 PREFILL_STAGES = ["pool", "cmp_attn_scores", "topn", "sel_bucket", "sel_tile", "win", "sel_merge_combine",
                   "dense_text"]
 # kernels of ours launched per prefill step: pool, compressed tile, top-n, bucket count / scan / scatter,
 # selected tiles, window tile, merge + gated combine (+ the dense text tile)
 PREFILL_KERNELS = 9
 # DRAM bytes per launch of a stage's kernel on the 128K workload, from one ncu capture of the
-# current kernel version (profiles/dram_traffic_v128k.md); an entry is removed when its kernel
-# changes, and the roofline then reports traffic null.
+# current kernel version (the full-size traffic summary kept with the profiles); an entry is
+# removed when its kernel changes, and the roofline then reports traffic null.
 STAGE_TRAFFIC_V128K = {"cmp_attn_scores": 4043696128}
 DECODE_STAGES = ["dec_cmp_and_window", "dec_select", "dec_selected_and_combine"]
 
@@ -211,19 +216,92 @@ def stage_times(stage_ev, names, nrec):
 
 # ---------------------------------------------------------------------------- arms
 
+def measure_prefill(w, q, k, v, g, args, world, peaks, peaks_src, flush, dev):
+    """Time one nsa_prefill per step on workload w (inputs resident, L2 flushed before every
+    step); returns the line's timing, stage times and the dominant stage's roofline."""
+    counts = prefill_counts(w)
+    p = nsa.make_params(w.n_tokens, w.n_video, w.hq, w.hkv, w.d, w.cmp_len, w.cmp_stride, w.sel_len, w.top_n,
+                        w.window, out_dtype=nsa.NSA_OUT_BF16)
+    ws = nsa.alloc_workspace(p, False, dev)
+    out = torch.empty((w.n_tokens, w.hq, w.d), dtype=torch.bfloat16, device=dev)
+    has_text = w.n_tokens > w.n_video
+    n_stages = (7 if w.n_video > 0 else 0) + (1 if has_text else 0)
+    stage_names = (PREFILL_STAGES[:7] if w.n_video > 0 else []) + (["dense_text"] if has_text else [])
+
+    def step(events):
+        nsa.nsa_profile_stages(events or [])
+        rc = nsa.nsa_prefill(q, k, v, g, p, out, None, ws, ws.numel())
+        if rc != nsa.NSA_OK:
+            raise nsa.NsaError(rc, "nsa_prefill")
+
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    step_ms, stage_ev = timed_steps(step, args.steps, args.warmup, flush, n_stages + 1)
+    clk = clocks.stop()
+    nsa.nsa_profile_stages([])
+    barrier(world)
+    assert nsa.nsa_get_device_error(clear=True) == 0, "device error word set during the benchmark"
+    ms_per_step = max_over_ranks(sum(step_ms), world) / args.steps
+    stages = stage_times(stage_ev, stage_names, n_stages)
+    flops = counts["cmp_flops"] + counts["sel_flops"] + counts["win_flops"] + counts["text_flops"]
+    tflops = flops / (sum(step_ms) / args.steps / 1e3) / 1e12
+    # the step lasts tens of milliseconds and the timed loop well under a second: the burst peak
+    peak_t, peak_name = peaks["bf16_tflops"], "bf16_tflops (burst: the step is short)"
+    dom = max(stages, key=stages.get)
+    stage_flops = {"cmp_attn_scores": counts["cmp_flops"], "sel_tile": counts["sel_flops"],
+                   "win": counts["win_flops"], "dense_text": counts["text_flops"]}
+    if dom in stage_flops:
+        ach = stage_flops[dom] / (stages[dom] / 1e3) / 1e12
+        traffic = STAGE_TRAFFIC_V128K.get(dom) if w.name == "v128k" else None
+        roofline = {"kernel": dom, "bound": "tensor", "achieved": round(ach, 2), "peak": peak_t, "unit": "TFLOP/s",
+                    "frac": round(ach / peak_t, 4), "traffic": traffic,
+                    "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one full-size launch"
+                    if traffic else None,
+                    "peak_source": f"{peaks_src} {peak_name}",
+                    "frac_of_datasheet": round(ach / DATASHEET["bf16_tflops"], 4),
+                    "datasheet_peak": DATASHEET["bf16_tflops"],
+                    "algorithmic": f"{stage_flops[dom]:.4e} FLOP per launch (attended keys only)"}
+    else:
+        roofline = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": None, "traffic": None}
+    del ws, out
+    return {"ms_per_step": ms_per_step, "stages": stages, "roofline": roofline, "clocks": clk, "counts": counts,
+            "tflops": tflops, "peak_t": peak_t, "n_kernels": PREFILL_KERNELS * (w.n_video > 0) + has_text}
+
+
+def run_config_lines(args, dev, peaks, peaks_src, flush, world, rank):
+    """The small prefill workloads, timed like the headline: the 2,048-token tiny case and
+    the 36K hybrid (its 256 trailing text rows run the dense stage)."""
+    lines = []
+    for name in ("tiny", "qwen36k_hybrid"):
+        w = WORKLOADS[name]
+        q, k, v, g = prefill_inputs(w, seed=10 + rank, device=dev)
+        m = measure_prefill(w, q, k, v, g, args, world, peaks, peaks_src, flush, dev)
+        lines.append({
+            "workload": name, "n_tokens": w.n_tokens, "n_video": w.n_video, "hq": w.hq, "hkv": w.hkv, "d": w.d,
+            "top_n": w.top_n, "window": w.window, "ms_per_step": round(m["ms_per_step"], 4),
+            "value": round(w.n_video * world / (m["ms_per_step"] / 1e3), 1), "unit": "video tokens/s",
+            "all_tokens_per_s": round(w.n_tokens * world / (m["ms_per_step"] / 1e3), 1),
+            "attended_tflops": round(m["tflops"], 2), "attended_frac_of_peak": round(m["tflops"] / m["peak_t"], 4),
+            "stages_ms": {kk: round(vv, 4) for kk, vv in m["stages"].items()}, "roofline": m["roofline"],
+            "launches": m["n_kernels"] * args.steps})
+        del q, k, v, g
+    return lines
+
+
 def run_b200(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks, peaks_src = load_peaks()
     w = WORKLOADS[args.workload]
-    counts = prefill_counts(w)
     q, k, v, g = prefill_inputs(w, seed=2 + rank, device=dev)
     p = nsa.make_params(w.n_tokens, w.n_video, w.hq, w.hkv, w.d, w.cmp_len, w.cmp_stride, w.sel_len, w.top_n,
                         w.window, out_dtype=nsa.NSA_OUT_BF16)
     ws = nsa.alloc_workspace(p, False, dev)
     out = torch.empty((w.n_tokens, w.hq, w.d), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    n_stages = 7 + (1 if w.n_tokens > w.n_video else 0)
     n_kernels = PREFILL_KERNELS + (1 if w.n_tokens > w.n_video else 0)
 
     def step(events):
@@ -232,40 +310,11 @@ def run_b200(args, world, rank, local):
         if rc != nsa.NSA_OK:
             raise nsa.NsaError(rc, "nsa_prefill")
 
-    clocks = ClockSampler(local)
-    barrier(world)
-    torch.cuda.synchronize()
-    clocks.start()
-    step_ms, stage_ev = timed_steps(step, args.steps, args.warmup, flush, n_stages + 1)
-    clk = clocks.stop()
-    nsa.nsa_profile_stages([])
-    barrier(world)
-    assert nsa.nsa_get_device_error(clear=True) == 0, "device error word set during the benchmark"
-    total_ms = max_over_ranks(sum(step_ms), world)
-    ms_per_step = total_ms / args.steps
+    m = measure_prefill(w, q, k, v, g, args, world, peaks, peaks_src, flush, dev)
+    ms_per_step, stages, counts, peak_t = m["ms_per_step"], m["stages"], m["counts"], m["peak_t"]
     tokens = w.n_video * world
     value = dist_helpers.aggregate_rate(w.n_video, world, ms_per_step / 1e3)
-    stages = stage_times(stage_ev, PREFILL_STAGES, n_stages)
-    flops = counts["cmp_flops"] + counts["sel_flops"] + counts["win_flops"] + counts["text_flops"]
-    tflops = flops / (sum(step_ms) / args.steps / 1e3) / 1e12
-
-    # dominant kernel and its roofline (live CUDA-event durations of this run)
-    dom = max(stages, key=stages.get)
-    stage_flops = {"cmp_attn_scores": counts["cmp_flops"], "sel_tile": counts["sel_flops"],
-                   "win": counts["win_flops"], "dense_text": counts["text_flops"]}
-    peak_t = peaks["bf16_tflops_sustained"]
-    if dom in stage_flops:
-        ach = stage_flops[dom] / (stages[dom] / 1e3) / 1e12
-        traffic = STAGE_TRAFFIC_V128K.get(dom) if w.name == "v128k" else None
-        roofline = {"kernel": dom, "bound": "tensor", "achieved": round(ach, 2), "peak": peak_t, "unit": "TFLOP/s",
-                    "frac": round(ach / peak_t, 4), "traffic": traffic,
-                    "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one full-size launch"
-                    if traffic else None,
-                    "peak_source": f"{peaks_src} bf16_tflops_sustained (kernel timed inside a long step loop)",
-                    "algorithmic": f"{stage_flops[dom]:.4e} FLOP per launch (attended keys only)"}
-    else:
-        roofline = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": None, "traffic": None}
+    tflops = m["tflops"]
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "video tokens/s", "n_gpus": world, "steps": args.steps,
@@ -278,10 +327,11 @@ def run_b200(args, world, rank, local):
                    "l2": "flushed (256 MiB write) before every timed step; inputs also exceed L2",
                    "parallelism": f"independent sequence per rank x{world}"},
         "attended_tflops": round(tflops, 2), "attended_frac_of_peak": round(tflops / peak_t, 4),
+        "attended_frac_of_datasheet": round(tflops / DATASHEET["bf16_tflops"], 4),
         "attended_keys_per_head": counts["keys_per_head"],
         "attended_fraction_of_dense_pairs": round(sum(counts["keys_per_head"].values()) / counts["dense_causal_pairs"], 4),
         "stages_ms": {kk: round(vv, 4) for kk, vv in stages.items()},
-        "roofline": roofline, "clocks": clk, "gpu_launches": n_kernels * args.steps,
+        "roofline": m["roofline"], "clocks": m["clocks"], "gpu_launches": n_kernels * args.steps,
     }
 
     # end to end through the public call: pinned host inputs in, bf16 output back, every step.
@@ -360,6 +410,10 @@ def run_b200(args, world, rank, local):
     if not args.no_sweep and w.name == "v128k":
         result["sweep"] = run_sweep(args, dev, q, k, v, g, flush, peak_t, world)
         result["gpu_launches"] += PREFILL_KERNELS * args.steps * len(result["sweep"]["points"])
+
+    if not args.no_configs:
+        result["configs"] = run_config_lines(args, dev, peaks, peaks_src, flush, world, rank)
+        result["gpu_launches"] += sum(c["launches"] for c in result["configs"])
 
     if not args.no_decode:
         result["decode"] = run_decode(args, dev, peaks, peaks_src, flush, world)
@@ -523,6 +577,7 @@ def run_backward(args, dev, q, k, v, g, peaks, flush, world):
     # QK^T, dO V^T, P^T dO, dS K and dS^T Q against the forward's QK^T and PV: 2.5x its FLOPs
     flops = 2.5 * (c["cmp_flops"] + c["sel_flops"] + c["win_flops"] + c["text_flops"])
     tf = flops / (ms / 1e3) / 1e12
+    # the timed loop runs for seconds at 360 ms a step: the sustained peak
     peak = peaks["bf16_tflops_sustained"]
     del bws, dq, dk, dv, dgates, d_out, ws
     return {"workload": "v128k backward: dq, dk, dv and the gates' gradient of the headline prefill "
@@ -531,6 +586,8 @@ def run_backward(args, dev, q, k, v, g, peaks, flush, world):
             "unit": "video tokens/s", "steps": args.steps, "warmup": args.warmup,
             "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(tf / peak, 4),
+                         "peak_source": "measured bf16_tflops_sustained (a seconds-long timed loop)",
+                         "frac_of_datasheet": round(tf / DATASHEET["bf16_tflops"], 4),
                          "algorithmic": f"{flops:.4e} FLOP per step (2.5x the forward's attended FLOPs)"},
             "launches": BACKWARD_KERNELS * args.steps}
 
@@ -571,6 +628,7 @@ def run_decode(args, dev, peaks, peaks_src, flush, world):
     return {"workload": "decode64x128k: 64 sequences x 131,072-token bf16 cache, Hq=28, Hkv=4, d=128, n=16, w=512",
             "ms_per_step": round(ms, 4), "hbm_gbs": round(gbs * world, 1), "unit": "GB/s",
             "algorithmic_bytes_per_step": nbytes, "frac_of_peak": round(gbs / peaks["hbm_gbs"], 4),
+            "frac_of_datasheet": round(gbs / DATASHEET["hbm_gbs"], 4), "datasheet_gbs": DATASHEET["hbm_gbs"],
             "peak_gbs": peaks["hbm_gbs"], "peak_source": f"{peaks_src} hbm_gbs",
             "steps": steps, "stages_ms": {kk: round(vv, 4) for kk, vv in stages.items()},
             "dec_cmp_roofline": {"bound": "hbm", "achieved": round(cmp_gbs, 1), "peak": peaks["hbm_gbs"],
@@ -652,6 +710,19 @@ def run_reference(args, world, rank):
     }
 
 
+def relaunch_ranks(n: int) -> int:
+    """Run this command again as n ranks on this node (torch.distributed.run, rendezvous on
+    127.0.0.1); rank 0 prints the JSON line. Returns the launcher's exit status."""
+    import socket
+
+    with socket.socket() as sck:
+        sck.bind(("127.0.0.1", 0))
+        port = sck.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -663,13 +734,19 @@ def main():
     ap.add_argument("--no-sweep", action="store_true", help="skip the 128K (n, w) budget sweep")
     ap.add_argument("--no-gates", action="store_true", help="skip the gate-network and learnable-compression lines")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward measurement")
+    ap.add_argument("--no-configs", action="store_true", help="skip the tiny and 36K-hybrid prefill lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "b200":
         ap.error("--warmup must be >= 3")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # one process per GPU: start the ranks here when no launcher did
+        sys.exit(relaunch_ranks(args.gpus))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} does not match the launcher's WORLD_SIZE={world}")
     if args.impl == "reference":
         res = run_reference(args, world, rank)
         if res is not None:

@@ -142,7 +142,9 @@ int nsa_decode(const void* q, const void* kcache, const void* vcache, const void
  * until the process exits.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call before any
- *     stream capture on the device.
+ *     stream capture on the device. The address is kept for the life of the process: do
+ *     not call nsa_decode_noalloc on a device after cudaDeviceReset (or any other reset of
+ *     its primary context) in the same process, since the array then moves.
  *   - A problem whose scratch (nsa_workspace_size(params, 1)) exceeds the array returns
  *     NSA_ERR_NOALLOC_TOO_LARGE before anything is enqueued; use nsa_decode for it.
  *   - All calls share the one array and it keeps the last call's contents; no kernel reads
@@ -278,6 +280,18 @@ const char* nsa_error_string(int status);
 int nsa_get_device_error(uint32_t* word, int clear);
 
 /*
+ * Self-test of failure detection. Every wait inside this library's kernels is bounded; a
+ * wait that runs out records bit 0 of the device error word and its kernel returns early
+ * instead of hanging. This entry point exercises exactly that path without any fault: it
+ * launches one warp that waits, through the library's bounded wait, on a barrier nothing
+ * ever arrives at, with a budget of `limit_cycles` GPU clock cycles (1 .. 4e9; e.g. 2e6 is
+ * about 1 ms). After the stream drains, nsa_get_device_error reports bit 0 set; the
+ * context stays usable. Returns NSA_OK, NSA_ERR_INVALID_ARG (limit out of range),
+ * NSA_ERR_UNSUPPORTED (not sm_100) or NSA_ERR_CUDA.
+ */
+int nsa_selftest_wait_timeout(int64_t limit_cycles, void* stream);
+
+/*
  * Stage timing (diagnostics). After nsa_profile_stages(events, count) with count > 0,
  * every nsa_prefill / nsa_decode call records events[i] (cudaEvent_t handles owned by
  * the caller) on its stream at its stage boundaries: events[0] before the first kernel,
@@ -286,7 +300,8 @@ int nsa_get_device_error(uint32_t* word, int clear);
  * decode: compressed split, select, branches + gated combine). Stages that do not run
  * record nothing; events beyond `count` are not recorded. count = 0 (or events = NULL)
  * switches recording off. The
- * registration is process-wide and not thread-safe. Returns NSA_OK or NSA_ERR_INVALID_ARG.
+ * registration belongs to the calling host thread: it applies to the calls that thread
+ * makes, and other threads' calls record nothing. Returns NSA_OK or NSA_ERR_INVALID_ARG.
  */
 int nsa_profile_stages(void* const* events, int count);
 

@@ -21,6 +21,27 @@
 #include "gate.cuh"
 #include "backward.cuh"
 
+namespace nsa {
+
+// Self-test of the failure-detection path: one warp waits, through the same bounded wait
+// every kernel of the library uses, on an mbarrier that nothing ever arrives at. The wait
+// gives up after `limit` clock cycles, sets the timeout bit of the device error word and
+// the kernel returns normally, leaving the context usable.
+__global__ void __launch_bounds__(32) bounded_wait_selftest_kernel(long long limit) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // phase 0 never completes: no thread arrives and no copy is counted on the barrier
+  (void)mbar_wait(&bar, 0, &abort_flag, limit);
+}
+
+}  // namespace nsa
+
 namespace {
 
 using nsa::AttnArgs;
@@ -162,10 +183,11 @@ bool debug_sync() {
 }
 
 // Caller-registered stage events (nsa_profile_stages); g_stage_next counts the events
-// recorded by the current call.
-void* const* g_stage_events = nullptr;
-int g_stage_count = 0;
-int g_stage_next = 0;
+// recorded by the current call. Per host thread: a registration made on one thread never
+// records events for calls made on another.
+thread_local void* const* g_stage_events = nullptr;
+thread_local int g_stage_count = 0;
+thread_local int g_stage_next = 0;
 
 void stage_begin(cudaStream_t st) {
   g_stage_next = 0;
@@ -675,7 +697,9 @@ int nsa_decode(const void* q, const void* kcache, const void* vcache, const void
 // workspace. Every GPU that loads the library holds the array until the process exits.
 // Host code must not pass the symbol itself to a kernel: on the host it is only a
 // stand-in, so the device address is looked up with cudaGetSymbolAddress, once per
-// device, with that device current.
+// device, with that device current. The cached address is valid for as long as the
+// device's primary context lives; a reset of that context (cudaDeviceReset) moves the array,
+// and the header forbids calls after one.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[NSA_NOALLOC_SCRATCH_BYTES];
 
 static int noalloc_scratch_address(void** out) {
@@ -1064,6 +1088,14 @@ int nsa_profile_stages(void* const* events, int count) {
   g_stage_count = count > 0 ? count : 0;
   g_stage_next = 0;
   return NSA_OK;
+}
+
+int nsa_selftest_wait_timeout(int64_t limit_cycles, void* stream) {
+  if (limit_cycles < 1 || limit_cycles > nsa::kWaitCycles) return NSA_ERR_INVALID_ARG;
+  int rc = check_device();
+  if (rc != NSA_OK) return rc;
+  nsa::bounded_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_cycles);
+  return launch_status("bounded_wait_selftest", static_cast<cudaStream_t>(stream), false);
 }
 
 int nsa_get_device_error(uint32_t* word, int clear) {

@@ -87,14 +87,16 @@ __device__ __forceinline__ bool mbar_test_suspend(uint64_t* bar, uint32_t parity
   return ok != 0;
 }
 // Bounded wait for the phase with the given parity. `abort_flag` (shared) lets one
-// role that timed out release every other waiter promptly.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+// role that timed out release every other waiter promptly. `limit` is the wait's budget in
+// clock cycles (the kernels use kWaitCycles; the self-test of this path passes a short one).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          long long limit = kWaitCycles) {
   if (mbar_test(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_test_suspend(bar, parity, 20000)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       *abort_flag = 1;
       record_error(kErrWaitTimeout);
       return false;

@@ -31,7 +31,7 @@ EXPORTED = (
     "nsa_error_string", "nsa_get_device_error", "nsa_version", "nsa_profile_stages", "nsa_decode_noalloc",
     "nsa_prefill_varlen", "nsa_prefill_varlen_workspace_size", "nsa_compress_weighted", "nsa_prefill_phi",
     "nsa_gate_mlp", "nsa_gate_mlp_pooled", "nsa_gate_mlp_pooled_workspace_size", "nsa_backward",
-    "nsa_backward_workspace_size",
+    "nsa_backward_workspace_size", "nsa_selftest_wait_timeout",
 )
 
 
@@ -115,6 +115,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.nsa_version.restype = ctypes.c_char_p
     lib.nsa_profile_stages.argtypes = [ctypes.POINTER(ctypes.c_void_p), I]
     lib.nsa_profile_stages.restype = I
+    lib.nsa_selftest_wait_timeout.argtypes = [ctypes.c_int64, P]
+    lib.nsa_selftest_wait_timeout.restype = I
     _lib = lib
     return lib
 
@@ -254,6 +256,12 @@ def nsa_get_device_error(clear: bool = True) -> int:
     if rc != NSA_OK:
         raise NsaError(rc, "nsa_get_device_error")
     return int(w.value)
+
+
+def nsa_selftest_wait_timeout(limit_cycles: int, stream=None) -> int:
+    """Launch the failure-detection self-test: a bounded wait on a barrier nothing arrives
+    at, which must give up after limit_cycles and set bit 0 of the device error word."""
+    return load_library().nsa_selftest_wait_timeout(int(limit_cycles), _stream(stream))
 
 
 def nsa_version() -> str:

@@ -204,3 +204,10 @@ def test_gate_kernel_erf_constants_meet_their_published_bound():
         poly = ((((a5 * t + a4) * t + a3) * t + a2) * t + a1) * t
         worst = max(worst, abs(1.0 - poly * math.exp(-x * x) - math.erf(x)))
     assert worst <= 1.5e-7, worst
+
+
+def test_selftest_budget_validated_before_any_launch():
+    # limits outside 1 .. 4e9 cycles are rejected on the host, before the device is touched
+    assert nsa.nsa_selftest_wait_timeout(0) == nsa.NSA_ERR_INVALID_ARG
+    assert nsa.nsa_selftest_wait_timeout(-5) == nsa.NSA_ERR_INVALID_ARG
+    assert nsa.nsa_selftest_wait_timeout(4_000_000_001) == nsa.NSA_ERR_INVALID_ARG

@@ -21,3 +21,24 @@ def test_reference_arm_prints_one_contract_line():
     assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_gpus_flag_starts_its_own_ranks():
+    """--gpus 2 without a launcher starts two ranks itself (rendezvous on 127.0.0.1); the
+    reference arm's rank 0 prints the one JSON line with n_gpus = 2, rank 1 exits quietly."""
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                          "--steps", "1", "--warmup", "1", "--gpus", "2"], capture_output=True, text=True, check=True,
+                         cwd=ROOT, timeout=600, env=env).stdout
+    lines = [ln for ln in out.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, out
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2
+
+
+def test_gpus_flag_must_match_the_launcher():
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                        "--steps", "1", "--warmup", "1", "--gpus", "2"], capture_output=True, text=True, cwd=ROOT,
+                       timeout=600, env=env)
+    assert r.returncode != 0 and "does not match" in r.stderr

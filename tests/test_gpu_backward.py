@@ -66,6 +66,8 @@ def _compare(w, q, k, v, g, d_out, sel, grads, phi=None):
     ("qwen36k_hybrid", 1200, 1000, 28, 4, 128, 16, 512),  # trailing text rows (dense branch)
     ("v128k", 300, 0, 4, 2, 64, 4, 64),               # all text
     ("v128k", 40, 40, 4, 2, 128, 3, 16),              # shorter than two compression blocks
+    ("v128k", 600, 600, 48, 4, 128, 16, 256),         # G = 12: one token per warp in the row pass
+    ("qwen36k_hybrid", 520, 450, 32, 2, 64, 12, 128),  # G = 16, d = 64, with text rows
 ])
 @pytest.mark.parametrize("saved", [False, True])
 def test_backward_every_element(name, n, nv, hq, hkv, d, top_n, window, saved):

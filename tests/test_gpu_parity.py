@@ -58,6 +58,9 @@ def test_prefill_tiny_all_rows():
     (777, 8, 1, 64, 5, 100),         # G = 8, d = 64, tiny window
     (1500, 16, 16, 128, 4, 300),     # G = 1 (no GQA)
     (640, 12, 3, 128, 64, 2048),     # top_n and window cover everything: dense special case
+    (1100, 48, 4, 128, 16, 512),     # G = 12: 16-lane head groups (4 padding heads), 10-token tiles
+    (900, 32, 2, 128, 12, 256),      # G = 16: 8-token tiles, every lane a real head
+    (700, 24, 2, 64, 8, 200),        # G = 12 with d = 64
 ])
 def test_prefill_shapes_all_rows(n, hq, hkv, d, top_n, window):
     w = scaled(WORKLOADS["v128k"], n_tokens=n, n_video=n, hq=hq, hkv=hkv, d=d, top_n=top_n, window=window)
@@ -183,6 +186,19 @@ def test_decode_small_varied_lengths():
 def test_decode_d64_window_covers_all():
     w = scaled(WORKLOADS["decode64x128k"], batch=4, n_tokens=700, hq=8, hkv=2, d=64, top_n=12, window=1024)
     print(_decode_case(w, seed=22, seq_lens=[700, 350, 64, 129]))
+
+
+def test_decode_top_n_48_shared_memory_selection():
+    """top_n > 32 takes the shared-memory warp selection in decode."""
+    w = scaled(WORKLOADS["decode64x128k"], batch=6, n_tokens=9000, top_n=48, window=512)
+    print(_decode_case(w, seed=23, seq_lens=[9000, 8999, 4000, 3100, 2047, 1]))
+
+
+@pytest.mark.parametrize("hq,hkv,d", [(48, 4, 128), (32, 2, 64)])
+def test_decode_large_groups(hq, hkv, d):
+    """G = 12 and G = 16 query heads per group in the decode tiles."""
+    w = scaled(WORKLOADS["decode64x128k"], batch=5, n_tokens=5000, hq=hq, hkv=hkv, d=d, top_n=16, window=512)
+    print(_decode_case(w, seed=24, seq_lens=[5000, 4097, 1000, 65, 30]))
 
 
 def test_decode_64x128k_sampled():
