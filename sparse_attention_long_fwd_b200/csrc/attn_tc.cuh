@@ -562,38 +562,45 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
         // slice; rows without keys (head padding, past the end) follow the others, their
         // probabilities being forced to 0 through lse2 = +inf
         const bool full = __all_sync(0xffffffffu, !row_valid || (kbase >= rb && kbase + kColsPerWG <= re));
-        // 32 columns at a time (an online max across the chunks keeps one chunk in registers)
+        // the slice's columns are loaded with one wait, and S is released at once; then 32
+        // columns at a time (an online max across the chunks)
         static_assert(kColsPerWG % 32 == 0, "phase 1 reads 32-column chunks");
+        float s_all[kColsPerWG];
+        __syncwarp();
 #pragma unroll
-        for (int hc = 0; hc < kColsPerWG / 32; ++hc) {
-          float s[32];
-          __syncwarp();
-          tmem_ld32(trow + b * kBN + col0 + 32 * hc, s);
-          tmem_wait_ld();
-          if (hc == kColsPerWG / 32 - 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.s_free[b]);  // S is in registers: the buffer may be reused
-          }
-          if (!full) {
+        for (int hc = 0; hc < kColsPerWG / 32; ++hc)
+          tmem_ld32(trow + b * kBN + col0 + 32 * hc, *reinterpret_cast<float(*)[32]>(&s_all[32 * hc]));
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.s_free[b]);  // S is in registers: the buffer may be reused
+        if (!full) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int kidx = kbase + 32 * hc + i;
-              s[i] = (kidx >= rb && kidx < re) ? s[i] : -INFINITY;
-            }
+          for (int i = 0; i < kColsPerWG; ++i) {
+            const int kidx = kbase + i;
+            s_all[i] = (kidx >= rb && kidx < re) ? s_all[i] : -INFINITY;
           }
-          float mx[8];
+        }
+        // one max over the whole slice (eight independent chains), then one rescale of the sum
+        float mx[8];
 #pragma unroll
-          for (int c = 0; c < 8; ++c) mx[c] = fmax3f(fmaxf(s[c], s[c + 8]), s[c + 16], s[c + 24]);
-          const float cmax = fmax3f(fmax3f(mx[0], mx[1], mx[2]), fmax3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-          const float mnew = fmaxf(m, cmax);
-          if (MODE != kModeCmp) {
-            m = mnew;  // the window and dense branches need only the row max here
-          } else if (mnew != -INFINITY) {
-            const float ms = mnew * sl2;
-            lsum = lsum * ex2_approx((m - mnew) * sl2) + chunk_sum_ex2(s, sl2, ms);
-            m = mnew;
-          }
+        for (int c = 0; c < 8; ++c) mx[c] = fmaxf(s_all[c], s_all[c + 8]);
+#pragma unroll
+        for (int c = 16; c < kColsPerWG; c += 16)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) mx[u] = fmax3f(mx[u], s_all[c + u], s_all[c + 8 + u]);
+        const float cmax = fmax3f(fmax3f(mx[0], mx[1], mx[2]), fmax3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+        const float mnew = fmaxf(m, cmax);
+        if (MODE != kModeCmp) {
+          m = mnew;  // the window and dense branches need only the row max here
+        } else if (mnew != -INFINITY) {
+          const float ms = mnew * sl2;
+          float part = 0.f;
+#pragma unroll
+          for (int hc = 0; hc < kColsPerWG / 32; ++hc)
+            part += chunk_sum_ex2(*reinterpret_cast<float(*)[32]>(&s_all[32 * hc]), sl2, ms);
+          lsum = lsum * ex2_approx((m - mnew) * sl2) + part;
+          m = mnew;
         }
       }
       sm.lse_x[wg][r][0] = (m == -INFINITY) ? -INFINITY : m * sl2;
@@ -651,19 +658,33 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
         static_assert(kColsPerWG % 32 == 0, "P is stored 16 columns (32 keys) at a time");
         uint32_t pk[kColsPerWG / 2];
         float prev_last = 0.f;  // (kModeCmp) p of the previous chunk's last column
+        // window / dense: the slice's columns with one wait, S released at once. Compressed:
+        // chunk by chunk (its P and block scores leave no registers for a second chunk)
+        float s2_all[kColsPerWG];
+        uint32_t xv = 0;
+        auto release_s = [&]() {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.s_free[b]);  // S is in registers: the buffer may be reused
+        };
+        if constexpr (MODE != kModeCmp) {
+          __syncwarp();
+#pragma unroll
+          for (int hc = 0; hc < kColsPerWG / 32; ++hc)
+            tmem_ld32(trow + b * kBN + col0 + 32 * hc, *reinterpret_cast<float(*)[32]>(&s2_all[32 * hc]));
+          tmem_wait_ld();
+          release_s();
+        }
 #pragma unroll
         for (int hc = 0; hc < kColsPerWG / 32; ++hc) {
-          float sc[32];
-          uint32_t xv = 0;
-          __syncwarp();
-          tmem_ld32(trow + b * kBN + col0 + 32 * hc, sc);
-          if (MODE == kModeCmp && hc == 0 && half > 0)
-            asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(xv) : "r"(trow + b * kBN + col0 - 1));
-          tmem_wait_ld();
-          if (hc == kColsPerWG / 32 - 1) {
-            tc_fence_before();
+          float(&sc)[32] = *reinterpret_cast<float(*)[32]>(&s2_all[32 * hc]);
+          if constexpr (MODE == kModeCmp) {
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.s_free[b]);  // S is in registers: the buffer may be reused
+            tmem_ld32(trow + b * kBN + col0 + 32 * hc, sc);
+            if (hc == 0 && half > 0)
+              asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(xv) : "r"(trow + b * kBN + col0 - 1));
+            tmem_wait_ld();
+            if (hc == kColsPerWG / 32 - 1) release_s();
           }
           if (MODE == kModeCmp && hc == 0 && half > 0) {
             const int xk = kb + kt2 * kBN + col0 - 1;

@@ -83,6 +83,19 @@ def test_prefill_edge_lengths():
     _prefill_case(w, seed=7)
 
 
+def test_prefill_g16_9k_sampled():
+    """G = 16 (every lane of a 16-lane head group a real head) at 9,000 tokens: many
+    compressed key tiles and selected buckets of mixed sizes; the first rows, rows around
+    4K and 8K, the last row and random rows, every intermediate."""
+    w = scaled(WORKLOADS["v128k"], n_tokens=9000, n_video=9000, hq=32, hkv=2, d=128, top_n=16, window=512)
+    q, k, v, g = prefill_inputs(w, seed=31, device=DEV)
+    out, sel, ws, lay = run_prefill(w, q, k, v, g)
+    rows = set(range(0, 70)) | {4094, 4095, 4096, 4097, 8190, 8191, 8192, 8193, 8999}
+    rows |= set(int(x) for x in np.random.default_rng(31).integers(0, 9000, 60))
+    st = compare_prefill_rows(w, q, k, v, g, np.array(sorted(rows), dtype=np.int32), out, sel, ws, lay)
+    print(st)
+
+
 def test_prefill_bf16_output():
     w = scaled(WORKLOADS["qwen36k_hybrid"], n_tokens=900, n_video=800)
     _prefill_case(w, seed=9, out_dtype=torch.bfloat16)
