@@ -631,3 +631,102 @@ def test_backward_value_gradient_sums_to_gated_output_gradient():
         hs = slice(grp * G, (grp + 1) * G)
         want = (w[:, hs, None] * do[:, hs]).sum(axis=(0, 1))
         assert np.allclose(r["dv"][:, grp].sum(0), want, atol=1e-10)
+
+
+# ---------------------------------------------------------------- packed batches, interleaved segments
+
+from oracle import packed as pk_orc  # noqa: E402
+
+
+def _packed_case(seqs, hq=4, hkv=2, d=16, seed=71, **kw):
+    """seqs: per sequence a list of (length, is_video) segments."""
+    lens = [sum(n for n, _ in s) for s in seqs]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    seg_lens = [n for s in seqs for n, _ in s]
+    seg_vid = [vid for s in seqs for _, vid in s]
+    N = int(cu[-1])
+    cfg, q, k, v, g = _case(N, hq, hkv, d, seed, **kw)
+    return cfg, _bits(q), _bits(k), _bits(v), g.numpy(), cu, seg_lens, seg_vid
+
+
+def test_packed_trailing_text_equals_the_single_sequence_hybrid():
+    """[video][text] in one sequence is the hybrid layout prefill_rows already computes."""
+    cfg, q, k, v, g, cu, sl, sv = _packed_case([[(190, True), (70, False)]], top_n=4, window=40)
+    o = pk_orc.packed_prefill(cfg, q, k, v, g, cu, sl, sv)
+    from dataclasses import replace
+    ref = orc.prefill_rows(replace(cfg, n_tokens=260, n_video=190), q, k, v, g, np.arange(260))
+    assert np.allclose(o["out"], ref["out"], atol=1e-12, rtol=0)
+    assert np.array_equal(o["sel"], ref["sel"][:190])
+
+
+def test_packed_text_rows_are_dense_over_every_earlier_token():
+    """Text rows between and after video segments attend densely to all earlier tokens of
+    their own sequence (numpy fp64 softmax, independent of the oracle's C code)."""
+    seqs = [[(70, True), (20, False), (90, True), (15, False)], [(40, False), (64, True), (9, False)]]
+    cfg, q, k, v, g, cu, sl, sv = _packed_case(seqs, top_n=3, window=32, seed=72)
+    o = pk_orc.packed_prefill(cfg, q, k, v, g, cu, sl, sv)
+    qd, kd, vd = (orc.bf16_bits_to_f64(x) for x in (q, k, v))
+    G = cfg.hq // cfg.hkv
+    per = pk_orc.segments_of(cu, sl, sv)
+    for b, segs in enumerate(per):
+        s0 = int(cu[b])
+        for t in pk_orc.text_positions(segs):
+            for h in range(cfg.hq):
+                z = kd[s0: t + 1, h // G] @ qd[t, h] / math.sqrt(cfg.d)
+                p = np.exp(z - z.max())
+                ref = (p / p.sum()) @ vd[s0: t + 1, h // G]
+                assert np.allclose(o["out"][t, h], ref, atol=1e-12, rtol=0), (b, t, h)
+
+
+def test_packed_video_rows_ignore_text_segments():
+    """Taking the text segments out of a sequence leaves every video row unchanged: video
+    positions count in the video stream."""
+    seqs = [[(100, True), (30, False), (80, True), (11, False), (50, True)]]
+    cfg, q, k, v, g, cu, sl, sv = _packed_case(seqs, top_n=4, window=48, seed=73)
+    o = pk_orc.packed_prefill(cfg, q, k, v, g, cu, sl, sv)
+    vp = o["video_rows"]
+    o2 = pk_orc.packed_prefill(cfg, q[vp], k[vp], v[vp], g[vp], [0, len(vp)], [len(vp)], [True])
+    assert np.array_equal(o["out"][vp], o2["out"])
+    assert np.array_equal(o["sel"], o2["sel"])
+
+
+def test_packed_full_budget_video_rows_are_dense_over_the_video_stream():
+    """With every block selected and a window covering the stream, the selected and window
+    branches of a video row are dense causal attention over the earlier video tokens only
+    (torch SDPA on the video tokens alone); text tokens between them are invisible."""
+    seqs = [[(80, True), (25, False), (60, True), (7, False), (33, True)]]
+    nv = 173
+    lens = [n for n, _ in seqs[0]]
+    N = sum(lens)
+    cfg, q, k, v, _, cu, sl, sv = _packed_case(seqs, top_n=orc.num_sel(nv, 64) + 1, window=nv + 3, seed=74)
+    for which in (1, 2):
+        g = np.zeros((N, cfg.hq, 3), dtype=np.float32)
+        g[..., which] = 1.0
+        o = pk_orc.packed_prefill(cfg, q, k, v, g, cu, sl, sv)
+        vp = o["video_rows"]
+        ref = _sdpa_causal(_f64(q[vp]), _f64(k[vp]), _f64(v[vp]), 1 / math.sqrt(cfg.d)).numpy()
+        assert np.allclose(o["out"][vp], ref, atol=1e-12, rtol=0)
+
+
+def test_packed_sequences_are_independent():
+    """A packed batch equals its sequences evaluated one at a time (positions restart)."""
+    seqs = [[(120, True), (10, False)], [(33, True)], [(12, False), (70, True), (5, False), (40, True)]]
+    cfg, q, k, v, g, cu, sl, sv = _packed_case(seqs, top_n=5, window=60, seed=75)
+    o = pk_orc.packed_prefill(cfg, q, k, v, g, cu, sl, sv)
+    si = 0
+    sels = []
+    for b, segs in enumerate(seqs):
+        s0, s1 = int(cu[b]), int(cu[b + 1])
+        n = len(segs)
+        ob = pk_orc.packed_prefill(cfg, q[s0:s1], k[s0:s1], v[s0:s1], g[s0:s1], [0, s1 - s0], sl[si: si + n],
+                                   sv[si: si + n])
+        assert np.array_equal(o["out"][s0:s1], ob["out"])
+        sels.append(ob["sel"])
+        si += n
+    assert np.array_equal(o["sel"], np.concatenate(sels))
+
+
+def test_packed_rejects_segments_that_cross_sequences():
+    cfg, q, k, v, g, cu, sl, sv = _packed_case([[(50, True)], [(30, False)]])
+    with pytest.raises(ValueError):
+        pk_orc.packed_prefill(cfg, q, k, v, g, cu, [60, 20], [True, False])
