@@ -257,7 +257,8 @@ size_t nsa_workspace_size(const nsa_params_t* params, int is_decode);
  * inspection after the stream has been synchronised. Every field is an offset from the
  * workspace base; layouts are row-major:
  *   kc, vc   [Ncmp(N_v)][Hkv][d] bf16     o_cmp [N_v][Hq][d] fp16     lse [N_v][Hq] fp32 (natural log)
- *   scores   [N_v][Hkv][Nsel] fp32, Nsel = ceil(N_v / l'); only entries j <= t/l' are written
+ *   scores   [N_v][Hkv][score_stride] fp32: block j of row (t, g) at j, Nsel = ceil(N_v / l')
+ *            blocks (score_stride = Nsel rounded up to a multiple of 4); only j <= t/l' is written
  *   sel_idx  [N_v][Hkv][top_n] int32      o_win [N_v][Hq][d] fp16 (window branch)
  * The selected branch's output goes straight into the gated combine and is not kept.
  * Returns NSA_OK or NSA_ERR_INVALID_ARG.
@@ -265,6 +266,7 @@ size_t nsa_workspace_size(const nsa_params_t* params, int is_decode);
 typedef struct {
   size_t kc, vc, o_cmp, lse, scores, sel_idx, o_win, total;
   int32_t n_cmp, n_sel;
+  int32_t score_stride;  /* floats between consecutive (t, g) score rows */
 } nsa_prefill_layout_t;
 int nsa_prefill_workspace_layout(const nsa_params_t* params, nsa_prefill_layout_t* layout);
 

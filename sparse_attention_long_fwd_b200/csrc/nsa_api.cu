@@ -102,6 +102,7 @@ struct PrefillLayout {
   size_t sel_cnt, sel_eoff, sel_toff, sel_list, sel_row, part_o, part_ml;
   long long part_rows;  // 128 x the bound on selected-branch tiles
   int ncmp, nsel;
+  int score_stride;     // floats per score row: nsel rounded up to 4, so rows are 16-byte aligned
 };
 
 PrefillLayout prefill_layout(const nsa_params_t* p) {
@@ -120,7 +121,8 @@ PrefillLayout prefill_layout(const nsa_params_t* p) {
   L.vc = take(cmp_rows * hkv * d * 2);
   L.o_cmp = take(static_cast<size_t>(nv) * hq * d * 2);
   L.lse = take(static_cast<size_t>(nv) * hq * 4);
-  L.scores = take(static_cast<size_t>(nv) * hkv * (L.nsel > 0 ? L.nsel : 1) * 4);
+  L.score_stride = (L.nsel + 3) / 4 * 4;
+  L.scores = take(static_cast<size_t>(nv) * hkv * (L.score_stride > 0 ? L.score_stride : 4) * 4);
   L.sel_idx = take(static_cast<size_t>(nv) * hkv * p->top_n * 4);
   L.o_win = take(static_cast<size_t>(nv) * hq * d * 2);
   const size_t buckets = static_cast<size_t>(hkv) * (L.nsel > 0 ? L.nsel : 1);
@@ -293,7 +295,7 @@ int prefill_impl(const nsa_params_t* p, const void* q, const void* k, const void
   a.cmp_stride = p->cmp_stride;
   a.window = p->window;
   a.sel_len = p->sel_block;
-  a.nsel = L.nsel;
+  a.nsel = L.score_stride;  // the score rows' stride
   a.out = out;
   a.out_f32 = p->out_dtype == NSA_OUT_F32;
   if (nv > 0) {
@@ -335,8 +337,9 @@ int prefill_impl(const nsa_params_t* p, const void* q, const void* k, const void
       if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
       int blocks = (nitems + nsa::kTopnWarps - 1) / nsa::kTopnWarps;
       if (blocks > 148 * 32) blocks = 148 * 32;
-      kern<<<blocks, nsa::kTopnWarps * 32, smem, st>>>(a.scores, nitems, hkv, L.nsel, p->sel_block, p->top_n,
-                                                        reinterpret_cast<int32_t*>(ws + L.sel_idx), out_sel_idx);
+      kern<<<blocks, nsa::kTopnWarps * 32, smem, st>>>(a.scores, nitems, hkv, L.nsel, L.score_stride, p->sel_block,
+                                                        p->top_n, reinterpret_cast<int32_t*>(ws + L.sel_idx),
+                                                        out_sel_idx);
       if ((rc = launch_status("topn", st)) != NSA_OK) return rc;
     }
     // 4. selected branch, block-major: bucket (token, slot) pairs by (group, block),
@@ -576,6 +579,7 @@ int nsa_prefill_workspace_layout(const nsa_params_t* params, nsa_prefill_layout_
   layout->total = L.total;
   layout->n_cmp = L.ncmp;
   layout->n_sel = L.nsel;
+  layout->score_stride = L.score_stride;
   return NSA_OK;
 }
 

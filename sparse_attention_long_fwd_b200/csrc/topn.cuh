@@ -294,7 +294,8 @@ __device__ __forceinline__ void warp_topn_regs(int* list, const float* __restric
   __syncwarp();
 }
 
-// scores: [nitems][nsel] fp32 (item = row * hkv + g); idx / idx_copy: [nitems][top_n].
+// scores: [nitems][stride] fp32 (item = row * hkv + g; stride >= nsel); idx / idx_copy:
+// [nitems][top_n].
 // Row position t = row (prefill rows are token positions).
 // One warp per (row, group). kRegsOnly: every row has fewer than 2,048 candidate blocks and
 // top_n <= 32 (checked by the host), so only the register path runs and each warp needs just
@@ -302,7 +303,7 @@ __device__ __forceinline__ void warp_topn_regs(int* list, const float* __restric
 // the list and the bitmap of the shared-memory path.
 template <bool kRegsOnly>
 __global__ void __launch_bounds__(kTopnWarps * 32) topn_kernel(const float* __restrict__ scores, int nitems, int hkv,
-                                                                int nsel, int sel_len, int top_n,
+                                                                int nsel, int stride, int sel_len, int top_n,
                                                                 int32_t* __restrict__ idx,
                                                                 int32_t* __restrict__ idx_copy) {
   extern __shared__ float tsm[];
@@ -319,7 +320,7 @@ __global__ void __launch_bounds__(kTopnWarps * 32) topn_kernel(const float* __re
       if (lane == 0) record_error(kErrBadIndex);
       continue;
     }
-    const float* src = scores + static_cast<size_t>(item) * nsel;
+    const float* src = scores + static_cast<size_t>(item) * stride;
     int32_t* d = idx + static_cast<size_t>(item) * top_n;
     int32_t* d2 = idx_copy ? idx_copy + static_cast<size_t>(item) * top_n : nullptr;
     if (!kRegsOnly && (top_n > 32 || jt >= 32 * 64)) warp_topn(sc, bits, list, src, jt, top_n, d, d2, lane);

@@ -57,7 +57,7 @@ class NsaParams(ctypes.Structure):
 
 class NsaPrefillLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in ("kc", "vc", "o_cmp", "lse", "scores", "sel_idx", "o_win", "total")] + [
-        ("n_cmp", ctypes.c_int32), ("n_sel", ctypes.c_int32)]
+        ("n_cmp", ctypes.c_int32), ("n_sel", ctypes.c_int32), ("score_stride", ctypes.c_int32)]
 
 
 _lib = None

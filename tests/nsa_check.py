@@ -118,7 +118,8 @@ def compare_prefill_rows(w: Workload, q, k, v, gates, rows, out, sel, ws, layout
             if fin.any():
                 assert np.abs(lse[fin] - o["lse"][vid][fin]).max() < 1e-3
             nsel = layout["n_sel"]
-            sc = ws_view(ws, layout["scores"], (w.n_video, w.hkv, nsel), torch.float32)[vrows].cpu().numpy()
+            sc = ws_view(ws, layout["scores"], (w.n_video, w.hkv, layout["score_stride"]),
+                         torch.float32)[vrows, :, :nsel].cpu().numpy()
             for i, t in enumerate(vrows):
                 jt = t // w.sel_len
                 ref = o["scores"][vid][i][:, : jt + 1]

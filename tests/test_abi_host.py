@@ -79,10 +79,13 @@ def test_prefill_layout_is_aligned_and_disjoint():
         assert lay["total"] == nsa.nsa_workspace_size(p, False)
         ncmp = (nv - 32) // 16 + 1 if nv >= 32 else 0
         assert lay["n_cmp"] == ncmp and lay["n_sel"] == (nv + 63) // 64
+        # score rows are 16-byte aligned: the stride is n_sel rounded up to a multiple of 4
+        assert lay["score_stride"] % 4 == 0 and 0 <= lay["score_stride"] - lay["n_sel"] < 4
         keys = ["kc", "vc", "o_cmp", "lse", "scores", "sel_idx", "o_win"]
         offs = [lay[k] for k in keys] + [lay["total"]]
         assert all(o % 256 == 0 for o in offs)
-        sizes = [max(ncmp, 1) * 4 * 128 * 2] * 2 + [nv * 28 * 128 * 2, nv * 28 * 4, nv * 4 * max(lay["n_sel"], 1) * 4,
+        sizes = [max(ncmp, 1) * 4 * 128 * 2] * 2 + [nv * 28 * 128 * 2, nv * 28 * 4,
+                                                    nv * 4 * max(lay["score_stride"], 4) * 4,
                                                     nv * 4 * 16 * 4, nv * 28 * 128 * 2]
         for i, sz in enumerate(sizes):
             assert offs[i] + sz <= offs[i + 1], keys[i]
