@@ -291,6 +291,46 @@ def run_config_lines(args, dev, peaks, peaks_src, flush, world, rank):
     return lines
 
 
+VARLEN_KERNELS = 11  # table and gather kernels, then the nine NSA stages (all-video batch: no text stage)
+
+
+def run_varlen(args, dev, peaks, flush, world, rank):
+    """A serving batch: 64 all-video clips of 2,048 tokens packed back to back, one
+    nsa_prefill_varlen call per step (every stage launched once for the whole batch)."""
+    B, L = 64, 2048
+    w = WORKLOADS["v128k"]
+    from sparse_attention_long_fwd_b200.inputs import scaled
+    wb = scaled(w, n_tokens=B * L, n_video=B * L)
+    q, k, v, g = prefill_inputs(wb, seed=30 + rank, device=dev)
+    cu = [b * L for b in range(B + 1)]
+    nvs = [L] * B
+    p = nsa.make_params(B * L, 0, w.hq, w.hkv, w.d, w.cmp_len, w.cmp_stride, w.sel_len, w.top_n, w.window,
+                        out_dtype=nsa.NSA_OUT_BF16)
+    need = nsa.nsa_prefill_varlen_workspace_size(p, cu, nvs)
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    out = torch.empty((B * L, w.hq, w.d), dtype=torch.bfloat16, device=dev)
+
+    def step(events):
+        rc = nsa.nsa_prefill_varlen(q, k, v, g, cu, nvs, p, out, None, ws, need)
+        if rc != nsa.NSA_OK:
+            raise nsa.NsaError(rc, "nsa_prefill_varlen")
+
+    barrier(world)
+    step_ms, _ = timed_steps(step, args.steps, args.warmup, flush, 0)
+    assert nsa.nsa_get_device_error(clear=True) == 0, "device error word set during the varlen run"
+    ms = max_over_ranks(sum(step_ms), world) / args.steps
+    # attended FLOPs: each clip counted as its own 2,048-token sequence
+    c = prefill_counts(scaled(w, n_tokens=L, n_video=L))
+    flops = B * (c["cmp_flops"] + c["sel_flops"] + c["win_flops"])
+    tf = flops / (ms / 1e3) / 1e12
+    del ws, out, q, k, v, g
+    return {"workload": f"{B} clips x {L} video tokens packed back to back (nsa_prefill_varlen), Hq={w.hq}, "
+                        f"Hkv={w.hkv}, d={w.d}, n={w.top_n}, w={w.window}",
+            "ms_per_step": round(ms, 4), "value": round(B * L * world / (ms / 1e3), 1), "unit": "video tokens/s",
+            "attended_tflops": round(tf, 2), "attended_frac_of_peak": round(tf / peaks["bf16_tflops"], 4),
+            "launches_per_step": VARLEN_KERNELS, "steps": args.steps, "warmup": args.warmup}
+
+
 def run_b200(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
@@ -414,6 +454,8 @@ def run_b200(args, world, rank, local):
     if not args.no_configs:
         result["configs"] = run_config_lines(args, dev, peaks, peaks_src, flush, world, rank)
         result["gpu_launches"] += sum(c["launches"] for c in result["configs"])
+        result["varlen"] = run_varlen(args, dev, peaks, flush, world, rank)
+        result["gpu_launches"] += VARLEN_KERNELS * args.steps
 
     if not args.no_decode:
         result["decode"] = run_decode(args, dev, peaks, peaks_src, flush, world)

@@ -103,18 +103,57 @@ int nsa_prefill(const void* q, const void* k, const void* v, const float* gates,
  *   out_sel_idx NULL, or [sum of n_video][Hkv][top_n] int32: the video rows of every sequence,
  *               sequence after sequence.
  *   workspace   at least nsa_prefill_varlen_workspace_size(params, cu_seqlens, n_video, B) bytes.
- * Each sequence gets exactly what nsa_prefill computes for it alone; positions restart at 0
- * in every sequence. The sequences run one after another on `stream` and share the workspace,
- * so the caller must not run two calls on one workspace concurrently. Errors as nsa_prefill,
- * plus NSA_ERR_INVALID_ARG for malformed cu_seqlens / n_video; nothing is enqueued then.
+ * Each sequence gets what nsa_prefill computes for it alone (the same selection, outputs equal
+ * up to fp32 summation order); positions restart at 0 in every sequence. This is
+ * nsa_prefill_packed with each sequence's video prefix and trailing text as its two
+ * segments: every stage is launched once for the whole batch. Errors as nsa_prefill, plus
+ * NSA_ERR_INVALID_ARG for malformed cu_seqlens / n_video; nothing is enqueued then.
  */
 int nsa_prefill_varlen(const void* q, const void* k, const void* v, const float* gates, const int32_t* cu_seqlens,
                        const int32_t* n_video, int batch, const nsa_params_t* params, void* out,
                        int32_t* out_sel_idx, void* workspace, size_t workspace_bytes, void* stream);
 
-/* Workspace bytes nsa_prefill_varlen needs (the largest single sequence's); 0 if the arguments are invalid. */
+/* Workspace bytes nsa_prefill_varlen needs; 0 if the arguments are invalid. */
 size_t nsa_prefill_varlen_workspace_size(const nsa_params_t* params, const int32_t* cu_seqlens,
                                          const int32_t* n_video, int batch);
+
+/*
+ * Packed prefill with video and text segments in any order: B sequences back to back, each a
+ * run of segments. Video tokens get NSA and text tokens dense attention (shd-paper.top page
+ * "VideoNSA: Native Sparse Attention Scales Video Understanding", abstract); clip lengths vary
+ * from request to request (CSDN blog on VideoNSA, vcloud.csdn.net, section 5.2, item 3). The
+ * pages never put text between video segments; this library's reading, which reduces to the
+ * trailing-text layout of nsa_prefill:
+ *   - a video row gets NSA over its sequence's video tokens only, taken in order as one
+ *     stream: compression and selection blocks, the window and causality count positions in
+ *     that stream, exactly as for a sequence made of those video tokens alone;
+ *   - a text row gets dense causal attention over every earlier token of its sequence, video
+ *     and text, and itself (gates unused).
+ * Arguments:
+ *   cu_seqlens  HOST [B+1]: sequence b owns packed rows [cu_seqlens[b], cu_seqlens[b+1]);
+ *               cu_seqlens[0] = 0, non-decreasing, cu_seqlens[B] = params->n_tokens.
+ *   seg_lens    HOST [nseg]: segment lengths (> 0) in packed order; the segments tile every
+ *               sequence exactly (an empty sequence has none).
+ *   seg_video   HOST [nseg]: 1 for a video segment, 0 for a text segment.
+ *   q, k, v, gates, out: as nsa_prefill over the params->n_tokens packed rows (params->n_video
+ *               is ignored; gates may be NULL when there is no video row).
+ *   out_sel_idx NULL, or [total video rows][Hkv][top_n] int32: every video row's selection,
+ *               in packed order (sequence after sequence, segment after segment).
+ *   workspace   at least nsa_prefill_packed_workspace_size(...) bytes, 256-byte aligned.
+ * Every stage is launched once for the whole batch (tiles span sequences); the plan (two small
+ * tables) is copied to the workspace with cudaMemcpyAsync from host memory first. Errors as
+ * nsa_prefill, plus NSA_ERR_INVALID_ARG for malformed sequence or segment arrays, and
+ * NSA_ERR_UNSUPPORTED when a video stream has more than 8,192 selection blocks; nothing is
+ * enqueued then.
+ */
+int nsa_prefill_packed(const void* q, const void* k, const void* v, const float* gates, const int32_t* cu_seqlens,
+                       int batch, const int32_t* seg_lens, const uint8_t* seg_video, int nseg,
+                       const nsa_params_t* params, void* out, int32_t* out_sel_idx, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/* Workspace bytes nsa_prefill_packed needs; 0 if the arguments are invalid. */
+size_t nsa_prefill_packed_workspace_size(const nsa_params_t* params, const int32_t* cu_seqlens, int batch,
+                                         const int32_t* seg_lens, const uint8_t* seg_video, int nseg);
 
 /*
  * Decode: one query token per sequence against a KV cache and its compressed cache.

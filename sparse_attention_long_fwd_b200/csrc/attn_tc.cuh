@@ -59,6 +59,13 @@ struct AttnArgs {
   __half* o_win;           // kModeWin: write [N_v][Hq][d]
   void* out;               // kModeDense: write [N][Hq][d]
   int out_f32;
+  // Packed batches (null for one sequence). vinfo [video stream tokens]: per token the stream
+  // index of its sequence's first video token (x), its sequence's first compressed-key row (y,
+  // a multiple of 128), its sequence's first selection block (z) and its row in the packed
+  // batch (w). tinfo [text stream rows] (kModeDense): per row its row in the packed batch (x)
+  // and its sequence's first row there (y); keys are then rows of the packed batch.
+  const int4* vinfo;
+  const int2* tinfo;
 };
 
 // Softmax warpgroups, by mode. Two warpgroups share each S tile, one per 64-column half.
@@ -199,7 +206,9 @@ __device__ __forceinline__ void group_reduce_scatter(float (&bin)[NB], int lane)
   }
 }
 
-template <int D, int MODE>
+// PACKED: the rows belong to a packed batch (AttnArgs::vinfo / tinfo); a single sequence
+// compiles without those lookups.
+template <int D, int MODE, bool PACKED = false>
 __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
     attn_tile_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap vmap, const AttnArgs args) {
@@ -236,13 +245,24 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
     const int tile = (MODE == kModeWin) ? rank : (args.n_tiles - 1 - rank);
     t0 = args.q_begin + tile * T;
     const int t_last = min(t0 + T, args.q_end) - 1;
+    // the tile's key range runs from its first row's first key to its last row's last key
+    // (rows are in order, and so are their sequences)
     int ke;
     if (MODE == kModeCmp) {
-      kb = 0;
-      ke = ncmp_visible(t_last, args.cmp_len, args.cmp_stride);
+      if ((PACKED && args.vinfo != nullptr)) {
+        const int4 a = args.vinfo[t0], z = args.vinfo[t_last];
+        kb = a.y;
+        ke = z.y + ncmp_visible(t_last - z.x, args.cmp_len, args.cmp_stride);
+      } else {
+        kb = 0;
+        ke = ncmp_visible(t_last, args.cmp_len, args.cmp_stride);
+      }
     } else if (MODE == kModeWin) {
-      kb = max(0, t0 - args.window + 1);
+      kb = max((PACKED && args.vinfo != nullptr) ? args.vinfo[t0].x : 0, t0 - args.window + 1);
       ke = t_last + 1;
+    } else if ((PACKED && args.tinfo != nullptr)) {
+      kb = args.tinfo[t0].y;
+      ke = args.tinfo[t_last].x + 1;
     } else {
       kb = 0;
       ke = t_last + 1;
@@ -539,12 +559,25 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
       const int h = g * G + hh;
       const bool row_valid = (r < T * Gp) && (hh < G) && (t < args.q_end);
       int rb = 0, re = 0;  // visible key range of this row
+      int s_first = 0;     // (packed) stream index of the first video token of the row's sequence
       if (row_valid) {
         if (MODE == kModeCmp) {
-          re = ncmp_visible(t, args.cmp_len, args.cmp_stride);
+          if ((PACKED && args.vinfo != nullptr)) {
+            const int4 a = args.vinfo[t];
+            s_first = a.x;
+            rb = a.y;
+            re = a.y + ncmp_visible(t - a.x, args.cmp_len, args.cmp_stride);
+          } else {
+            re = ncmp_visible(t, args.cmp_len, args.cmp_stride);
+          }
         } else if (MODE == kModeWin) {
-          rb = max(0, t - args.window + 1);
+          if ((PACKED && args.vinfo != nullptr)) s_first = args.vinfo[t].x;
+          rb = max(s_first, t - args.window + 1);
           re = t + 1;
+        } else if ((PACKED && args.tinfo != nullptr)) {
+          const int2 a = args.tinfo[t];
+          rb = a.y;
+          re = a.x + 1;
         } else {
           re = t + 1;
         }
@@ -640,7 +673,15 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
       // reduce-scatter sums them.
       float carry_last = 0.f;  // upper half, last tile: half of its last compressed block
       const bool sc_store = MODE == kModeCmp && t < args.q_end && (hh % sc_share) == 0;
-      const int sc_jt = t / args.sel_len;
+      // (packed) a row whose sequence starts after the tile's first key row sees its own
+      // blocks from column (rb - kb) on, a multiple of 128: its block indices are offset by
+      // sc_joff; rows padding the tile hold no position
+      int sc_jt = t / args.sel_len, sc_joff = 0;
+      if (MODE == kModeCmp && (PACKED && args.vinfo != nullptr)) {
+        const int4 a = args.vinfo[min(t, args.q_end - 1)];
+        sc_jt = (t - a.x) / args.sel_len;
+        sc_joff = (a.y - kb) / 4;
+      }
       float* const sc_dst = args.scores + (static_cast<size_t>(t) * args.hkv + g) * args.nsel;
       // this pair's phase-2 jobs are those of parity `pair`: job nkt + kt2
       for (int kt2 = kPairs == 1 ? 0 : ((pair + nkt) & 1); ok && kt2 < nkt; kt2 += kPairs) {
@@ -737,13 +778,13 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
               default: break;
             }
             if (sc_store) {
-              const int j0 = kt2 * 32 + hc * kChunkBins + sc_j0;
+              const int j0 = kt2 * 32 + hc * kChunkBins + sc_j0 - sc_joff;
               if (sc_bpl == 1) {
-                if (j0 <= sc_jt) sc_dst[j0] = bin[0];
+                if (j0 >= 0 && j0 <= sc_jt) sc_dst[j0] = bin[0];
               } else {
 #pragma unroll
                 for (int i = 0; i < kChunkBins; ++i)
-                  if (i < sc_bpl && j0 + i <= sc_jt) sc_dst[j0 + i] = bin[i];
+                  if (i < sc_bpl && j0 + i >= 0 && j0 + i <= sc_jt) sc_dst[j0 + i] = bin[i];
               }
             }
           }
@@ -789,8 +830,8 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
 #pragma unroll
         for (int o = 1; o < 16; o <<= 1)
           if (o < Gp) c += __shfl_xor_sync(0xffffffffu, c, o);
-        const int j = nkt * 32;
-        if (hh == 0 && t < args.q_end && j <= t / args.sel_len)
+        const int j = nkt * 32 - sc_joff;
+        if (hh == 0 && t < args.q_end && j >= 0 && j <= sc_jt)
           args.scores[(static_cast<size_t>(t) * args.hkv + g) * args.nsel + j] = c;
       }
       float inv_l = 1.f;  // (window, dense) 1 / row sum of P over all column slices
@@ -811,6 +852,10 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
       }
       // (after a failed wait the work below is skipped, but the named barrier is still passed)
       const size_t orow = (static_cast<size_t>(t) * args.hq + h) * D;
+      // (packed text rows) the dense output goes to the row's place in the packed batch
+      const size_t drow = (MODE == kModeDense && (PACKED && args.tinfo != nullptr) && row_valid)
+                              ? (static_cast<size_t>(args.tinfo[t].x) * args.hq + h) * D
+                              : orow;
       constexpr int kOC = D / kSoftmaxWG < 32 ? D / kSoftmaxWG : 32;  // output columns per load
       constexpr int kOLoads = (D / kSoftmaxWG + 31) / 32;
       float o[kOLoads][32];
@@ -885,12 +930,12 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
 #pragma unroll
             for (int u = 0; u < kOC; ++u) oc_[u] *= inv_l;
             if (args.out_f32) {
-              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.out) + orow + c0);
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.out) + drow + c0);
 #pragma unroll
               for (int u = 0; u < kOC / 4; ++u)
                 dst[u] = make_float4(oc_[4 * u], oc_[4 * u + 1], oc_[4 * u + 2], oc_[4 * u + 3]);
             } else {
-              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) + orow + c0);
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) + drow + c0);
 #pragma unroll
               for (int u = 0; u < kOC / 8; ++u)
                 dst[u] = make_uint4(pack_bf16x2(oc_[8 * u], oc_[8 * u + 1]), pack_bf16x2(oc_[8 * u + 2], oc_[8 * u + 3]),

@@ -8,6 +8,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "nsa.h"
 #include "sm100.cuh"
@@ -20,6 +21,7 @@
 #include "decode.cuh"
 #include "gate.cuh"
 #include "backward.cuh"
+#include "pack.cuh"
 
 namespace nsa {
 
@@ -105,11 +107,13 @@ struct PrefillLayout {
   int score_stride;     // floats per score row: nsel rounded up to 4, so rows are 16-byte aligned
 };
 
-PrefillLayout prefill_layout(const nsa_params_t* p) {
+// Workspace layout of the NSA rows of one call: nv stream rows, ncmp_rows compressed rows,
+// nsel_cols selection-block columns per group (the bucket space) and score rows of up to
+// nsel_max blocks (one sequence: ncmp_rows = Ncmp(nv), nsel_cols = nsel_max = Nsel(nv)).
+PrefillLayout video_layout(int nv, int ncmp_rows, int nsel_cols, int nsel_max, int hq, int hkv, int d, int top_n) {
   PrefillLayout L{};
-  const int nv = p->n_video, hq = p->num_q_heads, hkv = p->num_kv_heads, d = p->head_dim;
-  L.ncmp = ncmp_of(nv, p->cmp_block, p->cmp_stride);
-  L.nsel = nsel_of(nv, p->sel_block);
+  L.ncmp = ncmp_rows;
+  L.nsel = nsel_cols;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t at = off;
@@ -121,12 +125,12 @@ PrefillLayout prefill_layout(const nsa_params_t* p) {
   L.vc = take(cmp_rows * hkv * d * 2);
   L.o_cmp = take(static_cast<size_t>(nv) * hq * d * 2);
   L.lse = take(static_cast<size_t>(nv) * hq * 4);
-  L.score_stride = (L.nsel + 3) / 4 * 4;
+  L.score_stride = (nsel_max + 3) / 4 * 4;
   L.scores = take(static_cast<size_t>(nv) * hkv * (L.score_stride > 0 ? L.score_stride : 4) * 4);
-  L.sel_idx = take(static_cast<size_t>(nv) * hkv * p->top_n * 4);
+  L.sel_idx = take(static_cast<size_t>(nv) * hkv * top_n * 4);
   L.o_win = take(static_cast<size_t>(nv) * hq * d * 2);
   const size_t buckets = static_cast<size_t>(hkv) * (L.nsel > 0 ? L.nsel : 1);
-  const size_t entries = static_cast<size_t>(nv) * hkv * p->top_n;
+  const size_t entries = static_cast<size_t>(nv) * hkv * top_n;
   L.sel_cnt = take(2 * buckets * 4);
   L.sel_eoff = take((buckets + 1) * 4);
   L.sel_toff = take((buckets + 1) * 4);
@@ -141,6 +145,13 @@ PrefillLayout prefill_layout(const nsa_params_t* p) {
   L.part_ml = take(static_cast<size_t>(L.part_rows) * 16);
   L.total = off;
   return L;
+}
+
+PrefillLayout prefill_layout(const nsa_params_t* p) {
+  const int nv = p->n_video;
+  const int ns = nsel_of(nv, p->sel_block);
+  return video_layout(nv, ncmp_of(nv, p->cmp_block, p->cmp_stride), ns, ns, p->num_q_heads, p->num_kv_heads,
+                      p->head_dim, p->top_n);
 }
 
 struct DecodeLayout {
@@ -236,13 +247,14 @@ int set_smem(K kernel, size_t bytes) {
 // ------------------------------------------------------------------ launchers
 // wk, wv: per-head block weights [hkv][l] of the learnable compression, or null for the mean
 int launch_pool(const void* k, const void* v, void* kc, void* vc, int nseq, int T, int hkv, int d, int ncmp, int l,
-                int s, cudaStream_t st, const float* wk = nullptr, const float* wv = nullptr) {
+                int s, cudaStream_t st, const float* wk = nullptr, const float* wv = nullptr,
+                const int* row_tok = nullptr) {
   if (ncmp <= 0) return NSA_OK;
   const long long threads = static_cast<long long>(nseq) * ncmp * hkv * (d / 2);
   const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
   nsa::pool_kernel<<<dim3(blocks, 1, 2), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(kc),
-      static_cast<__nv_bfloat16*>(vc), wk, wv, nseq, T, hkv, d, ncmp, l, s);
+      static_cast<__nv_bfloat16*>(vc), wk, wv, nseq, T, hkv, d, ncmp, l, s, row_tok);
   return launch_status("pool", st);
 }
 
@@ -251,7 +263,8 @@ int launch_attn(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap&
                 cudaStream_t st) {
   if (a.n_tiles <= 0) return NSA_OK;
   const size_t smem = sizeof(nsa::AttnSmem<D, MODE>) + 1024;
-  auto kern = nsa::attn_tile_kernel<D, MODE>;
+  const bool packed = a.vinfo != nullptr || a.tinfo != nullptr;
+  auto kern = packed ? nsa::attn_tile_kernel<D, MODE, true> : nsa::attn_tile_kernel<D, MODE, false>;
   if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
   // persistent modes: one CTA per SM walks the (tile, group) items; otherwise one CTA per item
   const long long items = static_cast<long long>(a.n_tiles) * a.hkv;
@@ -263,12 +276,33 @@ int launch_attn(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap&
   return launch_status(MODE == nsa::kModeCmp ? "attn_cmp" : MODE == nsa::kModeWin ? "attn_win" : "attn_dense", st);
 }
 
+// What one prefill call computes, stage by stage: NSA over the rows of a video stream and
+// dense causal attention over a set of text rows. One sequence: the stream is the video
+// prefix itself and the text rows follow it. A packed batch: the stream is every sequence's
+// video tokens back to back (tables give each token its sequence), and the text rows are
+// gathered into a stream of their own whose keys are the rows of the packed batch.
+struct StageGeo {
+  const void *q, *k, *v;   // video stream: q [rows][hq][D], k, v [rows][hkv][D]
+  int rows;                // rows of those tensors (the extent of their TMA maps)
+  int nv;                  // NSA rows: stream rows [0, nv)
+  const int4* vinfo;       // packed: per stream row (sequence's first row, first compressed row,
+                           // first selection block, row in the batch); null: one sequence
+  const int* row_tok;      // packed: first stream token of every compressed row (-1: padding)
+  const int* blk_tok;      // packed: first stream token of every selection block
+  int nsel_max;            // selection blocks of the longest sequence
+  const void* qt;          // text rows: queries [qt_rows][hq][D]
+  int qt_rows, t_begin, t_end;  // dense rows [t_begin, t_end) of qt
+  const int2* tinfo;       // packed: per text row (row in the batch, first row of its sequence)
+  const void *kd, *vd;     // keys and values of the dense rows [kd_rows][hkv][D]
+  int kd_rows;
+  const float* gates;      // [rows of the batch][hq][3]
+  void* out;               // [rows of the batch][hq][D]
+};
+
 template <int D>
-int prefill_impl(const nsa_params_t* p, const void* q, const void* k, const void* v, const float* gates, void* out,
-                 int32_t* out_sel_idx, uint8_t* ws, cudaStream_t st, const float* phi_k = nullptr,
-                 const float* phi_v = nullptr) {
-  const PrefillLayout L = prefill_layout(p);
-  const int N = p->n_tokens, nv = p->n_video, hq = p->num_q_heads, hkv = p->num_kv_heads;
+int video_stages(const nsa_params_t* p, const StageGeo& geo, const PrefillLayout& L, int32_t* out_sel_idx,
+                 uint8_t* ws, cudaStream_t st, const float* phi_k, const float* phi_v) {
+  const int nv = geo.nv, hq = p->num_q_heads, hkv = p->num_kv_heads;
   const int G = hq / hkv;
   const int T = 128 / G;
   int Gc = 1;  // compressed mode: G rounded up to a power of two, so a token's heads share a warp
@@ -280,9 +314,15 @@ int prefill_impl(const nsa_params_t* p, const void* q, const void* k, const void
   CUtensorMap qmap, qcmap, kmap, vmap, kcmap, vcmap;
   const uint64_t qs1 = static_cast<uint64_t>(D) * 2, qs2 = static_cast<uint64_t>(hq) * D * 2;
   const uint64_t ks1 = static_cast<uint64_t>(D) * 2, ks2 = static_cast<uint64_t>(hkv) * D * 2;
-  if (!nsa::make_tmap_bf16_3d(&qmap, q, D, hq, N, qs1, qs2, 64, G, T) ||
-      !nsa::make_tmap_bf16_3d(&kmap, k, D, hkv, N, ks1, ks2, 64, 1, nsa::kBN) ||
-      !nsa::make_tmap_bf16_3d(&vmap, v, D, hkv, N, ks1, ks2, 64, 1, nsa::kBN))
+  auto* kc = ws + L.kc;
+  auto* vc = ws + L.vc;
+  const int ncmp_rows = L.ncmp > 0 ? L.ncmp : 1;
+  if (!nsa::make_tmap_bf16_3d(&qmap, geo.q, D, hq, geo.rows, qs1, qs2, 64, G, T) ||
+      !nsa::make_tmap_bf16_3d(&kmap, geo.k, D, hkv, geo.rows, ks1, ks2, 64, 1, nsa::kBN) ||
+      !nsa::make_tmap_bf16_3d(&vmap, geo.v, D, hkv, geo.rows, ks1, ks2, 64, 1, nsa::kBN) ||
+      !nsa::make_tmap_bf16_3d(&kcmap, kc, D, hkv, ncmp_rows, ks1, ks2, 64, 1, nsa::kBN) ||
+      !nsa::make_tmap_bf16_3d(&vcmap, vc, D, hkv, ncmp_rows, ks1, ks2, 64, 1, nsa::kBN) ||
+      !nsa::make_tmap_bf16_3d(&qcmap, geo.q, D, hq, geo.rows, qs1, qs2, 64, Gc, Tc))
     return NSA_ERR_CUDA;
   AttnArgs a{};
   a.hq = hq;
@@ -296,130 +336,181 @@ int prefill_impl(const nsa_params_t* p, const void* q, const void* k, const void
   a.window = p->window;
   a.sel_len = p->sel_block;
   a.nsel = L.score_stride;  // the score rows' stride
-  a.out = out;
+  a.out = geo.out;
   a.out_f32 = p->out_dtype == NSA_OUT_F32;
-  if (nv > 0) {
-    auto* kc = ws + L.kc;
-    auto* vc = ws + L.vc;
-    const int ncmp_rows = L.ncmp > 0 ? L.ncmp : 1;
-    if (!nsa::make_tmap_bf16_3d(&kcmap, kc, D, hkv, ncmp_rows, ks1, ks2, 64, 1, nsa::kBN) ||
-        !nsa::make_tmap_bf16_3d(&vcmap, vc, D, hkv, ncmp_rows, ks1, ks2, 64, 1, nsa::kBN) ||
-        !nsa::make_tmap_bf16_3d(&qcmap, q, D, hq, N, qs1, qs2, 64, Gc, Tc))
-      return NSA_ERR_CUDA;
-    // 1. compression: Kc, Vc of the video prefix
-    if ((rc = launch_pool(k, v, kc, vc, 1, nv, hkv, D, L.ncmp, p->cmp_block, p->cmp_stride, st, phi_k, phi_v)) !=
-        NSA_OK)
-      return rc;
-    // 2. compressed branch + block scores
-    a.q_begin = 0;
-    a.q_end = nv;
-    a.o_cmp = reinterpret_cast<__half*>(ws + L.o_cmp);
-    a.lse = reinterpret_cast<float*>(ws + L.lse);
-    a.scores = reinterpret_cast<float*>(ws + L.scores);
-    {
-      AttnArgs ac = a;
-      ac.Gp = Gc;
-      ac.T = Tc;
-      ac.n_tiles = (nv + Tc - 1) / Tc;
-      if ((rc = launch_attn<D, nsa::kModeCmp>(qcmap, kcmap, vcmap, ac, st)) != NSA_OK) return rc;
-    }
-    a.n_tiles = (nv + T - 1) / T;
-    // 3. top-n selection
-    {
-      const int nitems = nv * hkv;
-      const int nwords = (L.nsel + 31) / 32;
-      // every row on the register path (fewer than 2,048 blocks, top_n <= 32): 64 list
-      // entries per warp, so shared memory does not limit the warps per SM
-      const bool regs_only = L.nsel <= 32 * 64 && p->top_n <= 32;
-      const size_t smem =
-          static_cast<size_t>(nsa::kTopnWarps) * (regs_only ? 64 : 2 * L.nsel + nwords) * 4;
-      auto kern = regs_only ? nsa::topn_kernel<true> : nsa::topn_kernel<false>;
-      if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
-      int blocks = (nitems + nsa::kTopnWarps - 1) / nsa::kTopnWarps;
-      if (blocks > 148 * 32) blocks = 148 * 32;
-      kern<<<blocks, nsa::kTopnWarps * 32, smem, st>>>(a.scores, nitems, hkv, L.nsel, L.score_stride, p->sel_block,
-                                                        p->top_n, reinterpret_cast<int32_t*>(ws + L.sel_idx),
-                                                        out_sel_idx);
-      if ((rc = launch_status("topn", st)) != NSA_OK) return rc;
-    }
-    // 4. selected branch, block-major: bucket (token, slot) pairs by (group, block),
-    //    one tensor-core tile per bucket tile, then merge each row's partials
-    {
-      const int m = hkv * L.nsel;
-      const int Gp = G;  // tile rows token * G + head: no padding heads
-      const int TT = 128 / Gp;
-      const long long entries = static_cast<long long>(nv) * hkv * p->top_n;
-      nsa::SelInvArgs sa{};
-      sa.nv = nv;
-      sa.hq = hq;
-      sa.hkv = hkv;
-      sa.G = G;
-      sa.Gp = Gp;
-      sa.TT = TT;
-      sa.nsel = L.nsel;
-      sa.top_n = p->top_n;
-      sa.sel_len = p->sel_block;
-      sa.sl2 = sl2;
-      sa.sel_idx = reinterpret_cast<const int32_t*>(ws + L.sel_idx);
-      sa.cnt = reinterpret_cast<int*>(ws + L.sel_cnt);
-      sa.cursor = sa.cnt + m;
-      sa.ent_off = reinterpret_cast<int*>(ws + L.sel_eoff);
-      sa.tile_off = reinterpret_cast<int*>(ws + L.sel_toff);
-      sa.list = reinterpret_cast<int*>(ws + L.sel_list);
-      sa.row_of = reinterpret_cast<int*>(ws + L.sel_row);
-      sa.part_rows = L.part_rows;
-      sa.part_o = reinterpret_cast<const __half*>(ws + L.part_o);
-      sa.part_ml = reinterpret_cast<float4*>(ws + L.part_ml);
-      sa.o_cmp = reinterpret_cast<const __half*>(ws + L.o_cmp);
-      sa.o_win = reinterpret_cast<const __half*>(ws + L.o_win);
-      sa.gates = gates;
-      sa.out = out;
-      sa.out_f32 = p->out_dtype == NSA_OUT_F32;
-      sa.q = static_cast<const __nv_bfloat16*>(q);
-      CUtensorMap k64map, v64map, omap;
-      if (!nsa::make_tmap_f16_3d(&omap, ws + L.part_o, 64, static_cast<uint64_t>(L.part_rows), D / 64, 128,
-                                 static_cast<uint64_t>(L.part_rows) * 128, 64, 32, 1) ||
-          !nsa::make_tmap_bf16_3d(&k64map, k, D, hkv, N, ks1, ks2, 64, 1, 64) ||
-          !nsa::make_tmap_bf16_3d(&v64map, v, D, hkv, N, ks1, ks2, 64, 1, 64))
-        return NSA_ERR_CUDA;
-      if (cudaMemsetAsync(sa.cnt, 0, 2 * static_cast<size_t>(m) * 4, st) != cudaSuccess) return NSA_ERR_CUDA;
-      long long eb = (entries + 255) / 256;
-      const unsigned ebl = static_cast<unsigned>(eb < 148 * 16 ? (eb > 0 ? eb : 1) : 148 * 16);
-      nsa::sel_count_kernel<<<ebl, 256, 0, st>>>(sa);
-      if ((rc = launch_status("sel_count", st, false)) != NSA_OK) return rc;
-      nsa::sel_scan_kernel<<<1, 1024, 0, st>>>(sa);
-      if ((rc = launch_status("sel_scan", st, false)) != NSA_OK) return rc;
-      nsa::sel_scatter_kernel<<<ebl, 256, 0, st>>>(sa);
-      if ((rc = launch_status("sel_scatter", st)) != NSA_OK) return rc;
-      // persistent: one CTA per SM (512 TMEM columns each; the shared-memory request keeps
-      // a second CTA off the SM)
-      size_t smem = sizeof(nsa::SelTileSmem<D>) + 1024;
-      if (smem < 116 * 1024) smem = 116 * 1024;
-      auto kern = nsa::sel_tile_kernel<D>;
-      if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
-      const long long max_tiles = L.part_rows / 128;
-      const int nsm = sm_count();
-      if (nsm <= 0) return NSA_ERR_CUDA;
-      const unsigned grid = static_cast<unsigned>(max_tiles < nsm ? max_tiles : nsm);
-      kern<<<grid, nsa::kSelTileThreads, smem, st>>>(k64map, v64map, omap, sa);
-      if ((rc = launch_status("sel_tile", st)) != NSA_OK) return rc;
-      // 5. sliding window -> o_win
-      a.o_win = reinterpret_cast<__half*>(ws + L.o_win);
-      if ((rc = launch_attn<D, nsa::kModeWin>(qmap, kmap, vmap, a, st)) != NSA_OK) return rc;
-      // 6. merge of the selected partials + gated combine -> out rows [0, N_v)
-      const long long rows = static_cast<long long>(nv) * hq;
-      nsa::sel_merge_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(sa);
-      if ((rc = launch_status("sel_merge", st)) != NSA_OK) return rc;
-    }
+  a.vinfo = geo.vinfo;
+  // 1. compression: Kc, Vc of the video stream
+  if ((rc = launch_pool(geo.k, geo.v, kc, vc, 1, nv, hkv, D, L.ncmp, p->cmp_block, p->cmp_stride, st, phi_k, phi_v,
+                        geo.row_tok)) != NSA_OK)
+    return rc;
+  // 2. compressed branch + block scores
+  a.q_begin = 0;
+  a.q_end = nv;
+  a.o_cmp = reinterpret_cast<__half*>(ws + L.o_cmp);
+  a.lse = reinterpret_cast<float*>(ws + L.lse);
+  a.scores = reinterpret_cast<float*>(ws + L.scores);
+  {
+    AttnArgs ac = a;
+    ac.Gp = Gc;
+    ac.T = Tc;
+    ac.n_tiles = (nv + Tc - 1) / Tc;
+    if ((rc = launch_attn<D, nsa::kModeCmp>(qcmap, kcmap, vcmap, ac, st)) != NSA_OK) return rc;
   }
-  // 7. trailing text rows: dense causal attention -> out rows [N_v, N)
-  if (N > nv) {
-    a.q_begin = nv;
-    a.q_end = N;
-    a.n_tiles = (N - nv + T - 1) / T;
-    if ((rc = launch_attn<D, nsa::kModeDense>(qmap, kmap, vmap, a, st)) != NSA_OK) return rc;
+  a.n_tiles = (nv + T - 1) / T;
+  // 3. top-n selection
+  {
+    const int nitems = nv * hkv;
+    const int nwords = (geo.nsel_max + 31) / 32;
+    // every row on the register path (fewer than 2,048 blocks, top_n <= 32): 64 list
+    // entries per warp, so shared memory does not limit the warps per SM
+    const bool regs_only = geo.nsel_max <= 32 * 64 && p->top_n <= 32;
+    const size_t smem =
+        static_cast<size_t>(nsa::kTopnWarps) * (regs_only ? 64 : 2 * geo.nsel_max + nwords) * 4;
+    const bool packed = geo.vinfo != nullptr;
+    auto kern = regs_only ? (packed ? nsa::topn_kernel<true, true> : nsa::topn_kernel<true, false>)
+                          : (packed ? nsa::topn_kernel<false, true> : nsa::topn_kernel<false, false>);
+    if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
+    int blocks = (nitems + nsa::kTopnWarps - 1) / nsa::kTopnWarps;
+    if (blocks > 148 * 32) blocks = 148 * 32;
+    kern<<<blocks, nsa::kTopnWarps * 32, smem, st>>>(a.scores, nitems, hkv, geo.nsel_max, L.score_stride,
+                                                      p->sel_block, p->top_n,
+                                                      reinterpret_cast<int32_t*>(ws + L.sel_idx), out_sel_idx,
+                                                      geo.vinfo);
+    if ((rc = launch_status("topn", st)) != NSA_OK) return rc;
   }
-  return NSA_OK;
+  // 4. selected branch, block-major: bucket (token, slot) pairs by (group, block),
+  //    one tensor-core tile per bucket tile, then merge each row's partials
+  const int m = hkv * L.nsel;
+  const int Gp = G;  // tile rows token * G + head: no padding heads
+  const int TT = 128 / Gp;
+  const long long entries = static_cast<long long>(nv) * hkv * p->top_n;
+  nsa::SelInvArgs sa{};
+  sa.nv = nv;
+  sa.hq = hq;
+  sa.hkv = hkv;
+  sa.G = G;
+  sa.Gp = Gp;
+  sa.TT = TT;
+  sa.nsel = L.nsel;
+  sa.top_n = p->top_n;
+  sa.sel_len = p->sel_block;
+  sa.sl2 = sl2;
+  sa.sel_idx = reinterpret_cast<const int32_t*>(ws + L.sel_idx);
+  sa.cnt = reinterpret_cast<int*>(ws + L.sel_cnt);
+  sa.cursor = sa.cnt + m;
+  sa.ent_off = reinterpret_cast<int*>(ws + L.sel_eoff);
+  sa.tile_off = reinterpret_cast<int*>(ws + L.sel_toff);
+  sa.list = reinterpret_cast<int*>(ws + L.sel_list);
+  sa.row_of = reinterpret_cast<int*>(ws + L.sel_row);
+  sa.part_rows = L.part_rows;
+  sa.part_o = reinterpret_cast<const __half*>(ws + L.part_o);
+  sa.part_ml = reinterpret_cast<float4*>(ws + L.part_ml);
+  sa.o_cmp = reinterpret_cast<const __half*>(ws + L.o_cmp);
+  sa.o_win = reinterpret_cast<const __half*>(ws + L.o_win);
+  sa.gates = geo.gates;
+  sa.out = geo.out;
+  sa.out_f32 = p->out_dtype == NSA_OUT_F32;
+  sa.q = static_cast<const __nv_bfloat16*>(geo.q);
+  sa.vinfo = geo.vinfo;
+  sa.blk_tok = geo.blk_tok;
+  CUtensorMap k64map, v64map, omap;
+  if (!nsa::make_tmap_f16_3d(&omap, ws + L.part_o, 64, static_cast<uint64_t>(L.part_rows), D / 64, 128,
+                             static_cast<uint64_t>(L.part_rows) * 128, 64, 32, 1) ||
+      !nsa::make_tmap_bf16_3d(&k64map, geo.k, D, hkv, geo.rows, ks1, ks2, 64, 1, 64) ||
+      !nsa::make_tmap_bf16_3d(&v64map, geo.v, D, hkv, geo.rows, ks1, ks2, 64, 1, 64))
+    return NSA_ERR_CUDA;
+  if (cudaMemsetAsync(sa.cnt, 0, 2 * static_cast<size_t>(m) * 4, st) != cudaSuccess) return NSA_ERR_CUDA;
+  long long eb = (entries + 255) / 256;
+  const unsigned ebl = static_cast<unsigned>(eb < 148 * 16 ? (eb > 0 ? eb : 1) : 148 * 16);
+  nsa::sel_count_kernel<<<ebl, 256, 0, st>>>(sa);
+  if ((rc = launch_status("sel_count", st, false)) != NSA_OK) return rc;
+  nsa::sel_scan_kernel<<<1, 1024, 0, st>>>(sa);
+  if ((rc = launch_status("sel_scan", st, false)) != NSA_OK) return rc;
+  nsa::sel_scatter_kernel<<<ebl, 256, 0, st>>>(sa);
+  if ((rc = launch_status("sel_scatter", st)) != NSA_OK) return rc;
+  {
+    // persistent: one CTA per SM (512 TMEM columns each; the shared-memory request keeps
+    // a second CTA off the SM)
+    size_t smem = sizeof(nsa::SelTileSmem<D>) + 1024;
+    if (smem < 116 * 1024) smem = 116 * 1024;
+    auto kern = nsa::sel_tile_kernel<D>;
+    if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
+    const long long max_tiles = L.part_rows / 128;
+    const int nsm = sm_count();
+    if (nsm <= 0) return NSA_ERR_CUDA;
+    const unsigned grid = static_cast<unsigned>(max_tiles < nsm ? max_tiles : nsm);
+    kern<<<grid, nsa::kSelTileThreads, smem, st>>>(k64map, v64map, omap, sa);
+    if ((rc = launch_status("sel_tile", st)) != NSA_OK) return rc;
+  }
+  // 5. sliding window -> o_win
+  a.o_win = reinterpret_cast<__half*>(ws + L.o_win);
+  if ((rc = launch_attn<D, nsa::kModeWin>(qmap, kmap, vmap, a, st)) != NSA_OK) return rc;
+  // 6. merge of the selected partials + gated combine -> out (the NSA rows)
+  const long long rows = static_cast<long long>(nv) * hq;
+  nsa::sel_merge_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(sa);
+  return launch_status("sel_merge", st);
+}
+
+// Dense causal attention of the text rows [t_begin, t_end) of geo.qt.
+template <int D>
+int text_stage(const nsa_params_t* p, const StageGeo& geo, cudaStream_t st) {
+  if (geo.t_end <= geo.t_begin) return NSA_OK;
+  const int hq = p->num_q_heads, hkv = p->num_kv_heads;
+  const int G = hq / hkv;
+  const int T = 128 / G;
+  const float scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(D));
+  CUtensorMap qmap, kmap, vmap;
+  const uint64_t qs1 = static_cast<uint64_t>(D) * 2, qs2 = static_cast<uint64_t>(hq) * D * 2;
+  const uint64_t ks1 = static_cast<uint64_t>(D) * 2, ks2 = static_cast<uint64_t>(hkv) * D * 2;
+  if (!nsa::make_tmap_bf16_3d(&qmap, geo.qt, D, hq, geo.qt_rows, qs1, qs2, 64, G, T) ||
+      !nsa::make_tmap_bf16_3d(&kmap, geo.kd, D, hkv, geo.kd_rows, ks1, ks2, 64, 1, nsa::kBN) ||
+      !nsa::make_tmap_bf16_3d(&vmap, geo.vd, D, hkv, geo.kd_rows, ks1, ks2, 64, 1, nsa::kBN))
+    return NSA_ERR_CUDA;
+  AttnArgs a{};
+  a.hq = hq;
+  a.hkv = hkv;
+  a.G = G;
+  a.T = T;
+  a.Gp = G;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.cmp_len = p->cmp_block;
+  a.cmp_stride = p->cmp_stride;
+  a.window = p->window;
+  a.sel_len = p->sel_block;
+  a.out = geo.out;
+  a.out_f32 = p->out_dtype == NSA_OUT_F32;
+  a.tinfo = geo.tinfo;
+  a.q_begin = geo.t_begin;
+  a.q_end = geo.t_end;
+  a.n_tiles = (geo.t_end - geo.t_begin + T - 1) / T;
+  return launch_attn<D, nsa::kModeDense>(qmap, kmap, vmap, a, st);
+}
+
+template <int D>
+int prefill_impl(const nsa_params_t* p, const void* q, const void* k, const void* v, const float* gates, void* out,
+                 int32_t* out_sel_idx, uint8_t* ws, cudaStream_t st, const float* phi_k = nullptr,
+                 const float* phi_v = nullptr) {
+  const PrefillLayout L = prefill_layout(p);
+  const int N = p->n_tokens, nv = p->n_video;
+  StageGeo geo{};
+  geo.q = q;
+  geo.k = k;
+  geo.v = v;
+  geo.rows = N;
+  geo.nv = nv;
+  geo.nsel_max = L.nsel;
+  geo.qt = q;
+  geo.qt_rows = N;
+  geo.t_begin = nv;  // the trailing text rows
+  geo.t_end = N;
+  geo.kd = k;
+  geo.vd = v;
+  geo.kd_rows = N;
+  geo.gates = gates;
+  geo.out = out;
+  int rc;
+  if (nv > 0 && (rc = video_stages<D>(p, geo, L, out_sel_idx, ws, st, phi_k, phi_v)) != NSA_OK) return rc;
+  return text_stage<D>(p, geo, st);
 }
 
 // Launch with programmatic stream serialisation: the kernel may start while the previous
@@ -509,24 +600,222 @@ int decode_impl(const nsa_params_t* p, const void* q, const void* kcache, const 
   return NSA_OK;
 }
 
-// Host-side checks of a packed batch; on success the per-sequence parameter sets are valid.
-int check_varlen(const nsa_params_t* params, const int32_t* cu, const int32_t* nv, int batch) {
-  int rc = check_common(params);
+// ------------------------------------------------------------------ packed batches
+// A plan of a packed batch, built on the host from cu_seqlens and the segment list.
+struct PackPlan {
+  int B = 0, S = 0;
+  long long N = 0;
+  int nv = 0, nt = 0;         // video stream rows, text stream rows
+  int kc_rows = 0;            // compressed rows of all sequences, each padded to 128
+  int nsel_cols = 0;          // selection blocks of all sequences
+  int nsel_max = 0;           // selection blocks of the longest video stream
+  bool gather = false;        // the video stream is not the batch itself (text precedes video)
+  std::vector<int> seg, seq;  // nsa::kPackSeg ints per segment, nsa::kPackSeq per sequence
+};
+
+int build_plan(const nsa_params_t* p, const int32_t* cu, int batch, const int32_t* seg_lens, const uint8_t* seg_video,
+               int nseg, PackPlan& P) {
+  int rc = check_common(p);
   if (rc != NSA_OK) return rc;
-  if (!cu || !nv || batch < 1 || cu[0] != 0 || cu[batch] != params->n_tokens) return NSA_ERR_INVALID_ARG;
+  if (!cu || batch < 1 || cu[0] != 0 || cu[batch] != p->n_tokens || nseg < 0 || (nseg > 0 && (!seg_lens || !seg_video)))
+    return NSA_ERR_INVALID_ARG;
+  P = PackPlan{};
+  P.B = batch;
+  P.S = nseg;
+  P.N = p->n_tokens;
+  P.seg.resize(static_cast<size_t>(nseg) * nsa::kPackSeg);
+  P.seq.resize(static_cast<size_t>(batch) * nsa::kPackSeq);
+  long long pos = 0;
+  int s = 0;
+  bool text_seen = false;
   for (int b = 0; b < batch; ++b) {
-    const int len = cu[b + 1] - cu[b];
-    if (len < 0 || nv[b] < 0 || nv[b] > len) return NSA_ERR_INVALID_ARG;
-    if (nsel_of(nv[b], params->sel_block) > 8192) return NSA_ERR_UNSUPPORTED;
+    if (cu[b + 1] < cu[b]) return NSA_ERR_INVALID_ARG;
+    const int v0 = P.nv;
+    int nvb = 0;
+    // the sequence's segments: first pass for its video count, second for the table
+    const int s_first = s;
+    while (pos < cu[b + 1]) {
+      if (s >= nseg || seg_lens[s] <= 0 || pos + seg_lens[s] > cu[b + 1]) return NSA_ERR_INVALID_ARG;
+      if (seg_video[s] > 1) return NSA_ERR_INVALID_ARG;
+      if (seg_video[s]) {
+        nvb += seg_lens[s];
+        if (text_seen) P.gather = true;
+      } else {
+        text_seen = true;
+      }
+      pos += seg_lens[s];
+      ++s;
+    }
+    const int ncmp = ncmp_of(nvb, p->cmp_block, p->cmp_stride);
+    const int nsel = nsel_of(nvb, p->sel_block);
+    int* sq = &P.seq[static_cast<size_t>(b) * nsa::kPackSeq];
+    sq[0] = v0;
+    sq[1] = nvb;
+    sq[2] = P.kc_rows;
+    sq[3] = ncmp;
+    sq[4] = P.nsel_cols;
+    sq[5] = nsel;
+    long long sp = cu[b];
+    int vidx = v0;
+    for (int x = s_first; x < s; ++x) {
+      int* sg = &P.seg[static_cast<size_t>(x) * nsa::kPackSeg];
+      sg[0] = static_cast<int>(sp);
+      sg[1] = seg_lens[x];
+      sg[2] = seg_video[x] ? 1 : 0;
+      sg[3] = seg_video[x] ? vidx : P.nt;
+      sg[4] = cu[b];
+      sg[5] = v0;
+      sg[6] = sq[2];
+      sg[7] = sq[4];
+      if (seg_video[x]) vidx += seg_lens[x];
+      else P.nt += seg_lens[x];
+      sp += seg_lens[x];
+    }
+    P.nv += nvb;
+    P.kc_rows += (ncmp + 127) / 128 * 128;
+    P.nsel_cols += nsel;
+    if (nsel > P.nsel_max) P.nsel_max = nsel;
   }
+  if (s != nseg) return NSA_ERR_INVALID_ARG;
+  if (P.nsel_max > 8192) return NSA_ERR_UNSUPPORTED;
+  // the packed video stream keeps every stage's indices in 32 bits
+  if (static_cast<long long>(P.nsel_cols) * p->num_kv_heads > (1LL << 30)) return NSA_ERR_UNSUPPORTED;
   return NSA_OK;
 }
 
-nsa_params_t varlen_sequence(const nsa_params_t* params, const int32_t* cu, const int32_t* nv, int b) {
-  nsa_params_t pb = *params;
-  pb.n_tokens = cu[b + 1] - cu[b];
-  pb.n_video = nv[b];
-  return pb;
+// Workspace of a packed call: the plan, the tables, the stream copies, then the NSA rows.
+struct PackLayout {
+  size_t seg, seq, vinfo, tinfo, row_tok, blk_tok, qv, kv, vv, qt, video, total;
+  PrefillLayout L;
+};
+
+PackLayout pack_layout(const nsa_params_t* p, const PackPlan& P) {
+  PackLayout W{};
+  const size_t hq = p->num_q_heads, hkv = p->num_kv_heads, d = p->head_dim;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + (bytes > 0 ? bytes : 1));
+    return at;
+  };
+  W.seg = take(P.seg.size() * 4);
+  W.seq = take(P.seq.size() * 4);
+  W.vinfo = take(static_cast<size_t>(P.nv) * 16);
+  W.tinfo = take(static_cast<size_t>(P.nt) * 8);
+  W.row_tok = take(static_cast<size_t>(P.kc_rows) * 4);
+  W.blk_tok = take(static_cast<size_t>(P.nsel_cols) * 4);
+  const size_t nvg = P.gather ? static_cast<size_t>(P.nv) : 0;
+  W.qv = take(nvg * hq * d * 2);
+  W.kv = take(nvg * hkv * d * 2);
+  W.vv = take(nvg * hkv * d * 2);
+  W.qt = take(static_cast<size_t>(P.nt) * hq * d * 2);
+  W.L = video_layout(P.nv, P.kc_rows, P.nsel_cols, P.nsel_max, p->num_q_heads, p->num_kv_heads, p->head_dim,
+                     p->top_n);
+  W.video = take(W.L.total);
+  W.total = off;
+  return W;
+}
+
+template <int D>
+int packed_impl(const nsa_params_t* p, const PackPlan& P, const PackLayout& W, const void* q, const void* k,
+                const void* v, const float* gates, void* out, int32_t* out_sel_idx, uint8_t* ws, cudaStream_t st) {
+  int rc;
+  // the plan's two tables, one copy each from host memory (a copy from pageable memory is
+  // staged by the driver before cudaMemcpyAsync returns, so the plan may go out of scope)
+  if (P.seg.size() > 0 &&
+      cudaMemcpyAsync(ws + W.seg, P.seg.data(), P.seg.size() * 4, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return NSA_ERR_CUDA;
+  if (cudaMemcpyAsync(ws + W.seq, P.seq.data(), P.seq.size() * 4, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return NSA_ERR_CUDA;
+  nsa::PackArgs pa{};
+  pa.seg = reinterpret_cast<const int*>(ws + W.seg);
+  pa.seq = reinterpret_cast<const int*>(ws + W.seq);
+  pa.nseg = P.S;
+  pa.nseq = P.B;
+  pa.ntok = P.N;
+  pa.hq = p->num_q_heads;
+  pa.hkv = p->num_kv_heads;
+  pa.d = D;
+  pa.cmp_stride = p->cmp_stride;
+  pa.sel_len = p->sel_block;
+  pa.q = static_cast<const __nv_bfloat16*>(q);
+  pa.k = static_cast<const __nv_bfloat16*>(k);
+  pa.v = static_cast<const __nv_bfloat16*>(v);
+  pa.qv = P.gather ? reinterpret_cast<__nv_bfloat16*>(ws + W.qv) : nullptr;
+  pa.kv = P.gather ? reinterpret_cast<__nv_bfloat16*>(ws + W.kv) : nullptr;
+  pa.vv = P.gather ? reinterpret_cast<__nv_bfloat16*>(ws + W.vv) : nullptr;
+  pa.qt = P.nt > 0 ? reinterpret_cast<__nv_bfloat16*>(ws + W.qt) : nullptr;
+  pa.vinfo = reinterpret_cast<int4*>(ws + W.vinfo);
+  pa.tinfo = reinterpret_cast<int2*>(ws + W.tinfo);
+  pa.row_tok = reinterpret_cast<int*>(ws + W.row_tok);
+  pa.blk_tok = reinterpret_cast<int*>(ws + W.blk_tok);
+  if (P.N > 0) {
+    nsa::pack_rows_kernel<<<static_cast<unsigned>((P.N + 7) / 8), 256, 0, st>>>(pa);
+    if ((rc = launch_status("pack_rows", st, false)) != NSA_OK) return rc;
+  }
+  if (P.nv > 0) {
+    nsa::pack_blocks_kernel<<<P.B, 256, 0, st>>>(pa);
+    if ((rc = launch_status("pack_blocks", st, false)) != NSA_OK) return rc;
+  }
+  StageGeo geo{};
+  geo.q = P.gather ? static_cast<const void*>(pa.qv) : q;
+  geo.k = P.gather ? static_cast<const void*>(pa.kv) : k;
+  geo.v = P.gather ? static_cast<const void*>(pa.vv) : v;
+  geo.rows = P.gather ? P.nv : static_cast<int>(P.N);
+  geo.nv = P.nv;
+  geo.vinfo = pa.vinfo;
+  geo.row_tok = pa.row_tok;
+  geo.blk_tok = pa.blk_tok;
+  geo.nsel_max = P.nsel_max;
+  geo.qt = pa.qt;
+  geo.qt_rows = P.nt;
+  geo.t_begin = 0;
+  geo.t_end = P.nt;
+  geo.tinfo = pa.tinfo;
+  geo.kd = k;
+  geo.vd = v;
+  geo.kd_rows = static_cast<int>(P.N);
+  geo.gates = gates;
+  geo.out = out;
+  if (P.nv > 0 && (rc = video_stages<D>(p, geo, W.L, out_sel_idx, ws + W.video, st, nullptr, nullptr)) != NSA_OK)
+    return rc;
+  return text_stage<D>(p, geo, st);
+}
+
+int packed_entry(const void* q, const void* k, const void* v, const float* gates, const int32_t* cu, int batch,
+                 const int32_t* seg_lens, const uint8_t* seg_video, int nseg, const nsa_params_t* params, void* out,
+                 int32_t* out_sel_idx, void* workspace, size_t workspace_bytes, void* stream) {
+  PackPlan P;
+  int rc = build_plan(params, cu, batch, seg_lens, seg_video, nseg, P);
+  if (rc != NSA_OK) return rc;
+  if (!q || !k || !v || !out || !workspace || (!gates && P.nv > 0)) return NSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (gates && !aligned16(gates)) ||
+      (out_sel_idx && !aligned16(out_sel_idx)) || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+    return NSA_ERR_INVALID_ARG;
+  const PackLayout W = pack_layout(params, P);
+  if (workspace_bytes < W.total) return NSA_ERR_WORKSPACE_TOO_SMALL;
+  if ((rc = check_device()) != NSA_OK) return rc;
+  auto* ws = static_cast<uint8_t*>(workspace);
+  auto st = static_cast<cudaStream_t>(stream);
+  stage_begin(st);
+  if (params->head_dim == 64) return packed_impl<64>(params, P, W, q, k, v, gates, out, out_sel_idx, ws, st);
+  return packed_impl<128>(params, P, W, q, k, v, gates, out, out_sel_idx, ws, st);
+}
+
+// The varlen layout (video prefix, then text, per sequence) as a segment list.
+void varlen_segments(const int32_t* cu, const int32_t* nv, int batch, std::vector<int32_t>& lens,
+                     std::vector<uint8_t>& vid) {
+  for (int b = 0; b < batch; ++b) {
+    const int len = cu[b + 1] - cu[b];
+    if (nv[b] > 0) {
+      lens.push_back(nv[b]);
+      vid.push_back(1);
+    }
+    if (len > nv[b]) {
+      lens.push_back(len - nv[b]);
+      vid.push_back(0);
+    }
+  }
 }
 
 }  // namespace
@@ -622,54 +911,58 @@ int nsa_prefill_phi(const void* q, const void* k, const void* v, const float* ga
   return prefill_entry(q, k, v, gates, phi_k, phi_v, params, out, out_sel_idx, workspace, workspace_bytes, stream);
 }
 
+size_t nsa_prefill_packed_workspace_size(const nsa_params_t* params, const int32_t* cu_seqlens, int batch,
+                                         const int32_t* seg_lens, const uint8_t* seg_video, int nseg) {
+  PackPlan P;
+  if (build_plan(params, cu_seqlens, batch, seg_lens, seg_video, nseg, P) != NSA_OK) return 0;
+  return pack_layout(params, P).total;
+}
+
+int nsa_prefill_packed(const void* q, const void* k, const void* v, const float* gates, const int32_t* cu_seqlens,
+                       int batch, const int32_t* seg_lens, const uint8_t* seg_video, int nseg,
+                       const nsa_params_t* params, void* out, int32_t* out_sel_idx, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  return packed_entry(q, k, v, gates, cu_seqlens, batch, seg_lens, seg_video, nseg, params, out, out_sel_idx,
+                      workspace, workspace_bytes, stream);
+}
+
+}  // extern "C"
+
+namespace {
+// The varlen call's host arrays as a segment list, after checking them.
+int varlen_to_segments(const nsa_params_t* params, const int32_t* cu, const int32_t* nv, int batch,
+                       std::vector<int32_t>& lens, std::vector<uint8_t>& vid) {
+  if (params == nullptr || !cu || !nv || batch < 1 || cu[0] != 0 || cu[batch] != params->n_tokens)
+    return NSA_ERR_INVALID_ARG;
+  for (int b = 0; b < batch; ++b) {
+    const int len = cu[b + 1] - cu[b];
+    if (len < 0 || nv[b] < 0 || nv[b] > len) return NSA_ERR_INVALID_ARG;
+  }
+  varlen_segments(cu, nv, batch, lens, vid);
+  return NSA_OK;
+}
+}  // namespace
+
+extern "C" {
+
 size_t nsa_prefill_varlen_workspace_size(const nsa_params_t* params, const int32_t* cu_seqlens,
                                          const int32_t* n_video, int batch) {
-  if (check_varlen(params, cu_seqlens, n_video, batch) != NSA_OK) return 0;
-  size_t most = 0;
-  for (int b = 0; b < batch; ++b) {
-    const nsa_params_t pb = varlen_sequence(params, cu_seqlens, n_video, b);
-    const size_t need = prefill_layout(&pb).total;
-    if (need > most) most = need;
-  }
-  return most;
+  std::vector<int32_t> lens;
+  std::vector<uint8_t> vid;
+  if (varlen_to_segments(params, cu_seqlens, n_video, batch, lens, vid) != NSA_OK) return 0;
+  return nsa_prefill_packed_workspace_size(params, cu_seqlens, batch, lens.data(), vid.data(),
+                                           static_cast<int>(lens.size()));
 }
 
 int nsa_prefill_varlen(const void* q, const void* k, const void* v, const float* gates, const int32_t* cu_seqlens,
                        const int32_t* n_video, int batch, const nsa_params_t* params, void* out,
                        int32_t* out_sel_idx, void* workspace, size_t workspace_bytes, void* stream) {
-  int rc = check_varlen(params, cu_seqlens, n_video, batch);
+  std::vector<int32_t> lens;
+  std::vector<uint8_t> vid;
+  const int rc = varlen_to_segments(params, cu_seqlens, n_video, batch, lens, vid);
   if (rc != NSA_OK) return rc;
-  long long video_rows = 0;
-  for (int b = 0; b < batch; ++b) video_rows += n_video[b];
-  if (!q || !k || !v || !out || !workspace || (!gates && video_rows > 0)) return NSA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (gates && !aligned16(gates)) ||
-      (out_sel_idx && !aligned16(out_sel_idx)) || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
-    return NSA_ERR_INVALID_ARG;
-  if (workspace_bytes < nsa_prefill_varlen_workspace_size(params, cu_seqlens, n_video, batch))
-    return NSA_ERR_WORKSPACE_TOO_SMALL;
-  if ((rc = check_device()) != NSA_OK) return rc;
-  auto* ws = static_cast<uint8_t*>(workspace);
-  auto st = static_cast<cudaStream_t>(stream);
-  const size_t hq = params->num_q_heads, hkv = params->num_kv_heads, d = params->head_dim;
-  const size_t out_elem = params->out_dtype == NSA_OUT_F32 ? 4 : 2;
-  stage_begin(st);
-  long long sel_row = 0;  // video rows of the earlier sequences
-  for (int b = 0; b < batch; ++b) {
-    const nsa_params_t pb = varlen_sequence(params, cu_seqlens, n_video, b);
-    if (pb.n_tokens == 0) continue;
-    const size_t t0 = static_cast<size_t>(cu_seqlens[b]);
-    const auto* qb = static_cast<const uint8_t*>(q) + t0 * hq * d * 2;
-    const auto* kb = static_cast<const uint8_t*>(k) + t0 * hkv * d * 2;
-    const auto* vb = static_cast<const uint8_t*>(v) + t0 * hkv * d * 2;
-    const float* gb = gates ? gates + t0 * hq * 3 : nullptr;
-    auto* ob = static_cast<uint8_t*>(out) + t0 * hq * d * out_elem;
-    int32_t* sb = out_sel_idx ? out_sel_idx + static_cast<size_t>(sel_row) * hkv * params->top_n : nullptr;
-    rc = params->head_dim == 64 ? prefill_impl<64>(&pb, qb, kb, vb, gb, ob, sb, ws, st)
-                                : prefill_impl<128>(&pb, qb, kb, vb, gb, ob, sb, ws, st);
-    if (rc != NSA_OK) return rc;
-    sel_row += pb.n_video;
-  }
-  return NSA_OK;
+  return packed_entry(q, k, v, gates, cu_seqlens, batch, lens.data(), vid.data(), static_cast<int>(lens.size()),
+                      params, out, out_sel_idx, workspace, workspace_bytes, stream);
 }
 
 int nsa_decode(const void* q, const void* kcache, const void* vcache, const void* kcmp, const void* vcmp,

@@ -36,11 +36,14 @@ __device__ __forceinline__ __nv_bfloat16 f64_to_bf16_rne(double x) {
 // src: [nseq][T][hkv][d] bf16; dst: [nseq][ncmp][hkv][d] bf16. blockIdx.z: 0 -> K, 1 -> V.
 // wk, wv: [hkv][l] fp32 weights of the learnable form, or both null for the mean.
 // Each thread handles one bf16x2 column pair of one (seq, block i, head g).
+// row_tok (packed batches; nseq = 1): [ncmp] the token row of every summary's first token,
+// or -1 for a row that pads a sequence's summaries to a multiple of 128 (written as zeros).
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ k,
                                                    const __nv_bfloat16* __restrict__ v,
                                                    __nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict__ vc,
                                                    const float* __restrict__ wk, const float* __restrict__ wv,
-                                                   int nseq, int T, int hkv, int d, int ncmp, int l, int s) {
+                                                   int nseq, int T, int hkv, int d, int ncmp, int l, int s,
+                                                   const int* __restrict__ row_tok) {
   const __nv_bfloat16* src = blockIdx.z == 0 ? k : v;
   __nv_bfloat16* dst = blockIdx.z == 0 ? kc : vc;
   const float* w = blockIdx.z == 0 ? wk : wv;
@@ -55,8 +58,14 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   const int i = static_cast<int>(rest % ncmp);
   const int b = static_cast<int>(rest / ncmp);
   const size_t row_elems = static_cast<size_t>(hkv) * d;
+  const long long tok0 = row_tok != nullptr ? row_tok[i] : static_cast<long long>(b) * T + static_cast<long long>(i) * s;
+  __nv_bfloat16* const out_row = dst + ((static_cast<size_t>(b) * ncmp + i) * hkv + g) * d;
+  if (tok0 < 0) {
+    reinterpret_cast<__nv_bfloat162*>(out_row)[p] = __floats2bfloat162_rn(0.f, 0.f);
+    return;
+  }
   const __nv_bfloat162* in = reinterpret_cast<const __nv_bfloat162*>(
-      src + (static_cast<size_t>(b) * T + static_cast<size_t>(i) * s) * row_elems + static_cast<size_t>(g) * d) + p;
+      src + static_cast<size_t>(tok0) * row_elems + static_cast<size_t>(g) * d) + p;
   double a0 = 0.0, a1 = 0.0;
   __nv_bfloat162 o;
   if (w == nullptr) {
@@ -79,7 +88,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
     o.x = f64_to_bf16_rne(a0);
     o.y = f64_to_bf16_rne(a1);
   }
-  reinterpret_cast<__nv_bfloat162*>(dst + ((static_cast<size_t>(b) * ncmp + i) * hkv + g) * d)[p] = o;
+  reinterpret_cast<__nv_bfloat162*>(out_row)[p] = o;
 }
 
 }  // namespace nsa

@@ -49,7 +49,19 @@ struct SelInvArgs {
   const float* gates;           // [N][hq][3] (g_cmp, g_sel, g_win)
   void* out;                    // [N][hq][D] rows < nv: the gated combine, bf16 or fp32
   int out_f32;
+  // Packed batches (null for one sequence): vinfo as in AttnArgs (token -> its sequence's
+  // first stream token, first selection block and its row in the batch); blk_tok [nsel]: the
+  // stream token where each selection block starts. Block j of a row's sequence is bucket
+  // column vinfo.z + j (nsel counts the blocks of all sequences), and out / gates use the
+  // row in the batch.
+  const int4* vinfo;
+  const int* blk_tok;
 };
+
+// Bucket column of block j of token t: its sequence's blocks come after the earlier sequences'.
+__device__ __forceinline__ int sel_block_col(const SelInvArgs& a, int t, int j) {
+  return a.vinfo != nullptr ? a.vinfo[t].z + j : j;
+}
 
 // Block 0 is kept by every token, so its buckets take one entry per token of their group:
 // those entries are counted (and, in the scatter, placed) per CTA in shared memory and
@@ -63,8 +75,12 @@ __global__ void __launch_bounds__(256) sel_count_kernel(const SelInvArgs a) {
        e += static_cast<long long>(gridDim.x) * blockDim.x) {
     const int j = a.sel_idx[e];
     const int g = static_cast<int>((e / a.top_n) % a.hkv);
-    if (j == 0 && g < 16) atomicAdd(&zero_cnt[g], 1);
-    else if (j >= 0 && j < a.nsel) atomicAdd(&a.cnt[g * a.nsel + j], 1);
+    if (j == 0 && g < 16 && a.vinfo == nullptr) {
+      atomicAdd(&zero_cnt[g], 1);
+    } else if (j >= 0 && j < a.nsel) {
+      const int t = static_cast<int>(e / (static_cast<long long>(a.top_n) * a.hkv));
+      atomicAdd(&a.cnt[g * a.nsel + sel_block_col(a, t, j)], 1);
+    }
   }
   __syncthreads();
   if (threadIdx.x < min(a.hkv, 16) && zero_cnt[threadIdx.x] > 0)
@@ -150,8 +166,9 @@ __global__ void __launch_bounds__(256) sel_scatter_kernel(const SelInvArgs a) {
     const long long tg = e / a.top_n;
     const int g = static_cast<int>(tg % a.hkv);
     const int t = static_cast<int>(tg / a.hkv);
-    const int key = g * a.nsel + (valid ? j : 0);
-    const bool agg = valid && j == 0 && g < 16;  // groups past 16 use the global counter directly
+    const int key = g * a.nsel + (valid ? sel_block_col(a, t, j) : 0);
+    // groups past 16, and the per-sequence block 0 of packed batches, use the global counter
+    const bool agg = valid && j == 0 && g < 16 && a.vinfo == nullptr;
     int local = 0;
     if (agg) local = atomicAdd(&zero_cnt[g], 1);
     else if (valid) local = atomicAdd(&a.cursor[key], 1);
@@ -389,10 +406,11 @@ __global__ void __launch_bounds__(kSelTileThreads, 1)
           if (u >= kSelKVStages && !warp_wait(&sm.kv_empty[kvs], ((u / kSelKVStages) - 1) & 1, abort_flag)) return false;
           if (lane == 0) {
             const int g = cur.key / a.nsel, j = cur.key % a.nsel;
+            const int k0 = a.blk_tok != nullptr ? a.blk_tok[j] : j * a.sel_len;  // first key token
             mbar_arrive_expect_tx(&sm.kv_full[kvs], kChunks * 2 * 64 * 128);
             for (int c = 0; c < kChunks; ++c) {
-              tma_load_3d(&kmap, &sm.kv_full[kvs], sm.k[kvs][c], c * 64, g, j * a.sel_len);
-              tma_load_3d(&vmap, &sm.kv_full[kvs], sm.v[kvs][c], c * 64, g, j * a.sel_len);
+              tma_load_3d(&kmap, &sm.kv_full[kvs], sm.k[kvs][c], c * 64, g, k0);
+              tma_load_3d(&vmap, &sm.kv_full[kvs], sm.v[kvs][c], c * 64, g, k0);
             }
           }
           __syncwarp();
@@ -490,7 +508,8 @@ __global__ void __launch_bounds__(kSelTileThreads, 1)
       const bool valid = tok < cnt && hh < G;
       const int ent = tok < cnt ? inf.ent[tok] : 0;
       const int t = ent >> 6;
-      const int key_hi = valid ? min(64, t + 1 - j * a.sel_len) : 0;  // keys j*64 + c, c < key_hi
+      const int k0 = a.blk_tok != nullptr ? a.blk_tok[j] : j * a.sel_len;
+      const int key_hi = valid ? min(64, t + 1 - k0) : 0;  // keys k0 + c, c < key_hi
       if (!warp_wait(&sm.s_full[w], jj & 1, abort_flag)) break;
       tc_fence_after();
       float s[64];
@@ -648,9 +667,12 @@ __global__ void __launch_bounds__(256, 4) sel_merge_kernel(const SelInvArgs a) {
   const size_t base = (static_cast<size_t>(t) * a.hkv + g) * a.top_n;
   // the combine's other inputs go out first: their latency overlaps the partials' loads
   const size_t orow = static_cast<size_t>(row) * D + lane * kPer;
-  const float gc = __ldg(a.gates + static_cast<size_t>(row) * 3 + 0);
-  const float gs = __ldg(a.gates + static_cast<size_t>(row) * 3 + 1);
-  const float gw = __ldg(a.gates + static_cast<size_t>(row) * 3 + 2);
+  // (packed) gates and out use the row's place in the batch
+  const size_t brow = a.vinfo != nullptr ? static_cast<size_t>(a.vinfo[t].w) * a.hq + h : static_cast<size_t>(row);
+  const size_t out_off = brow * D + lane * kPer;
+  const float gc = __ldg(a.gates + brow * 3 + 0);
+  const float gs = __ldg(a.gates + brow * 3 + 1);
+  const float gw = __ldg(a.gates + brow * 3 + 2);
   float oc[kPer], ow[kPer];
   if constexpr (kPer == 4) {
     const uint2 c2 = __ldg(reinterpret_cast<const uint2*>(a.o_cmp + orow));
@@ -742,13 +764,13 @@ __global__ void __launch_bounds__(256, 4) sel_merge_kernel(const SelInvArgs a) {
 #pragma unroll
   for (int u = 0; u < kPer; ++u) res[u] = gc * oc[u] + gs * (acc[u] * inv) + gw * ow[u];
   if (a.out_f32) {
-    float* dst = static_cast<float*>(a.out) + orow;
+    float* dst = static_cast<float*>(a.out) + out_off;
     if constexpr (kPer == 4)
       *reinterpret_cast<float4*>(dst) = make_float4(res[0], res[1], res[2], res[3]);
     else
       *reinterpret_cast<float2*>(dst) = make_float2(res[0], res[1]);
   } else {
-    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + orow;
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + out_off;
     if constexpr (kPer == 4)
       *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(res[0], res[1]), pack_bf16x2(res[2], res[3]));
     else

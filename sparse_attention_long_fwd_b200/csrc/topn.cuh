@@ -296,16 +296,18 @@ __device__ __forceinline__ void warp_topn_regs(int* list, const float* __restric
 
 // scores: [nitems][stride] fp32 (item = row * hkv + g; stride >= nsel); idx / idx_copy:
 // [nitems][top_n].
-// Row position t = row (prefill rows are token positions).
+// Row position t = row (prefill rows are token positions); in a packed batch (vinfo, see
+// AttnArgs) t is the row's position in its own sequence's video stream.
 // One warp per (row, group). kRegsOnly: every row has fewer than 2,048 candidate blocks and
 // top_n <= 32 (checked by the host), so only the register path runs and each warp needs just
 // the 64-entry candidate list in shared memory; otherwise each warp also has the score row,
 // the list and the bitmap of the shared-memory path.
-template <bool kRegsOnly>
+template <bool kRegsOnly, bool kPacked = false>
 __global__ void __launch_bounds__(kTopnWarps * 32) topn_kernel(const float* __restrict__ scores, int nitems, int hkv,
                                                                 int nsel, int stride, int sel_len, int top_n,
                                                                 int32_t* __restrict__ idx,
-                                                                int32_t* __restrict__ idx_copy) {
+                                                                int32_t* __restrict__ idx_copy,
+                                                                const int4* __restrict__ vinfo) {
   extern __shared__ float tsm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwords = (nsel + 31) / 32;
@@ -313,7 +315,8 @@ __global__ void __launch_bounds__(kTopnWarps * 32) topn_kernel(const float* __re
   int* list = kRegsOnly ? reinterpret_cast<int*>(sc) : reinterpret_cast<int*>(sc + nsel);
   uint32_t* bits = reinterpret_cast<uint32_t*>(list + nsel);
   for (int item = blockIdx.x * kTopnWarps + warp; item < nitems; item += gridDim.x * kTopnWarps) {
-    const int t = item / hkv;
+    const int row = item / hkv;
+    const int t = kPacked ? row - vinfo[row].x : row;
     const int jt = t / sel_len;
     if (jt >= nsel || (kRegsOnly && (top_n > 32 || jt >= 32 * 64))) {
       // cannot happen for valid arguments; never index past the row

@@ -31,7 +31,8 @@ EXPORTED = (
     "nsa_error_string", "nsa_get_device_error", "nsa_version", "nsa_profile_stages", "nsa_decode_noalloc",
     "nsa_prefill_varlen", "nsa_prefill_varlen_workspace_size", "nsa_compress_weighted", "nsa_prefill_phi",
     "nsa_gate_mlp", "nsa_gate_mlp_pooled", "nsa_gate_mlp_pooled_workspace_size", "nsa_backward",
-    "nsa_backward_workspace_size", "nsa_selftest_wait_timeout",
+    "nsa_backward_workspace_size", "nsa_selftest_wait_timeout", "nsa_prefill_packed",
+    "nsa_prefill_packed_workspace_size",
 )
 
 
@@ -83,6 +84,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.nsa_prefill_varlen.restype = I
     lib.nsa_prefill_varlen_workspace_size.argtypes = [PP, I32P, I32P, I]
     lib.nsa_prefill_varlen_workspace_size.restype = S
+    U8P = ctypes.POINTER(ctypes.c_uint8)
+    lib.nsa_prefill_packed.argtypes = [P, P, P, P, I32P, I, I32P, U8P, I, PP, P, P, P, S, P]
+    lib.nsa_prefill_packed.restype = I
+    lib.nsa_prefill_packed_workspace_size.argtypes = [PP, I32P, I, I32P, U8P, I]
+    lib.nsa_prefill_packed_workspace_size.restype = S
     lib.nsa_decode.argtypes = [P, P, P, P, P, P, P, PP, P, P, P, S, P]
     lib.nsa_decode.restype = I
     lib.nsa_decode_noalloc.argtypes = [P, P, P, P, P, P, P, PP, P, P, P]
@@ -171,6 +177,27 @@ def nsa_prefill_varlen(q, k, v, gates, cu_seqlens, n_video, params: NsaParams, o
 def nsa_prefill_varlen_workspace_size(params: NsaParams, cu_seqlens, n_video) -> int:
     cu, nv = _host_i32(cu_seqlens), _host_i32(n_video)
     return load_library().nsa_prefill_varlen_workspace_size(ctypes.byref(params), cu, nv, len(nv))
+
+
+def _host_u8(values):
+    vals = [int(x) for x in values]
+    return (ctypes.c_uint8 * max(len(vals), 1))(*vals)
+
+
+def nsa_prefill_packed(q, k, v, gates, cu_seqlens, seg_lens, seg_video, params: NsaParams, out, out_sel_idx,
+                       workspace, workspace_bytes: int, stream=None) -> int:
+    """Packed batch with video and text segments in any order; cu_seqlens ([B+1]), seg_lens and
+    seg_video ([S]) are host integer sequences."""
+    cu, sl, sv = _host_i32(cu_seqlens), _host_i32(seg_lens), _host_u8(seg_video)
+    return load_library().nsa_prefill_packed(_addr(q), _addr(k), _addr(v), _addr(gates), cu, len(cu) - 1, sl, sv,
+                                             len(seg_lens), ctypes.byref(params), _addr(out), _addr(out_sel_idx),
+                                             _addr(workspace), workspace_bytes, _stream(stream))
+
+
+def nsa_prefill_packed_workspace_size(params: NsaParams, cu_seqlens, seg_lens, seg_video) -> int:
+    cu, sl, sv = _host_i32(cu_seqlens), _host_i32(seg_lens), _host_u8(seg_video)
+    return int(load_library().nsa_prefill_packed_workspace_size(ctypes.byref(params), cu, len(cu) - 1, sl, sv,
+                                                                 len(seg_lens)))
 
 
 def nsa_decode(q, kcache, vcache, kcmp, vcmp, seq_lens, gates, params: NsaParams, out, out_sel_idx, workspace,
