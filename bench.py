@@ -636,6 +636,9 @@ def run_backward(args, dev, q, k, v, g, peaks, flush, world):
 
 def run_decode(args, dev, peaks, peaks_src, flush, world):
     w = WORKLOADS["decode64x128k"]
+    if args.decode_batch != w.batch:
+        from sparse_attention_long_fwd_b200.inputs import scaled
+        w = scaled(w, batch=args.decode_batch)
     q, kc, vc, g, sl = decode_inputs(w, seed=4, device=dev)
     kcmp, vcmp = nsa.compress(kc, vc)
     p = nsa.make_params(w.n_tokens, w.n_tokens, w.hq, w.hkv, w.d, top_n=w.top_n, window=w.window,
@@ -667,7 +670,8 @@ def run_decode(args, dev, peaks, peaks_src, flush, world):
     cmp_bytes += w.batch * min(w.window, w.n_tokens) * w.hkv * w.d * 2 * 2
     cmp_gbs = cmp_bytes / (stages["dec_cmp_and_window"] / 1e3) / 1e9
     del kc, vc
-    return {"workload": "decode64x128k: 64 sequences x 131,072-token bf16 cache, Hq=28, Hkv=4, d=128, n=16, w=512",
+    return {"workload": f"decode{w.batch}x128k: {w.batch} sequences x 131,072-token bf16 cache, Hq=28, Hkv=4, "
+                        f"d=128, n=16, w=512",
             "ms_per_step": round(ms, 4), "hbm_gbs": round(gbs * world, 1), "unit": "GB/s",
             "algorithmic_bytes_per_step": nbytes, "frac_of_peak": round(gbs / peaks["hbm_gbs"], 4),
             "frac_of_datasheet": round(gbs / DATASHEET["hbm_gbs"], 4), "datasheet_gbs": DATASHEET["hbm_gbs"],
@@ -777,6 +781,8 @@ def main():
     ap.add_argument("--no-gates", action="store_true", help="skip the gate-network and learnable-compression lines")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward measurement")
     ap.add_argument("--no-configs", action="store_true", help="skip the tiny and 36K-hybrid prefill lines")
+    ap.add_argument("--decode-batch", type=int, default=64,
+                    help="sequences of the decode line (a smaller batch for profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     args = ap.parse_args()

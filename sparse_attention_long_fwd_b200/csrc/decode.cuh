@@ -235,9 +235,10 @@ __global__ void __launch_bounds__(kDecWarps * 32) dec_cmp_kernel(const __nv_bflo
   }
 }
 
-// One CTA (256 threads) per (sequence, group).
+// One CTA (256 threads) per (sequence, group); two CTAs per SM, so the 64 x 4 (sequence,
+// group) pairs of a full batch run as one wave on 148 SMs.
 template <int D>
-__global__ void __launch_bounds__(256) dec_select_kernel(const int32_t* __restrict__ seq_lens, const DecArgs a,
+__global__ void __launch_bounds__(256, 2) dec_select_kernel(const int32_t* __restrict__ seq_lens, const DecArgs a,
                                                          int32_t* __restrict__ out_sel_idx) {
   grid_dependency_wait();  // dec_cmp_kernel's partials and logits
   grid_launch_dependents();

@@ -414,8 +414,9 @@ int video_stages(const nsa_params_t* p, const StageGeo& geo, const PrefillLayout
   sa.vinfo = geo.vinfo;
   sa.blk_tok = geo.blk_tok;
   CUtensorMap k64map, v64map, omap;
-  if (!nsa::make_tmap_f16_3d(&omap, ws + L.part_o, 64, static_cast<uint64_t>(L.part_rows), D / 64, 128,
-                             static_cast<uint64_t>(L.part_rows) * 128, 64, 32, 1) ||
+  // partial rows [part_rows][D] fp16: a store box is 32 rows x one 64-column half
+  if (!nsa::make_tmap_f16_3d(&omap, ws + L.part_o, 64, D / 64, static_cast<uint64_t>(L.part_rows), 128,
+                             static_cast<uint64_t>(D) * 2, 64, 1, 32) ||
       !nsa::make_tmap_bf16_3d(&k64map, geo.k, D, hkv, geo.rows, ks1, ks2, 64, 1, 64) ||
       !nsa::make_tmap_bf16_3d(&v64map, geo.v, D, hkv, geo.rows, ks1, ks2, 64, 1, 64))
     return NSA_ERR_CUDA;

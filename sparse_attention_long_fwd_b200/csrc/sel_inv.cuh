@@ -41,8 +41,9 @@ struct SelInvArgs {
   int* list;                    // [nv*hkv*top_n] bucketed entries: t * 64 + slot
   int* row_of;                  // [nv][hkv][top_n] first partial row of each (token, group, slot)
   const __nv_bfloat16* q;       // [nv][hq][D]
-  long long part_rows;          // rows per 64-column half of part_o (128 x the tile bound)
-  const __half* part_o;         // [D/64][part_rows][64] output / (sum * c_half) of each partial
+  long long part_rows;          // partial rows (128 x the tile bound)
+  const __half* part_o;         // [part_rows][D] output / (sum * c_half) of each partial, half h in
+                                // columns [64h, 64h+64): a row is one contiguous 2D-byte segment
   float4* part_ml;              // [part_rows] (max in log2 units, sum, c of half 0, c of half 1)
   const __half* o_cmp;          // [nv][hq][D] compressed branch
   const __half* o_win;          // [nv][hq][D] sliding-window branch
@@ -602,7 +603,7 @@ __global__ void __launch_bounds__(kSelTileThreads, 1)
         fence_proxy_async_smem();  // the TMA store reads the staged rows (async proxy)
         __syncwarp();
         if (lane == 0) {
-          tma_store_3d(&omap, stg, 0, (tile_begin + i) * 128 + q4 * 32, h);
+          tma_store_3d(&omap, stg, 0, h, (tile_begin + i) * 128 + q4 * 32);
           bulk_commit_group();
         }
       }
@@ -708,7 +709,7 @@ __global__ void __launch_bounds__(256, 4) sel_merge_kernel(const SelInvArgs a) {
   const float4 x1 = r1 >= 0 ? a.part_ml[r1] : none;
   const int half = (lane * kPer) >> 6;
   const int col = (lane * kPer) & 63;
-  const __half* po = a.part_o + static_cast<size_t>(half) * a.part_rows * 64 + col;
+  const __half* po = a.part_o + static_cast<size_t>(half) * 64 + col;
   float acc[kPer];
 #pragma unroll
   for (int u = 0; u < kPer; ++u) acc[u] = 0.f;
@@ -723,7 +724,7 @@ __global__ void __launch_bounds__(256, 4) sel_merge_kernel(const SelInvArgs a) {
     for (int k = 0; k < kMB; ++k) {
       prow[k] = __shfl_sync(0xffffffffu, lo ? r0 : r1, (s0 + k) & 31);
       if (s0 + k >= a.top_n) prow[k] = -1;
-      const __half* p = po + static_cast<size_t>(prow[k] < 0 ? 0 : prow[k]) * 64;
+      const __half* p = po + static_cast<size_t>(prow[k] < 0 ? 0 : prow[k]) * D;
       if (prow[k] >= 0) {
         if constexpr (kPer == 4) {
           const uint2 v = *reinterpret_cast<const uint2*>(p);
