@@ -1,0 +1,326 @@
+// backward_tc.cuh -- the compressed branch's key pass of the backward on tcgen05.
+//
+// For the compressed keys Kc, Vc (the block summaries the forward attended) the key pass
+// accumulates, over every (token, head) row r that sees key i,
+//   dVc[i] += g_r P[r, i] dO_r,   dKc[i] += dS[r, i] q_r,
+//   P[r, i] = 2^(scale log2e <q_r, Kc_i> - lse2_r),  dS = g_r P scale (<dO_r, Vc_i> - D_r),
+// with lse2_r and D_r = <dO_r, o_cmp_r> from the row pass (the gradient of the forward
+// defined in this library; the pages train the model end to end, shd-paper.top page
+// "VideoNSA: Native Sparse Attention Scales Video Understanding", abstract).
+//
+// One CTA per (tile of 128 compressed keys, KV group, segment of tokens). Its keys sit in
+// the 128 TMEM lanes (M = 128) for the whole item; the rows stream in chunks of 64 (T
+// tokens x G heads, a 3-D TMA box like the forward's query tiles) through two stages:
+//   S^T = Kc Q^T and dP^T = Vc dO^T   (M = 128 keys, N = 64 rows, K = d; TMEM columns 0, 64)
+//   softmax warps: P g and dS as bf16 into TMEM (columns 128 and 160)
+//   dV += (P g)^T-rows x dO, dK += dS x Q   (A from TMEM, B = the stage's dO / Q read
+//                                            MN-major; accumulators in columns 256, 384)
+// The score MMAs of chunk c are issued before the value MMAs of chunk c-1, so they overlap
+// its softmax. P and dS of chunk c are stored only once the MMAs of chunk c-1 that read
+// those columns have finished (write-after-read on the same TMEM columns). At the end each
+// key's dVc, dKc rows are added to the global sums (segments of one key tile share rows).
+// Warp roles: warp 0 loads (TMA, and the rows' lse2 / D / gate / token), warp 1 owns TMEM
+// and issues the MMAs, warps 2..9 (two warpgroups) take 32 of a chunk's 64 rows each.
+// Every wait is bounded (sm100.cuh).
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+#include "sm100.cuh"
+#include "attn_tc.cuh"
+#include "backward.cuh"
+
+namespace nsa {
+
+constexpr int kBtKeys = 128;   // compressed keys per item (MMA M)
+constexpr int kBtRows = 64;    // rows per chunk (MMA N of the score products)
+constexpr int kBtThreads = 64 + 256;
+constexpr int kBtSegTokens = 4096;  // tokens per item segment
+
+template <int D>
+struct BtSmem {
+  static constexpr int kChunks = D / 64;
+  alignas(1024) uint8_t kc[kChunks][kBtKeys * 128];
+  alignas(1024) uint8_t vc[kChunks][kBtKeys * 128];
+  alignas(1024) uint8_t q[2][kChunks][kBtRows * 128];
+  alignas(1024) uint8_t dout[2][kChunks][kBtRows * 128];
+  float4 rowc[2][kBtRows];  // per row: (lse2, D, gate, token as int bits; -1: no row)
+  uint64_t kv_full, q_full[2], q_empty[2], sd_full, sd_free, p_full, pv_done, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kBtThreads, 1)
+    bwd_cmp_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap dmap,
+                      const __grid_constant__ CUtensorMap kcmap, const __grid_constant__ CUtensorMap vcmap,
+                      const BwdArgs a, int nseg) {
+  using Smem = BtSmem<D>;
+  constexpr int kChunks = Smem::kChunks;
+  constexpr uint32_t kColS = 0, kColDP = 64, kColP = 128, kColDS = 160, kColDV = 256, kColDK = 384;
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = a.G;
+  const int T = kBtRows / G;  // tokens per chunk
+  // ---- the item: key tile (heaviest first: early keys are seen by the most tokens), group, segment
+  const int nkt = (a.ncmp + kBtKeys - 1) / kBtKeys;
+  const int seg = blockIdx.x % nseg;
+  const int g = (blockIdx.x / nseg) % a.hkv;
+  const int kt = blockIdx.x / (nseg * a.hkv);
+  if (kt >= nkt) return;
+  const int key0 = kt * kBtKeys;
+  const int nkeys = min(kBtKeys, a.ncmp - key0);
+  const int tok_lo = max(seg * kBtSegTokens, key0 * a.cmp_stride + a.cmp_len - 1);
+  const int tok_hi = min((seg + 1) * kBtSegTokens, a.nv);
+  if (tok_lo >= tok_hi) return;  // uniform across the CTA, before any barrier or TMEM
+  const int nch = (tok_hi - tok_lo + T - 1) / T;
+
+  if (tid == 0) {
+    mbar_init(&sm.kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.q_full[s], 1 + 32);  // the TMA's expect_tx arrival + the 32 row-constant lanes
+      mbar_init(&sm.q_empty[s], 1);
+    }
+    mbar_init(&sm.sd_full, 1);
+    mbar_init(&sm.sd_free, 8);
+    mbar_init(&sm.p_full, 8);
+    mbar_init(&sm.pv_done, 1);
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp >= 2) {
+    // rows T*G .. 63 of the row stages are never written by TMA: keep them finite (zero), as
+    // the value products multiply them by P = dS = 0
+    const int r0 = T * G;
+    const int per = (kBtRows - r0) * 8;  // 16-byte units per (stage, tensor, chunk)
+    for (int i = tid - 64; i < 2 * 2 * kChunks * per; i += 256) {
+      const int u = i % per, rest = i / per;
+      const int c = rest % kChunks, tq = (rest / kChunks) % 2, s = rest / (2 * kChunks);
+      uint8_t* base = tq == 0 ? sm.q[s][c] : sm.dout[s][c];
+      *reinterpret_cast<uint4*>(base + (r0 + u / 8) * 128 + (u % 8) * 16) = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort_flag = &sm.abort_flag;
+  int q_issued = 0;     // producer: row chunks whose TMA was issued
+  bool leader = false;  // MMA warp: the lane that issues every tcgen05 op
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ loads
+    if (lane == 0) {
+      tma_prefetch_desc(&qmap);
+      tma_prefetch_desc(&dmap);
+      mbar_arrive_expect_tx(&sm.kv_full, 2 * kChunks * kBtKeys * 128);
+      for (int c = 0; c < kChunks; ++c) {
+        tma_load_3d(&kcmap, &sm.kv_full, sm.kc[c], c * 64, g, key0);
+        tma_load_3d(&vcmap, &sm.kv_full, sm.vc[c], c * 64, g, key0);
+      }
+    }
+    for (int c = 0; c < nch; ++c) {
+      const int s = c & 1;
+      if (c >= 2 && !__all_sync(0xffffffffu, mbar_wait(&sm.q_empty[s], ((c - 2) >> 1) & 1, abort_flag))) break;
+      const int t0 = tok_lo + c * T;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&sm.q_full[s], 2 * kChunks * T * G * 128);
+        for (int ch = 0; ch < kChunks; ++ch) {
+          tma_load_3d(&qmap, &sm.q_full[s], sm.q[s][ch], ch * 64, g * G, t0);
+          tma_load_3d(&dmap, &sm.q_full[s], sm.dout[s][ch], ch * 64, g * G, t0);
+        }
+      }
+      q_issued = c + 1;
+      // the rows' constants: (lse2, D) from the row pass, the compressed branch's gate, token
+#pragma unroll
+      for (int k = 0; k < kBtRows / 32; ++k) {
+        const int r = lane + 32 * k;
+        const int t = t0 + r / G, h = g * G + r % G;
+        float4 v = make_float4(-INFINITY, 0.f, 0.f, __int_as_float(-1));
+        if (r < T * G && t < tok_hi) {
+          const size_t o = (static_cast<size_t>(t) * a.hq + h) * 3;
+          const float2 st = a.stats[o + kBwdCmp];
+          v = make_float4(st.x, st.y, a.gates[o + kBwdCmp], __int_as_float(t));
+        }
+        sm.rowc[s][r] = v;
+      }
+      mbar_arrive(&sm.q_full[s]);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    leader = elect_one_sync();
+    constexpr uint32_t idS = idesc_bf16_f32(kBtKeys, kBtRows, false, false);
+    constexpr uint32_t idV = idesc_bf16_f32(kBtKeys, D, false, true);
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+    };
+    bool ok = wait_all(&sm.kv_full, 0);
+    for (int c = 0; ok && c <= nch; ++c) {
+      if (c < nch) {
+        // S^T and dP^T of chunk c (their columns were read by the softmax of chunk c - 1)
+        const int s = c & 1;
+        if (!wait_all(&sm.q_full[s], (c >> 1) & 1) || (c >= 1 && !wait_all(&sm.sd_free, (c - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (leader) {
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const int ch = k >> 2, kk = k & 3;
+            umma_bf16_ss(tmem + kColS, sdesc_sw128(smem_u32(sm.kc[ch]) + kk * 32, 16, 1024),
+                         sdesc_sw128(smem_u32(sm.q[s][ch]) + kk * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const int ch = k >> 2, kk = k & 3;
+            umma_bf16_ss(tmem + kColDP, sdesc_sw128(smem_u32(sm.vc[ch]) + kk * 32, 16, 1024),
+                         sdesc_sw128(smem_u32(sm.dout[s][ch]) + kk * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
+          }
+          umma_commit(&sm.sd_full);
+        }
+        __syncwarp();
+      }
+      if (c >= 1) {
+        // dV += (P g) x dO and dK += dS x Q over chunk c - 1's 64 rows (16 per MMA)
+        const int cp = c - 1, sp = cp & 1;
+        if (!wait_all(&sm.p_full, cp & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (leader) {
+          const uint64_t ddesc = sdesc_sw128(smem_u32(sm.dout[sp][0]), kBtRows * 128, 1024);
+          const uint64_t qdesc = sdesc_sw128(smem_u32(sm.q[sp][0]), kBtRows * 128, 1024);
+#pragma unroll
+          for (int k = 0; k < kBtRows / 16; ++k) {
+            const uint32_t acc = (cp > 0 || k > 0) ? 1u : 0u;
+            umma_bf16_ts(tmem + kColDV, tmem + kColP + k * 8, ddesc + static_cast<uint64_t>(k * (2048 >> 4)), idV,
+                         acc);
+            umma_bf16_ts(tmem + kColDK, tmem + kColDS + k * 8, qdesc + static_cast<uint64_t>(k * (2048 >> 4)), idV,
+                         acc);
+          }
+          umma_commit(&sm.pv_done);
+          umma_commit(&sm.q_empty[sp]);
+        }
+        __syncwarp();
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax warps
+    const int sw = warp - 2;
+    const int wg = sw >> 2;          // rows [32 wg, 32 wg + 32) of each chunk
+    const int q4 = warp & 3;         // TMEM lane quadrant
+    const int kl = q4 * 32 + lane;   // this thread's key (TMEM lane)
+    const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const int key = key0 + kl;
+    const bool key_ok = kl < nkeys;
+    const int tk = key * a.cmp_stride + a.cmp_len - 1;  // first token that sees this key
+    const float sl2 = a.sl2, scale = a.scale;
+    bool ok = true;
+    for (int c = 0; c < nch && ok; ++c) {
+      const int s = c & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.sd_full, c & 1, abort_flag) &&
+                                       mbar_wait(&sm.q_full[s], (c >> 1) & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      float sv[32], dp[32];
+      __syncwarp();
+      tmem_ld32(trow + kColS + 32 * wg, sv);
+      tmem_ld32(trow + kColDP + 32 * wg, dp);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.sd_free);
+      uint32_t pp[16], pd[16];
+#pragma unroll
+      for (int j = 0; j < 32; j += 2) {
+        float pg[2], ds[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float4 rc = sm.rowc[s][32 * wg + j + e];
+          const int t = __float_as_int(rc.w);
+          const bool vis = key_ok && t >= tk && rc.x != -INFINITY;
+          const float p = vis ? ex2_approx(fmaf(sv[j + e], sl2, -rc.x)) : 0.f;
+          pg[e] = p * rc.z;
+          ds[e] = pg[e] * scale * (dp[j + e] - rc.y);
+        }
+        pp[j / 2] = pack_bf16x2(pg[0], pg[1]);
+        pd[j / 2] = pack_bf16x2(ds[0], ds[1]);
+      }
+      // P and dS of chunk c go over the columns the value MMAs of chunk c - 1 read
+      if (c >= 1) ok = mbar_wait(&sm.pv_done, (c - 1) & 1, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      tmem_st16(trow + kColP + 16 * wg, pp);
+      tmem_st16(trow + kColDS + 16 * wg, pd);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.p_full);
+    }
+    // ---- the item's sums: this warpgroup's half of the key's dVc and dKc rows
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done, (nch - 1) & 1, abort_flag));
+    if (ok) {
+      tc_fence_after();
+      constexpr int kHalf = D / 2;
+      float* dvr = a.dvc + (static_cast<size_t>(key) * a.hkv + g) * D + wg * kHalf;
+      float* dkr = a.dkc + (static_cast<size_t>(key) * a.hkv + g) * D + wg * kHalf;
+#pragma unroll
+      for (int x = 0; x < kHalf / 32; ++x) {
+        float v[32], kk[32];
+        __syncwarp();
+        tmem_ld32(trow + kColDV + wg * kHalf + 32 * x, v);
+        tmem_ld32(trow + kColDK + wg * kHalf + 32 * x, kk);
+        tmem_wait_ld();
+        if (key_ok) {
+#pragma unroll
+          for (int u = 0; u < 32; u += 4) {
+            atomicAdd(reinterpret_cast<float4*>(dvr + 32 * x + u), make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]));
+            atomicAdd(reinterpret_cast<float4*>(dkr + 32 * x + u),
+                      make_float4(kk[u], kk[u + 1], kk[u + 2], kk[u + 3]));
+          }
+        }
+      }
+    }
+    tc_fence_before();
+  }
+
+  // ------------------------------------------------------------------ teardown
+  __syncthreads();
+  if (*abort_flag) {
+    // drain: wait (bounded) for the loads issued and for MMAs in flight, so no async write
+    // lands after the CTA exits
+    if (warp == 0 && lane == 0) {
+      long long t_start = clock64();
+      while (!mbar_test(&sm.kv_full, 0) && clock64() - t_start < kWaitCycles) {
+      }
+      for (int c = q_issued - 2 > 0 ? q_issued - 2 : 0; c < q_issued; ++c) {
+        t_start = clock64();
+        while (!mbar_test(&sm.q_full[c & 1], (c >> 1) & 1) && clock64() - t_start < kWaitCycles) {
+        }
+      }
+    }
+    if (warp == 1 && leader) {
+      umma_commit(&sm.drain);
+      const long long t_start = clock64();
+      while (!mbar_test(&sm.drain, 0) && clock64() - t_start < kWaitCycles) {
+      }
+    }
+    __syncwarp();
+    __syncthreads();
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace nsa

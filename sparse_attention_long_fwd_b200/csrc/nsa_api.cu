@@ -21,6 +21,7 @@
 #include "decode.cuh"
 #include "gate.cuh"
 #include "backward.cuh"
+#include "backward_tc.cuh"
 #include "pack.cuh"
 
 namespace nsa {
@@ -1309,11 +1310,26 @@ int backward_impl(const nsa_params_t* p, const void* q, const void* k, const voi
     if ((rc = launch_status("bwd_sel_scan", st, false)) != NSA_OK) return rc;
     nsa::sel_scatter_kernel<<<ebl, 256, 0, st>>>(sa);
     if ((rc = launch_status("bwd_sel_scatter", st)) != NSA_OK) return rc;
-    // key pass, one launch per branch
+    // key pass, one launch per branch; the compressed keys' on tcgen05 (128 keys x 64 rows)
     if (L.ncmp > 0) {
-      const long long items = static_cast<long long>((L.ncmp + nsa::kBwdChunk - 1) / nsa::kBwdChunk) * hkv *
-                              ((nv + nsa::kBwdSegCmp - 1) / nsa::kBwdSegCmp);
-      if ((rc = launch_bwd_key<D, nsa::kBwdCmp>(a, items, st)) != NSA_OK) return rc;
+      CUtensorMap bqmap, bdmap, bkcmap, bvcmap;
+      const int Tb = nsa::kBtRows / G;
+      const uint64_t qs1 = static_cast<uint64_t>(D) * 2, qs2 = static_cast<uint64_t>(hq) * D * 2;
+      const uint64_t ks1 = static_cast<uint64_t>(D) * 2, ks2 = static_cast<uint64_t>(hkv) * D * 2;
+      if (!nsa::make_tmap_bf16_3d(&bqmap, q, D, hq, N, qs1, qs2, 64, G, Tb) ||
+          !nsa::make_tmap_bf16_3d(&bdmap, d_out, D, hq, N, qs1, qs2, 64, G, Tb) ||
+          !nsa::make_tmap_bf16_3d(&bkcmap, ws + L.kc, D, hkv, L.ncmp, ks1, ks2, 64, 1, nsa::kBtKeys) ||
+          !nsa::make_tmap_bf16_3d(&bvcmap, ws + L.vc, D, hkv, L.ncmp, ks1, ks2, 64, 1, nsa::kBtKeys))
+        return NSA_ERR_CUDA;
+      const int nseg = (nv + nsa::kBtSegTokens - 1) / nsa::kBtSegTokens;
+      const long long items =
+          static_cast<long long>((L.ncmp + nsa::kBtKeys - 1) / nsa::kBtKeys) * hkv * nseg;
+      const size_t smem = sizeof(nsa::BtSmem<D>) + 1024;
+      auto kern = nsa::bwd_cmp_tc_kernel<D>;
+      if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
+      if (items > 0x7fffffffLL) return NSA_ERR_UNSUPPORTED;
+      kern<<<static_cast<unsigned>(items), nsa::kBtThreads, smem, st>>>(bqmap, bdmap, bkcmap, bvcmap, a, nseg);
+      if ((rc = launch_status("bwd_key_cmp", st)) != NSA_OK) return rc;
     }
     {
       const long long segs = entries / nsa::kBwdSegSel + m + 1;  // >= sum over buckets of ceil(count / segment)
