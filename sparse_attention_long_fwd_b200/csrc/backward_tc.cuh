@@ -1,14 +1,18 @@
-// backward_tc.cuh -- the compressed branch's key pass of the backward on tcgen05.
+// backward_tc.cuh -- key passes of the backward on tcgen05: the compressed branch, the
+// sliding window and the dense text rows (the branches whose rows are runs of consecutive
+// tokens).
 //
-// For the compressed keys Kc, Vc (the block summaries the forward attended) the key pass
-// accumulates, over every (token, head) row r that sees key i,
-//   dVc[i] += g_r P[r, i] dO_r,   dKc[i] += dS[r, i] q_r,
-//   P[r, i] = 2^(scale log2e <q_r, Kc_i> - lse2_r),  dS = g_r P scale (<dO_r, Vc_i> - D_r),
-// with lse2_r and D_r = <dO_r, o_cmp_r> from the row pass (the gradient of the forward
+// For a branch's keys K, V the key pass accumulates, over every (token, head) row r that
+// sees key i,
+//   dV[i] += g_r P[r, i] dO_r,   dK[i] += dS[r, i] q_r,
+//   P[r, i] = 2^(scale log2e <q_r, K_i> - lse2_r),  dS = g_r P scale (<dO_r, V_i> - D_r),
+// with lse2_r and D_r = <dO_r, o_b,r> from the row pass (the gradient of the forward
 // defined in this library; the pages train the model end to end, shd-paper.top page
-// "VideoNSA: Native Sparse Attention Scales Video Understanding", abstract).
+// "VideoNSA: Native Sparse Attention Scales Video Understanding", abstract). The keys are
+// the compressed summaries Kc, Vc (row r of token t sees block i iff i*s + l - 1 <= t), the
+// tokens of the window (t - w < i <= t) or, for text rows, every token i <= t (gate 1).
 //
-// One CTA per (tile of 128 compressed keys, KV group, segment of tokens). Its keys sit in
+// One CTA per (tile of 128 keys, KV group, segment of tokens). Its keys sit in
 // the 128 TMEM lanes (M = 128) for the whole item; the rows stream in chunks of 64 (T
 // tokens x G heads, a 3-D TMA box like the forward's query tiles) through two stages:
 //   S^T = Kc Q^T and dP^T = Vc dO^T   (M = 128 keys, N = 64 rows, K = d; TMEM columns 0, 64)
@@ -49,9 +53,12 @@ struct BtSmem {
   int abort_flag;
 };
 
-template <int D>
+// BR: kBwdCmp (keys: compressed rows, rows: video tokens), kBwdWin (keys: video tokens,
+// rows: the video tokens within the window after them), kBwdDense (keys: all tokens, rows: the
+// text tokens after them).
+template <int D, int BR>
 __global__ void __launch_bounds__(kBtThreads, 1)
-    bwd_cmp_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap dmap,
+    bwd_key_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap dmap,
                       const __grid_constant__ CUtensorMap kcmap, const __grid_constant__ CUtensorMap vcmap,
                       const BwdArgs a, int nseg) {
   using Smem = BtSmem<D>;
@@ -63,15 +70,26 @@ __global__ void __launch_bounds__(kBtThreads, 1)
   const int G = a.G;
   const int T = kBtRows / G;  // tokens per chunk
   // ---- the item: key tile (heaviest first: early keys are seen by the most tokens), group, segment
-  const int nkt = (a.ncmp + kBtKeys - 1) / kBtKeys;
+  const int nkeys_all = BR == kBwdCmp ? a.ncmp : (BR == kBwdWin ? a.nv : a.N);
+  const int nkt = (nkeys_all + kBtKeys - 1) / kBtKeys;
   const int seg = blockIdx.x % nseg;
   const int g = (blockIdx.x / nseg) % a.hkv;
   const int kt = blockIdx.x / (nseg * a.hkv);
   if (kt >= nkt) return;
   const int key0 = kt * kBtKeys;
-  const int nkeys = min(kBtKeys, a.ncmp - key0);
-  const int tok_lo = max(seg * kBtSegTokens, key0 * a.cmp_stride + a.cmp_len - 1);
-  const int tok_hi = min((seg + 1) * kBtSegTokens, a.nv);
+  const int nkeys = min(kBtKeys, nkeys_all - key0);
+  // rows: the tokens that see at least one of the tile's keys, cut into segments
+  int tok_lo, tok_hi;
+  if (BR == kBwdCmp) {
+    tok_lo = max(seg * kBtSegTokens, key0 * a.cmp_stride + a.cmp_len - 1);
+    tok_hi = min((seg + 1) * kBtSegTokens, a.nv);
+  } else if (BR == kBwdWin) {
+    tok_lo = max(key0 + seg * kBtSegTokens, key0);
+    tok_hi = min(min(key0 + (seg + 1) * kBtSegTokens, key0 + nkeys - 1 + a.window), a.nv);
+  } else {
+    tok_lo = max(a.nv + seg * kBtSegTokens, key0);
+    tok_hi = min(a.nv + (seg + 1) * kBtSegTokens, a.N);
+  }
   if (tok_lo >= tok_hi) return;  // uniform across the CTA, before any barrier or TMEM
   const int nch = (tok_hi - tok_lo + T - 1) / T;
 
@@ -144,9 +162,10 @@ __global__ void __launch_bounds__(kBtThreads, 1)
         const int t = t0 + r / G, h = g * G + r % G;
         float4 v = make_float4(-INFINITY, 0.f, 0.f, __int_as_float(-1));
         if (r < T * G && t < tok_hi) {
+          // text rows keep their statistics in slot 0 and have no gate
           const size_t o = (static_cast<size_t>(t) * a.hq + h) * 3;
-          const float2 st = a.stats[o + kBwdCmp];
-          v = make_float4(st.x, st.y, a.gates[o + kBwdCmp], __int_as_float(t));
+          const float2 st = a.stats[o + (BR == kBwdDense ? 0 : BR)];
+          v = make_float4(st.x, st.y, BR == kBwdDense ? 1.f : a.gates[o + BR], __int_as_float(t));
         }
         sm.rowc[s][r] = v;
       }
@@ -221,7 +240,9 @@ __global__ void __launch_bounds__(kBtThreads, 1)
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int key = key0 + kl;
     const bool key_ok = kl < nkeys;
-    const int tk = key * a.cmp_stride + a.cmp_len - 1;  // first token that sees this key
+    // the tokens that see this key: [tk, tk_end]
+    const int tk = BR == kBwdCmp ? key * a.cmp_stride + a.cmp_len - 1 : key;
+    const int tk_end = BR == kBwdWin ? key + a.window - 1 : 0x7fffffff;
     const float sl2 = a.sl2, scale = a.scale;
     bool ok = true;
     for (int c = 0; c < nch && ok; ++c) {
@@ -246,7 +267,7 @@ __global__ void __launch_bounds__(kBtThreads, 1)
         for (int e = 0; e < 2; ++e) {
           const float4 rc = sm.rowc[s][32 * wg + j + e];
           const int t = __float_as_int(rc.w);
-          const bool vis = key_ok && t >= tk && rc.x != -INFINITY;
+          const bool vis = key_ok && t >= tk && t <= tk_end && rc.x != -INFINITY;
           const float p = vis ? ex2_approx(fmaf(sv[j + e], sl2, -rc.x)) : 0.f;
           pg[e] = p * rc.z;
           ds[e] = pg[e] * scale * (dp[j + e] - rc.y);
@@ -271,8 +292,8 @@ __global__ void __launch_bounds__(kBtThreads, 1)
     if (ok) {
       tc_fence_after();
       constexpr int kHalf = D / 2;
-      float* dvr = a.dvc + (static_cast<size_t>(key) * a.hkv + g) * D + wg * kHalf;
-      float* dkr = a.dkc + (static_cast<size_t>(key) * a.hkv + g) * D + wg * kHalf;
+      float* dvr = (BR == kBwdCmp ? a.dvc : a.dv) + (static_cast<size_t>(key) * a.hkv + g) * D + wg * kHalf;
+      float* dkr = (BR == kBwdCmp ? a.dkc : a.dk) + (static_cast<size_t>(key) * a.hkv + g) * D + wg * kHalf;
 #pragma unroll
       for (int x = 0; x < kHalf / 32; ++x) {
         float v[32], kk[32];
@@ -324,3 +345,4 @@ __global__ void __launch_bounds__(kBtThreads, 1)
 }
 
 }  // namespace nsa
+

@@ -1211,6 +1211,33 @@ int launch_bwd_key(const nsa::BwdArgs& a, long long n_items, cudaStream_t st) {
                        st);
 }
 
+// The tcgen05 key pass of one branch: keys from (kk, vk) with `key_rows` rows in their tensor
+// maps; `span` tokens of rows bound the segments per key tile.
+template <int D, int BR>
+int launch_bwd_key_tc(const nsa::BwdArgs& a, const void* q, const void* d_out, const void* kk, const void* vk,
+                      int key_rows, int span, cudaStream_t st) {
+  const int G = a.G, hq = a.hq, hkv = a.hkv, N = a.N;
+  const int nkeys = BR == nsa::kBwdCmp ? a.ncmp : (BR == nsa::kBwdWin ? a.nv : a.N);
+  if (nkeys <= 0) return NSA_OK;
+  CUtensorMap qmap, dmap, kmap, vmap;
+  const int Tb = nsa::kBtRows / G;
+  const uint64_t qs1 = static_cast<uint64_t>(D) * 2, qs2 = static_cast<uint64_t>(hq) * D * 2;
+  const uint64_t ks1 = static_cast<uint64_t>(D) * 2, ks2 = static_cast<uint64_t>(hkv) * D * 2;
+  if (!nsa::make_tmap_bf16_3d(&qmap, q, D, hq, N, qs1, qs2, 64, G, Tb) ||
+      !nsa::make_tmap_bf16_3d(&dmap, d_out, D, hq, N, qs1, qs2, 64, G, Tb) ||
+      !nsa::make_tmap_bf16_3d(&kmap, kk, D, hkv, key_rows, ks1, ks2, 64, 1, nsa::kBtKeys) ||
+      !nsa::make_tmap_bf16_3d(&vmap, vk, D, hkv, key_rows, ks1, ks2, 64, 1, nsa::kBtKeys))
+    return NSA_ERR_CUDA;
+  const int nseg = (span + nsa::kBtSegTokens - 1) / nsa::kBtSegTokens;
+  const long long items = static_cast<long long>((nkeys + nsa::kBtKeys - 1) / nsa::kBtKeys) * hkv * nseg;
+  if (items > 0x7fffffffLL) return NSA_ERR_UNSUPPORTED;
+  const size_t smem = sizeof(nsa::BtSmem<D>) + 1024;
+  auto kern = nsa::bwd_key_tc_kernel<D, BR>;
+  if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
+  kern<<<static_cast<unsigned>(items), nsa::kBtThreads, smem, st>>>(qmap, dmap, kmap, vmap, a, nseg);
+  return launch_status(BR == nsa::kBwdCmp ? "bwd_key_cmp" : BR == nsa::kBwdWin ? "bwd_key_win" : "bwd_key_dense", st);
+}
+
 template <int D>
 int backward_impl(const nsa_params_t* p, const void* q, const void* k, const void* v, const float* gates,
                   const void* d_out, const int32_t* sel_idx, const uint8_t* fwd_ws, const float* phi_k,
@@ -1310,41 +1337,20 @@ int backward_impl(const nsa_params_t* p, const void* q, const void* k, const voi
     if ((rc = launch_status("bwd_sel_scan", st, false)) != NSA_OK) return rc;
     nsa::sel_scatter_kernel<<<ebl, 256, 0, st>>>(sa);
     if ((rc = launch_status("bwd_sel_scatter", st)) != NSA_OK) return rc;
-    // key pass, one launch per branch; the compressed keys' on tcgen05 (128 keys x 64 rows)
-    if (L.ncmp > 0) {
-      CUtensorMap bqmap, bdmap, bkcmap, bvcmap;
-      const int Tb = nsa::kBtRows / G;
-      const uint64_t qs1 = static_cast<uint64_t>(D) * 2, qs2 = static_cast<uint64_t>(hq) * D * 2;
-      const uint64_t ks1 = static_cast<uint64_t>(D) * 2, ks2 = static_cast<uint64_t>(hkv) * D * 2;
-      if (!nsa::make_tmap_bf16_3d(&bqmap, q, D, hq, N, qs1, qs2, 64, G, Tb) ||
-          !nsa::make_tmap_bf16_3d(&bdmap, d_out, D, hq, N, qs1, qs2, 64, G, Tb) ||
-          !nsa::make_tmap_bf16_3d(&bkcmap, ws + L.kc, D, hkv, L.ncmp, ks1, ks2, 64, 1, nsa::kBtKeys) ||
-          !nsa::make_tmap_bf16_3d(&bvcmap, ws + L.vc, D, hkv, L.ncmp, ks1, ks2, 64, 1, nsa::kBtKeys))
-        return NSA_ERR_CUDA;
-      const int nseg = (nv + nsa::kBtSegTokens - 1) / nsa::kBtSegTokens;
-      const long long items =
-          static_cast<long long>((L.ncmp + nsa::kBtKeys - 1) / nsa::kBtKeys) * hkv * nseg;
-      const size_t smem = sizeof(nsa::BtSmem<D>) + 1024;
-      auto kern = nsa::bwd_cmp_tc_kernel<D>;
-      if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
-      if (items > 0x7fffffffLL) return NSA_ERR_UNSUPPORTED;
-      kern<<<static_cast<unsigned>(items), nsa::kBtThreads, smem, st>>>(bqmap, bdmap, bkcmap, bvcmap, a, nseg);
-      if ((rc = launch_status("bwd_key_cmp", st)) != NSA_OK) return rc;
-    }
+    // key pass, one launch per branch: the compressed keys and the window on tcgen05 (128 keys
+    // x 64-row chunks), the selected blocks' on warp tiles over their buckets
+    if (L.ncmp > 0 &&
+        (rc = launch_bwd_key_tc<D, nsa::kBwdCmp>(a, q, d_out, ws + L.kc, ws + L.vc, L.ncmp, nv, st)) != NSA_OK)
+      return rc;
     {
       const long long segs = entries / nsa::kBwdSegSel + m + 1;  // >= sum over buckets of ceil(count / segment)
       if ((rc = launch_bwd_key<D, nsa::kBwdSel>(a, segs * (p->sel_block / nsa::kBwdChunk), st)) != NSA_OK) return rc;
     }
-    {
-      const long long items = static_cast<long long>((nv + nsa::kBwdChunk - 1) / nsa::kBwdChunk) * hkv;
-      if ((rc = launch_bwd_key<D, nsa::kBwdWin>(a, items, st)) != NSA_OK) return rc;
-    }
+    // a window key tile's rows span 128 + w - 1 tokens
+    if ((rc = launch_bwd_key_tc<D, nsa::kBwdWin>(a, q, d_out, k, v, N, nsa::kBtKeys + p->window, st)) != NSA_OK)
+      return rc;
   }
-  if (N > nv) {
-    const long long items = static_cast<long long>((N + nsa::kBwdChunk - 1) / nsa::kBwdChunk) * hkv *
-                            ((N - nv + nsa::kBwdSegDense - 1) / nsa::kBwdSegDense);
-    if ((rc = launch_bwd_key<D, nsa::kBwdDense>(a, items, st)) != NSA_OK) return rc;
-  }
+  if (N > nv && (rc = launch_bwd_key_tc<D, nsa::kBwdDense>(a, q, d_out, k, v, N, N - nv, st)) != NSA_OK) return rc;
   if (L.ncmp > 0) {
     const long long total = static_cast<long long>(nv) * hkv * D;
     nsa::pool_bwd_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(
