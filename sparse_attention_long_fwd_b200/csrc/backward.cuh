@@ -65,6 +65,8 @@ struct BwdArgs {
   const int* list;            // bucketed entries t * 64 + slot
   const float* fwd_lse;       // [nv][hq] the forward's compressed-branch log-sum-exp (natural log),
   const __half* fwd_ocmp;     // [nv][hq][D] and its output, or both null: pass A recomputes them
+  int cmp_rows_done;          // 1: the video rows' compressed-branch dq, statistics and gate gradient
+                              // are already written; the row pass adds the other branches to dq
 };
 
 // ---------------------------------------------------------------- row pass
@@ -373,7 +375,8 @@ __global__ void __launch_bounds__(32 * kBwdWarps) bwd_row_kernel(const BwdArgs a
     __syncwarp();
   }
   const int per_block = a.sel_len / kBwdChunk;
-  for (int b = 0; b < nb; ++b) {
+  const int b0 = video && a.cmp_rows_done ? 1 : 0;
+  for (int b = b0; b < nb; ++b) {
     const int br = video ? b : static_cast<int>(kBwdDense);
     const __nv_bfloat16* kb = (br == kBwdCmp) ? a.kc + g * D : a.k + g * D;
     const __nv_bfloat16* vb = (br == kBwdCmp) ? a.vc + g * D : a.v + g * D;
@@ -485,8 +488,15 @@ __global__ void __launch_bounds__(32 * kBwdWarps) bwd_row_kernel(const BwdArgs a
     if (!ok[r]) continue;
     float* dst = a.dq + (static_cast<size_t>(tok[r]) * a.hq + h0 + head[r]) * D + c;
 #pragma unroll
-    for (int n = 0; n < D / 8; ++n)
-      *reinterpret_cast<float2*>(dst + n * 8) = make_float2(dq[n][2 * r], dq[n][2 * r + 1]);
+    for (int n = 0; n < D / 8; ++n) {
+      float2 acc = make_float2(dq[n][2 * r], dq[n][2 * r + 1]);
+      if (b0 == 1) {
+        const float2 prev = *reinterpret_cast<const float2*>(dst + n * 8);
+        acc.x += prev.x;
+        acc.y += prev.y;
+      }
+      *reinterpret_cast<float2*>(dst + n * 8) = acc;
+    }
   }
 }
 

@@ -346,3 +346,318 @@ __global__ void __launch_bounds__(kBtThreads, 1)
 
 }  // namespace nsa
 
+namespace nsa {
+
+// ---------------------------------------------------------------- row pass, compressed branch
+// dq of the video rows from the compressed branch, on tcgen05, given the forward's saved
+// log-sum-exp and output of that branch: per row r (token t, head h) and visible compressed
+// block i,
+//   P = 2^(scale log2e <q_r, Kc_i> - lse2_r),  dS = g_r scale P (<dO_r, Vc_i> - D_r),
+//   dq_r = sum_i dS Kc_i,   D_r = <dO_r, o_cmp,r>.
+// One CTA per (query tile of T = 128 / G tokens x G heads, KV group): its Q and dO tiles load
+// once, the visible compressed keys stream in 128-key tiles through a two-slot ring:
+//   S = Q Kc^T, dP = dO Vc^T   (M = 128 rows, N = 128 keys; TMEM columns 0 and 128)
+//   softmax warps: dS as bf16 into TMEM (column 384)
+//   dQ += dS Kc                (A = dS from TMEM, B = the slot's Kc read MN-major; column 256)
+// It writes dq for these rows (the row pass then adds the other branches) and the branch's
+// (lse2, D) statistics and gate gradient. Same warp roles and bounded waits as the key pass.
+constexpr int kBrThreads = 64 + 256;
+constexpr int kBrSlots = 2;
+
+template <int D>
+struct BrSmem {
+  static constexpr int kChunks = D / 64;
+  alignas(1024) uint8_t q[kChunks][128 * 128];
+  alignas(1024) uint8_t dout[kChunks][128 * 128];
+  alignas(1024) uint8_t kc[kBrSlots][kChunks][128 * 128];
+  alignas(1024) uint8_t vc[kBrSlots][kChunks][128 * 128];
+  float rowc[2][128];  // per row: the two warpgroups' halves of <dO, o_cmp>
+  uint64_t q_full, kv_full[kBrSlots], kv_empty[kBrSlots], sd_full, sd_free, p_full, pv_done, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kBrThreads, 1)
+    bwd_row_cmp_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap dmap,
+                          const __grid_constant__ CUtensorMap kcmap, const __grid_constant__ CUtensorMap vcmap,
+                          const BwdArgs a) {
+  using Smem = BrSmem<D>;
+  constexpr int kChunks = Smem::kChunks;
+  constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256, kColDS = 384;
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = a.G;
+  const int T = 128 / G;
+  // the item: query tile (latest first: they see the most keys), group
+  const int ntiles = (a.nv + T - 1) / T;
+  const int g = blockIdx.x % a.hkv;
+  const int tile = ntiles - 1 - static_cast<int>(blockIdx.x / a.hkv);
+  if (tile < 0) return;
+  const int t0 = tile * T;
+  const int t_last = min(t0 + T, a.nv) - 1;
+  const int ke = t_last + 1 >= a.cmp_len ? min((t_last + 1 - a.cmp_len) / a.cmp_stride + 1, a.ncmp) : 0;
+  const int nkt = (ke + 127) / 128;
+
+  if (tid == 0) {
+    mbar_init(&sm.q_full, 1);
+    for (int s = 0; s < kBrSlots; ++s) {
+      mbar_init(&sm.kv_full[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
+    }
+    mbar_init(&sm.sd_full, 1);
+    mbar_init(&sm.sd_free, 8);
+    mbar_init(&sm.p_full, 8);
+    mbar_init(&sm.pv_done, 1);
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp >= 2) {
+    // rows T*G .. 127 of the Q and dO tiles are never written by TMA: keep them finite (zero)
+    const int r0 = T * G;
+    const int per = (128 - r0) * 8;
+    for (int i = tid - 64; i < 2 * kChunks * per; i += 256) {
+      const int u = i % per, rest = i / per;
+      const int c = rest % kChunks, tq = rest / kChunks;
+      uint8_t* base = tq == 0 ? sm.q[c] : sm.dout[c];
+      *reinterpret_cast<uint4*>(base + (r0 + u / 8) * 128 + (u % 8) * 16) = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort_flag = &sm.abort_flag;
+  int kv_issued = 0;
+  bool leader = false;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ loads
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&sm.q_full, 2 * kChunks * T * G * 128);
+      for (int c = 0; c < kChunks; ++c) {
+        tma_load_3d(&qmap, &sm.q_full, sm.q[c], c * 64, g * G, t0);
+        tma_load_3d(&dmap, &sm.q_full, sm.dout[c], c * 64, g * G, t0);
+      }
+      for (int kt = 0; kt < nkt; ++kt) {
+        const int s = kt % kBrSlots;
+        if (kt >= kBrSlots && !mbar_wait(&sm.kv_empty[s], ((kt / kBrSlots) - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&sm.kv_full[s], 2 * kChunks * 128 * 128);
+        for (int c = 0; c < kChunks; ++c) {
+          tma_load_3d(&kcmap, &sm.kv_full[s], sm.kc[s][c], c * 64, g, kt * 128);
+          tma_load_3d(&vcmap, &sm.kv_full[s], sm.vc[s][c], c * 64, g, kt * 128);
+        }
+        kv_issued = kt + 1;
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    leader = elect_one_sync();
+    constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
+    constexpr uint32_t idQ = idesc_bf16_f32(128, D, false, true);
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+    };
+    bool ok = wait_all(&sm.q_full, 0);
+    for (int kt = 0; ok && kt <= nkt; ++kt) {
+      if (kt < nkt) {
+        const int s = kt % kBrSlots;
+        if (!wait_all(&sm.kv_full[s], (kt / kBrSlots) & 1) || (kt >= 1 && !wait_all(&sm.sd_free, (kt - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (leader) {
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const int ch = k >> 2, kk = k & 3;
+            umma_bf16_ss(tmem + kColS, sdesc_sw128(smem_u32(sm.q[ch]) + kk * 32, 16, 1024),
+                         sdesc_sw128(smem_u32(sm.kc[s][ch]) + kk * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const int ch = k >> 2, kk = k & 3;
+            umma_bf16_ss(tmem + kColDP, sdesc_sw128(smem_u32(sm.dout[ch]) + kk * 32, 16, 1024),
+                         sdesc_sw128(smem_u32(sm.vc[s][ch]) + kk * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
+          }
+          umma_commit(&sm.sd_full);
+        }
+        __syncwarp();
+      }
+      if (kt >= 1) {
+        // dQ += dS Kc over the previous key tile (16 keys per MMA)
+        const int kp = kt - 1, sp = kp % kBrSlots;
+        if (!wait_all(&sm.p_full, kp & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (leader) {
+          const uint64_t kdesc = sdesc_sw128(smem_u32(sm.kc[sp][0]), 128 * 128, 1024);
+#pragma unroll
+          for (int k = 0; k < 128 / 16; ++k)
+            umma_bf16_ts(tmem + kColDQ, tmem + kColDS + k * 8, kdesc + static_cast<uint64_t>(k * (2048 >> 4)), idQ,
+                         (kp > 0 || k > 0) ? 1u : 0u);
+          umma_commit(&sm.pv_done);
+          umma_commit(&sm.kv_empty[sp]);
+        }
+        __syncwarp();
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax warps
+    const int sw = warp - 2;
+    const int wg = sw >> 2;          // key columns [64 wg, 64 wg + 64) of each tile
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;    // this thread's row (TMEM lane)
+    const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const int tok = r / G, hh = r % G;
+    const int t = t0 + tok;
+    const int h = g * G + hh;
+    const bool row_valid = r < T * G && t < a.nv;
+    bool ok = true;
+    // ---- the row's constants: D = <dO, o_cmp> from the forward's fp16 output, each warpgroup
+    // over half of the head dimension, summed through shared memory
+    float lse2 = -INFINITY, gs = 0.f;
+    int re = 0;
+    {
+      float part = 0.f;
+      if (row_valid) {
+        const size_t row = static_cast<size_t>(t) * a.hq + h;
+        const __half* o = a.fwd_ocmp + row * D + wg * (D / 2);
+        const __nv_bfloat16* dop = a.dout + row * D + wg * (D / 2);
+#pragma unroll 4
+        for (int c = 0; c < D / 2; c += 8) {
+          const uint4 ov = *reinterpret_cast<const uint4*>(o + c);
+          const uint4 dv = *reinterpret_cast<const uint4*>(dop + c);
+          const __half2* oh = reinterpret_cast<const __half2*>(&ov);
+          const __nv_bfloat162* dh = reinterpret_cast<const __nv_bfloat162*>(&dv);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            const float2 of = __half22float2(oh[x]);
+            const float2 df = __bfloat1622float2(dh[x]);
+            part += of.x * df.x + of.y * df.y;
+          }
+        }
+        lse2 = a.fwd_lse[row] * 1.4426950408889634f;
+        gs = a.gates[row * 3 + kBwdCmp] * a.scale;
+        re = t >= a.cmp_len - 1 ? min((t - a.cmp_len + 1) / a.cmp_stride + 1, a.ncmp) : 0;
+      }
+      sm.rowc[wg][r] = part;
+      named_bar_sync(1, 256);
+    }
+    const float dgr = sm.rowc[0][r] + sm.rowc[1][r];
+    if (wg == 0 && row_valid) {
+      const size_t o = (static_cast<size_t>(t) * a.hq + h) * 3;
+      a.stats[o + kBwdCmp] = make_float2(lse2, dgr);
+      a.dgates[o + kBwdCmp] = dgr;
+    }
+    for (int kt = 0; ok && kt < nkt; ++kt) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.sd_full, kt & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const int kbase = kt * 128 + wg * 64;
+      const bool full = __all_sync(0xffffffffu, !row_valid || kbase + 64 <= re);
+      uint32_t pd[32];
+#pragma unroll
+      for (int hc = 0; hc < 2; ++hc) {
+        float sv[32], dp[32];
+        __syncwarp();
+        tmem_ld32(trow + kColS + wg * 64 + 32 * hc, sv);
+        tmem_ld32(trow + kColDP + wg * 64 + 32 * hc, dp);
+        tmem_wait_ld();
+        if (hc == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.sd_free);
+        }
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          float ds[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int kidx = kbase + 32 * hc + j + e;
+            const bool vis = row_valid && (full || kidx < re) && lse2 != -INFINITY;
+            const float p = vis ? ex2_approx(fmaf(sv[j + e], a.sl2, -lse2)) : 0.f;
+            ds[e] = p * gs * (dp[j + e] - dgr);
+          }
+          pd[16 * hc + j / 2] = pack_bf16x2(ds[0], ds[1]);
+        }
+      }
+      // dS of this tile goes over the columns the previous tile's dQ MMAs read
+      if (kt >= 1) ok = mbar_wait(&sm.pv_done, (kt - 1) & 1, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      tmem_st16(trow + kColDS + wg * 32, *reinterpret_cast<const uint32_t(*)[16]>(&pd[0]));
+      tmem_st16(trow + kColDS + wg * 32 + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pd[16]));
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.p_full);
+    }
+    // ---- dq of this row: this warpgroup's half of D (zero when no key was visible)
+    if (ok && nkt > 0) ok = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done, (nkt - 1) & 1, abort_flag));
+    if (ok) {
+      tc_fence_after();
+      constexpr int kHalf = D / 2;
+      float* dst = a.dq + (static_cast<size_t>(t) * a.hq + h) * D + wg * kHalf;
+#pragma unroll
+      for (int x = 0; x < kHalf / 32; ++x) {
+        float v[32];
+        __syncwarp();
+        if (nkt > 0) {
+          tmem_ld32(trow + kColDQ + wg * kHalf + 32 * x, v);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) v[u] = 0.f;
+        }
+        if (row_valid) {
+#pragma unroll
+          for (int u = 0; u < 32; u += 4)
+            *reinterpret_cast<float4*>(dst + 32 * x + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+        }
+      }
+    }
+    tc_fence_before();
+  }
+
+  // ------------------------------------------------------------------ teardown
+  __syncthreads();
+  if (*abort_flag) {
+    if (warp == 0 && lane == 0) {
+      long long t_start = clock64();
+      while (!mbar_test(&sm.q_full, 0) && clock64() - t_start < kWaitCycles) {
+      }
+      for (int kt = kv_issued - kBrSlots > 0 ? kv_issued - kBrSlots : 0; kt < kv_issued; ++kt) {
+        t_start = clock64();
+        while (!mbar_test(&sm.kv_full[kt % kBrSlots], (kt / kBrSlots) & 1) && clock64() - t_start < kWaitCycles) {
+        }
+      }
+    }
+    if (warp == 1 && leader) {
+      umma_commit(&sm.drain);
+      const long long t_start = clock64();
+      while (!mbar_test(&sm.drain, 0) && clock64() - t_start < kWaitCycles) {
+      }
+    }
+    __syncwarp();
+    __syncthreads();
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace nsa
+

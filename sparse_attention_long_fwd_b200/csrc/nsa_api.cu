@@ -1238,6 +1238,30 @@ int launch_bwd_key_tc(const nsa::BwdArgs& a, const void* q, const void* d_out, c
   return launch_status(BR == nsa::kBwdCmp ? "bwd_key_cmp" : BR == nsa::kBwdWin ? "bwd_key_win" : "bwd_key_dense", st);
 }
 
+// The compressed branch's row pass on tcgen05 (dq, the branch's statistics and gate gradient of the
+// video rows), from the forward's saved log-sum-exp and output of that branch.
+template <int D>
+int launch_bwd_row_cmp_tc(const nsa::BwdArgs& a, const void* q, const void* d_out, cudaStream_t st) {
+  const int G = a.G, hq = a.hq, hkv = a.hkv;
+  if (G > 128) return NSA_ERR_UNSUPPORTED;
+  const int T = 128 / G;
+  CUtensorMap qmap, dmap, kmap, vmap;
+  const uint64_t qs1 = static_cast<uint64_t>(D) * 2, qs2 = static_cast<uint64_t>(hq) * D * 2;
+  const uint64_t ks1 = static_cast<uint64_t>(D) * 2, ks2 = static_cast<uint64_t>(hkv) * D * 2;
+  if (!nsa::make_tmap_bf16_3d(&qmap, q, D, hq, a.N, qs1, qs2, 64, G, T) ||
+      !nsa::make_tmap_bf16_3d(&dmap, d_out, D, hq, a.N, qs1, qs2, 64, G, T) ||
+      !nsa::make_tmap_bf16_3d(&kmap, a.kc, D, hkv, a.ncmp, ks1, ks2, 64, 1, 128) ||
+      !nsa::make_tmap_bf16_3d(&vmap, a.vc, D, hkv, a.ncmp, ks1, ks2, 64, 1, 128))
+    return NSA_ERR_CUDA;
+  const long long items = static_cast<long long>((a.nv + T - 1) / T) * hkv;
+  if (items > 0x7fffffffLL) return NSA_ERR_UNSUPPORTED;
+  const size_t smem = sizeof(nsa::BrSmem<D>) + 1024;
+  auto kern = nsa::bwd_row_cmp_tc_kernel<D>;
+  if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
+  kern<<<static_cast<unsigned>(items), nsa::kBrThreads, smem, st>>>(qmap, dmap, kmap, vmap, a);
+  return launch_status("bwd_row_cmp", st);
+}
+
 template <int D>
 int backward_impl(const nsa_params_t* p, const void* q, const void* k, const void* v, const float* gates,
                   const void* d_out, const int32_t* sel_idx, const uint8_t* fwd_ws, const float* phi_k,
@@ -1297,7 +1321,12 @@ int backward_impl(const nsa_params_t* p, const void* q, const void* k, const voi
                           phi_v)) != NSA_OK)
       return rc;
   }
-  // row pass: dq, the gates' gradient and the per-branch statistics
+  // row pass: dq, the gates' gradient and the per-branch statistics; with the forward's saved
+  // compressed-branch statistics, that branch's share runs first on tcgen05
+  if (a.fwd_lse != nullptr && L.ncmp > 0) {
+    if ((rc = launch_bwd_row_cmp_tc<D>(a, q, d_out, st)) != NSA_OK) return rc;
+    a.cmp_rows_done = 1;
+  }
   {
     const size_t smem = nsa::kBwdWarps * sizeof(nsa::BwdRowSmem<D>);
     auto kern = nsa::bwd_row_kernel<D>;

@@ -68,6 +68,7 @@ def _compare(w, q, k, v, g, d_out, sel, grads, phi=None):
     ("v128k", 40, 40, 4, 2, 128, 3, 16),              # shorter than two compression blocks
     ("v128k", 600, 600, 48, 4, 128, 16, 256),         # G = 12: one token per warp in the row pass
     ("qwen36k_hybrid", 520, 450, 32, 2, 64, 12, 128),  # G = 16, d = 64, with text rows
+    ("v128k", 4300, 4300, 8, 2, 64, 8, 64),           # 267 compressed blocks: three 128-key tiles
 ])
 @pytest.mark.parametrize("saved", [False, True])
 def test_backward_every_element(name, n, nv, hq, hkv, d, top_n, window, saved):
