@@ -32,6 +32,7 @@
 #include "sm100.cuh"
 #include "attn_tc.cuh"
 #include "backward.cuh"
+#include "sel_inv.cuh"
 
 namespace nsa {
 
@@ -661,3 +662,414 @@ __global__ void __launch_bounds__(kBrThreads, 1)
 
 }  // namespace nsa
 
+namespace nsa {
+
+// ---------------------------------------------------------------- key pass, selected branch
+// dK and dV of the selected blocks on tcgen05, over the buckets of (group, block j) that list
+// the tokens which chose block j. A tile is 128 gathered rows (T = 128 / G tokens x G heads)
+// against the block's 64 keys:
+//   S = Q K_j^T, dP = dO V_j^T           (M = 128 rows, N = 64 keys; TMEM, double-buffered)
+//   softmax warps: g P and dS = g scale P (dP - D) as bf16 tiles in shared memory
+//   dV_j^T += dO^T (g P), dK_j^T += Q^T dS  (M = D = 128 dims, N = 64 keys, K = 128 rows: A and
+//                                            B both read MN-major from the tiles already there)
+// so all four products run at M = 128 with no padding. dV^T and dK^T accumulate in TMEM over
+// the consecutive tiles of one bucket and are added to dv, dk (fp32, lane = dimension, so a
+// warp's reductions cover 128 contiguous bytes) after the bucket's last tile in this CTA.
+// Persistent: CTA c takes tiles [total c / grid, total (c + 1) / grid).
+//   warps 0..2   producers: warp 0 writes the tile records and loads K_j, V_j by TMA once per
+//                bucket run; all three gather the tile's Q and dO rows with 16-byte cp.async
+//                into the 128-byte-swizzled layout
+//   warp 3       MMA issuer
+//   warps 4..11  two warpgroups, thread = row; warpgroup w takes keys 32w .. 32w + 31 of each
+//                tile and, at a bucket's end, the dV^T (w = 0) or dK^T (w = 1) columns
+constexpr int kBsProducers = 3;
+constexpr int kBsMmaWarp = 3;
+constexpr int kBsFirstSmx = 4;
+constexpr int kBsThreads = 32 * kBsFirstSmx + 256;
+constexpr int kBsQStages = 2;
+constexpr int kBsInfo = 8;
+
+template <int D>
+struct BsSmem {
+  static constexpr int kChunks = D / 64;
+  alignas(1024) uint8_t q[kBsQStages][kChunks][128 * 128];
+  alignas(1024) uint8_t dout[kBsQStages][kChunks][128 * 128];
+  alignas(1024) uint8_t k[kChunks][64 * 128];
+  alignas(1024) uint8_t v[kChunks][64 * 128];
+  alignas(1024) uint8_t p[128 * 128];   // g P: 128 rows x 64 keys bf16, 128-byte swizzled rows
+  alignas(1024) uint8_t ds[128 * 128];  // dS, the same layout
+  SelTileInfo info[kBsInfo];
+  uint64_t q_full[kBsQStages], q_empty[kBsQStages], kv_full, kv_empty;
+  uint64_t info_full[kBsInfo], info_empty[kBsInfo];
+  uint64_t s_full[2], s_free[2], pd_full, pd_free, acc_full, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kBsThreads, 1)
+    bwd_sel_key_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                          const BwdArgs a) {
+  static_assert(D == 128, "the dV^T and dK^T products take M = D = 128");
+  using Smem = BsSmem<D>;
+  constexpr int kChunks = Smem::kChunks;
+  constexpr int kCpr = D / 8;  // 16-byte pieces per row
+  constexpr uint32_t kColAcc = 256;  // dV^T at 256, dK^T at 320; S and dP of tile i at 128 (i % 2) (+ 64)
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = a.G, TT = 128 / G;
+  const int m = a.hkv * a.nsel;
+  const long long total = a.seg_off[m];
+  const int tile_begin = static_cast<int>(total * blockIdx.x / gridDim.x);
+  const int tile_end = static_cast<int>(total * (blockIdx.x + 1) / gridDim.x);
+  const int n = tile_end - tile_begin;
+  if (n <= 0) return;  // uniform across the CTA
+  if (tid == 0) {
+    for (int s = 0; s < kBsQStages; ++s) {
+      mbar_init(&sm.q_full[s], kBsProducers * 32);  // one cp.async arrival per producer lane
+      mbar_init(&sm.q_empty[s], 1);
+    }
+    mbar_init(&sm.kv_full, 1);
+    mbar_init(&sm.kv_empty, 1);
+    for (int s = 0; s < kBsInfo; ++s) {
+      mbar_init(&sm.info_full[s], 1);
+      mbar_init(&sm.info_empty[s], 8);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.s_full[b], 1);
+      mbar_init(&sm.s_free[b], 8);
+    }
+    mbar_init(&sm.pd_full, 8);
+    mbar_init(&sm.pd_free, 1);
+    mbar_init(&sm.acc_full, 1);
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kBsMmaWarp) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  {
+    // rows a tile does not load keep what the stage held before: zero them once so that they
+    // are finite (their P and dS are zero, and 0 x NaN would not be)
+    uint4* z = reinterpret_cast<uint4*>(&sm.q[0][0][0]);
+    const int nq = static_cast<int>(sizeof(sm.q) / 16);
+    for (int i = tid; i < nq; i += kBsThreads) z[i] = make_uint4(0, 0, 0, 0);
+    z = reinterpret_cast<uint4*>(&sm.dout[0][0][0]);
+    for (int i = tid; i < nq; i += kBsThreads) z[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort_flag = &sm.abort_flag;
+  int kv_issued = 0;  // warp 0: K-V loads issued
+
+  if (warp < kBsProducers) {
+    // ------------------------------------------------------------------ producers
+    int key = 0, t_base = 0, t_next = 0, e_base = 0, e_next = 0;
+    auto fetch = [&](int tile) {
+      SelTileMeta r;
+      while (t_next <= tile) {  // next bucket with tiles
+        ++key;
+        t_base = t_next;
+        e_base = e_next;
+        t_next = a.seg_off[key + 1];
+        e_next = a.ent_off[key + 1];
+      }
+      r.key = key;
+      r.e0 = e_base + (tile - t_base) * TT;
+      r.cnt = min(TT, e_next - r.e0);
+      r.last = (tile == tile_end - 1) || (t_next == tile + 1);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) r.e[k] = (lane + 32 * k < r.cnt) ? a.list[r.e0 + lane + 32 * k] : 0;
+      return r;
+    };
+    SelTileMeta cur{};
+    if (warp == 0) {
+      if (lane == 0) {
+        tma_prefetch_desc(&kmap);
+        tma_prefetch_desc(&vmap);
+        int lo = 0, hi = m - 1;  // bucket of the first tile: the last key with seg_off[key] <= tile_begin
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (a.seg_off[mid] <= tile_begin) lo = mid; else hi = mid - 1;
+        }
+        key = lo;
+      }
+      key = __shfl_sync(0xffffffffu, key, 0);
+      t_base = a.seg_off[key];
+      t_next = a.seg_off[key + 1];
+      e_base = a.ent_off[key];
+      e_next = a.ent_off[key + 1];
+      cur = fetch(tile_begin);
+    }
+    int kv_key = -1;
+    for (int i = 0; i < n; ++i) {
+      const int si = i % kBsInfo, sq = i % kBsQStages;
+      SelTileInfo& inf = sm.info[si];
+      if (warp == 0) {
+        if (i >= kBsInfo && !warp_wait(&sm.info_empty[si], ((i / kBsInfo) - 1) & 1, abort_flag)) break;
+        const bool first = cur.key != kv_key;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (lane + 32 * k < cur.cnt) inf.ent[lane + 32 * k] = cur.e[k];
+        if (lane == 0) {
+          inf.key = cur.key;
+          inf.cnt = cur.cnt;
+          inf.kvs = 0;
+          inf.flags = (first ? 1 : 0) | (cur.last ? 2 : 0);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.info_full[si]);
+      } else if (!warp_wait(&sm.info_full[si], (i / kBsInfo) & 1, abort_flag)) {
+        break;
+      }
+      // Q and dO rows: row R = token slot R / G, head slot R % G; this warp takes the 32-row
+      // blocks b with b % 3 == (warp + 1) % 3 (warp 0, which also writes the records, the fewest)
+      if (i >= kBsQStages && !warp_wait(&sm.q_empty[sq], ((i / kBsQStages) - 1) & 1, abort_flag)) break;
+      {
+        const int cnt = inf.cnt;
+        const int g = inf.key / a.nsel;
+        for (int b = (warp + 1) % kBsProducers; b < 4; b += kBsProducers) {
+          const int rbase = b * 32;
+          int my_row = -1;
+          {
+            const int R = rbase + lane;
+            const int tok = R / G, hh = R - tok * G;
+            if (tok < cnt) my_row = (inf.ent[tok] >> 6) * a.hq + g * G + hh;
+          }
+          constexpr int kRpi = 32 / kCpr;  // rows per iteration
+          const int sub = lane / kCpr, c16 = lane % kCpr;
+          const char* q_lane = reinterpret_cast<const char*>(a.q) + c16 * 16;
+          const char* d_lane = reinterpret_cast<const char*>(a.dout) + c16 * 16;
+          // 128-byte swizzle: piece (c16 & 7) of row R sits at unit (c16 & 7) ^ (R & 7)
+          const uint32_t off_lane = (c16 >> 3) * (128 * 128) + (rbase + sub) * 128;
+          const uint32_t qdst = smem_u32(sm.q[sq][0]) + off_lane, ddst = smem_u32(sm.dout[sq][0]) + off_lane;
+          const uint32_t x_lane = (c16 & 7) ^ sub;
+#pragma unroll
+          for (int it = 0; it < kCpr; ++it) {
+            const int row = __shfl_sync(0xffffffffu, my_row, it * kRpi + sub);
+            const uint32_t o = it * kRpi * 128 + ((x_lane ^ ((it * kRpi) & 7)) << 4);
+            if (row >= 0) {
+              cp_async16_cg(qdst + o, q_lane + static_cast<size_t>(row) * (D * 2));
+              cp_async16_cg(ddst + o, d_lane + static_cast<size_t>(row) * (D * 2));
+            }
+          }
+        }
+        cp_async_arrive_noinc(&sm.q_full[sq]);
+      }
+      if (warp == 0) {
+        if (cur.key != kv_key) {
+          const int u = kv_issued;  // K-V load number
+          if (u >= 1 && !warp_wait(&sm.kv_empty, (u - 1) & 1, abort_flag)) break;
+          if (lane == 0) {
+            const int g = cur.key / a.nsel, j = cur.key % a.nsel;
+            mbar_arrive_expect_tx(&sm.kv_full, kChunks * 2 * 64 * 128);
+            for (int c = 0; c < kChunks; ++c) {
+              tma_load_3d(&kmap, &sm.kv_full, sm.k[c], c * 64, g, j * a.sel_len);
+              tma_load_3d(&vmap, &sm.kv_full, sm.v[c], c * 64, g, j * a.sel_len);
+            }
+          }
+          __syncwarp();
+          kv_issued = u + 1;
+          kv_key = cur.key;
+        }
+        if (i + 1 < n) cur = fetch(tile_begin + i + 1);
+      }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  } else if (warp == kBsMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, 64, false, false);
+      constexpr uint32_t idT = idesc_bf16_f32(128, 64, true, true);
+      int ns = 0, np = 0, kv_seen = 0;  // next S tile, next dV/dK tile, K-V loads consumed
+      int flags_even = 0, flags_odd = 0;  // flags of the last tiles whose S was issued
+      long long last = clock64();
+      while (np < n) {
+        if (*abort_flag) break;
+        bool did = false;
+        if (np < ns && mbar_ready(&sm.pd_full, np & 1)) {
+          const int sq = np % kBsQStages, flags = (np & 1) ? flags_odd : flags_even;
+          tc_fence_after();
+          const uint64_t pdesc = sdesc_sw128(smem_u32(sm.p), 128 * 128, 1024);
+          const uint64_t sdesc = sdesc_sw128(smem_u32(sm.ds), 128 * 128, 1024);
+          const uint64_t odesc = sdesc_sw128(smem_u32(sm.dout[sq][0]), 128 * 128, 1024);
+          const uint64_t qdesc = sdesc_sw128(smem_u32(sm.q[sq][0]), 128 * 128, 1024);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {  // 128 rows, 16 per MMA
+            const uint64_t adv = static_cast<uint64_t>(k * (2048 >> 4));
+            const uint32_t acc = ((flags & 1) && k == 0) ? 0u : 1u;
+            umma_bf16_ss(tmem + kColAcc, odesc + adv, pdesc + adv, idT, acc);
+            umma_bf16_ss(tmem + kColAcc + 64, qdesc + adv, sdesc + adv, idT, acc);
+          }
+          umma_commit(&sm.pd_free);
+          umma_commit(&sm.q_empty[sq]);
+          if (flags & 2) umma_commit(&sm.acc_full);
+          ++np;
+          did = true;
+        } else if (ns < n && ns < np + 2) {
+          const int b = ns & 1;
+          const int si = ns % kBsInfo, sq = ns % kBsQStages;
+          bool ready = mbar_ready(&sm.info_full[si], (ns / kBsInfo) & 1);
+          int flags = 0;
+          if (ready) {
+            flags = sm.info[si].flags;
+            if (flags & 1) ready = mbar_ready(&sm.kv_full, kv_seen & 1);
+          }
+          if (ready) ready = mbar_ready(&sm.q_full[sq], (ns / kBsQStages) & 1);
+          if (ready && ns >= 2) ready = mbar_ready(&sm.s_free[b], ((ns >> 1) - 1) & 1);
+          if (ready) {
+            if (flags & 1) ++kv_seen;
+            if (b) flags_odd = flags; else flags_even = flags;
+            fence_proxy_async_smem();  // Q and dO were written by cp.async (generic proxy)
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+              const int c = k >> 2, kk = k & 3;
+              umma_bf16_ss(tmem + b * 128, sdesc_sw128(smem_u32(sm.q[sq][c]) + kk * 32, 16, 1024),
+                           sdesc_sw128(smem_u32(sm.k[c]) + kk * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
+            }
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+              const int c = k >> 2, kk = k & 3;
+              umma_bf16_ss(tmem + b * 128 + 64, sdesc_sw128(smem_u32(sm.dout[sq][c]) + kk * 32, 16, 1024),
+                           sdesc_sw128(smem_u32(sm.v[c]) + kk * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
+            }
+            umma_commit(&sm.s_full[b]);
+            if (flags & 2) umma_commit(&sm.kv_empty);  // K_j and V_j are no longer needed
+            ++ns;
+            did = true;
+          }
+        }
+        if (did) {
+          last = clock64();
+        } else if (clock64() - last > kWaitCycles) {
+          *abort_flag = 1;
+          record_error(kErrWaitTimeout);
+          break;
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ softmax / epilogue
+    const int wg = (warp - kBsFirstSmx) >> 2;  // keys 32 wg .. 32 wg + 31
+    const int q4 = warp & 3;                   // TMEM lane quadrant
+    const int r = q4 * 32 + lane;              // tile row
+    const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    uint8_t* prow = sm.p + r * 128;
+    uint8_t* drow = sm.ds + r * 128;
+    int nepi = 0;
+    for (int i = 0; i < n; ++i) {
+      const int si = i % kBsInfo, b = i & 1;
+      if (!warp_wait(&sm.info_full[si], (i / kBsInfo) & 1, abort_flag)) break;
+      const SelTileInfo& inf = sm.info[si];
+      const int cnt = inf.cnt, key = inf.key, flags = inf.flags;
+      const int g = key / a.nsel, j = key % a.nsel;
+      const int tok = r / G, hh = r - (r / G) * G;
+      const bool valid = tok < cnt;
+      const int t = valid ? inf.ent[tok] >> 6 : 0;
+      const int k0 = j * a.sel_len;
+      const int key_hi = valid ? min(64, t + 1 - k0) - 32 * wg : 0;  // this thread's keys c < key_hi
+      float lse2 = 0.f, dgr = 0.f, gate = 0.f;
+      if (valid) {
+        const size_t o = (static_cast<size_t>(t) * a.hq + g * G + hh) * 3 + kBwdSel;
+        const float2 st = a.stats[o];
+        lse2 = st.x;
+        dgr = st.y;
+        gate = a.gates[o];
+      }
+      const float gs = gate * a.scale;
+      if (!warp_wait(&sm.s_full[b], (i >> 1) & 1, abort_flag)) break;
+      tc_fence_after();
+      float sv[32], dp[32];
+      tmem_ld32(trow + b * 128 + 32 * wg, sv);
+      tmem_ld32(trow + b * 128 + 64 + 32 * wg, dp);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.s_free[b]);
+      uint32_t pw[16], dw[16];
+#pragma unroll
+      for (int c = 0; c < 32; c += 2) {
+        float pv[2], dv[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const bool vis = c + e < key_hi && lse2 != -INFINITY;
+          const float p = vis ? ex2_approx(fmaf(sv[c + e], a.sl2, -lse2)) : 0.f;
+          pv[e] = p * gate;
+          dv[e] = p * gs * (dp[c + e] - dgr);
+        }
+        pw[c / 2] = pack_bf16x2(pv[0], pv[1]);
+        dw[c / 2] = pack_bf16x2(dv[0], dv[1]);
+      }
+      // the previous tile's dV/dK products read the P and dS tiles
+      if (i >= 1 && !warp_wait(&sm.pd_free, (i - 1) & 1, abort_flag)) break;
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {  // 8 keys = one 16-byte unit of the swizzled row
+        const int unit = wg * 4 + x;
+        const uint32_t off = static_cast<uint32_t>((unit ^ (r & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(prow) + off), "r"(pw[4 * x]),
+                     "r"(pw[4 * x + 1]), "r"(pw[4 * x + 2]), "r"(pw[4 * x + 3])
+                     : "memory");
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(drow) + off), "r"(dw[4 * x]),
+                     "r"(dw[4 * x + 1]), "r"(dw[4 * x + 2]), "r"(dw[4 * x + 3])
+                     : "memory");
+      }
+      fence_proxy_async_smem();  // read by the tensor core (async proxy)
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.pd_full);
+      if (flags & 2) {
+        // the bucket's sums: lane = dimension, column = key; warpgroup 0 dV, warpgroup 1 dK
+        if (!warp_wait(&sm.acc_full, nepi & 1, abort_flag)) break;
+        ++nepi;
+        tc_fence_after();
+        float accv[64];
+        tmem_ld32(trow + kColAcc + 64 * wg, *reinterpret_cast<float(*)[32]>(&accv[0]));
+        tmem_ld32(trow + kColAcc + 64 * wg + 32, *reinterpret_cast<float(*)[32]>(&accv[32]));
+        tmem_wait_ld();
+        tc_fence_before();
+        float* dst = (wg == 0 ? a.dv : a.dk) + (static_cast<size_t>(k0) * a.hkv + g) * D + r;
+        const size_t kstride = static_cast<size_t>(a.hkv) * D;
+        const int nk = min(64, a.nv - k0);
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (c < nk) atomicAdd(dst + c * kstride, accv[c]);  // result unused: a reduction
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.info_empty[si]);
+    }
+  }
+
+  // ------------------------------------------------------------------ teardown
+  __syncthreads();
+  if (*abort_flag) {
+    // drain: wait (bounded) for the last K-V load and for MMAs in flight, so that no async
+    // write lands after the CTA exits
+    if (warp == 0 && lane == 0 && kv_issued > 0) {
+      const long long t_start = clock64();
+      while (!mbar_test(&sm.kv_full, (kv_issued - 1) & 1) && clock64() - t_start < kWaitCycles) {
+      }
+    }
+    if (warp == kBsMmaWarp && lane == 0) {
+      umma_commit(&sm.drain);
+      const long long t_start = clock64();
+      while (!mbar_test(&sm.drain, 0) && clock64() - t_start < kWaitCycles) {
+      }
+    }
+    __syncwarp();
+    __syncthreads();
+  }
+  if (warp == kBsMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace nsa

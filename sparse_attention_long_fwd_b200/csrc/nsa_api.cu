@@ -1238,6 +1238,24 @@ int launch_bwd_key_tc(const nsa::BwdArgs& a, const void* q, const void* d_out, c
   return launch_status(BR == nsa::kBwdCmp ? "bwd_key_cmp" : BR == nsa::kBwdWin ? "bwd_key_win" : "bwd_key_dense", st);
 }
 
+// The selected blocks' key pass on tcgen05 (d = 128): persistent, one CTA per SM over the bucket
+// tiles, whose count the bucket scan left on the device.
+int launch_bwd_sel_key_tc(const nsa::BwdArgs& a, const void* k, const void* v, cudaStream_t st) {
+  constexpr int D = 128;
+  CUtensorMap kmap, vmap;
+  const uint64_t ks1 = static_cast<uint64_t>(D) * 2, ks2 = static_cast<uint64_t>(a.hkv) * D * 2;
+  if (!nsa::make_tmap_bf16_3d(&kmap, k, D, a.hkv, a.N, ks1, ks2, 64, 1, 64) ||
+      !nsa::make_tmap_bf16_3d(&vmap, v, D, a.hkv, a.N, ks1, ks2, 64, 1, 64))
+    return NSA_ERR_CUDA;
+  const size_t smem = sizeof(nsa::BsSmem<D>) + 1024;
+  auto kern = nsa::bwd_sel_key_tc_kernel<D>;
+  if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
+  const int nsm = sm_count();
+  if (nsm <= 0) return NSA_ERR_CUDA;
+  kern<<<static_cast<unsigned>(nsm), nsa::kBsThreads, smem, st>>>(kmap, vmap, a);
+  return launch_status("bwd_key_sel", st);
+}
+
 // The compressed branch's row pass on tcgen05 (dq, the branch's statistics and gate gradient of the
 // video rows), from the forward's saved log-sum-exp and output of that branch.
 template <int D>
@@ -1345,7 +1363,8 @@ int backward_impl(const nsa_params_t* p, const void* q, const void* k, const voi
     sa.hkv = hkv;
     sa.G = G;
     sa.Gp = G;
-    sa.TT = nsa::kBwdSegSel;
+    // d = 128: buckets cut into tcgen05 tiles of 128 rows (128 / G tokens); else warp segments
+    sa.TT = D == 128 ? 128 / G : nsa::kBwdSegSel;
     sa.nsel = L.nsel;
     sa.top_n = p->top_n;
     sa.sel_len = p->sel_block;
@@ -1371,7 +1390,9 @@ int backward_impl(const nsa_params_t* p, const void* q, const void* k, const voi
     if (L.ncmp > 0 &&
         (rc = launch_bwd_key_tc<D, nsa::kBwdCmp>(a, q, d_out, ws + L.kc, ws + L.vc, L.ncmp, nv, st)) != NSA_OK)
       return rc;
-    {
+    if constexpr (D == 128) {
+      if ((rc = launch_bwd_sel_key_tc(a, k, v, st)) != NSA_OK) return rc;
+    } else {
       const long long segs = entries / nsa::kBwdSegSel + m + 1;  // >= sum over buckets of ceil(count / segment)
       if ((rc = launch_bwd_key<D, nsa::kBwdSel>(a, segs * (p->sel_block / nsa::kBwdChunk), st)) != NSA_OK) return rc;
     }
