@@ -75,6 +75,11 @@ typedef struct {
   float softmax_scale;   /* <= 0 selects 1/sqrt(head_dim) */
   int32_t out_dtype;     /* enum nsa_out_dtype */
   int32_t batch;         /* decode / compress: number of sequences B (prefill: ignored) */
+  int32_t keep_branch_stats; /* prefill (one sequence) and backward: 1 = the prefill also keeps the
+                                selected branch's output and the selected and window branches'
+                                log-sum-exp in its workspace (larger workspace, one more fp16
+                                write of the selected rows), and nsa_backward, given that
+                                workspace and the same params, reuses them; 0 = neither */
 } nsa_params_t;
 
 /*
@@ -271,7 +276,10 @@ size_t nsa_gate_mlp_pooled_workspace_size(int batch, int seq_len, int heads, int
  *   sel_idx  [N_v][Hkv][top_n] int32: the forward's selection (nsa_prefill's out_sel_idx)
  *   fwd_workspace  NULL, or the workspace of the nsa_prefill / nsa_prefill_phi call being
  *            differentiated, unchanged since: its compressed-branch log-sum-exp and output
- *            (nsa_prefill_workspace_layout: lse, o_cmp) then replace a recomputation
+ *            (nsa_prefill_workspace_layout: lse, o_cmp) then replace a recomputation; if
+ *            params.keep_branch_stats = 1 (for both calls) the selected and window branches'
+ *            too (o_sel, lse_sel, o_win, lse_win), and every video row's dq, statistics and
+ *            gate gradient come from single passes on the tensor cores
  *   phi_k, phi_v  both NULL (mean compression) or both the learnable weights [Hkv][l] fp32
  *   dq       [N][Hq][d] fp32     dk, dv [N][Hkv][d] fp32    (written, not accumulated)
  *   dgates   [N][Hq][3] fp32: <dL/dout, o_b> per branch; 0 for text rows
@@ -299,13 +307,17 @@ size_t nsa_workspace_size(const nsa_params_t* params, int is_decode);
  *   scores   [N_v][Hkv][score_stride] fp32: block j of row (t, g) at j, Nsel = ceil(N_v / l')
  *            blocks (score_stride = Nsel rounded up to a multiple of 4); only j <= t/l' is written
  *   sel_idx  [N_v][Hkv][top_n] int32      o_win [N_v][Hq][d] fp16 (window branch)
- * The selected branch's output goes straight into the gated combine and is not kept.
+ * With params.keep_branch_stats = 1 the selected branch's output and the two other
+ * log-sum-exps are kept too (else these offsets are 0 and the selected output goes straight
+ * into the gated combine):
+ *   o_sel [N_v][Hq][d] fp16     lse_sel, lse_win [N_v][Hq] fp32 (natural log; -inf: no key)
  * Returns NSA_OK or NSA_ERR_INVALID_ARG.
  */
 typedef struct {
   size_t kc, vc, o_cmp, lse, scores, sel_idx, o_win, total;
   int32_t n_cmp, n_sel;
   int32_t score_stride;  /* floats between consecutive (t, g) score rows */
+  size_t o_sel, lse_sel, lse_win;
 } nsa_prefill_layout_t;
 int nsa_prefill_workspace_layout(const nsa_params_t* params, nsa_prefill_layout_t* layout);
 

@@ -204,6 +204,8 @@ typedef struct {
   double* o_sel;   /* [hq][d] */
   double* o_win;   /* [hq][d] */
   double* tie_gap; /* [hkv] */
+  double* lse_sel; /* [hq] selected-branch log-sum-exp */
+  double* lse_win; /* [hq] window-branch log-sum-exp */
 } row_out_t;
 
 /* One NSA (video) row at position t. K, V: [*][hkv][d] token rows of the sequence;
@@ -296,8 +298,10 @@ static void video_row(const oracle_cfg* c, int t, const uint16_t* qrow, const ui
       for (int e = 0; e < d; ++e) w->qd[e] = oracle_bf16_to_double(qrow[(size_t)h * d + e]);
       double* osel = w->osel + (size_t)h * d;
       double* owin = w->owin + (size_t)h * d;
-      attend_list(w->qd, K, V, stride, (size_t)g * d, d, c->scale, w->keys, nsk, w->z, NULL, osel);
-      attend_list(w->qd, K, V, stride, (size_t)g * d, d, c->scale, wkeys, nwk, w->z, NULL, owin);
+      const double lsel = attend_list(w->qd, K, V, stride, (size_t)g * d, d, c->scale, w->keys, nsk, w->z, NULL, osel);
+      const double lwin = attend_list(w->qd, K, V, stride, (size_t)g * d, d, c->scale, wkeys, nwk, w->z, NULL, owin);
+      if (ro->lse_sel) ro->lse_sel[h] = lsel;
+      if (ro->lse_win) ro->lse_win[h] = lwin;
       /* gated combine, gates ordered (cmp, sel, win), used as given */
       const double g0 = grow[h * 3 + 0], g1 = grow[h * 3 + 1], g2 = grow[h * 3 + 2];
       const double* ocmp = w->ocmp + (size_t)h * d;
@@ -355,12 +359,14 @@ static void free_scratch(scratch_t* w) {
  * kc, vc: [Ncmp(N_v)][hkv][d] from oracle_compress over the video prefix.
  * rows: nrows token positions. Per-row outputs are indexed by the position in rows[]:
  * out [nrows][hq][d]; sel [nrows][hkv][top_n]; scores [nrows][hkv][nsel_w];
- * o_cmp/o_sel/o_win [nrows][hq][d]; lse [nrows][hq]; tie_gap [nrows][hkv].
- * For text rows only out is written. Returns 0, or -1 on invalid arguments. */
+ * o_cmp/o_sel/o_win [nrows][hq][d]; lse (compressed branch), lse_sel, lse_win [nrows][hq];
+ * tie_gap [nrows][hkv]. For text rows only out is written. Returns 0, or -1 on invalid
+ * arguments. */
 int oracle_prefill_rows(const oracle_cfg* c, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                         const float* gates, const uint16_t* kc, const uint16_t* vc, int nrows, const int* rows,
                         const int* sel_override, double* out, int* sel, double* scores, int nsel_w, double* o_cmp,
-                        double* lse, double* o_sel, double* o_win, double* tie_gap, int nthreads) {
+                        double* lse, double* o_sel, double* o_win, double* tie_gap, double* lse_sel,
+                        double* lse_win, int nthreads) {
   if (!cfg_ok(c) || !q || !k || !v || !gates || !out || nrows < 0 || (nrows > 0 && !rows)) return -1;
   for (int r = 0; r < nrows; ++r)
     if (rows[r] < 0 || rows[r] >= c->n_tokens) return -1;
@@ -390,6 +396,8 @@ int oracle_prefill_rows(const oracle_cfg* c, const uint16_t* q, const uint16_t* 
         ro.o_sel = o_sel ? o_sel + (size_t)r * hq * d : NULL;
         ro.o_win = o_win ? o_win + (size_t)r * hq * d : NULL;
         ro.tie_gap = tie_gap ? tie_gap + (size_t)r * hkv : NULL;
+        ro.lse_sel = lse_sel ? lse_sel + (size_t)r * hq : NULL;
+        ro.lse_win = lse_win ? lse_win + (size_t)r * hq : NULL;
         const uint16_t* qrow = q + (size_t)t * hq * d;
         if (t < c->n_video) {
           video_row(c, t, qrow, k, v, kc, vc, gates + (size_t)t * hq * 3,
@@ -446,6 +454,8 @@ int oracle_decode(const oracle_cfg* c, const uint16_t* q, const uint16_t* kcache
         ro.o_sel = o_sel ? o_sel + (size_t)r * hq * d : NULL;
         ro.o_win = o_win ? o_win + (size_t)r * hq * d : NULL;
         ro.tie_gap = tie_gap ? tie_gap + (size_t)r * hkv : NULL;
+        ro.lse_sel = NULL;
+        ro.lse_win = NULL;
         const size_t seq_off = (size_t)b * Lmax * hkv * d;
         const size_t cmp_off = (size_t)b * ncmax * hkv * d;
         video_row(c, L - 1, q + (size_t)b * hq * d, kcache + seq_off, vcache + seq_off, kcmp + cmp_off,

@@ -55,7 +55,7 @@ def _load():
         lib.oracle_compress_weighted.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                  ctypes.c_int, P]
         lib.oracle_prefill_rows.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, P, P, ctypes.c_int, P, P, P, P, P,
-                                            ctypes.c_int, P, P, P, P, P, ctypes.c_int]
+                                            ctypes.c_int, P, P, P, P, P, P, P, ctypes.c_int]
         lib.oracle_decode.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, P, P, P, ctypes.c_int, P, P, P, P, P,
                                       ctypes.c_int, P, P, P, P, P, ctypes.c_int]
         _lib = lib
@@ -152,8 +152,9 @@ def _alloc_outputs(n: int, cfg: OracleConfig, nsel_w: int, want: tuple):
     for key in ("o_cmp", "o_sel", "o_win"):
         if key in want:
             o[key] = np.zeros((n, cfg.hq, cfg.d))
-    if "lse" in want:
-        o["lse"] = np.zeros((n, cfg.hq))
+    for key in ("lse", "lse_sel", "lse_win"):
+        if key in want:
+            o[key] = np.zeros((n, cfg.hq))
     if "tie_gap" in want:
         o["tie_gap"] = np.zeros((n, cfg.hkv))
     return o
@@ -181,7 +182,8 @@ def prefill_rows(cfg: OracleConfig, q, k, v, gates, rows, kc=None, vc=None, sel_
     rc = _load().oracle_prefill_rows(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(kc), _ptr(vc),
                                      len(rows), _ptr(rows), _ptr(so), _ptr(o["out"]), _ptr(o.get("sel")),
                                      _ptr(o.get("scores")), nsel_w, _ptr(o.get("o_cmp")), _ptr(o.get("lse")),
-                                     _ptr(o.get("o_sel")), _ptr(o.get("o_win")), _ptr(o.get("tie_gap")), nthreads)
+                                     _ptr(o.get("o_sel")), _ptr(o.get("o_win")), _ptr(o.get("tie_gap")),
+                                     _ptr(o.get("lse_sel")), _ptr(o.get("lse_win")), nthreads)
     if rc != 0:
         raise ValueError("oracle_prefill_rows rejected its arguments")
     return o

@@ -57,6 +57,7 @@ struct AttnArgs {
   float* scores;           // kModeCmp: write [N_v][Hkv][nsel]
   int nsel;
   __half* o_win;           // kModeWin: write [N_v][Hq][d]
+  float* lse_win;          // kModeWin: write [N_v][Hq] (natural log) when not null
   void* out;               // kModeDense: write [N][Hq][d]
   int out_f32;
   // Packed batches (null for one sequence). vinfo [video stream tokens]: per token the stream
@@ -946,6 +947,10 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
       }
       if (MODE == kModeCmp && ok && row_valid && wg == 0)
         args.lse[static_cast<size_t>(t) * args.hq + h] = has_keys ? lse2 * 0.69314718055994530942f : -INFINITY;
+      // (window) lse2 holds the row max and 1 / inv_l the row sum of exp2(S*sl2 - max)
+      if (MODE == kModeWin && args.lse_win != nullptr && ok && row_valid && wg == 0)
+        args.lse_win[static_cast<size_t>(t) * args.hq + h] =
+            has_keys && inv_l > 0.f ? (lse2 - __log2f(inv_l)) * 0.69314718055994530942f : -INFINITY;
       base += nkt;
       other_pv += (nkt + ((pair ^ 1) == (nkt & 1) ? 1 : 0)) >> 1;
     }

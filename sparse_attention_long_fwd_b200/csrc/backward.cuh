@@ -67,6 +67,16 @@ struct BwdArgs {
   const __half* fwd_ocmp;     // [nv][hq][D] and its output, or both null: pass A recomputes them
   int cmp_rows_done;          // 1: the video rows' compressed-branch dq, statistics and gate gradient
                               // are already written; the row pass adds the other branches to dq
+  // kept by the forward (nsa_params_t.keep_branch_stats), else null
+  const float* fwd_lse_sel;   // [nv][hq] natural log
+  const __half* fwd_osel;     // [nv][hq][D]
+  const float* fwd_lse_win;   // [nv][hq] natural log
+  const __half* fwd_owin;     // [nv][hq][D]
+  int video_rows_done;        // 1: the tensor-core kernels write every video row; the row pass
+                              // takes the text rows only
+  const int* row_of;          // [nv][hkv][top_n] first partial row of each (token, group, slot)
+  __half* dq_part;            // [part rows][D] the selected branch's dq per (row, block), fp16
+  float2* part_scale;         // [part rows] the factor of each 64-column half of a partial row
 };
 
 // ---------------------------------------------------------------- row pass
@@ -303,6 +313,7 @@ __global__ void __launch_bounds__(32 * kBwdWarps) bwd_row_kernel(const BwdArgs a
   const int g = static_cast<int>(item % a.hkv);
   const int pi = static_cast<int>(item / a.hkv);
   const bool video = pi < nv_items;
+  if (video && a.video_rows_done) return;  // warp-uniform
   const int t_end = video ? a.nv : a.N;
   const int tA = video ? pi * tpw : a.nv + (pi - nv_items) * tpw;
   const int h0 = g * G;

@@ -40,16 +40,17 @@ constexpr int kBtKeys = 128;   // compressed keys per item (MMA M)
 constexpr int kBtRows = 64;    // rows per chunk (MMA N of the score products)
 constexpr int kBtThreads = 64 + 256;
 constexpr int kBtSegTokens = 4096;  // tokens per item segment
+constexpr int kBtStages = 4;        // row chunks in flight (a chunk's loads take longer than its MMAs)
 
 template <int D>
 struct BtSmem {
   static constexpr int kChunks = D / 64;
   alignas(1024) uint8_t kc[kChunks][kBtKeys * 128];
   alignas(1024) uint8_t vc[kChunks][kBtKeys * 128];
-  alignas(1024) uint8_t q[2][kChunks][kBtRows * 128];
-  alignas(1024) uint8_t dout[2][kChunks][kBtRows * 128];
-  float4 rowc[2][kBtRows];  // per row: (lse2, D, gate, token as int bits; -1: no row)
-  uint64_t kv_full, q_full[2], q_empty[2], sd_full, sd_free, p_full, pv_done, drain;
+  alignas(1024) uint8_t q[kBtStages][kChunks][kBtRows * 128];
+  alignas(1024) uint8_t dout[kBtStages][kChunks][kBtRows * 128];
+  float4 rowc[kBtStages][kBtRows];  // per row: (lse2, D, gate, token as int bits; -1: no row)
+  uint64_t kv_full, q_full[kBtStages], q_empty[kBtStages], sd_full, sd_free, p_full, pv_done, drain;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -96,7 +97,7 @@ __global__ void __launch_bounds__(kBtThreads, 1)
 
   if (tid == 0) {
     mbar_init(&sm.kv_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kBtStages; ++s) {
       mbar_init(&sm.q_full[s], 1 + 32);  // the TMA's expect_tx arrival + the 32 row-constant lanes
       mbar_init(&sm.q_empty[s], 1);
     }
@@ -117,7 +118,7 @@ __global__ void __launch_bounds__(kBtThreads, 1)
     // the value products multiply them by P = dS = 0
     const int r0 = T * G;
     const int per = (kBtRows - r0) * 8;  // 16-byte units per (stage, tensor, chunk)
-    for (int i = tid - 64; i < 2 * 2 * kChunks * per; i += 256) {
+    for (int i = tid - 64; i < kBtStages * 2 * kChunks * per; i += 256) {
       const int u = i % per, rest = i / per;
       const int c = rest % kChunks, tq = (rest / kChunks) % 2, s = rest / (2 * kChunks);
       uint8_t* base = tq == 0 ? sm.q[s][c] : sm.dout[s][c];
@@ -145,8 +146,10 @@ __global__ void __launch_bounds__(kBtThreads, 1)
       }
     }
     for (int c = 0; c < nch; ++c) {
-      const int s = c & 1;
-      if (c >= 2 && !__all_sync(0xffffffffu, mbar_wait(&sm.q_empty[s], ((c - 2) >> 1) & 1, abort_flag))) break;
+      const int s = c % kBtStages;
+      if (c >= kBtStages &&
+          !__all_sync(0xffffffffu, mbar_wait(&sm.q_empty[s], ((c / kBtStages) - 1) & 1, abort_flag)))
+        break;
       const int t0 = tok_lo + c * T;
       if (lane == 0) {
         mbar_arrive_expect_tx(&sm.q_full[s], 2 * kChunks * T * G * 128);
@@ -184,8 +187,8 @@ __global__ void __launch_bounds__(kBtThreads, 1)
     for (int c = 0; ok && c <= nch; ++c) {
       if (c < nch) {
         // S^T and dP^T of chunk c (their columns were read by the softmax of chunk c - 1)
-        const int s = c & 1;
-        if (!wait_all(&sm.q_full[s], (c >> 1) & 1) || (c >= 1 && !wait_all(&sm.sd_free, (c - 1) & 1))) {
+        const int s = c % kBtStages;
+        if (!wait_all(&sm.q_full[s], (c / kBtStages) & 1) || (c >= 1 && !wait_all(&sm.sd_free, (c - 1) & 1))) {
           ok = false;
           break;
         }
@@ -209,7 +212,7 @@ __global__ void __launch_bounds__(kBtThreads, 1)
       }
       if (c >= 1) {
         // dV += (P g) x dO and dK += dS x Q over chunk c - 1's 64 rows (16 per MMA)
-        const int cp = c - 1, sp = cp & 1;
+        const int cp = c - 1, sp = cp % kBtStages;
         if (!wait_all(&sm.p_full, cp & 1)) {
           ok = false;
           break;
@@ -247,9 +250,9 @@ __global__ void __launch_bounds__(kBtThreads, 1)
     const float sl2 = a.sl2, scale = a.scale;
     bool ok = true;
     for (int c = 0; c < nch && ok; ++c) {
-      const int s = c & 1;
+      const int s = c % kBtStages;
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.sd_full, c & 1, abort_flag) &&
-                                       mbar_wait(&sm.q_full[s], (c >> 1) & 1, abort_flag));
+                                       mbar_wait(&sm.q_full[s], (c / kBtStages) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       float sv[32], dp[32];
@@ -324,9 +327,9 @@ __global__ void __launch_bounds__(kBtThreads, 1)
       long long t_start = clock64();
       while (!mbar_test(&sm.kv_full, 0) && clock64() - t_start < kWaitCycles) {
       }
-      for (int c = q_issued - 2 > 0 ? q_issued - 2 : 0; c < q_issued; ++c) {
+      for (int c = q_issued - kBtStages > 0 ? q_issued - kBtStages : 0; c < q_issued; ++c) {
         t_start = clock64();
-        while (!mbar_test(&sm.q_full[c & 1], (c >> 1) & 1) && clock64() - t_start < kWaitCycles) {
+        while (!mbar_test(&sm.q_full[c % kBtStages], (c / kBtStages) & 1) && clock64() - t_start < kWaitCycles) {
         }
       }
     }
@@ -349,19 +352,21 @@ __global__ void __launch_bounds__(kBtThreads, 1)
 
 namespace nsa {
 
-// ---------------------------------------------------------------- row pass, compressed branch
-// dq of the video rows from the compressed branch, on tcgen05, given the forward's saved
-// log-sum-exp and output of that branch: per row r (token t, head h) and visible compressed
-// block i,
-//   P = 2^(scale log2e <q_r, Kc_i> - lse2_r),  dS = g_r scale P (<dO_r, Vc_i> - D_r),
-//   dq_r = sum_i dS Kc_i,   D_r = <dO_r, o_cmp,r>.
+// ---------------------------------------------------------------- row pass, contiguous keys
+// dq of the video rows on tcgen05 from branches whose keys are contiguous, given the forward's
+// saved log-sum-exp and output of each: per row r (token t, head h) and visible key i of
+// branch b,
+//   P = 2^(scale log2e <q_r, K_i> - lse2_r,b),  dS = g_r,b scale P (<dO_r, V_i> - D_r,b),
+//   dq_r = sum_b sum_i dS K_i,   D_r,b = <dO_r, o_b,r>.
+// kFull = false: the compressed branch only (its statistics and gate gradient are written here,
+// the warp row pass adds the other branches to dq); kFull = true: the compressed blocks, then
+// the window's tokens [t - w + 1, t], with every branch's statistics already in `stats`.
 // One CTA per (query tile of T = 128 / G tokens x G heads, KV group): its Q and dO tiles load
-// once, the visible compressed keys stream in 128-key tiles through a two-slot ring:
-//   S = Q Kc^T, dP = dO Vc^T   (M = 128 rows, N = 128 keys; TMEM columns 0 and 128)
+// once, the keys stream in 128-key tiles through a two-slot ring:
+//   S = Q K^T, dP = dO V^T     (M = 128 rows, N = 128 keys; TMEM columns 0 and 128)
 //   softmax warps: dS as bf16 into TMEM (column 384)
-//   dQ += dS Kc                (A = dS from TMEM, B = the slot's Kc read MN-major; column 256)
-// It writes dq for these rows (the row pass then adds the other branches) and the branch's
-// (lse2, D) statistics and gate gradient. Same warp roles and bounded waits as the key pass.
+//   dQ += dS K                 (A = dS from TMEM, B = the slot's K read MN-major; column 256)
+// It writes dq for these rows. Same warp roles and bounded waits as the key pass.
 constexpr int kBrThreads = 64 + 256;
 constexpr int kBrSlots = 2;
 
@@ -378,11 +383,12 @@ struct BrSmem {
   int abort_flag;
 };
 
-template <int D>
+template <int D, bool kFull>
 __global__ void __launch_bounds__(kBrThreads, 1)
-    bwd_row_cmp_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap dmap,
-                          const __grid_constant__ CUtensorMap kcmap, const __grid_constant__ CUtensorMap vcmap,
-                          const BwdArgs a) {
+    bwd_row_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap dmap,
+                      const __grid_constant__ CUtensorMap kcmap, const __grid_constant__ CUtensorMap vcmap,
+                      const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                      const BwdArgs a) {
   using Smem = BrSmem<D>;
   constexpr int kChunks = Smem::kChunks;
   constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256, kColDS = 384;
@@ -399,7 +405,9 @@ __global__ void __launch_bounds__(kBrThreads, 1)
   const int t0 = tile * T;
   const int t_last = min(t0 + T, a.nv) - 1;
   const int ke = t_last + 1 >= a.cmp_len ? min((t_last + 1 - a.cmp_len) / a.cmp_stride + 1, a.ncmp) : 0;
-  const int nkt = (ke + 127) / 128;
+  const int nkt_c = (ke + 127) / 128;
+  const int kb_w = kFull ? max(0, t0 - a.window + 1) : 0;  // window keys [kb_w, t_last]
+  const int nkt = nkt_c + (kFull ? (t_last + 1 - kb_w + 127) / 128 : 0);
 
   if (tid == 0) {
     mbar_init(&sm.q_full, 1);
@@ -451,9 +459,11 @@ __global__ void __launch_bounds__(kBrThreads, 1)
         const int s = kt % kBrSlots;
         if (kt >= kBrSlots && !mbar_wait(&sm.kv_empty[s], ((kt / kBrSlots) - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(&sm.kv_full[s], 2 * kChunks * 128 * 128);
+        const bool win = kFull && kt >= nkt_c;
+        const int k0 = win ? kb_w + (kt - nkt_c) * 128 : kt * 128;
         for (int c = 0; c < kChunks; ++c) {
-          tma_load_3d(&kcmap, &sm.kv_full[s], sm.kc[s][c], c * 64, g, kt * 128);
-          tma_load_3d(&vcmap, &sm.kv_full[s], sm.vc[s][c], c * 64, g, kt * 128);
+          tma_load_3d(win ? &kmap : &kcmap, &sm.kv_full[s], sm.kc[s][c], c * 64, g, k0);
+          tma_load_3d(win ? &vmap : &vcmap, &sm.kv_full[s], sm.vc[s][c], c * 64, g, k0);
         }
         kv_issued = kt + 1;
       }
@@ -526,10 +536,24 @@ __global__ void __launch_bounds__(kBrThreads, 1)
     const bool row_valid = r < T * G && t < a.nv;
     bool ok = true;
     // ---- the row's constants: D = <dO, o_cmp> from the forward's fp16 output, each warpgroup
-    // over half of the head dimension, summed through shared memory
-    float lse2 = -INFINITY, gs = 0.f;
+    // over half of the head dimension, summed through shared memory (kFull: every branch's
+    // statistics are in `stats` already)
+    float lse2 = -INFINITY, gs = 0.f, dgr = 0.f;
+    float lse2_w = -INFINITY, gs_w = 0.f, dgr_w = 0.f;
     int re = 0;
-    {
+    if constexpr (kFull) {
+      if (row_valid) {
+        const size_t o = (static_cast<size_t>(t) * a.hq + h) * 3;
+        const float2 sc = a.stats[o + kBwdCmp], sw_ = a.stats[o + kBwdWin];
+        lse2 = sc.x;
+        dgr = sc.y;
+        gs = a.gates[o + kBwdCmp] * a.scale;
+        lse2_w = sw_.x;
+        dgr_w = sw_.y;
+        gs_w = a.gates[o + kBwdWin] * a.scale;
+        re = t >= a.cmp_len - 1 ? min((t - a.cmp_len + 1) / a.cmp_stride + 1, a.ncmp) : 0;
+      }
+    } else {
       float part = 0.f;
       if (row_valid) {
         const size_t row = static_cast<size_t>(t) * a.hq + h;
@@ -554,19 +578,23 @@ __global__ void __launch_bounds__(kBrThreads, 1)
       }
       sm.rowc[wg][r] = part;
       named_bar_sync(1, 256);
-    }
-    const float dgr = sm.rowc[0][r] + sm.rowc[1][r];
-    if (wg == 0 && row_valid) {
-      const size_t o = (static_cast<size_t>(t) * a.hq + h) * 3;
-      a.stats[o + kBwdCmp] = make_float2(lse2, dgr);
-      a.dgates[o + kBwdCmp] = dgr;
+      dgr = sm.rowc[0][r] + sm.rowc[1][r];
+      if (wg == 0 && row_valid) {
+        const size_t o = (static_cast<size_t>(t) * a.hq + h) * 3;
+        a.stats[o + kBwdCmp] = make_float2(lse2, dgr);
+        a.dgates[o + kBwdCmp] = dgr;
+      }
     }
     for (int kt = 0; ok && kt < nkt; ++kt) {
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.sd_full, kt & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      const int kbase = kt * 128 + wg * 64;
-      const bool full = __all_sync(0xffffffffu, !row_valid || kbase + 64 <= re);
+      const bool win = kFull && kt >= nkt_c;
+      // this thread's 64 keys: [kbase, kbase + 64), visible in [lo, hi)
+      const int kbase = (win ? kb_w + (kt - nkt_c) * 128 : kt * 128) + wg * 64;
+      const int lo = win ? t - a.window + 1 : 0, hi = win ? t + 1 : re;
+      const float l2 = win ? lse2_w : lse2, dg = win ? dgr_w : dgr, gsb = win ? gs_w : gs;
+      const bool full = __all_sync(0xffffffffu, !row_valid || (kbase >= lo && kbase + 64 <= hi));
       uint32_t pd[32];
 #pragma unroll
       for (int hc = 0; hc < 2; ++hc) {
@@ -586,9 +614,9 @@ __global__ void __launch_bounds__(kBrThreads, 1)
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int kidx = kbase + 32 * hc + j + e;
-            const bool vis = row_valid && (full || kidx < re) && lse2 != -INFINITY;
-            const float p = vis ? ex2_approx(fmaf(sv[j + e], a.sl2, -lse2)) : 0.f;
-            ds[e] = p * gs * (dp[j + e] - dgr);
+            const bool vis = row_valid && (full || (kidx >= lo && kidx < hi)) && l2 != -INFINITY;
+            const float p = vis ? ex2_approx(fmaf(sv[j + e], a.sl2, -l2)) : 0.f;
+            ds[e] = p * gsb * (dp[j + e] - dg);
           }
           pd[16 * hc + j / 2] = pack_bf16x2(ds[0], ds[1]);
         }
@@ -675,6 +703,10 @@ namespace nsa {
 // so all four products run at M = 128 with no padding. dV^T and dK^T accumulate in TMEM over
 // the consecutive tiles of one bucket and are added to dv, dk (fp32, lane = dimension, so a
 // warp's reductions cover 128 contiguous bytes) after the bucket's last tile in this CTA.
+// kDq: also dQ = dS K_j (M = 128 rows, N = D, K = 64 keys; TMEM, double-buffered), stored
+// per tile row as an fp16 partial (each 64-column half with a power-of-two factor that keeps
+// it finite), which a merge adds to the row's dq: the selected branch's share of dq.
+// TMEM columns: S 0, dP 64, dV^T 128, dK^T 192, dQ 256 and 384.
 // Persistent: CTA c takes tiles [total c / grid, total (c + 1) / grid).
 //   warps 0..2   producers: warp 0 writes the tile records and loads K_j, V_j by TMA once per
 //                bucket run; all three gather the tile's Q and dO rows with 16-byte cp.async
@@ -701,12 +733,12 @@ struct BsSmem {
   SelTileInfo info[kBsInfo];
   uint64_t q_full[kBsQStages], q_empty[kBsQStages], kv_full, kv_empty;
   uint64_t info_full[kBsInfo], info_empty[kBsInfo];
-  uint64_t s_full[2], s_free[2], pd_full, pd_free, acc_full, drain;
+  uint64_t s_full, s_free, pd_full, pd_free, acc_full, dq_full[2], dq_free[2], drain;
   uint32_t tmem_base;
   int abort_flag;
 };
 
-template <int D>
+template <int D, bool kDq>
 __global__ void __launch_bounds__(kBsThreads, 1)
     bwd_sel_key_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                           const BwdArgs a) {
@@ -714,7 +746,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
   using Smem = BsSmem<D>;
   constexpr int kChunks = Smem::kChunks;
   constexpr int kCpr = D / 8;  // 16-byte pieces per row
-  constexpr uint32_t kColAcc = 256;  // dV^T at 256, dK^T at 320; S and dP of tile i at 128 (i % 2) (+ 64)
+  constexpr uint32_t kColAcc = 128, kColDQ = 256;
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -736,9 +768,11 @@ __global__ void __launch_bounds__(kBsThreads, 1)
       mbar_init(&sm.info_full[s], 1);
       mbar_init(&sm.info_empty[s], 8);
     }
+    mbar_init(&sm.s_full, 1);
+    mbar_init(&sm.s_free, 8);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&sm.s_full[b], 1);
-      mbar_init(&sm.s_free[b], 8);
+      mbar_init(&sm.dq_full[b], 1);
+      mbar_init(&sm.dq_free[b], 8);
     }
     mbar_init(&sm.pd_full, 8);
     mbar_init(&sm.pd_free, 1);
@@ -887,13 +921,15 @@ __global__ void __launch_bounds__(kBsThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 64, false, false);
       constexpr uint32_t idT = idesc_bf16_f32(128, 64, true, true);
-      int ns = 0, np = 0, kv_seen = 0;  // next S tile, next dV/dK tile, K-V loads consumed
+      constexpr uint32_t idQ = idesc_bf16_f32(128, D, false, true);
+      int ns = 0, np = 0, kv_seen = 0;    // next S tile, next dV/dK tile, K-V loads consumed
       int flags_even = 0, flags_odd = 0;  // flags of the last tiles whose S was issued
       long long last = clock64();
       while (np < n) {
         if (*abort_flag) break;
         bool did = false;
-        if (np < ns && mbar_ready(&sm.pd_full, np & 1)) {
+        if (np < ns && mbar_ready(&sm.pd_full, np & 1) &&
+            (!kDq || np < 2 || mbar_ready(&sm.dq_free[np & 1], ((np >> 1) - 1) & 1))) {
           const int sq = np % kBsQStages, flags = (np & 1) ? flags_odd : flags_even;
           tc_fence_after();
           const uint64_t pdesc = sdesc_sw128(smem_u32(sm.p), 128 * 128, 1024);
@@ -907,13 +943,23 @@ __global__ void __launch_bounds__(kBsThreads, 1)
             umma_bf16_ss(tmem + kColAcc, odesc + adv, pdesc + adv, idT, acc);
             umma_bf16_ss(tmem + kColAcc + 64, qdesc + adv, sdesc + adv, idT, acc);
           }
+          if constexpr (kDq) {
+            const uint64_t kdesc = sdesc_sw128(smem_u32(sm.k[0]), 64 * 128, 1024);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)  // 64 keys, 16 per MMA
+              umma_bf16_ss(tmem + kColDQ + (np & 1) * 128, sdesc_sw128(smem_u32(sm.ds) + k * 32, 16, 1024),
+                           kdesc + static_cast<uint64_t>(k * (2048 >> 4)), idQ, k > 0 ? 1u : 0u);
+            umma_commit(&sm.dq_full[np & 1]);
+          }
           umma_commit(&sm.pd_free);
           umma_commit(&sm.q_empty[sq]);
-          if (flags & 2) umma_commit(&sm.acc_full);
+          if (flags & 2) {
+            umma_commit(&sm.acc_full);
+            umma_commit(&sm.kv_empty);  // K_j and V_j are no longer needed
+          }
           ++np;
           did = true;
         } else if (ns < n && ns < np + 2) {
-          const int b = ns & 1;
           const int si = ns % kBsInfo, sq = ns % kBsQStages;
           bool ready = mbar_ready(&sm.info_full[si], (ns / kBsInfo) & 1);
           int flags = 0;
@@ -922,26 +968,25 @@ __global__ void __launch_bounds__(kBsThreads, 1)
             if (flags & 1) ready = mbar_ready(&sm.kv_full, kv_seen & 1);
           }
           if (ready) ready = mbar_ready(&sm.q_full[sq], (ns / kBsQStages) & 1);
-          if (ready && ns >= 2) ready = mbar_ready(&sm.s_free[b], ((ns >> 1) - 1) & 1);
+          if (ready && ns >= 1) ready = mbar_ready(&sm.s_free, (ns - 1) & 1);
           if (ready) {
             if (flags & 1) ++kv_seen;
-            if (b) flags_odd = flags; else flags_even = flags;
+            if (ns & 1) flags_odd = flags; else flags_even = flags;
             fence_proxy_async_smem();  // Q and dO were written by cp.async (generic proxy)
             tc_fence_after();
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
               const int c = k >> 2, kk = k & 3;
-              umma_bf16_ss(tmem + b * 128, sdesc_sw128(smem_u32(sm.q[sq][c]) + kk * 32, 16, 1024),
+              umma_bf16_ss(tmem, sdesc_sw128(smem_u32(sm.q[sq][c]) + kk * 32, 16, 1024),
                            sdesc_sw128(smem_u32(sm.k[c]) + kk * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
             }
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
               const int c = k >> 2, kk = k & 3;
-              umma_bf16_ss(tmem + b * 128 + 64, sdesc_sw128(smem_u32(sm.dout[sq][c]) + kk * 32, 16, 1024),
+              umma_bf16_ss(tmem + 64, sdesc_sw128(smem_u32(sm.dout[sq][c]) + kk * 32, 16, 1024),
                            sdesc_sw128(smem_u32(sm.v[c]) + kk * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
             }
-            umma_commit(&sm.s_full[b]);
-            if (flags & 2) umma_commit(&sm.kv_empty);  // K_j and V_j are no longer needed
+            umma_commit(&sm.s_full);
             ++ns;
             did = true;
           }
@@ -965,8 +1010,42 @@ __global__ void __launch_bounds__(kBsThreads, 1)
     uint8_t* prow = sm.p + r * 128;
     uint8_t* drow = sm.ds + r * 128;
     int nepi = 0;
+    // the fp16 partial of tile x, this warpgroup's half of row r
+    auto dq_out = [&](int x) -> bool {
+      if (!warp_wait(&sm.dq_full[x & 1], (x >> 1) & 1, abort_flag)) return false;
+      tc_fence_after();
+      float v[64];
+      tmem_ld32(trow + kColDQ + (x & 1) * 128 + 64 * wg, *reinterpret_cast<float(*)[32]>(&v[0]));
+      tmem_ld32(trow + kColDQ + (x & 1) * 128 + 64 * wg + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.dq_free[x & 1]);
+      float am = 0.f;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) am = fmaxf(am, fabsf(v[c]));
+      // 65504 is the largest finite fp16 value; rare rows are scaled down by a power of two
+      float c = 1.f;
+      if (am > 32768.f && am <= 3.0e38f) c = exp2f(ceilf(log2f(am / 32768.f)));
+      const float inv = 1.f / c;
+      const size_t prow_g = static_cast<size_t>(tile_begin + x) * 128 + r;
+      uint4* dst = reinterpret_cast<uint4*>(a.dq_part + prow_g * D + 64 * wg);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        uint4 w4;
+        uint32_t* wp = reinterpret_cast<uint32_t*>(&w4);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __half2 hv = __floats2half2_rn(v[8 * u + 2 * e] * inv, v[8 * u + 2 * e + 1] * inv);
+          wp[e] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
+        dst[u] = w4;
+      }
+      reinterpret_cast<float*>(a.part_scale)[2 * prow_g + wg] = c;
+      return true;
+    };
     for (int i = 0; i < n; ++i) {
-      const int si = i % kBsInfo, b = i & 1;
+      const int si = i % kBsInfo;
       if (!warp_wait(&sm.info_full[si], (i / kBsInfo) & 1, abort_flag)) break;
       const SelTileInfo& inf = sm.info[si];
       const int cnt = inf.cnt, key = inf.key, flags = inf.flags;
@@ -985,15 +1064,15 @@ __global__ void __launch_bounds__(kBsThreads, 1)
         gate = a.gates[o];
       }
       const float gs = gate * a.scale;
-      if (!warp_wait(&sm.s_full[b], (i >> 1) & 1, abort_flag)) break;
+      if (!warp_wait(&sm.s_full, i & 1, abort_flag)) break;
       tc_fence_after();
       float sv[32], dp[32];
-      tmem_ld32(trow + b * 128 + 32 * wg, sv);
-      tmem_ld32(trow + b * 128 + 64 + 32 * wg, dp);
+      tmem_ld32(trow + 32 * wg, sv);
+      tmem_ld32(trow + 64 + 32 * wg, dp);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.s_free[b]);
+      if (lane == 0) mbar_arrive(&sm.s_free);
       uint32_t pw[16], dw[16];
 #pragma unroll
       for (int c = 0; c < 32; c += 2) {
@@ -1025,6 +1104,8 @@ __global__ void __launch_bounds__(kBsThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.pd_full);
+      // the previous tile's dq partial: read while this tile's products run
+      if (kDq && i >= 1 && !dq_out(i - 1)) break;
       if (flags & 2) {
         // the bucket's sums: lane = dimension, column = key; warpgroup 0 dV, warpgroup 1 dK
         if (!warp_wait(&sm.acc_full, nepi & 1, abort_flag)) break;
@@ -1044,6 +1125,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.info_empty[si]);
+      if (kDq && i == n - 1) dq_out(i);
     }
   }
 
@@ -1069,6 +1151,113 @@ __global__ void __launch_bounds__(kBsThreads, 1)
   if (warp == kBsMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace nsa
+
+namespace nsa {
+
+// ---------------------------------------------------------------- kept statistics
+// Per video row (t, h), from what the forward kept: stats[row][b] = (lse_b log2 e, <dO, o_b>)
+// and dgates[row][b] = <dO, o_b> for b = compressed, selected, window. One warp per row;
+// lane l takes elements [l D/32, (l + 1) D/32).
+template <int D>
+__global__ void __launch_bounds__(256) bwd_stats_kernel(const BwdArgs a) {
+  constexpr int kPer = D / 32;
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= static_cast<long long>(a.nv) * a.hq) return;
+  const size_t off = static_cast<size_t>(row) * D + lane * kPer;
+  float dov[kPer];
+#pragma unroll
+  for (int u = 0; u < kPer; u += 2) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(a.dout + off + u));
+    dov[u] = f.x;
+    dov[u + 1] = f.y;
+  }
+  const __half* ob[3] = {a.fwd_ocmp, a.fwd_osel, a.fwd_owin};
+  const float* lb[3] = {a.fwd_lse, a.fwd_lse_sel, a.fwd_lse_win};
+#pragma unroll
+  for (int b = 0; b < 3; ++b) {
+    float dot = 0.f;
+#pragma unroll
+    for (int u = 0; u < kPer; u += 2) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(ob[b] + off + u));
+      dot = fmaf(dov[u], f.x, fmaf(dov[u + 1], f.y, dot));
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    if (lane == 0) {
+      const size_t o3 = static_cast<size_t>(row) * 3 + b;
+      a.stats[o3] = make_float2(lb[b][row] * 1.4426950408889634f, dot);
+      a.dgates[o3] = dot;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- selected dq merge
+// dq[t][h] += sum over the row's selected slots of its fp16 partial (times each half's factor).
+// One warp per row; lane l takes elements [l D/32, (l + 1) D/32), in half (l D/32) / 64.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_sel_dq_merge_kernel(const BwdArgs a) {
+  constexpr int kPer = D / 32;
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= static_cast<long long>(a.nv) * a.hq) return;
+  const int t = static_cast<int>(row / a.hq), h = static_cast<int>(row % a.hq);
+  const int g = h / a.G, hh = h - g * a.G;
+  const size_t base = (static_cast<size_t>(t) * a.hkv + g) * a.top_n;
+  // lane s holds slot s (and s + 32): its partial row, or -1; top_n <= 64
+  int r0 = -1, r1 = -1;
+  if (lane < a.top_n && a.sel_idx[base + lane] >= 0) r0 = a.row_of[base + lane] + hh;
+  if (lane + 32 < a.top_n && a.sel_idx[base + lane + 32] >= 0) r1 = a.row_of[base + lane + 32] + hh;
+  const int half = (lane * kPer) >> 6;
+  float acc[kPer];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) acc[u] = 0.f;
+  for (int s0 = 0; s0 < a.top_n; s0 += 8) {
+    uint2 raw[8];
+    float c[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int s = s0 + k;
+      int pr = __shfl_sync(0xffffffffu, s < 32 ? r0 : r1, s & 31);
+      if (s >= a.top_n) pr = -1;
+      raw[k] = make_uint2(0u, 0u);
+      c[k] = 0.f;
+      if (pr >= 0) {
+        const __half* p = a.dq_part + static_cast<size_t>(pr) * D + lane * kPer;
+        if constexpr (kPer == 4) raw[k] = *reinterpret_cast<const uint2*>(p);
+        else raw[k].x = *reinterpret_cast<const uint32_t*>(p);
+        c[k] = reinterpret_cast<const float*>(a.part_scale)[2 * static_cast<size_t>(pr) + half];
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&raw[k].x));
+      acc[0] = fmaf(c[k], f0.x, acc[0]);
+      acc[1] = fmaf(c[k], f0.y, acc[1]);
+      if constexpr (kPer == 4) {
+        const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&raw[k].y));
+        acc[2] = fmaf(c[k], f1.x, acc[2]);
+        acc[3] = fmaf(c[k], f1.y, acc[3]);
+      }
+    }
+  }
+  float* dst = a.dq + static_cast<size_t>(row) * D + lane * kPer;
+  if constexpr (kPer == 4) {
+    float4 v = *reinterpret_cast<float4*>(dst);
+    v.x += acc[0];
+    v.y += acc[1];
+    v.z += acc[2];
+    v.w += acc[3];
+    *reinterpret_cast<float4*>(dst) = v;
+  } else {
+    float2 v = *reinterpret_cast<float2*>(dst);
+    v.x += acc[0];
+    v.y += acc[1];
+    *reinterpret_cast<float2*>(dst) = v;
   }
 }
 

@@ -68,6 +68,7 @@ int check_common(const nsa_params_t* p) {
   if (p->cmp_block < 1 || p->cmp_stride < 1 || p->sel_block < 1 || p->window < 1 || p->top_n < 1)
     return NSA_ERR_INVALID_ARG;
   if (p->out_dtype != NSA_OUT_BF16 && p->out_dtype != NSA_OUT_F32) return NSA_ERR_INVALID_ARG;
+  if (p->keep_branch_stats != 0 && p->keep_branch_stats != 1) return NSA_ERR_INVALID_ARG;
   if (p->head_dim != 64 && p->head_dim != 128) return NSA_ERR_UNSUPPORTED;
   if (p->num_q_heads / p->num_kv_heads > 16) return NSA_ERR_UNSUPPORTED;
   if (p->cmp_block != 32 || p->cmp_stride != 16 || p->sel_block != 64) return NSA_ERR_UNSUPPORTED;
@@ -101,6 +102,7 @@ int check_device() {
 
 struct PrefillLayout {
   size_t kc, vc, o_cmp, lse, scores, sel_idx, o_win, total;
+  size_t o_sel, lse_sel, lse_win;  // kept branch statistics, or 0
   // block-major selected branch: bucket counters, offsets, bucketed entries, partials
   size_t sel_cnt, sel_eoff, sel_toff, sel_list, sel_row, part_o, part_ml;
   long long part_rows;  // 128 x the bound on selected-branch tiles
@@ -111,7 +113,8 @@ struct PrefillLayout {
 // Workspace layout of the NSA rows of one call: nv stream rows, ncmp_rows compressed rows,
 // nsel_cols selection-block columns per group (the bucket space) and score rows of up to
 // nsel_max blocks (one sequence: ncmp_rows = Ncmp(nv), nsel_cols = nsel_max = Nsel(nv)).
-PrefillLayout video_layout(int nv, int ncmp_rows, int nsel_cols, int nsel_max, int hq, int hkv, int d, int top_n) {
+PrefillLayout video_layout(int nv, int ncmp_rows, int nsel_cols, int nsel_max, int hq, int hkv, int d, int top_n,
+                           bool keep = false) {
   PrefillLayout L{};
   L.ncmp = ncmp_rows;
   L.nsel = nsel_cols;
@@ -144,6 +147,11 @@ PrefillLayout video_layout(int nv, int ncmp_rows, int nsel_cols, int nsel_max, i
   }
   L.part_o = take(static_cast<size_t>(L.part_rows) * d * 2);
   L.part_ml = take(static_cast<size_t>(L.part_rows) * 16);
+  if (keep) {
+    L.o_sel = take(static_cast<size_t>(nv) * hq * d * 2);
+    L.lse_sel = take(static_cast<size_t>(nv) * hq * 4);
+    L.lse_win = take(static_cast<size_t>(nv) * hq * 4);
+  }
   L.total = off;
   return L;
 }
@@ -152,7 +160,7 @@ PrefillLayout prefill_layout(const nsa_params_t* p) {
   const int nv = p->n_video;
   const int ns = nsel_of(nv, p->sel_block);
   return video_layout(nv, ncmp_of(nv, p->cmp_block, p->cmp_stride), ns, ns, p->num_q_heads, p->num_kv_heads,
-                      p->head_dim, p->top_n);
+                      p->head_dim, p->top_n, p->keep_branch_stats != 0);
 }
 
 struct DecodeLayout {
@@ -408,6 +416,8 @@ int video_stages(const nsa_params_t* p, const StageGeo& geo, const PrefillLayout
   sa.part_ml = reinterpret_cast<float4*>(ws + L.part_ml);
   sa.o_cmp = reinterpret_cast<const __half*>(ws + L.o_cmp);
   sa.o_win = reinterpret_cast<const __half*>(ws + L.o_win);
+  sa.o_sel = L.o_sel != 0 ? reinterpret_cast<__half*>(ws + L.o_sel) : nullptr;
+  sa.lse_sel = L.lse_sel != 0 ? reinterpret_cast<float*>(ws + L.lse_sel) : nullptr;
   sa.gates = geo.gates;
   sa.out = geo.out;
   sa.out_f32 = p->out_dtype == NSA_OUT_F32;
@@ -446,6 +456,7 @@ int video_stages(const nsa_params_t* p, const StageGeo& geo, const PrefillLayout
   }
   // 5. sliding window -> o_win
   a.o_win = reinterpret_cast<__half*>(ws + L.o_win);
+  a.lse_win = L.lse_win != 0 ? reinterpret_cast<float*>(ws + L.lse_win) : nullptr;
   if ((rc = launch_attn<D, nsa::kModeWin>(qmap, kmap, vmap, a, st)) != NSA_OK) return rc;
   // 6. merge of the selected partials + gated combine -> out (the NSA rows)
   const long long rows = static_cast<long long>(nv) * hq;
@@ -871,6 +882,9 @@ int nsa_prefill_workspace_layout(const nsa_params_t* params, nsa_prefill_layout_
   layout->n_cmp = L.ncmp;
   layout->n_sel = L.nsel;
   layout->score_stride = L.score_stride;
+  layout->o_sel = L.o_sel;
+  layout->lse_sel = L.lse_sel;
+  layout->lse_win = L.lse_win;
   return NSA_OK;
 }
 
@@ -1166,6 +1180,8 @@ namespace {
 
 struct BwdLayout {
   size_t kc, vc, dkc, dvc, stats, cnt, ent_off, seg_off, list, row_of, total;
+  size_t dq_part, part_scale;  // (kept statistics, d = 128) the selected branch's dq partials
+  long long part_rows;
   int ncmp, nsel;
 };
 
@@ -1193,6 +1209,12 @@ BwdLayout bwd_layout(const nsa_params_t* p) {
   L.seg_off = take((buckets + 1) * 4);
   L.list = take(entries * 4);
   L.row_of = take(entries * 4);
+  if (p->keep_branch_stats && d == 128 && nv > 0) {
+    const size_t G = hq / hkv;  // 128-row tiles of 128 / G tokens, at most one partial tile per bucket
+    L.part_rows = static_cast<long long>((entries + (128 / G) - 1) / (128 / G) + buckets) * 128;
+    L.dq_part = take(static_cast<size_t>(L.part_rows) * d * 2);
+    L.part_scale = take(static_cast<size_t>(L.part_rows) * 8);
+  }
   L.total = off;
   return L;
 }
@@ -1239,7 +1261,9 @@ int launch_bwd_key_tc(const nsa::BwdArgs& a, const void* q, const void* d_out, c
 }
 
 // The selected blocks' key pass on tcgen05 (d = 128): persistent, one CTA per SM over the bucket
-// tiles, whose count the bucket scan left on the device.
+// tiles, whose count the bucket scan left on the device; kDq also writes the selected branch's
+// dq partials.
+template <bool kDq>
 int launch_bwd_sel_key_tc(const nsa::BwdArgs& a, const void* k, const void* v, cudaStream_t st) {
   constexpr int D = 128;
   CUtensorMap kmap, vmap;
@@ -1248,7 +1272,7 @@ int launch_bwd_sel_key_tc(const nsa::BwdArgs& a, const void* k, const void* v, c
       !nsa::make_tmap_bf16_3d(&vmap, v, D, a.hkv, a.N, ks1, ks2, 64, 1, 64))
     return NSA_ERR_CUDA;
   const size_t smem = sizeof(nsa::BsSmem<D>) + 1024;
-  auto kern = nsa::bwd_sel_key_tc_kernel<D>;
+  auto kern = nsa::bwd_sel_key_tc_kernel<D, kDq>;
   if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
   const int nsm = sm_count();
   if (nsm <= 0) return NSA_ERR_CUDA;
@@ -1256,28 +1280,32 @@ int launch_bwd_sel_key_tc(const nsa::BwdArgs& a, const void* k, const void* v, c
   return launch_status("bwd_key_sel", st);
 }
 
-// The compressed branch's row pass on tcgen05 (dq, the branch's statistics and gate gradient of the
-// video rows), from the forward's saved log-sum-exp and output of that branch.
-template <int D>
-int launch_bwd_row_cmp_tc(const nsa::BwdArgs& a, const void* q, const void* d_out, cudaStream_t st) {
+// The video rows' dq on tcgen05 from branches with contiguous keys and kept statistics: the
+// compressed branch (kFull = false: also its statistics and gate gradient), or the compressed
+// branch and the window (kFull = true: every branch's statistics are in a.stats already).
+template <int D, bool kFull>
+int launch_bwd_row_tc(const nsa::BwdArgs& a, const void* q, const void* d_out, cudaStream_t st) {
   const int G = a.G, hq = a.hq, hkv = a.hkv;
   if (G > 128) return NSA_ERR_UNSUPPORTED;
   const int T = 128 / G;
-  CUtensorMap qmap, dmap, kmap, vmap;
+  CUtensorMap qmap, dmap, kcmap, vcmap, kmap, vmap;
   const uint64_t qs1 = static_cast<uint64_t>(D) * 2, qs2 = static_cast<uint64_t>(hq) * D * 2;
   const uint64_t ks1 = static_cast<uint64_t>(D) * 2, ks2 = static_cast<uint64_t>(hkv) * D * 2;
+  const int crows = a.ncmp > 0 ? a.ncmp : 1;  // the workspace holds at least one compressed row
   if (!nsa::make_tmap_bf16_3d(&qmap, q, D, hq, a.N, qs1, qs2, 64, G, T) ||
       !nsa::make_tmap_bf16_3d(&dmap, d_out, D, hq, a.N, qs1, qs2, 64, G, T) ||
-      !nsa::make_tmap_bf16_3d(&kmap, a.kc, D, hkv, a.ncmp, ks1, ks2, 64, 1, 128) ||
-      !nsa::make_tmap_bf16_3d(&vmap, a.vc, D, hkv, a.ncmp, ks1, ks2, 64, 1, 128))
+      !nsa::make_tmap_bf16_3d(&kcmap, a.kc, D, hkv, crows, ks1, ks2, 64, 1, 128) ||
+      !nsa::make_tmap_bf16_3d(&vcmap, a.vc, D, hkv, crows, ks1, ks2, 64, 1, 128) ||
+      !nsa::make_tmap_bf16_3d(&kmap, a.k, D, hkv, a.N, ks1, ks2, 64, 1, 128) ||
+      !nsa::make_tmap_bf16_3d(&vmap, a.v, D, hkv, a.N, ks1, ks2, 64, 1, 128))
     return NSA_ERR_CUDA;
   const long long items = static_cast<long long>((a.nv + T - 1) / T) * hkv;
   if (items > 0x7fffffffLL) return NSA_ERR_UNSUPPORTED;
   const size_t smem = sizeof(nsa::BrSmem<D>) + 1024;
-  auto kern = nsa::bwd_row_cmp_tc_kernel<D>;
+  auto kern = nsa::bwd_row_tc_kernel<D, kFull>;
   if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
-  kern<<<static_cast<unsigned>(items), nsa::kBrThreads, smem, st>>>(qmap, dmap, kmap, vmap, a);
-  return launch_status("bwd_row_cmp", st);
+  kern<<<static_cast<unsigned>(items), nsa::kBrThreads, smem, st>>>(qmap, dmap, kcmap, vcmap, kmap, vmap, a);
+  return launch_status(kFull ? "bwd_row_tc" : "bwd_row_cmp", st);
 }
 
 template <int D>
@@ -1322,10 +1350,24 @@ int backward_impl(const nsa_params_t* p, const void* q, const void* k, const voi
   a.ent_off = reinterpret_cast<const int*>(ws + L.ent_off);
   a.seg_off = reinterpret_cast<const int*>(ws + L.seg_off);
   a.list = reinterpret_cast<const int*>(ws + L.list);
+  // full: the forward kept every branch's statistics, and every video row runs on the tensor
+  // cores (d = 128)
+  bool full = false;
   if (fwd_ws != nullptr && nv > 0) {
     const PrefillLayout F = prefill_layout(p);
     a.fwd_lse = reinterpret_cast<const float*>(fwd_ws + F.lse);
     a.fwd_ocmp = reinterpret_cast<const __half*>(fwd_ws + F.o_cmp);
+    if (D == 128 && p->keep_branch_stats && F.o_sel != 0) {
+      full = true;
+      a.fwd_osel = reinterpret_cast<const __half*>(fwd_ws + F.o_sel);
+      a.fwd_lse_sel = reinterpret_cast<const float*>(fwd_ws + F.lse_sel);
+      a.fwd_owin = reinterpret_cast<const __half*>(fwd_ws + F.o_win);
+      a.fwd_lse_win = reinterpret_cast<const float*>(fwd_ws + F.lse_win);
+      a.video_rows_done = 1;
+      a.row_of = reinterpret_cast<const int*>(ws + L.row_of);
+      a.dq_part = reinterpret_cast<__half*>(ws + L.dq_part);
+      a.part_scale = reinterpret_cast<float2*>(ws + L.part_scale);
+    }
   }
   const size_t kv_bytes = static_cast<size_t>(N) * hkv * D * 4;
   if (cudaMemsetAsync(dk, 0, kv_bytes, st) != cudaSuccess || cudaMemsetAsync(dv, 0, kv_bytes, st) != cudaSuccess)
@@ -1339,13 +1381,19 @@ int backward_impl(const nsa_params_t* p, const void* q, const void* k, const voi
                           phi_v)) != NSA_OK)
       return rc;
   }
-  // row pass: dq, the gates' gradient and the per-branch statistics; with the forward's saved
-  // compressed-branch statistics, that branch's share runs first on tcgen05
-  if (a.fwd_lse != nullptr && L.ncmp > 0) {
-    if ((rc = launch_bwd_row_cmp_tc<D>(a, q, d_out, st)) != NSA_OK) return rc;
+  // row pass: dq, the gates' gradient and the per-branch statistics. full: the statistics of
+  // the video rows come from the forward's, the warp row pass takes the text rows only, and
+  // the video rows' dq is written by the tensor-core kernels below. Else, with the forward's
+  // compressed-branch statistics, that branch's share runs first on tcgen05.
+  if (full) {
+    const long long rows = static_cast<long long>(nv) * hq;
+    nsa::bwd_stats_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(a);
+    if ((rc = launch_status("bwd_stats", st)) != NSA_OK) return rc;
+  } else if (a.fwd_lse != nullptr && L.ncmp > 0) {
+    if ((rc = launch_bwd_row_tc<D, false>(a, q, d_out, st)) != NSA_OK) return rc;
     a.cmp_rows_done = 1;
   }
-  {
+  if (!full || N > nv) {
     const size_t smem = nsa::kBwdWarps * sizeof(nsa::BwdRowSmem<D>);
     auto kern = nsa::bwd_row_kernel<D>;
     if (set_smem(kern, smem) != NSA_OK) return NSA_ERR_CUDA;
@@ -1391,7 +1439,16 @@ int backward_impl(const nsa_params_t* p, const void* q, const void* k, const voi
         (rc = launch_bwd_key_tc<D, nsa::kBwdCmp>(a, q, d_out, ws + L.kc, ws + L.vc, L.ncmp, nv, st)) != NSA_OK)
       return rc;
     if constexpr (D == 128) {
-      if ((rc = launch_bwd_sel_key_tc(a, k, v, st)) != NSA_OK) return rc;
+      if ((rc = full ? launch_bwd_sel_key_tc<true>(a, k, v, st) : launch_bwd_sel_key_tc<false>(a, k, v, st)) !=
+          NSA_OK)
+        return rc;
+      if (full) {
+        // the video rows' dq: compressed and window tiles, then the selected partials
+        if ((rc = launch_bwd_row_tc<D, true>(a, q, d_out, st)) != NSA_OK) return rc;
+        const long long rows = static_cast<long long>(nv) * hq;
+        nsa::bwd_sel_dq_merge_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(a);
+        if ((rc = launch_status("bwd_sel_dq_merge", st)) != NSA_OK) return rc;
+      }
     } else {
       const long long segs = entries / nsa::kBwdSegSel + m + 1;  // >= sum over buckets of ceil(count / segment)
       if ((rc = launch_bwd_key<D, nsa::kBwdSel>(a, segs * (p->sel_block / nsa::kBwdChunk), st)) != NSA_OK) return rc;

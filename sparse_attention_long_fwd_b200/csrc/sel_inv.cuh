@@ -50,6 +50,8 @@ struct SelInvArgs {
   const float* gates;           // [N][hq][3] (g_cmp, g_sel, g_win)
   void* out;                    // [N][hq][D] rows < nv: the gated combine, bf16 or fp32
   int out_f32;
+  __half* o_sel;                // [nv][hq][D] the selected branch's output, kept when not null
+  float* lse_sel;               // [nv][hq] its log-sum-exp (natural log), kept with o_sel
   // Packed batches (null for one sequence): vinfo as in AttnArgs (token -> its sequence's
   // first stream token, first selection block and its row in the batch); blk_tok [nsel]: the
   // stream token where each selection block starts. Block j of a row's sequence is bucket
@@ -761,6 +763,19 @@ __global__ void __launch_bounds__(256, 4) sel_merge_kernel(const SelInvArgs a) {
     }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
+  if (a.o_sel != nullptr) {
+    __half* dst = a.o_sel + orow;
+    if constexpr (kPer == 4) {
+      const __half2 h0 = __floats2half2_rn(acc[0] * inv, acc[1] * inv), h1 = __floats2half2_rn(acc[2] * inv, acc[3] * inv);
+      *reinterpret_cast<uint2*>(dst) =
+          make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
+    } else {
+      const __half2 h0 = __floats2half2_rn(acc[0] * inv, acc[1] * inv);
+      *reinterpret_cast<uint32_t*>(dst) = *reinterpret_cast<const uint32_t*>(&h0);
+    }
+    // M is the largest partial max in log2 units, L the sum in those units
+    if (lane == 0) a.lse_sel[row] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994530942f : -INFINITY;
+  }
   float res[kPer];
 #pragma unroll
   for (int u = 0; u < kPer; ++u) res[u] = gc * oc[u] + gs * (acc[u] * inv) + gw * ow[u];

@@ -52,13 +52,14 @@ class NsaParams(ctypes.Structure):
         ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("cmp_block", ctypes.c_int32),
         ("cmp_stride", ctypes.c_int32), ("sel_block", ctypes.c_int32), ("top_n", ctypes.c_int32),
         ("window", ctypes.c_int32), ("softmax_scale", ctypes.c_float), ("out_dtype", ctypes.c_int32),
-        ("batch", ctypes.c_int32),
+        ("batch", ctypes.c_int32), ("keep_branch_stats", ctypes.c_int32),
     ]
 
 
 class NsaPrefillLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in ("kc", "vc", "o_cmp", "lse", "scores", "sel_idx", "o_win", "total")] + [
-        ("n_cmp", ctypes.c_int32), ("n_sel", ctypes.c_int32), ("score_stride", ctypes.c_int32)]
+        ("n_cmp", ctypes.c_int32), ("n_sel", ctypes.c_int32), ("score_stride", ctypes.c_int32)] + [
+        (n, ctypes.c_size_t) for n in ("o_sel", "lse_sel", "lse_win")]
 
 
 _lib = None
@@ -130,9 +131,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
 def make_params(n_tokens: int, n_video: int | None = None, num_q_heads: int = 28, num_kv_heads: int = 4,
                 head_dim: int = 128, cmp_block: int = 32, cmp_stride: int = 16, sel_block: int = 64, top_n: int = 16,
                 window: int = 512, softmax_scale: float = 0.0, out_dtype: int = NSA_OUT_F32,
-                batch: int = 0) -> NsaParams:
+                batch: int = 0, keep_branch_stats: bool = False) -> NsaParams:
     return NsaParams(n_tokens, n_tokens if n_video is None else n_video, num_q_heads, num_kv_heads, head_dim,
-                     cmp_block, cmp_stride, sel_block, top_n, window, softmax_scale, out_dtype, batch)
+                     cmp_block, cmp_stride, sel_block, top_n, window, softmax_scale, out_dtype, batch,
+                     1 if keep_branch_stats else 0)
 
 
 def _addr(x) -> int | None:
@@ -324,13 +326,16 @@ def alloc_workspace(params: NsaParams, is_decode: bool, device) -> torch.Tensor:
 
 def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gates: torch.Tensor, *, n_video: int | None = None,
             top_n: int = 16, window: int = 512, softmax_scale: float = 0.0, out_dtype=torch.float32,
-            return_sel: bool = False, workspace: torch.Tensor | None = None, phi=None, stream=None):
+            return_sel: bool = False, workspace: torch.Tensor | None = None, phi=None,
+            keep_branch_stats: bool = False, stream=None):
     """NSA prefill of one sequence: q [N,Hq,d], k/v [N,Hkv,d] bf16, gates [N,Hq,3] fp32 (device tensors).
-    phi = (phi_k, phi_v), each [Hkv, 32] fp32, selects the learnable compression."""
+    phi = (phi_k, phi_v), each [Hkv, 32] fp32, selects the learnable compression.
+    keep_branch_stats keeps in the workspace what backward(..., keep_branch_stats=True) reuses."""
     N, hq, d = q.shape
     hkv = k.shape[1]
     p = make_params(N, n_video, hq, hkv, d, top_n=top_n, window=window, softmax_scale=softmax_scale,
-                    out_dtype=NSA_OUT_F32 if out_dtype == torch.float32 else NSA_OUT_BF16)
+                    out_dtype=NSA_OUT_F32 if out_dtype == torch.float32 else NSA_OUT_BF16,
+                    keep_branch_stats=keep_branch_stats)
     out = torch.empty((N, hq, d), dtype=out_dtype, device=q.device)
     sel = torch.empty((p.n_video, hkv, top_n), dtype=torch.int32, device=q.device) if return_sel else None
     if workspace is None:
@@ -380,13 +385,15 @@ def decode(q, kcache, vcache, kcmp, vcmp, seq_lens, gates, *, top_n: int = 16, w
 
 def backward(q, k, v, gates, d_out, sel_idx, *, n_video: int | None = None, top_n: int = 16, window: int = 512,
              softmax_scale: float = 0.0, phi=None, fwd_workspace: torch.Tensor | None = None,
-             workspace: torch.Tensor | None = None, stream=None):
+             keep_branch_stats: bool = False, workspace: torch.Tensor | None = None, stream=None):
     """Gradients of the prefill: returns dq [N,Hq,d], dk, dv [N,Hkv,d] and dgates [N,Hq,3] (fp32),
     given dL/dout (bf16) and the forward's selection sel_idx [N_v,Hkv,top_n]; fwd_workspace, the
-    forward call's workspace, lets the compressed branch reuse its saved statistics."""
+    forward call's workspace, lets the compressed branch reuse its saved statistics, and every
+    branch when both calls pass keep_branch_stats=True."""
     N, hq, d = q.shape
     hkv = k.shape[1]
-    p = make_params(N, n_video, hq, hkv, d, top_n=top_n, window=window, softmax_scale=softmax_scale)
+    p = make_params(N, n_video, hq, hkv, d, top_n=top_n, window=window, softmax_scale=softmax_scale,
+                    keep_branch_stats=keep_branch_stats)
     dq = torch.empty((N, hq, d), dtype=torch.float32, device=q.device)
     dk = torch.empty((N, hkv, d), dtype=torch.float32, device=q.device)
     dv = torch.empty_like(dk)

@@ -22,11 +22,13 @@ def oracle_cfg(w: Workload) -> orc.OracleConfig:
                             w.window)
 
 
-def run_prefill(w: Workload, q, k, v, gates, out_dtype=torch.float32, phi=None):
+def run_prefill(w: Workload, q, k, v, gates, out_dtype=torch.float32, phi=None, keep=False):
     """Call nsa_prefill (nsa_prefill_phi when phi = (phi_k, phi_v) is given) through the C ABI;
-    returns (out, sel, workspace, layout)."""
+    returns (out, sel, workspace, layout). keep: the workspace also keeps the selected and window
+    branches' statistics."""
     p = nsa.make_params(w.n_tokens, w.n_video, w.hq, w.hkv, w.d, w.cmp_len, w.cmp_stride, w.sel_len, w.top_n,
-                        w.window, out_dtype=nsa.NSA_OUT_F32 if out_dtype == torch.float32 else nsa.NSA_OUT_BF16)
+                        w.window, out_dtype=nsa.NSA_OUT_F32 if out_dtype == torch.float32 else nsa.NSA_OUT_BF16,
+                        keep_branch_stats=keep)
     ws = nsa.alloc_workspace(p, False, q.device)
     out = torch.empty((w.n_tokens, w.hq, w.d), dtype=out_dtype, device=q.device)
     sel = torch.full((max(w.n_video, 1), w.hkv, w.top_n), -7, dtype=torch.int32, device=q.device)

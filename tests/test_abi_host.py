@@ -91,6 +91,29 @@ def test_prefill_layout_is_aligned_and_disjoint():
             assert offs[i] + sz <= offs[i + 1], keys[i]
 
 
+def test_kept_branch_statistics_layout():
+    nv = 5000
+    p0 = nsa.make_params(nv)
+    p1 = nsa.make_params(nv, keep_branch_stats=True)
+    l0, l1 = nsa.nsa_prefill_workspace_layout(p0), nsa.nsa_prefill_workspace_layout(p1)
+    assert l0["o_sel"] == l0["lse_sel"] == l0["lse_win"] == 0
+    # the kept arrays follow everything else, 256-byte aligned, and do not overlap
+    offs = [l1["o_sel"], l1["lse_sel"], l1["lse_win"], l1["total"]]
+    sizes = [nv * 28 * 128 * 2, nv * 28 * 4, nv * 28 * 4]
+    assert offs[0] >= l0["total"] and all(o % 256 == 0 for o in offs)
+    for i, sz in enumerate(sizes):
+        assert offs[i] + sz <= offs[i + 1]
+    assert {k: l1[k] for k in ("kc", "o_cmp", "o_win", "scores")} == {k: l0[k] for k in ("kc", "o_cmp", "o_win", "scores")}
+    # the backward keeps the selected branch's dq partials (d = 128 only)
+    assert nsa.nsa_backward_workspace_size(p1) > nsa.nsa_backward_workspace_size(p0)
+    p64 = nsa.make_params(nv, head_dim=64)
+    p64k = nsa.make_params(nv, head_dim=64, keep_branch_stats=True)
+    assert nsa.nsa_backward_workspace_size(p64k) == nsa.nsa_backward_workspace_size(p64)
+    bad = nsa.make_params(nv)
+    bad.keep_branch_stats = 2
+    assert nsa.nsa_workspace_size(bad, False) == 0
+
+
 def test_decode_workspace_scales_with_batch():
     a = nsa.nsa_workspace_size(nsa.make_params(131072, batch=1), True)
     b = nsa.nsa_workspace_size(nsa.make_params(131072, batch=64), True)

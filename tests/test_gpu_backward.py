@@ -35,13 +35,17 @@ def _grad_close(got, ref, what):
 
 
 def _run(w, seed, phi=None, saved=False):
+    """saved: False (the backward recomputes every statistic), True (the forward's compressed-branch
+    statistics) or "keep" (the forward keeps every branch's statistics for the backward)."""
+    keep = saved == "keep"
     q, k, v, g = prefill_inputs(w, seed=seed, device=DEV)
-    out, sel, ws, lay = run_prefill(w, q, k, v, g, phi=phi)
+    out, sel, ws, lay = run_prefill(w, q, k, v, g, phi=phi, keep=keep)
     gen = torch.Generator(device=DEV).manual_seed(seed + 100)
     d_out = torch.randn((w.n_tokens, w.hq, w.d), generator=gen, device=DEV).to(torch.bfloat16)
     sel_arg = sel if w.n_video > 0 else torch.zeros(1, dtype=torch.int32, device=DEV)
     dq, dk, dv, dgates = nsa.backward(q, k, v, g, d_out, sel_arg, n_video=w.n_video, top_n=w.top_n,
-                                      window=w.window, phi=phi, fwd_workspace=ws if saved else None)
+                                      window=w.window, phi=phi, fwd_workspace=ws if saved else None,
+                                      keep_branch_stats=keep)
     torch.cuda.synchronize()
     assert nsa.nsa_get_device_error(clear=True) == 0
     return q, k, v, g, d_out, sel, (dq, dk, dv, dgates)
@@ -70,9 +74,9 @@ def _compare(w, q, k, v, g, d_out, sel, grads, phi=None):
     ("qwen36k_hybrid", 520, 450, 32, 2, 64, 12, 128),  # G = 16, d = 64, with text rows
     ("v128k", 4300, 4300, 8, 2, 64, 8, 64),           # 267 compressed blocks: three 128-key tiles
 ])
-@pytest.mark.parametrize("saved", [False, True])
+@pytest.mark.parametrize("saved", [False, True, "keep"])
 def test_backward_every_element(name, n, nv, hq, hkv, d, top_n, window, saved):
-    """saved: the compressed branch takes the forward's saved log-sum-exp and output."""
+    """saved: see _run; "keep" with d = 128 runs every video row on the tensor-core kernels."""
     w = WORKLOADS[name] if n is None else scaled(WORKLOADS[name], n_tokens=n, n_video=nv, hq=hq, hkv=hkv, d=d,
                                                     top_n=top_n, window=window)
     q, k, v, g, d_out, sel, grads = _run(w, seed=21, saved=saved)
@@ -80,11 +84,23 @@ def test_backward_every_element(name, n, nv, hq, hkv, d, top_n, window, saved):
     print(_compare(w, q, k, v, g, d_out, sel, grads))
 
 
-def test_backward_learnable_compression():
+@pytest.mark.parametrize("saved", [True, "keep"])
+def test_backward_learnable_compression(saved):
     w = scaled(WORKLOADS["v128k"], n_tokens=900, n_video=900)
     phi = phi_weights(w.hkv, 32, seed=22, device=DEV)
-    q, k, v, g, d_out, sel, grads = _run(w, seed=23, phi=phi, saved=True)
+    q, k, v, g, d_out, sel, grads = _run(w, seed=23, phi=phi, saved=saved)
     print(_compare(w, q, k, v, g, d_out, sel, grads, phi=phi))
+
+
+def test_backward_kept_statistics_agree_with_recomputed():
+    """The two saved modes differ only in where the statistics come from; at a size past the
+    oracle's reach (several 128-key tiles in every branch) their gradients agree to the
+    tolerance of the bf16 operands."""
+    w = scaled(WORKLOADS["v16k"], n_tokens=6000, n_video=6000)
+    a = _run(w, seed=25, saved=True)[-1]
+    b = _run(w, seed=25, saved="keep")[-1]
+    for name, x, y in zip(("dq", "dk", "dv", "dgates"), a, b):
+        _grad_close(y, x.detach().cpu().numpy().astype(np.float64), name)
 
 
 def test_backward_sum_identities_at_16k():
@@ -92,7 +108,7 @@ def test_backward_sum_identities_at_16k():
     zero and the mean's weights sum to one), and the value gradients sum to the dO of each
     row weighted by the gates of its non-empty branches."""
     w = WORKLOADS["v16k"]
-    q, k, v, g, d_out, sel, (dq, dk, dv, dgates) = _run(w, seed=24, saved=True)
+    q, k, v, g, d_out, sel, (dq, dk, dv, dgates) = _run(w, seed=24, saved="keep")
     G = w.hq // w.hkv
     do = d_out.double()
     rows = torch.arange(w.n_tokens, device=DEV)

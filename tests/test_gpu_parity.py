@@ -126,6 +126,32 @@ def test_prefill_one_hot_gates_isolate_branches():
     assert_close(outs[1][0][rows].cpu().numpy(), o["o_sel"], "o_sel through g_sel = 1")
 
 
+@pytest.mark.parametrize("n,nv,hq,hkv,d", [(1000, 1000, 28, 4, 128), (777, 700, 8, 1, 64)])
+def test_prefill_kept_branch_statistics(n, nv, hq, hkv, d):
+    """keep_branch_stats: the output is bit-identical to a run without it, and the kept o_sel,
+    lse_sel and lse_win match the oracle's selected and window branches (on the blocks this run
+    selected, so near-ties cannot differ)."""
+    from nsa_check import ws_view, host_bits
+    w = scaled(WORKLOADS["qwen36k_hybrid"], n_tokens=n, n_video=nv, hq=hq, hkv=hkv, d=d)
+    q, k, v, g = prefill_inputs(w, seed=13, device=DEV)
+    out0, sel0, _, _ = run_prefill(w, q, k, v, g)
+    out, sel, ws, lay = run_prefill(w, q, k, v, g, keep=True)
+    assert torch.equal(out, out0) and torch.equal(sel, sel0)
+    assert lay["o_sel"] > 0 and lay["lse_sel"] > 0 and lay["lse_win"] > 0
+    o_sel = ws_view(ws, lay["o_sel"], (nv, hq, d), torch.float16).float().cpu().numpy()
+    lse_sel = ws_view(ws, lay["lse_sel"], (nv, hq), torch.float32).cpu().numpy()
+    lse_win = ws_view(ws, lay["lse_win"], (nv, hq), torch.float32).cpu().numpy()
+    qb, kb, vb = host_bits(q, k, v)
+    rows = np.concatenate([np.arange(0, 70), np.arange(70, nv, 5), [nv - 1]]).astype(np.int32)
+    o = orc.prefill_rows(oracle_cfg(w), qb, kb, vb, g.cpu().numpy(), rows, sel_override=sel[rows].cpu().numpy(),
+                         want=("o_sel", "lse_sel", "lse_win"))
+    assert_close(o_sel[rows], o["o_sel"], "kept o_sel")
+    # log-sum-exp: the kernels sum P as the bf16 value the tensor core multiplies (relative
+    # rounding <= 2^-9 per term), so with one dominant key ln(sum) is off by up to ln(1 + 2^-8)
+    assert_close(lse_sel[rows], o["lse_sel"], "kept lse_sel", max_abs=4e-3, mean_abs=2e-4)
+    assert_close(lse_win[rows], o["lse_win"], "kept lse_win", max_abs=4e-3, mean_abs=2e-4)
+
+
 @pytest.mark.parametrize("n", [9000, 40000])
 def test_prefill_constant_keys_exact_ties(n):
     """Every key equal: the compressed probabilities are uniform, so all interior selection

@@ -187,10 +187,47 @@ def test_cmp_branch_with_unit_blocks_is_dense_causal_attention():
 def test_full_budget_selection_and_window_are_dense_attention():
     N = 200
     cfg, q, k, v, g = _case(N, 6, 2, 16, 21, top_n=orc.num_sel(N, 64) + 2, window=N + 5)
-    o = orc.prefill_rows(cfg, _bits(q), _bits(k), _bits(v), g.numpy(), np.arange(N))
-    ref = _sdpa_causal(_f64(_bits(q)), _f64(_bits(k)), _f64(_bits(v)), 1 / 4.0).numpy()
+    o = orc.prefill_rows(cfg, _bits(q), _bits(k), _bits(v), g.numpy(), np.arange(N),
+                         want=orc.ALL + ("lse_sel", "lse_win"))
+    qd, kd, vd = _f64(_bits(q)), _f64(_bits(k)), _f64(_bits(v))
+    ref = _sdpa_causal(qd, kd, vd, 1 / 4.0).numpy()
     assert np.allclose(o["o_sel"], ref, atol=1e-12, rtol=0)
     assert np.allclose(o["o_win"], ref, atol=1e-12, rtol=0)
+    # both branches' log-sum-exp: torch.logsumexp of the causal score rows
+    for t in (0, 63, 64, 199):
+        for h in range(6):
+            want = torch.logsumexp((kd[: t + 1, h // 3] @ qd[t, h]) / 4.0, 0).item()
+            assert abs(o["lse_sel"][t, h] - want) < 1e-12
+            assert abs(o["lse_win"][t, h] - want) < 1e-12
+
+
+def test_unit_window_log_sum_exp_is_the_own_score():
+    # w = 1: the window holds the query token alone, so its log-sum-exp is that one scaled score
+    cfg, q, k, v, g = _case(130, 4, 2, 16, 23, top_n=3, window=1)
+    rows = np.array([0, 1, 64, 129])
+    o = orc.prefill_rows(cfg, _bits(q), _bits(k), _bits(v), g.numpy(), rows, want=("lse_win", "o_win"))
+    qd, kd, vd = _f64(_bits(q)), _f64(_bits(k)), _f64(_bits(v))
+    for r, t in enumerate(rows):
+        for h in range(4):
+            assert abs(o["lse_win"][r, h] - float(qd[t, h] @ kd[t, h // 2]) / 4.0) < 1e-12
+            assert np.array_equal(o["o_win"][r, h], vd[t, h // 2].numpy())
+
+
+def test_constant_keys_log_sum_exp_counts_the_keys():
+    # every key equal: each branch's log-sum-exp is the common score plus the log of its key count
+    N, w = 300, 40
+    cfg, q, k, v, g = _case(N, 2, 1, 16, 25, top_n=3, window=w)
+    k = k[:1].expand(N, -1, -1).contiguous()
+    rows = np.array([0, 10, 39, 40, 63, 64, 150, 299])
+    o = orc.prefill_rows(cfg, _bits(q), _bits(k), _bits(v), g.numpy(), rows,
+                         want=("sel", "lse_sel", "lse_win"))
+    qd, kd = _f64(_bits(q)), _f64(_bits(k))
+    for r, t in enumerate(rows):
+        nsel_keys = sum(min(64, t + 1 - 64 * j) for j in o["sel"][r, 0] if j >= 0)
+        for h in range(2):
+            z = float(qd[t, h] @ kd[0, 0]) / 4.0
+            assert abs(o["lse_win"][r, h] - (z + math.log(min(w, t + 1)))) < 1e-12
+            assert abs(o["lse_sel"][r, h] - (z + math.log(nsel_keys))) < 1e-12
 
 
 def test_first_token_attends_to_itself_only():
