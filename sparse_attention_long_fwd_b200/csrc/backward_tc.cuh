@@ -38,9 +38,17 @@ namespace nsa {
 
 constexpr int kBtKeys = 128;   // compressed keys per item (MMA M)
 constexpr int kBtRows = 64;    // rows per chunk (MMA N of the score products)
-constexpr int kBtThreads = 64 + 256;
+constexpr int kBtWG = 4;  // softmax warpgroups: each takes 64 / kBtWG rows of every chunk
+constexpr int kBtThreads = 64 + 128 * kBtWG;
 constexpr int kBtSegTokens = 4096;  // tokens per item segment
 constexpr int kBtStages = 4;        // row chunks in flight (a chunk's loads take longer than its MMAs)
+
+__device__ __forceinline__ void cp_async_ca8(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_ca4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
 
 template <int D>
 struct BtSmem {
@@ -49,7 +57,7 @@ struct BtSmem {
   alignas(1024) uint8_t vc[kChunks][kBtKeys * 128];
   alignas(1024) uint8_t q[kBtStages][kChunks][kBtRows * 128];
   alignas(1024) uint8_t dout[kBtStages][kChunks][kBtRows * 128];
-  float4 rowc[kBtStages][kBtRows];  // per row: (lse2, D, gate, token as int bits; -1: no row)
+  float4 rowc[kBtStages][kBtRows];  // per row: (lse2, D, gate, -); only rows that exist are written
   uint64_t kv_full, q_full[kBtStages], q_empty[kBtStages], sd_full, sd_free, p_full, pv_done, drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -102,8 +110,8 @@ __global__ void __launch_bounds__(kBtThreads, 1)
       mbar_init(&sm.q_empty[s], 1);
     }
     mbar_init(&sm.sd_full, 1);
-    mbar_init(&sm.sd_free, 8);
-    mbar_init(&sm.p_full, 8);
+    mbar_init(&sm.sd_free, 4 * kBtWG);
+    mbar_init(&sm.p_full, 4 * kBtWG);
     mbar_init(&sm.pv_done, 1);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
@@ -118,7 +126,7 @@ __global__ void __launch_bounds__(kBtThreads, 1)
     // the value products multiply them by P = dS = 0
     const int r0 = T * G;
     const int per = (kBtRows - r0) * 8;  // 16-byte units per (stage, tensor, chunk)
-    for (int i = tid - 64; i < kBtStages * 2 * kChunks * per; i += 256) {
+    for (int i = tid - 64; i < kBtStages * 2 * kChunks * per; i += 128 * kBtWG) {
       const int u = i % per, rest = i / per;
       const int c = rest % kChunks, tq = (rest / kChunks) % 2, s = rest / (2 * kChunks);
       uint8_t* base = tq == 0 ? sm.q[s][c] : sm.dout[s][c];
@@ -159,21 +167,21 @@ __global__ void __launch_bounds__(kBtThreads, 1)
         }
       }
       q_issued = c + 1;
-      // the rows' constants: (lse2, D) from the row pass, the compressed branch's gate, token
+      // the rows' constants, (lse2, D) from the row pass and the branch's gate, copied without
+      // waiting: each lane's barrier arrival lands with its copies (text rows keep their
+      // statistics in slot 0 and have no gate)
 #pragma unroll
       for (int k = 0; k < kBtRows / 32; ++k) {
         const int r = lane + 32 * k;
         const int t = t0 + r / G, h = g * G + r % G;
-        float4 v = make_float4(-INFINITY, 0.f, 0.f, __int_as_float(-1));
         if (r < T * G && t < tok_hi) {
-          // text rows keep their statistics in slot 0 and have no gate
           const size_t o = (static_cast<size_t>(t) * a.hq + h) * 3;
-          const float2 st = a.stats[o + (BR == kBwdDense ? 0 : BR)];
-          v = make_float4(st.x, st.y, BR == kBwdDense ? 1.f : a.gates[o + BR], __int_as_float(t));
+          const uint32_t dst = smem_u32(&sm.rowc[s][r]);
+          cp_async_ca8(dst, a.stats + o + (BR == kBwdDense ? 0 : BR));
+          if (BR != kBwdDense) cp_async_ca4(dst + 8, a.gates + o + BR);
         }
-        sm.rowc[s][r] = v;
       }
-      mbar_arrive(&sm.q_full[s]);
+      cp_async_arrive_noinc(&sm.q_full[s]);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -237,8 +245,11 @@ __global__ void __launch_bounds__(kBtThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ softmax warps
+    constexpr int kRows = kBtRows / kBtWG;  // rows per thread and chunk
+    constexpr int kPart = D / kBtWG;        // dV, dK columns per thread
+    static_assert(kRows == 16 && (kPart == 32 || kPart == 16), "16-column TMEM loads per chunk");
     const int sw = warp - 2;
-    const int wg = sw >> 2;          // rows [32 wg, 32 wg + 32) of each chunk
+    const int wg = sw >> 2;          // rows [kRows wg, kRows wg + kRows) of each chunk
     const int q4 = warp & 3;         // TMEM lane quadrant
     const int kl = q4 * 32 + lane;   // this thread's key (TMEM lane)
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
@@ -255,26 +266,33 @@ __global__ void __launch_bounds__(kBtThreads, 1)
                                        mbar_wait(&sm.q_full[s], (c / kBtStages) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      float sv[32], dp[32];
+      float sv[kRows], dp[kRows];
       __syncwarp();
-      tmem_ld32(trow + kColS + 32 * wg, sv);
-      tmem_ld32(trow + kColDP + 32 * wg, dp);
+      tmem_ld16(trow + kColS + kRows * wg, sv);
+      tmem_ld16(trow + kColDP + kRows * wg, dp);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.sd_free);
-      uint32_t pp[16], pd[16];
+      // the chunk's rows r = token slot * G + head that exist and see this key: [r_lo, r_hi)
+      // (row token t0 + r / G sees it iff tk <= t <= tk_end; those rows' lse is finite)
+      const int t0 = tok_lo + c * T;
+      const int r_lo = min(max(tk - t0, 0), T) * G;
+      const int n_end = tk_end - t0 >= T ? T : max(tk_end - t0 + 1, 0);  // (tk_end may be INT_MAX)
+      const int r_hi = key_ok ? min(n_end, tok_hi - t0) * G : 0;
+      uint32_t pp[kRows / 2], pd[kRows / 2];
 #pragma unroll
-      for (int j = 0; j < 32; j += 2) {
+      for (int j = 0; j < kRows; j += 2) {
         float pg[2], ds[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const float4 rc = sm.rowc[s][32 * wg + j + e];
-          const int t = __float_as_int(rc.w);
-          const bool vis = key_ok && t >= tk && t <= tk_end && rc.x != -INFINITY;
-          const float p = vis ? ex2_approx(fmaf(sv[j + e], sl2, -rc.x)) : 0.f;
-          pg[e] = p * rc.z;
-          ds[e] = pg[e] * scale * (dp[j + e] - rc.y);
+          const int r = kRows * wg + j + e;
+          const bool vis = r >= r_lo && r < r_hi;
+          const float4 rc = sm.rowc[s][r];
+          const float p = ex2_approx(fmaf(sv[j + e], sl2, -rc.x));
+          const float gate = BR == kBwdDense ? 1.f : rc.z;
+          pg[e] = vis ? p * gate : 0.f;
+          ds[e] = vis ? pg[e] * scale * (dp[j + e] - rc.y) : 0.f;
         }
         pp[j / 2] = pack_bf16x2(pg[0], pg[1]);
         pd[j / 2] = pack_bf16x2(ds[0], ds[1]);
@@ -284,34 +302,34 @@ __global__ void __launch_bounds__(kBtThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      tmem_st16(trow + kColP + 16 * wg, pp);
-      tmem_st16(trow + kColDS + 16 * wg, pd);
+      tmem_st8(trow + kColP + (kRows / 2) * wg, pp);
+      tmem_st8(trow + kColDS + (kRows / 2) * wg, pd);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full);
     }
-    // ---- the item's sums: this warpgroup's half of the key's dVc and dKc rows
+    // ---- the item's sums: this warpgroup's part of the key's dV and dK rows
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done, (nch - 1) & 1, abort_flag));
     if (ok) {
       tc_fence_after();
-      constexpr int kHalf = D / 2;
-      float* dvr = (BR == kBwdCmp ? a.dvc : a.dv) + (static_cast<size_t>(key) * a.hkv + g) * D + wg * kHalf;
-      float* dkr = (BR == kBwdCmp ? a.dkc : a.dk) + (static_cast<size_t>(key) * a.hkv + g) * D + wg * kHalf;
+      float* dvr = (BR == kBwdCmp ? a.dvc : a.dv) + (static_cast<size_t>(key) * a.hkv + g) * D + wg * kPart;
+      float* dkr = (BR == kBwdCmp ? a.dkc : a.dk) + (static_cast<size_t>(key) * a.hkv + g) * D + wg * kPart;
+      float v[kPart], kk[kPart];
+      __syncwarp();
+      if constexpr (kPart == 32) {
+        tmem_ld32(trow + kColDV + wg * kPart, v);
+        tmem_ld32(trow + kColDK + wg * kPart, kk);
+      } else {
+        tmem_ld16(trow + kColDV + wg * kPart, v);
+        tmem_ld16(trow + kColDK + wg * kPart, kk);
+      }
+      tmem_wait_ld();
+      if (key_ok) {
 #pragma unroll
-      for (int x = 0; x < kHalf / 32; ++x) {
-        float v[32], kk[32];
-        __syncwarp();
-        tmem_ld32(trow + kColDV + wg * kHalf + 32 * x, v);
-        tmem_ld32(trow + kColDK + wg * kHalf + 32 * x, kk);
-        tmem_wait_ld();
-        if (key_ok) {
-#pragma unroll
-          for (int u = 0; u < 32; u += 4) {
-            atomicAdd(reinterpret_cast<float4*>(dvr + 32 * x + u), make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]));
-            atomicAdd(reinterpret_cast<float4*>(dkr + 32 * x + u),
-                      make_float4(kk[u], kk[u + 1], kk[u + 2], kk[u + 3]));
-          }
+        for (int u = 0; u < kPart; u += 4) {
+          atomicAdd(reinterpret_cast<float4*>(dvr + u), make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]));
+          atomicAdd(reinterpret_cast<float4*>(dkr + u), make_float4(kk[u], kk[u + 1], kk[u + 2], kk[u + 3]));
         }
       }
     }
@@ -366,8 +384,10 @@ namespace nsa {
 //   S = Q K^T, dP = dO V^T     (M = 128 rows, N = 128 keys; TMEM columns 0 and 128)
 //   softmax warps: dS as bf16 into TMEM (column 384)
 //   dQ += dS K                 (A = dS from TMEM, B = the slot's K read MN-major; column 256)
-// It writes dq for these rows. Same warp roles and bounded waits as the key pass.
-constexpr int kBrThreads = 64 + 256;
+// It writes dq for these rows. Warp 0 loads, warp 1 issues the MMAs, kBrWG softmax warpgroups
+// (thread = row) split each tile's key columns; every wait is bounded.
+constexpr int kBrWG = 4;  // softmax warpgroups: each takes 128 / kBrWG key columns of every tile
+constexpr int kBrThreads = 64 + 128 * kBrWG;
 constexpr int kBrSlots = 2;
 
 template <int D>
@@ -377,7 +397,7 @@ struct BrSmem {
   alignas(1024) uint8_t dout[kChunks][128 * 128];
   alignas(1024) uint8_t kc[kBrSlots][kChunks][128 * 128];
   alignas(1024) uint8_t vc[kBrSlots][kChunks][128 * 128];
-  float rowc[2][128];  // per row: the two warpgroups' halves of <dO, o_cmp>
+  float rowc[kBrWG][128];  // per row: the warpgroups' parts of <dO, o_cmp>
   uint64_t q_full, kv_full[kBrSlots], kv_empty[kBrSlots], sd_full, sd_free, p_full, pv_done, drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -416,8 +436,8 @@ __global__ void __launch_bounds__(kBrThreads, 1)
       mbar_init(&sm.kv_empty[s], 1);
     }
     mbar_init(&sm.sd_full, 1);
-    mbar_init(&sm.sd_free, 8);
-    mbar_init(&sm.p_full, 8);
+    mbar_init(&sm.sd_free, 4 * kBrWG);
+    mbar_init(&sm.p_full, 4 * kBrWG);
     mbar_init(&sm.pv_done, 1);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
@@ -431,7 +451,7 @@ __global__ void __launch_bounds__(kBrThreads, 1)
     // rows T*G .. 127 of the Q and dO tiles are never written by TMA: keep them finite (zero)
     const int r0 = T * G;
     const int per = (128 - r0) * 8;
-    for (int i = tid - 64; i < 2 * kChunks * per; i += 256) {
+    for (int i = tid - 64; i < 2 * kChunks * per; i += 128 * kBrWG) {
       const int u = i % per, rest = i / per;
       const int c = rest % kChunks, tq = rest / kChunks;
       uint8_t* base = tq == 0 ? sm.q[c] : sm.dout[c];
@@ -525,8 +545,11 @@ __global__ void __launch_bounds__(kBrThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ softmax warps
+    constexpr int kCols = 128 / kBrWG;  // key columns per thread and tile
+    constexpr int kPart = D / kBrWG;    // dq columns per thread
+    static_assert(kCols == 32 && (kPart == 32 || kPart == 16), "one 32-column TMEM load per tile");
     const int sw = warp - 2;
-    const int wg = sw >> 2;          // key columns [64 wg, 64 wg + 64) of each tile
+    const int wg = sw >> 2;          // key columns [kCols wg, kCols wg + kCols) of each tile
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;    // this thread's row (TMEM lane)
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
@@ -536,7 +559,7 @@ __global__ void __launch_bounds__(kBrThreads, 1)
     const bool row_valid = r < T * G && t < a.nv;
     bool ok = true;
     // ---- the row's constants: D = <dO, o_cmp> from the forward's fp16 output, each warpgroup
-    // over half of the head dimension, summed through shared memory (kFull: every branch's
+    // over a part of the head dimension, summed through shared memory (kFull: every branch's
     // statistics are in `stats` already)
     float lse2 = -INFINITY, gs = 0.f, dgr = 0.f;
     float lse2_w = -INFINITY, gs_w = 0.f, dgr_w = 0.f;
@@ -557,10 +580,10 @@ __global__ void __launch_bounds__(kBrThreads, 1)
       float part = 0.f;
       if (row_valid) {
         const size_t row = static_cast<size_t>(t) * a.hq + h;
-        const __half* o = a.fwd_ocmp + row * D + wg * (D / 2);
-        const __nv_bfloat16* dop = a.dout + row * D + wg * (D / 2);
-#pragma unroll 4
-        for (int c = 0; c < D / 2; c += 8) {
+        const __half* o = a.fwd_ocmp + row * D + wg * kPart;
+        const __nv_bfloat16* dop = a.dout + row * D + wg * kPart;
+#pragma unroll
+        for (int c = 0; c < kPart; c += 8) {
           const uint4 ov = *reinterpret_cast<const uint4*>(o + c);
           const uint4 dv = *reinterpret_cast<const uint4*>(dop + c);
           const __half2* oh = reinterpret_cast<const __half2*>(&ov);
@@ -577,8 +600,9 @@ __global__ void __launch_bounds__(kBrThreads, 1)
         re = t >= a.cmp_len - 1 ? min((t - a.cmp_len + 1) / a.cmp_stride + 1, a.ncmp) : 0;
       }
       sm.rowc[wg][r] = part;
-      named_bar_sync(1, 256);
-      dgr = sm.rowc[0][r] + sm.rowc[1][r];
+      named_bar_sync(1, 128 * kBrWG);
+#pragma unroll
+      for (int w = 0; w < kBrWG; ++w) dgr += sm.rowc[w][r];
       if (wg == 0 && row_valid) {
         const size_t o = (static_cast<size_t>(t) * a.hq + h) * 3;
         a.stats[o + kBwdCmp] = make_float2(lse2, dgr);
@@ -590,35 +614,32 @@ __global__ void __launch_bounds__(kBrThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const bool win = kFull && kt >= nkt_c;
-      // this thread's 64 keys: [kbase, kbase + 64), visible in [lo, hi)
-      const int kbase = (win ? kb_w + (kt - nkt_c) * 128 : kt * 128) + wg * 64;
+      // this thread's keys: [kbase, kbase + kCols), visible in [lo, hi)
+      const int kbase = (win ? kb_w + (kt - nkt_c) * 128 : kt * 128) + wg * kCols;
       const int lo = win ? t - a.window + 1 : 0, hi = win ? t + 1 : re;
       const float l2 = win ? lse2_w : lse2, dg = win ? dgr_w : dgr, gsb = win ? gs_w : gs;
-      const bool full = __all_sync(0xffffffffu, !row_valid || (kbase >= lo && kbase + 64 <= hi));
-      uint32_t pd[32];
-#pragma unroll
-      for (int hc = 0; hc < 2; ++hc) {
-        float sv[32], dp[32];
+      const bool full = __all_sync(0xffffffffu, !row_valid || (kbase >= lo && kbase + kCols <= hi));
+      uint32_t pd[kCols / 2];
+      {
+        float sv[kCols], dp[kCols];
         __syncwarp();
-        tmem_ld32(trow + kColS + wg * 64 + 32 * hc, sv);
-        tmem_ld32(trow + kColDP + wg * 64 + 32 * hc, dp);
+        tmem_ld32(trow + kColS + wg * kCols, sv);
+        tmem_ld32(trow + kColDP + wg * kCols, dp);
         tmem_wait_ld();
-        if (hc == 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.sd_free);
-        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.sd_free);
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
+        for (int j = 0; j < kCols; j += 2) {
           float ds[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int kidx = kbase + 32 * hc + j + e;
+            const int kidx = kbase + j + e;
             const bool vis = row_valid && (full || (kidx >= lo && kidx < hi)) && l2 != -INFINITY;
             const float p = vis ? ex2_approx(fmaf(sv[j + e], a.sl2, -l2)) : 0.f;
             ds[e] = p * gsb * (dp[j + e] - dg);
           }
-          pd[16 * hc + j / 2] = pack_bf16x2(ds[0], ds[1]);
+          pd[j / 2] = pack_bf16x2(ds[0], ds[1]);
         }
       }
       // dS of this tile goes over the columns the previous tile's dQ MMAs read
@@ -626,35 +647,31 @@ __global__ void __launch_bounds__(kBrThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      tmem_st16(trow + kColDS + wg * 32, *reinterpret_cast<const uint32_t(*)[16]>(&pd[0]));
-      tmem_st16(trow + kColDS + wg * 32 + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pd[16]));
+      tmem_st16(trow + kColDS + wg * (kCols / 2), pd);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full);
     }
-    // ---- dq of this row: this warpgroup's half of D (zero when no key was visible)
+    // ---- dq of this row: this warpgroup's part of D (zero when no key was visible)
     if (ok && nkt > 0) ok = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done, (nkt - 1) & 1, abort_flag));
     if (ok) {
       tc_fence_after();
-      constexpr int kHalf = D / 2;
-      float* dst = a.dq + (static_cast<size_t>(t) * a.hq + h) * D + wg * kHalf;
+      float* dst = a.dq + (static_cast<size_t>(t) * a.hq + h) * D + wg * kPart;
+      float v[kPart];
+      __syncwarp();
+      if (nkt > 0) {
+        if constexpr (kPart == 32) tmem_ld32(trow + kColDQ + wg * kPart, v);
+        else tmem_ld16(trow + kColDQ + wg * kPart, v);
+        tmem_wait_ld();
+      } else {
 #pragma unroll
-      for (int x = 0; x < kHalf / 32; ++x) {
-        float v[32];
-        __syncwarp();
-        if (nkt > 0) {
-          tmem_ld32(trow + kColDQ + wg * kHalf + 32 * x, v);
-          tmem_wait_ld();
-        } else {
+        for (int u = 0; u < kPart; ++u) v[u] = 0.f;
+      }
+      if (row_valid) {
 #pragma unroll
-          for (int u = 0; u < 32; ++u) v[u] = 0.f;
-        }
-        if (row_valid) {
-#pragma unroll
-          for (int u = 0; u < 32; u += 4)
-            *reinterpret_cast<float4*>(dst + 32 * x + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
-        }
+        for (int u = 0; u < kPart; u += 4)
+          *reinterpret_cast<float4*>(dst + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
       }
     }
     tc_fence_before();
