@@ -44,7 +44,8 @@ struct DecArgs {
   int nsplit;           // CTAs per (sequence, group) in dec_cmp_kernel
   int cmp_len, cmp_stride, sel_len, top_n, window, nsel_max;
   float sl2;            // softmax scale * log2(e)
-  float* logits;        // [B][hkv][G][ncmax] base-2 scaled logits of the compressed branch
+  int lstride;          // floats between logit rows: ncmax rounded up to 4 (16-byte rows)
+  float* logits;        // [B][hkv][G][lstride] base-2 scaled logits of the compressed branch
   float* part;          // [B][hkv][nsplit][G][2 + D] (m, l, o[D])
   float* o_cmp;         // [B][hq][D]
   float* lse;           // [B][hq] natural log
@@ -146,12 +147,13 @@ __device__ __forceinline__ void dec_branch_body(DecSmem<D>& sm, const __nv_bfloa
   const __nv_bfloat16* kb = kcache + static_cast<size_t>(b) * a.lmax * rs + static_cast<size_t>(g) * D;
   const __nv_bfloat16* vb = vcache + static_cast<size_t>(b) * a.lmax * rs + static_cast<size_t>(g) * D;
   auto& buf = sm.buf[warp];
+  const uint64_t pol = l2_evict_first_policy();  // the cache rows are read once per step
   WarpAttnState<D> st;
   state_init(st);
   const int my = nch > warp ? (nch - warp + kDecWarps - 1) / kDecWarps : 0;
   dec_stream(
       my,
-      [&](int stg, int x) { load_chunk<D>(buf, stg, kb, vb, rs, list[warp + x * kDecWarps], t + 1, lane); },
+      [&](int stg, int x) { load_chunk<D>(buf, stg, kb, vb, rs, list[warp + x * kDecWarps], t + 1, lane, pol); },
       [&](int stg, int x) { attend_chunk<D>(st, qa, buf, stg, list[warp + x * kDecWarps], key_lo, t + 1, a.sl2, lane); });
   state_reduce_l(st);
   cp_async_wait_0();
@@ -162,8 +164,11 @@ __device__ __forceinline__ void dec_branch_body(DecSmem<D>& sm, const __nv_bfloa
     float M, Lsum, wts[kDecWarps];
     merge_rows<D>(sm.part, kDecWarps, a.G, row, M, Lsum, wts);
     const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+    // (unrolled: the callback's global loads for all of the lane's columns go out together)
+#pragma unroll
     for (int c = lane; c < D; c += 32) {
       float acc = 0.f;
+#pragma unroll
       for (int w = 0; w < kDecWarps; ++w) acc += sm.part[w].o[row][c] * wts[w];
       f(row, c, acc * inv);
     }
@@ -203,15 +208,18 @@ __global__ void __launch_bounds__(kDecWarps * 32) dec_cmp_kernel(const __nv_bflo
   const size_t rs = static_cast<size_t>(a.hkv) * D;
   const __nv_bfloat16* kb = kcmp + static_cast<size_t>(b) * a.ncmax * rs + static_cast<size_t>(g) * D;
   const __nv_bfloat16* vb = vcmp + static_cast<size_t>(b) * a.ncmax * rs + static_cast<size_t>(g) * D;
-  float* lg = a.logits + static_cast<size_t>(bg) * a.G * a.ncmax;
+  float* lg = a.logits + static_cast<size_t>(bg) * a.G * a.lstride;
   auto& buf = sm.buf[warp];
+  // the compressed cache is read once per step: its lines go first, so the logits and partials
+  // this grid writes are still in L2 for dec_select_kernel
+  const uint64_t pol = l2_evict_first_policy();
   WarpAttnState<D> st;
   state_init(st);
   const int nch = w1 > w0 ? (w1 - w0 + kDecChunk - 1) / kDecChunk : 0;
   dec_stream(
-      nch, [&](int stg, int ci) { load_chunk<D>(buf, stg, kb, vb, rs, w0 + ci * kDecChunk, w1, lane); },
+      nch, [&](int stg, int ci) { load_chunk<D>(buf, stg, kb, vb, rs, w0 + ci * kDecChunk, w1, lane, pol); },
       [&](int stg, int ci) {
-        attend_chunk<D>(st, qa, buf, stg, w0 + ci * kDecChunk, w0, w1, a.sl2, lane, lg, a.ncmax, 0, a.G);
+        attend_chunk<D>(st, qa, buf, stg, w0 + ci * kDecChunk, w0, w1, a.sl2, lane, lg, a.lstride, 0, a.G);
       });
   state_reduce_l(st);
   cp_async_wait_0();
@@ -227,8 +235,10 @@ __global__ void __launch_bounds__(kDecWarps * 32) dec_cmp_kernel(const __nv_bflo
       pr[0] = M;
       pr[1] = Lsum;
     }
+#pragma unroll
     for (int c = lane; c < D; c += 32) {
       float acc = 0.f;
+#pragma unroll
       for (int w = 0; w < kDecWarps; ++w) acc += sm.part[w].o[row][c] * wts[w];
       pr[2 + c] = acc;
     }
@@ -277,12 +287,17 @@ __global__ void __launch_bounds__(256, 2) dec_select_kernel(const int32_t* __res
     float acc[kPer];
 #pragma unroll
     for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
-#pragma unroll 4
-    for (int s = 0; s < a.nsplit; ++s) {
-      const float w = __shfl_sync(0xffffffffu, s < 32 ? w0 : w1, s & 31);
-      const float* pr = part + (static_cast<size_t>(s) * a.G + row) * (2 + D) + 2;
+    // (the split loop unrolled 16-wide: its loads go out together)
+    for (int s0 = 0; s0 < a.nsplit; s0 += 16) {
 #pragma unroll
-      for (int k = 0; k < kPer; ++k) acc[k] += w * pr[lane + 32 * k];
+      for (int s = s0; s < s0 + 16; ++s) {
+        const float w = __shfl_sync(0xffffffffu, s < 32 ? w0 : w1, s & 31);
+        if (s < a.nsplit) {
+          const float* pr = part + (static_cast<size_t>(s) * a.G + row) * (2 + D) + 2;
+#pragma unroll
+          for (int k = 0; k < kPer; ++k) acc[k] += w * pr[lane + 32 * k];
+        }
+      }
     }
 #pragma unroll
     for (int k = 0; k < kPer; ++k) a.o_cmp[(static_cast<size_t>(b) * a.hq + h) * D + lane + 32 * k] = acc[k] * inv;
@@ -293,18 +308,55 @@ __global__ void __launch_bounds__(256, 2) dec_select_kernel(const int32_t* __res
   }
   __syncthreads();
   // ---- selection-block scores: compressed block i covers tokens [16i, 16i+32);
-  // block j gets half of blocks 4j-1 and 4j+3 and all of 4j..4j+2.
-  const float* lg = a.logits + static_cast<size_t>(bg) * a.G * a.ncmax;
-  for (int j = tid; j <= jt; j += blockDim.x) {
-    float acc = 0.f;
-    for (int row = 0; row < a.G; ++row) {
-      const float* lr = lg + static_cast<size_t>(row) * a.ncmax;
-      const float l2 = lse2[row];
-      auto p = [&](int i) -> float { return (i >= 0 && i < nc) ? ex2_approx(lr[i] - l2) : 0.f; };
-      acc += 0.5f * p(4 * j - 1) + p(4 * j) + p(4 * j + 1) + p(4 * j + 2) + 0.5f * p(4 * j + 3);
+  // block j gets half of blocks 4j-1 and 4j+3 and all of 4j..4j+2. Thread tid takes the 8
+  // blocks j0 .. j0+7 (j0 = 8 tid + 2048 pass): per head row it needs compressed blocks
+  // 4 j0 - 1 .. 4 j0 + 31, read as 8 aligned float4 and one scalar, and the next row's loads
+  // are issued before this row is binned, so a row costs about one load latency.
+  {
+    const float* lg = a.logits + static_cast<size_t>(bg) * a.G * a.lstride;
+    for (int j0 = 8 * tid; j0 <= jt; j0 += 8 * 256) {  // (uniform trip count per warp is not needed)
+      const int i0 = 4 * j0;  // first of the 32 aligned values
+      float4 cur[8], nxt[8];
+      float hcur = 0.f, hnxt = 0.f;
+      auto load = [&](int row, float4 (&v)[8], float& halo) {
+        const float* lr = lg + static_cast<size_t>(row) * a.lstride;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          v[k] = (i0 + 4 * k < nc) ? *reinterpret_cast<const float4*>(lr + i0 + 4 * k)
+                                   : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        halo = (i0 >= 1 && i0 - 1 < nc) ? lr[i0 - 1] : -INFINITY;
+      };
+      float acc[8];
+#pragma unroll
+      for (int b2 = 0; b2 < 8; ++b2) acc[b2] = 0.f;
+      load(0, cur, hcur);
+      for (int row = 0; row < a.G; ++row) {
+        if (row + 1 < a.G) load(row + 1, nxt, hnxt);
+        const float l2 = lse2[row];
+        float p[33];
+        p[0] = i0 >= 1 && i0 - 1 < nc ? ex2_approx(hcur - l2) : 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float x[4] = {cur[k].x, cur[k].y, cur[k].z, cur[k].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) p[1 + 4 * k + e] = (i0 + 4 * k + e < nc) ? ex2_approx(x[e] - l2) : 0.f;
+        }
+#pragma unroll
+        for (int b2 = 0; b2 < 8; ++b2)
+          acc[b2] += 0.5f * p[4 * b2] + p[4 * b2 + 1] + p[4 * b2 + 2] + p[4 * b2 + 3] + 0.5f * p[4 * b2 + 4];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) cur[k] = nxt[k];
+        hcur = hnxt;
+      }
+#pragma unroll
+      for (int b2 = 0; b2 < 8; ++b2) {
+        const int j = j0 + b2;
+        if (j <= jt) {
+          sc[j] = acc[b2];
+          a.scores[static_cast<size_t>(bg) * a.nsel_max + j] = acc[b2];
+        }
+      }
     }
-    sc[j] = acc;
-    a.scores[static_cast<size_t>(bg) * a.nsel_max + j] = acc;
   }
   __syncthreads();
   if (tid < 32) {
@@ -335,7 +387,8 @@ __global__ void __launch_bounds__(kDecWarps * 32) dec_branch_kernel(const __nv_b
   dec_branch_body<D>(sm, q, kcache, vcache, a, b, g, L, false, [&](int row, int c, float v) {
     const size_t r = row0 + row;
     const size_t e = r * D + c;
-    const float o = a.gates[r * 3 + 0] * a.o_cmp[e] + a.gates[r * 3 + 1] * v + a.gates[r * 3 + 2] * a.o_win[e];
+    const float o = __ldg(a.gates + r * 3 + 0) * __ldcg(a.o_cmp + e) + __ldg(a.gates + r * 3 + 1) * v +
+                    __ldg(a.gates + r * 3 + 2) * __ldcg(a.o_win + e);
     if (a.out_f32)
       static_cast<float*>(a.out)[e] = o;
     else

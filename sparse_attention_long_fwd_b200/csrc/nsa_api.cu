@@ -183,7 +183,8 @@ DecodeLayout decode_layout(const nsa_params_t* p) {
     off = align_up(off + (bytes > 0 ? bytes : 1));
     return at;
   };
-  L.logits = take(static_cast<size_t>(B) * hkv * G * (L.ncmax > 0 ? L.ncmax : 1) * 4);
+  // logit rows of ncmax rounded up to 4 floats (16-byte rows: dec_select reads them as float4)
+  L.logits = take(static_cast<size_t>(B) * hkv * G * ((L.ncmax + 3) / 4 * 4 > 0 ? (L.ncmax + 3) / 4 * 4 : 4) * 4);
   L.part = take(static_cast<size_t>(B) * hkv * L.nsplit * G * (2 + d) * 4);
   L.o_cmp = take(static_cast<size_t>(B) * hq * d * 4);
   L.lse = take(static_cast<size_t>(B) * hq * 4);
@@ -558,6 +559,7 @@ int decode_impl(const nsa_params_t* p, const void* q, const void* kcache, const 
   a.G = a.hq / a.hkv;
   a.d = D;
   a.ncmax = L.ncmax;
+  a.lstride = (L.ncmax + 3) / 4 * 4;
   a.nsplit = L.nsplit;
   a.cmp_len = p->cmp_block;
   a.cmp_stride = p->cmp_stride;

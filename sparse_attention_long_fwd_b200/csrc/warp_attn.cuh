@@ -39,6 +39,20 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src, bool vali
   const int n = valid ? 16 : 0;  // zero-fill when the source row is out of range
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(n) : "memory");
 }
+// L2 policy for data read once (a stream): its lines are the first evicted, so what the
+// stream's kernel writes for the next kernel stays in L2.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void cp_async16_hint(void* dst, const void* src, bool valid, uint64_t policy) {
+  const uint32_t d = smem_u32(dst);
+  const int n = valid ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(d), "l"(src), "r"(n),
+               "l"(policy)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
@@ -79,10 +93,11 @@ __device__ __forceinline__ void load_q_frags(uint32_t (&a)[D / 16][4], const __n
 // Copy CK key rows (and value rows) starting at token `start` into ring stage `st`.
 // Rows at or beyond `row_end` are zero-filled and never read from global memory.
 // K/V row `tok` of the head lives at base + tok * row_stride.
+// policy: 0, or an L2 policy the copies carry (l2_evict_first_policy for data read once).
 template <int D, int CK, int NST>
 __device__ __forceinline__ void load_chunk(WarpChunkBuf<D, CK, NST>& buf, int st, const __nv_bfloat16* kbase,
                                            const __nv_bfloat16* vbase, size_t row_stride, int start, int row_end,
-                                           int lane) {
+                                           int lane, uint64_t policy = 0) {
   constexpr int kUnits = D / 8;  // 16-byte units per row
 #pragma unroll
   for (int i = lane; i < CK * kUnits; i += 32) {
@@ -91,8 +106,13 @@ __device__ __forceinline__ void load_chunk(WarpChunkBuf<D, CK, NST>& buf, int st
     const bool valid = tok < row_end;
     const size_t src = static_cast<size_t>(valid ? tok : 0) * row_stride + unit * 8;
     const int dst = row * D + static_cast<int>(swz_unit(row, unit)) * 8;
-    cp_async16(&buf.kv[st][0][dst], kbase + src, valid);
-    cp_async16(&buf.kv[st][1][dst], vbase + src, valid);
+    if (policy != 0) {
+      cp_async16_hint(&buf.kv[st][0][dst], kbase + src, valid, policy);
+      cp_async16_hint(&buf.kv[st][1][dst], vbase + src, valid, policy);
+    } else {
+      cp_async16(&buf.kv[st][0][dst], kbase + src, valid);
+      cp_async16(&buf.kv[st][1][dst], vbase + src, valid);
+    }
   }
 }
 
