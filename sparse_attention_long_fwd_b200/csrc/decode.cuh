@@ -227,20 +227,21 @@ __global__ void __launch_bounds__(kDecWarps * 32) dec_cmp_kernel(const __nv_bflo
   state_store(st, sm.part[warp], lane);
   __syncthreads();
   float* dst = a.part + (static_cast<size_t>(bg) * a.nsplit + split) * a.G * (2 + D);
+  const uint64_t keep = l2_evict_last_policy();  // dec_select_kernel reads the partials back
   for (int row = warp; row < a.G; row += kDecWarps) {
     float M, Lsum, wts[kDecWarps];
     merge_rows<D>(sm.part, kDecWarps, a.G, row, M, Lsum, wts);
     float* pr = dst + static_cast<size_t>(row) * (2 + D);
     if (lane == 0) {
-      pr[0] = M;
-      pr[1] = Lsum;
+      st_f32_hint(pr, M, keep);
+      st_f32_hint(pr + 1, Lsum, keep);
     }
 #pragma unroll
     for (int c = lane; c < D; c += 32) {
       float acc = 0.f;
 #pragma unroll
       for (int w = 0; w < kDecWarps; ++w) acc += sm.part[w].o[row][c] * wts[w];
-      pr[2 + c] = acc;
+      st_f32_hint(pr + 2 + c, acc, keep);
     }
   }
 }

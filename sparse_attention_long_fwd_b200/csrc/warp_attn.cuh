@@ -46,6 +46,15 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
+// L2 policy for data the next kernel reads back: its lines are the last evicted.
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void st_f32_hint(float* dst, float v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(dst), "f"(v), "l"(policy) : "memory");
+}
 __device__ __forceinline__ void cp_async16_hint(void* dst, const void* src, bool valid, uint64_t policy) {
   const uint32_t d = smem_u32(dst);
   const int n = valid ? 16 : 0;
@@ -166,6 +175,8 @@ __device__ __forceinline__ void attend_chunk(WarpAttnState<D>& s, const uint32_t
     }
   }
   if (logits != nullptr) {
+    // the next kernel reads these back: they are stored with an L2 evict-last policy
+    const uint64_t keep = l2_evict_last_policy();
     const int r0 = lane >> 2;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -174,7 +185,7 @@ __device__ __forceinline__ void attend_chunk(WarpAttnState<D>& s, const uint32_t
         const int row = r0 + (e >> 1) * 8;
         const int key = start + nt * 8 + 2 * (lane & 3) + (e & 1);
         if (row < G && key >= key_lo && key < key_hi)
-          logits[static_cast<size_t>(row) * logit_stride + (key - logit_base)] = sc[nt][e];
+          st_f32_hint(logits + static_cast<size_t>(row) * logit_stride + (key - logit_base), sc[nt][e], keep);
       }
     }
   }
