@@ -356,7 +356,7 @@ def compress(k: torch.Tensor, v: torch.Tensor, phi=None, stream=None):
         k, v = k.unsqueeze(0), v.unsqueeze(0)
     B, L, hkv, d = k.shape
     p = make_params(L, L, hkv, hkv, d, batch=B)
-    nc = (L - 32) // 16 + 1 if L >= 32 else 0
+    nc = (L - p.cmp_block) // p.cmp_stride + 1 if L >= p.cmp_block else 0  # Ncmp(L) of the params' l and s
     kc = torch.empty((B, nc, hkv, d), dtype=k.dtype, device=k.device)
     vc = torch.empty_like(kc)
     if phi is None:
