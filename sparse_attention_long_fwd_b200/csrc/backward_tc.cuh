@@ -165,6 +165,13 @@ __global__ void __launch_bounds__(kBtThreads, 1)
           tma_load_3d(&qmap, &sm.q_full[s], sm.q[s][ch], ch * 64, g * G, t0);
           tma_load_3d(&dmap, &sm.q_full[s], sm.dout[s][ch], ch * 64, g * G, t0);
         }
+        // the rows a ring's depth further on go to L2 now (they come from HBM)
+        if (c + kBtStages < nch) {
+          for (int ch = 0; ch < kChunks; ++ch) {
+            tma_prefetch_3d(&qmap, ch * 64, g * G, t0 + kBtStages * T);
+            tma_prefetch_3d(&dmap, ch * 64, g * G, t0 + kBtStages * T);
+          }
+        }
       }
       q_issued = c + 1;
       // the rows' constants, (lse2, D) from the row pass and the branch's gate, copied without
@@ -484,6 +491,14 @@ __global__ void __launch_bounds__(kBrThreads, 1)
         for (int c = 0; c < kChunks; ++c) {
           tma_load_3d(win ? &kmap : &kcmap, &sm.kv_full[s], sm.kc[s][c], c * 64, g, k0);
           tma_load_3d(win ? &vmap : &vcmap, &sm.kv_full[s], sm.vc[s][c], c * 64, g, k0);
+        }
+        // the window's key tiles come from HBM: the one two tiles on goes to L2 now
+        if (kFull && kt + 2 >= nkt_c && kt + 2 < nkt) {
+          const int kp = kb_w + (kt + 2 - nkt_c) * 128;
+          for (int c = 0; c < kChunks; ++c) {
+            tma_prefetch_3d(&kmap, c * 64, g, kp);
+            tma_prefetch_3d(&vmap, c * 64, g, kp);
+          }
         }
         kv_issued = kt + 1;
       }
