@@ -184,6 +184,46 @@ def test_prefill_v128k_sampled():
     print(st)
 
 
+def test_prefill_and_decode_graph_replay_match_direct_calls():
+    """The C ABI only enqueues work on the given stream, so a call can be captured in a CUDA
+    graph: its replay gives the direct call's output and selection bit for bit."""
+    w = scaled(WORKLOADS["qwen36k_hybrid"], n_tokens=1500, n_video=1300)
+    q, k, v, g = prefill_inputs(w, seed=17, device=DEV)
+    p = nsa.make_params(w.n_tokens, w.n_video, w.hq, w.hkv, w.d, w.cmp_len, w.cmp_stride, w.sel_len, w.top_n,
+                        w.window, out_dtype=nsa.NSA_OUT_F32)
+    ws = nsa.alloc_workspace(p, False, q.device)
+    out0 = torch.empty((w.n_tokens, w.hq, w.d), device=DEV)
+    sel0 = torch.empty((w.n_video, w.hkv, w.top_n), dtype=torch.int32, device=DEV)
+    assert nsa.nsa_prefill(q, k, v, g, p, out0, sel0, ws, ws.numel()) == nsa.NSA_OK
+    torch.cuda.synchronize()
+    out1, sel1 = torch.full_like(out0, float("nan")), torch.full_like(sel0, -7)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        assert nsa.nsa_prefill(q, k, v, g, p, out1, sel1, ws, ws.numel()) == nsa.NSA_OK
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out1, out0) and torch.equal(sel1, sel0)
+    del graph
+    # decode (three kernels with dependent launches) the same way
+    wd = scaled(WORKLOADS["decode64x128k"], batch=4, n_tokens=3000)
+    qd, kc, vc, gd, sl = decode_inputs(wd, seed=18, device=DEV)
+    kcmp, vcmp = nsa.compress(kc, vc)
+    pd = nsa.make_params(wd.n_tokens, wd.n_tokens, wd.hq, wd.hkv, wd.d, top_n=wd.top_n, window=wd.window,
+                         out_dtype=nsa.NSA_OUT_F32, batch=wd.batch)
+    wsd = nsa.alloc_workspace(pd, True, qd.device)
+    d0 = torch.empty((wd.batch, wd.hq, wd.d), device=DEV)
+    assert nsa.nsa_decode(qd, kc, vc, kcmp, vcmp, sl, gd, pd, d0, None, wsd, wsd.numel()) == nsa.NSA_OK
+    torch.cuda.synchronize()
+    d1 = torch.full_like(d0, float("nan"))
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        assert nsa.nsa_decode(qd, kc, vc, kcmp, vcmp, sl, gd, pd, d1, None, wsd, wsd.numel()) == nsa.NSA_OK
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(d1, d0)
+    assert nsa.nsa_get_device_error(clear=True) == 0
+
+
 @pytest.mark.parametrize("n", [8192, 32768, 131072])
 def test_prefill_error_by_length(n):
     """The fp16 intermediates (o_cmp, o_win, the selected partials) against sequence length:
