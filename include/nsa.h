@@ -90,6 +90,9 @@ typedef struct {
  *                row, ascending, padded with -1.
  *   workspace    device scratch of at least nsa_workspace_size(params, 0) bytes (256-byte aligned).
  * Rows t < N_v follow NSA; rows t >= N_v get dense causal attention (gates unused).
+ * The call only enqueues kernels and device memsets on `stream` (no host copies, no
+ * synchronisation), so it can be captured in a CUDA graph and replayed; nsa_decode,
+ * nsa_compress and nsa_backward can be captured the same way.
  */
 int nsa_prefill(const void* q, const void* k, const void* v, const float* gates, const nsa_params_t* params,
                 void* out, int32_t* out_sel_idx, void* workspace, size_t workspace_bytes, void* stream);
@@ -146,7 +149,9 @@ size_t nsa_prefill_varlen_workspace_size(const nsa_params_t* params, const int32
  *               in packed order (sequence after sequence, segment after segment).
  *   workspace   at least nsa_prefill_packed_workspace_size(...) bytes, 256-byte aligned.
  * Every stage is launched once for the whole batch (tiles span sequences); the plan (two small
- * tables) is copied to the workspace with cudaMemcpyAsync from host memory first. Errors as
+ * tables) is copied to the workspace with cudaMemcpyAsync from host memory first, from a host
+ * buffer that lives only during the call: do not capture this call (or nsa_prefill_varlen) in a
+ * CUDA graph. Errors as
  * nsa_prefill, plus NSA_ERR_INVALID_ARG for malformed sequence or segment arrays, and
  * NSA_ERR_UNSUPPORTED when a video stream has more than 8,192 selection blocks; nothing is
  * enqueued then.
