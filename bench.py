@@ -655,7 +655,8 @@ def run_backward(args, dev, w, q, k, v, g, peaks, flush, world):
     bws = torch.empty(nsa.nsa_backward_workspace_size(p), dtype=torch.uint8, device=dev)
 
     def step(events):
-        rc = nsa.nsa_backward(q, k, v, g, d_out, sel, ws, None, None, p, dq, dk, dv, dgates, bws, bws.numel())
+        rc = nsa.nsa_backward(q, k, v, g, d_out, sel, ws, ws.numel(), None, None, p, dq, dk, dv, dgates, bws,
+                              bws.numel())
         if rc != nsa.NSA_OK:
             raise nsa.NsaError(rc, "nsa_backward")
 

@@ -285,6 +285,9 @@ size_t nsa_gate_mlp_pooled_workspace_size(int batch, int seq_len, int heads, int
  *            params.keep_branch_stats = 1 (for both calls) the selected and window branches'
  *            too (o_sel, lse_sel, o_win, lse_win), and every video row's dq, statistics and
  *            gate gradient come from single passes on the tensor cores
+ *   fwd_workspace_bytes  its size; smaller than nsa_workspace_size(params, 0) (for example a
+ *            workspace of a forward call without keep_branch_stats, given to a backward call
+ *            with it) returns NSA_ERR_WORKSPACE_TOO_SMALL; ignored when fwd_workspace is NULL
  *   phi_k, phi_v  both NULL (mean compression) or both the learnable weights [Hkv][l] fp32
  *   dq       [N][Hq][d] fp32     dk, dv [N][Hkv][d] fp32    (written, not accumulated)
  *   dgates   [N][Hq][3] fp32: <dL/dout, o_b> per branch; 0 for text rows
@@ -294,9 +297,9 @@ size_t nsa_gate_mlp_pooled_workspace_size(int batch, int seq_len, int heads, int
  * last bits vary from run to run.
  */
 int nsa_backward(const void* q, const void* k, const void* v, const float* gates, const void* d_out,
-                 const int32_t* sel_idx, const void* fwd_workspace, const float* phi_k, const float* phi_v,
-                 const nsa_params_t* params, float* dq, float* dk, float* dv, float* dgates, void* workspace,
-                 size_t workspace_bytes, void* stream);
+                 const int32_t* sel_idx, const void* fwd_workspace, size_t fwd_workspace_bytes, const float* phi_k,
+                 const float* phi_v, const nsa_params_t* params, float* dq, float* dk, float* dv, float* dgates,
+                 void* workspace, size_t workspace_bytes, void* stream);
 
 /* Workspace bytes nsa_backward needs; 0 if params are invalid. */
 size_t nsa_backward_workspace_size(const nsa_params_t* params);

@@ -1479,9 +1479,9 @@ size_t nsa_backward_workspace_size(const nsa_params_t* params) {
 }
 
 int nsa_backward(const void* q, const void* k, const void* v, const float* gates, const void* d_out,
-                 const int32_t* sel_idx, const void* fwd_workspace, const float* phi_k, const float* phi_v,
-                 const nsa_params_t* params, float* dq, float* dk, float* dv, float* dgates, void* workspace,
-                 size_t workspace_bytes, void* stream) {
+                 const int32_t* sel_idx, const void* fwd_workspace, size_t fwd_workspace_bytes, const float* phi_k,
+                 const float* phi_v, const nsa_params_t* params, float* dq, float* dk, float* dv, float* dgates,
+                 void* workspace, size_t workspace_bytes, void* stream) {
   int rc = check_common(params);
   if (rc != NSA_OK) return rc;
   if (params->n_video < 0 || params->n_video > params->n_tokens) return NSA_ERR_INVALID_ARG;
@@ -1496,6 +1496,10 @@ int nsa_backward(const void* q, const void* k, const void* v, const float* gates
     return NSA_ERR_INVALID_ARG;
   if (nsel_of(params->n_video, params->sel_block) > 8192) return NSA_ERR_UNSUPPORTED;
   if (workspace_bytes < bwd_layout(params).total) return NSA_ERR_WORKSPACE_TOO_SMALL;
+  // the forward's workspace must hold the layout these params give it (with keep_branch_stats,
+  // the kept statistics too): a workspace from a call with other params is refused, not read past
+  if (fwd_workspace != nullptr && fwd_workspace_bytes < prefill_layout(params).total)
+    return NSA_ERR_WORKSPACE_TOO_SMALL;
   if ((rc = check_device()) != NSA_OK) return rc;
   auto* ws = static_cast<uint8_t*>(workspace);
   auto st = static_cast<cudaStream_t>(stream);

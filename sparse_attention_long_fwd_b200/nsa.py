@@ -106,7 +106,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.nsa_gate_mlp_pooled.restype = I
     lib.nsa_gate_mlp_pooled_workspace_size.argtypes = [I, I, I, I]
     lib.nsa_gate_mlp_pooled_workspace_size.restype = S
-    lib.nsa_backward.argtypes = [P, P, P, P, P, P, P, P, P, PP, P, P, P, P, P, S, P]
+    lib.nsa_backward.argtypes = [P, P, P, P, P, P, P, S, P, P, PP, P, P, P, P, P, S, P]
     lib.nsa_backward.restype = I
     lib.nsa_backward_workspace_size.argtypes = [PP]
     lib.nsa_backward_workspace_size.restype = S
@@ -251,12 +251,12 @@ def nsa_gate_mlp_pooled_workspace_size(batch: int, seq_len: int, heads: int, dim
     return int(load_library().nsa_gate_mlp_pooled_workspace_size(batch, seq_len, heads, dim))
 
 
-def nsa_backward(q, k, v, gates, d_out, sel_idx, fwd_workspace, phi_k, phi_v, params: NsaParams, dq, dk, dv, dgates,
-                 workspace, workspace_bytes: int, stream=None) -> int:
+def nsa_backward(q, k, v, gates, d_out, sel_idx, fwd_workspace, fwd_workspace_bytes: int, phi_k, phi_v,
+                 params: NsaParams, dq, dk, dv, dgates, workspace, workspace_bytes: int, stream=None) -> int:
     return load_library().nsa_backward(_addr(q), _addr(k), _addr(v), _addr(gates), _addr(d_out), _addr(sel_idx),
-                                       _addr(fwd_workspace), _addr(phi_k), _addr(phi_v), ctypes.byref(params),
-                                       _addr(dq), _addr(dk), _addr(dv), _addr(dgates), _addr(workspace),
-                                       workspace_bytes, _stream(stream))
+                                       _addr(fwd_workspace), fwd_workspace_bytes, _addr(phi_k), _addr(phi_v),
+                                       ctypes.byref(params), _addr(dq), _addr(dk), _addr(dv), _addr(dgates),
+                                       _addr(workspace), workspace_bytes, _stream(stream))
 
 
 def nsa_backward_workspace_size(params: NsaParams) -> int:
@@ -404,8 +404,9 @@ def backward(q, k, v, gates, d_out, sel_idx, *, n_video: int | None = None, top_
             raise NsaError(NSA_ERR_INVALID_ARG, "nsa_backward_workspace_size")
         workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
     pk, pv = (None, None) if phi is None else phi
-    _check(nsa_backward(q, k, v, gates, d_out, sel_idx, fwd_workspace, pk, pv, p, dq, dk, dv, dgates, workspace,
-                        workspace.numel(), stream), "nsa_backward")
+    fwd_bytes = fwd_workspace.numel() if fwd_workspace is not None else 0
+    _check(nsa_backward(q, k, v, gates, d_out, sel_idx, fwd_workspace, fwd_bytes, pk, pv, p, dq, dk, dv, dgates,
+                        workspace, workspace.numel(), stream), "nsa_backward")
     return dq, dk, dv, dgates
 
 

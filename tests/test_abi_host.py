@@ -196,20 +196,31 @@ def test_backward_validation():
     p = _p()
     need = nsa.nsa_backward_workspace_size(p)
     assert need > 0 and need % 256 == 0
-    ok_args = [f] * 6 + [None, None, None, p] + [f] * 5
+    ok_args = [f] * 6 + [None, 0, None, None, p] + [f] * 5
     assert nsa.nsa_backward(*ok_args, need - 1, None) == nsa.NSA_ERR_WORKSPACE_TOO_SMALL
     bad = list(ok_args)
     bad[5] = None  # the forward's selection is required when there are video rows
     assert nsa.nsa_backward(*bad, need, None) == nsa.NSA_ERR_INVALID_ARG
     bad = list(ok_args)
-    bad[7] = f  # phi_k without phi_v
+    bad[8] = f  # phi_k without phi_v
     assert nsa.nsa_backward(*bad, need, None) == nsa.NSA_ERR_INVALID_ARG
     bad = list(ok_args)
-    bad[10] = f + 4  # dq misaligned
+    bad[11] = f + 4  # dq misaligned
     assert nsa.nsa_backward(*bad, need, None) == nsa.NSA_ERR_INVALID_ARG
     bad = list(ok_args)
     bad[6] = f + 128  # the forward's workspace must be 256-byte aligned
+    bad[7] = 1 << 40
     assert nsa.nsa_backward(*bad, need, None) == nsa.NSA_ERR_INVALID_ARG
+    # the forward's workspace must hold the layout of these params: one from a call without
+    # keep_branch_stats is too small for a backward with it
+    fwd_plain = nsa.nsa_workspace_size(p, False)
+    pk = _p()
+    pk.keep_branch_stats = 1
+    fwd_keep = nsa.nsa_workspace_size(pk, False)
+    assert fwd_keep > fwd_plain
+    need_k = nsa.nsa_backward_workspace_size(pk)
+    args = [f] * 6 + [f, fwd_plain, None, None, pk] + [f] * 5
+    assert nsa.nsa_backward(*args, need_k, None) == nsa.NSA_ERR_WORKSPACE_TOO_SMALL
     assert nsa.nsa_backward_workspace_size(_p(head_dim=96)) == 0
 
 
