@@ -135,22 +135,62 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 }
 
 // Sum over 32 columns of 2^(s*sl2 - ms), in 8 independent chains.
+// Two fp32 values in one 64-bit register: sm_100 issues the pair's FMA (or ADD) as one
+// instruction, which halves the FMA-pipe work of the softmax warps on these paths.
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b, float c) {
+  asm("{\n\t.reg .b64 pa, pb, pc, pd;\n\t"
+      "mov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %4};\n\tmov.b64 pc, {%5, %5};\n\t"
+      "fma.rn.f32x2 pd, pa, pb, pc;\n\tmov.b64 {%0, %1}, pd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+__device__ __forceinline__ void fma2v(float& d0, float& d1, float a0, float a1, float b, float c0, float c1) {
+  asm("{\n\t.reg .b64 pa, pb, pc, pd;\n\t"
+      "mov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %4};\n\tmov.b64 pc, {%5, %6};\n\t"
+      "fma.rn.f32x2 pd, pa, pb, pc;\n\tmov.b64 {%0, %1}, pd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 pa, pb;\n\tmov.b64 pa, {%0, %1};\n\tmov.b64 pb, {%2, %3};\n\t"
+      "add.rn.f32x2 pa, pa, pb;\n\tmov.b64 {%0, %1}, pa;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(b0), "f"(b1));
+}
+
 __device__ __forceinline__ float chunk_sum_ex2(const float (&s)[32], float sl2, float ms) {
   float acc[8];
 #pragma unroll
-  for (int c = 0; c < 8; ++c) acc[c] = ex2_approx(fmaf(s[c], sl2, -ms));
+  for (int c = 0; c < 8; c += 2) {
+    float x0, x1;
+    fma2(x0, x1, s[c], s[c + 1], sl2, -ms);
+    acc[c] = ex2_approx(x0);
+    acc[c + 1] = ex2_approx(x1);
+  }
 #pragma unroll
   for (int i = 8; i < 32; i += 8)
 #pragma unroll
-    for (int c = 0; c < 8; ++c) acc[c] += ex2_approx(fmaf(s[i + c], sl2, -ms));
-  return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+    for (int c = 0; c < 8; c += 2) {
+      float x0, x1;
+      fma2(x0, x1, s[i + c], s[i + c + 1], sl2, -ms);
+      add2(acc[c], acc[c + 1], ex2_approx(x0), ex2_approx(x1));
+    }
+  add2(acc[0], acc[1], acc[2], acc[3]);
+  add2(acc[4], acc[5], acc[6], acc[7]);
+  add2(acc[0], acc[1], acc[4], acc[5]);
+  return acc[0] + acc[1];
 }
 
 // s[i] = 2^(s[i]*sl2 - off) for the columns kbase+i in [rb, re), 0 elsewhere.
 __device__ __forceinline__ void chunk_ex2(float (&s)[32], float sl2, float off, bool full, int kbase, int rb, int re) {
   if (full) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) s[i] = ex2_approx(fmaf(s[i], sl2, -off));
+    for (int i = 0; i < 32; i += 2) {
+      float x0, x1;
+      fma2(x0, x1, s[i], s[i + 1], sl2, -off);
+      s[i] = ex2_approx(x0);
+      s[i + 1] = ex2_approx(x1);
+    }
   } else {
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
@@ -764,11 +804,19 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
                 carry_last = c127;
               }
             }
+            // bins u and u + 1 in one paired pass; the compressed block between them (4u + 3)
+            // gives half to each
             float bin[kChunkBins];
+            static_assert(kChunkBins % 2 == 0, "bins are computed in pairs");
 #pragma unroll
-            for (int u = 0; u < kChunkBins; ++u) {
-              const float left = u > 0 ? 0.5f * sc[4 * u - 1] : (hc == 0 ? half_in : 0.5f * prev_last);
-              bin[u] = left + sc[4 * u] + sc[4 * u + 1] + sc[4 * u + 2] + 0.5f * sc[4 * u + 3];
+            for (int u = 0; u < kChunkBins; u += 2) {
+              // the outer halves: block 4u - 1 (left of bin u; 2 x half_in is exact) and 4u + 7
+              const float outer = u > 0 ? sc[4 * u - 1] : (hc == 0 ? 2.f * half_in : prev_last);
+              float b0 = sc[4 * u], b1 = sc[4 * u + 4];
+              add2(b0, b1, sc[4 * u + 1], sc[4 * u + 5]);
+              add2(b0, b1, sc[4 * u + 2], sc[4 * u + 6]);
+              fma2v(b0, b1, sc[4 * u + 3], sc[4 * u + 3], 0.5f, b0, b1);
+              fma2v(bin[u], bin[u + 1], outer, sc[4 * u + 7], 0.5f, b0, b1);
             }
             prev_last = sc[31];
             switch (Gp) {
