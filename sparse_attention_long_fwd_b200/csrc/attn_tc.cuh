@@ -135,29 +135,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 }
 
 // Sum over 32 columns of 2^(s*sl2 - ms), in 8 independent chains.
-// Two fp32 values in one 64-bit register: sm_100 issues the pair's FMA (or ADD) as one
-// instruction, which halves the FMA-pipe work of the softmax warps on these paths.
-__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b, float c) {
-  asm("{\n\t.reg .b64 pa, pb, pc, pd;\n\t"
-      "mov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %4};\n\tmov.b64 pc, {%5, %5};\n\t"
-      "fma.rn.f32x2 pd, pa, pb, pc;\n\tmov.b64 {%0, %1}, pd;\n\t}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(a0), "f"(a1), "f"(b), "f"(c));
-}
-__device__ __forceinline__ void fma2v(float& d0, float& d1, float a0, float a1, float b, float c0, float c1) {
-  asm("{\n\t.reg .b64 pa, pb, pc, pd;\n\t"
-      "mov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %4};\n\tmov.b64 pc, {%5, %6};\n\t"
-      "fma.rn.f32x2 pd, pa, pb, pc;\n\tmov.b64 {%0, %1}, pd;\n\t}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(a0), "f"(a1), "f"(b), "f"(c0), "f"(c1));
-}
-__device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 pa, pb;\n\tmov.b64 pa, {%0, %1};\n\tmov.b64 pb, {%2, %3};\n\t"
-      "add.rn.f32x2 pa, pa, pb;\n\tmov.b64 {%0, %1}, pa;\n\t}"
-      : "+f"(a0), "+f"(a1)
-      : "f"(b0), "f"(b1));
-}
-
 __device__ __forceinline__ float chunk_sum_ex2(const float (&s)[32], float sl2, float ms) {
   float acc[8];
 #pragma unroll
@@ -774,10 +751,14 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::kThreads, 1)
           }
           chunk_ex2(sc, sl2, lse2, full, kbase + 32 * hc, rb, re);
           if (MODE != kModeCmp) {
-            float ps[4] = {0.f, 0.f, 0.f, 0.f};
+            float ps[4] = {sc[0], sc[1], sc[2], sc[3]};
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ps[i & 3] += sc[i];
-            psum += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+            for (int i = 4; i < 32; i += 4) {
+              add2(ps[0], ps[1], sc[i], sc[i + 1]);
+              add2(ps[2], ps[3], sc[i + 2], sc[i + 3]);
+            }
+            add2(ps[0], ps[1], ps[2], ps[3]);
+            psum += ps[0] + ps[1];
           }
           if (MODE == kModeCmp) {
             if (hc == 0 && half == 0 && kt2 > 0) {

@@ -646,15 +646,18 @@ __global__ void __launch_bounds__(kBrThreads, 1)
         if (lane == 0) mbar_arrive(&sm.sd_free);
 #pragma unroll
         for (int j = 0; j < kCols; j += 2) {
-          float ds[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int kidx = kbase + j + e;
-            const bool vis = row_valid && (full || (kidx >= lo && kidx < hi)) && l2 != -INFINITY;
-            const float p = vis ? ex2_approx(fmaf(sv[j + e], a.sl2, -l2)) : 0.f;
-            ds[e] = p * gsb * (dp[j + e] - dg);
-          }
-          pd[j / 2] = pack_bf16x2(ds[0], ds[1]);
+          // keys j and j + 1 in paired fp32 arithmetic: P = 2^(S sl2 - lse2), dS = P g scale (dP - D)
+          const int kidx = kbase + j;
+          const bool ok_row = row_valid && l2 != -INFINITY;
+          const bool vis0 = ok_row && (full || (kidx >= lo && kidx < hi));
+          const bool vis1 = ok_row && (full || (kidx + 1 >= lo && kidx + 1 < hi));
+          float x0, x1, d0, d1;
+          fma2(x0, x1, sv[j], sv[j + 1], a.sl2, -l2);
+          const float p0 = vis0 ? ex2_approx(x0) : 0.f, p1 = vis1 ? ex2_approx(x1) : 0.f;
+          sub2v(d0, d1, dp[j], dp[j + 1], dg, dg);
+          mul2v(d0, d1, d0, d1, gsb, gsb);
+          mul2v(d0, d1, d0, d1, p0, p1);
+          pd[j / 2] = pack_bf16x2(d0, d1);
         }
       }
       // dS of this tile goes over the columns the previous tile's dQ MMAs read
