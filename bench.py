@@ -52,7 +52,7 @@ PREFILL_KERNELS = 9
 # DRAM bytes per launch of a stage's kernel on the 128K workload, from one ncu capture of the
 # current kernel version (the full-size traffic summary kept with the profiles); an entry is
 # removed when its kernel changes, and the roofline then reports traffic null.
-STAGE_TRAFFIC_V128K = {"cmp_attn_scores": 4037673472}
+STAGE_TRAFFIC_V128K = {"cmp_attn_scores": 4065668352}
 DECODE_STAGES = ["dec_cmp_and_window", "dec_select", "dec_selected_and_combine"]
 
 
