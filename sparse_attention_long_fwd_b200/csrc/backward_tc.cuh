@@ -57,7 +57,9 @@ struct BtSmem {
   alignas(1024) uint8_t vc[kChunks][kBtKeys * 128];
   alignas(1024) uint8_t q[kBtStages][kChunks][kBtRows * 128];
   alignas(1024) uint8_t dout[kBtStages][kChunks][kBtRows * 128];
-  float4 rowc[kBtStages][kBtRows];  // per row: (lse2, D, gate, -); only rows that exist are written
+  // per row: lse2, D and the gate, each field its own array so that two adjacent rows' values
+  // load as one register pair; only rows that exist are written
+  float rlse[kBtStages][kBtRows], rd[kBtStages][kBtRows], rg[kBtStages][kBtRows];
   uint64_t kv_full, q_full[kBtStages], q_empty[kBtStages], sd_full, sd_free, p_full, pv_done, drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -183,9 +185,10 @@ __global__ void __launch_bounds__(kBtThreads, 1)
         const int t = t0 + r / G, h = g * G + r % G;
         if (r < T * G && t < tok_hi) {
           const size_t o = (static_cast<size_t>(t) * a.hq + h) * 3;
-          const uint32_t dst = smem_u32(&sm.rowc[s][r]);
-          cp_async_ca8(dst, a.stats + o + (BR == kBwdDense ? 0 : BR));
-          if (BR != kBwdDense) cp_async_ca4(dst + 8, a.gates + o + BR);
+          const float* st2 = reinterpret_cast<const float*>(a.stats + o + (BR == kBwdDense ? 0 : BR));
+          cp_async_ca4(smem_u32(&sm.rlse[s][r]), st2);
+          cp_async_ca4(smem_u32(&sm.rd[s][r]), st2 + 1);
+          if (BR != kBwdDense) cp_async_ca4(smem_u32(&sm.rg[s][r]), a.gates + o + BR);
         }
       }
       cp_async_arrive_noinc(&sm.q_full[s]);
@@ -290,19 +293,27 @@ __global__ void __launch_bounds__(kBtThreads, 1)
       uint32_t pp[kRows / 2], pd[kRows / 2];
 #pragma unroll
       for (int j = 0; j < kRows; j += 2) {
-        float pg[2], ds[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int r = kRows * wg + j + e;
-          const bool vis = r >= r_lo && r < r_hi;
-          const float4 rc = sm.rowc[s][r];
-          const float p = ex2_approx(fmaf(sv[j + e], sl2, -rc.x));
-          const float gate = BR == kBwdDense ? 1.f : rc.z;
-          pg[e] = vis ? p * gate : 0.f;
-          ds[e] = vis ? pg[e] * scale * (dp[j + e] - rc.y) : 0.f;
+        // rows r and r + 1 in paired fp32 arithmetic (their constants load as register pairs):
+        // P = 2^(S sl2 - lse2), P g, dS = P g scale (dP - D)
+        const int r = kRows * wg + j;
+        const float2 l2 = *reinterpret_cast<const float2*>(&sm.rlse[s][r]);
+        const float2 dd = *reinterpret_cast<const float2*>(&sm.rd[s][r]);
+        float x0, x1, pg0, pg1, d0, d1;
+        fma2v(x0, x1, sv[j], sv[j + 1], sl2, -l2.x, -l2.y);
+        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+        if (BR == kBwdDense) {
+          pg0 = p0;
+          pg1 = p1;
+        } else {
+          const float2 gg = *reinterpret_cast<const float2*>(&sm.rg[s][r]);
+          mul2v(pg0, pg1, p0, p1, gg.x, gg.y);
         }
-        pp[j / 2] = pack_bf16x2(pg[0], pg[1]);
-        pd[j / 2] = pack_bf16x2(ds[0], ds[1]);
+        sub2v(d0, d1, dp[j], dp[j + 1], dd.x, dd.y);
+        mul2v(d0, d1, d0, d1, scale, scale);
+        mul2v(d0, d1, d0, d1, pg0, pg1);
+        const bool vis0 = r >= r_lo && r < r_hi, vis1 = r + 1 >= r_lo && r + 1 < r_hi;
+        pp[j / 2] = pack_bf16x2(vis0 ? pg0 : 0.f, vis1 ? pg1 : 0.f);
+        pd[j / 2] = pack_bf16x2(vis0 ? d0 : 0.f, vis1 ? d1 : 0.f);
       }
       // P and dS of chunk c go over the columns the value MMAs of chunk c - 1 read
       if (c >= 1) ok = mbar_wait(&sm.pv_done, (c - 1) & 1, abort_flag);
