@@ -1,20 +1,21 @@
-// backward_tc.cuh -- key passes of the backward on tcgen05: the compressed branch, the
-// sliding window and the dense text rows (the branches whose rows are runs of consecutive
-// tokens).
+// backward_tc.cuh -- the backward on tcgen05: key passes (dK, dV) of the compressed branch,
+// the sliding window and the dense text rows; the row pass (dq) over compressed and window
+// tiles; the selected blocks' key pass, which also emits the selected branch's dq partials;
+// the kept-statistics kernel and the dq merge.
 //
 // For a branch's keys K, V the key pass accumulates, over every (token, head) row r that
 // sees key i,
 //   dV[i] += g_r P[r, i] dO_r,   dK[i] += dS[r, i] q_r,
 //   P[r, i] = 2^(scale log2e <q_r, K_i> - lse2_r),  dS = g_r P scale (<dO_r, V_i> - D_r),
-// with lse2_r and D_r = <dO_r, o_b,r> from the row pass (the gradient of the forward
+// with lse2_r and D_r = <dO_r, o_b,r> from the row statistics (the gradient of the forward
 // defined in this library; the pages train the model end to end, shd-paper.top page
 // "VideoNSA: Native Sparse Attention Scales Video Understanding", abstract). The keys are
 // the compressed summaries Kc, Vc (row r of token t sees block i iff i*s + l - 1 <= t), the
 // tokens of the window (t - w < i <= t) or, for text rows, every token i <= t (gate 1).
 //
-// One CTA per (tile of 128 keys, KV group, segment of tokens). Its keys sit in
+// Key pass: one CTA per (tile of 128 keys, KV group, segment of tokens). Its keys sit in
 // the 128 TMEM lanes (M = 128) for the whole item; the rows stream in chunks of 64 (T
-// tokens x G heads, a 3-D TMA box like the forward's query tiles) through two stages:
+// tokens x G heads, a 3-D TMA box like the forward's query tiles) through a four-stage ring:
 //   S^T = Kc Q^T and dP^T = Vc dO^T   (M = 128 keys, N = 64 rows, K = d; TMEM columns 0, 64)
 //   softmax warps: P g and dS as bf16 into TMEM (columns 128 and 160)
 //   dV += (P g)^T-rows x dO, dK += dS x Q   (A from TMEM, B = the stage's dO / Q read
@@ -23,9 +24,9 @@
 // its softmax. P and dS of chunk c are stored only once the MMAs of chunk c-1 that read
 // those columns have finished (write-after-read on the same TMEM columns). At the end each
 // key's dVc, dKc rows are added to the global sums (segments of one key tile share rows).
-// Warp roles: warp 0 loads (TMA, and the rows' lse2 / D / gate / token), warp 1 owns TMEM
-// and issues the MMAs, warps 2..9 (two warpgroups) take 32 of a chunk's 64 rows each.
-// Every wait is bounded (sm100.cuh).
+// Warp roles: warp 0 loads (the TMA boxes, an L2 prefetch a ring's depth ahead, and the rows'
+// lse2 / D / gate by cp.async), warp 1 owns TMEM and issues the MMAs, warps 2..17 (four
+// warpgroups) take 16 of a chunk's 64 rows each. Every wait is bounded (sm100.cuh).
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
